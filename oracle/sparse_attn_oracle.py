@@ -1,0 +1,369 @@
+"""Float64 CPU oracle for indexer-driven top-k block-sparse attention.
+
+TEST INFRASTRUCTURE ONLY.  This module is the plain, slow, obviously-correct
+definition that the CUDA library is checked against.  Only ``tests/``,
+``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py`` may import it.  It shares no code with the CUDA path and
+imports nothing from ``top_block_sparse_b200``.
+
+Every step works on ONE (sequence, KV head) slab at a time, in float64
+(bf16 and fp32 inputs convert exactly), with no tiling, no online softmax and
+no fusion.  Library primitives used as steps: numpy matmul / dot, sort, exp,
+log.
+
+Sources (web pages on the method; each function cites the passage it restates):
+
+* [S3R review]   "港科大(广州)S3R:稀疏起草+稠密验证,RL训练吞吐1.39倍"
+                 (longzhangge.com PaperDaily), section "稀疏起草": the
+                 sparse-attention formula over a retained index set T and the
+                 KV-selection formula (recent window + top-K); the k=6 draft
+                 chunk with the selection held fixed.
+* [LSA review]   "精读:LSA——当稀疏注意力的账单从「算」搬到「找」"
+                 (tuntang.top), §2.2 (L2-normalise, sum 4 keys into a pool key,
+                 centroid = normalised sum), §2.3 (normalised query scores
+                 centroids, top buckets + 4 sink keys + 512 window keys, one
+                 index table shared by the heads), §2.4 (query heads summed
+                 into one index query).
+* [SparDA]       hyper.ai paper summary 2606.04511 (SparDA on InfLLM-V2),
+                 section "方法": attention = initial tokens + local sliding
+                 window + top-k selected blocks; keys mean-pooled into
+                 compressed keys; one forecast (index) head per GQA group.
+* [PulseCol]     "PulseCol:周期性刷新的列稀疏注意力机制..." (bittide), §3.1
+                 eq. (1) Z = QK^T/sqrt(d_h) and eq. (2) masked softmax
+                 softmax(Z + M(S)) V.
+
+Readings taken where the pages leave a step open (each is also listed in the
+design notes of the repository):
+
+* R1  GQA aggregation: the index query is the plain SUM of the group's query
+      vectors; block score s_j = qbar . Kc_j * scale  (LSA §2.4 sums heads).
+* R2  Prefill tile aggregation: a 64-query tile scores block j with the MAX
+      over its rows of the GQA-summed logit (the pages do not say; max keeps
+      any block some row needs, cf. N-LSA's max aggregation in LSA §2.5).
+* R3  Window = the last W keys of the context [C-W, C); the new tokens
+      (decode token, draft chunk, prefill diagonal tile) are attended causally
+      in addition.
+* R4  Blocks lying wholly inside sink or window are not candidates; a block
+      partly covered stays a candidate and its covered keys count once.
+* R5  Only complete blocks (b keys inside the context) are candidates.
+* R6  Ties: score descending, then lower block index first.  A pair whose
+      k-th and (k+1)-th candidate scores differ by less than 1e-4*|s_k| is a
+      near-tie; more than one selected set is then correct.
+* R7  LSA pooling order: normalise each raw key, sum 4 consecutive unit keys
+      into a pool key, centroid = normalise(sum of the block's pool keys);
+      score = (qbar/|qbar|) . c_j (cosine).  normalise(0) = 0.
+* R8  Softmax scale 1/sqrt(d) unless given (PulseCol eq. (1)).
+* R9  Multi-token chunk: the selection is made once from the chunk's FIRST
+      query and reused by every token of the chunk (S3R draft chunk); token j
+      of the chunk also sees chunk keys C..C+j.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+NEAR_TIE_REL = 1e-4
+
+
+@dataclass
+class OracleParams:
+    """Selection and attention parameters of one problem (sizes in keys)."""
+
+    block_size: int            # b: raw keys per selectable block
+    top_k: int                 # k: blocks chosen by score
+    sink_keys: int             # S: keys [0, S) always attended
+    window_keys: int           # W: keys [C-W, C) always attended
+    pool: str = "mean"         # "mean" (SparDA) or "lsa" (LSA §2.2)
+    pool_stride: int = 4       # raw keys summed into one LSA pool key
+    scale: Optional[float] = None   # softmax scale; None -> 1/sqrt(d)
+
+
+# --------------------------------------------------------------------------
+# 1. Compression (one slab: K [T, d] float64)
+# --------------------------------------------------------------------------
+
+def pool_mean(K: np.ndarray, b: int) -> np.ndarray:
+    """Compressed keys by mean pooling  [SparDA, "方法"].
+
+    Kc[j] = (1/b) * sum_{t = j*b}^{j*b + b - 1} K[t]  for every COMPLETE block j
+    of the rows given (reading R5: a partial trailing block has no compressed
+    key).  Returns [nb, d] with nb = len(K) // b.
+    """
+    K = np.asarray(K, dtype=np.float64)
+    nb = K.shape[0] // b
+    out = np.zeros((nb, K.shape[1]), dtype=np.float64)
+    for j in range(nb):
+        out[j] = K[j * b:(j + 1) * b].sum(axis=0) / b
+    return out
+
+
+def _normalise(x: np.ndarray) -> np.ndarray:
+    """x / ||x||_2 along the last axis, with normalise(0) = 0 (reading R7)."""
+    n = np.sqrt((x * x).sum(axis=-1, keepdims=True))
+    return np.where(n > 0, x / np.where(n > 0, n, 1.0), 0.0)
+
+
+def pool_lsa(K: np.ndarray, b: int, stride: int = 4) -> np.ndarray:
+    """LSA centroids  [LSA review, §2.2].
+
+    Steps in the page's order: (1) L2-normalise every raw key; (2) sum each
+    ``stride`` consecutive unit keys into one pool key; (3) a block of b raw
+    keys holds b/stride pool keys and its centroid is the normalised sum of
+    them.  Returns [nb, d] unit vectors (or zero rows), nb = len(K) // b.
+    """
+    assert b % stride == 0
+    K = np.asarray(K, dtype=np.float64)
+    nb = K.shape[0] // b
+    khat = _normalise(K[:nb * b])                                   # (1)
+    pool_keys = khat.reshape(nb * b // stride, stride, -1).sum(1)   # (2)
+    per_block = b // stride
+    cent = np.zeros((nb, K.shape[1]), dtype=np.float64)
+    for j in range(nb):                                             # (3)
+        cent[j] = pool_keys[j * per_block:(j + 1) * per_block].sum(axis=0)
+    return _normalise(cent)
+
+
+def compress(K: np.ndarray, p: OracleParams) -> np.ndarray:
+    if p.pool == "mean":
+        return pool_mean(K, p.block_size)
+    if p.pool == "lsa":
+        return pool_lsa(K, p.block_size, p.pool_stride)
+    raise ValueError(p.pool)
+
+
+# --------------------------------------------------------------------------
+# 2. Scoring
+# --------------------------------------------------------------------------
+
+def index_query(q_group: np.ndarray) -> np.ndarray:
+    """One index query per GQA group: the sum of the group's query vectors.
+
+    [LSA review, §2.4] (the query side sums the heads into one index query);
+    [SparDA, "方法"] (one forecast head per GQA group).  q_group: [G, d].
+    """
+    return np.asarray(q_group, dtype=np.float64).sum(axis=0)
+
+
+def softmax_scale(d: int, p: OracleParams) -> float:
+    """1/sqrt(d_h)  [PulseCol, §3.1 eq. (1)] unless the caller fixes it."""
+    return (1.0 / math.sqrt(d)) if p.scale is None else float(p.scale)
+
+
+def block_scores(qbar: np.ndarray, Kc: np.ndarray, p: OracleParams) -> np.ndarray:
+    """Score of every compressed key.
+
+    mean pooling: s_j = qbar . Kc_j * scale   (reading R1)
+    LSA pooling : s_j = (qbar / |qbar|) . c_j (LSA §2.3: the query is
+                  normalised before it scores the centroids; reading R7)
+    """
+    qbar = np.asarray(qbar, dtype=np.float64)
+    if p.pool == "lsa":
+        return Kc @ _normalise(qbar)
+    return (Kc @ qbar) * softmax_scale(Kc.shape[1], p)
+
+
+# --------------------------------------------------------------------------
+# 3. Candidates and top-k
+# --------------------------------------------------------------------------
+
+def sink_window(C: int, p: OracleParams):
+    """Always-attended context keys: sink [0, S) and window [C-W, C), clipped
+    to the context [0, C)  [SparDA, "方法" (initial tokens + local window);
+    LSA review §2.3 (4 sink keys + 512 window keys); S3R review, KV-selection
+    formula (recent window R)]."""
+    s_end = min(p.sink_keys, C)
+    w_begin = max(C - p.window_keys, 0)
+    return s_end, w_begin
+
+
+def candidate_blocks(C: int, p: OracleParams) -> List[int]:
+    """Blocks that compete in top-k (readings R4, R5): complete blocks of the
+    context whose keys are not ALL inside sink or window.
+
+    Sink is the prefix [0, s_end) and window the suffix [w_begin, C), so the
+    context keys outside both form the interval [s_end, w_begin); a complete
+    block [j*b, j*b + b) competes iff it shares at least one key with it.
+    """
+    b = p.block_size
+    s_end, w_begin = sink_window(C, p)
+    out = []
+    for j in range(C // b):
+        lo, hi = j * b, (j + 1) * b
+        if lo < w_begin and hi > s_end:
+            out.append(j)
+    return out
+
+
+@dataclass
+class Selection:
+    selected: List[int]          # ascending block ids
+    n_candidates: int
+    kth_score: Optional[float]   # score of the k-th ranked candidate
+    gap: Optional[float]         # s_(k) - s_(k+1); None when all are taken
+    near_tie: bool               # gap < 1e-4 * |s_(k)|  (reading R6)
+
+
+def select_topk(scores: np.ndarray, candidates: Sequence[int], k: int) -> Selection:
+    """Top-k block selection [SparDA, "方法"; S3R review, KV-selection
+    formula]: rank candidates by (score descending, block index ascending)
+    and keep the first min(k, #candidates).  Returns them in ascending block
+    order with the k-th/(k+1)-th gap used for near-tie accounting."""
+    cand = list(candidates)
+    ranked = sorted(cand, key=lambda j: (-float(scores[j]), j))
+    take = ranked[:min(k, len(ranked))]
+    kth = float(scores[take[-1]]) if take else None
+    gap = None
+    near = False
+    if len(ranked) > k and k > 0:
+        gap = float(scores[ranked[k - 1]]) - float(scores[ranked[k]])
+        near = gap < NEAR_TIE_REL * abs(float(scores[ranked[k - 1]]))
+    return Selection(sorted(take), len(cand), kth, gap, near)
+
+
+# --------------------------------------------------------------------------
+# 4. Attended set and masked softmax attention
+# --------------------------------------------------------------------------
+
+def attended_positions(C: int, p: OracleParams, selected: Sequence[int],
+                       last_pos: int) -> np.ndarray:
+    """Key positions one query at position ``last_pos`` (>= C) attends:
+
+    {t < S} U {C-W <= t < C} U {t in a selected block} U {C <= t <= last_pos}
+
+    [SparDA, "方法" (initial + local + top-k blocks); S3R review, the retained
+    set T = recent window U top-K; reading R3 for the new tokens].  A key
+    covered twice is listed once (reading R4).
+    """
+    b = p.block_size
+    s_end, w_begin = sink_window(C, p)
+    mask = np.zeros(last_pos + 1, dtype=bool)
+    mask[0:s_end] = True
+    mask[w_begin:C] = True
+    for j in selected:
+        mask[j * b:(j + 1) * b] = True
+    mask[C:last_pos + 1] = True
+    return np.flatnonzero(mask)
+
+
+def masked_softmax_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray,
+                             positions: np.ndarray, scale: float):
+    """Attention over the retained set only.
+
+    z_t = q . K_t * scale for t in the set; w = exp(z - max z) / sum exp;
+    O = sum_t w_t V_t; lse = max z + log sum exp(z - max z).
+    [S3R review, sparse-attention formula: softmax over K_T, weighted sum of
+    V_T; PulseCol §3.1 eq. (1)-(2): keys outside the mask get -inf logits, so
+    they receive zero weight.]
+    Returns (O [d], lse, w [len(positions)]).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    Ks = np.asarray(K[positions], dtype=np.float64)
+    Vs = np.asarray(V[positions], dtype=np.float64)
+    z = (Ks @ q) * scale
+    m = z.max()
+    e = np.exp(z - m)
+    den = e.sum()
+    w = e / den
+    O = w @ Vs
+    lse = m + math.log(den)
+    return O, lse, w
+
+
+# --------------------------------------------------------------------------
+# 5. One (sequence, KV head) pair: decode, draft chunk
+# --------------------------------------------------------------------------
+
+def decode_pair(q_tokens: np.ndarray, K: np.ndarray, V: np.ndarray, C: int,
+                p: OracleParams, Kc: Optional[np.ndarray] = None) -> Dict:
+    """Decode / multi-token chunk for one (sequence, KV head).
+
+    q_tokens: [n_q, G, d] queries of the new tokens for the G query heads of
+              this KV head (token j sits at position C + j).
+    K, V:     [>= C + n_q, d] this pair's cache rows (new tokens' keys at C..).
+    Steps: compress the context keys [0, C) -> index query of token 0 ->
+    scores -> candidates -> top-k -> per token j and head g, attention over
+    sink U window U selected U chunk keys C..C+j  (reading R9).
+    """
+    n_q, G, d = q_tokens.shape
+    if Kc is None:
+        Kc = compress(K[:C], p)
+    qbar = index_query(q_tokens[0])
+    s = block_scores(qbar, Kc, p)
+    cand = candidate_blocks(C, p)
+    sel = select_topk(s, cand, p.top_k)
+    scale = softmax_scale(d, p)
+    O = np.zeros((n_q, G, d))
+    lse = np.zeros((n_q, G))
+    wsum = np.zeros((n_q, G))
+    pos_list = []
+    for j in range(n_q):
+        pos = attended_positions(C, p, sel.selected, C + j)
+        pos_list.append(pos)
+        for g in range(G):
+            O[j, g], lse[j, g], w = masked_softmax_attention(
+                q_tokens[j, g], K, V, pos, scale)
+            wsum[j, g] = w.sum()
+    return dict(Kc=Kc, qbar=qbar, scores=s, candidates=cand, sel=sel,
+                O=O, lse=lse, wsum=wsum, positions=pos_list)
+
+
+# --------------------------------------------------------------------------
+# 6. Prefill (one KV head): 64-query tiles, tile-max scoring
+# --------------------------------------------------------------------------
+
+def prefill_tile_scores(q_rows: np.ndarray, Kc: np.ndarray, p: OracleParams) -> np.ndarray:
+    """Tile score of each block: max over the tile's rows of the row's
+    GQA-summed block score (readings R1, R2).  q_rows: [rows, G, d]."""
+    per_row = np.stack([block_scores(index_query(q_rows[r]), Kc, p)
+                        for r in range(q_rows.shape[0])])
+    return per_row.max(axis=0)
+
+
+def prefill_tile(q_tile: np.ndarray, K: np.ndarray, V: np.ndarray, i: int,
+                 p: OracleParams, Kc_all: Optional[np.ndarray] = None) -> Dict:
+    """Query tile i of a causal prefill (tile size = block size b).
+
+    The tile's queries sit at positions [i*b, i*b + rows); the tile's context
+    is C_i = i*b (blocks 0..i-1).  Its selection uses the tile-max score over
+    the context's complete blocks; every query row then attends sink U window
+    U selected blocks U the causal part of its own tile (readings R2, R3).
+    q_tile: [rows, G, d];  K, V: this KV head's rows [T, d].
+    """
+    b = p.block_size
+    C = i * b
+    rows, G, d = q_tile.shape
+    if Kc_all is None:
+        Kc_all = compress(K, p)
+    Kc = Kc_all[:C // b]
+    s = prefill_tile_scores(q_tile, Kc, p) if C // b > 0 else np.zeros(0)
+    cand = candidate_blocks(C, p)
+    sel = select_topk(s, cand, p.top_k)
+    scale = softmax_scale(d, p)
+    O = np.zeros((rows, G, d))
+    lse = np.zeros((rows, G))
+    wsum = np.zeros((rows, G))
+    for r in range(rows):
+        pos = attended_positions(C, p, sel.selected, C + r)
+        for g in range(G):
+            O[r, g], lse[r, g], w = masked_softmax_attention(
+                q_tile[r, g], K, V, pos, scale)
+            wsum[r, g] = w.sum()
+    return dict(scores=s, candidates=cand, sel=sel, O=O, lse=lse, wsum=wsum)
+
+
+def prefill_head_selection(q_head_rows: np.ndarray, Kc_all: np.ndarray,
+                           p: OracleParams, tiles: Sequence[int]) -> Dict[int, Selection]:
+    """Selections only (no attention) for the given tiles of one KV head.
+    q_head_rows: [T, G, d]."""
+    b = p.block_size
+    out = {}
+    for i in tiles:
+        q_tile = q_head_rows[i * b:(i + 1) * b]
+        C = i * b
+        Kc = Kc_all[:C // b]
+        s = prefill_tile_scores(q_tile, Kc, p) if C // b > 0 else np.zeros(0)
+        out[i] = select_topk(s, candidate_blocks(C, p), p.top_k)
+    return out

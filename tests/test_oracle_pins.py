@@ -1,0 +1,433 @@
+"""Pins of the float64 oracle against things other than itself.
+
+Each test checks the oracle against a closed form, an invariant the
+definitions imply, a library routine the definition reduces to in a special
+case, brute force on tiny inputs, or the hand-worked examples in
+tests/golden/hand_worked.json.  No expected value here comes from the CUDA
+library.  A final group plants plausible mistakes in (a copy of) the oracle
+and checks that some pin catches each one.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import logsumexp
+
+from oracle import sparse_attn_oracle as orc
+from top_block_sparse_b200.inputs import WORKLOADS, make_inputs
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+GOLD = json.load(open(os.path.join(HERE, "golden", "hand_worked.json")))["cases"]
+
+
+def P(w, **kw):
+    p = orc.OracleParams(block_size=w.block_size, top_k=w.top_k,
+                         sink_keys=w.sink_keys, window_keys=w.window_keys,
+                         pool=w.pool)
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- golden ---
+
+def _case(name):
+    return next(c for c in GOLD if c["name"] == name)
+
+
+@pytest.mark.parametrize("name", ["decode_k1", "decode_k2", "decode_tie"])
+def test_hand_worked_decode(name):
+    c = _case(name)
+    pr = c["params"]
+    p = orc.OracleParams(block_size=pr["block_size"], top_k=pr["top_k"],
+                         sink_keys=pr["sink_keys"], window_keys=pr["window_keys"])
+    K = np.array(c["K"], float)
+    V = np.array(c["V"], float)
+    q = np.array(c["q"], float)[None]          # [n_q=1, G=1, d]
+    r = orc.decode_pair(q, K, V, pr["C"], p)
+    e = c["expect"]
+    if "Kc" in e:
+        np.testing.assert_allclose(r["Kc"], e["Kc"], atol=1e-15)
+    if "scores" in e:
+        np.testing.assert_allclose(r["scores"], e["scores"], atol=1e-15)
+    if "candidates" in e:
+        assert r["candidates"] == e["candidates"]
+    assert r["sel"].selected == e["selected"]
+    if "positions" in e:
+        assert r["positions"][0].tolist() == e["positions"]
+    np.testing.assert_allclose(r["O"][0, 0], e["O"], rtol=1e-14, atol=1e-14)
+    assert abs(r["lse"][0, 0] - e["lse"]) < 1e-14
+
+
+def test_hand_worked_lsa_centroid():
+    c = _case("lsa_centroid")
+    K = np.array(c["K"], float)
+    cent = orc.pool_lsa(K, c["params"]["block_size"], c["params"]["pool_stride"])
+    np.testing.assert_allclose(cent[0], c["expect"]["centroid"], atol=1e-15)
+    p = orc.OracleParams(block_size=8, top_k=1, sink_keys=0, window_keys=0, pool="lsa")
+    s = orc.block_scores(np.array(c["qbar"], float), cent, p)
+    assert abs(s[0] - c["expect"]["score"]) < 1e-15
+
+
+# ----------------------------------------------------------- compression ---
+
+def test_pool_mean_equals_library_avg_pool():
+    """Non-overlapping mean pooling is avg_pool1d with kernel = stride = b
+    (a partial trailing block is dropped by both)."""
+    K = rng(1).standard_normal((1000, 16))
+    ref = torch.nn.functional.avg_pool1d(torch.from_numpy(K).T[None], 64, 64)[0].T
+    got = orc.pool_mean(K, 64)
+    assert got.shape == (15, 16)
+    np.testing.assert_allclose(got, ref.numpy(), atol=1e-14)
+
+
+def test_pool_mean_invariants():
+    r = rng(2)
+    K = r.standard_normal((256, 8))
+    base = orc.pool_mean(K, 32)
+    # permuting keys inside a block leaves the compressed key unchanged
+    Kp = K.copy()
+    for j in range(8):
+        Kp[j * 32:(j + 1) * 32] = Kp[j * 32 + r.permutation(32)]
+    np.testing.assert_allclose(orc.pool_mean(Kp, 32), base, atol=1e-14)
+    # a block of identical keys compresses to that key; b = 1 is the identity
+    x = r.standard_normal(8)
+    assert np.allclose(orc.pool_mean(np.tile(x, (32, 1)), 32)[0], x, atol=1e-15)
+    np.testing.assert_array_equal(orc.pool_mean(K, 1), K)
+
+
+def test_pool_lsa_invariants():
+    r = rng(3)
+    K = r.standard_normal((2048, 16))
+    c = orc.pool_lsa(K, 512, 4)
+    assert c.shape == (4, 16)
+    np.testing.assert_allclose(np.linalg.norm(c, axis=1), 1.0, atol=1e-14)
+    # step (1) normalises every raw key: positive per-key scaling changes nothing
+    a = r.uniform(0.01, 100.0, size=(2048, 1))
+    np.testing.assert_allclose(orc.pool_lsa(K * a, 512, 4), c, atol=1e-13)
+    # the pool-key sums are plain sums: centroid = normalise(sum of unit keys)
+    unit = K / np.linalg.norm(K, axis=1, keepdims=True)
+    direct = unit.reshape(4, 512, 16).sum(1)
+    direct /= np.linalg.norm(direct, axis=1, keepdims=True)
+    np.testing.assert_allclose(c, direct, atol=1e-13)
+    # keys all pointing one way -> that direction; negation flips the sign
+    x = r.standard_normal(16)
+    same = np.outer(r.uniform(0.5, 2, 512), x)
+    np.testing.assert_allclose(orc.pool_lsa(same, 512)[0], x / np.linalg.norm(x), atol=1e-14)
+    np.testing.assert_allclose(orc.pool_lsa(-K, 512, 4), -c, atol=1e-13)
+
+
+# --------------------------------------------------------------- scoring ---
+
+def test_scores_brute_force_loops():
+    """s_j = scale * (1/b) * sum_{t in block j} sum_h q_h . K_t, written as
+    explicit Python loops over heads, keys and coordinates."""
+    r = rng(4)
+    G, d, b, T = 3, 8, 4, 32
+    q = r.standard_normal((G, d))
+    K = r.standard_normal((T, d))
+    p = orc.OracleParams(block_size=b, top_k=2, sink_keys=0, window_keys=0)
+    s = orc.block_scores(orc.index_query(q), orc.pool_mean(K, b), p)
+    scale = 1 / math.sqrt(d)
+    for j in range(T // b):
+        acc = 0.0
+        for t in range(j * b, (j + 1) * b):
+            for h in range(G):
+                for c in range(d):
+                    acc += q[h, c] * K[t, c]
+        assert abs(s[j] - scale * acc / b) < 1e-13
+
+
+def test_lsa_scores_are_cosines():
+    r = rng(5)
+    K = r.standard_normal((4096, 16))
+    p = orc.OracleParams(block_size=512, top_k=2, sink_keys=4, window_keys=512, pool="lsa")
+    c = orc.compress(K, p)
+    qbar = r.standard_normal(16)
+    s = orc.block_scores(qbar, c, p)
+    assert np.all(np.abs(s) <= 1 + 1e-15)
+    np.testing.assert_allclose(orc.block_scores(7.5 * qbar, c, p), s, atol=1e-15)
+    assert abs(orc.block_scores(c[2] * 3.0, c, p)[2] - 1.0) < 1e-14
+
+
+# -------------------------------------------------- candidates and top-k ---
+
+def _candidates_by_key_enumeration(C, p):
+    b = p.block_size
+    s_end, w_begin = min(p.sink_keys, C), max(C - p.window_keys, 0)
+    return [j for j in range(C // b)
+            if any(not (t < s_end or t >= w_begin) for t in range(j * b, (j + 1) * b))]
+
+
+@pytest.mark.parametrize("C,b,S,W", [(4096, 64, 64, 128), (1000, 64, 64, 256), (640, 64, 100, 70),
+                                     (300, 64, 0, 0), (64, 64, 64, 64), (2048, 512, 4, 512),
+                                     (130, 64, 200, 10)])
+def test_candidates_match_key_enumeration(C, b, S, W):
+    p = orc.OracleParams(block_size=b, top_k=1, sink_keys=S, window_keys=W)
+    assert orc.candidate_blocks(C, p) == _candidates_by_key_enumeration(C, p)
+
+
+def test_candidate_counts_of_workloads():
+    w = WORKLOADS
+    assert len(orc.candidate_blocks(4096, P(w["tiny_decode"]))) == 61
+    c1 = orc.candidate_blocks(32768, P(w["decode_32k"]))
+    assert len(c1) == 507 and c1[0] == 1 and c1[-1] == 507
+    c3 = orc.candidate_blocks(1048576, P(w["decode_1m"]))
+    assert len(c3) == 2047 and c3[0] == 0          # block 0 only partly sink
+    assert len(orc.candidate_blocks(16384, P(w["draft_chunk_16k"]))) == 251
+    pp = P(w["prefill_64k"])
+    for i in [0, 5, 6, 7, 100, 1023]:
+        assert len(orc.candidate_blocks(64 * i, pp)) == max(0, i - 5)
+
+
+def test_topk_matches_exhaustive_rank_count():
+    """Selected iff fewer than k candidates beat it, where i beats j when
+    s_i > s_j or (s_i == s_j and i < j); scores drawn with many exact ties."""
+    r = rng(6)
+    for trial in range(300):
+        nb = int(r.integers(1, 13))
+        s = r.integers(-3, 4, size=nb).astype(float) / 2.0
+        cand = sorted(r.choice(nb, size=int(r.integers(0, nb + 1)), replace=False).tolist())
+        for k in range(0, nb + 2):
+            sel = orc.select_topk(s, cand, k).selected
+            want = [j for j in cand
+                    if sum(1 for i in cand if s[i] > s[j] or (s[i] == s[j] and i < j)) < k]
+            assert sel == sorted(want)
+
+
+def test_topk_subset_maximises_score_sum():
+    """Brute force over all k-subsets: the chosen set has the largest total
+    score (distinct scores, so the optimum is unique)."""
+    r = rng(7)
+    for trial in range(50):
+        nb = 9
+        s = r.standard_normal(nb)
+        cand = list(range(nb))
+        for k in range(1, 5):
+            best = max(itertools.combinations(cand, k), key=lambda c: sum(s[list(c)]))
+            assert orc.select_topk(s, cand, k).selected == sorted(best)
+
+
+def test_near_tie_flag():
+    s = np.array([1.0, 0.99999999, 0.5, 2.0])
+    sel = orc.select_topk(s, [0, 1, 2, 3], 1)
+    assert sel.selected == [3] and sel.near_tie is False and sel.gap == 1.0
+    sel = orc.select_topk(s, [0, 1, 2, 3], 2)
+    assert sel.selected == [0, 3] and sel.near_tie is True
+    sel = orc.select_topk(s, [0, 1, 2], 1)
+    assert sel.selected == [0] and sel.near_tie is True
+    sel = orc.select_topk(s, [0, 1, 2], 3)
+    assert sel.selected == [0, 1, 2] and sel.gap is None and sel.near_tie is False
+
+
+# ----------------------------------------------------------- attention ---
+
+def _slab(inp, b, h, G, dt=np.float64):
+    q = inp["Q"][b, :, h * G:(h + 1) * G].double().numpy()
+    K = inp["K"][b, h].double().numpy()
+    V = inp["V"][b, h].double().numpy()
+    return q, K, V
+
+
+def _sdpa(q, K, V, n_keys):
+    """Library dense attention of one query over keys [0, n_keys)."""
+    qt = torch.from_numpy(q)[None, None, None]          # [1,1,1,d]
+    kt = torch.from_numpy(K[:n_keys])[None, None]
+    vt = torch.from_numpy(V[:n_keys])[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)[0, 0, 0].numpy()
+
+
+def test_needles_selected_tiny_decode():
+    w = WORKLOADS["tiny_decode"]
+    inp = make_inputs(w, seed=11)
+    q, K, V = _slab(inp, 0, 0, w.group)
+    r = orc.decode_pair(q, K, V, w.ctx_len, P(w))
+    assert set(inp["needles"][0, 0].tolist()) <= set(r["sel"].selected)
+    assert len(r["sel"].selected) == 8
+    assert all(len(pz) == 705 for pz in r["positions"])       # (8+1+2)*64 + 1
+
+
+def test_needles_selected_decode_32k_slab():
+    w = WORKLOADS["decode_32k"].scaled(batch=1, num_q_heads=8, num_kv_heads=2)
+    inp = make_inputs(w, seed=12)
+    for h in range(2):
+        q, K, V = _slab(inp, 0, h, w.group)
+        r = orc.decode_pair(q, K, V, w.ctx_len, P(w))
+        assert set(inp["needles"][0, h].tolist()) <= set(r["sel"].selected)
+        assert len(r["positions"][0]) == 2369                 # (32+1+4)*64 + 1
+        np.testing.assert_allclose(r["wsum"], 1.0, atol=1e-12)
+
+
+def test_sink_window_always_attended_and_chunk_causal():
+    w = WORKLOADS["draft_chunk_16k"].scaled(batch=1, num_kv_heads=1, num_q_heads=2, ctx_len=4096)
+    inp = make_inputs(w, seed=13)
+    q, K, V = _slab(inp, 0, 0, w.group)
+    p = P(w)
+    r = orc.decode_pair(q, K, V, w.ctx_len, p)
+    C = w.ctx_len
+    for j, pos in enumerate(r["positions"]):
+        s = set(pos.tolist())
+        assert set(range(64)) <= s and set(range(C - 256, C)) <= s
+        assert set(range(C, C + j + 1)) <= s and max(s) == C + j
+        assert len(pos) == (16 + 1 + 4) * 64 + j + 1
+
+
+@pytest.mark.parametrize("pool", ["mean", "lsa"])
+def test_dense_equivalence_when_topk_covers_all(pool):
+    """With k >= #candidates the sparse result is dense causal attention
+    (the special case S = all-ones causal of the masked softmax)."""
+    b = 64 if pool == "mean" else 512
+    w = WORKLOADS["draft_chunk_16k"].scaled(batch=1, num_kv_heads=1, num_q_heads=3,
+                                            ctx_len=2048 + 37, block_size=b, pool=pool)
+    inp = make_inputs(w, seed=14)
+    q, K, V = _slab(inp, 0, 0, w.group)
+    p = P(w, top_k=10_000)
+    r = orc.decode_pair(q, K, V, w.ctx_len, p)
+    for j in range(w.n_q):
+        for g in range(w.group):
+            ref = _sdpa(q[j, g], K, V, w.ctx_len + j + 1)
+            np.testing.assert_allclose(r["O"][j, g], ref, atol=1e-12)
+            z = K[:w.ctx_len + j + 1] @ q[j, g] / math.sqrt(128)
+            assert abs(r["lse"][j, g] - logsumexp(z)) < 1e-12
+
+
+def test_block_size_one_full_window_is_dense():
+    r_ = rng(8)
+    C, d = 50, 8
+    K = r_.standard_normal((C + 1, d))
+    V = r_.standard_normal((C + 1, d))
+    q = r_.standard_normal((1, 2, d))
+    p = orc.OracleParams(block_size=1, top_k=0, sink_keys=0, window_keys=C)
+    r = orc.decode_pair(q, K, V, C, p)
+    for g in range(2):
+        np.testing.assert_allclose(r["O"][0, g], _sdpa(q[0, g], K, V, C + 1), atol=1e-13)
+
+
+def test_constant_values_and_equal_keys():
+    w = WORKLOADS["tiny_decode"]
+    inp = make_inputs(w, seed=15)
+    q, K, V = _slab(inp, 0, 0, w.group)
+    p = P(w)
+    Vc = np.tile(np.arange(128, dtype=float), (K.shape[0], 1))
+    r = orc.decode_pair(q, K, Vc, w.ctx_len, p)
+    np.testing.assert_allclose(r["O"], np.broadcast_to(Vc[0], r["O"].shape), atol=1e-12)
+    Ke = np.tile(K[0], (K.shape[0], 1))
+    r2 = orc.decode_pair(q, Ke, V, w.ctx_len, p)
+    pos = r2["positions"][0]
+    np.testing.assert_allclose(r2["O"][0, 0], V[pos].mean(axis=0), atol=1e-12)
+
+
+def test_attention_pure_python_loops():
+    """Brute-force softmax with explicit loops on a tiny case."""
+    r_ = rng(9)
+    C, d = 24, 4
+    K = r_.standard_normal((C + 2, d))
+    V = r_.standard_normal((C + 2, d))
+    q = r_.standard_normal((2, 1, d))
+    p = orc.OracleParams(block_size=4, top_k=2, sink_keys=4, window_keys=4)
+    r = orc.decode_pair(q, K, V, C, p)
+    for j in range(2):
+        pos = r["positions"][j].tolist()
+        z = [sum(q[j, 0, c] * K[t, c] for c in range(d)) / math.sqrt(d) for t in pos]
+        m = max(z)
+        e = [math.exp(x - m) for x in z]
+        tot = sum(e)
+        for c in range(d):
+            o = sum(e[i] * V[t, c] for i, t in enumerate(pos)) / tot
+            assert abs(o - r["O"][j, 0, c]) < 1e-13
+        assert abs(m + math.log(tot) - r["lse"][j, 0]) < 1e-13
+
+
+# --------------------------------------------------------------- prefill ---
+
+def test_prefill_tile_score_is_max_of_row_scores():
+    r_ = rng(10)
+    G, d, b = 4, 16, 8
+    K = r_.standard_normal((10 * b, d))
+    q_tile = r_.standard_normal((b, G, d))
+    p = orc.OracleParams(block_size=b, top_k=2, sink_keys=b, window_keys=2 * b)
+    Kc = orc.pool_mean(K, b)[:7]
+    s = orc.prefill_tile_scores(q_tile, Kc, p)
+    for j in range(7):
+        rows = [sum(float(q_tile[r, h] @ Kc[j]) for h in range(G)) / math.sqrt(d) for r in range(b)]
+        assert abs(s[j] - max(rows)) < 1e-13
+
+
+def test_prefill_dense_equivalence_and_needles():
+    w = WORKLOADS["prefill_64k"].scaled(n_q=1024 + 40, num_q_heads=2, num_kv_heads=1, n_needles=3)
+    inp = make_inputs(w, seed=16)
+    q = inp["Q"][0, :, 0:2].double().numpy()             # [T, G, d]
+    K = inp["K"][0, 0].double().numpy()
+    V = inp["V"][0, 0].double().numpy()
+    T = w.n_q
+    # dense equivalence: k covers every candidate
+    p = P(w, top_k=10_000)
+    Kc = orc.compress(K, p)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).permute(1, 0, 2)[None],
+        torch.from_numpy(K)[None, None].expand(1, 2, T, 128),
+        torch.from_numpy(V)[None, None].expand(1, 2, T, 128), is_causal=True)[0].permute(1, 0, 2).numpy()
+    for i in [0, 3, 7, 16]:
+        rows = slice(i * 64, min((i + 1) * 64, T))
+        r = orc.prefill_tile(q[rows], K, V, i, p, Kc)
+        np.testing.assert_allclose(r["O"], ref[rows], atol=1e-12)
+        np.testing.assert_allclose(r["wsum"], 1.0, atol=1e-12)
+    # the last (ragged) tile selects every needle with the real k
+    p = P(w)
+    i = (T - 1) // 64
+    r = orc.prefill_tile(q[i * 64:], K, V, i, p, Kc)
+    assert set(inp["needles"][0, 0].tolist()) <= set(r["sel"].selected)
+    assert len(r["sel"].selected) == min(64, i - 5)
+
+
+# ---------------------------------------------- planted-mistake checks ---
+
+def _fails(fn):
+    try:
+        fn()
+    except AssertionError:
+        return True
+    return False
+
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    """Each plausible mistake planted in the oracle makes some pin fail."""
+    mistakes = {
+        "mean instead of sum over the GQA group":
+            ("index_query", lambda qg: np.asarray(qg, float).mean(axis=0),
+             test_scores_brute_force_loops),
+        "LSA pooling without key normalisation":
+            ("pool_lsa", lambda K, b, stride=4: orc._normalise(
+                np.asarray(K, float)[:(len(K) // b) * b].reshape(len(K) // b, b, -1).sum(1)),
+             test_pool_lsa_invariants),
+        "ties broken towards the higher index":
+            ("select_topk", lambda s, c, k: orc.Selection(
+                sorted(sorted(c, key=lambda j: (-float(s[j]), -j))[:min(k, len(c))]), len(c), None, None, False),
+             test_topk_matches_exhaustive_rank_count),
+        "window dropped from the attended set":
+            ("attended_positions", lambda C, p, sel, last: np.flatnonzero(np.isin(
+                np.arange(last + 1),
+                list(range(min(p.sink_keys, C))) + [t for j in sel for t in range(j * p.block_size, (j + 1) * p.block_size)]
+                + list(range(C, last + 1)))),
+             test_sink_window_always_attended_and_chunk_causal),
+    }
+    for what, (name, bad, pin) in mistakes.items():
+        with monkeypatch.context() as m:
+            m.setattr(orc, name, bad)
+            assert _fails(pin), f"no pin caught: {what}"
+    # scale 1/d instead of 1/sqrt(d): the hand-worked example catches it
+    with monkeypatch.context() as m:
+        m.setattr(orc, "softmax_scale", lambda d, p: 1.0 / d)
+        assert _fails(lambda: test_hand_worked_decode("decode_k1"))
+    # summed chunk queries instead of the chunk's first query for selection
+    with monkeypatch.context() as m:
+        m.setattr(orc, "index_query", lambda qg: np.asarray(qg, float).sum(axis=0) * 0.0)
+        assert _fails(test_needles_selected_tiny_decode)
