@@ -1,0 +1,428 @@
+"""Benchmark of the sparse-attention decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode_32k] [--no-cpu-baseline] [--no-prefill]
+
+Workload (default): batched decode, batch 32, 32 query / 8 KV heads, d = 128,
+context T = 32768, bf16 KV cache with fp32 accumulation, block 64, top-k 32 +
+1 sink block + 4-block window (2369 keys per query), synthetic N(0,1) inputs
+with 16 planted needle blocks per (sequence, KV head).  One step = one
+``sa_sparse_attn_decode`` call (scoring + top-k kernel, then the split-KV
+sparse attention kernel) over the whole batch, compressed keys maintained.
+
+Timing: W untimed warm-up steps, then K steps; before every step a 256 MB
+buffer is written to flush the 126 MB L2, and each step is bracketed by CUDA
+events on the launching stream (the flush is outside the events).  Multi-GPU
+(torchrun): every rank runs its own batch (weak scaling, no collective on the
+data path); the per-rank device times are max-reduced.
+
+Printed: one JSON line (rank 0).  ``value`` = sequences decoded per second
+(whole job).  Also: achieved HBM GB/s of the step and of the attention kernel
+(its roofline against the measured copy bandwidth), the end-to-end number
+through the C ABI with host buffers, clocks sampled during the timed region,
+and the float64 CPU oracle timed on a bounded sample (rank 0, N = 1).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from top_block_sparse_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ----------------------------------------------------------------- helpers --
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0) or 0), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def decode_bytes(w) -> dict:
+    """Algorithmic HBM bytes of one decode step (per the whole batch)."""
+    el = 2 if w.dtype == "bf16" else 4
+    b = w.block_size
+    C = w.ctx_len
+    s_end = min(w.sink_keys, C)
+    w_begin = max(C - w.window_keys, s_end)
+    nb = C // b
+    cand = sum(1 for j in range(nb) if j * b < w_begin and (j + 1) * b > s_end)
+    k = min(w.top_k, cand)
+    keys = s_end + k * b + (C + w.n_q - w_begin)       # block keys inside sink/window are disjoint here
+    pairs = w.batch * w.num_kv_heads
+    kv = pairs * keys * w.head_dim * el * 2
+    kc = pairs * nb * w.head_dim * 4
+    q = w.batch * w.n_q * w.num_q_heads * w.head_dim * el
+    o = w.batch * w.n_q * w.num_q_heads * w.head_dim * el
+    return dict(kv=kv, kc=kc, q=q, o=o, keys_per_query=keys, attn=kv + q + o, step=kv + kc + 2 * q + o)
+
+
+def src_hash(*names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "top_block_sparse_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_file: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(path))[kernel_file]
+        if d["src_sha"] == src_hash(kernel_file, "common.cuh"):
+            return float(d["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def timed_steps(fn, steps, warmup, stream, flush_buf):
+    """W warm-ups, then K steps each preceded by an L2 flush; returns the
+    per-step device times (ms) from CUDA events on `stream`."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for s, e in evs:
+            flush_buf.fill_(1)
+            s.record(stream)
+            fn()
+            e.record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in evs]
+
+
+# ------------------------------------------------------------- CPU oracle --
+
+def oracle_sample(w, inp_cpu_pairs, n_pairs_total):
+    """Times the float64 oracle (one thread) on the sampled pairs; returns
+    (seconds per full step extrapolated, seconds measured, pairs)."""
+    from threadpoolctl import threadpool_limits
+    from oracle import sparse_attn_oracle as orc
+    p = orc.OracleParams(block_size=w.block_size, top_k=w.top_k, sink_keys=w.sink_keys,
+                         window_keys=w.window_keys, pool=w.pool)
+    with threadpool_limits(limits=1):
+        # compressed keys are maintained state of a decode step, as on the GPU
+        Kcs = [orc.compress(K[:w.ctx_len], p) for (_, K, _) in inp_cpu_pairs]
+        t0 = time.perf_counter()
+        for (q, K, V), Kc in zip(inp_cpu_pairs, Kcs):
+            orc.decode_pair(q, K, V, w.ctx_len, p, Kc=Kc)
+        dt = time.perf_counter() - t0
+    per_pair = dt / len(inp_cpu_pairs)
+    return per_pair * n_pairs_total, dt, len(inp_cpu_pairs)
+
+
+def cpu_pairs(w, inp, n):
+    G = w.group
+    out = []
+    pairs = [(b, h) for b in range(w.batch) for h in range(w.num_kv_heads)]
+    step = max(1, len(pairs) // n)
+    for (b, h) in pairs[::step][:n]:
+        q = inp["Q"][b, :, h * G:(h + 1) * G].double().cpu().numpy()
+        K = inp["K"][b, h, :w.kv_len].double().cpu().numpy()
+        V = inp["V"][b, h, :w.kv_len].double().cpu().numpy()
+        out.append((q, K, V))
+    return out
+
+
+def cpu_info():
+    model = ""
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except Exception:
+        pass
+    return model, os.cpu_count()
+
+
+# ------------------------------------------------------------------- arms ---
+
+def run_reference(args, w, rank, world):
+    """The float64 oracle on the host cores: each step is a bounded sample of
+    the workload's (sequence, KV head) pairs; value extrapolated per step."""
+    if rank != 0:
+        return None
+    inp = make_inputs(w.scaled(batch=1), seed=1000 + 1, device="cpu")
+    n = min(args.ref_pairs, w.num_kv_heads)
+    pairs = cpu_pairs(w.scaled(batch=1), inp, n)
+    pairs_total = w.batch * w.num_kv_heads
+    for _ in range(args.warmup):
+        oracle_sample(w, pairs[:1], pairs_total)
+    times = []
+    for _ in range(args.steps):
+        full, _, _ = oracle_sample(w, pairs, pairs_total)
+        times.append(full)
+    sec = statistics.mean(times)
+    q_per_s = w.batch * w.n_q / sec
+    model, ncpu = cpu_info()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": q_per_s, "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w),
+        "cpu_baseline": {"value": q_per_s, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{len(pairs)} of {pairs_total} (sequence, KV head) pairs per step, "
+                                   f"extrapolated to the full batch; {model}, {ncpu} host cores, 1 used"},
+        "e2e": {"value": q_per_s, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+METRIC = "sparse-attn decode queries/s + achieved HBM GB/s at T=32k; prefill TFLOP/s"
+
+
+def config_of(w):
+    return {"workload": f"{w.name}: batched decode B={w.batch}, Hq={w.num_q_heads}, Hkv={w.num_kv_heads}, "
+                        f"d={w.head_dim}, T={w.ctx_len}, {w.dtype} KV, block {w.block_size}, top-k {w.top_k} "
+                        f"+ sink {w.sink_keys} keys + window {w.window_keys} keys",
+            "batch": w.batch, "seq_len": w.ctx_len, "n_q": w.n_q, "num_q_heads": w.num_q_heads,
+            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+            "top_k": w.top_k, "sink_keys": w.sink_keys, "window_keys": w.window_keys,
+            "l2": "256 MB buffer written before every timed step (outside the step's events)",
+            "parallelism": "replicas (weak scaling)"}
+
+
+def run_ours(args, w, rank, world, local_rank):
+    from top_block_sparse_b200 import sa
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    inp = make_inputs(w, seed=1000 + 1 + rank, device=dev)
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    p = sa.params_for(w)
+    nb = w.ctx_len // w.block_size
+    Kc = torch.empty((w.batch, w.num_kv_heads, nb, w.head_dim), device=dev, dtype=torch.float32)
+    O = torch.empty((w.batch, w.n_q, w.num_q_heads, w.head_dim), device=dev, dtype=Q.dtype)
+    lse = torch.empty((w.batch, w.n_q, w.num_q_heads), device=dev, dtype=torch.float32)
+    idx = torch.empty((w.batch, w.num_kv_heads, w.top_k), device=dev, dtype=torch.int32)
+    ws = sa.alloc_workspace(p, sa.SA_OP_DECODE, device=dev)
+    ws_g = sa.alloc_workspace(p, sa.SA_OP_GIVEN_IDX, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
+    with torch.cuda.stream(stream):
+        sa.pool_keys(p, K, Kc, stream=stream)
+    torch.cuda.synchronize()
+
+    def step():
+        sa.sparse_attn_decode(p, Q, K, V, Kc, O, lse, idx, ws, stream=stream)
+
+    def attn_only():
+        sa.sparse_attn_given_idx(p, Q, K, V, idx, O, lse, ws_g, stream=stream)
+
+    def pool_only():
+        sa.pool_keys(p, K, Kc, stream=stream)
+
+    # --- the timed decode steps -------------------------------------------
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        step_ms = timed_steps(step, args.steps, args.warmup, stream, flush)
+    if sa.read_status(ws, stream) != sa.SA_OK:
+        raise RuntimeError("device status word set during the timed steps")
+    ms = sum(step_ms) / len(step_ms)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    # --- kernels alone (roofline), rank-local -----------------------------
+    attn_ms = statistics.mean(timed_steps(attn_only, max(50, args.steps // 4), 3, stream, flush))
+    pool_ms = statistics.mean(timed_steps(pool_only, 10, 2, stream, flush))
+    # --- end to end through the C ABI with host buffers -------------------
+    e2e = e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush)
+    if world > 1:
+        t = torch.tensor([e2e["ms"]], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e["ms"] = float(t.item())
+    if rank != 0:
+        return None
+
+    hbm, tfl, tfl_s, src = peaks()
+    by = decode_bytes(w)
+    q_per_s = world * w.batch * w.n_q / (ms * 1e-3)
+    attn_gbs = by["attn"] / (attn_ms * 1e-3) / 1e9
+    step_gbs = by["step"] / (ms * 1e-3) / 1e9
+    pool_bytes = w.batch * w.num_kv_heads * (nb * w.block_size * w.head_dim * 2 + nb * w.head_dim * 4)
+    line = {
+        "metric": METRIC, "value": q_per_s, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) + needle blocks)",
+        "config": config_of(w),
+        "decode_hbm_gbs": step_gbs, "decode_hbm_frac": step_gbs / hbm,
+        "decode_bytes_per_step": by["step"], "keys_per_query": by["keys_per_query"],
+        "roofline": {"bound": "hbm", "kernel": "decode_attn_kernel (split-KV sparse attention)",
+                     "achieved": attn_gbs, "peak": hbm, "unit": "GB/s", "frac": attn_gbs / hbm,
+                     "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs, burst copy)" if src == "measured" else src,
+                     "algorithmic_bytes_per_launch": by["attn"], "launch_ms": attn_ms,
+                     "traffic": profiled_traffic("decode_attn.cu"),
+                     "frac_of_spec_8tbs": attn_gbs / 8000.0},
+        "pool": {"kernel": "pool_kernel", "ms": pool_ms, "gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
+                 "note": "compression runs once after prefill / when a block fills; not part of a decode step"},
+        "e2e": {"value": world * w.batch * w.n_q / (e2e["ms"] * 1e-3), "unit": "queries/s",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                "note": "per step: pinned host -> device copy of the new tokens' Q, K, V rows, the decode "
+                        "call through the C ABI, device -> pinned host copy of O; the KV cache and the "
+                        "compressed keys stay resident in HBM"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    return line
+
+
+def e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush):
+    from top_block_sparse_b200 import sa
+    C = w.ctx_len
+    hQ = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
+    hK = torch.empty((w.batch, w.num_kv_heads, w.n_q, w.head_dim), dtype=K.dtype, pin_memory=True)
+    hV = torch.empty_like(hK, pin_memory=True)
+    hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    hQ.copy_(Q.cpu())
+    hK.copy_(K[:, :, C:C + w.n_q].cpu())
+    hV.copy_(V[:, :, C:C + w.n_q].cpu())
+    Kn = K[:, :, C:C + w.n_q]
+    Vn = V[:, :, C:C + w.n_q]
+
+    def one():
+        Q.copy_(hQ, non_blocking=True)
+        Kn.copy_(hK, non_blocking=True)
+        Vn.copy_(hV, non_blocking=True)
+        sa.sparse_attn_decode(p, Q, K, V, Kc, O, lse, idx, ws, stream=stream)
+        hO.copy_(O, non_blocking=True)
+
+    n = max(50, args.steps // 4)
+    with torch.cuda.stream(stream):
+        ms = statistics.mean(timed_steps(one, n, args.warmup, stream, flush))
+    el = Q.element_size()
+    h2d = hQ.numel() * el + 2 * hK.numel() * el
+    return {"ms": ms, "h2d": h2d, "d2h": hO.numel() * O.element_size()}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode_32k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-pairs", type=int, default=16)
+    ap.add_argument("--ref-pairs", type=int, default=4)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        line = run_reference(args, w, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, w, rank, world, local_rank)
+        if line is not None and world == 1 and not args.no_cpu_baseline:
+            inp = make_inputs(w.scaled(batch=2), seed=1000 + 1, device="cuda")
+            pairs = cpu_pairs(w.scaled(batch=2), inp, args.cpu_pairs)
+            full, dt, n = oracle_sample(w, pairs, w.batch * w.num_kv_heads)
+            model, ncpu = cpu_info()
+            line["cpu_baseline"] = {
+                "value": w.batch * w.n_q / full, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                "sample": f"float64 oracle on {n} of {w.batch * w.num_kv_heads} (sequence, KV head) pairs "
+                          f"({dt:.1f} s), extrapolated to the full step; {model}, {ncpu} host cores, 1 used"}
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

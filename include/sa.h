@@ -1,0 +1,197 @@
+/*
+ * sa.h - C ABI of the B200 (sm_100a) indexer-driven top-k block-sparse
+ * attention library (libsa.so).
+ *
+ * The method (sources are web pages on it; each entry point cites the passage
+ * that defines its operation):
+ *   1. keys of every complete block of b keys are compressed: mean-pooled
+ *      (SparDA summary on hyper.ai 2606.04511, section "方法": keys are
+ *      average-pooled into compressed keys), or LSA-style: each key
+ *      L2-normalised, 4 consecutive unit keys summed into a pool key, the
+ *      block centroid = the normalised sum of its pool keys (LSA review,
+ *      §2.2);
+ *   2. one index query per (sequence, KV head) = the SUM of the query vectors
+ *      of the GQA group (LSA review §2.4; SparDA "方法": one forecast head per
+ *      GQA group) scores every compressed key: s_j = qbar.Kc_j * scale, or the
+ *      cosine (qbar/|qbar|).c_j for LSA centroids (LSA review §2.3);
+ *   3. the top-k candidate blocks (score descending, lower block id on ties)
+ *      are united with the sink keys [0, S) and the window keys [C-W, C)
+ *      (SparDA "方法": initial tokens + local sliding window + top-k blocks;
+ *      LSA review §2.3: 4 sink keys + 512 window keys; S3R review, section
+ *      "稀疏起草", KV-selection formula: recent window + top-K).  Blocks lying
+ *      wholly inside sink or window are not candidates; only complete blocks
+ *      of the context are;
+ *   4. softmax attention runs over the retained keys only (S3R review,
+ *      "稀疏起草", sparse-attention formula; PulseCol §3.1 eq. (1)-(2): logits
+ *      QK^T/sqrt(d_h), keys outside the mask get zero weight).  The n_q new
+ *      tokens sit at positions C..C+n_q-1 and token j also sees the new keys
+ *      C..C+j (a multi-token draft chunk keeps one selection, made from its
+ *      first query, for all its tokens: S3R review, "稀疏起草").
+ *
+ * Layouts (all row-major, contiguous, element strides implied):
+ *   K, V : [B, Hkv, kv_capacity, d]   dtype = params.dtype
+ *   Q    : [B, n_q, Hq, d]            dtype = params.dtype
+ *   O    : [B, n_q, Hq, d]            dtype = params.out_dtype
+ *   lse  : [B, n_q, Hq] float32, natural log of the softmax denominator
+ *   Kc   : [B, Hkv, nb, d] float32, nb = number of complete blocks
+ *          (decode: floor(ctx_len / b); prefill: floor(n_q / b))
+ *   idx  : decode / chunk: [B, Hkv, top_k] int32; prefill: [B, Hkv,
+ *          n_tiles, top_k] int32 with n_tiles = ceil(n_q / b).  Block ids in
+ *          ascending order, unused entries -1 at the end.
+ *   Query head h uses KV head h / (Hq / Hkv).
+ *
+ * Ownership: the caller allocates every buffer, including the workspace; the
+ * library allocates no device or host memory and keeps no state besides a
+ * per-thread error string and cached device attributes.  Every call is
+ * asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream).
+ * Pointers are device pointers unless stated; K, V, Q, O, Kc must be 16-byte
+ * aligned.
+ *
+ * Errors: arguments are validated on the host before any launch
+ * (SA_ERR_INVALID / SA_ERR_UNSUPPORTED / SA_ERR_WORKSPACE, with a message in
+ * sa_last_error()); a failed launch returns SA_ERR_CUDA.  Conditions found on
+ * the device (an out-of-range or repeated block id in a caller's index table,
+ * a bounded wait that ran out) set bits of a status word kept in the
+ * workspace; the affected block is skipped and sa_read_status() reports
+ * them.  No kernel traps or asserts.
+ */
+#ifndef SA_H_
+#define SA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID = 1,      /* bad argument (null, shape, alignment, range) */
+  SA_ERR_UNSUPPORTED = 2,  /* valid but not built (head_dim != 128, sizes above limits) */
+  SA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than sa_workspace_size() */
+  SA_ERR_INDEX = 4,        /* device: a caller's block id was out of range or repeated */
+  SA_ERR_CUDA = 5,         /* a CUDA launch or runtime call failed */
+  SA_ERR_TIMEOUT = 6       /* device: a bounded wait inside a kernel ran out */
+} sa_status;
+
+enum { SA_F32 = 0, SA_BF16 = 1 };                 /* element types */
+enum { SA_POOL_MEAN = 0, SA_POOL_LSA = 1 };       /* compression (step 1) */
+enum { SA_SEL_QUERY0 = 0, SA_SEL_TILE_MAX = 1 };  /* how the index query is formed */
+enum {                                            /* ops for sa_workspace_size */
+  SA_OP_SCORE_TOPK = 0,
+  SA_OP_GIVEN_IDX = 1,
+  SA_OP_DECODE = 2,
+  SA_OP_PREFILL = 3
+};
+
+/* Problem description shared by every entry point (88 bytes). */
+typedef struct sa_params {
+  int32_t batch;          /* B >= 1 */
+  int32_t num_q_heads;    /* Hq, a multiple of Hkv */
+  int32_t num_kv_heads;   /* Hkv >= 1 */
+  int32_t head_dim;       /* d; only 128 is built */
+  int64_t ctx_len;        /* C: keys cached before the new tokens (prefill: 0) */
+  int64_t kv_capacity;    /* token stride of K and V, >= ctx_len + n_q */
+  int32_t n_q;            /* new tokens per sequence (decode 1, draft chunk m, prefill T) */
+  int32_t block_size;     /* b: keys per selectable block (a multiple of 16) */
+  int32_t pool;           /* SA_POOL_MEAN or SA_POOL_LSA */
+  int32_t pool_stride;    /* LSA: raw keys per pool key (divides b); ignored for mean */
+  int32_t top_k;          /* k >= 0 blocks chosen by score */
+  int32_t dtype;          /* SA_F32 or SA_BF16: element type of Q, K, V */
+  int32_t out_dtype;      /* SA_F32 or SA_BF16: element type of O */
+  int32_t select;         /* SA_SEL_QUERY0: decode / chunk (index query of the
+                             chunk's first token); SA_SEL_TILE_MAX: causal
+                             prefill (query tiles of b rows, ctx_len == 0) */
+  int64_t sink_keys;      /* S >= 0 */
+  int64_t window_keys;    /* W >= 0 */
+  float softmax_scale;    /* <= 0 selects 1/sqrt(head_dim) */
+  int32_t reserved;       /* must be 0 */
+} sa_params;
+
+/* Version of this ABI (major * 100 + minor). */
+int32_t sa_version(void);
+
+/* Bytes of workspace `op` needs for `p` (0 if p is invalid).  The workspace
+ * also carries the device status word and self-resetting counters, so it
+ * must be zero-filled once before its first use (sa_workspace_init) and may
+ * then be reused by later calls on the same stream.  Calls that share one
+ * workspace must not overlap on the device. */
+size_t sa_workspace_size(const sa_params* p, int32_t op);
+
+/* Zero-fills `ws_bytes` bytes at device pointer `ws` on `stream`. */
+sa_status sa_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Step 1 (compression) for every complete block of the context:
+ * SA_POOL_MEAN: Kc[j] = (1/b) sum_{t=jb}^{jb+b-1} K[t] (SparDA "方法");
+ * SA_POOL_LSA : Kc[j] = normalise(sum over the block's pool keys), a pool
+ *               key being the sum of pool_stride consecutive L2-normalised
+ *               keys (LSA review §2.2).
+ * Blocks counted over ctx_len keys (prefill: over n_q keys).  Reads K,
+ * writes Kc (fp32, see layouts).  No workspace. */
+sa_status sa_pool_keys(const sa_params* p, const void* K, float* Kc, void* stream);
+
+/* Steps 2-3 (scoring and selection).  SA_SEL_QUERY0: one table row per
+ * (sequence, KV head) from the first new token's GQA-summed query.
+ * SA_SEL_TILE_MAX: one row per (sequence, KV head, query tile of b rows),
+ * the tile score of block j being the max over the tile's rows (reading of
+ * the pages, which do not fix the tile aggregation).  Writes idx (see
+ * layouts).  scores (optional, may be NULL): fp32 block scores,
+ * [B, Hkv, nb] for SA_SEL_QUERY0 or [B, Hkv, n_tiles, nb] for
+ * SA_SEL_TILE_MAX.  Kc may be NULL when the context holds no complete
+ * block. */
+sa_status sa_score_topk(const sa_params* p, const void* Q, const float* Kc,
+                        int32_t* idx, float* scores, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* Step 4 alone with the CALLER's index table (a page table of selected
+ * blocks, as LSA review §2.6 feeds its attention kernel).  idx holds
+ * idx_len entries per row (layout as above with top_k replaced by idx_len);
+ * entries are block ids in [0, nb) in strictly ascending order, -1 for none.
+ * Attended set per token = sink U window U listed blocks U new keys up to the
+ * token; keys of a listed block that lie in sink or window count once.  An
+ * entry is used only if it is in [0, nb) and larger than every earlier
+ * in-range entry of its row; any other entry except -1 sets SA_ERR_INDEX in
+ * the status word and is skipped.  Writes O and (if non-NULL) lse.  The
+ * workspace size reported for SA_OP_GIVEN_IDX assumes idx_len == top_k. */
+sa_status sa_sparse_attn_given_idx(const sa_params* p, const void* Q,
+                                   const void* K, const void* V,
+                                   const int32_t* idx, int32_t idx_len,
+                                   void* O, float* lse, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* Steps 2-4 for decode and draft chunks (select == SA_SEL_QUERY0) with the
+ * compressed keys Kc kept up to date by the caller (sa_pool_keys).  Writes
+ * O, lse (optional) and the index table (optional idx_out, [B, Hkv, top_k]). */
+sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q,
+                                const void* K, const void* V, const float* Kc,
+                                void* O, float* lse, int32_t* idx_out,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* Steps 1-4 for a causal prefill (select == SA_SEL_TILE_MAX, ctx_len == 0,
+ * n_q = T): pools K into Kc (caller-provided, [B, Hkv, floor(T/b), d] fp32),
+ * scores every query tile of b rows against the compressed keys of the
+ * blocks before it, selects per (tile, KV head) and runs causal sparse
+ * attention: tile i attends sink U window U selected U its own keys
+ * (causal).  Writes O, lse (optional), idx_out (optional). */
+sa_status sa_sparse_attn_prefill(const sa_params* p, const void* Q,
+                                 const void* K, const void* V, float* Kc,
+                                 void* O, float* lse, int32_t* idx_out,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, returns the worst device condition recorded in the
+ * workspace status word since the last call (SA_OK, SA_ERR_INDEX or
+ * SA_ERR_TIMEOUT) and clears it. */
+sa_status sa_read_status(void* ws, void* stream);
+
+/* Static name of a status code. */
+const char* sa_status_string(sa_status s);
+
+/* Message of the last error returned on the calling thread ("" if none). */
+const char* sa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_H_ */

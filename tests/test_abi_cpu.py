@@ -1,0 +1,113 @@
+"""CPU-only checks of the C ABI: the library loads without a GPU, exports
+every symbol include/sa.h declares, the params struct matches, and host-side
+validation rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from top_block_sparse_b200 import sa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = open(os.path.join(ROOT, "include", "sa.h")).read()
+
+FAKE = ctypes.c_void_p(0x10000)          # 16-byte aligned, never dereferenced
+FAKE_ODD = ctypes.c_void_p(0x10008)
+
+
+def declared_functions():
+    body = re.sub(r"/\*.*?\*/", "", HEADER, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z0-9_]+)\s*\(", body)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for must in ["sa_pool_keys", "sa_score_topk", "sa_sparse_attn_decode", "sa_sparse_attn_prefill",
+                 "sa_sparse_attn_given_idx"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(sa.lib_path())
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) <= set(sa.EXPORTED) | set(declared_functions())
+    assert sa.version() == 100
+
+
+def test_params_struct_layout():
+    assert ctypes.sizeof(sa.SaParams) == 88
+    assert sa.SaParams.sink_keys.offset == 64
+    assert sa.SaParams.softmax_scale.offset == 80
+
+
+def _p(**kw):
+    base = dict(batch=2, num_q_heads=8, num_kv_heads=2, ctx_len=4096, n_q=1, block_size=64,
+                top_k=8, sink_keys=64, window_keys=128, dtype="bf16")
+    base.update(kw)
+    return sa.make_params(**base)
+
+
+def _decode(p, ws_bytes=1 << 30, q=FAKE, kc=FAKE):
+    return sa.raw_call("sa_sparse_attn_decode", ctypes.byref(p), q, FAKE, FAKE, kc, FAKE, None, None,
+                       FAKE, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(head_dim=64), sa.SA_ERR_UNSUPPORTED),
+    (dict(num_q_heads=7), sa.SA_ERR_INVALID),
+    (dict(kv_capacity=100), sa.SA_ERR_INVALID),
+    (dict(block_size=40), sa.SA_ERR_INVALID),
+    (dict(top_k=-1), sa.SA_ERR_INVALID),
+    (dict(sink_keys=-1), sa.SA_ERR_INVALID),
+    (dict(n_q=0), sa.SA_ERR_INVALID),
+    (dict(n_q=5), sa.SA_ERR_UNSUPPORTED),       # 5 tokens x GQA 4 = 20 rows > 16
+    (dict(prefill=True), sa.SA_ERR_INVALID),     # decode entry point with the prefill selector
+])
+def test_validation_rejects(kw, status):
+    assert _decode(_p(**kw)) == status
+    assert sa.raw_call("sa_last_error").decode() != ""
+
+
+def test_validation_null_and_alignment():
+    p = _p()
+    assert sa.raw_call("sa_sparse_attn_decode", None, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
+                       1 << 30, None) == sa.SA_ERR_INVALID
+    assert _decode(p, q=None) == sa.SA_ERR_INVALID
+    assert _decode(p, q=FAKE_ODD) == sa.SA_ERR_INVALID
+    p2 = _p()
+    p2.reserved = 1
+    assert _decode(p2) == sa.SA_ERR_INVALID
+
+
+def test_workspace_too_small():
+    p = _p()
+    need = sa.workspace_size(p, sa.SA_OP_DECODE)
+    assert need > 0
+    assert _decode(p, ws_bytes=need - 1) == sa.SA_ERR_WORKSPACE
+    assert "workspace" in sa.raw_call("sa_last_error").decode()
+
+
+def test_workspace_sizes_grow_with_the_problem():
+    a = sa.workspace_size(_p(), sa.SA_OP_DECODE)
+    b = sa.workspace_size(_p(batch=8), sa.SA_OP_DECODE)
+    assert 0 < a < b
+    assert sa.workspace_size(_p(head_dim=64), sa.SA_OP_DECODE) == 0
+    assert sa.workspace_size(_p(), sa.SA_OP_GIVEN_IDX) > 0
+    assert sa.workspace_size(_p(), sa.SA_OP_SCORE_TOPK) > 0
+
+
+def test_given_idx_validation():
+    p = _p()
+    st = sa.raw_call("sa_sparse_attn_given_idx", ctypes.byref(p), FAKE, FAKE, FAKE, None, 4, FAKE, None,
+                     FAKE, 1 << 30, None)
+    assert st == sa.SA_ERR_INVALID                  # idx NULL with idx_len > 0
+    st = sa.raw_call("sa_sparse_attn_given_idx", ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, -2, FAKE, None,
+                     FAKE, 1 << 30, None)
+    assert st == sa.SA_ERR_INVALID
+
+
+def test_status_strings():
+    for code, name in [(0, "SA_OK"), (4, "SA_ERR_INDEX"), (6, "SA_ERR_TIMEOUT")]:
+        assert sa.raw_call("sa_status_string", code).decode() == name

@@ -1,0 +1,267 @@
+"""GPU parity of the decode / draft-chunk path against the float64 oracle.
+
+Every case draws seeded inputs on the GPU, runs the CUDA library through the
+C ABI, copies the same inputs to the host and runs the oracle on them.
+Bars (bf16 inputs, fp32 accumulation): max abs <= 5e-3 and relative L2 <=
+1e-2; fp32 inputs: max abs <= 1e-5.  Selected block sets must be identical
+except where the oracle's k-th/(k+1)-th gap is a near-tie (< 1e-4 |s_k|);
+such pairs are counted and reported.
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import (assert_close, compare_sets, errors, oracle_decode, oracle_params, slab)
+from oracle import sparse_attn_oracle as orc
+from top_block_sparse_b200.inputs import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+sa = pytest.importorskip("top_block_sparse_b200.sa")
+
+
+def dev_inputs(w, seed, kv_capacity=None):
+    return make_inputs(w, seed=seed, device="cuda", kv_capacity=kv_capacity)
+
+
+def run_pool(w, inp, p):
+    nb = w.ctx_len // w.block_size
+    Kc = torch.empty((w.batch, w.num_kv_heads, nb, 128), device="cuda", dtype=torch.float32)
+    sa.pool_keys(p, inp["K"], Kc)
+    return Kc
+
+
+def run_decode(w, inp, p, Kc, out_dtype=torch.float32):
+    O = torch.empty((w.batch, w.n_q, w.num_q_heads, 128), device="cuda", dtype=out_dtype)
+    lse = torch.empty((w.batch, w.n_q, w.num_q_heads), device="cuda", dtype=torch.float32)
+    idx = torch.empty((w.batch, w.num_kv_heads, w.top_k), device="cuda", dtype=torch.int32)
+    ws = sa.alloc_workspace(p, sa.SA_OP_DECODE)
+    sa.sparse_attn_decode(p, inp["Q"], inp["K"], inp["V"], Kc, O, lse, idx, ws)
+    assert sa.read_status(ws) == sa.SA_OK
+    return O, lse, idx, ws
+
+
+def all_pairs(w):
+    return [(b, h) for b in range(w.batch) for h in range(w.num_kv_heads)]
+
+
+def check_decode(w, seed, pairs=None, out_dtype=torch.float32, p_over=None):
+    inp = dev_inputs(w, seed)
+    p = sa.params_for(w, out_dtype="bf16" if out_dtype == torch.bfloat16 else "f32")
+    if p_over:
+        for k, v in p_over.items():
+            setattr(p, k, v)
+    Kc = run_pool(w, inp, p)
+    O, lse, idx, _ = run_decode(w, inp, p, Kc, out_dtype)
+    torch.cuda.synchronize()
+    pairs = pairs or all_pairs(w)
+    op = oracle_params(w, **({"top_k": p_over["top_k"]} if p_over and "top_k" in p_over else {}))
+    ref = oracle_decode(w, inp, pairs, op)
+    G = w.group
+    n_match = n_tie = 0
+    for (b, h), r in ref.items():
+        # compressed keys
+        np.testing.assert_allclose(Kc[b, h].double().cpu().numpy(), r["Kc"], atol=2e-6, rtol=1e-5)
+        verdict = compare_sets(idx[b, h].cpu().numpy(), r["sel"])
+        assert verdict != "mismatch", (b, h, idx[b, h].tolist(), r["sel"].selected)
+        if verdict == "near_tie":
+            n_tie += 1
+            continue
+        n_match += 1
+        dt = "f32" if (w.dtype == "f32" and out_dtype == torch.float32) else "bf16"
+        assert_close(O[b, :, h * G:(h + 1) * G], r["O"], dt, f"O pair {(b, h)}")
+        lse_err = np.abs(lse[b, :, h * G:(h + 1) * G].double().cpu().numpy() - r["lse"]).max()
+        assert lse_err < (2e-5 if w.dtype == "f32" else 2e-4), lse_err
+    print(f"\n{w.name}: {n_match} pairs matched, {n_tie} near-ties")
+    return inp, p, Kc, O, lse, idx
+
+
+# ------------------------------------------------------------------ pooling --
+
+@pytest.mark.parametrize("dtype,pool,b,C", [("bf16", "mean", 64, 64 * 37 + 19), ("f32", "mean", 64, 64 * 21),
+                                            ("bf16", "lsa", 512, 512 * 9 + 100), ("f32", "lsa", 128, 128 * 5),
+                                            ("bf16", "mean", 16, 16 * 50 + 3)])
+def test_pool_keys_parity(dtype, pool, b, C):
+    w = WORKLOADS["decode_32k"].scaled(batch=2, num_q_heads=8, num_kv_heads=2, ctx_len=C, dtype=dtype,
+                                       pool=pool, block_size=b, n_needles=2, sink_keys=b, window_keys=b)
+    inp = dev_inputs(w, 21)
+    p = sa.params_for(w)
+    Kc = run_pool(w, inp, p)
+    torch.cuda.synchronize()
+    for (bi, h) in all_pairs(w):
+        K = inp["K"][bi, h, :C].double().cpu().numpy()
+        ref = orc.pool_lsa(K, b, 4) if pool == "lsa" else orc.pool_mean(K, b)
+        np.testing.assert_allclose(Kc[bi, h].double().cpu().numpy(), ref, atol=2e-6, rtol=1e-5)
+
+
+# ------------------------------------------------------------- score + top-k --
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny_decode", {}),
+    ("decode_32k", dict(batch=2)),
+    ("draft_chunk_16k", dict(batch=2)),
+    ("decode_1m", dict(batch=1, ctx_len=512 * 300 + 77, num_kv_heads=2, num_q_heads=8)),
+])
+def test_score_topk_parity(name, over):
+    w = WORKLOADS[name].scaled(**over)
+    inp = dev_inputs(w, 31)
+    p = sa.params_for(w)
+    Kc = run_pool(w, inp, p)
+    nb = w.ctx_len // w.block_size
+    idx = torch.empty((w.batch, w.num_kv_heads, w.top_k), device="cuda", dtype=torch.int32)
+    scores = torch.empty((w.batch, w.num_kv_heads, nb), device="cuda", dtype=torch.float32)
+    ws = sa.alloc_workspace(p, sa.SA_OP_SCORE_TOPK)
+    sa.score_topk(p, inp["Q"], Kc, idx, scores, ws)
+    torch.cuda.synchronize()
+    ref = oracle_decode(w, inp, all_pairs(w))
+    ties = 0
+    for (b, h), r in ref.items():
+        np.testing.assert_allclose(scores[b, h].double().cpu().numpy(), r["scores"], atol=2e-5, rtol=2e-5)
+        v = compare_sets(idx[b, h].cpu().numpy(), r["sel"])
+        assert v != "mismatch", (b, h)
+        ties += v == "near_tie"
+        if w.n_needles <= w.top_k:
+            assert set(inp["needles"][b, h].tolist()) <= set(idx[b, h].tolist())
+    print(f"\n{name}: near-ties {ties}/{len(ref)}")
+
+
+# -------------------------------------------------------- given index table --
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny_decode", {}),
+    ("decode_32k", dict(batch=2)),
+    ("draft_chunk_16k", dict(batch=2, ctx_len=4096 + 5)),
+    ("decode_1m", dict(batch=1, ctx_len=512 * 64 + 300, num_kv_heads=2, num_q_heads=8)),
+])
+def test_given_idx_with_oracle_indices(name, over):
+    """The attention step alone, fed the oracle's own selection."""
+    w = WORKLOADS[name].scaled(**over)
+    inp = dev_inputs(w, 41)
+    pairs = all_pairs(w)
+    ref = oracle_decode(w, inp, pairs)
+    idx = torch.full((w.batch, w.num_kv_heads, w.top_k), -1, dtype=torch.int32)
+    for (b, h), r in ref.items():
+        s = r["sel"].selected
+        idx[b, h, :len(s)] = torch.tensor(s, dtype=torch.int32)
+    idx = idx.cuda()
+    p = sa.params_for(w, out_dtype="f32")
+    O = torch.empty((w.batch, w.n_q, w.num_q_heads, 128), device="cuda", dtype=torch.float32)
+    lse = torch.empty((w.batch, w.n_q, w.num_q_heads), device="cuda", dtype=torch.float32)
+    ws = sa.alloc_workspace(p, sa.SA_OP_GIVEN_IDX)
+    sa.sparse_attn_given_idx(p, inp["Q"], inp["K"], inp["V"], idx, O, lse, ws)
+    assert sa.read_status(ws) == sa.SA_OK
+    G = w.group
+    worst = (0.0, 0.0)
+    for (b, h), r in ref.items():
+        e = assert_close(O[b, :, h * G:(h + 1) * G], r["O"], w.dtype, f"pair {(b, h)}")
+        worst = (max(worst[0], e[0]), max(worst[1], e[1]))
+        assert np.abs(lse[b, :, h * G:(h + 1) * G].double().cpu().numpy() - r["lse"]).max() < 2e-4
+    print(f"\n{name}: worst max-abs {worst[0]:.2e} rel-L2 {worst[1]:.2e}")
+
+
+# ------------------------------------------------------------ end to end ----
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny_decode", {}),
+    ("decode_32k", dict(batch=2)),
+    ("draft_chunk_16k", dict(batch=2)),
+    ("decode_1m", dict(batch=1, ctx_len=512 * 200, num_kv_heads=2, num_q_heads=8)),
+])
+def test_decode_end_to_end(name, over):
+    check_decode(WORKLOADS[name].scaled(**over), seed=51)
+
+
+def test_decode_bf16_output():
+    check_decode(WORKLOADS["decode_32k"].scaled(batch=1), seed=52, out_dtype=torch.bfloat16)
+
+
+@pytest.mark.parametrize("over", [
+    dict(top_k=0),                                      # sink + window + new token only
+    dict(top_k=600),                                    # k above #candidates: dense equivalence
+    dict(ctx_len=40),                                   # no complete block
+    dict(ctx_len=0),                                    # the new token attends itself only
+    dict(ctx_len=64 * 33 + 7, sink_keys=100, window_keys=70),   # ragged sink / window / context
+    dict(num_q_heads=2, num_kv_heads=2),                # GQA 1
+    dict(num_q_heads=16, num_kv_heads=2, n_q=2),        # GQA 8 x 2 tokens = 16 rows
+    dict(num_q_heads=4, num_kv_heads=2, n_q=6, top_k=5),  # draft chunk, 12 rows
+    dict(block_size=128, top_k=3),
+])
+def test_decode_edge_cases(over):
+    base = dict(batch=2, num_q_heads=8, num_kv_heads=2, ctx_len=4096, n_needles=2)
+    base.update(over)
+    w = WORKLOADS["decode_32k"].scaled(**base)
+    if w.top_k > 64 or w.ctx_len < 4096:
+        w = w.scaled(n_needles=0)
+    check_decode(w, seed=61)
+
+
+def test_decode_fp32_dense_equivalence_torch():
+    """k covering every candidate: the GPU result equals dense attention
+    computed by torch in float64 (a library routine, independent of both)."""
+    w = WORKLOADS["tiny_decode"].scaled(top_k=100, ctx_len=1500)
+    inp = dev_inputs(w, 62)
+    p = sa.params_for(w)
+    Kc = run_pool(w, inp, p)
+    O, lse, idx, _ = run_decode(w, inp, p, Kc)
+    q = inp["Q"][0, 0].double()                    # [4, d]
+    K = inp["K"][0, 0, :w.kv_len].double()
+    V = inp["V"][0, 0, :w.kv_len].double()
+    ref = torch.nn.functional.scaled_dot_product_attention(q[:, None], K[None].expand(4, -1, -1),
+                                                           V[None].expand(4, -1, -1))[:, 0]
+    assert (O[0, 0].double() - ref).abs().max().item() <= 1e-5
+
+
+def test_workspace_reuse_is_deterministic():
+    w = WORKLOADS["decode_32k"].scaled(batch=2)
+    inp = dev_inputs(w, 71)
+    p = sa.params_for(w, out_dtype="f32")
+    Kc = run_pool(w, inp, p)
+    O1, lse1, idx1, ws = run_decode(w, inp, p, Kc)
+    O2 = torch.empty_like(O1)
+    lse2 = torch.empty_like(lse1)
+    idx2 = torch.empty_like(idx1)
+    for _ in range(3):
+        sa.sparse_attn_decode(p, inp["Q"], inp["K"], inp["V"], Kc, O2, lse2, idx2, ws)
+    assert sa.read_status(ws) == sa.SA_OK
+    assert torch.equal(idx1, idx2) and torch.equal(O1, O2) and torch.equal(lse1, lse2)
+
+
+def test_given_idx_bad_entries_are_reported_and_skipped():
+    w = WORKLOADS["decode_32k"].scaled(batch=1, num_kv_heads=2, num_q_heads=8, ctx_len=4096, top_k=6,
+                                       n_needles=0)
+    inp = dev_inputs(w, 81)
+    nb = w.ctx_len // 64
+    rows = [[3, 9, 9, 20, -1, -1],            # repeated id
+            [5, 2, 30, nb + 4, 40, -1]]       # descending pair and an out-of-range id
+    keep = [[3, 9, 20], [5, 30, 40]]
+    idx = torch.tensor(rows, dtype=torch.int32, device="cuda")[None]
+    p = sa.params_for(w, out_dtype="f32")
+    O = torch.empty((1, 1, 8, 128), device="cuda")
+    ws = sa.alloc_workspace(p, sa.SA_OP_GIVEN_IDX)
+    sa.sparse_attn_given_idx(p, inp["Q"], inp["K"], inp["V"], idx, O, None, ws)
+    assert sa.read_status(ws) == sa.SA_ERR_INDEX
+    assert sa.read_status(ws) == sa.SA_OK            # the status word was cleared
+    op = oracle_params(w)
+    for h in range(2):
+        q, K, V = slab(inp, 0, h, 4, w.kv_len)
+        pos = orc.attended_positions(w.ctx_len, op, keep[h], w.ctx_len)
+        for g in range(4):
+            ref, _, _ = orc.masked_softmax_attention(q[0, g], K, V, pos, 1 / np.sqrt(128))
+            err = np.abs(O[0, 0, h * 4 + g].double().cpu().numpy() - ref).max()
+            assert err < 5e-3
+
+
+# ------------------------------------------------------- full-size samples --
+
+def _sampled(w):
+    return sorted({(0, 0), (w.batch - 1, w.num_kv_heads - 1), (w.batch // 2, w.num_kv_heads // 2),
+                   (1 % w.batch, (3 % w.num_kv_heads)), (w.batch // 3, w.num_kv_heads - 1)})
+
+
+@pytest.mark.parametrize("name", ["decode_32k", "draft_chunk_16k", "decode_1m"])
+def test_full_size_sampled(name):
+    """The benchmark's launch configuration at full size; the oracle checks a
+    sample of (sequence, KV head) pairs one by one."""
+    w = WORKLOADS[name]
+    check_decode(w, seed=91, pairs=_sampled(w), out_dtype=torch.bfloat16)
+    torch.cuda.empty_cache()

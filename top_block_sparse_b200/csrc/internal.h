@@ -1,0 +1,98 @@
+// Host-side interface between the C ABI layer (sa_api.cu) and the kernel
+// translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "sa.h"
+
+namespace sa {
+
+// Geometry of one decode / chunk problem, derived from sa_params on the host.
+struct DecodeGeom {
+  int B, Hq, Hkv, G, n_q, R;       // R = n_q * G query rows per (sequence, KV head)
+  int64_t C, cap, kv_end;          // context length, token stride, C + n_q
+  int b;                           // block size
+  int64_t nb;                      // complete blocks of the context
+  int64_t s_end, w_begin;          // sink [0, s_end), window [w_begin, C)
+  int pairs;                       // B * Hkv
+};
+
+// ---- pooling ----------------------------------------------------------------
+struct PoolArgs {
+  const void* K;
+  float* Kc;
+  int pairs;
+  int64_t cap;      // token stride of K
+  int64_t nb;       // blocks per pair
+  int b;
+  int lsa;          // 0 mean, 1 LSA centroid
+};
+cudaError_t launch_pool(const PoolArgs& a, bool bf16, cudaStream_t s);
+
+// ---- decode scoring + top-k --------------------------------------------------
+struct ScoreArgs {
+  const void* Q;
+  const float* Kc;
+  float* scores;          // [pairs, nb]
+  int32_t* idx;           // [pairs, top_k]
+  unsigned* counters;     // [pairs], zero between calls
+  int B, Hq, Hkv, G, n_q;
+  int64_t nb;
+  int b;
+  int64_t s_end, w_begin;
+  int top_k;
+  float scale;            // softmax scale (mean pooling)
+  int lsa;                // cosine scores
+  int chunks;             // CTAs per pair
+  int blocks_per_chunk;
+};
+constexpr int kScoreBlocksPerChunk = 128;
+constexpr int64_t kMaxSelectBlocks = 16384;
+cudaError_t launch_score_topk_query0(const ScoreArgs& a, bool bf16, cudaStream_t s);
+
+// ---- decode / chunk sparse attention ---------------------------------------
+struct DecodeAttnArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const int32_t* idx;     // [pairs, idx_stride]
+  int idx_stride;         // entries per pair
+  void* O;
+  float* lse;             // may be null
+  float* part_O;          // [pairs, n_slots, R4, 128]
+  float* part_ml;         // [pairs, n_slots, R4, 2]
+  unsigned* counters;     // [pairs], zero between calls
+  unsigned* status;
+  int B, Hq, Hkv, G, n_q, R, R4;
+  int64_t C, cap, kv_end;
+  int b;
+  int64_t nb;
+  int64_t s_end, w_begin;
+  int n_sink_tiles, tpb, n_wc_tiles, MT;
+  int64_t total_tiles;
+  int tpc;                // tiles per CTA
+  int n_slots;            // partial slots per pair
+  int n_stages;
+  float qscale;           // softmax scale * log2(e)
+  int check_idx;          // validate caller-provided ids
+  int pdl;                // launched as a programmatic dependent of the scorer
+};
+
+struct DecodePlan {
+  int R, R4, RG, KG;
+  int n_sink_tiles, tpb, n_wc_tiles, MT;
+  int64_t total_tiles;
+  int grid, tpc, n_slots, n_stages;
+  size_t smem;
+  int threads;
+};
+// Fills `plan`; returns false (with a reason) if the shape is not built.
+bool plan_decode(const DecodeGeom& g, int idx_slots, bool bf16, int num_sms, DecodePlan* plan,
+                 const char** why);
+cudaError_t launch_decode_attn(const DecodeAttnArgs& a, const DecodePlan& p, bool bf16,
+                               bool out_bf16, cudaStream_t s);
+
+}  // namespace sa

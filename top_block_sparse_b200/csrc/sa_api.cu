@@ -1,0 +1,385 @@
+// C ABI of libsa.so: argument validation, workspace layout, launch planning.
+// Every entry point validates on the host before launching anything and
+// never allocates memory; see include/sa.h for the contract.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sa.h"
+
+namespace sa {
+namespace {
+
+thread_local char g_err[512] = "";
+
+sa_status fail(sa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+sa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static int cached[64] = {0};
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared validation of sa_params.  `prefill` selects the SA_SEL_TILE_MAX rules.
+sa_status check_params(const sa_params* p, bool prefill) {
+  if (!p) return fail(SA_ERR_INVALID, "params is NULL");
+  if (p->reserved != 0) return fail(SA_ERR_INVALID, "params.reserved must be 0");
+  if (p->batch < 1 || p->num_kv_heads < 1 || p->num_q_heads < 1)
+    return fail(SA_ERR_INVALID, "batch, num_q_heads and num_kv_heads must be >= 1");
+  if (p->num_q_heads % p->num_kv_heads != 0)
+    return fail(SA_ERR_INVALID, "num_q_heads (%d) must be a multiple of num_kv_heads (%d)", p->num_q_heads,
+                p->num_kv_heads);
+  if (p->head_dim != kHeadDim) return fail(SA_ERR_UNSUPPORTED, "head_dim %d: only 128 is built", p->head_dim);
+  if (p->dtype != SA_F32 && p->dtype != SA_BF16) return fail(SA_ERR_INVALID, "dtype %d", p->dtype);
+  if (p->out_dtype != SA_F32 && p->out_dtype != SA_BF16) return fail(SA_ERR_INVALID, "out_dtype %d", p->out_dtype);
+  if (p->n_q < 1) return fail(SA_ERR_INVALID, "n_q must be >= 1");
+  if (p->ctx_len < 0) return fail(SA_ERR_INVALID, "ctx_len must be >= 0");
+  if (p->kv_capacity < p->ctx_len + p->n_q)
+    return fail(SA_ERR_INVALID, "kv_capacity (%lld) < ctx_len + n_q (%lld)", (long long)p->kv_capacity,
+                (long long)(p->ctx_len + p->n_q));
+  if (p->block_size < 16 || p->block_size % 16 != 0 || p->block_size > 65536)
+    return fail(SA_ERR_INVALID, "block_size %d must be a multiple of 16 in [16, 65536]", p->block_size);
+  if (p->pool != SA_POOL_MEAN && p->pool != SA_POOL_LSA) return fail(SA_ERR_INVALID, "pool %d", p->pool);
+  if (p->pool == SA_POOL_LSA && (p->pool_stride < 1 || p->block_size % p->pool_stride != 0))
+    return fail(SA_ERR_INVALID, "pool_stride %d must divide block_size %d", p->pool_stride, p->block_size);
+  if (p->top_k < 0 || p->top_k > 4096) return fail(SA_ERR_INVALID, "top_k %d must be in [0, 4096]", p->top_k);
+  if (p->sink_keys < 0 || p->window_keys < 0) return fail(SA_ERR_INVALID, "sink_keys and window_keys must be >= 0");
+  if (p->select != SA_SEL_QUERY0 && p->select != SA_SEL_TILE_MAX) return fail(SA_ERR_INVALID, "select %d", p->select);
+  if (prefill) {
+    if (p->select != SA_SEL_TILE_MAX) return fail(SA_ERR_INVALID, "prefill needs select = SA_SEL_TILE_MAX");
+    if (p->ctx_len != 0) return fail(SA_ERR_INVALID, "prefill needs ctx_len = 0 (n_q is the sequence length)");
+  } else if (p->select != SA_SEL_QUERY0) {
+    return fail(SA_ERR_INVALID, "decode / chunk calls need select = SA_SEL_QUERY0");
+  }
+  return SA_OK;
+}
+
+DecodeGeom decode_geom(const sa_params* p) {
+  DecodeGeom g;
+  g.B = p->batch;
+  g.Hq = p->num_q_heads;
+  g.Hkv = p->num_kv_heads;
+  g.G = p->num_q_heads / p->num_kv_heads;
+  g.n_q = p->n_q;
+  g.R = g.n_q * g.G;
+  g.C = p->ctx_len;
+  g.cap = p->kv_capacity;
+  g.kv_end = p->ctx_len + p->n_q;
+  g.b = p->block_size;
+  g.nb = p->ctx_len / p->block_size;
+  g.s_end = p->sink_keys < g.C ? p->sink_keys : g.C;
+  const int64_t wb = g.C - p->window_keys;
+  g.w_begin = wb > g.s_end ? wb : g.s_end;
+  g.pairs = g.B * g.Hkv;
+  return g;
+}
+
+float scale_of(const sa_params* p) {
+  return p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf(static_cast<float>(p->head_dim));
+}
+
+// Workspace layout of the decode-type ops.
+struct DecodeWs {
+  size_t score_cnt, attn_cnt, scores, idx, part_O, part_ml, total;
+};
+
+DecodeWs decode_ws(const DecodeGeom& g, const DecodePlan& plan, int top_k, int op) {
+  DecodeWs w = {};
+  size_t off = kWsHeader;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  const size_t pairs = static_cast<size_t>(g.pairs);
+  w.score_cnt = take(pairs * 4);
+  w.attn_cnt = take(pairs * 4);
+  if (op == SA_OP_SCORE_TOPK || op == SA_OP_DECODE) {
+    w.scores = take(pairs * static_cast<size_t>(g.nb) * 4);
+  }
+  if (op == SA_OP_DECODE) w.idx = take(pairs * static_cast<size_t>(top_k) * 4);
+  if (op == SA_OP_DECODE || op == SA_OP_GIVEN_IDX) {
+    const size_t slots = pairs * static_cast<size_t>(plan.n_slots) * plan.R4;
+    w.part_O = take(slots * kHeadDim * 4);
+    w.part_ml = take(slots * 2 * 4);
+  }
+  w.total = off;
+  return w;
+}
+
+sa_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (!ws) return fail(SA_ERR_WORKSPACE, "workspace is NULL (needs %zu bytes)", need);
+  if (!aligned16(ws)) return fail(SA_ERR_INVALID, "workspace must be 16-byte aligned");
+  if (ws_bytes < need) return fail(SA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  return SA_OK;
+}
+
+sa_status plan_for(const sa_params* p, int idx_slots, DecodeGeom* g, DecodePlan* plan) {
+  *g = decode_geom(p);
+  const char* why = "";
+  if (!plan_decode(*g, idx_slots, p->dtype == SA_BF16, device_sms(), plan, &why))
+    return fail(SA_ERR_UNSUPPORTED, "%s", why);
+  return SA_OK;
+}
+
+ScoreArgs score_args(const sa_params* p, const DecodeGeom& g, const void* Q, const float* Kc,
+                     float* scores, int32_t* idx, unsigned* counters) {
+  ScoreArgs a = {};
+  a.Q = Q;
+  a.Kc = Kc;
+  a.scores = scores;
+  a.idx = idx;
+  a.counters = counters;
+  a.B = g.B;
+  a.Hq = g.Hq;
+  a.Hkv = g.Hkv;
+  a.G = g.G;
+  a.n_q = g.n_q;
+  a.nb = g.nb;
+  a.b = g.b;
+  a.s_end = g.s_end;
+  a.w_begin = g.w_begin;
+  a.top_k = p->top_k;
+  a.scale = scale_of(p);
+  a.lsa = p->pool == SA_POOL_LSA;
+  a.blocks_per_chunk = kScoreBlocksPerChunk;
+  a.chunks = static_cast<int>((g.nb + kScoreBlocksPerChunk - 1) / kScoreBlocksPerChunk);
+  if (a.chunks < 1) a.chunks = 1;
+  return a;
+}
+
+DecodeAttnArgs attn_args(const sa_params* p, const DecodeGeom& g, const DecodePlan& plan, const void* Q,
+                         const void* K, const void* V, const int32_t* idx, int idx_stride, void* O, float* lse,
+                         unsigned char* ws, const DecodeWs& L) {
+  DecodeAttnArgs a = {};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.idx = idx;
+  a.idx_stride = idx_stride;
+  a.O = O;
+  a.lse = lse;
+  a.part_O = reinterpret_cast<float*>(ws + L.part_O);
+  a.part_ml = reinterpret_cast<float*>(ws + L.part_ml);
+  a.counters = reinterpret_cast<unsigned*>(ws + L.attn_cnt);
+  a.status = reinterpret_cast<unsigned*>(ws);
+  a.B = g.B;
+  a.Hq = g.Hq;
+  a.Hkv = g.Hkv;
+  a.G = g.G;
+  a.n_q = g.n_q;
+  a.R = g.R;
+  a.R4 = plan.R4;
+  a.C = g.C;
+  a.cap = g.cap;
+  a.kv_end = g.kv_end;
+  a.b = g.b;
+  a.nb = g.nb;
+  a.s_end = g.s_end;
+  a.w_begin = g.w_begin;
+  a.n_sink_tiles = plan.n_sink_tiles;
+  a.tpb = plan.tpb;
+  a.n_wc_tiles = plan.n_wc_tiles;
+  a.MT = plan.MT;
+  a.total_tiles = plan.total_tiles;
+  a.tpc = plan.tpc;
+  a.n_slots = plan.n_slots;
+  a.n_stages = plan.n_stages;
+  a.qscale = scale_of(p) * 1.4426950408889634f;
+  return a;
+}
+
+}  // namespace
+}  // namespace sa
+
+using namespace sa;
+
+extern "C" {
+
+int32_t sa_version(void) { return 100; }
+
+const char* sa_last_error(void) { return g_err; }
+
+const char* sa_status_string(sa_status s) {
+  switch (s) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID: return "SA_ERR_INVALID";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED";
+    case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE";
+    case SA_ERR_INDEX: return "SA_ERR_INDEX";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA";
+    case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT";
+  }
+  return "SA_ERR_UNKNOWN";
+}
+
+size_t sa_workspace_size(const sa_params* p, int32_t op) {
+  const bool prefill = (op == SA_OP_PREFILL) || (p && p->select == SA_SEL_TILE_MAX);
+  if (check_params(p, prefill) != SA_OK) return 0;
+  if (prefill) return 0;   // prefill is not built in this library version
+  DecodeGeom g;
+  DecodePlan plan;
+  int slots = (op == SA_OP_DECODE) ? p->top_k : 0;
+  if (op == SA_OP_GIVEN_IDX) slots = p->top_k;   // sized for idx_len == top_k
+  if (op == SA_OP_SCORE_TOPK) slots = 0;
+  if (plan_for(p, slots, &g, &plan) != SA_OK) return 0;
+  return decode_ws(g, plan, p->top_k, op).total;
+}
+
+sa_status sa_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws) return fail(SA_ERR_INVALID, "workspace is NULL");
+  cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  return SA_OK;
+}
+
+sa_status sa_pool_keys(const sa_params* p, const void* K, float* Kc, void* stream) {
+  const bool prefill = p && p->select == SA_SEL_TILE_MAX;
+  sa_status st = check_params(p, prefill);
+  if (st != SA_OK) return st;
+  const int64_t nb = (prefill ? static_cast<int64_t>(p->n_q) : p->ctx_len) / p->block_size;
+  if (nb == 0) return SA_OK;   // no complete block: nothing to write
+  if (!K || !Kc) return fail(SA_ERR_INVALID, "K and Kc must be non-NULL");
+  if (!aligned16(K) || !aligned16(Kc)) return fail(SA_ERR_INVALID, "K and Kc must be 16-byte aligned");
+  PoolArgs a = {};
+  a.K = K;
+  a.Kc = Kc;
+  a.pairs = p->batch * p->num_kv_heads;
+  a.cap = p->kv_capacity;
+  a.nb = nb;
+  a.b = p->block_size;
+  a.lsa = p->pool == SA_POOL_LSA;
+  cudaError_t e = launch_pool(a, p->dtype == SA_BF16, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pool kernel launch");
+  return SA_OK;
+}
+
+sa_status sa_score_topk(const sa_params* p, const void* Q, const float* Kc, int32_t* idx, float* scores, void* ws,
+                        size_t ws_bytes, void* stream) {
+  const bool prefill = p && p->select == SA_SEL_TILE_MAX;
+  sa_status st = check_params(p, prefill);
+  if (st != SA_OK) return st;
+  if (prefill) return fail(SA_ERR_UNSUPPORTED, "SA_SEL_TILE_MAX scoring is not built in this library version");
+  if (!Q || (!Kc && p->ctx_len >= p->block_size) || (!idx && p->top_k > 0))
+    return fail(SA_ERR_INVALID, "Q, Kc and idx must be non-NULL (Kc may be NULL without a complete block)");
+  if (!aligned16(Q) || !aligned16(Kc)) return fail(SA_ERR_INVALID, "Q and Kc must be 16-byte aligned");
+  DecodeGeom g;
+  DecodePlan plan;
+  if ((st = plan_for(p, 0, &g, &plan)) != SA_OK) return st;
+  if (g.nb > kMaxSelectBlocks)
+    return fail(SA_ERR_UNSUPPORTED, "%lld blocks per sequence exceed the %lld the selector handles",
+                (long long)g.nb, (long long)kMaxSelectBlocks);
+  const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_SCORE_TOPK);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != SA_OK) return st;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  float* sc = scores ? scores : reinterpret_cast<float*>(w + L.scores);
+  ScoreArgs a = score_args(p, g, Q, Kc, sc, idx, reinterpret_cast<unsigned*>(w + L.score_cnt));
+  cudaError_t e = launch_score_topk_query0(a, p->dtype == SA_BF16, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "score/top-k kernel launch");
+  return SA_OK;
+}
+
+sa_status sa_sparse_attn_given_idx(const sa_params* p, const void* Q, const void* K, const void* V,
+                                   const int32_t* idx, int32_t idx_len, void* O, float* lse, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  const bool prefill = p && p->select == SA_SEL_TILE_MAX;
+  sa_status st = check_params(p, prefill);
+  if (st != SA_OK) return st;
+  if (prefill) return fail(SA_ERR_UNSUPPORTED, "prefill index tables are not built in this library version");
+  if (!Q || !K || !V || !O) return fail(SA_ERR_INVALID, "Q, K, V and O must be non-NULL");
+  if (idx_len < 0 || idx_len > 4096) return fail(SA_ERR_INVALID, "idx_len %d must be in [0, 4096]", idx_len);
+  if (idx_len > 0 && !idx) return fail(SA_ERR_INVALID, "idx is NULL");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return fail(SA_ERR_INVALID, "Q, K, V and O must be 16-byte aligned");
+  DecodeGeom g;
+  DecodePlan plan;
+  if ((st = plan_for(p, idx_len, &g, &plan)) != SA_OK) return st;
+  const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_GIVEN_IDX);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != SA_OK) return st;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, idx, idx_len, O, lse, w, L);
+  a.check_idx = 1;
+  a.pdl = 0;
+  cudaError_t e = launch_decode_attn(a, plan, p->dtype == SA_BF16, p->out_dtype == SA_BF16,
+                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+  return SA_OK;
+}
+
+sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q, const void* K, const void* V, const float* Kc,
+                                void* O, float* lse, int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  sa_status st = check_params(p, false);
+  if (st != SA_OK) return st;
+  if (!Q || !K || !V || !O || (!Kc && p->ctx_len >= p->block_size))
+    return fail(SA_ERR_INVALID, "Q, K, V, Kc and O must be non-NULL (Kc may be NULL without a complete block)");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(Kc))
+    return fail(SA_ERR_INVALID, "Q, K, V, Kc and O must be 16-byte aligned");
+  DecodeGeom g;
+  DecodePlan plan;
+  if ((st = plan_for(p, p->top_k, &g, &plan)) != SA_OK) return st;
+  if (g.nb > kMaxSelectBlocks)
+    return fail(SA_ERR_UNSUPPORTED, "%lld blocks per sequence exceed the %lld the selector handles",
+                (long long)g.nb, (long long)kMaxSelectBlocks);
+  const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_DECODE);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != SA_OK) return st;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + L.idx);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ScoreArgs sa_ = score_args(p, g, Q, Kc, reinterpret_cast<float*>(w + L.scores), idx,
+                             reinterpret_cast<unsigned*>(w + L.score_cnt));
+  cudaError_t e = launch_score_topk_query0(sa_, p->dtype == SA_BF16, s);
+  if (e != cudaSuccess) return cuda_fail(e, "score/top-k kernel launch");
+  DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, idx, p->top_k, O, lse, w, L);
+  a.check_idx = 0;
+  a.pdl = 1;
+  e = launch_decode_attn(a, plan, p->dtype == SA_BF16, p->out_dtype == SA_BF16, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+  return SA_OK;
+}
+
+sa_status sa_sparse_attn_prefill(const sa_params* p, const void* Q, const void* K, const void* V, float* Kc,
+                                 void* O, float* lse, int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  sa_status st = check_params(p, true);
+  if (st != SA_OK) return st;
+  (void)Q; (void)K; (void)V; (void)Kc; (void)O; (void)lse; (void)idx_out; (void)ws; (void)ws_bytes; (void)stream;
+  return fail(SA_ERR_UNSUPPORTED, "prefill is not built in this library version");
+}
+
+sa_status sa_read_status(void* ws, void* stream) {
+  if (!ws) return fail(SA_ERR_INVALID, "workspace is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned word = 0;
+  e = cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy (status word)");
+  if (word) {
+    e = cudaMemset(ws, 0, sizeof(word));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset (status word)");
+  }
+  if (word & kStatusTimeout) return fail(SA_ERR_TIMEOUT, "a bounded wait inside a kernel ran out");
+  if (word & kStatusIndex) return fail(SA_ERR_INDEX, "an index-table entry was out of range or repeated");
+  return SA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,190 @@
+"""Thin ctypes binding of libsa.so (include/sa.h).
+
+Argument marshalling only: torch tensors are passed as raw device pointers
+with the current CUDA stream; every step runs in the library's kernels.
+Importing this module loads libsa.so and raises ImportError if it is missing
+(build it with ``python -m top_block_sparse_b200.build``).  There is no CPU
+fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsa.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libsa.so not found at {_LIB_PATH}; run python -m top_block_sparse_b200.build")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+# ---- constants mirrored from sa.h ------------------------------------------
+SA_OK, SA_ERR_INVALID, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_INDEX, SA_ERR_CUDA, SA_ERR_TIMEOUT = range(7)
+SA_F32, SA_BF16 = 0, 1
+SA_POOL_MEAN, SA_POOL_LSA = 0, 1
+SA_SEL_QUERY0, SA_SEL_TILE_MAX = 0, 1
+SA_OP_SCORE_TOPK, SA_OP_GIVEN_IDX, SA_OP_DECODE, SA_OP_PREFILL = 0, 1, 2, 3
+
+EXPORTED = ["sa_version", "sa_workspace_size", "sa_workspace_init", "sa_pool_keys", "sa_score_topk",
+            "sa_sparse_attn_given_idx", "sa_sparse_attn_decode", "sa_sparse_attn_prefill",
+            "sa_read_status", "sa_status_string", "sa_last_error"]
+
+
+class SaParams(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("ctx_len", ctypes.c_int64), ("kv_capacity", ctypes.c_int64),
+        ("n_q", ctypes.c_int32), ("block_size", ctypes.c_int32),
+        ("pool", ctypes.c_int32), ("pool_stride", ctypes.c_int32),
+        ("top_k", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("out_dtype", ctypes.c_int32), ("select", ctypes.c_int32),
+        ("sink_keys", ctypes.c_int64), ("window_keys", ctypes.c_int64),
+        ("softmax_scale", ctypes.c_float), ("reserved", ctypes.c_int32),
+    ]
+
+
+assert ctypes.sizeof(SaParams) == 88
+
+_vp, _sz, _i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
+_P = ctypes.POINTER(SaParams)
+_sig = {
+    "sa_version": (_i32, []),
+    "sa_workspace_size": (_sz, [_P, _i32]),
+    "sa_workspace_init": (_i32, [_vp, _sz, _vp]),
+    "sa_pool_keys": (_i32, [_P, _vp, _vp, _vp]),
+    "sa_score_topk": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "sa_sparse_attn_given_idx": (_i32, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "sa_sparse_attn_decode": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "sa_sparse_attn_prefill": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "sa_read_status": (_i32, [_vp, _vp]),
+    "sa_status_string": (ctypes.c_char_p, [_i32]),
+    "sa_last_error": (ctypes.c_char_p, []),
+}
+for _name, (_res, _args) in _sig.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class SaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_lib.sa_status_string(status).decode()}: {msg}")
+        self.status = status
+
+
+def _check(st: int):
+    if st != SA_OK:
+        raise SaError(st, _lib.sa_last_error().decode())
+
+
+def version() -> int:
+    return int(_lib.sa_version())
+
+
+def make_params(*, batch, num_q_heads, num_kv_heads, ctx_len, n_q, block_size, top_k,
+                sink_keys, window_keys, dtype="bf16", out_dtype=None, pool="mean",
+                pool_stride=4, kv_capacity=None, prefill=False, softmax_scale=0.0,
+                head_dim=128) -> SaParams:
+    dt = SA_BF16 if dtype == "bf16" else SA_F32
+    odt = dt if out_dtype is None else (SA_BF16 if out_dtype == "bf16" else SA_F32)
+    return SaParams(batch=batch, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
+                    head_dim=head_dim, ctx_len=ctx_len,
+                    kv_capacity=(ctx_len + n_q) if kv_capacity is None else kv_capacity,
+                    n_q=n_q, block_size=block_size,
+                    pool=SA_POOL_LSA if pool == "lsa" else SA_POOL_MEAN, pool_stride=pool_stride,
+                    top_k=top_k, dtype=dt, out_dtype=odt,
+                    select=SA_SEL_TILE_MAX if prefill else SA_SEL_QUERY0,
+                    sink_keys=sink_keys, window_keys=window_keys,
+                    softmax_scale=softmax_scale, reserved=0)
+
+
+def params_for(w, kv_capacity=None, out_dtype=None) -> SaParams:
+    """SaParams for a Workload from top_block_sparse_b200.inputs."""
+    return make_params(batch=w.batch, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
+                       ctx_len=w.ctx_len, n_q=w.n_q, block_size=w.block_size, top_k=w.top_k,
+                       sink_keys=w.sink_keys, window_keys=w.window_keys, dtype=w.dtype,
+                       out_dtype=out_dtype, pool=w.pool, kv_capacity=kv_capacity,
+                       prefill=w.prefill, head_dim=w.head_dim)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to libsa must be CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libsa must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_size(p: SaParams, op: int) -> int:
+    return int(_lib.sa_workspace_size(ctypes.byref(p), op))
+
+
+def alloc_workspace(p: SaParams, op: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace of the size op needs (the status word and the
+    self-resetting tickets start at zero)."""
+    n = workspace_size(p, op)
+    if n == 0:
+        _check(SA_ERR_INVALID if _lib.sa_last_error() else SA_ERR_UNSUPPORTED)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def workspace_init(ws: torch.Tensor, stream=None):
+    _check(_lib.sa_workspace_init(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+def pool_keys(p: SaParams, K: torch.Tensor, Kc: torch.Tensor, stream=None):
+    _check(_lib.sa_pool_keys(ctypes.byref(p), _ptr(K), _ptr(Kc), _stream(stream)))
+
+
+def score_topk(p: SaParams, Q, Kc, idx, scores=None, ws=None, stream=None):
+    _check(_lib.sa_score_topk(ctypes.byref(p), _ptr(Q), _ptr(Kc), _ptr(idx), _ptr(scores),
+                              _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def sparse_attn_given_idx(p: SaParams, Q, K, V, idx, O, lse=None, ws=None, stream=None):
+    idx_len = 0 if idx is None else int(idx.shape[-1])
+    _check(_lib.sa_sparse_attn_given_idx(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
+                                         idx_len, _ptr(O), _ptr(lse), _ptr(ws),
+                                         0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def sparse_attn_decode(p: SaParams, Q, K, V, Kc, O, lse=None, idx_out=None, ws=None, stream=None):
+    _check(_lib.sa_sparse_attn_decode(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kc), _ptr(O),
+                                      _ptr(lse), _ptr(idx_out), _ptr(ws),
+                                      0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def sparse_attn_prefill(p: SaParams, Q, K, V, Kc, O, lse=None, idx_out=None, ws=None, stream=None):
+    _check(_lib.sa_sparse_attn_prefill(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kc), _ptr(O),
+                                       _ptr(lse), _ptr(idx_out), _ptr(ws),
+                                       0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def read_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronises and returns (then clears) the device status of the
+    workspace: SA_OK, SA_ERR_INDEX or SA_ERR_TIMEOUT."""
+    return int(_lib.sa_read_status(_ptr(ws), _stream(stream)))
+
+
+def num_blocks(p: SaParams) -> int:
+    n = p.n_q if p.select == SA_SEL_TILE_MAX else p.ctx_len
+    return n // p.block_size
+
+
+def raw_call(name: str, *args):
+    """Direct access to an exported C function (ctypes-typed as in sa.h)."""
+    return getattr(_lib, name)(*args)
+
+
+def lib_path() -> str:
+    return _LIB_PATH
