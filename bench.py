@@ -389,6 +389,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-pairs", type=int, default=16)
     ap.add_argument("--ref-pairs", type=int, default=4)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller cases for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -397,6 +399,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = WORKLOADS[args.workload]
+    if args.batch is not None:
+        w = w.scaled(batch=args.batch)
 
     if args.impl == "reference":
         line = run_reference(args, w, rank, world)
