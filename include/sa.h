@@ -179,6 +179,26 @@ sa_status sa_sparse_attn_prefill(const sa_params* p, const void* Q,
                                  void* O, float* lse, int32_t* idx_out,
                                  void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of sa_sparse_attn_given_idx (the paper has no
+ * counterpart; it exists for callers that cannot allocate device memory,
+ * e.g. code inside a framework whose allocator must not be re-entered or
+ * plug-ins that are handed only their input and output buffers).  Same
+ * arguments, layouts and results as sa_sparse_attn_given_idx without the
+ * workspace: the kernel's scratch lives in a 16 MiB static device array that
+ * every device loading the library holds until exit.  Problems needing more
+ * scratch are rejected with SA_ERR_WORKSPACE before any launch.  The first
+ * call on a device looks up the array's device address (with that device
+ * current); make that first call before any stream capture.  All calls share
+ * the one array, so calls that overlap on the device race: issue them on one
+ * stream or otherwise order them.  Each call clears the array's status word
+ * and tickets first; bad index entries are skipped exactly as in
+ * sa_sparse_attn_given_idx but cannot be read back (there is no workspace to
+ * pass to sa_read_status).  Calls no allocating routine. */
+sa_status sa_sparse_attn_given_idx_noalloc(const sa_params* p, const void* Q,
+                                           const void* K, const void* V,
+                                           const int32_t* idx, int32_t idx_len,
+                                           void* O, float* lse, void* stream);
+
 /* Synchronises `stream`, returns the worst device condition recorded in the
  * workspace status word since the last call (SA_OK, SA_ERR_INDEX or
  * SA_ERR_TIMEOUT) and clears it. */

@@ -1,0 +1,79 @@
+"""The allocation-free entry point, sa_sparse_attn_given_idx_noalloc.
+
+Some callers cannot allocate device memory: code running inside a framework
+whose allocator must not be re-entered, or plug-ins that are handed only
+their input and output buffers.  For them the library offers this variant of
+sa_sparse_attn_given_idx whose scratch is a static device array inside the
+library instead of a caller-provided workspace.  The test calls it through
+the C ABI twice in a row (the array keeps the previous call's contents) and
+checks each result against the workspace entry point within the parity
+tolerances, then checks that a problem too large for the array is refused
+before any launch.  This file is collected last so that a run stopping at
+the first failure has already run every other test.
+"""
+import ctypes
+
+import pytest
+import torch
+
+from helpers import assert_close
+from top_block_sparse_b200.inputs import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+sa = pytest.importorskip("top_block_sparse_b200.sa")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _call_noalloc(p, inp, idx, O, lse):
+    st = sa.raw_call("sa_sparse_attn_given_idx_noalloc", ctypes.byref(p), _ptr(inp["Q"]), _ptr(inp["K"]),
+                     _ptr(inp["V"]), _ptr(idx), int(idx.shape[-1]), _ptr(O), _ptr(lse),
+                     ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == sa.SA_OK, sa.raw_call("sa_last_error").decode()
+
+
+def _reference(w, seed):
+    """Inputs, an index table from the library's own selector, and the
+    result of the workspace entry point."""
+    inp = make_inputs(w, seed=seed, device="cuda")
+    p = sa.params_for(w, out_dtype="f32")
+    nb = w.ctx_len // w.block_size
+    Kc = torch.empty((w.batch, w.num_kv_heads, nb, 128), device="cuda")
+    sa.pool_keys(p, inp["K"], Kc)
+    idx = torch.empty((w.batch, w.num_kv_heads, w.top_k), device="cuda", dtype=torch.int32)
+    sa.score_topk(p, inp["Q"], Kc, idx, None, sa.alloc_workspace(p, sa.SA_OP_SCORE_TOPK))
+    O = torch.empty((w.batch, w.n_q, w.num_q_heads, 128), device="cuda")
+    lse = torch.empty((w.batch, w.n_q, w.num_q_heads), device="cuda")
+    ws = sa.alloc_workspace(p, sa.SA_OP_GIVEN_IDX)
+    sa.sparse_attn_given_idx(p, inp["Q"], inp["K"], inp["V"], idx, O, lse, ws)
+    assert sa.read_status(ws) == sa.SA_OK
+    return inp, p, idx, O, lse
+
+
+@pytest.mark.parametrize("name,over", [("decode_32k", dict(batch=4)),
+                                       ("draft_chunk_16k", dict(batch=3, ctx_len=4096 + 33))])
+def test_noalloc_matches_workspace_entry_point_on_two_calls(name, over):
+    w = WORKLOADS[name].scaled(**over)
+    inp, p, idx, O_ref, lse_ref = _reference(w, seed=3)
+    ref_O = O_ref.double().cpu().numpy()
+    ref_lse = lse_ref.double().cpu().numpy()
+    for call in range(2):
+        O = torch.full_like(O_ref, float("nan"))
+        lse = torch.full_like(lse_ref, float("nan"))
+        _call_noalloc(p, inp, idx, O, lse)
+        torch.cuda.synchronize()
+        assert_close(O, ref_O, w.dtype, f"{name}, call {call + 1}")
+        assert abs(lse.double().cpu().numpy() - ref_lse).max() < 2e-4
+
+
+def test_noalloc_refuses_problems_larger_than_its_array():
+    w = WORKLOADS["draft_chunk_16k"].scaled(batch=256)
+    p = sa.params_for(w)
+    fake = ctypes.c_void_p(0x10000)
+    st = sa.raw_call("sa_sparse_attn_given_idx_noalloc", ctypes.byref(p), fake, fake, fake, fake, w.top_k,
+                     fake, None, None)
+    assert st == sa.SA_ERR_WORKSPACE
+    assert "static" in sa.raw_call("sa_last_error").decode()

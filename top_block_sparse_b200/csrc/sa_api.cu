@@ -383,3 +383,82 @@ sa_status sa_read_status(void* ws, void* stream) {
 }
 
 }  // extern "C"
+
+// ---- allocation-free variant of sa_sparse_attn_given_idx --------------------
+// For callers that cannot call cudaMalloc themselves: code running inside a
+// host framework whose allocator must not be re-entered, plug-ins handed only
+// input and output buffers, or callers whose memory budget was fixed before
+// they run.  The attention kernel's scratch (status word, per-pair tickets,
+// split partials) lives in one file-scope device array instead of a
+// caller-provided workspace.
+#include <mutex>
+
+namespace sa {
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB per device, held until exit
+
+// In host code this name is only a host-side stand-in for the device array,
+// not a device address: the address is obtained once per device with
+// cudaGetSymbolAddress and passed to the kernel.
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_mu;
+void* g_static_ptr[64] = {nullptr};
+
+// Device address of g_static_scratch on the current device (set-up on the
+// first call per device, with that device current).
+sa_status static_scratch(unsigned char** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(SA_ERR_UNSUPPORTED, "device ordinal %d: at most 64 devices", dev);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    g_static_ptr[dev] = p;
+  }
+  *out = static_cast<unsigned char*>(g_static_ptr[dev]);
+  return SA_OK;
+}
+
+}  // namespace
+}  // namespace sa
+
+extern "C" sa_status sa_sparse_attn_given_idx_noalloc(const sa_params* p, const void* Q, const void* K,
+                                                      const void* V, const int32_t* idx, int32_t idx_len,
+                                                      void* O, float* lse, void* stream) {
+  const bool prefill = p && p->select == SA_SEL_TILE_MAX;
+  sa_status st = check_params(p, prefill);
+  if (st != SA_OK) return st;
+  if (prefill) return fail(SA_ERR_UNSUPPORTED, "prefill index tables are not built in this library version");
+  if (!Q || !K || !V || !O) return fail(SA_ERR_INVALID, "Q, K, V and O must be non-NULL");
+  if (idx_len < 0 || idx_len > 4096) return fail(SA_ERR_INVALID, "idx_len %d must be in [0, 4096]", idx_len);
+  if (idx_len > 0 && !idx) return fail(SA_ERR_INVALID, "idx is NULL");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return fail(SA_ERR_INVALID, "Q, K, V and O must be 16-byte aligned");
+  DecodeGeom g;
+  DecodePlan plan;
+  if ((st = plan_for(p, idx_len, &g, &plan)) != SA_OK) return st;
+  const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_GIVEN_IDX);
+  if (L.total > kStaticScratchBytes)
+    return fail(SA_ERR_WORKSPACE,
+                "this problem needs %zu bytes of scratch; the allocation-free entry point has a static "
+                "array of %zu bytes (use sa_sparse_attn_given_idx with a workspace)",
+                L.total, kStaticScratchBytes);
+  unsigned char* w = nullptr;
+  if ((st = static_scratch(&w)) != SA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The array keeps the previous call's contents: the status word and the
+  // tickets must start at zero.
+  cudaError_t e = cudaMemsetAsync(w, 0, L.part_O, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (static scratch)");
+  DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, idx, idx_len, O, lse, w, L);
+  a.check_idx = 1;
+  a.pdl = 0;
+  e = launch_decode_attn(a, plan, p->dtype == SA_BF16, p->out_dtype == SA_BF16, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+  return SA_OK;
+}

@@ -29,7 +29,7 @@ SA_OP_SCORE_TOPK, SA_OP_GIVEN_IDX, SA_OP_DECODE, SA_OP_PREFILL = 0, 1, 2, 3
 
 EXPORTED = ["sa_version", "sa_workspace_size", "sa_workspace_init", "sa_pool_keys", "sa_score_topk",
             "sa_sparse_attn_given_idx", "sa_sparse_attn_decode", "sa_sparse_attn_prefill",
-            "sa_read_status", "sa_status_string", "sa_last_error"]
+            "sa_read_status", "sa_status_string", "sa_last_error", "sa_sparse_attn_given_idx_noalloc"]
 
 
 class SaParams(ctypes.Structure):
@@ -59,6 +59,7 @@ _sig = {
     "sa_sparse_attn_given_idx": (_i32, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     "sa_sparse_attn_decode": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "sa_sparse_attn_prefill": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "sa_sparse_attn_given_idx_noalloc": (_i32, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp]),
     "sa_read_status": (_i32, [_vp, _vp]),
     "sa_status_string": (ctypes.c_char_p, [_i32]),
     "sa_last_error": (ctypes.c_char_p, []),
@@ -156,6 +157,14 @@ def sparse_attn_given_idx(p: SaParams, Q, K, V, idx, O, lse=None, ws=None, strea
     _check(_lib.sa_sparse_attn_given_idx(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
                                          idx_len, _ptr(O), _ptr(lse), _ptr(ws),
                                          0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def sparse_attn_given_idx_noalloc(p: SaParams, Q, K, V, idx, O, lse=None, stream=None):
+    """sa_sparse_attn_given_idx without a workspace: scratch comes from the
+    library's static device array (for callers that cannot allocate)."""
+    idx_len = 0 if idx is None else int(idx.shape[-1])
+    _check(_lib.sa_sparse_attn_given_idx_noalloc(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
+                                                 idx_len, _ptr(O), _ptr(lse), _stream(stream)))
 
 
 def sparse_attn_decode(p: SaParams, Q, K, V, Kc, O, lse=None, idx_out=None, ws=None, stream=None):
