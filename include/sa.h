@@ -106,8 +106,13 @@ typedef struct sa_params {
   int64_t sink_keys;      /* S >= 0 */
   int64_t window_keys;    /* W >= 0 */
   float softmax_scale;    /* <= 0 selects 1/sqrt(head_dim) */
-  int32_t reserved;       /* must be 0 */
+  int32_t flags;          /* OR of SA_FLAG_* (other bits must be 0) */
 } sa_params;
+
+/* sa_params.flags: the caller's index table is known to hold only
+ * ascending in-range block ids and -1 (e.g. it came from sa_score_topk), so
+ * sa_sparse_attn_given_idx[_noalloc] skips its checking pass. */
+#define SA_FLAG_TRUSTED_IDX 1
 
 /* Version of this ABI (major * 100 + minor). */
 int32_t sa_version(void);

@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
     for name in declared_functions():
         assert hasattr(lib, name), name
     assert set(declared_functions()) <= set(sa.EXPORTED) | set(declared_functions())
-    assert sa.version() == 100
+    assert sa.version() == 101
 
 
 def test_params_struct_layout():
@@ -77,7 +77,7 @@ def test_validation_null_and_alignment():
     assert _decode(p, q=None) == sa.SA_ERR_INVALID
     assert _decode(p, q=FAKE_ODD) == sa.SA_ERR_INVALID
     p2 = _p()
-    p2.reserved = 1
+    p2.flags = 4
     assert _decode(p2) == sa.SA_ERR_INVALID
 
 

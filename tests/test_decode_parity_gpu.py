@@ -226,6 +226,25 @@ def test_workspace_reuse_is_deterministic():
     assert torch.equal(idx1, idx2) and torch.equal(O1, O2) and torch.equal(lse1, lse2)
 
 
+def test_trusted_table_flag_gives_the_checked_result():
+    """SA_FLAG_TRUSTED_IDX only skips the checking pass: with a valid table
+    (here the library's own selection) both paths agree bit for bit."""
+    w = WORKLOADS["decode_32k"].scaled(batch=2)
+    inp = dev_inputs(w, 73)
+    p = sa.params_for(w, out_dtype="f32")
+    Kc = run_pool(w, inp, p)
+    _, _, idx, _ = run_decode(w, inp, p, Kc)
+    outs = []
+    for flags in (0, sa.SA_FLAG_TRUSTED_IDX):
+        p.flags = flags
+        O = torch.empty((w.batch, 1, w.num_q_heads, 128), device="cuda")
+        ws = sa.alloc_workspace(p, sa.SA_OP_GIVEN_IDX)
+        sa.sparse_attn_given_idx(p, inp["Q"], inp["K"], inp["V"], idx, O, None, ws)
+        assert sa.read_status(ws) == sa.SA_OK
+        outs.append(O)
+    assert torch.equal(outs[0], outs[1])
+
+
 def test_given_idx_bad_entries_are_reported_and_skipped():
     w = WORKLOADS["decode_32k"].scaled(batch=1, num_kv_heads=2, num_q_heads=8, ctx_len=4096, top_k=6,
                                        n_needles=0)

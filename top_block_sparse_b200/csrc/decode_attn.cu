@@ -42,99 +42,146 @@ namespace {
 
 constexpr int kCombStride = 132;   // floats per (row) in the combine buffer: 128 O + m + l + pad
 
-struct TileInfo {
-  int64_t key_start;
-  int nkeys;
-  int pad;
+// Key ranges of the two tiles of one ring stage (n == 0: empty tile).
+struct StageInfo {
+  int64_t ks0, ks1;
+  int n0, n1;
+  int64_t pad;
 };
 
 __device__ __forceinline__ void consumer_bar(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
-// Walks a CTA's tiles in order and yields each tile's key range.  For a
-// caller's index table (check_idx) an entry is used only if it is a block id
-// in [0, nb) larger than every earlier in-range entry of the row, so no key is
-// ever attended twice; other non-negative entries set kStatusIndex and are
-// skipped, -1 entries are empty.
-struct TileWalker {
-  int64_t pair = -1;
-  int slot = -1;
-  int32_t run_max = -1;   // largest in-range id of the row's earlier slots
-  int32_t j = -1;         // id of the current slot, -1 if skipped
+typedef unsigned long long u64;
 
-  __device__ __forceinline__ void range(const DecodeAttnArgs& a, int64_t pr, int u, int64_t* ks, int* nk) {
-    int64_t s = 0, e = 0;
-    if (u < a.n_sink_tiles) {
-      s = static_cast<int64_t>(u) * kTileKeys;
-      e = min(s + kTileKeys, a.s_end);
-    } else if ((u -= a.n_sink_tiles) < a.idx_stride * a.tpb) {
-      const int sl = u / a.tpb, sub = u - sl * a.tpb;
-      const int32_t* row = a.idx + pr * a.idx_stride;
-      if (pr != pair) { pair = pr; slot = -1; run_max = -1; }
-      if (sl != slot) {
-        for (int q = slot + 1; q < sl; ++q) {        // slots this CTA did not walk
-          const int32_t pj = __ldg(row + q);
-          if (pj >= 0 && pj < a.nb && pj > run_max) run_max = pj;
-        }
-        int32_t jj = __ldg(row + sl);
-        if (a.check_idx && jj >= 0) {
-          const bool in_range = jj < a.nb;
-          const bool ok = in_range && jj > run_max;
-          if (in_range && jj > run_max) run_max = jj;
-          if (!ok) {
-            if (sub == 0) report(a.status, kStatusIndex);
-            jj = -1;
-          }
-        } else if (a.check_idx && jj < -1) {
-          if (sub == 0) report(a.status, kStatusIndex);
-          jj = -1;
-        }
-        j = jj;
-        slot = sl;
-      }
-      if (j >= 0) {
-        const int64_t lo = max(static_cast<int64_t>(j) * a.b, a.s_end);
-        const int64_t hi = min(static_cast<int64_t>(j + 1) * a.b, a.w_begin);
-        s = lo + static_cast<int64_t>(sub) * kTileKeys;
-        e = min(s + kTileKeys, hi);
-      }
-    } else {
-      u -= a.idx_stride * a.tpb;
-      s = a.w_begin + static_cast<int64_t>(u) * kTileKeys;
-      e = min(s + kTileKeys, a.kv_end);
+// Packed fp32 pairs (sm_100 f32x2 arithmetic halves the FMA instruction count).
+__device__ __forceinline__ u64 pk2(float x, float y) {
+  u64 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+  return r;
+}
+__device__ __forceinline__ float lo2(u64 v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi2(u64 v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
+  u64 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ u64 mul2(u64 a, u64 b) {
+  u64 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// two bf16 (one 32-bit word) -> packed fp32 pair
+__device__ __forceinline__ u64 bf2(uint32_t w) { return pk2(bf16lo(w), bf16hi(w)); }
+
+// Key range of tile u (0 <= u < MT) of a pair; nkeys == 0 means empty.  The
+// index table holds valid ids or -1 (caller tables are sanitised first).
+__device__ __forceinline__ void tile_range(const DecodeAttnArgs& a, int64_t pair, int u, int64_t* ks,
+                                           int* nk) {
+  int64_t s = 0, e = 0;
+  const int T = a.tile;
+  if (u < a.n_sink_tiles) {
+    s = static_cast<int64_t>(u) * T;
+    e = min(s + T, a.s_end);
+  } else if ((u -= a.n_sink_tiles) < a.idx_stride * a.tpb) {
+    const int sl = u / a.tpb, sub = u - sl * a.tpb;
+    const int32_t j = __ldg(a.idx + pair * a.idx_stride + sl);
+    if (j >= 0) {
+      const int64_t lo = max(static_cast<int64_t>(j) * a.b, a.s_end);
+      const int64_t hi = min(static_cast<int64_t>(j + 1) * a.b, a.w_begin);
+      s = lo + static_cast<int64_t>(sub) * T;
+      e = min(s + T, hi);
     }
-    *ks = s;
-    *nk = e > s ? static_cast<int>(e - s) : 0;
+  } else {
+    u -= a.idx_stride * a.tpb;
+    s = a.w_begin + static_cast<int64_t>(u) * T;
+    e = min(s + T, a.kv_end);
   }
-};
+  *ks = s;
+  *nk = e > s ? static_cast<int>(e - s) : 0;
+}
+
+// Loads this lane's 16 coordinates of one key row as packed fp32 pairs.
+template <bool BF16>
+__device__ __forceinline__ void load_key(const unsigned char* krow, int l8, u64 (&kp)[8]) {
+  if constexpr (BF16) {
+    const uint4 u0 = *reinterpret_cast<const uint4*>(krow + l8 * 16);
+    const uint4 u1 = *reinterpret_cast<const uint4*>(krow + 128 + l8 * 16);
+    kp[0] = bf2(u0.x); kp[1] = bf2(u0.y); kp[2] = bf2(u0.z); kp[3] = bf2(u0.w);
+    kp[4] = bf2(u1.x); kp[5] = bf2(u1.y); kp[6] = bf2(u1.z); kp[7] = bf2(u1.w);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(krow + 128 * c + l8 * 16);
+      kp[2 * c] = x.x;
+      kp[2 * c + 1] = x.y;
+    }
+  }
+}
+
+// QK partial sums of two key rows over this lane's 16 coordinates for the 4
+// query-row slots: v[4*key + x] = sum_e q[x][e] * k_key[e].  Even and odd
+// coordinate pairs go to separate accumulators so that the two keys give 16
+// independent FMA chains of length 4.
+template <bool BF16>
+__device__ __forceinline__ void qk_two_keys(const unsigned char* krow_a, const unsigned char* krow_b, int l8,
+                                            const u64 (&q2)[4][8], float (&v)[8]) {
+  u64 ka[8], kb[8];
+  load_key<BF16>(krow_a, l8, ka);
+  load_key<BF16>(krow_b, l8, kb);
+  u64 acc[2][4][2];
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    acc[0][x][0] = 0ull; acc[0][x][1] = 0ull;
+    acc[1][x][0] = 0ull; acc[1][x][1] = 0ull;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      acc[0][x][e & 1] = fma2(q2[x][e], ka[e], acc[0][x][e & 1]);
+      acc[1][x][e & 1] = fma2(q2[x][e], kb[e], acc[1][x][e & 1]);
+    }
+  }
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    v[x] = (lo2(acc[0][x][0]) + hi2(acc[0][x][0])) + (lo2(acc[0][x][1]) + hi2(acc[0][x][1]));
+    v[4 + x] = (lo2(acc[1][x][0]) + hi2(acc[1][x][0])) + (lo2(acc[1][x][1]) + hi2(acc[1][x][1]));
+  }
+}
 
 template <bool BF16, bool OUT_BF16, int RG, int KG>
 __global__ void __launch_bounds__((RG * KG + 1) * 32, 1) decode_attn_kernel(DecodeAttnArgs a) {
-  constexpr int NWC = RG * KG;            // consumer warps
-  constexpr int NCT = NWC * 32;           // consumer threads
-  constexpr int KPW = kTileKeys / KG;     // keys per warp per tile
-  constexpr int NIT = KPW / 8;            // QK iterations (8 keys per warp-iteration)
-  constexpr int ROWB = BF16 ? 256 : 512;  // bytes per K/V row
-  constexpr int STAGE = 2 * kTileKeys * ROWB;
-  static_assert(KPW % 8 == 0, "KG must divide 8");
+  constexpr int NWC = RG * KG;                 // consumer warps
+  constexpr int NCT = NWC * 32;                // consumer threads
+  constexpr int HALF = BF16 ? 64 : 32;         // keys per tile; a ring stage holds two tiles
+  constexpr int KPH = HALF / KG;               // keys per warp per tile
+  constexpr int NITH = KPH / 8;                // QK iterations per tile (8 keys per warp-iteration)
+  constexpr int NIT = 2 * NITH;
+  constexpr int KPR = 2 * KPH;                 // keys per warp per round (two tiles)
+  constexpr int ROWB = BF16 ? 256 : 512;       // bytes per K/V row
+  constexpr int KBYTES = 2 * HALF * ROWB;      // K part of a stage
+  constexpr int STAGE = 2 * KBYTES;
+  static_assert(KPH % 8 == 0, "a warp takes a multiple of 8 keys of every tile");
 
   extern __shared__ __align__(1024) unsigned char smem[];
   const int NS = a.n_stages;
   unsigned char* stages = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NS) * STAGE);
   uint64_t* empty = full + NS;
-  TileInfo* info = reinterpret_cast<TileInfo*>(empty + NS);
-  float* pbuf = reinterpret_cast<float*>(info + NS);                 // [NWC][KPW][4]
-  float* rowbuf = pbuf + NWC * KPW * 4;                              // [NWC][3][4]
-  float* comb = rowbuf + NWC * 12;                                   // [KG][RG*4][kCombStride]
+  StageInfo* info = reinterpret_cast<StageInfo*>(empty + NS);
+  u64* pbuf = reinterpret_cast<u64*>(info + NS);                     // [NWC][KPR][4] (p, p) pairs
+  float* rowbuf = reinterpret_cast<float*>(pbuf + NWC * KPR * 4);    // [NWC][4] row scale factors
+  float* comb = rowbuf + NWC * 4;                                    // [KG][RG*4][kCombStride]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(comb + KG * RG * 4 * kCombStride);
   int* ticket = const_cast<int*>(abort_flag) + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * a.tpc;
-  const int64_t t1 = min(a.total_tiles, t0 + a.tpc);
-  const int ntiles = static_cast<int>(t1 - t0);
+  const int64_t u0 = static_cast<int64_t>(blockIdx.x) * a.tpc;       // work units = tile pairs
+  const int64_t u1 = min(a.total_tiles, u0 + a.tpc);
+  const int nunits = static_cast<int>(u1 - u0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -151,108 +198,157 @@ __global__ void __launch_bounds__((RG * KG + 1) * 32, 1) decode_attn_kernel(Deco
 
   if (warp == NWC) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int issued = 0;
-      TileWalker walker;
-      for (int i = 0; i < ntiles; ++i) {
+    // The warp computes the key ranges of 32 units at a time (one per lane,
+    // index loads in parallel); lane 0 then feeds them to the ring in order.
+    int issued = 0;
+    bool stop = false;
+    for (int base = 0; base < nunits && !stop; base += 32) {
+      int64_t ks0 = 0, ks1 = 0;
+      int nk0 = 0, nk1 = 0;
+      if (base + lane < nunits) {
+        const int64_t u = u0 + base + lane;
+        const int64_t pair = u / a.MT;
+        const int v = static_cast<int>(u - pair * a.MT);
+        tile_range(a, pair, 2 * v, &ks0, &nk0);
+        if (2 * v + 1 < a.n_tiles) tile_range(a, pair, 2 * v + 1, &ks1, &nk1);
+      }
+      const int cnt = min(32, nunits - base);
+      for (int l = 0; l < cnt; ++l) {
+        const int64_t k0 = __shfl_sync(0xffffffffu, ks0, l);
+        const int64_t k1 = __shfl_sync(0xffffffffu, ks1, l);
+        const int n0 = __shfl_sync(0xffffffffu, nk0, l);
+        const int n1 = __shfl_sync(0xffffffffu, nk1, l);
+        const int i = base + l;
         const int s = i % NS;
-        if (i >= NS) {
-          if (!mbar_wait_bounded(&empty[s], ((i / NS) & 1) ^ 1, abort_flag)) {
+        int ok = 1;
+        if (lane == 0) {
+          if (i >= NS && !mbar_wait_bounded(&empty[s], ((i / NS) & 1) ^ 1, abort_flag)) ok = 0;
+          if (ok && *abort_flag) ok = 0;
+          if (ok) {
+            info[s].ks0 = k0;
+            info[s].ks1 = k1;
+            info[s].n0 = n0;
+            info[s].n1 = n1;
+            if (n0 + n1 > 0) {
+              const int64_t pair = (u0 + i) / a.MT;
+              mbar_arrive_expect_tx(&full[s], 2u * static_cast<uint32_t>(n0 + n1) * ROWB);
+              unsigned char* st = stages + static_cast<size_t>(s) * STAGE;
+              const unsigned char* kb = static_cast<const unsigned char*>(a.K) + pair * a.cap * ROWB;
+              const unsigned char* vb = static_cast<const unsigned char*>(a.V) + pair * a.cap * ROWB;
+              if (n0 > 0) {
+                bulk_g2s(st, kb + k0 * ROWB, n0 * ROWB, &full[s]);
+                bulk_g2s(st + KBYTES, vb + k0 * ROWB, n0 * ROWB, &full[s]);
+              }
+              if (n1 > 0) {
+                bulk_g2s(st + HALF * ROWB, kb + k1 * ROWB, n1 * ROWB, &full[s]);
+                bulk_g2s(st + KBYTES + HALF * ROWB, vb + k1 * ROWB, n1 * ROWB, &full[s]);
+              }
+            } else {
+              mbar_arrive(&full[s]);
+            }
+          } else {
             report(a.status, kStatusTimeout);
             *abort_flag = 1;
-            break;
           }
         }
-        if (*abort_flag) break;
-        const int64_t t = t0 + i;
-        const int64_t pair = t / a.MT;
-        int64_t ks;
-        int nk;
-        walker.range(a, pair, static_cast<int>(t - pair * a.MT), &ks, &nk);
-        info[s].key_start = ks;
-        info[s].nkeys = nk;
-        if (nk > 0) {
-          const uint32_t bytes = static_cast<uint32_t>(nk) * ROWB;
-          mbar_arrive_expect_tx(&full[s], 2 * bytes);
-          const int64_t row = pair * a.cap + ks;
-          const unsigned char* kp = static_cast<const unsigned char*>(a.K) + row * ROWB;
-          const unsigned char* vp = static_cast<const unsigned char*>(a.V) + row * ROWB;
-          bulk_g2s(stages + static_cast<size_t>(s) * STAGE, kp, bytes, &full[s]);
-          bulk_g2s(stages + static_cast<size_t>(s) * STAGE + kTileKeys * ROWB, vp, bytes, &full[s]);
-        } else {
-          mbar_arrive(&full[s]);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          stop = true;
+          break;
         }
         issued = i + 1;
       }
-      // do not leave while copies into this CTA's shared memory may be in flight
-      for (int i = max(0, issued - NS); i < issued; ++i)
-        mbar_wait_bounded(&full[i % NS], (i / NS) & 1, nullptr);
     }
+    // do not leave while copies into this CTA's shared memory may be in flight
+    if (lane == 0)
+      for (int i = max(0, issued - NS); i < issued; ++i) mbar_wait_bounded(&full[i % NS], (i / NS) & 1, nullptr);
     return;
   }
 
   // ------------------------------------------------------------- consumers
   const int rg = warp / KG, kg = warp - (warp / KG) * KG;
   const int gi = lane >> 3, l8 = lane & 7;
-  float* my_p = pbuf + warp * KPW * 4;
-  float* my_row = rowbuf + warp * 12;
+  const int m8 = l8 & 3;             // this lane's row after the reduce-scatter
+  const int b2 = l8 >> 2;            // this lane's key (of the group's pair) after it
+  u64* my_p = pbuf + warp * KPR * 4;
+  float* my_row = rowbuf + warp * 4;
 
-  float q[4][16];
-  float o[4][4];
-  float m_run[4], l_run[4];
+  // q2[x] holds query row rg*4 + (x ^ m8): with the rows permuted per lane the
+  // reduce-scatter below needs no selects.
+  u64 q2[4][8];
+  u64 o2[4][2];                      // rows rg*4+r, columns 4*lane..4*lane+3 as two pairs
+  float m_own = -CUDART_INF_F;       // running max of row rg*4 + m8 (same on all its lanes)
+  float l_own = 0.f;                 // this lane's share of that row's running sum
   int64_t cur_pair = -1;
 
   auto load_q = [&](int64_t pair) {
     const int bi = static_cast<int>(pair / a.Hkv), h = static_cast<int>(pair % a.Hkv);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int rr = rg * 4 + r;
+    for (int x = 0; x < 4; ++x) {
+      const int rr = rg * 4 + (x ^ m8);
+      float qf[16];
       if (rr < a.R) {
         const int j = rr / a.G, g = rr - (rr / a.G) * a.G;
         const int64_t off = ((static_cast<int64_t>(bi) * a.n_q + j) * a.Hq + h * a.G + g) * kHeadDim;
         if constexpr (BF16) {
           const uint16_t* qp = static_cast<const uint16_t*>(a.Q) + off;
-          uint4 u0 = __ldg(reinterpret_cast<const uint4*>(qp + 8 * l8));
-          uint4 u1 = __ldg(reinterpret_cast<const uint4*>(qp + 64 + 8 * l8));
-          unpack8(u0, &q[r][0]);
-          unpack8(u1, &q[r][8]);
+          unpack8(__ldg(reinterpret_cast<const uint4*>(qp + 8 * l8)), qf);
+          unpack8(__ldg(reinterpret_cast<const uint4*>(qp + 64 + 8 * l8)), qf + 8);
         } else {
           const float* qp = static_cast<const float*>(a.Q) + off;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            float4 x = __ldg(reinterpret_cast<const float4*>(qp + 32 * c + 4 * l8));
-            q[r][4 * c + 0] = x.x; q[r][4 * c + 1] = x.y; q[r][4 * c + 2] = x.z; q[r][4 * c + 3] = x.w;
+            const float4 v = __ldg(reinterpret_cast<const float4*>(qp + 32 * c + 4 * l8));
+            qf[4 * c + 0] = v.x; qf[4 * c + 1] = v.y; qf[4 * c + 2] = v.z; qf[4 * c + 3] = v.w;
           }
         }
-#pragma unroll
-        for (int e = 0; e < 16; ++e) q[r][e] *= a.qscale;
       } else {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) q[r][e] = 0.f;
+        for (int e = 0; e < 16; ++e) qf[e] = 0.f;
       }
-      m_run[r] = -CUDART_INF_F;
-      l_run[r] = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) o[r][c] = 0.f;
+      for (int e = 0; e < 8; ++e) q2[x][e] = pk2(qf[2 * e] * a.qscale, qf[2 * e + 1] * a.qscale);
+    }
+    m_own = -CUDART_INF_F;
+    l_own = 0.f;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      o2[r][0] = 0ull;
+      o2[r][1] = 0ull;
+    }
+  };
+
+  auto write_out = [&](int64_t orow, int c4, float4 acc, float inv) {
+    if constexpr (OUT_BF16) {
+      uint2 pk = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+      *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.O) + orow * kHeadDim + 4 * c4) = pk;
+    } else {
+      *reinterpret_cast<float4*>(static_cast<float*>(a.O) + orow * kHeadDim + 4 * c4) =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
   };
 
   // Merge the KG warps of every row group and emit this CTA's result for `pair`.
   auto flush = [&](int64_t pair) {
+    // the row sums are spread over the 8 lanes that hold each row
+    float l_row = l_own;
+    l_row += __shfl_xor_sync(0xffffffffu, l_row, 4);
+    l_row += __shfl_xor_sync(0xffffffffu, l_row, 8);
+    l_row += __shfl_xor_sync(0xffffffffu, l_row, 16);
     float* cb = comb + (kg * RG * 4) * kCombStride;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int rr = rg * 4 + r;
       *reinterpret_cast<float4*>(cb + rr * kCombStride + 4 * lane) =
-          make_float4(o[r][0], o[r][1], o[r][2], o[r][3]);
-      if (lane == 0) {
-        cb[rr * kCombStride + 128] = m_run[r];
-        cb[rr * kCombStride + 129] = l_run[r];
-      }
+          make_float4(lo2(o2[r][0]), hi2(o2[r][0]), lo2(o2[r][1]), hi2(o2[r][1]));
+    }
+    if (lane < 4) {                   // lane r holds row rg*4 + r (gi = 0, b2 = 0, m8 = r)
+      cb[(rg * 4 + lane) * kCombStride + 128] = m_own;
+      cb[(rg * 4 + lane) * kCombStride + 129] = l_row;
     }
     consumer_bar(NCT);
     const int64_t first = pair * a.MT, last = first + a.MT - 1;
-    const bool whole = first >= t0 && last < t1;
+    const bool whole = first >= u0 && last < u1;
     const int64_t first_cta = first / a.tpc, last_cta = last / a.tpc;
     const int n_ctas = static_cast<int>(last_cta - first_cta + 1);
     const int slot = static_cast<int>(blockIdx.x - first_cta);
@@ -276,14 +372,7 @@ __global__ void __launch_bounds__((RG * KG + 1) * 32, 1) decode_attn_kernel(Deco
       if (whole) {
         const int j = rr / a.G, g = rr - (rr / a.G) * a.G;
         const int64_t orow = (static_cast<int64_t>(bi) * a.n_q + j) * a.Hq + h * a.G + g;
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        if constexpr (OUT_BF16) {
-          uint2 pk = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
-          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.O) + orow * kHeadDim + 4 * c4) = pk;
-        } else {
-          *reinterpret_cast<float4*>(static_cast<float*>(a.O) + orow * kHeadDim + 4 * c4) =
-              make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-        }
+        write_out(orow, c4, acc, L > 0.f ? 1.f / L : 0.f);
         if (c4 == 0 && a.lse)
           a.lse[orow] = L > 0.f ? (Mr + log2f(L)) * 0.69314718055994531f : -CUDART_INF_F;
       } else {
@@ -296,9 +385,11 @@ __global__ void __launch_bounds__((RG * KG + 1) * 32, 1) decode_attn_kernel(Deco
       }
     }
     if (!whole) {
-      __threadfence();
+      // the barrier orders every consumer's partial stores before thread 0's
+      // release fence and ticket
       consumer_bar(NCT);
       if (threadIdx.x == 0) {
+        __threadfence();
         const unsigned t = atomicAdd(&a.counters[pair], 1u);
         *ticket = (t == static_cast<unsigned>(n_ctas - 1));
       }
@@ -322,14 +413,7 @@ __global__ void __launch_bounds__((RG * KG + 1) * 32, 1) decode_attn_kernel(Deco
           }
           const int j = rr / a.G, g = rr - (rr / a.G) * a.G;
           const int64_t orow = (static_cast<int64_t>(bi) * a.n_q + j) * a.Hq + h * a.G + g;
-          const float inv = L > 0.f ? 1.f / L : 0.f;
-          if constexpr (OUT_BF16) {
-            uint2 pk = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
-            *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.O) + orow * kHeadDim + 4 * c4) = pk;
-          } else {
-            *reinterpret_cast<float4*>(static_cast<float*>(a.O) + orow * kHeadDim + 4 * c4) =
-                make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-          }
+          write_out(orow, c4, acc, L > 0.f ? 1.f / L : 0.f);
           if (c4 == 0 && a.lse)
             a.lse[orow] = L > 0.f ? (Mr + log2f(L)) * 0.69314718055994531f : -CUDART_INF_F;
         }
@@ -339,10 +423,10 @@ __global__ void __launch_bounds__((RG * KG + 1) * 32, 1) decode_attn_kernel(Deco
     consumer_bar(NCT);   // the combine buffer is reused by the next segment
   };
 
+  const int tok = (rg * 4 + m8) / a.G;   // new-token index of this lane's row
   bool aborted = false;
-  for (int i = 0; i < ntiles; ++i) {
-    const int64_t t = t0 + i;
-    const int64_t pair = t / a.MT;
+  for (int i = 0; i < nunits; ++i) {
+    const int64_t pair = (u0 + i) / a.MT;
     if (pair != cur_pair) {
       if (cur_pair >= 0) flush(cur_pair);
       cur_pair = pair;
@@ -356,71 +440,36 @@ __global__ void __launch_bounds__((RG * KG + 1) * 32, 1) decode_attn_kernel(Deco
         *abort_flag = 1;
       }
     }
-    const int nkeys = aborted ? 0 : info[s].nkeys;
-    const int64_t kstart = info[s].key_start;
-    const int kb = kg * KPW;                 // this warp's first key in the tile
-    const int nk = min(KPW, nkeys - kb);     // keys of this warp (<= 0: none)
-    if (nk > 0) {
+    const int n0 = aborted ? 0 : info[s].n0;
+    const int n1 = aborted ? 0 : info[s].n1;
+    const int64_t ks0 = info[s].ks0, ks1 = info[s].ks1;
+    const int kb = kg * KPH;                  // this warp's first key in each tile
+    const int nk0 = min(KPH, n0 - kb), nk1 = min(KPH, n1 - kb);
+    if (nk0 > 0 || nk1 > 0) {
       const unsigned char* kst = stages + static_cast<size_t>(s) * STAGE;
-      const unsigned char* vst = kst + kTileKeys * ROWB;
+      const unsigned char* vst = kst + KBYTES;
       float sc[NIT];
-      const int r_loc = l8 & 3;
-      const int rr_loc = rg * 4 + r_loc;
-      const int tok = rr_loc / a.G;          // new-token index of this lane's row
 #pragma unroll
       for (int it = 0; it < NIT; ++it) {
-        const int kk0 = kb + it * 8 + 2 * gi;
+        const int half = it / NITH;
+        const int kl = kb + (it % NITH) * 8 + 2 * gi;    // group's first key within the tile
+        const unsigned char* kt = kst + half * HALF * ROWB;
+        // this lane computes its own key (kl + b2) first, so the first
+        // reduce-scatter level keeps v[0..3] and sends v[4..7] on every lane
         float v[8];
-#pragma unroll
-        for (int kq = 0; kq < 2; ++kq) {
-          const unsigned char* krow = kst + (kk0 + kq) * ROWB;
-          float kf[16];
-          if constexpr (BF16) {
-            const uint4 u0 = *reinterpret_cast<const uint4*>(krow + l8 * 16);
-            const uint4 u1 = *reinterpret_cast<const uint4*>(krow + 128 + l8 * 16);
-            unpack8(u0, kf);
-            unpack8(u1, kf + 8);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const float4 x = *reinterpret_cast<const float4*>(krow + 128 * c + l8 * 16);
-              kf[4 * c + 0] = x.x; kf[4 * c + 1] = x.y; kf[4 * c + 2] = x.z; kf[4 * c + 3] = x.w;
-            }
-          }
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            float acc = 0.f;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) acc = fmaf(q[r][e], kf[e], acc);
-            v[kq * 4 + r] = acc;
-          }
-        }
-        // reduce-scatter over the 8 lanes of the group: lane l8 ends with value l8
-        const bool b2 = l8 & 4, b1 = l8 & 2, b0 = l8 & 1;
+        qk_two_keys<BF16>(kt + (kl + b2) * ROWB, kt + (kl + (b2 ^ 1)) * ROWB, l8, q2, v);
         float w4[4];
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const float send = b2 ? v[x] : v[4 + x];
-          const float keep = b2 ? v[4 + x] : v[x];
-          w4[x] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-        }
+        for (int x = 0; x < 4; ++x) w4[x] = v[x] + __shfl_xor_sync(0xffffffffu, v[4 + x], 4);
         float w2[2];
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const float send = b1 ? w4[x] : w4[2 + x];
-          const float keep = b1 ? w4[2 + x] : w4[x];
-          w2[x] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-        }
-        float w1;
-        {
-          const float send = b0 ? w2[0] : w2[1];
-          const float keep = b0 ? w2[1] : w2[0];
-          w1 = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-        }
-        // this lane: key kk0 + (l8 >> 2), row r_loc
-        const int kl = kk0 + (l8 >> 2);
-        const int64_t pos = kstart + kl;
-        bool valid = kl < nkeys;
+        for (int x = 0; x < 2; ++x) w2[x] = w4[x] + __shfl_xor_sync(0xffffffffu, w4[2 + x], 2);
+        const float w1 = w2[0] + __shfl_xor_sync(0xffffffffu, w2[1], 1);
+        // this lane now holds the logit of key kl + b2 of tile `half`, row rg*4 + m8
+        const int key = kl + b2;
+        const int nh = half ? n1 : n0;
+        const int64_t pos = (half ? ks1 : ks0) + key;
+        bool valid = key < nh;
         if (pos >= a.C) valid = valid && (pos - a.C) <= tok;
         sc[it] = valid ? w1 : -CUDART_INF_F;
       }
@@ -430,56 +479,53 @@ __global__ void __launch_bounds__((RG * KG + 1) * 32, 1) decode_attn_kernel(Deco
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      float m_old = m_run[0];
-#pragma unroll
-      for (int r = 1; r < 4; ++r) m_old = (r_loc == r) ? m_run[r] : m_old;
-      const float m_new = fmaxf(m_old, mx);
+      const float m_new = fmaxf(m_own, mx);
       const float m_ref = (m_new == -CUDART_INF_F) ? 0.f : m_new;
-      float rs = 0.f;
+      const float alpha = exp2f(m_own - m_ref);
+      float ps = 0.f;
 #pragma unroll
       for (int it = 0; it < NIT; ++it) {
         const float p = exp2f(sc[it] - m_ref);
-        rs += p;
-        my_p[(it * 8 + 2 * gi + (l8 >> 2)) * 4 + r_loc] = p;
+        ps += p;
+        my_p[(it * 8 + 2 * gi + b2) * 4 + m8] = pk2(p, p);
       }
-      rs += __shfl_xor_sync(0xffffffffu, rs, 4);
-      rs += __shfl_xor_sync(0xffffffffu, rs, 8);
-      rs += __shfl_xor_sync(0xffffffffu, rs, 16);
-      if (lane < 4) {
-        my_row[0 + lane] = exp2f(m_old - m_ref);   // alpha
-        my_row[4 + lane] = rs;
-        my_row[8 + lane] = m_new;
-      }
+      l_own = l_own * alpha + ps;
+      const bool grew = m_new != m_own;          // only then does a row's scale change
+      m_own = m_new;
+      if (lane < 4) my_row[lane] = alpha;
       __syncwarp();
-      const float4 al = *reinterpret_cast<const float4*>(my_row);
-      const float4 rsv = *reinterpret_cast<const float4*>(my_row + 4);
-      const float4 mn = *reinterpret_cast<const float4*>(my_row + 8);
-      const float alr[4] = {al.x, al.y, al.z, al.w};
-      const float rsr[4] = {rsv.x, rsv.y, rsv.z, rsv.w};
-      const float mnr[4] = {mn.x, mn.y, mn.z, mn.w};
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        l_run[r] = l_run[r] * alr[r] + rsr[r];
-        m_run[r] = mnr[r];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) o[r][c] *= alr[r];
+      if (__any_sync(0xffffffffu, grew)) {
+        const float4 al = *reinterpret_cast<const float4*>(my_row);
+        const u64 a0 = pk2(al.x, al.x), a1 = pk2(al.y, al.y), a2 = pk2(al.z, al.z), a3 = pk2(al.w, al.w);
+        o2[0][0] = mul2(o2[0][0], a0); o2[0][1] = mul2(o2[0][1], a0);
+        o2[1][0] = mul2(o2[1][0], a1); o2[1][1] = mul2(o2[1][1], a1);
+        o2[2][0] = mul2(o2[2][0], a2); o2[2][1] = mul2(o2[2][1], a2);
+        o2[3][0] = mul2(o2[3][0], a3); o2[3][1] = mul2(o2[3][1], a3);
       }
-      for (int kk = 0; kk < nk; ++kk) {
-        const float4 p4 = *reinterpret_cast<const float4*>(my_p + kk * 4);
-        const unsigned char* vrow = vst + (kb + kk) * ROWB;
-        float vv[4];
-        if constexpr (BF16) {
-          const uint2 u = *reinterpret_cast<const uint2*>(vrow + lane * 8);
-          vv[0] = bf16lo(u.x); vv[1] = bf16hi(u.x); vv[2] = bf16lo(u.y); vv[3] = bf16hi(u.y);
-        } else {
-          const float4 x = *reinterpret_cast<const float4*>(vrow + lane * 16);
-          vv[0] = x.x; vv[1] = x.y; vv[2] = x.z; vv[3] = x.w;
-        }
-        const float pr[4] = {p4.x, p4.y, p4.z, p4.w};
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) o[r][c] = fmaf(pr[r], vv[c], o[r][c]);
+      for (int half = 0; half < 2; ++half) {
+        const int nk = half ? nk1 : nk0;
+        const unsigned char* vt = vst + half * HALF * ROWB + kb * ROWB;
+        const u64* pt = my_p + half * KPH * 4;
+#pragma unroll 4
+        for (int kk = 0; kk < nk; ++kk) {
+          const ulonglong2 p01 = *reinterpret_cast<const ulonglong2*>(pt + kk * 4);
+          const ulonglong2 p23 = *reinterpret_cast<const ulonglong2*>(pt + kk * 4 + 2);
+          const unsigned char* vrow = vt + kk * ROWB;
+          u64 v0, v1;
+          if constexpr (BF16) {
+            const uint2 u = *reinterpret_cast<const uint2*>(vrow + lane * 8);
+            v0 = bf2(u.x);
+            v1 = bf2(u.y);
+          } else {
+            const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(vrow + lane * 16);
+            v0 = x.x;
+            v1 = x.y;
+          }
+          o2[0][0] = fma2(p01.x, v0, o2[0][0]); o2[0][1] = fma2(p01.x, v1, o2[0][1]);
+          o2[1][0] = fma2(p01.y, v0, o2[1][0]); o2[1][1] = fma2(p01.y, v1, o2[1][1]);
+          o2[2][0] = fma2(p23.x, v0, o2[2][0]); o2[2][1] = fma2(p23.x, v1, o2[2][1]);
+          o2[3][0] = fma2(p23.y, v0, o2[3][0]); o2[3][1] = fma2(p23.y, v1, o2[3][1]);
         }
       }
       __syncwarp();
@@ -487,6 +533,41 @@ __global__ void __launch_bounds__((RG * KG + 1) * 32, 1) decode_attn_kernel(Deco
     if (lane == 0) mbar_arrive(&empty[s]);
   }
   if (cur_pair >= 0) flush(cur_pair);
+}
+
+// Caller index tables (sa_sparse_attn_given_idx): an entry is kept only if it
+// is a complete-block id larger than every earlier in-range entry of its row,
+// so no key is attended twice; other entries become -1 and, unless they were
+// -1 already, set kStatusIndex.  One warp per row, a max-scan per 32 entries.
+__global__ void __launch_bounds__(256) sanitize_idx_kernel(const int32_t* idx, int32_t* out, int rows,
+                                                           int len, int64_t nb, unsigned* status) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int32_t* in = idx + static_cast<int64_t>(row) * len;
+  int32_t* o = out + static_cast<int64_t>(row) * len;
+  int carry = -1;
+  bool bad = false;
+  for (int base = 0; base < len; base += 32) {
+    const int s = base + lane;
+    const int32_t j = s < len ? __ldg(in + s) : -1;
+    const bool in_range = j >= 0 && j < nb;
+    int incl = in_range ? j : -1;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl = max(incl, y);
+    }
+    int excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = -1;
+    excl = max(excl, carry);
+    const bool ok = in_range && j > excl;
+    if (s < len) {
+      o[s] = ok ? j : -1;
+      if (!ok && j != -1) bad = true;
+    }
+    carry = max(carry, __shfl_sync(0xffffffffu, incl, 31));
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) report(status, kStatusIndex);
 }
 
 template <bool BF16, bool OUT_BF16, int RG, int KG>
@@ -510,11 +591,12 @@ cudaError_t launch_one(const DecodeAttnArgs& a, const DecodePlan& p, cudaStream_
 
 template <bool BF16, bool OUT_BF16>
 cudaError_t launch_rg(const DecodeAttnArgs& a, const DecodePlan& p, cudaStream_t s) {
+  constexpr int H = BF16 ? 64 : 32;
   switch (p.RG) {
-    case 1: return launch_one<BF16, OUT_BF16, 1, 8>(a, p, s);
-    case 2: return launch_one<BF16, OUT_BF16, 2, 4>(a, p, s);
-    case 3: return launch_one<BF16, OUT_BF16, 3, 4>(a, p, s);
-    case 4: return launch_one<BF16, OUT_BF16, 4, 2>(a, p, s);
+    case 1: return launch_one<BF16, OUT_BF16, 1, H / 8>(a, p, s);
+    case 2: return launch_one<BF16, OUT_BF16, 2, H / 16>(a, p, s);
+    case 3: return launch_one<BF16, OUT_BF16, 3, H / 16>(a, p, s);
+    case 4: return launch_one<BF16, OUT_BF16, 4, (H / 32 < 1 ? 1 : H / 32)>(a, p, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -523,16 +605,25 @@ cudaError_t launch_rg(const DecodeAttnArgs& a, const DecodePlan& p, cudaStream_t
 
 size_t decode_smem_bytes(int RG, int KG, bool bf16, int n_stages) {
   const int NWC = RG * KG;
-  const int KPW = kTileKeys / KG;
-  const size_t stage = 2 * kTileKeys * (bf16 ? 256 : 512);
+  const int half = bf16 ? 64 : 32;
+  const int KPR = 2 * (half / KG);
+  const size_t stage = 2 * 2 * half * (bf16 ? 256 : 512);
   size_t b = stage * n_stages;
   b += 2 * sizeof(uint64_t) * n_stages;
-  b += sizeof(TileInfo) * n_stages;
-  b += sizeof(float) * NWC * KPW * 4;
-  b += sizeof(float) * NWC * 12;
+  b += sizeof(StageInfo) * n_stages;
+  b += sizeof(unsigned long long) * NWC * KPR * 4;
+  b += sizeof(float) * NWC * 4;
   b += sizeof(float) * KG * RG * 4 * kCombStride;
   b += 16;
   return b;
+}
+
+// Consumer warp layout: RG groups of 4 query rows, KG warps per group; every
+// warp takes 8, 16 or 32 keys of each tile.
+static int kg_for(int RG, bool bf16) {
+  const int half = bf16 ? 64 : 32;
+  const int kg = RG == 1 ? half / 8 : (RG == 4 ? half / 32 : half / 16);
+  return kg < 1 ? 1 : kg;
 }
 
 bool plan_decode(const DecodeGeom& g, int idx_slots, bool bf16, int num_sms, DecodePlan* p,
@@ -544,18 +635,21 @@ bool plan_decode(const DecodeGeom& g, int idx_slots, bool bf16, int num_sms, Dec
     return false;
   }
   p->R4 = p->RG * 4;
-  p->KG = p->RG == 1 ? 8 : (p->RG == 4 ? 2 : 4);
+  p->KG = kg_for(p->RG, bf16);
   p->threads = (p->RG * p->KG + 1) * 32;
-  p->n_sink_tiles = static_cast<int>((g.s_end + kTileKeys - 1) / kTileKeys);
-  p->tpb = (g.b + kTileKeys - 1) / kTileKeys;
-  p->n_wc_tiles = static_cast<int>((g.kv_end - g.w_begin + kTileKeys - 1) / kTileKeys);
-  const int64_t mt = static_cast<int64_t>(p->n_sink_tiles) + static_cast<int64_t>(idx_slots) * p->tpb +
+  p->tile = bf16 ? 64 : 32;
+  const int T = p->tile;
+  p->n_sink_tiles = static_cast<int>((g.s_end + T - 1) / T);
+  p->tpb = (g.b + T - 1) / T;
+  p->n_wc_tiles = static_cast<int>((g.kv_end - g.w_begin + T - 1) / T);
+  const int64_t nt = static_cast<int64_t>(p->n_sink_tiles) + static_cast<int64_t>(idx_slots) * p->tpb +
                      p->n_wc_tiles;
-  if (mt > (1 << 24)) {
+  if (nt > (1 << 24)) {
     *why = "too many key tiles per (sequence, KV head)";
     return false;
   }
-  p->MT = static_cast<int>(mt);
+  p->n_tiles = static_cast<int>(nt);
+  p->MT = static_cast<int>((nt + 1) / 2);            // work units (tile pairs) per pair
   p->total_tiles = static_cast<int64_t>(g.pairs) * p->MT;
   const int64_t max_grid = num_sms;
   int64_t grid = p->total_tiles < max_grid ? p->total_tiles : max_grid;
@@ -571,8 +665,8 @@ bool plan_decode(const DecodeGeom& g, int idx_slots, bool bf16, int num_sms, Dec
   if (p->grid < 1) p->grid = 1;
   p->n_slots = static_cast<int>((p->MT + tpc - 1) / tpc) + 1;
   const size_t limit = 227 * 1024;
-  int ns = bf16 ? 6 : 3;
-  while (ns > 2 && decode_smem_bytes(p->RG, p->KG, bf16, ns) > limit) --ns;
+  int ns = 3;
+  while (ns > 1 && decode_smem_bytes(p->RG, p->KG, bf16, ns) > limit) --ns;
   p->n_stages = ns;
   p->smem = decode_smem_bytes(p->RG, p->KG, bf16, ns);
   if (p->smem > limit) {
@@ -580,6 +674,13 @@ bool plan_decode(const DecodeGeom& g, int idx_slots, bool bf16, int num_sms, Dec
     return false;
   }
   return true;
+}
+
+cudaError_t launch_sanitize_idx(const int32_t* idx, int32_t* out, int rows, int len, int64_t nb,
+                                unsigned* status, cudaStream_t s) {
+  if (rows == 0 || len == 0) return cudaSuccess;
+  sanitize_idx_kernel<<<(rows + 7) / 8, 256, 0, s>>>(idx, out, rows, len, nb, status);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode_attn(const DecodeAttnArgs& a, const DecodePlan& p, bool bf16, bool out_bf16,

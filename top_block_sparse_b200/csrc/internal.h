@@ -71,19 +71,20 @@ struct DecodeAttnArgs {
   int b;
   int64_t nb;
   int64_t s_end, w_begin;
-  int n_sink_tiles, tpb, n_wc_tiles, MT;
-  int64_t total_tiles;
-  int tpc;                // tiles per CTA
+  int tile;               // keys per tile (64 bf16, 32 fp32); a ring stage holds two
+  int n_sink_tiles, tpb, n_wc_tiles, n_tiles;
+  int MT;                 // work units (tile pairs) per (sequence, KV head)
+  int64_t total_tiles;    // work units over all pairs
+  int tpc;                // work units per CTA
   int n_slots;            // partial slots per pair
   int n_stages;
   float qscale;           // softmax scale * log2(e)
-  int check_idx;          // validate caller-provided ids
   int pdl;                // launched as a programmatic dependent of the scorer
 };
 
 struct DecodePlan {
   int R, R4, RG, KG;
-  int n_sink_tiles, tpb, n_wc_tiles, MT;
+  int tile, n_sink_tiles, tpb, n_wc_tiles, n_tiles, MT;
   int64_t total_tiles;
   int grid, tpc, n_slots, n_stages;
   size_t smem;
@@ -94,5 +95,9 @@ bool plan_decode(const DecodeGeom& g, int idx_slots, bool bf16, int num_sms, Dec
                  const char** why);
 cudaError_t launch_decode_attn(const DecodeAttnArgs& a, const DecodePlan& p, bool bf16,
                                bool out_bf16, cudaStream_t s);
+// Copies a caller's [rows, len] index table to `out`, keeping only entries
+// that are in [0, nb) and above every earlier in-range entry of the row.
+cudaError_t launch_sanitize_idx(const int32_t* idx, int32_t* out, int rows, int len, int64_t nb,
+                                unsigned* status, cudaStream_t s);
 
 }  // namespace sa

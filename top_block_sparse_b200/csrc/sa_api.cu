@@ -43,7 +43,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Shared validation of sa_params.  `prefill` selects the SA_SEL_TILE_MAX rules.
 sa_status check_params(const sa_params* p, bool prefill) {
   if (!p) return fail(SA_ERR_INVALID, "params is NULL");
-  if (p->reserved != 0) return fail(SA_ERR_INVALID, "params.reserved must be 0");
+  if ((p->flags & ~SA_FLAG_TRUSTED_IDX) != 0) return fail(SA_ERR_INVALID, "params.flags has unknown bits");
   if (p->batch < 1 || p->num_kv_heads < 1 || p->num_q_heads < 1)
     return fail(SA_ERR_INVALID, "batch, num_q_heads and num_kv_heads must be >= 1");
   if (p->num_q_heads % p->num_kv_heads != 0)
@@ -100,10 +100,11 @@ float scale_of(const sa_params* p) {
 
 // Workspace layout of the decode-type ops.
 struct DecodeWs {
-  size_t score_cnt, attn_cnt, scores, idx, part_O, part_ml, total;
+  size_t score_cnt, attn_cnt, scores, idx, clean_idx, part_O, part_ml, total;
 };
 
-DecodeWs decode_ws(const DecodeGeom& g, const DecodePlan& plan, int top_k, int op) {
+// idx_len: entries per row of a caller's index table (SA_OP_GIVEN_IDX).
+DecodeWs decode_ws(const DecodeGeom& g, const DecodePlan& plan, int top_k, int op, int idx_len = 0) {
   DecodeWs w = {};
   size_t off = kWsHeader;
   auto take = [&](size_t bytes) {
@@ -118,6 +119,7 @@ DecodeWs decode_ws(const DecodeGeom& g, const DecodePlan& plan, int top_k, int o
     w.scores = take(pairs * static_cast<size_t>(g.nb) * 4);
   }
   if (op == SA_OP_DECODE) w.idx = take(pairs * static_cast<size_t>(top_k) * 4);
+  if (op == SA_OP_GIVEN_IDX) w.clean_idx = take(pairs * static_cast<size_t>(idx_len) * 4);
   if (op == SA_OP_DECODE || op == SA_OP_GIVEN_IDX) {
     const size_t slots = pairs * static_cast<size_t>(plan.n_slots) * plan.R4;
     w.part_O = take(slots * kHeadDim * 4);
@@ -197,6 +199,8 @@ DecodeAttnArgs attn_args(const sa_params* p, const DecodeGeom& g, const DecodePl
   a.nb = g.nb;
   a.s_end = g.s_end;
   a.w_begin = g.w_begin;
+  a.tile = plan.tile;
+  a.n_tiles = plan.n_tiles;
   a.n_sink_tiles = plan.n_sink_tiles;
   a.tpb = plan.tpb;
   a.n_wc_tiles = plan.n_wc_tiles;
@@ -216,7 +220,7 @@ using namespace sa;
 
 extern "C" {
 
-int32_t sa_version(void) { return 100; }
+int32_t sa_version(void) { return 101; }
 
 const char* sa_last_error(void) { return g_err; }
 
@@ -243,7 +247,7 @@ size_t sa_workspace_size(const sa_params* p, int32_t op) {
   if (op == SA_OP_GIVEN_IDX) slots = p->top_k;   // sized for idx_len == top_k
   if (op == SA_OP_SCORE_TOPK) slots = 0;
   if (plan_for(p, slots, &g, &plan) != SA_OK) return 0;
-  return decode_ws(g, plan, p->top_k, op).total;
+  return decode_ws(g, plan, p->top_k, op, p->top_k).total;
 }
 
 sa_status sa_workspace_init(void* ws, size_t ws_bytes, void* stream) {
@@ -314,14 +318,21 @@ sa_status sa_sparse_attn_given_idx(const sa_params* p, const void* Q, const void
   DecodeGeom g;
   DecodePlan plan;
   if ((st = plan_for(p, idx_len, &g, &plan)) != SA_OK) return st;
-  const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_GIVEN_IDX);
+  const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_GIVEN_IDX, idx_len);
   if ((st = check_ws(ws, ws_bytes, L.total)) != SA_OK) return st;
   unsigned char* w = static_cast<unsigned char*>(ws);
-  DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, idx, idx_len, O, lse, w, L);
-  a.check_idx = 1;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int32_t* table = idx;
+  cudaError_t e = cudaSuccess;
+  if (!(p->flags & SA_FLAG_TRUSTED_IDX)) {
+    int32_t* clean = reinterpret_cast<int32_t*>(w + L.clean_idx);
+    e = launch_sanitize_idx(idx, clean, g.pairs, idx_len, g.nb, reinterpret_cast<unsigned*>(w), s);
+    if (e != cudaSuccess) return cuda_fail(e, "index-table check launch");
+    table = clean;
+  }
+  DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, table, idx_len, O, lse, w, L);
   a.pdl = 0;
-  cudaError_t e = launch_decode_attn(a, plan, p->dtype == SA_BF16, p->out_dtype == SA_BF16,
-                                     static_cast<cudaStream_t>(stream));
+  e = launch_decode_attn(a, plan, p->dtype == SA_BF16, p->out_dtype == SA_BF16, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
   return SA_OK;
 }
@@ -350,7 +361,6 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q, const void* K
   cudaError_t e = launch_score_topk_query0(sa_, p->dtype == SA_BF16, s);
   if (e != cudaSuccess) return cuda_fail(e, "score/top-k kernel launch");
   DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, idx, p->top_k, O, lse, w, L);
-  a.check_idx = 0;
   a.pdl = 1;
   e = launch_decode_attn(a, plan, p->dtype == SA_BF16, p->out_dtype == SA_BF16, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
@@ -442,7 +452,7 @@ extern "C" sa_status sa_sparse_attn_given_idx_noalloc(const sa_params* p, const 
   DecodeGeom g;
   DecodePlan plan;
   if ((st = plan_for(p, idx_len, &g, &plan)) != SA_OK) return st;
-  const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_GIVEN_IDX);
+  const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_GIVEN_IDX, idx_len);
   if (L.total > kStaticScratchBytes)
     return fail(SA_ERR_WORKSPACE,
                 "this problem needs %zu bytes of scratch; the allocation-free entry point has a static "
@@ -453,10 +463,16 @@ extern "C" sa_status sa_sparse_attn_given_idx_noalloc(const sa_params* p, const 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // The array keeps the previous call's contents: the status word and the
   // tickets must start at zero.
-  cudaError_t e = cudaMemsetAsync(w, 0, L.part_O, s);
+  cudaError_t e = cudaMemsetAsync(w, 0, L.clean_idx, s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (static scratch)");
-  DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, idx, idx_len, O, lse, w, L);
-  a.check_idx = 1;
+  const int32_t* table = idx;
+  if (!(p->flags & SA_FLAG_TRUSTED_IDX)) {
+    int32_t* clean = reinterpret_cast<int32_t*>(w + L.clean_idx);
+    e = launch_sanitize_idx(idx, clean, g.pairs, idx_len, g.nb, reinterpret_cast<unsigned*>(w), s);
+    if (e != cudaSuccess) return cuda_fail(e, "index-table check launch");
+    table = clean;
+  }
+  DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, table, idx_len, O, lse, w, L);
   a.pdl = 0;
   e = launch_decode_attn(a, plan, p->dtype == SA_BF16, p->out_dtype == SA_BF16, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");

@@ -25,104 +25,104 @@ namespace {
 constexpr int kScoreThreads = 256;
 constexpr int kScoreWarps = kScoreThreads / 32;
 
-// Block-wide exclusive scan of one value per thread (kScoreThreads threads).
-__device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* warp_tot,
-                                                         unsigned* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ __forceinline__ unsigned warp_sum(unsigned v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ unsigned warp_exclusive_scan(unsigned v) {
+  const int lane = threadIdx.x & 31;
   unsigned x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    unsigned y = __shfl_up_sync(0xffffffffu, x, o);
+    const unsigned y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) warp_tot[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    unsigned t = lane < kScoreWarps ? warp_tot[lane] : 0u;
-    unsigned s = t;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      unsigned y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    if (lane < kScoreWarps) warp_tot[lane] = s - t;   // exclusive warp offsets
-    if (lane == kScoreWarps - 1) *total = s;
-  }
-  __syncthreads();
-  const unsigned r = warp_tot[warp] + x - v;
-  __syncthreads();
-  return r;
+  return x - v;
 }
 
-// Exact top-k of `nb` keys in shared memory (key 0 = not a candidate;
-// candidates have keys >= 1).  Writes ascending block ids to out[0..k).
-__device__ void radix_select_write(const uint32_t* keys, int nb, int k, int32_t* out,
-                                   unsigned* hist, unsigned* scratch) {
-  const int tid = threadIdx.x;
-  unsigned* warp_tot = scratch;          // [kScoreWarps]
-  unsigned* total = scratch + 16;
-  unsigned* bcast = scratch + 20;        // digit, count above
-
-  // number of candidates
+// Exact top-k of `nb` keys in shared memory by ONE warp (key 0 = not a
+// candidate, candidates have keys >= 1): a 4-pass, 8-bit-digit radix select
+// finds the k-th largest key tau and how many keys equal to tau are taken
+// (the lowest block ids first); a prefix scan in block-id order then writes
+// the selected ids ascending to out[0..k), -1 padded.
+__device__ void warp_radix_select(const uint32_t* keys, int nb, int k, int32_t* out, unsigned* hist) {
+  const int lane = threadIdx.x & 31;
   unsigned nc = 0;
-  for (int j = tid; j < nb; j += kScoreThreads) nc += keys[j] != 0u;
-  block_exclusive_scan(nc, warp_tot, total);
-  const unsigned n_cand = *total;
-  const unsigned keff = n_cand < static_cast<unsigned>(k) ? n_cand : static_cast<unsigned>(k);
+#pragma unroll 8
+  for (int j = lane; j < nb; j += 32) nc += keys[j] != 0u;
+  nc = warp_sum(nc);
+  const unsigned keff = nc < static_cast<unsigned>(k) ? nc : static_cast<unsigned>(k);
 
   uint32_t tau = 0u;          // keff-th largest key
-  unsigned need = keff;       // how many keys equal to tau are taken
+  unsigned need = keff;       // keys equal to tau that are taken
   if (keff > 0u) {
     uint32_t prefix = 0u;
     for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += kScoreThreads) hist[i] = 0u;
-      __syncthreads();
-      for (int j = tid; j < nb; j += kScoreThreads) {
-        const uint32_t key = keys[j];
-        if (key == 0u) continue;
-        const bool match = (shift == 24) || ((key ^ prefix) >> (shift + 8)) == 0u;
-        if (match) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hist[lane + 32 * i] = 0u;
+      __syncwarp();
+      // scores cluster in a few digit values (sign and exponent bits first), so
+      // lanes with equal digits are merged and one of them adds their count
+#pragma unroll 8
+      for (int j0 = 0; j0 < nb; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t key = j < nb ? keys[j] : 0u;
+        const bool take = key != 0u && (shift == 24 || ((key ^ prefix) >> (shift + 8)) == 0u);
+        const unsigned digit = take ? ((key >> shift) & 255u) : 256u;
+        const unsigned peers = __match_any_sync(0xffffffffu, digit);
+        if (take && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], static_cast<unsigned>(__popc(peers)));
       }
-      __syncthreads();
-      if (tid < 32) {
-        // lane owns bins [8*lane, 8*lane + 8); find the digit holding the need-th largest
-        unsigned own = 0;
+      __syncwarp();
+      // lane owns bins [8*lane, 8*lane + 8): find the digit holding the need-th largest
+      unsigned h8[8], own = 0;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) own += hist[8 * tid + q];
-        unsigned suf = own;
+      for (int q = 0; q < 8; ++q) {
+        h8[q] = hist[8 * lane + q];
+        own += h8[q];
+      }
+      unsigned suf = own;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          unsigned y = __shfl_down_sync(0xffffffffu, suf, o);
-          if (tid + o < 32) suf += y;
-        }
-        unsigned above = suf - own;    // keys with a digit in a higher lane's bins
-        if (above < need && need <= above + own) {
-          unsigned c = above;
-          for (int q = 7; q >= 0; --q) {
-            const unsigned h = hist[8 * tid + q];
-            if (c + h >= need) {
-              bcast[0] = static_cast<unsigned>(8 * tid + q);
-              bcast[1] = c;
-              break;
-            }
-            c += h;
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_down_sync(0xffffffffu, suf, o);
+        if (lane + o < 32) suf += y;
+      }
+      const unsigned above = suf - own;          // keys in higher lanes' bins
+      unsigned digit = 0, cnt_above = 0;
+      const bool mine = above < need && need <= above + own;
+      if (mine) {
+        unsigned c = above;
+        bool found = false;
+#pragma unroll
+        for (int q = 7; q >= 0; --q) {
+          if (!found && c + h8[q] >= need) {
+            digit = static_cast<unsigned>(8 * lane + q);
+            cnt_above = c;
+            found = true;
           }
+          c += h8[q];
         }
       }
-      __syncthreads();
-      prefix |= bcast[0] << shift;
-      need -= bcast[1];
-      __syncthreads();
+      const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      cnt_above = __shfl_sync(0xffffffffu, cnt_above, src);
+      prefix |= digit << shift;
+      need -= cnt_above;
+      __syncwarp();
     }
     tau = prefix;
   }
 
-  // Each thread owns a contiguous run of block ids so that scans follow id order.
-  const int per = (nb + kScoreThreads - 1) / kScoreThreads;
-  const int j0 = tid * per, j1 = min(nb, j0 + per);
+  // Each lane owns a contiguous run of block ids so that scans follow id order.
+  const int per = (nb + 31) / 32;
+  const int j0 = lane * per, j1 = min(nb, j0 + per);
   unsigned eq = 0;
-  for (int j = j0; j < j1; ++j) eq += (keff > 0u && keys[j] == tau) ? 1u : 0u;
-  unsigned eq_before = block_exclusive_scan(eq, warp_tot, total);
+  if (keff > 0u) {
+#pragma unroll 8
+    for (int j = j0; j < j1; ++j) eq += keys[j] == tau;
+  }
+  const unsigned eq_before = warp_exclusive_scan(eq);
   unsigned sel = 0;
   {
     unsigned e = eq_before;
@@ -136,7 +136,7 @@ __device__ void radix_select_write(const uint32_t* keys, int nb, int k, int32_t*
       sel += s;
     }
   }
-  unsigned pos = block_exclusive_scan(sel, warp_tot, total);
+  unsigned pos = warp_exclusive_scan(sel);
   {
     unsigned e = eq_before;
     for (int j = j0; j < j1; ++j) {
@@ -149,7 +149,7 @@ __device__ void radix_select_write(const uint32_t* keys, int nb, int k, int32_t*
       if (s) out[pos++] = j;
     }
   }
-  for (int s = static_cast<int>(keff) + tid; s < k; s += kScoreThreads) out[s] = -1;
+  for (int s = static_cast<int>(keff) + lane; s < k; s += 32) out[s] = -1;
 }
 
 template <bool BF16>
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_query0_kernel(ScoreA
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw);                        // [nb] (last CTA)
   __shared__ __align__(16) float qs[kHeadDim];
   __shared__ unsigned hist[256];
-  __shared__ unsigned scratch[32];
+  __shared__ unsigned scratch[4];
   __shared__ int is_last;
 
   const int pair = blockIdx.y;
@@ -166,6 +166,8 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_query0_kernel(ScoreA
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bi = pair / a.Hkv, h = pair % a.Hkv;
 
+  static_assert(kScoreBlocksPerChunk % kScoreWarps == 0 && kScoreBlocksPerChunk / kScoreWarps <= 32,
+                "rows per warp");
   // index query of the first new token: sum over the GQA group
   if (tid < kHeadDim) {
     float s = 0.f;
@@ -199,46 +201,62 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_query0_kernel(ScoreA
   const int64_t j_end = min(a.nb, j_begin + a.blocks_per_chunk);
   const float* kc = a.Kc + static_cast<int64_t>(pair) * a.nb * kHeadDim;
   float* sc = a.scores + static_cast<int64_t>(pair) * a.nb;
-  for (int64_t j0 = j_begin + warp * 4; j0 < j_end; j0 += kScoreWarps * 4) {
-    float4 r[4];
+  // every warp streams kRowsPerWarp rows; all their loads are issued first
+  constexpr int kRowsPerWarp = kScoreBlocksPerChunk / kScoreWarps;
+  const int64_t jw = j_begin + static_cast<int64_t>(warp) * kRowsPerWarp;
+  float4 r[kRowsPerWarp];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      r[u] = (j0 + u < j_end) ? __ldcs(reinterpret_cast<const float4*>(kc + (j0 + u) * kHeadDim) + lane)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-    float d[4];
+  for (int u = 0; u < kRowsPerWarp; ++u)
+    r[u] = (jw + u < j_end) ? __ldcs(reinterpret_cast<const float4*>(kc + (jw + u) * kHeadDim) + lane)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+  float d[kRowsPerWarp];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) d[u] = r[u].x * q4.x + r[u].y * q4.y + r[u].z * q4.z + r[u].w * q4.w;
+  for (int u = 0; u < kRowsPerWarp; ++u) d[u] = r[u].x * q4.x + r[u].y * q4.y + r[u].z * q4.z + r[u].w * q4.w;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
+  for (int o = 16; o > 0; o >>= 1) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) d[u] += __shfl_xor_sync(0xffffffffu, d[u], o);
-    }
-    if (lane < 4 && j0 + lane < j_end)
-      sc[j0 + lane] = lane == 0 ? d[0] : lane == 1 ? d[1] : lane == 2 ? d[2] : d[3];
+    for (int u = 0; u < kRowsPerWarp; ++u) d[u] += __shfl_xor_sync(0xffffffffu, d[u], o);
   }
+  float mine = d[0];
+#pragma unroll
+  for (int u = 1; u < kRowsPerWarp; ++u) mine = (lane == u) ? d[u] : mine;
+  if (lane < kRowsPerWarp && jw + lane < j_end) sc[jw + lane] = mine;
 
-  // ticket: the last CTA of this pair selects
-  __threadfence();
+  // ticket: the last CTA of this pair selects (one warp; the others leave).
+  // The barrier orders the CTA's score stores before thread 0's release fence.
   __syncthreads();
   if (tid == 0) {
+    __threadfence();
     const unsigned t = atomicAdd(&a.counters[pair], 1u);
     is_last = (t == static_cast<unsigned>(a.chunks - 1));
   }
   __syncthreads();
-  if (!is_last) return;
+  if (!is_last || warp != 0) return;
   __threadfence();
-  if (tid == 0) a.counters[pair] = 0u;
+  if (lane == 0) a.counters[pair] = 0u;
 
   const int nb = static_cast<int>(a.nb);
-  for (int j = tid; j < nb; j += kScoreThreads) {
-    const int64_t lo = static_cast<int64_t>(j) * a.b, hi = lo + a.b;
-    const bool cand = (lo < a.w_begin) && (hi > a.s_end);
-    const float s = __ldcg(sc + j);
-    uint32_t key = float_key(s);
-    keys[j] = cand ? (key == 0u ? 1u : key) : 0u;
+  // the pair's scores come from L2; keep 8 loads per lane in flight
+  for (int j0 = 0; j0 < nb; j0 += 8 * 32) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * 32 + lane;
+      v[u] = j < nb ? __ldcg(sc + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * 32 + lane;
+      if (j < nb) {
+        const int64_t lo = static_cast<int64_t>(j) * a.b, hi = lo + a.b;
+        const bool cand = (lo < a.w_begin) && (hi > a.s_end);
+        const uint32_t key = float_key(v[u]);
+        keys[j] = cand ? (key == 0u ? 1u : key) : 0u;
+      }
+    }
   }
-  __syncthreads();
-  radix_select_write(keys, nb, a.top_k, a.idx + static_cast<int64_t>(pair) * a.top_k, hist, scratch);
+  __syncwarp();
+  warp_radix_select(keys, nb, a.top_k, a.idx + static_cast<int64_t>(pair) * a.top_k, hist);
 }
 
 }  // namespace

@@ -26,6 +26,7 @@ SA_F32, SA_BF16 = 0, 1
 SA_POOL_MEAN, SA_POOL_LSA = 0, 1
 SA_SEL_QUERY0, SA_SEL_TILE_MAX = 0, 1
 SA_OP_SCORE_TOPK, SA_OP_GIVEN_IDX, SA_OP_DECODE, SA_OP_PREFILL = 0, 1, 2, 3
+SA_FLAG_TRUSTED_IDX = 1
 
 EXPORTED = ["sa_version", "sa_workspace_size", "sa_workspace_init", "sa_pool_keys", "sa_score_topk",
             "sa_sparse_attn_given_idx", "sa_sparse_attn_decode", "sa_sparse_attn_prefill",
@@ -42,7 +43,7 @@ class SaParams(ctypes.Structure):
         ("top_k", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("out_dtype", ctypes.c_int32), ("select", ctypes.c_int32),
         ("sink_keys", ctypes.c_int64), ("window_keys", ctypes.c_int64),
-        ("softmax_scale", ctypes.c_float), ("reserved", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float), ("flags", ctypes.c_int32),
     ]
 
 
@@ -99,7 +100,7 @@ def make_params(*, batch, num_q_heads, num_kv_heads, ctx_len, n_q, block_size, t
                     top_k=top_k, dtype=dt, out_dtype=odt,
                     select=SA_SEL_TILE_MAX if prefill else SA_SEL_QUERY0,
                     sink_keys=sink_keys, window_keys=window_keys,
-                    softmax_scale=softmax_scale, reserved=0)
+                    softmax_scale=softmax_scale, flags=0)
 
 
 def params_for(w, kv_capacity=None, out_dtype=None) -> SaParams:
