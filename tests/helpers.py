@@ -64,10 +64,25 @@ def compare_sets(gpu_idx_row: np.ndarray, sel: orc.Selection) -> str:
     return "near_tie" if sel.near_tie else "mismatch"
 
 
+def bf16_half_step(x: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 numbers around |x| (8 significant bits)."""
+    ax = np.abs(x)
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, np.exp2(e - 8), 0.0)
+
+
 def errors(got: torch.Tensor, ref: np.ndarray):
+    """Max abs and relative L2 error against the float64 reference.  For a
+    bf16 output the max abs error is counted beyond half a bf16 step of the
+    exact value (the output format cannot come closer), so the bar measures
+    the kernel's arithmetic, not the format."""
     g = got.double().cpu().numpy().reshape(ref.shape)
     d = g - ref
-    max_abs = float(np.abs(d).max()) if d.size else 0.0
+    if got.dtype == torch.bfloat16:
+        excess = np.maximum(np.abs(d) - bf16_half_step(ref), 0.0)
+        max_abs = float(excess.max()) if d.size else 0.0
+    else:
+        max_abs = float(np.abs(d).max()) if d.size else 0.0
     den = float(np.sqrt((ref * ref).sum()))
     rel = float(np.sqrt((d * d).sum()) / den) if den > 0 else float(np.sqrt((d * d).sum()))
     return max_abs, rel

@@ -1,0 +1,172 @@
+"""GPU parity of the causal prefill path (tensor-core scoring and attention)
+against the float64 oracle, tile by tile.
+
+Bars: tile scores within 2e-5 (fp32 accumulation of split-bf16 products);
+selected sets identical except oracle near-ties; attention outputs (bf16
+inputs, bf16 probabilities into the P.V product, fp32 accumulation) within
+max abs 5e-3 and relative L2 1e-2.
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_close, compare_sets, oracle_params
+from oracle import sparse_attn_oracle as orc
+from top_block_sparse_b200.inputs import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+sa = pytest.importorskip("top_block_sparse_b200.sa")
+
+
+def pf(T, Hkv=2, k=8, **kw):
+    return WORKLOADS["prefill_64k"].scaled(n_q=T, num_kv_heads=Hkv, num_q_heads=4 * Hkv, top_k=k,
+                                           n_needles=min(k, 4), **kw)
+
+
+def head_arrays(inp, h, w):
+    q = inp["Q"][0, :, 4 * h:4 * h + 4].double().cpu().numpy()     # [T, G, d]
+    K = inp["K"][0, h, :w.n_q].double().cpu().numpy()
+    V = inp["V"][0, h, :w.n_q].double().cpu().numpy()
+    return q, K, V
+
+
+def run_prefill(w, inp, out_dtype="f32"):
+    p = sa.params_for(w, out_dtype=out_dtype)
+    T = w.n_q
+    nb, nt = T // 64, (T + 63) // 64
+    Kc = torch.empty((w.batch, w.num_kv_heads, max(nb, 1), 128), device="cuda")
+    O = torch.empty((w.batch, T, w.num_q_heads, 128), device="cuda",
+                    dtype=torch.float32 if out_dtype == "f32" else torch.bfloat16)
+    lse = torch.empty((w.batch, T, w.num_q_heads), device="cuda")
+    idx = torch.empty((w.batch, w.num_kv_heads, nt, w.top_k), device="cuda", dtype=torch.int32)
+    ws = sa.alloc_workspace(p, sa.SA_OP_PREFILL)
+    sa.sparse_attn_prefill(p, inp["Q"], inp["K"], inp["V"], Kc, O, lse, idx, ws)
+    assert sa.read_status(ws) == sa.SA_OK
+    return p, Kc, O, lse, idx
+
+
+def check_tiles(w, inp, O, lse, idx, tiles, Kc_gpu=None):
+    op = oracle_params(w)
+    ties = 0
+    for h in range(w.num_kv_heads):
+        q, K, V = head_arrays(inp, h, w)
+        Kc_all = orc.compress(K, op)
+        if Kc_gpu is not None:
+            np.testing.assert_allclose(Kc_gpu[0, h, :len(Kc_all)].double().cpu().numpy(), Kc_all, atol=2e-6, rtol=1e-5)
+        for i in tiles:
+            rows = slice(i * 64, min((i + 1) * 64, w.n_q))
+            r = orc.prefill_tile(q[rows], K, V, i, op, Kc_all)
+            v = compare_sets(idx[0, h, i].cpu().numpy(), r["sel"])
+            assert v != "mismatch", (h, i, idx[0, h, i].tolist(), r["sel"].selected)
+            if v == "near_tie":
+                ties += 1
+                continue
+            assert_close(O[0, rows, 4 * h:4 * h + 4], r["O"], "bf16", f"head {h} tile {i}")
+            lerr = np.abs(lse[0, rows, 4 * h:4 * h + 4].double().cpu().numpy() - r["lse"]).max()
+            assert lerr < 2e-3, (h, i, lerr)
+    return ties
+
+
+def test_prefill_scores_and_selection():
+    w = pf(64 * 40 + 17, k=8)
+    inp = make_inputs(w, seed=5, device="cuda")
+    p = sa.params_for(w)
+    T = w.n_q
+    nb, nt = T // 64, (T + 63) // 64
+    Kc = torch.empty((1, w.num_kv_heads, nb, 128), device="cuda")
+    sa.pool_keys(p, inp["K"], Kc)
+    idx = torch.empty((1, w.num_kv_heads, nt, w.top_k), device="cuda", dtype=torch.int32)
+    scores = torch.full((1, w.num_kv_heads, nt, nb), float("nan"), device="cuda")
+    ws = sa.alloc_workspace(p, sa.SA_OP_SCORE_TOPK)
+    sa.score_topk(p, inp["Q"], Kc, idx, scores, ws)
+    torch.cuda.synchronize()
+    op = oracle_params(w)
+    ties = 0
+    for h in range(w.num_kv_heads):
+        q, K, V = head_arrays(inp, h, w)
+        Kc_all = orc.compress(K, op)
+        sel = orc.prefill_head_selection(q, Kc_all, op, range(nt))
+        for i in range(nt):
+            cand = sel[i].n_candidates and orc.candidate_blocks(64 * i, op)
+            if cand:
+                ref = orc.prefill_tile_scores(q[i * 64:(i + 1) * 64], Kc_all[:i], op)
+                got = scores[0, h, i, cand].double().cpu().numpy()
+                np.testing.assert_allclose(got, ref[cand], atol=2e-5, rtol=2e-5)
+            v = compare_sets(idx[0, h, i].cpu().numpy(), sel[i])
+            assert v != "mismatch", (h, i)
+            ties += v == "near_tie"
+    print(f"\nprefill selection: near-ties {ties}")
+
+
+def test_prefill_given_idx_with_oracle_indices():
+    w = pf(64 * 24, k=6)
+    inp = make_inputs(w, seed=6, device="cuda")
+    op = oracle_params(w)
+    nt = w.n_q // 64
+    idx = torch.full((1, w.num_kv_heads, nt, w.top_k), -1, dtype=torch.int32)
+    refs = {}
+    for h in range(w.num_kv_heads):
+        q, K, V = head_arrays(inp, h, w)
+        Kc_all = orc.compress(K, op)
+        for i in range(nt):
+            r = orc.prefill_tile(q[i * 64:(i + 1) * 64], K, V, i, op, Kc_all)
+            s = r["sel"].selected
+            idx[0, h, i, :len(s)] = torch.tensor(s, dtype=torch.int32)
+            refs[(h, i)] = r
+    p = sa.params_for(w, out_dtype="f32")
+    O = torch.empty((1, w.n_q, w.num_q_heads, 128), device="cuda")
+    lse = torch.empty((1, w.n_q, w.num_q_heads), device="cuda")
+    ws = sa.alloc_workspace(p, sa.SA_OP_GIVEN_IDX)
+    sa.sparse_attn_given_idx(p, inp["Q"], inp["K"], inp["V"], idx.cuda(), O, lse, ws)
+    assert sa.read_status(ws) == sa.SA_OK
+    worst = 0.0
+    for (h, i), r in refs.items():
+        e = assert_close(O[0, i * 64:(i + 1) * 64, 4 * h:4 * h + 4], r["O"], "bf16", f"head {h} tile {i}")
+        worst = max(worst, e[0])
+    print(f"\nprefill given-idx worst max abs {worst:.2e}")
+
+
+@pytest.mark.parametrize("T,k", [(64 * 32, 8), (64 * 20 + 33, 4), (100, 8), (64 * 12, 100)])
+def test_prefill_end_to_end(T, k):
+    w = pf(T, k=k)
+    inp = make_inputs(w, seed=7, device="cuda")
+    _, Kc, O, lse, idx = run_prefill(w, inp)
+    ties = check_tiles(w, inp, O, lse, idx, range((T + 63) // 64), Kc)
+    print(f"\nprefill T={T}: near-ties {ties}")
+
+
+def test_prefill_bf16_output_and_reuse():
+    w = pf(64 * 16, k=4)
+    inp = make_inputs(w, seed=8, device="cuda")
+    p, Kc, O1, lse1, idx1 = run_prefill(w, inp, out_dtype="bf16")
+    check_tiles(w, inp, O1, lse1, idx1, range(16))
+    _, _, O2, _, idx2 = run_prefill(w, inp, out_dtype="bf16")
+    assert torch.equal(idx1, idx2) and torch.equal(O1, O2)
+
+
+def test_prefill_full_size_sampled():
+    """The benchmark configuration (T = 65536, 8 KV heads); the oracle checks
+    sampled tiles of every head."""
+    w = WORKLOADS["prefill_64k"]
+    inp = make_inputs(w, seed=9, device="cuda")
+    _, Kc, O, lse, idx = run_prefill(w, inp, out_dtype="bf16")
+    torch.cuda.synchronize()
+    op = oracle_params(w)
+    tiles = [0, 5, 6, 70, 511, 1022, 1023]
+    ties = 0
+    for h in [0, 3, 7]:
+        q, K, V = head_arrays(inp, h, w)
+        Kc_all = orc.compress(K, op)
+        for i in tiles:
+            rows = slice(i * 64, (i + 1) * 64)
+            r = orc.prefill_tile(q[rows], K, V, i, op, Kc_all)
+            v = compare_sets(idx[0, h, i].cpu().numpy(), r["sel"])
+            assert v != "mismatch", (h, i)
+            if v == "near_tie":
+                ties += 1
+                continue
+            assert_close(O[0, rows, 4 * h:4 * h + 4], r["O"], "bf16", f"head {h} tile {i}")
+        if h == 0:
+            assert set(inp["needles"][0, h].tolist()) <= set(idx[0, h, 1023].tolist())
+    print(f"\nprefill 64k sampled: near-ties {ties}")

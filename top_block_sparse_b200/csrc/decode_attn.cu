@@ -570,6 +570,48 @@ __global__ void __launch_bounds__(256) sanitize_idx_kernel(const int32_t* idx, i
   if (__any_sync(0xffffffffu, bad) && lane == 0) report(status, kStatusIndex);
 }
 
+// Caller prefill tables: row (pair, tile t) may list blocks j < t (complete
+// blocks before the tile); an entry is kept if it is above every earlier
+// in-range entry of the row and is not one of the tile's sink / window blocks
+// (their keys are attended anyway).  Entries >= t or < -1, and repeated or
+// descending ones, set kStatusIndex.
+__global__ void __launch_bounds__(256) sanitize_prefill_idx_kernel(const int32_t* idx, int32_t* out, int P,
+                                                                   int n_tiles, int len, int64_t S, int64_t W,
+                                                                   unsigned* status) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= P * n_tiles) return;
+  const int t = row % n_tiles;
+  const int64_t C = static_cast<int64_t>(t) * 64;
+  const int64_t s_end = S < C ? S : C;
+  const int64_t w_begin = (C - W) > s_end ? (C - W) : s_end;
+  const int lo = static_cast<int>(s_end / 64), hi = static_cast<int>(w_begin / 64);
+  const int32_t* in = idx + static_cast<int64_t>(row) * len;
+  int32_t* o = out + static_cast<int64_t>(row) * len;
+  int carry = -1;
+  bool bad = false;
+  for (int base = 0; base < len; base += 32) {
+    const int s = base + lane;
+    const int32_t j = s < len ? __ldg(in + s) : -1;
+    const bool in_range = j >= 0 && j < t;
+    int incl = in_range ? j : -1;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl = max(incl, y);
+    }
+    int excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = -1;
+    excl = max(excl, carry);
+    const bool ok = in_range && j > excl;
+    if (s < len) {
+      o[s] = (ok && j >= lo && j < hi) ? j : -1;
+      if (!ok && j != -1) bad = true;
+    }
+    carry = max(carry, __shfl_sync(0xffffffffu, incl, 31));
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) report(status, kStatusIndex);
+}
+
 template <bool BF16, bool OUT_BF16, int RG, int KG>
 cudaError_t launch_one(const DecodeAttnArgs& a, const DecodePlan& p, cudaStream_t s) {
   auto kern = decode_attn_kernel<BF16, OUT_BF16, RG, KG>;
@@ -680,6 +722,14 @@ cudaError_t launch_sanitize_idx(const int32_t* idx, int32_t* out, int rows, int 
                                 unsigned* status, cudaStream_t s) {
   if (rows == 0 || len == 0) return cudaSuccess;
   sanitize_idx_kernel<<<(rows + 7) / 8, 256, 0, s>>>(idx, out, rows, len, nb, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sanitize_prefill_idx(const int32_t* idx, int32_t* out, int P, int n_tiles, int len,
+                                        int64_t S, int64_t W, unsigned* status, cudaStream_t s) {
+  const int rows = P * n_tiles;
+  if (rows == 0 || len == 0) return cudaSuccess;
+  sanitize_prefill_idx_kernel<<<(rows + 7) / 8, 256, 0, s>>>(idx, out, P, n_tiles, len, S, W, status);
   return cudaGetLastError();
 }
 

@@ -100,4 +100,31 @@ cudaError_t launch_decode_attn(const DecodeAttnArgs& a, const DecodePlan& p, boo
 cudaError_t launch_sanitize_idx(const int32_t* idx, int32_t* out, int rows, int len, int64_t nb,
                                 unsigned* status, cudaStream_t s);
 
+// ---- prefill (tensor cores) -------------------------------------------------
+struct PrefillArgs {
+  const void* Q;          // [B, T, Hq, 128] bf16
+  const void* K;          // [B, Hkv, cap, 128] bf16
+  const void* V;
+  const float* Kc;        // [B, Hkv, nb, 128] fp32
+  uint16_t* kc2;          // workspace: [B*Hkv, nb, 256] bf16 (hi | lo)
+  float* scores;          // workspace or caller: [B*Hkv, n_tiles, nb]
+  int32_t* idx;           // [B*Hkv, n_tiles, top_k]
+  void* O;                // [B, T, Hq, 128]
+  float* lse;             // [B, T, Hq] or null
+  unsigned* status;
+  int B, Hq, Hkv, T, nb, n_tiles, top_k, out_bf16, num_sms;
+  int64_t cap, S, W;
+  float scale;
+};
+// Kc split, tile scoring (tcgen05) and per-tile top-k into pa.idx.
+cudaError_t launch_prefill_score(const PrefillArgs& pa, cudaStream_t s);
+// Causal sparse attention of every tile over pa.idx (tcgen05).
+cudaError_t launch_prefill_attn(const PrefillArgs& pa, cudaStream_t s);
+size_t prefill_score_smem();
+size_t prefill_attn_smem();
+// Caller prefill tables [P, n_tiles, len]: keeps ids j < tile that are above
+// every earlier such id of the row and outside sink / window of the tile.
+cudaError_t launch_sanitize_prefill_idx(const int32_t* idx, int32_t* out, int P, int n_tiles, int len,
+                                        int64_t S, int64_t W, unsigned* status, cudaStream_t s);
+
 }  // namespace sa

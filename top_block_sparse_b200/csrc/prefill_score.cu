@@ -1,0 +1,453 @@
+// Prefill steps 2-3 on tensor cores: tile scoring and per-tile top-k.
+//
+// Scoring (LSA review §2.4 and SparDA "方法": one index query per GQA group =
+// the sum of the group's query vectors; the pages do not say how the rows of
+// a 64-query tile are combined -- the reading taken is the max over rows):
+//   s[t][j] = max_{r in tile t} ( sum_g q_{r,g} ) . Kc_j * scale
+// for every candidate block j of tile t (complete, before the tile, not
+// wholly inside sink / window).
+//
+// This is a dense contraction, so it runs on tcgen05 tensor cores.  The GEMM
+// is transposed -- M = 128 compressed keys (TMEM lanes), N = 128 query rows
+// (two tiles, TMEM columns), K = 128 -- so that a TMEM lane holds one block's
+// scores against all query rows and the tile max is a per-thread reduction.
+// Both operands are split into bf16 hi + lo parts (x = hi + lo exactly up to
+// 2^-16 relative) and three products hi*hi + lo*hi + hi*lo are accumulated in
+// fp32: single-pass bf16 scores would be ~1e-3 off and flip top-k choices.
+//
+// CTA roles (persistent, one CTA per SM, work items = (sequence x KV head,
+// pair of query tiles) in decreasing-cost order):
+//   warp 0      TMA producer: Kc hi / lo chunks of 128 blocks (128-byte swizzle)
+//   warp 1      TMEM owner and MMA issuer (one thread)
+//   warps 2-5   build the B operand: GQA sum x scale of 128 query rows, split
+//               into hi / lo, written to swizzled shared memory
+//   warps 6-9   epilogue: TMEM -> registers, max over each 64-row tile,
+//               candidate mask, fp32 scores to global
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "select.cuh"
+#include "tc.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kTile = 64;                      // query rows per tile = block size
+constexpr int kNSA = 3;                        // A stages (32 KB: hi or lo of a 128-block chunk)
+constexpr int kAStage = 32768;
+constexpr int kBBuf = 65536;                   // B operand: hi atoms 0,1 then lo atoms 0,1
+constexpr int kScoreThreadsTC = 320;
+constexpr uint32_t kIdesc = tc::idesc_bf16(128, 128, false, false);
+
+struct PSArgs {
+  const uint16_t* Q;        // [B, T, Hq, 128] bf16
+  float* scores;            // [P, n_tiles, nb]
+  unsigned* status;
+  int B, Hq, Hkv, G, T, nb, n_tiles, n_tpairs, P;
+  int64_t S, W;
+  float scale;
+};
+
+// Candidate test of block j for query tile t (context C = 64 t).
+__device__ __forceinline__ bool is_candidate(const PSArgs& a, int t, int j) {
+  const int64_t C = static_cast<int64_t>(t) * kTile;
+  const int64_t s_end = a.S < C ? a.S : C;
+  const int64_t w_begin = (C - a.W) > s_end ? (C - a.W) : s_end;
+  const int64_t lo = static_cast<int64_t>(j) * kTile;
+  return j < a.nb && lo < w_begin && lo + kTile > s_end;
+}
+
+// Blocks [0, j_lim) contain every candidate of tiles 2n and 2n+1.
+__device__ __forceinline__ int chunk_count(const PSArgs& a, int n) {
+  int t = min(2 * n + 1, a.n_tiles - 1);
+  const int64_t C = static_cast<int64_t>(t) * kTile;
+  const int64_t s_end = a.S < C ? a.S : C;
+  const int64_t w_begin = (C - a.W) > s_end ? (C - a.W) : s_end;
+  int64_t j_lim = (w_begin + kTile - 1) / kTile;
+  if (j_lim > a.nb) j_lim = a.nb;
+  if (j_lim * kTile <= s_end) return 0;      // no block reaches past the sink
+  return static_cast<int>((j_lim + 127) / 128);
+}
+
+// Work item k -> (tile pair n, pair p), most expensive first.
+__device__ __forceinline__ void item_of(const PSArgs& a, int k, int* n, int* p) {
+  *n = a.n_tpairs - 1 - k / a.P;
+  *p = k % a.P;
+}
+
+__global__ void __launch_bounds__(kScoreThreadsTC, 1)
+    prefill_score_kernel(const __grid_constant__ CUtensorMap kc_map, PSArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte alignment for the swizzled operand atoms
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* A = smem;                                     // kNSA x 32 KB
+  unsigned char* Bop = A + kNSA * kAStage;                     // 2 x 64 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Bop + 2 * kBBuf);
+  uint64_t* a_full = bars;
+  uint64_t* a_empty = a_full + kNSA;
+  uint64_t* b_full = a_empty + kNSA;
+  uint64_t* b_empty = b_full + 2;
+  uint64_t* d_full = b_empty + 2;
+  uint64_t* d_empty = d_full + 2;
+  uint64_t* mma_done = d_empty + 2;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = a.n_tpairs * a.P;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNSA; ++s) {
+      mbar_init(&a_full[s], 1);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&b_full[b], 4);
+      mbar_init(&b_empty[b], 1);
+      mbar_init(&d_full[b], 1);
+      mbar_init(&d_empty[b], 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_base_slot, 256);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tmem_base_slot;
+
+  auto fail = [&]() {
+    report(a.status, kStatusTimeout);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- A producer
+    if (lane == 0) {
+      int use = 0;
+      bool ok = true;
+      for (int k = blockIdx.x; k < n_items && ok; k += gridDim.x) {
+        int n, p;
+        item_of(a, k, &n, &p);
+        const int mc = chunk_count(a, n);
+        for (int m = 0; m < mc && ok; ++m) {
+          for (int part = 0; part < 2 && ok; ++part, ++use) {
+            const int s = use % kNSA;
+            if (use >= kNSA && !mbar_wait_bounded(&a_empty[s], ((use / kNSA) & 1) ^ 1, abort_flag)) {
+              fail();
+              ok = false;
+              break;
+            }
+            unsigned char* dst = A + s * kAStage;
+            mbar_arrive_expect_tx(&a_full[s], kAStage);
+            tc::tma_load_3d(dst, &kc_map, part * 128, 128 * m, p, &a_full[s]);
+            tc::tma_load_3d(dst + 16384, &kc_map, part * 128 + 64, 128 * m, p, &a_full[s]);
+          }
+        }
+      }
+      // drain copies still in flight before the CTA may exit
+      for (int u = max(0, use - kNSA); u < use; ++u) mbar_wait_bounded(&a_full[u % kNSA], (u / kNSA) & 1, nullptr);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int use = 0, mc_all = 0, it = 0;
+      bool ok = true;
+      const uint32_t bbase = smem_u32(Bop);
+      const uint32_t abase = smem_u32(A);
+      for (int k = blockIdx.x; k < n_items && ok; k += gridDim.x) {
+        int n, p;
+        item_of(a, k, &n, &p);
+        const int mc = chunk_count(a, n);
+        if (mc == 0) continue;
+        const int b = it & 1;
+        if (!mbar_wait_bounded(&b_full[b], (it >> 1) & 1, abort_flag)) { fail(); break; }
+        tc::fence_after_sync();
+        const uint32_t bhi = bbase + b * kBBuf, blo = bhi + 32768;
+        for (int m = 0; m < mc; ++m, ++mc_all) {
+          const int d = mc_all & 1;
+          if (mc_all >= 2 && !mbar_wait_bounded(&d_empty[d], ((mc_all >> 1) & 1) ^ 1, abort_flag)) {
+            fail();
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t dt = tbase + d * 128;
+          // hi part of Kc: hi*hi then hi*lo
+          int s = use % kNSA;
+          if (!mbar_wait_bounded(&a_full[s], (use / kNSA) & 1, abort_flag)) { fail(); ok = false; break; }
+          tc::fence_after_sync();
+          const uint32_t ahi = abase + s * kAStage;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            tc::mma_bf16(dt, tc::smem_desc(ahi + off, 16, 1024), tc::smem_desc(bhi + off, 16, 1024), kIdesc, kk > 0);
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            tc::mma_bf16(dt, tc::smem_desc(ahi + off, 16, 1024), tc::smem_desc(blo + off, 16, 1024), kIdesc, true);
+          }
+          tc::mma_commit(&a_empty[s]);
+          ++use;
+          // lo part of Kc: lo*hi
+          s = use % kNSA;
+          if (!mbar_wait_bounded(&a_full[s], (use / kNSA) & 1, abort_flag)) { fail(); ok = false; break; }
+          tc::fence_after_sync();
+          const uint32_t alo = abase + s * kAStage;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            tc::mma_bf16(dt, tc::smem_desc(alo + off, 16, 1024), tc::smem_desc(bhi + off, 16, 1024), kIdesc, true);
+          }
+          tc::mma_commit(&a_empty[s]);
+          ++use;
+          tc::mma_commit(&d_full[d]);
+        }
+        tc::mma_commit(&b_empty[b]);
+        ++it;
+      }
+      // every MMA issued has completed before the CTA tears TMEM down
+      tc::mma_commit(mma_done);
+      mbar_wait_bounded(mma_done, 0, nullptr);
+    }
+  } else if (warp < 6) {
+    // ---------------------------------------------------- B operand builders
+    const int wq = warp - 2;                       // rows wq*32 .. wq*32+31 of the item
+    const int cc = lane & 15;                      // 16-byte column chunk (8 columns)
+    const bool write_lo = lane >= 16;
+    int it = 0;
+    for (int k = blockIdx.x; k < n_items; k += gridDim.x) {
+      int n, p;
+      item_of(a, k, &n, &p);
+      if (chunk_count(a, n) == 0) continue;
+      const int b = it & 1;
+      if (it >= 2 && !mbar_wait_bounded(&b_empty[b], ((it >> 1) & 1) ^ 1, abort_flag)) {
+        if (lane == 0) fail();
+        break;
+      }
+      const int bi = p / a.Hkv, h = p % a.Hkv;
+      unsigned char* dst = Bop + b * kBBuf + (write_lo ? 32768 : 0) + (cc >> 3) * 16384;
+      for (int rb = 0; rb < 32; rb += 4) {
+        float acc[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
+          const int row = 128 * n + wq * 32 + rb + u;
+          if (row < a.T) {
+            const uint16_t* src = a.Q + ((static_cast<int64_t>(bi) * a.T + row) * a.Hq + h * a.G) * kHeadDim;
+            for (int c = lane; c < 16 * a.G; c += 32) {   // chunk c: head c / 16, columns 8 * (c % 16)
+              float f[8];
+              unpack8(__ldg(reinterpret_cast<const uint4*>(src) + c), f);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc[u][e] += f[e];
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = wq * 32 + rb + u;
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = (acc[u][e] + __shfl_xor_sync(0xffffffffu, acc[u][e], 16)) * a.scale;
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * e]), h1 = __float2bfloat16_rn(x[2 * e + 1]);
+            if (write_lo) {
+              w[e] = pack_bf16x2(x[2 * e] - __bfloat162float(h0), x[2 * e + 1] - __bfloat162float(h1));
+            } else {
+              w[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                     (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+            }
+          }
+          *reinterpret_cast<uint4*>(dst + tc::sw128_off(r, cc & 7)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b_full[b]);
+      ++it;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                        // TMEM lane quadrant of this warp
+    int mc_all = 0;
+    bool ok = true;
+    for (int k = blockIdx.x; k < n_items && ok; k += gridDim.x) {
+      int n, p;
+      item_of(a, k, &n, &p);
+      const int mc = chunk_count(a, n);
+      for (int m = 0; m < mc; ++m, ++mc_all) {
+        const int d = mc_all & 1;
+        if (!mbar_wait_bounded(&d_full[d], (mc_all >> 1) & 1, abort_flag)) {
+          if (lane == 0) fail();
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const int j = 128 * m + 32 * q + lane;      // this thread's block
+        float best[2];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float v[64];
+          tc::tmem_ld64(tbase + (static_cast<uint32_t>(32 * q) << 16) + d * 128 + half * 64, v);
+          tc::tmem_wait_ld();
+          const int t = 2 * n + half;
+          const int rows = min(kTile, a.T - t * kTile);    // ragged last tile
+          float mx = -CUDART_INF_F;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) mx = (c < rows) ? fmaxf(mx, v[c]) : mx;
+          best[half] = mx;
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&d_empty[d]);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int t = 2 * n + half;
+          if (t < a.n_tiles && is_candidate(a, t, j))
+            a.scores[(static_cast<int64_t>(p) * a.n_tiles + t) * a.nb + j] = best[half];
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, 256);
+  }
+}
+
+// Kc (fp32) -> [hi | lo] bf16 rows of 256 elements for the TMA loads.
+__global__ void kc_split_kernel(const float* Kc, uint16_t* out, int64_t rows) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;   // one float4 each
+  if (i >= rows * 32) return;
+  const int64_t r = i / 32, c = i % 32;
+  const float4 x = reinterpret_cast<const float4*>(Kc)[i];
+  const float v[4] = {x.x, x.y, x.z, x.w};
+  uint16_t hi[4], lo[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(v[e]);
+    hi[e] = __bfloat16_as_ushort(h);
+    lo[e] = __bfloat16_as_ushort(__float2bfloat16_rn(v[e] - __bfloat162float(h)));
+  }
+  uint16_t* o = out + r * 256 + c * 4;
+  *reinterpret_cast<uint2*>(o) = make_uint2(hi[0] | (uint32_t(hi[1]) << 16), hi[2] | (uint32_t(hi[3]) << 16));
+  *reinterpret_cast<uint2*>(o + 128) = make_uint2(lo[0] | (uint32_t(lo[1]) << 16), lo[2] | (uint32_t(lo[3]) << 16));
+}
+
+// Per (pair, tile) top-k over the candidate scores, one warp each.
+__global__ void __launch_bounds__(256) prefill_topk_kernel(PSArgs a, int top_k, int32_t* idx) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+  if (row >= static_cast<int64_t>(a.P) * a.n_tiles) return;
+  const int t = static_cast<int>(row % a.n_tiles);
+  unsigned* hist = reinterpret_cast<unsigned*>(smem_raw) + warp * (256 + a.nb);
+  uint32_t* keys = hist + 256;
+  const float* sc = a.scores + row * a.nb;
+  // blocks at or after the tile are never candidates
+  const int nb_t = min(a.nb, t);
+  for (int j0 = 0; j0 < nb_t; j0 += 8 * 32) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * 32 + lane;
+      v[u] = (j < nb_t && is_candidate(a, t, j)) ? __ldcg(sc + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * 32 + lane;
+      if (j < nb_t) {
+        const uint32_t key = float_key(v[u]);
+        keys[j] = is_candidate(a, t, j) ? (key == 0u ? 1u : key) : 0u;
+      }
+    }
+  }
+  __syncwarp();
+  warp_radix_select(keys, nb_t, top_k, idx + row * top_k, hist);
+}
+
+using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+size_t prefill_score_smem() {
+  return 1024 + kNSA * kAStage + 2 * kBBuf + 16 * 8 + 64;
+}
+
+cudaError_t launch_prefill_score(const PrefillArgs& pa, cudaStream_t s) {
+  EncodeFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  PSArgs a = {};
+  a.Q = static_cast<const uint16_t*>(pa.Q);
+  a.scores = pa.scores;
+  a.status = pa.status;
+  a.B = pa.B;
+  a.Hq = pa.Hq;
+  a.Hkv = pa.Hkv;
+  a.G = pa.Hq / pa.Hkv;
+  a.T = pa.T;
+  a.nb = pa.nb;
+  a.n_tiles = pa.n_tiles;
+  a.n_tpairs = (pa.n_tiles + 1) / 2;
+  a.P = pa.B * pa.Hkv;
+  a.S = pa.S;
+  a.W = pa.W;
+  a.scale = pa.scale;
+  if (a.nb > 0) {
+    // Kc -> hi / lo bf16
+    const int64_t rows = static_cast<int64_t>(a.P) * a.nb;
+    kc_split_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, s>>>(pa.Kc, pa.kc2, rows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    CUtensorMap map;
+    cuuint64_t dims[3] = {256, static_cast<cuuint64_t>(a.nb), static_cast<cuuint64_t>(a.P)};
+    cuuint64_t strides[2] = {256 * 2, static_cast<cuuint64_t>(a.nb) * 256 * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, pa.kc2, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    const size_t smem = prefill_score_smem();
+    e = cudaFuncSetAttribute(prefill_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int items = a.n_tpairs * a.P;
+    const int grid = items < pa.num_sms ? items : pa.num_sms;
+    prefill_score_kernel<<<grid, kScoreThreadsTC, smem, s>>>(map, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t rows = static_cast<int64_t>(a.P) * a.n_tiles;
+  const size_t smem_k = 8 * (256 + static_cast<size_t>(a.nb)) * 4;
+  cudaError_t e = cudaFuncSetAttribute(prefill_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem_k));
+  if (e != cudaSuccess) return e;
+  prefill_topk_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, smem_k, s>>>(a, pa.top_k, pa.idx);
+  return cudaGetLastError();
+}
+
+}  // namespace sa

@@ -213,6 +213,76 @@ DecodeAttnArgs attn_args(const sa_params* p, const DecodeGeom& g, const DecodePl
   return a;
 }
 
+// ---- prefill -------------------------------------------------------------------
+struct PrefillGeom {
+  int B, Hq, Hkv, G, T, nb, n_tiles, P;
+  int64_t cap;
+};
+
+// Shape limits of the tensor-core prefill path (besides check_params).
+sa_status check_prefill(const sa_params* p, PrefillGeom* g) {
+  if (p->dtype != SA_BF16) return fail(SA_ERR_UNSUPPORTED, "prefill runs on bf16 tensor cores: dtype must be SA_BF16");
+  if (p->num_q_heads != 4 * p->num_kv_heads)
+    return fail(SA_ERR_UNSUPPORTED, "prefill is built for GQA groups of 4 query heads per KV head");
+  if (p->block_size != 64) return fail(SA_ERR_UNSUPPORTED, "prefill is built for block_size 64 (= query tile)");
+  if (p->sink_keys % 64 != 0 || p->window_keys % 64 != 0)
+    return fail(SA_ERR_UNSUPPORTED, "prefill needs sink_keys and window_keys to be multiples of 64");
+  if (p->pool != SA_POOL_MEAN) return fail(SA_ERR_UNSUPPORTED, "prefill scoring is built for mean pooling");
+  g->B = p->batch;
+  g->Hq = p->num_q_heads;
+  g->Hkv = p->num_kv_heads;
+  g->G = 4;
+  g->T = p->n_q;
+  g->nb = p->n_q / 64;
+  g->n_tiles = (p->n_q + 63) / 64;
+  g->P = p->batch * p->num_kv_heads;
+  g->cap = p->kv_capacity;
+  if (g->nb > 6144) return fail(SA_ERR_UNSUPPORTED, "prefill is built for sequences up to 393216 tokens");
+  if (static_cast<int64_t>(g->B) * g->T > 0x7fffffff) return fail(SA_ERR_UNSUPPORTED, "too many tokens");
+  return SA_OK;
+}
+
+struct PrefillWs {
+  size_t kc2, scores, idx, clean, total;
+};
+
+PrefillWs prefill_ws(const PrefillGeom& g, int top_k, int op, int idx_len) {
+  PrefillWs w = {};
+  size_t off = kWsHeader;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = align_up(off + bytes, 1024);
+    return at;
+  };
+  const size_t rows = static_cast<size_t>(g.P) * g.n_tiles;
+  if (op == SA_OP_PREFILL || op == SA_OP_SCORE_TOPK) {
+    w.kc2 = take(static_cast<size_t>(g.P) * g.nb * 512);
+    w.scores = take(rows * g.nb * 4);
+  }
+  if (op == SA_OP_PREFILL) w.idx = take(rows * static_cast<size_t>(top_k) * 4);
+  if (op == SA_OP_GIVEN_IDX) w.clean = take(rows * static_cast<size_t>(idx_len) * 4);
+  w.total = off;
+  return w;
+}
+
+PrefillArgs prefill_args(const sa_params* p, const PrefillGeom& g) {
+  PrefillArgs a = {};
+  a.B = g.B;
+  a.Hq = g.Hq;
+  a.Hkv = g.Hkv;
+  a.T = g.T;
+  a.nb = g.nb;
+  a.n_tiles = g.n_tiles;
+  a.top_k = p->top_k;
+  a.out_bf16 = p->out_dtype == SA_BF16;
+  a.num_sms = device_sms();
+  a.cap = g.cap;
+  a.S = p->sink_keys;
+  a.W = p->window_keys;
+  a.scale = scale_of(p);
+  return a;
+}
+
 }  // namespace
 }  // namespace sa
 
@@ -240,7 +310,11 @@ const char* sa_status_string(sa_status s) {
 size_t sa_workspace_size(const sa_params* p, int32_t op) {
   const bool prefill = (op == SA_OP_PREFILL) || (p && p->select == SA_SEL_TILE_MAX);
   if (check_params(p, prefill) != SA_OK) return 0;
-  if (prefill) return 0;   // prefill is not built in this library version
+  if (prefill) {
+    PrefillGeom g;
+    if (check_prefill(p, &g) != SA_OK) return 0;
+    return prefill_ws(g, p->top_k, op, p->top_k).total;
+  }
   DecodeGeom g;
   DecodePlan plan;
   int slots = (op == SA_OP_DECODE) ? p->top_k : 0;
@@ -283,7 +357,25 @@ sa_status sa_score_topk(const sa_params* p, const void* Q, const float* Kc, int3
   const bool prefill = p && p->select == SA_SEL_TILE_MAX;
   sa_status st = check_params(p, prefill);
   if (st != SA_OK) return st;
-  if (prefill) return fail(SA_ERR_UNSUPPORTED, "SA_SEL_TILE_MAX scoring is not built in this library version");
+  if (prefill) {
+    PrefillGeom g;
+    if ((st = check_prefill(p, &g)) != SA_OK) return st;
+    if (!Q || (!Kc && g.nb > 0) || (!idx && p->top_k > 0)) return fail(SA_ERR_INVALID, "Q, Kc and idx must be non-NULL");
+    if (!aligned16(Q) || !aligned16(Kc)) return fail(SA_ERR_INVALID, "Q and Kc must be 16-byte aligned");
+    const PrefillWs L = prefill_ws(g, p->top_k, SA_OP_SCORE_TOPK, 0);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != SA_OK) return st;
+    unsigned char* w = static_cast<unsigned char*>(ws);
+    PrefillArgs a = prefill_args(p, g);
+    a.Q = Q;
+    a.Kc = Kc;
+    a.kc2 = reinterpret_cast<uint16_t*>(w + L.kc2);
+    a.scores = scores ? scores : reinterpret_cast<float*>(w + L.scores);
+    a.idx = idx;
+    a.status = reinterpret_cast<unsigned*>(w);
+    cudaError_t e = launch_prefill_score(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "prefill scoring launch");
+    return SA_OK;
+  }
   if (!Q || (!Kc && p->ctx_len >= p->block_size) || (!idx && p->top_k > 0))
     return fail(SA_ERR_INVALID, "Q, Kc and idx must be non-NULL (Kc may be NULL without a complete block)");
   if (!aligned16(Q) || !aligned16(Kc)) return fail(SA_ERR_INVALID, "Q and Kc must be 16-byte aligned");
@@ -309,19 +401,45 @@ sa_status sa_sparse_attn_given_idx(const sa_params* p, const void* Q, const void
   const bool prefill = p && p->select == SA_SEL_TILE_MAX;
   sa_status st = check_params(p, prefill);
   if (st != SA_OK) return st;
-  if (prefill) return fail(SA_ERR_UNSUPPORTED, "prefill index tables are not built in this library version");
   if (!Q || !K || !V || !O) return fail(SA_ERR_INVALID, "Q, K, V and O must be non-NULL");
   if (idx_len < 0 || idx_len > 4096) return fail(SA_ERR_INVALID, "idx_len %d must be in [0, 4096]", idx_len);
   if (idx_len > 0 && !idx) return fail(SA_ERR_INVALID, "idx is NULL");
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
     return fail(SA_ERR_INVALID, "Q, K, V and O must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (prefill) {
+    PrefillGeom g;
+    if ((st = check_prefill(p, &g)) != SA_OK) return st;
+    const PrefillWs L = prefill_ws(g, p->top_k, SA_OP_GIVEN_IDX, idx_len);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != SA_OK) return st;
+    unsigned char* w = static_cast<unsigned char*>(ws);
+    const int32_t* table = idx;
+    if (!(p->flags & SA_FLAG_TRUSTED_IDX)) {
+      int32_t* clean = reinterpret_cast<int32_t*>(w + L.clean);
+      cudaError_t e = launch_sanitize_prefill_idx(idx, clean, g.P, g.n_tiles, idx_len, p->sink_keys, p->window_keys,
+                                                  reinterpret_cast<unsigned*>(w), s);
+      if (e != cudaSuccess) return cuda_fail(e, "index-table check launch");
+      table = clean;
+    }
+    PrefillArgs a = prefill_args(p, g);
+    a.Q = Q;
+    a.K = K;
+    a.V = V;
+    a.idx = const_cast<int32_t*>(table);
+    a.top_k = idx_len;
+    a.O = O;
+    a.lse = lse;
+    a.status = reinterpret_cast<unsigned*>(w);
+    cudaError_t e = launch_prefill_attn(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
+    return SA_OK;
+  }
   DecodeGeom g;
   DecodePlan plan;
   if ((st = plan_for(p, idx_len, &g, &plan)) != SA_OK) return st;
   const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_GIVEN_IDX, idx_len);
   if ((st = check_ws(ws, ws_bytes, L.total)) != SA_OK) return st;
   unsigned char* w = static_cast<unsigned char*>(ws);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int32_t* table = idx;
   cudaError_t e = cudaSuccess;
   if (!(p->flags & SA_FLAG_TRUSTED_IDX)) {
@@ -371,8 +489,33 @@ sa_status sa_sparse_attn_prefill(const sa_params* p, const void* Q, const void* 
                                  void* O, float* lse, int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
   sa_status st = check_params(p, true);
   if (st != SA_OK) return st;
-  (void)Q; (void)K; (void)V; (void)Kc; (void)O; (void)lse; (void)idx_out; (void)ws; (void)ws_bytes; (void)stream;
-  return fail(SA_ERR_UNSUPPORTED, "prefill is not built in this library version");
+  PrefillGeom g;
+  if ((st = check_prefill(p, &g)) != SA_OK) return st;
+  if (!Q || !K || !V || !O || (!Kc && g.nb > 0)) return fail(SA_ERR_INVALID, "Q, K, V, Kc and O must be non-NULL");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(Kc))
+    return fail(SA_ERR_INVALID, "Q, K, V, Kc and O must be 16-byte aligned");
+  const PrefillWs L = prefill_ws(g, p->top_k, SA_OP_PREFILL, 0);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != SA_OK) return st;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = sa_pool_keys(p, K, Kc, stream)) != SA_OK) return st;
+  PrefillArgs a = prefill_args(p, g);
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.Kc = Kc;
+  a.kc2 = reinterpret_cast<uint16_t*>(w + L.kc2);
+  a.scores = reinterpret_cast<float*>(w + L.scores);
+  a.idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + L.idx);
+  a.O = O;
+  a.lse = lse;
+  a.status = reinterpret_cast<unsigned*>(w);
+  cudaError_t e = launch_prefill_score(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill scoring launch");
+  e = launch_prefill_attn(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
+  return SA_OK;
+
 }
 
 sa_status sa_read_status(void* ws, void* stream) {
