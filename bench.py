@@ -331,6 +331,10 @@ def run_ours(args, w, rank, world, local_rank):
     # --- kernels alone (roofline), rank-local -----------------------------
     attn_ms = statistics.mean(timed_steps(attn_only, max(50, args.steps // 4), 3, stream, flush))
     pool_ms = statistics.mean(timed_steps(pool_only, 10, 2, stream, flush))
+    # --- causal prefill (tensor cores), rank-local --------------------------
+    prefill = None
+    if not args.no_prefill:
+        prefill = run_prefill_bench(args, dev, stream, flush)
     # --- end to end through the C ABI with host buffers -------------------
     e2e = e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush)
     if world > 1:
@@ -366,10 +370,103 @@ def run_ours(args, w, rank, world, local_rank):
                 "note": "per step: pinned host -> device copy of the new tokens' Q, K, V rows, the decode "
                         "call through the C ABI, device -> pinned host copy of O; the KV cache and the "
                         "compressed keys stay resident in HBM"},
+        "prefill": prefill,
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
     return line
+
+
+def prefill_counts(w):
+    """Algorithmic and executed tensor-core FLOPs of one causal prefill of
+    workload w (sink / window multiples of 64, tile = block = 64)."""
+    T, b, k = w.n_q, w.block_size, w.top_k
+    Hq, Hkv, G, d = w.num_q_heads, w.num_kv_heads, w.group, w.head_dim
+    nt, nb = (T + b - 1) // b, T // b
+    attn_alg = 0
+    blocks = 0
+    score_alg = 0
+    for t in range(nt):
+        C = t * b
+        s_end = min(w.sink_keys, C)
+        w_begin = max(C - w.window_keys, s_end)
+        cand = sum(1 for j in range(min(nb, t)) if j * b < w_begin and (j + 1) * b > s_end)
+        ke = min(k, cand)
+        rows = min(b, T - C)
+        ctx_keys = s_end + ke * b + (C - w_begin)
+        attn_alg += Hq * 4 * d * (rows * ctx_keys + rows * (rows + 1) // 2)
+        blocks += s_end // b + ke + (C - w_begin) // b + 1
+        score_alg += Hkv * cand * rows * 2 * d
+    attn_exec = Hkv * blocks * (G * b) * 4 * b * d            # S and PV, 256 rows x 64 keys x 128
+    npairs = (nt + 1) // 2
+    score_exec = 0
+    for n in range(npairs):
+        t = min(2 * n + 1, nt - 1)
+        C = t * b
+        s_end = min(w.sink_keys, C)
+        w_begin = max(C - w.window_keys, s_end)
+        j_lim = min(nb, -(-w_begin // b))
+        if j_lim * b > s_end:
+            score_exec += Hkv * (-(-j_lim // 128)) * 128 * 128 * 384 * 2
+    return dict(attn_alg=attn_alg, attn_exec=attn_exec, score_alg=score_alg, score_exec=score_exec)
+
+
+def run_prefill_bench(args, dev, stream, flush):
+    """Times the full causal prefill and its two tensor-core kernels alone."""
+    from top_block_sparse_b200 import sa
+    w = WORKLOADS["prefill_64k"]
+    if args.prefill_tokens:
+        w = w.scaled(n_q=args.prefill_tokens)
+    inp = make_inputs(w, seed=2001, device=dev)
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    del inp
+    p = sa.params_for(w)
+    T = w.n_q
+    nb, nt = T // 64, (T + 63) // 64
+    Kc = torch.empty((1, w.num_kv_heads, nb, 128), device=dev)
+    O = torch.empty((1, T, w.num_q_heads, 128), device=dev, dtype=torch.bfloat16)
+    lse = torch.empty((1, T, w.num_q_heads), device=dev)
+    idx = torch.empty((1, w.num_kv_heads, nt, w.top_k), device=dev, dtype=torch.int32)
+    ws = sa.alloc_workspace(p, sa.SA_OP_PREFILL, device=dev)
+    ws_s = sa.alloc_workspace(p, sa.SA_OP_SCORE_TOPK, device=dev)
+    pt = sa.params_for(w)
+    pt.flags = sa.SA_FLAG_TRUSTED_IDX
+    ws_g = sa.alloc_workspace(pt, sa.SA_OP_GIVEN_IDX, device=dev)
+
+    def full():
+        sa.sparse_attn_prefill(p, Q, K, V, Kc, O, lse, idx, ws, stream=stream)
+
+    def score():
+        sa.score_topk(p, Q, Kc, idx, None, ws_s, stream=stream)
+
+    def attn():
+        sa.sparse_attn_given_idx(pt, Q, K, V, idx, O, lse, ws_g, stream=stream)
+
+    n = args.prefill_steps
+    full_ms = statistics.mean(timed_steps(full, n, 3, stream, flush))
+    score_ms = statistics.mean(timed_steps(score, n, 3, stream, flush))
+    attn_ms = statistics.mean(timed_steps(attn, n, 3, stream, flush))
+    if sa.read_status(ws, stream) != sa.SA_OK:
+        raise RuntimeError("device status word set during the prefill runs")
+    c = prefill_counts(w)
+    hbm, tfl, tfl_s, src = peaks()
+    return {
+        "workload": f"prefill_64k: causal prefill T={w.n_q}, Hq=32, Hkv=8, d=128, bf16, tile = block 64, "
+                    "top-k 64 + sink 64 keys + window 256 keys",
+        "ms": full_ms,
+        "tflops": (c["attn_alg"] + c["score_alg"]) / (full_ms * 1e-3) / 1e12,
+        "tflops_note": "algorithmic attention + scoring FLOPs / whole prefill time (pool, score, top-k, attention)",
+        "attention": {"kernel": "prefill_attn_kernel (tcgen05)", "ms": attn_ms,
+                      "exec_tflops": c["attn_exec"] / (attn_ms * 1e-3) / 1e12,
+                      "alg_tflops": c["attn_alg"] / (attn_ms * 1e-3) / 1e12,
+                      "frac_of_bf16_peak": c["attn_exec"] / (attn_ms * 1e-3) / 1e12 / tfl,
+                      "exec_flop": c["attn_exec"], "alg_flop": c["attn_alg"]},
+        "scoring": {"kernel": "kc_split + prefill_score_kernel (tcgen05, split bf16 x3) + prefill_topk_kernel",
+                    "ms": score_ms, "exec_tflops": c["score_exec"] / (score_ms * 1e-3) / 1e12,
+                    "frac_of_bf16_peak": c["score_exec"] / (score_ms * 1e-3) / 1e12 / tfl,
+                    "alg_gflop": c["score_alg"] / 1e9, "exec_gflop": c["score_exec"] / 1e9},
+        "peak_bf16_tflops": tfl, "peak_source": src,
+    }
 
 
 def e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush):
@@ -410,6 +507,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-pairs", type=int, default=16)
     ap.add_argument("--ref-pairs", type=int, default=4)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--prefill-steps", type=int, default=10)
+    ap.add_argument("--prefill-tokens", type=int, default=None,
+                    help="override the prefill length (smaller cases for ncu captures)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for ncu captures)")
     args = ap.parse_args()
