@@ -40,6 +40,21 @@ constexpr uint32_t kIdescS = tc::idesc_bf16(128, 64, false, false);
 constexpr uint32_t kIdescO = tc::idesc_bf16(128, 128, false, true);
 constexpr float kLazy = 8.f;                   // rescale when the max grows by > 2^8
 
+// 2^x by the hardware approximation (ex2.approx, relative error ~2^-22);
+// 2^-inf = 0.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two fp32 -> packed bf16 pair (round to nearest even), lo in the low half.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 struct PAArgs {
   const int32_t* idx;       // [P, n_tiles, k]
   void* O;                  // [B, T, Hq, 128]
@@ -285,19 +300,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);
-        const bool diag = b == bl.n_blk - 1;
-        float mx = -CUDART_INF_F;
+        const bool diag = b == bl.n_blk - 1;          // the tile's own block: causal
+        if (diag) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          s[c] = (!diag || c <= r) ? s[c] * a.scale_log2 : -CUDART_INF_F;
-          mx = fmaxf(mx, s[c]);
+          for (int c = 0; c < 64; ++c) s[c] = (c <= r) ? s[c] : -CUDART_INF_F;
         }
+        // row max of the raw logits (8 independent chains; the scale is > 0)
+        float m8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8[e] = s[e];
+#pragma unroll
+        for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * a.scale_log2;
         float factor = 1.f;
         bool rescale = false;
         if (mx > m_ref + kLazy) {
           const float m_new = mx;
           if (m_ref != -CUDART_INF_F) {
-            factor = exp2f(m_ref - m_new);
+            factor = ex2(m_ref - m_new);
             rescale = true;
           }
           l *= factor;
@@ -311,30 +332,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::fence_after_sync();
         if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int c0 = 0; c0 < 128; c0 += 64) {
-            float o[64];
-            tc::tmem_ld64(t_o + c0, o);
+#pragma unroll 1
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            float o[32];
+            tc::tmem_ld32(t_o + c0, o);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 64; ++c) o[c] *= factor;
-            tc::tmem_st64(t_o + c0, o);
+            for (int c = 0; c < 32; ++c) o[c] *= factor;
+            tc::tmem_st32(t_o + c0, o);
           }
           tc::tmem_wait_st();
         }
-        float ls = 0.f;
+        // p = 2^(s * scale_log2 - m_ref): one FFMA and one ex2 per element; the
+        // row sum uses the fp32 values, P goes to the tensor cores in bf16
+        float ls0 = 0.f, ls1 = 0.f;
+        const float neg_m = -m_ref;
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat16 p0 = __float2bfloat16_rn(exp2f(s[8 * c8 + 2 * e] - m_ref));
-            const __nv_bfloat16 p1 = __float2bfloat16_rn(exp2f(s[8 * c8 + 2 * e + 1] - m_ref));
-            ls += __bfloat162float(p0) + __bfloat162float(p1);
-            w[e] = static_cast<uint32_t>(__bfloat16_as_ushort(p0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(p1)) << 16);
+            const float p0 = ex2(fmaf(s[8 * c8 + 2 * e], a.scale_log2, neg_m));
+            const float p1 = ex2(fmaf(s[8 * c8 + 2 * e + 1], a.scale_log2, neg_m));
+            ls0 += p0;
+            ls1 += p1;
+            w[e] = cvt_bf16x2(p0, p1);
           }
           *reinterpret_cast<uint4*>(prow + tc::sw128_off(q * 32 + lane, c8)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        const float ls = ls0 + ls1;
         l += ls;
         tc::fence_proxy_async_smem();
         tc::fence_before_sync();
@@ -353,23 +379,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = tok < a.T;
       const int64_t orow = (static_cast<int64_t>(bi) * a.T + tok) * a.Hq + h * kG + g;
       const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 64) {
-        float o[64];
-        tc::tmem_ld64(t_o + c0, o);
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        float o[32];
+        tc::tmem_ld32(t_o + c0, o);
         tc::tmem_wait_ld();
         if (valid) {
           if (a.out_bf16) {
             uint16_t* dst = static_cast<uint16_t*>(a.O) + orow * kHeadDim + c0;
 #pragma unroll
-            for (int c = 0; c < 64; c += 8)
+            for (int c = 0; c < 32; c += 8)
               *reinterpret_cast<uint4*>(dst + c) =
                   make_uint4(pack_bf16x2(o[c] * inv, o[c + 1] * inv), pack_bf16x2(o[c + 2] * inv, o[c + 3] * inv),
                              pack_bf16x2(o[c + 4] * inv, o[c + 5] * inv), pack_bf16x2(o[c + 6] * inv, o[c + 7] * inv));
           } else {
             float* dst = static_cast<float*>(a.O) + orow * kHeadDim + c0;
 #pragma unroll
-            for (int c = 0; c < 64; c += 4)
+            for (int c = 0; c < 32; c += 4)
               *reinterpret_cast<float4*>(dst + c) = make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
           }
         }

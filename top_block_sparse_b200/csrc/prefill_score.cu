@@ -19,9 +19,10 @@
 // pair of query tiles) in decreasing-cost order):
 //   warp 0      TMA producer: Kc hi / lo chunks of 128 blocks (128-byte swizzle)
 //   warp 1      TMEM owner and MMA issuer (one thread)
-//   warps 2-5   build the B operand: GQA sum x scale of 128 query rows, split
-//               into hi / lo, written to swizzled shared memory
-//   warps 6-9   epilogue: TMEM -> registers, max over each 64-row tile,
+//   warps 2-9   build the B operand: GQA sum x scale of 128 query rows, split
+//               into hi / lo, written to swizzled shared memory (16 rows per
+//               warp, 8 rows of loads in flight: Q is the kernel's HBM stream)
+//   warps 10-13 epilogue: TMEM -> registers, max over each 64-row tile,
 //               candidate mask, fp32 scores to global
 #include <cudaTypedefs.h>
 #include <math_constants.h>
@@ -38,7 +39,8 @@ constexpr int kTile = 64;                      // query rows per tile = block si
 constexpr int kNSA = 3;                        // A stages (32 KB: hi or lo of a 128-block chunk)
 constexpr int kAStage = 32768;
 constexpr int kBBuf = 65536;                   // B operand: hi atoms 0,1 then lo atoms 0,1
-constexpr int kScoreThreadsTC = 320;
+constexpr int kScoreThreadsTC = 448;
+constexpr int kBuilders = 8;                   // warps 2..9 build the B operand, 16 rows each
 constexpr uint32_t kIdesc = tc::idesc_bf16(128, 128, false, false);
 
 struct PSArgs {
@@ -104,7 +106,7 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
       mbar_init(&a_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&b_full[b], 4);
+      mbar_init(&b_full[b], kBuilders);
       mbar_init(&b_empty[b], 1);
       mbar_init(&d_full[b], 1);
       mbar_init(&d_empty[b], 4);
@@ -217,9 +219,12 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
       tc::mma_commit(mma_done);
       mbar_wait_bounded(mma_done, 0, nullptr);
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + kBuilders) {
     // ---------------------------------------------------- B operand builders
-    const int wq = warp - 2;                       // rows wq*32 .. wq*32+31 of the item
+    // A row's G = 4 query heads are 1 KB contiguous = 64 chunks of 16 B: lane l
+    // loads chunks l (head l / 16) and l + 32 (head l / 16 + 2), both of column
+    // chunk cc = l % 16; lanes l and l ^ 16 hold the other two heads.
+    const int wq = warp - 2;                       // rows wq*16 .. wq*16+15 of the item
     const int cc = lane & 15;                      // 16-byte column chunk (8 columns)
     const bool write_lo = lane >= 16;
     int it = 0;
@@ -234,35 +239,38 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
       }
       const int bi = p / a.Hkv, h = p % a.Hkv;
       unsigned char* dst = Bop + b * kBBuf + (write_lo ? 32768 : 0) + (cc >> 3) * 16384;
-      for (int rb = 0; rb < 32; rb += 4) {
-        float acc[4][8];
+#pragma unroll 1
+      for (int rb = 0; rb < 16; rb += 8) {
+        uint4 x[8][2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
-          const int row = 128 * n + wq * 32 + rb + u;
+        for (int u = 0; u < 8; ++u) {
+          const int row = 128 * n + wq * 16 + rb + u;
           if (row < a.T) {
-            const uint16_t* src = a.Q + ((static_cast<int64_t>(bi) * a.T + row) * a.Hq + h * a.G) * kHeadDim;
-            for (int c = lane; c < 16 * a.G; c += 32) {   // chunk c: head c / 16, columns 8 * (c % 16)
-              float f[8];
-              unpack8(__ldg(reinterpret_cast<const uint4*>(src) + c), f);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) acc[u][e] += f[e];
-            }
+            const uint4* src = reinterpret_cast<const uint4*>(
+                a.Q + ((static_cast<int64_t>(bi) * a.T + row) * a.Hq + h * 4) * kHeadDim);
+            x[u][0] = __ldg(src + lane);
+            x[u][1] = __ldg(src + lane + 32);
+          } else {
+            x[u][0] = make_uint4(0u, 0u, 0u, 0u);
+            x[u][1] = x[u][0];
           }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int r = wq * 32 + rb + u;
-          float x[8];
+        for (int u = 0; u < 8; ++u) {
+          const int r = wq * 16 + rb + u;
+          float f0[8], f1[8], v[8];
+          unpack8(x[u][0], f0);
+          unpack8(x[u][1], f1);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = (acc[u][e] + __shfl_xor_sync(0xffffffffu, acc[u][e], 16)) * a.scale;
+          for (int e = 0; e < 8; ++e) v[e] = f0[e] + f1[e];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = (v[e] + __shfl_xor_sync(0xffffffffu, v[e], 16)) * a.scale;
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * e]), h1 = __float2bfloat16_rn(x[2 * e + 1]);
+            const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * e]), h1 = __float2bfloat16_rn(v[2 * e + 1]);
             if (write_lo) {
-              w[e] = pack_bf16x2(x[2 * e] - __bfloat162float(h0), x[2 * e + 1] - __bfloat162float(h1));
+              w[e] = pack_bf16x2(v[2 * e] - __bfloat162float(h0), v[2 * e + 1] - __bfloat162float(h1));
             } else {
               w[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
                      (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
@@ -353,8 +361,7 @@ __global__ void __launch_bounds__(256) prefill_topk_kernel(PSArgs a, int top_k, 
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + warp;
   if (row >= static_cast<int64_t>(a.P) * a.n_tiles) return;
   const int t = static_cast<int>(row % a.n_tiles);
-  unsigned* hist = reinterpret_cast<unsigned*>(smem_raw) + warp * (256 + a.nb);
-  uint32_t* keys = hist + 256;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw) + warp * a.nb;
   const float* sc = a.scores + row * a.nb;
   // blocks at or after the tile are never candidates
   const int nb_t = min(a.nb, t);
@@ -375,7 +382,7 @@ __global__ void __launch_bounds__(256) prefill_topk_kernel(PSArgs a, int top_k, 
     }
   }
   __syncwarp();
-  warp_radix_select(keys, nb_t, top_k, idx + row * top_k, hist);
+  warp_topk(keys, nb_t, top_k, idx + row * top_k);
 }
 
 using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
@@ -442,7 +449,7 @@ cudaError_t launch_prefill_score(const PrefillArgs& pa, cudaStream_t s) {
     if (e != cudaSuccess) return e;
   }
   const int64_t rows = static_cast<int64_t>(a.P) * a.n_tiles;
-  const size_t smem_k = 8 * (256 + static_cast<size_t>(a.nb)) * 4;
+  const size_t smem_k = 8 * static_cast<size_t>(a.nb) * 4;
   cudaError_t e = cudaFuncSetAttribute(prefill_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem_k));
   if (e != cudaSuccess) return e;

@@ -42,6 +42,19 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_query0_kernel(ScoreA
 
   static_assert(kScoreBlocksPerChunk % kScoreWarps == 0 && kScoreBlocksPerChunk / kScoreWarps <= 32,
                 "rows per warp");
+  const int64_t j_begin = static_cast<int64_t>(chunk) * a.blocks_per_chunk;
+  const int64_t j_end = min(a.nb, j_begin + a.blocks_per_chunk);
+  const float* kc = a.Kc + static_cast<int64_t>(pair) * a.nb * kHeadDim;
+  float* sc = a.scores + static_cast<int64_t>(pair) * a.nb;
+  // every warp streams kRowsPerWarp rows; their loads are issued first, before
+  // the index query is formed, so the two latencies overlap
+  constexpr int kRowsPerWarp = kScoreBlocksPerChunk / kScoreWarps;
+  const int64_t jw = j_begin + static_cast<int64_t>(warp) * kRowsPerWarp;
+  float4 r[kRowsPerWarp];
+#pragma unroll
+  for (int u = 0; u < kRowsPerWarp; ++u)
+    r[u] = (jw + u < j_end) ? __ldcs(reinterpret_cast<const float4*>(kc + (jw + u) * kHeadDim) + lane)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
   // index query of the first new token: sum over the GQA group
   if (tid < kHeadDim) {
     float s = 0.f;
@@ -71,18 +84,6 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_query0_kernel(ScoreA
   __syncthreads();
 
   const float4 q4 = reinterpret_cast<const float4*>(qs)[lane];
-  const int64_t j_begin = static_cast<int64_t>(chunk) * a.blocks_per_chunk;
-  const int64_t j_end = min(a.nb, j_begin + a.blocks_per_chunk);
-  const float* kc = a.Kc + static_cast<int64_t>(pair) * a.nb * kHeadDim;
-  float* sc = a.scores + static_cast<int64_t>(pair) * a.nb;
-  // every warp streams kRowsPerWarp rows; all their loads are issued first
-  constexpr int kRowsPerWarp = kScoreBlocksPerChunk / kScoreWarps;
-  const int64_t jw = j_begin + static_cast<int64_t>(warp) * kRowsPerWarp;
-  float4 r[kRowsPerWarp];
-#pragma unroll
-  for (int u = 0; u < kRowsPerWarp; ++u)
-    r[u] = (jw + u < j_end) ? __ldcs(reinterpret_cast<const float4*>(kc + (jw + u) * kHeadDim) + lane)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
   float d[kRowsPerWarp];
 #pragma unroll
   for (int u = 0; u < kRowsPerWarp; ++u) d[u] = r[u].x * q4.x + r[u].y * q4.y + r[u].z * q4.z + r[u].w * q4.w;
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_query0_kernel(ScoreA
     }
   }
   __syncwarp();
-  warp_radix_select(keys, nb, a.top_k, a.idx + static_cast<int64_t>(pair) * a.top_k, hist);
+  warp_topk(keys, nb, a.top_k, a.idx + static_cast<int64_t>(pair) * a.top_k);
 }
 
 }  // namespace
