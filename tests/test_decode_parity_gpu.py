@@ -125,6 +125,52 @@ def test_score_topk_parity(name, over):
     print(f"\n{name}: near-ties {ties}/{len(ref)}")
 
 
+# ----------------------------------- scorer chunking and the two selectors --
+
+@pytest.mark.parametrize("B,Hkv,nb,k,dup", [
+    (1, 1, 2100, 32, False),      # one pair over many CTAs, CTA-wide selection
+    (1, 1, 16384, 200, False),    # the largest table the selector takes
+    (38, 8, 2100, 32, False),     # one CTA per pair, CTA-wide selection
+    (38, 8, 600, 32, False),      # one CTA per pair, warp selection
+    (1, 4, 600, 48, False),       # several CTAs per pair, warp selection
+    (1, 2, 3000, 64, True),       # duplicated rows: exact ties go to the lower id
+    (2, 2, 2500, 3000, False),    # k above the number of candidates
+])
+def test_score_topk_given_compressed_keys(B, Hkv, nb, k, dup):
+    C = nb * 64 + 17
+    w = WORKLOADS["decode_32k"].scaled(batch=B, num_kv_heads=Hkv, num_q_heads=4 * Hkv, ctx_len=C, top_k=k)
+    p = sa.params_for(w)
+    g = torch.Generator().manual_seed(1000 * nb + k)
+    Kc = torch.randn((B, Hkv, nb, 128), generator=g) * 0.125     # the spread of 64-key means
+    if dup:
+        Kc[:, :, 1::2] = Kc[:, :, 0::2]
+    Q = torch.randn((B, 1, 4 * Hkv, 128), generator=g).to(torch.bfloat16)
+    idx = torch.empty((B, Hkv, k), device="cuda", dtype=torch.int32)
+    scores = torch.empty((B, Hkv, nb), device="cuda")
+    ws = sa.alloc_workspace(p, sa.SA_OP_SCORE_TOPK)
+    sa.score_topk(p, Q.cuda(), Kc.cuda(), idx, scores, ws)
+    torch.cuda.synchronize()
+    op = oracle_params(w)
+    cand = orc.candidate_blocks(C, op)
+    idx_h, sc_h = idx.cpu().numpy(), scores.cpu().double().numpy()
+    ties = 0
+    for b in range(B):
+        for h in range(Hkv):
+            qbar = orc.index_query(Q[b, 0, 4 * h:4 * h + 4].double().numpy())
+            ref = orc.block_scores(qbar, Kc[b, h].double().numpy(), op)
+            np.testing.assert_allclose(sc_h[b, h], ref, atol=2e-5, rtol=2e-5)
+            sel = orc.select_topk(ref, cand, k)
+            v = compare_sets(idx_h[b, h], sel)
+            assert v != "mismatch", (b, h)
+            ties += v == "near_tie"
+            if dup:
+                got = set(int(j) for j in idx_h[b, h] if j >= 0)
+                for j in got:
+                    if j % 2 == 1 and (j - 1) in cand:
+                        assert j - 1 in got, (b, h, j)
+    print(f"\nnb={nb} k={k} pairs={B * Hkv}: near-ties {ties}")
+
+
 # -------------------------------------------------------- given index table --
 
 @pytest.mark.parametrize("name,over", [

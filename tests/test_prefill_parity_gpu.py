@@ -145,6 +145,17 @@ def test_prefill_bf16_output_and_reuse():
     assert torch.equal(idx1, idx2) and torch.equal(O1, O2)
 
 
+def test_prefill_long_rows_select_from_shared_memory():
+    """T = 2100 blocks + 5 tokens: tiles past block 2048 take the selector's
+    shared-memory path."""
+    w = pf(64 * 2100 + 5, Hkv=1, k=16)
+    inp = make_inputs(w, seed=10, device="cuda")
+    _, Kc, O, lse, idx = run_prefill(w, inp, out_dtype="bf16")
+    torch.cuda.synchronize()
+    ties = check_tiles(w, inp, O, lse, idx, [0, 6, 2047, 2048, 2049, 2099, 2100])
+    print(f"\nprefill T={w.n_q}: near-ties {ties}")
+
+
 def test_prefill_full_size_sampled():
     """The benchmark configuration (T = 65536, 8 KV heads); the oracle checks
     sampled tiles of every head."""

@@ -35,19 +35,13 @@
 #include <math_constants.h>
 
 #include "common.cuh"
+#include "decode_units.cuh"
 #include "internal.h"
 
 namespace sa {
 namespace {
 
 constexpr int kCombStride = 132;   // floats per (row) in the combine buffer: 128 O + m + l + pad
-
-// Key ranges of the two tiles of one ring stage (n == 0: empty tile).
-struct StageInfo {
-  int64_t ks0, ks1;
-  int n0, n1;
-  int64_t pad;
-};
 
 __device__ __forceinline__ void consumer_bar(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
@@ -75,33 +69,6 @@ __device__ __forceinline__ u64 mul2(u64 a, u64 b) {
 }
 // two bf16 (one 32-bit word) -> packed fp32 pair
 __device__ __forceinline__ u64 bf2(uint32_t w) { return pk2(bf16lo(w), bf16hi(w)); }
-
-// Key range of tile u (0 <= u < MT) of a pair; nkeys == 0 means empty.  The
-// index table holds valid ids or -1 (caller tables are sanitised first).
-__device__ __forceinline__ void tile_range(const DecodeAttnArgs& a, int64_t pair, int u, int64_t* ks,
-                                           int* nk) {
-  int64_t s = 0, e = 0;
-  const int T = a.tile;
-  if (u < a.n_sink_tiles) {
-    s = static_cast<int64_t>(u) * T;
-    e = min(s + T, a.s_end);
-  } else if ((u -= a.n_sink_tiles) < a.idx_stride * a.tpb) {
-    const int sl = u / a.tpb, sub = u - sl * a.tpb;
-    const int32_t j = __ldg(a.idx + pair * a.idx_stride + sl);
-    if (j >= 0) {
-      const int64_t lo = max(static_cast<int64_t>(j) * a.b, a.s_end);
-      const int64_t hi = min(static_cast<int64_t>(j + 1) * a.b, a.w_begin);
-      s = lo + static_cast<int64_t>(sub) * T;
-      e = min(s + T, hi);
-    }
-  } else {
-    u -= a.idx_stride * a.tpb;
-    s = a.w_begin + static_cast<int64_t>(u) * T;
-    e = min(s + T, a.kv_end);
-  }
-  *ks = s;
-  *nk = e > s ? static_cast<int>(e - s) : 0;
-}
 
 // Loads this lane's 16 coordinates of one key row as packed fp32 pairs.
 template <bool BF16>
@@ -736,6 +703,7 @@ cudaError_t launch_sanitize_prefill_idx(const int32_t* idx, int32_t* out, int P,
 cudaError_t launch_decode_attn(const DecodeAttnArgs& a, const DecodePlan& p, bool bf16, bool out_bf16,
                                cudaStream_t s) {
   if (p.total_tiles == 0) return cudaSuccess;
+  if (bf16 && decode_tc_supported(a)) return launch_decode_tc(a, p, out_bf16, s);
   if (bf16) return out_bf16 ? launch_rg<true, true>(a, p, s) : launch_rg<true, false>(a, p, s);
   return out_bf16 ? launch_rg<false, true>(a, p, s) : launch_rg<false, false>(a, p, s);
 }

@@ -1,0 +1,691 @@
+// Step 4 for decode and draft chunks on the tensor cores (bf16 K, V and Q):
+// softmax attention over the retained keys only (S3R review, section
+// "稀疏起草": softmax over K_T and the weighted sum of V_T for the retained
+// index set T; PulseCol §3.1 eq. (1)-(2): logits q.k/sqrt(d_h), keys outside
+// the mask get zero weight).  The retained set, the work units (two 64-key
+// tiles of one (sequence, KV head) pair), their stream-K split over one CTA
+// per SM and the combine of partial results are those of decode_attn.cu.
+//
+// The keys of a unit sit on the MMA's M axis and the pair's <= 16 query rows
+// (n_q tokens x G heads) on its N axis:
+//   S^T  = K Q^T       tcgen05.mma M 128 keys x N 16 rows x K 128 (d), fp32 in TMEM
+//   P    = softmax     4 warps, one key per thread (TMEM lane = key); the row
+//                      max is exchanged through shared memory once per unit,
+//                      the running max is raised lazily (only when a row's
+//                      max grows by more than 2^8, which rescales O in TMEM)
+//   O^T += V^T P^T     tcgen05.mma M 128 (d) x N 16 rows x K 128 keys; V is
+//                      the MN-major operand straight from its TMA tile
+// Every K/V byte is thus read from shared memory by the tensor cores alone;
+// the CUDA cores do O(keys x rows) work per unit instead of O(keys x rows x d).
+//
+// CTA roles: warp 0 TMA producer (Q once per pair into a double buffer; K and
+// V as 64-row x 128-byte boxes, two d-halves per tile, into a 3-stage ring of
+// 64 KB units; rows at or past the end of the cache are zero-filled by the
+// tensor map), warp 1 TMEM owner and MMA issuer, warps 2-5 softmax and
+// epilogue.  TMEM columns: S in [0,16) / [16,32) by unit parity, O^T in
+// [32,48) / [48,64) by pair parity.  All waits are bounded.
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "decode_units.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kN = 16;                          // query rows per pair on the MMA N axis
+constexpr int kKVHalf = 16384;                  // one d-half of a unit: 128 keys x 128 B
+constexpr int kStage = 4 * kKVHalf;             // K (two d-halves) + V (two d-halves)
+constexpr int kNS = 3;                          // ring stages
+constexpr int kQBuf = 2 * kN * 128;             // two d-halves of 16 rows x 128 B
+constexpr int kPBuf = 2 * kN * 128;             // two key-halves of 16 rows x 128 B
+constexpr int kThreads = 192;
+constexpr int kSoftThreads = 128;
+constexpr int kNumBars = 22;
+constexpr uint32_t kIdescS = tc::idesc_bf16(128, kN, false, false);
+constexpr uint32_t kIdescO = tc::idesc_bf16(128, kN, true, false);
+constexpr float kLazy = 8.f;                    // raise the running max when it grows by > 2^8
+constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kNS) * kStage + 2 * kQBuf + 2 * kPBuf +
+                              kNumBars * 8 + kNS * sizeof(StageInfo) + (2 * 4 * kN + 4 * kN) * 4 + 32;
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float float_of_key(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+__device__ __forceinline__ void softmax_bar() {
+  asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const float (&v)[4]) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+// The first NR columns of this warp's 32 TMEM lanes.
+template <int NR>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, float (&v)[NR]) {
+  if constexpr (NR == 4) tmem_ld4(taddr, v);
+  else if constexpr (NR == 8) tmem_ld8(taddr, v);
+  else tmem_ld16(taddr, v);
+}
+template <int NR>
+__device__ __forceinline__ void tmem_stn(uint32_t taddr, const float (&v)[NR]) {
+  if constexpr (NR == 4) tmem_st4(taddr, v);
+  else if constexpr (NR == 8) tmem_st8(taddr, v);
+  else tmem_st16(taddr, v);
+}
+
+// Unit bookkeeping without divisions: the pair of unit i changes at
+// next_start, which advances by MT.
+struct PairCursor {
+  int next_start;   // first unit (CTA-local) of the following pair
+  int ordinal;      // pair ordinal of the current unit within this CTA
+  int MT;
+  __device__ void init(int64_t u0, int mt) {
+    MT = mt;
+    next_start = static_cast<int>((u0 / mt + 1) * mt - u0);
+    ordinal = 0;
+  }
+  // call with the unit index before using the flags of unit i (i ascending)
+  __device__ void at(int i) {
+    if (i == next_start) {
+      next_start += MT;
+      ++ordinal;
+    }
+  }
+  __device__ bool first(int i) const { return i == 0 || i == next_start - MT; }
+  __device__ bool last(int i, int nunits) const { return i == nunits - 1 || i + 1 == next_start; }
+};
+
+template <bool OUT_BF16>
+__device__ __forceinline__ void store_out(void* O, int64_t idx, float v) {
+  if constexpr (OUT_BF16) static_cast<__nv_bfloat16*>(O)[idx] = __float2bfloat16_rn(v);
+  else static_cast<float*>(O)[idx] = v;
+}
+
+template <bool OUT_BF16, int NR>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
+                     const __grid_constant__ CUtensorMap v_map, DecodeAttnArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* ring = smem;                                   // kNS x 64 KB
+  unsigned char* Qs = ring + kNS * kStage;                      // 2 x 4 KB
+  unsigned char* Ps = Qs + 2 * kQBuf;                           // 2 x 4 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Ps + 2 * kPBuf);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + 3;
+  uint64_t* q_full = bars + 6;
+  uint64_t* q_empty = bars + 8;
+  uint64_t* s_full = bars + 10;
+  uint64_t* s_free = bars + 12;
+  uint64_t* p_full = bars + 14;
+  uint64_t* p_free = bars + 16;
+  uint64_t* o_full = bars + 18;
+  uint64_t* o_free = bars + 20;
+  StageInfo* info = reinterpret_cast<StageInfo*>(bars + kNumBars);
+  float* wmax = reinterpret_cast<float*>(info + kNS);          // [2][16 rows][4 warps]
+  float* lsum = wmax + 2 * 4 * kN;                              // [16 rows][4 warps]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lsum + 4 * kN);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* ticket = reinterpret_cast<int*>(tmem_slot + 2);
+  uint64_t* mma_done = reinterpret_cast<uint64_t*>(tmem_slot + 4);    // 8-byte aligned
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t u0 = static_cast<int64_t>(blockIdx.x) * a.tpc;
+  const int64_t u1 = min(a.total_tiles, u0 + a.tpc);
+  const int nunits = static_cast<int>(u1 - u0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_empty[b], 1);
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], kSoftThreads);
+      mbar_init(&p_full[b], kSoftThreads);
+      mbar_init(&p_free[b], 1);
+      mbar_init(&o_full[b], 1);
+      mbar_init(&o_free[b], kSoftThreads);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // V rows of a partly filled unit keep whatever the buffer held; they meet
+  // zero probabilities, so they must be finite: zero the V halves, Q and P.
+  {
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int s = 0; s < kNS; ++s) {
+      uint4* v = reinterpret_cast<uint4*>(ring + s * kStage + 2 * kKVHalf);
+      for (int i = threadIdx.x; i < 2 * kKVHalf / 16; i += kThreads) v[i] = z;
+    }
+    uint4* qp = reinterpret_cast<uint4*>(Qs);
+    for (int i = threadIdx.x; i < (2 * kQBuf + 2 * kPBuf) / 16; i += kThreads) qp[i] = z;
+    tc::fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, 64);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tmem_slot;
+
+  auto fail = [&]() {
+    report(a.status, kStatusTimeout);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0) {
+    // -------------------------------------------------------- TMA producer
+    // the index table is written by the scoring kernel launched before this one
+    if (a.pdl) pdl_wait_prior_grid();
+    int issued = 0;
+    PairCursor pc;
+    pc.init(u0, a.MT);
+    int64_t pair = u0 / a.MT;
+    bool stop = false;
+    for (int base = 0; base < nunits && !stop; base += 32) {
+      int64_t ks0 = 0, ks1 = 0;
+      int nk0 = 0, nk1 = 0;
+      if (base + lane < nunits) {
+        const int64_t u = u0 + base + lane;
+        const int64_t pair = u / a.MT;
+        const int v = static_cast<int>(u - pair * a.MT);
+        tile_range(a, pair, 2 * v, &ks0, &nk0);
+        if (2 * v + 1 < a.n_tiles) tile_range(a, pair, 2 * v + 1, &ks1, &nk1);
+      }
+      const int cnt = min(32, nunits - base);
+      for (int l = 0; l < cnt; ++l) {
+        const int64_t k0 = __shfl_sync(0xffffffffu, ks0, l);
+        const int64_t k1 = __shfl_sync(0xffffffffu, ks1, l);
+        const int n0 = __shfl_sync(0xffffffffu, nk0, l);
+        const int n1 = __shfl_sync(0xffffffffu, nk1, l);
+        const int i = base + l;
+        const int s = i % kNS;
+        const int prev_ord = pc.ordinal;
+        pc.at(i);
+        if (pc.ordinal != prev_ord) ++pair;
+        const int pk = pc.ordinal;
+        int ok = 1;
+        if (lane == 0) {
+          if (pc.first(i)) {
+            const int qb = pk & 1;
+            if (pk >= 2 && !mbar_wait_bounded(&q_empty[qb], ((pk >> 1) + 1) & 1, abort_flag)) ok = 0;
+            if (ok) {
+              const int bi = static_cast<int>(pair / a.Hkv), h = static_cast<int>(pair % a.Hkv);
+              mbar_arrive_expect_tx(&q_full[qb], static_cast<uint32_t>(2 * a.R * 128));
+              tc::tma_load_3d(Qs + qb * kQBuf, &q_map, 0, h * a.G, bi * a.n_q, &q_full[qb]);
+              tc::tma_load_3d(Qs + qb * kQBuf + kN * 128, &q_map, 64, h * a.G, bi * a.n_q, &q_full[qb]);
+            }
+          }
+          if (ok && i >= kNS && !mbar_wait_bounded(&kv_empty[s], ((i / kNS) & 1) ^ 1, abort_flag)) ok = 0;
+          if (ok) {
+            info[s].ks0 = k0;
+            info[s].ks1 = k1;
+            info[s].n0 = n0;
+            info[s].n1 = n1;
+            const int t0 = n0 > 0, t1 = n1 > 0;
+            if (t0 + t1 > 0) {
+              unsigned char* st = ring + s * kStage;
+              const int p32 = static_cast<int>(pair);
+              mbar_arrive_expect_tx(&kv_full[s], static_cast<uint32_t>((t0 + t1) * 4 * 8192));
+              if (t0) {
+                const int r0 = static_cast<int>(k0);
+                tc::tma_load_3d(st, &k_map, 0, r0, p32, &kv_full[s]);
+                tc::tma_load_3d(st + kKVHalf, &k_map, 64, r0, p32, &kv_full[s]);
+                tc::tma_load_3d(st + 2 * kKVHalf, &v_map, 0, r0, p32, &kv_full[s]);
+                tc::tma_load_3d(st + 3 * kKVHalf, &v_map, 64, r0, p32, &kv_full[s]);
+              }
+              if (t1) {
+                const int r1 = static_cast<int>(k1);
+                tc::tma_load_3d(st + 8192, &k_map, 0, r1, p32, &kv_full[s]);
+                tc::tma_load_3d(st + kKVHalf + 8192, &k_map, 64, r1, p32, &kv_full[s]);
+                tc::tma_load_3d(st + 2 * kKVHalf + 8192, &v_map, 0, r1, p32, &kv_full[s]);
+                tc::tma_load_3d(st + 3 * kKVHalf + 8192, &v_map, 64, r1, p32, &kv_full[s]);
+              }
+            } else {
+              mbar_arrive(&kv_full[s]);
+            }
+          } else {
+            fail();
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          stop = true;
+          break;
+        }
+        issued = i + 1;
+      }
+    }
+    // do not leave while copies into this CTA's shared memory may be in flight
+    if (lane == 0) {
+      for (int i = max(0, issued - kNS); i < issued; ++i) mbar_wait_bounded(&kv_full[i % kNS], (i / kNS) & 1, nullptr);
+      for (int k = max(0, pc.ordinal - 1); k <= pc.ordinal; ++k)
+        if (issued > 0) mbar_wait_bounded(&q_full[k & 1], (k >> 1) & 1, nullptr);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    // S(i) needs unit i's K and Q and a free S buffer; PV(i) needs P(i).  The
+    // thread polls both and issues whichever is ready, so a unit's ring stage
+    // (released when PV(i) completes) never waits for the next unit's data.
+    if (lane == 0) {
+      const uint32_t ring_a = smem_u32(ring), qa = smem_u32(Qs), pa = smem_u32(Ps);
+      int ns = 0, npv = 0;                  // next S / PV to issue
+      PairCursor cs, cp;                    // pair bookkeeping of units ns / npv
+      cs.init(u0, a.MT);
+      cp.init(u0, a.MT);
+      bool ok = true;
+      uint64_t t0 = global_ns();
+      for (uint32_t spin = 0; npv < nunits; ++spin) {
+        bool did = false;
+        if (ns < nunits) {
+          const bool fi = cs.first(ns);
+          const int pk = cs.ordinal, qb = pk & 1, s = ns % kNS;
+          if (mbar_test_wait(&kv_full[s], (ns / kNS) & 1) &&
+              (!fi || mbar_test_wait(&q_full[qb], (pk >> 1) & 1)) &&
+              (ns < 2 || mbar_test_wait(&s_free[ns & 1], ((ns >> 1) + 1) & 1))) {
+            tc::fence_after_sync();
+            const uint32_t kst = ring_a + s * kStage, qst = qa + qb * kQBuf;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              tc::mma_bf16(tbase + (ns & 1) * kN,
+                           tc::smem_desc(kst + (kk >> 2) * kKVHalf + (kk & 3) * 32, 16, 1024),
+                           tc::smem_desc(qst + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024), kIdescS, kk > 0);
+            tc::mma_commit(&s_full[ns & 1]);
+            // no later MMA reads this Q buffer for this pair
+            if (cs.last(ns, nunits)) tc::mma_commit(&q_empty[qb]);
+            ++ns;
+            cs.at(ns);
+            did = true;
+          }
+        }
+        if (npv < ns) {
+          const bool fi = cp.first(npv);
+          const int pk = cp.ordinal, ob = pk & 1;
+          if (mbar_test_wait(&p_full[npv & 1], (npv >> 1) & 1) &&
+              (!fi || pk < 2 || mbar_test_wait(&o_free[ob], ((pk >> 1) + 1) & 1))) {
+            tc::fence_after_sync();
+            const uint32_t vst = ring_a + (npv % kNS) * kStage + 2 * kKVHalf;
+            const uint32_t pb = pa + (npv & 1) * kPBuf;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              tc::mma_bf16(tbase + 32 + ob * kN, tc::smem_desc(vst + kk * 2048, kKVHalf, 1024),
+                           tc::smem_desc(pb + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024), kIdescO,
+                           !(fi && kk == 0));
+            tc::mma_commit(&kv_empty[npv % kNS]);
+            tc::mma_commit(&p_free[npv & 1]);
+            if (cp.last(npv, nunits)) tc::mma_commit(&o_full[ob]);
+            ++npv;
+            cp.at(npv);
+            did = true;
+          }
+        }
+        if (did) {
+          t0 = global_ns();
+        } else if ((spin & 63u) == 0) {
+          if (*abort_flag || global_ns() - t0 > kWaitLimitNs) {
+            ok = false;
+            break;
+          }
+        }
+      }
+      if (!ok) fail();
+      // every MMA must be complete before TMEM is released
+      tc::mma_commit(mma_done);
+      mbar_wait_bounded(mma_done, 0, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------- softmax and epilogue
+    const int qq = warp & 3;                  // TMEM lane quarter of this warp
+    const int t = qq * 32 + lane;             // key slot of the unit; output column d in the epilogue
+    const uint32_t tl = tbase + (static_cast<uint32_t>(qq * 32) << 16);
+    const int R = a.R, G = a.G;
+    const int C = static_cast<int>(a.C);
+    const float qscale = a.qscale;
+    const int tile = t >> 6, kc = t & 63;
+    // byte offsets of this key's P^T entries (row r, key kc of its 64-key half)
+    uint32_t poff[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) poff[r] = tile * (kN * 128) + tc::sw128_off(r, kc >> 3) + (kc & 7) * 2;
+    float m_run[NR], l_t[NR];
+    PairCursor pc;
+    pc.init(u0, a.MT);
+    int64_t pair = u0 / a.MT;
+    bool ok = true;
+
+    auto epilogue = [&]() -> bool {
+      // row sums over the unit's 128 key slots
+      float mine = 0.f;
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        float v = l_t[r];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        mine = (lane == r) ? v : mine;
+      }
+      if (lane < NR) lsum[lane * 4 + qq] = mine;
+      const int pkk = pc.ordinal, ob = pkk & 1;
+      if (!mbar_wait_bounded(&o_full[ob], (pkk >> 1) & 1, abort_flag)) return false;
+      tc::fence_after_sync();
+      float ov[NR];
+      tmem_ldn<NR>(tl + 32 + ob * kN, ov);
+      tc::tmem_wait_ld();
+      tc::fence_before_sync();
+      mbar_arrive(&o_free[ob]);
+      softmax_bar();
+      float L[NR];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        const float4 v = reinterpret_cast<const float4*>(lsum)[r];
+        L[r] = (v.x + v.y) + (v.z + v.w);
+      }
+      const int64_t first = pair * a.MT, last = first + a.MT - 1;
+      const bool whole = first >= u0 && last < u1;
+      const int64_t first_cta = first / a.tpc, last_cta = last / a.tpc;
+      const int n_ctas = static_cast<int>(last_cta - first_cta + 1);
+      const int slot = static_cast<int>(blockIdx.x - first_cta);
+      const int bi = static_cast<int>(pair / a.Hkv), h = static_cast<int>(pair % a.Hkv);
+      auto out_row = [&](int r) -> int64_t {
+        const int j = r / G, g = r - (r / G) * G;
+        return (static_cast<int64_t>(bi) * a.n_q + j) * a.Hq + h * G + g;
+      };
+      if (whole) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          if (r < R) {
+            const int64_t orow = out_row(r);
+            store_out<OUT_BF16>(a.O, orow * kHeadDim + t, ov[r] * (L[r] > 0.f ? 1.f / L[r] : 0.f));
+            if (t == r && a.lse)
+              a.lse[orow] = L[r] > 0.f ? (m_run[r] + log2f(L[r])) * 0.69314718055994531f : -CUDART_INF_F;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          if (r < R) {
+            const int64_t ps = (pair * a.n_slots + slot) * a.R4 + r;
+            a.part_O[ps * kHeadDim + t] = ov[r];
+            if (t == r) {
+              a.part_ml[ps * 2 + 0] = m_run[r];
+              a.part_ml[ps * 2 + 1] = L[r];
+            }
+          }
+        }
+        // the barrier orders every thread's partial stores before thread 0's
+        // release fence and ticket
+        softmax_bar();
+        if (t == 0) {
+          __threadfence();
+          const unsigned tk = atomicAdd(&a.counters[pair], 1u);
+          *ticket = (tk == static_cast<unsigned>(n_ctas - 1));
+        }
+        softmax_bar();
+        if (*ticket) {
+          __threadfence();
+          for (int r = 0; r < R; ++r) {
+            float M = -CUDART_INF_F;
+            for (int s2 = 0; s2 < n_ctas; ++s2)
+              M = fmaxf(M, __ldcg(a.part_ml + ((pair * a.n_slots + s2) * a.R4 + r) * 2));
+            const float Mr = (M == -CUDART_INF_F) ? 0.f : M;
+            float Ls = 0.f, acc = 0.f;
+            for (int s2 = 0; s2 < n_ctas; ++s2) {
+              const int64_t ps = (pair * a.n_slots + s2) * a.R4 + r;
+              const float sc = exp2f(__ldcg(a.part_ml + ps * 2) - Mr);
+              Ls += __ldcg(a.part_ml + ps * 2 + 1) * sc;
+              acc += __ldcg(a.part_O + ps * kHeadDim + t) * sc;
+            }
+            const int64_t orow = out_row(r);
+            store_out<OUT_BF16>(a.O, orow * kHeadDim + t, acc * (Ls > 0.f ? 1.f / Ls : 0.f));
+            if (t == 0 && a.lse)
+              a.lse[orow] = Ls > 0.f ? (Mr + log2f(Ls)) * 0.69314718055994531f : -CUDART_INF_F;
+          }
+          if (t == 0) a.counters[pair] = 0u;
+        }
+      }
+      softmax_bar();     // lsum and the ticket are reused by the next pair
+      return true;
+    };
+
+    for (int i = 0; i < nunits && ok; ++i) {
+      const int prev_ord = pc.ordinal;
+      pc.at(i);
+      if (pc.ordinal != prev_ord) ++pair;
+      const bool fi = pc.first(i);
+      if (fi) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          m_run[r] = -CUDART_INF_F;
+          l_t[r] = 0.f;
+        }
+      }
+      const int s = i % kNS, sb = i & 1;
+      if (!mbar_wait_bounded(&s_full[sb], (i >> 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      float sv[NR];
+      tmem_ldn<NR>(tl + sb * kN, sv);
+      tc::tmem_wait_ld();
+      tc::fence_before_sync();
+      mbar_arrive(&s_free[sb]);
+      // the unit's key ranges, published with the stage's full barrier
+      if (!mbar_wait_bounded(&kv_full[s], (i / kNS) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const int n = tile ? info[s].n1 : info[s].n0;
+      const int dnew = static_cast<int>(tile ? info[s].ks1 : info[s].ks0) + kc - C;   // >= 0: a new key
+      const int dn = dnew < 0 ? -1 : min(dnew, 64);
+      const bool kv = kc < n;
+      float x[NR];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        // new key C + dnew is seen by token r / G iff dnew <= r / G, i.e. dnew * G <= r
+        const bool v = kv && r < R && (dn < 0 || dn * G <= r);
+        x[r] = v ? sv[r] * qscale : -CUDART_INF_F;
+      }
+      // unit max of every row: warp reduction, then the four warps through
+      // shared memory (row r of this warp stored by lane r)
+      float* wm = wmax + sb * (kN * 4);
+      uint32_t mk = 0u;
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        const uint32_t k = __reduce_max_sync(0xffffffffu, float_key(x[r]));
+        mk = (lane == r) ? k : mk;
+      }
+      if (lane < NR) wm[lane * 4 + qq] = float_of_key(mk);
+      softmax_bar();
+      float alpha[NR];
+      bool grow_any = false;
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        const float4 w4 = reinterpret_cast<const float4*>(wm)[r];
+        const float M = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
+        const bool grow = M > m_run[r] + kLazy;
+        alpha[r] = grow ? ex2(m_run[r] - M) : 1.f;     // 0 for the first keys of a row
+        m_run[r] = grow ? M : m_run[r];
+        grow_any |= grow;
+      }
+      if (grow_any) {
+        if (!fi) {
+          // O^T holds earlier units of this pair: wait for PV(i-1), rescale
+          const int pj = i - 1;
+          if (!mbar_wait_bounded(&p_free[pj & 1], (pj >> 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          float ov[NR];
+          const uint32_t to = tl + 32 + (pc.ordinal & 1) * kN;
+          tmem_ldn<NR>(to, ov);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int r = 0; r < NR; ++r) ov[r] *= alpha[r];
+          tmem_stn<NR>(to, ov);
+          tc::tmem_wait_st();
+          tc::fence_before_sync();
+        }
+#pragma unroll
+        for (int r = 0; r < NR; ++r) l_t[r] *= alpha[r];
+      }
+      // P^T into this unit's P buffer once PV(i-2) has read it
+      if (i >= 2 && !mbar_wait_bounded(&p_free[sb], ((i >> 1) + 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      unsigned char* pbuf = Ps + sb * kPBuf;
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        const float p = ex2(x[r] - (m_run[r] == -CUDART_INF_F ? 0.f : m_run[r]));
+        l_t[r] += p;
+        *reinterpret_cast<__nv_bfloat16*>(pbuf + poff[r]) = __float2bfloat16_rn(p);
+      }
+      tc::fence_proxy_async_smem();
+      mbar_arrive(&p_full[sb]);
+      if (pc.last(i, nunits) && !epilogue()) {
+        ok = false;
+        break;
+      }
+    }
+    if (!ok && lane == 0) fail();
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, 64);
+  }
+}
+
+using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+size_t decode_tc_smem_bytes() { return kSmemBytes; }
+
+bool decode_tc_supported(const DecodeAttnArgs& a) {
+  return a.R >= 1 && a.R <= kN && a.kv_end < (int64_t(1) << 31) &&
+         static_cast<int64_t>(a.B) * a.n_q < (int64_t(1) << 31) && encode_fn() != nullptr;
+}
+
+cudaError_t launch_decode_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf16, cudaStream_t s) {
+  EncodeFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUtensorMap qm, km, vm;
+  {
+    // Q [B * n_q tokens][Hq heads][128]: box 64 columns x G heads x n_q tokens
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(a.Hq), static_cast<cuuint64_t>(a.B) * a.n_q};
+    cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(a.Hq) * 256};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(a.G), static_cast<cuuint32_t>(a.n_q)};
+    if (enc(&qm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.Q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    // K, V [pairs][cap keys][128], rows at or past kv_end read as zeros: box 64 columns x 64 keys
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(a.kv_end), static_cast<cuuint64_t>(a.B) * a.Hkv};
+    cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(a.cap) * 256};
+    cuuint32_t box[3] = {64, 64, 1};
+    if (enc(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.K), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    if (enc(&vm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.V), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, DecodeAttnArgs);
+  if (a.R <= 4) kern = out_bf16 ? decode_tc_kernel<true, 4> : decode_tc_kernel<false, 4>;
+  else if (a.R <= 8) kern = out_bf16 ? decode_tc_kernel<true, 8> : decode_tc_kernel<false, 8>;
+  else kern = out_bf16 ? decode_tc_kernel<true, 16> : decode_tc_kernel<false, 16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, qm, km, vm, a);
+}
+
+}  // namespace sa

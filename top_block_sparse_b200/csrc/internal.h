@@ -36,9 +36,10 @@ cudaError_t launch_pool(const PoolArgs& a, bool bf16, cudaStream_t s);
 struct ScoreArgs {
   const void* Q;
   const float* Kc;
-  float* scores;          // [pairs, nb]
+  float* scores;          // [pairs, nb]; may be null when chunks == 1
   int32_t* idx;           // [pairs, top_k]
   unsigned* counters;     // [pairs], zero between calls
+  unsigned* status;       // workspace status word
   int B, Hq, Hkv, G, n_q;
   int64_t nb;
   int b;
@@ -47,9 +48,9 @@ struct ScoreArgs {
   float scale;            // softmax scale (mean pooling)
   int lsa;                // cosine scores
   int chunks;             // CTAs per pair
-  int blocks_per_chunk;
+  int64_t rows_per_chunk; // a multiple of kScoreRowsPerPass
 };
-constexpr int kScoreBlocksPerChunk = 128;
+constexpr int kScoreRowsPerPass = 64;
 constexpr int64_t kMaxSelectBlocks = 16384;
 cudaError_t launch_score_topk_query0(const ScoreArgs& a, bool bf16, cudaStream_t s);
 
@@ -95,6 +96,11 @@ bool plan_decode(const DecodeGeom& g, int idx_slots, bool bf16, int num_sms, Dec
                  const char** why);
 cudaError_t launch_decode_attn(const DecodeAttnArgs& a, const DecodePlan& p, bool bf16,
                                bool out_bf16, cudaStream_t s);
+// Tensor-core variant for bf16 inputs (decode_tc.cu); launch_decode_attn
+// picks it whenever decode_tc_supported() holds.
+bool decode_tc_supported(const DecodeAttnArgs& a);
+size_t decode_tc_smem_bytes();
+cudaError_t launch_decode_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf16, cudaStream_t s);
 // Copies a caller's [rows, len] index table to `out`, keeping only entries
 // that are in [0, nb) and above every earlier in-range entry of the row.
 cudaError_t launch_sanitize_idx(const int32_t* idx, int32_t* out, int rows, int len, int64_t nb,

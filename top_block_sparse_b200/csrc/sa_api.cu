@@ -1,6 +1,7 @@
 // C ABI of libsa.so: argument validation, workspace layout, launch planning.
 // Every entry point validates on the host before launching anything and
 // never allocates memory; see include/sa.h for the contract.
+#include <algorithm>
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
@@ -144,14 +145,18 @@ sa_status plan_for(const sa_params* p, int idx_slots, DecodeGeom* g, DecodePlan*
   return SA_OK;
 }
 
+// caller_scores may be null; the workspace receives the scores when a pair
+// is split over several CTAs.
 ScoreArgs score_args(const sa_params* p, const DecodeGeom& g, const void* Q, const float* Kc,
-                     float* scores, int32_t* idx, unsigned* counters) {
+                     float* caller_scores, int32_t* idx, unsigned char* ws, const DecodeWs& L) {
+  float* ws_scores = reinterpret_cast<float*>(ws + L.scores);
+  unsigned* counters = reinterpret_cast<unsigned*>(ws + L.score_cnt);
   ScoreArgs a = {};
   a.Q = Q;
   a.Kc = Kc;
-  a.scores = scores;
   a.idx = idx;
   a.counters = counters;
+  a.status = reinterpret_cast<unsigned*>(ws);
   a.B = g.B;
   a.Hq = g.Hq;
   a.Hkv = g.Hkv;
@@ -164,9 +169,14 @@ ScoreArgs score_args(const sa_params* p, const DecodeGeom& g, const void* Q, con
   a.top_k = p->top_k;
   a.scale = scale_of(p);
   a.lsa = p->pool == SA_POOL_LSA;
-  a.blocks_per_chunk = kScoreBlocksPerChunk;
-  a.chunks = static_cast<int>((g.nb + kScoreBlocksPerChunk - 1) / kScoreBlocksPerChunk);
-  if (a.chunks < 1) a.chunks = 1;
+  // as many chunks per pair as keep every CTA resident (two per SM)
+  const int64_t pairs = std::max<int64_t>(1, g.pairs);
+  const int64_t passes = std::max<int64_t>(1, (g.nb + kScoreRowsPerPass - 1) / kScoreRowsPerPass);
+  const int64_t want = std::min<int64_t>(passes, std::max<int64_t>(1, 2 * device_sms() / pairs));
+  const int64_t per = (passes + want - 1) / want;
+  a.rows_per_chunk = per * kScoreRowsPerPass;
+  a.chunks = static_cast<int>((passes + per - 1) / per);
+  a.scores = caller_scores ? caller_scores : (a.chunks > 1 ? ws_scores : nullptr);
   return a;
 }
 
@@ -388,8 +398,7 @@ sa_status sa_score_topk(const sa_params* p, const void* Q, const float* Kc, int3
   const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_SCORE_TOPK);
   if ((st = check_ws(ws, ws_bytes, L.total)) != SA_OK) return st;
   unsigned char* w = static_cast<unsigned char*>(ws);
-  float* sc = scores ? scores : reinterpret_cast<float*>(w + L.scores);
-  ScoreArgs a = score_args(p, g, Q, Kc, sc, idx, reinterpret_cast<unsigned*>(w + L.score_cnt));
+  ScoreArgs a = score_args(p, g, Q, Kc, scores, idx, w, L);
   cudaError_t e = launch_score_topk_query0(a, p->dtype == SA_BF16, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "score/top-k kernel launch");
   return SA_OK;
@@ -474,8 +483,7 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q, const void* K
   unsigned char* w = static_cast<unsigned char*>(ws);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + L.idx);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  ScoreArgs sa_ = score_args(p, g, Q, Kc, reinterpret_cast<float*>(w + L.scores), idx,
-                             reinterpret_cast<unsigned*>(w + L.score_cnt));
+  ScoreArgs sa_ = score_args(p, g, Q, Kc, nullptr, idx, w, L);
   cudaError_t e = launch_score_topk_query0(sa_, p->dtype == SA_BF16, s);
   if (e != cudaSuccess) return cuda_fail(e, "score/top-k kernel launch");
   DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, idx, p->top_k, O, lse, w, L);

@@ -10,10 +10,15 @@
 // Selection: the k largest by (score desc, block id asc), written in
 // ascending block order, -1 padded.
 //
-// Grid (chunks, pairs): every CTA streams a chunk of one pair's compressed
-// keys (fp32, 128-bit loads, a warp per row with a shuffle reduction) and
-// writes scores; the CTA that finishes last for a pair (atomic ticket, no
-// waiting) runs the radix select over the pair's scores.
+// Grid (chunks, pairs), every CTA resident at once (2 per SM): each CTA
+// streams a contiguous chunk of one pair's compressed keys (fp32 rows of 512
+// bytes) through a 3-stage shared-memory ring of 64-row stages filled by
+// cp.async.bulk (the TMA engine keeps far more bytes in flight per SM than
+// per-thread loads); a warp scores 8 rows of a stage with a shuffle reduction
+// per row.  With one chunk per pair the CTA builds the selection keys in
+// shared memory and selects; with several, CTAs write scores and the CTA that
+// finishes last for the pair (atomic ticket, no waiting) reads them back and
+// selects.
 #include <math_constants.h>
 
 #include "common.cuh"
@@ -25,36 +30,65 @@ namespace {
 
 constexpr int kScoreThreads = 256;
 constexpr int kScoreWarps = kScoreThreads / 32;
+constexpr int kStageRows = kScoreRowsPerPass;                 // 64 rows = 32 KB
+constexpr int kStageBytes = kStageRows * kHeadDim * 4;
+constexpr int kScoreStages = 3;
+constexpr int kRowsPerWarp = kStageRows / kScoreWarps;        // 8
+constexpr size_t kRingBytes = static_cast<size_t>(kScoreStages) * kStageBytes;
+
+__device__ __forceinline__ uint32_t block_key(const ScoreArgs& a, int64_t j, float s) {
+  const int64_t lo = j * a.b, hi = lo + a.b;
+  const bool cand = (lo < a.w_begin) && (hi > a.s_end);
+  const uint32_t key = float_key(s);
+  return cand ? (key == 0u ? 1u : key) : 0u;
+}
 
 template <bool BF16>
-__global__ void __launch_bounds__(kScoreThreads) score_topk_query0_kernel(ScoreArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw);                        // [nb] (last CTA)
+__global__ void __launch_bounds__(kScoreThreads, 2) score_topk_query0_kernel(ScoreArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  unsigned char* ring = smem_raw;                                           // kScoreStages x 32 KB
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kRingBytes);     // [nb] (selecting CTA)
+  __shared__ uint64_t full[kScoreStages];
   __shared__ __align__(16) float qs[kHeadDim];
-  __shared__ unsigned hist[256];
-  __shared__ unsigned scratch[4];
+  __shared__ unsigned red[2 * kScoreWarps];
+  __shared__ float qinv;
   __shared__ int is_last;
+  __shared__ volatile int abort_flag;
+
+  // the attention kernel launched after this one may take SMs as they drain
+  pdl_launch_dependents();
 
   const int pair = blockIdx.y;
   const int chunk = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bi = pair / a.Hkv, h = pair % a.Hkv;
+  const bool single = a.chunks == 1;
 
-  static_assert(kScoreBlocksPerChunk % kScoreWarps == 0 && kScoreBlocksPerChunk / kScoreWarps <= 32,
-                "rows per warp");
-  const int64_t j_begin = static_cast<int64_t>(chunk) * a.blocks_per_chunk;
-  const int64_t j_end = min(a.nb, j_begin + a.blocks_per_chunk);
-  const float* kc = a.Kc + static_cast<int64_t>(pair) * a.nb * kHeadDim;
-  float* sc = a.scores + static_cast<int64_t>(pair) * a.nb;
-  // every warp streams kRowsPerWarp rows; their loads are issued first, before
-  // the index query is formed, so the two latencies overlap
-  constexpr int kRowsPerWarp = kScoreBlocksPerChunk / kScoreWarps;
-  const int64_t jw = j_begin + static_cast<int64_t>(warp) * kRowsPerWarp;
-  float4 r[kRowsPerWarp];
-#pragma unroll
-  for (int u = 0; u < kRowsPerWarp; ++u)
-    r[u] = (jw + u < j_end) ? __ldcs(reinterpret_cast<const float4*>(kc + (jw + u) * kHeadDim) + lane)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+  const int64_t j_begin = min(a.nb, static_cast<int64_t>(chunk) * a.rows_per_chunk);
+  const int64_t j_end = min(a.nb, j_begin + a.rows_per_chunk);
+  const int nrows = static_cast<int>(j_end - j_begin);
+  const int nst = (nrows + kStageRows - 1) / kStageRows;
+  const float* kc = a.Kc + (static_cast<int64_t>(pair) * a.nb + j_begin) * kHeadDim;
+  float* sc = a.scores ? a.scores + static_cast<int64_t>(pair) * a.nb : nullptr;
+
+  if (tid == 0) {
+    for (int s = 0; s < kScoreStages; ++s) mbar_init(&full[s], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](int st) {
+    const int s = st % kScoreStages;
+    const int rows = min(kStageRows, nrows - st * kStageRows);
+    const uint32_t bytes = static_cast<uint32_t>(rows) * kHeadDim * 4;
+    mbar_arrive_expect_tx(&full[s], bytes);
+    bulk_g2s(ring + static_cast<size_t>(s) * kStageBytes, kc + static_cast<int64_t>(st) * kStageRows * kHeadDim,
+             bytes, &full[s]);
+  };
+  // the first stages are requested before the index query is formed, so the
+  // two latencies overlap
+  if (tid == 0)
+    for (int st = 0; st < min(kScoreStages, nst); ++st) issue(st);
   // index query of the first new token: sum over the GQA group
   if (tid < kHeadDim) {
     float s = 0.f;
@@ -72,66 +106,85 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_query0_kernel(ScoreA
       for (int i = lane; i < kHeadDim; i += 32) ss += qs[i] * qs[i];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      if (lane == 0) scratch[0] = __float_as_uint(ss > 0.f ? rsqrtf(ss) : 0.f);
+      if (lane == 0) qinv = ss > 0.f ? rsqrtf(ss) : 0.f;
     }
     __syncthreads();
-    const float inv = __uint_as_float(scratch[0]);
-    __syncthreads();
-    if (tid < kHeadDim) qs[tid] *= inv;
-  } else {
-    if (tid < kHeadDim) qs[tid] *= a.scale;
   }
-  __syncthreads();
+  const float qmul = a.lsa ? qinv : a.scale;
+  float4 q4 = reinterpret_cast<const float4*>(qs)[lane];
+  q4.x *= qmul;
+  q4.y *= qmul;
+  q4.z *= qmul;
+  q4.w *= qmul;
 
-  const float4 q4 = reinterpret_cast<const float4*>(qs)[lane];
-  float d[kRowsPerWarp];
+  bool aborted = false;
+  for (int st = 0; st < nst; ++st) {
+    const int s = st % kScoreStages;
+    const bool ok = mbar_wait_bounded(&full[s], (st / kScoreStages) & 1, &abort_flag);
+    if (ok) {
+      const float* rows = reinterpret_cast<const float*>(ring + static_cast<size_t>(s) * kStageBytes);
+      const int r0 = warp * kRowsPerWarp;
+      float d[kRowsPerWarp];
 #pragma unroll
-  for (int u = 0; u < kRowsPerWarp; ++u) d[u] = r[u].x * q4.x + r[u].y * q4.y + r[u].z * q4.z + r[u].w * q4.w;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-    for (int u = 0; u < kRowsPerWarp; ++u) d[u] += __shfl_xor_sync(0xffffffffu, d[u], o);
-  }
-  float mine = d[0];
-#pragma unroll
-  for (int u = 1; u < kRowsPerWarp; ++u) mine = (lane == u) ? d[u] : mine;
-  if (lane < kRowsPerWarp && jw + lane < j_end) sc[jw + lane] = mine;
-
-  // ticket: the last CTA of this pair selects (one warp; the others leave).
-  // The barrier orders the CTA's score stores before thread 0's release fence.
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const unsigned t = atomicAdd(&a.counters[pair], 1u);
-    is_last = (t == static_cast<unsigned>(a.chunks - 1));
-  }
-  __syncthreads();
-  if (!is_last || warp != 0) return;
-  __threadfence();
-  if (lane == 0) a.counters[pair] = 0u;
-
-  const int nb = static_cast<int>(a.nb);
-  // the pair's scores come from L2; keep 8 loads per lane in flight
-  for (int j0 = 0; j0 < nb; j0 += 8 * 32) {
-    float v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j = j0 + u * 32 + lane;
-      v[u] = j < nb ? __ldcg(sc + j) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j = j0 + u * 32 + lane;
-      if (j < nb) {
-        const int64_t lo = static_cast<int64_t>(j) * a.b, hi = lo + a.b;
-        const bool cand = (lo < a.w_begin) && (hi > a.s_end);
-        const uint32_t key = float_key(v[u]);
-        keys[j] = cand ? (key == 0u ? 1u : key) : 0u;
+      for (int u = 0; u < kRowsPerWarp; ++u) {
+        const float4 r = reinterpret_cast<const float4*>(rows + (r0 + u) * kHeadDim)[lane];
+        d[u] = r.x * q4.x + r.y * q4.y + r.z * q4.z + r.w * q4.w;
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+        for (int u = 0; u < kRowsPerWarp; ++u) d[u] += __shfl_xor_sync(0xffffffffu, d[u], o);
+      }
+      float mine = d[0];
+#pragma unroll
+      for (int u = 1; u < kRowsPerWarp; ++u) mine = (lane == u) ? d[u] : mine;
+      const int64_t j = j_begin + static_cast<int64_t>(st) * kStageRows + r0 + lane;
+      if (lane < kRowsPerWarp && j < j_end) {
+        if (sc) sc[j] = mine;
+        if (single) keys[j] = block_key(a, j, mine);
+      }
+    } else if (lane == 0) {
+      report(a.status, kStatusTimeout);
+      abort_flag = 1;
     }
+    // every warp is done with stage s before it is refilled
+    if (__syncthreads_or(!ok)) {
+      aborted = true;
+      break;
+    }
+    if (tid == 0 && st + kScoreStages < nst) issue(st + kScoreStages);
   }
-  __syncwarp();
-  warp_topk(keys, nb, a.top_k, a.idx + static_cast<int64_t>(pair) * a.top_k);
+  if (aborted) {
+    // do not leave while copies into this CTA's shared memory may be in flight
+    if (tid == 0)
+      for (int st = 0; st < nst; ++st) mbar_wait_bounded(&full[st % kScoreStages], (st / kScoreStages) & 1, nullptr);
+    return;
+  }
+
+  if (!single) {
+    // ticket: the last CTA of this pair selects.  The barrier orders the
+    // CTA's score stores before thread 0's release fence.
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      const unsigned t = atomicAdd(&a.counters[pair], 1u);
+      is_last = (t == static_cast<unsigned>(a.chunks - 1));
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    if (tid == 0) a.counters[pair] = 0u;
+    // the pair's scores come back from L2
+    for (int64_t j = tid; j < a.nb; j += kScoreThreads) keys[j] = block_key(a, j, __ldcg(sc + j));
+  }
+  __syncthreads();
+  const int nb = static_cast<int>(a.nb);
+  int32_t* out = a.idx + static_cast<int64_t>(pair) * a.top_k;
+  if (nb <= 2048) {
+    if (warp == 0) warp_topk(keys, nb, a.top_k, out);
+  } else {
+    block_topk<kScoreThreads, kMaxSelectBlocks / kScoreThreads>(keys, nb, a.top_k, out, red);
+  }
 }
 
 }  // namespace
@@ -139,7 +192,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_query0_kernel(ScoreA
 cudaError_t launch_score_topk_query0(const ScoreArgs& a, bool bf16, cudaStream_t s) {
   if (a.B * a.Hkv == 0) return cudaSuccess;
   dim3 grid(a.chunks, a.B * a.Hkv), blk(kScoreThreads);
-  const size_t smem = align_up(static_cast<size_t>(a.nb) * 4, 16);
+  const size_t smem = kRingBytes + align_up(static_cast<size_t>(a.nb) * 4, 16);
   cudaError_t e;
   if (bf16) {
     e = cudaFuncSetAttribute(score_topk_query0_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -78,12 +78,164 @@ __device__ inline void warp_topk_bits(const uint32_t* keys, int nb, int k, int32
   for (int s = static_cast<int>(keff) + lane; s < k; s += 32) out[s] = -1;
 }
 
-// Dispatch on the number of keys per lane; nb <= 2048.
+// The same selection for any nb, by one warp, with the keys left in shared
+// memory (every step of the search re-reads them).
+__device__ inline void warp_topk_smem(const uint32_t* keys, int nb, int k, int32_t* out) {
+  const int lane = threadIdx.x & 31;
+  unsigned nc = 0;
+  for (int j = lane; j < nb; j += 32) nc += keys[j] != 0u;
+  nc = __reduce_add_sync(0xffffffffu, nc);
+  const unsigned keff = nc < static_cast<unsigned>(k) ? nc : static_cast<unsigned>(k);
+  uint32_t tau = 0xffffffffu;
+  unsigned need = 0;
+  if (keff > 0u) {
+    uint32_t prefix = 0u;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = prefix | (1u << bit);
+      unsigned c = 0;
+#pragma unroll 4
+      for (int j = lane; j < nb; j += 32) c += keys[j] >= cand;
+      if (__reduce_add_sync(0xffffffffu, c) >= keff) prefix = cand;
+    }
+    tau = prefix;
+    unsigned gt = 0;
+    for (int j = lane; j < nb; j += 32) gt += keys[j] > tau;
+    need = keff - __reduce_add_sync(0xffffffffu, gt);
+  }
+  const unsigned lt_mask = (1u << lane) - 1u;
+  unsigned base = 0, eq_base = 0;
+  if (keff > 0u) {
+    for (int j0 = 0; j0 < nb; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t key = j < nb ? keys[j] : 0u;
+      const bool eq = key == tau;
+      const unsigned b_eq = __ballot_sync(0xffffffffu, eq);
+      const bool take_eq = eq && (eq_base + __popc(b_eq & lt_mask)) < need;
+      eq_base += __popc(b_eq);
+      const bool sel = (key > tau) || take_eq;
+      const unsigned b = __ballot_sync(0xffffffffu, sel);
+      if (sel) out[base + __popc(b & lt_mask)] = j;
+      base += __popc(b);
+    }
+  }
+  for (int s = static_cast<int>(keff) + lane; s < k; s += 32) out[s] = -1;
+}
+
+// Dispatch on the number of keys per lane: registers up to 2048 keys, shared
+// memory beyond.
 __device__ inline void warp_topk(const uint32_t* keys, int nb, int k, int32_t* out) {
   if (nb <= 256) warp_topk_bits<8>(keys, nb, k, out);
   else if (nb <= 512) warp_topk_bits<16>(keys, nb, k, out);
   else if (nb <= 1024) warp_topk_bits<32>(keys, nb, k, out);
-  else warp_topk_bits<64>(keys, nb, k, out);
+  else if (nb <= 2048) warp_topk_bits<64>(keys, nb, k, out);
+  else warp_topk_smem(keys, nb, k, out);
+}
+
+// Sum over a CTA of NW warps.  `red` holds two rows of NW words used in turn,
+// so one barrier per call suffices: a row is rewritten two calls later, after
+// the barrier of the call in between, when every thread has read it.
+template <int NW>
+__device__ __forceinline__ unsigned block_sum(unsigned v, unsigned* red, int& row) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = __reduce_add_sync(0xffffffffu, v);
+  unsigned* r = red + row * NW;
+  row ^= 1;
+  if (lane == 0) r[warp] = v;
+  __syncthreads();
+  unsigned s = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) s += r[w];
+  return s;
+}
+
+// Exact top-k of nb <= NT * PER keys (in shared memory) by a whole CTA of NT
+// threads; the same rules as warp_topk_bits.  Thread t holds keys t, t + NT,
+// ... in registers, so the 32 keys of shared-memory word w (bits of keys
+// 32w..32w+31) sit in one warp's lanes and a ballot builds the word.  After the
+// search the keys array is reused for two bitmaps (keys above tau; keys equal
+// to tau), which warp 0 turns into ascending ids.  Every thread of the CTA
+// must call it; `red` is 2 * NT / 32 words of shared memory.
+template <int NT, int PER>
+__device__ inline void block_topk(uint32_t* keys, int nb, int k, int32_t* out, unsigned* red) {
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int row = 0;
+  uint32_t kr[PER];
+  unsigned nc = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int j = i * NT + tid;
+    kr[i] = j < nb ? keys[j] : 0u;
+    nc += kr[i] != 0u;
+  }
+  nc = block_sum<NW>(nc, red, row);
+  const unsigned keff = nc < static_cast<unsigned>(k) ? nc : static_cast<unsigned>(k);
+  uint32_t tau = 0xffffffffu;
+  unsigned need = 0;
+  if (keff > 0u) {
+    uint32_t prefix = 0u;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = prefix | (1u << bit);
+      unsigned c = 0;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) c += kr[i] >= cand;
+      if (block_sum<NW>(c, red, row) >= keff) prefix = cand;
+    }
+    tau = prefix;
+    unsigned gt = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) gt += kr[i] > tau;
+    need = keff - block_sum<NW>(gt, red, row);
+  }
+  // every thread has passed a barrier after loading its keys: reuse the array
+  const int W = (nb + 31) / 32;
+  uint32_t* gbits = keys;
+  uint32_t* ebits = keys + W;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int w = i * NW + warp;
+    const unsigned g = __ballot_sync(0xffffffffu, keff > 0u && kr[i] > tau);
+    const unsigned e = __ballot_sync(0xffffffffu, keff > 0u && kr[i] == tau);
+    if (lane == 0 && w < W) {
+      gbits[w] = g;
+      ebits[w] = e;
+    }
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  // lane l owns words [l * WL, (l + 1) * WL)
+  const int WL = (W + 31) / 32;
+  const int w0 = min(W, lane * WL), w1 = min(W, w0 + WL);
+  unsigned eq_cnt = 0;
+  for (int w = w0; w < w1; ++w) eq_cnt += __popc(ebits[w]);
+  unsigned eq_before = warp_exclusive_scan(eq_cnt);
+  unsigned n_sel = 0;
+  for (int w = w0; w < w1; ++w) {
+    unsigned e = ebits[w];
+    unsigned take = 0u;
+    while (e && eq_before < need) {
+      const unsigned low = e & (0u - e);
+      take |= low;
+      e ^= low;
+      ++eq_before;
+    }
+    eq_before += __popc(e);
+    const unsigned sel = gbits[w] | take;
+    gbits[w] = sel;
+    n_sel += __popc(sel);
+  }
+  unsigned pos = warp_exclusive_scan(n_sel);
+  for (int w = w0; w < w1; ++w) {
+    unsigned m = gbits[w];
+    while (m) {
+      const int b = __ffs(m) - 1;
+      out[pos++] = w * 32 + b;
+      m &= m - 1u;
+    }
+  }
+  for (int s = static_cast<int>(keff) + lane; s < k; s += 32) out[s] = -1;
 }
 
 }  // namespace sa
