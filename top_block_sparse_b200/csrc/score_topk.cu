@@ -50,7 +50,6 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_topk_query0_kernel(Sco
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kRingBytes);     // [nb] (selecting CTA)
   __shared__ uint64_t full[kScoreStages];
   __shared__ __align__(16) float qs[kHeadDim];
-  __shared__ unsigned red[2 * kScoreWarps];
   __shared__ float qinv;
   __shared__ int is_last;
   __shared__ volatile int abort_flag;
@@ -180,11 +179,10 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_topk_query0_kernel(Sco
   __syncthreads();
   const int nb = static_cast<int>(a.nb);
   int32_t* out = a.idx + static_cast<int64_t>(pair) * a.top_k;
-  if (nb <= 2048) {
-    if (warp == 0) warp_topk(keys, nb, a.top_k, out);
-  } else {
-    block_topk<kScoreThreads, kMaxSelectBlocks / kScoreThreads>(keys, nb, a.top_k, out, red);
-  }
+  // the ring is idle now: its first words hold the selection's histograms
+  unsigned* scratch = reinterpret_cast<unsigned*>(ring);
+  if (nb <= 2048) block_radix_topk<2048 / kScoreThreads>(keys, nb, a.top_k, out, scratch);
+  else block_radix_topk<kMaxSelectBlocks / kScoreThreads>(keys, nb, a.top_k, out, scratch);
 }
 
 }  // namespace

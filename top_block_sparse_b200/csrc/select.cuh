@@ -149,47 +149,17 @@ __device__ __forceinline__ unsigned block_sum(unsigned v, unsigned* red, int& ro
   return s;
 }
 
-// Exact top-k of nb <= NT * PER keys (in shared memory) by a whole CTA of NT
-// threads; the same rules as warp_topk_bits.  Thread t holds keys t, t + NT,
-// ... in registers, so the 32 keys of shared-memory word w (bits of keys
-// 32w..32w+31) sit in one warp's lanes and a ballot builds the word.  After the
-// search the keys array is reused for two bitmaps (keys above tau; keys equal
-// to tau), which warp 0 turns into ascending ids.  Every thread of the CTA
-// must call it; `red` is 2 * NT / 32 words of shared memory.
+// Ascending ids of the keys above tau plus the first `need` keys equal to
+// tau (lowest ids first), -1 padded to k; the CTA's keys are in registers
+// (thread t holds keys t, t + NT, ...).  The keys array (nb words) is reused
+// for two bitmaps: the 32 keys of word w sit in one warp's lanes, so a ballot
+// builds the word; warp 0 then turns the bitmaps into ids.  Every thread must
+// call it after a barrier that follows its last read of `keys`.
 template <int NT, int PER>
-__device__ inline void block_topk(uint32_t* keys, int nb, int k, int32_t* out, unsigned* red) {
+__device__ inline void block_emit(const uint32_t (&kr)[PER], uint32_t* keys, int nb, int k, unsigned keff,
+                                  uint32_t tau, unsigned need, int32_t* out) {
   constexpr int NW = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int row = 0;
-  uint32_t kr[PER];
-  unsigned nc = 0;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int j = i * NT + tid;
-    kr[i] = j < nb ? keys[j] : 0u;
-    nc += kr[i] != 0u;
-  }
-  nc = block_sum<NW>(nc, red, row);
-  const unsigned keff = nc < static_cast<unsigned>(k) ? nc : static_cast<unsigned>(k);
-  uint32_t tau = 0xffffffffu;
-  unsigned need = 0;
-  if (keff > 0u) {
-    uint32_t prefix = 0u;
-#pragma unroll 1
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = prefix | (1u << bit);
-      unsigned c = 0;
-#pragma unroll
-      for (int i = 0; i < PER; ++i) c += kr[i] >= cand;
-      if (block_sum<NW>(c, red, row) >= keff) prefix = cand;
-    }
-    tau = prefix;
-    unsigned gt = 0;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) gt += kr[i] > tau;
-    need = keff - block_sum<NW>(gt, red, row);
-  }
-  // every thread has passed a barrier after loading its keys: reuse the array
   const int W = (nb + 31) / 32;
   uint32_t* gbits = keys;
   uint32_t* ebits = keys + W;
@@ -236,6 +206,121 @@ __device__ inline void block_topk(uint32_t* keys, int nb, int k, int32_t* out, u
     }
   }
   for (int s = static_cast<int>(keff) + lane; s < k; s += 32) out[s] = -1;
+}
+
+// Exact top-k of nb <= NT * PER keys (in shared memory) by a whole CTA of NT
+// threads; the same rules as warp_topk_bits.  The k-th largest key tau is
+// found bit by bit (32 steps of a CTA-wide count); `red` is 2 * NT / 32 words
+// of shared memory.
+template <int NT, int PER>
+__device__ inline void block_topk(uint32_t* keys, int nb, int k, int32_t* out, unsigned* red) {
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x;
+  int row = 0;
+  uint32_t kr[PER];
+  unsigned nc = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int j = i * NT + tid;
+    kr[i] = j < nb ? keys[j] : 0u;
+    nc += kr[i] != 0u;
+  }
+  nc = block_sum<NW>(nc, red, row);
+  const unsigned keff = nc < static_cast<unsigned>(k) ? nc : static_cast<unsigned>(k);
+  uint32_t tau = 0xffffffffu;
+  unsigned need = 0;
+  if (keff > 0u) {
+    uint32_t prefix = 0u;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = prefix | (1u << bit);
+      unsigned c = 0;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) c += kr[i] >= cand;
+      if (block_sum<NW>(c, red, row) >= keff) prefix = cand;
+    }
+    tau = prefix;
+    unsigned gt = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) gt += kr[i] > tau;
+    need = keff - block_sum<NW>(gt, red, row);
+  }
+  // every thread has passed a barrier after loading its keys
+  block_emit<NT, PER>(kr, keys, nb, k, keff, tau, need, out);
+}
+
+// The same selection by a CTA of 256 threads with an 8-bit radix search for
+// tau: four passes, each a histogram of the next 8 bits of the keys that
+// still agree with tau on the bits above (one private histogram per warp,
+// then one bin per thread), and a suffix scan over the 256 bins that picks
+// the digit holding the k-th largest.  `scratch` is NW * 256 + NW + 4 words
+// of shared memory (not the keys array).
+template <int PER>
+__device__ inline void block_radix_topk(uint32_t* keys, int nb, int k, int32_t* out, unsigned* scratch) {
+  constexpr int NT = 256, NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned* hist = scratch;                 // [NW][256]
+  unsigned* wtot = scratch + NW * 256;      // [NW]
+  unsigned* ctl = wtot + NW;                // digit, need
+  uint32_t kr[PER];
+  unsigned nc = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int j = i * NT + tid;
+    kr[i] = j < nb ? keys[j] : 0u;
+    nc += kr[i] != 0u;
+  }
+  nc = __reduce_add_sync(0xffffffffu, nc);
+  if (lane == 0) wtot[warp] = nc;
+  __syncthreads();
+  nc = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) nc += wtot[w];
+  const unsigned keff = nc < static_cast<unsigned>(k) ? nc : static_cast<unsigned>(k);
+  uint32_t prefix = 0u, pmask = 0u;
+  unsigned need = keff;
+  if (keff > 0u) {
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      __syncthreads();                      // the previous pass has read hist, wtot and ctl
+#pragma unroll
+      for (int w = 0; w < NW; ++w) hist[w * 256 + tid] = 0u;
+      __syncthreads();
+      unsigned* my = hist + warp * 256;
+#pragma unroll
+      for (int i = 0; i < PER; ++i)
+        if (kr[i] != 0u && (kr[i] & pmask) == prefix) atomicAdd(&my[(kr[i] >> shift) & 255u], 1u);
+      __syncthreads();
+      // thread t takes bin b = 255 - t, so a prefix scan over t counts the
+      // keys whose digit is >= b
+      const int b = 255 - tid;
+      unsigned hb = 0;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) hb += hist[w * 256 + b];
+      unsigned x = hb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) wtot[warp] = x;
+      __syncthreads();
+      unsigned off = 0;
+      for (int w = 0; w < warp; ++w) off += wtot[w];
+      const unsigned incl = x + off, excl = incl - hb;
+      if (hb > 0u && excl < need && incl >= need) {
+        ctl[0] = static_cast<unsigned>(b);
+        ctl[1] = need - excl;
+      }
+      __syncthreads();
+      prefix |= ctl[0] << shift;
+      pmask |= 255u << shift;
+      need = ctl[1];
+    }
+  }
+  const uint32_t tau = keff > 0u ? prefix : 0xffffffffu;
+  if (keff == 0u) need = 0u;
+  block_emit<NT, PER>(kr, keys, nb, k, keff, tau, need, out);
 }
 
 }  // namespace sa
