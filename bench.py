@@ -30,6 +30,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -132,6 +133,10 @@ def decode_bytes(w) -> dict:
     return dict(kv=kv, kc=kc, q=q, o=o, keys_per_query=keys, attn=kv + q + o, step=kv + kc + 2 * q + o)
 
 
+# the sources a kernel's traffic record depends on
+TRAFFIC_SOURCES = {"decode_tc.cu": ("decode_tc.cu", "decode_units.cuh", "tc.cuh", "common.cuh", "internal.h")}
+
+
 def src_hash(*names) -> str:
     h = hashlib.sha256()
     for n in names:
@@ -139,17 +144,24 @@ def src_hash(*names) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_file: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current source of the kernel; else None."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+def profiled_traffic(kernel_file: str, pairs: int):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary (read + write of one launch at the captured batch, scaled by the
+    number of (sequence, KV head) pairs: the traffic is per pair), if the
+    summary was taken on the current source of the kernel; else None."""
+    path = os.path.join(ROOT, "profiles", "decode_tc_kernel__decode_32k_b16.md")
     try:
-        d = json.load(open(path))[kernel_file]
-        if d["src_sha"] == src_hash(kernel_file, "common.cuh"):
-            return float(d["dram_bytes_per_launch"])
+        text = open(path).read()
+        sha = re.search(r"source hash: `([0-9a-f]+)`", text).group(1)
+        cap_pairs = int(re.search(r"captured pairs: (\d+)", text).group(1))
+        if sha != src_hash(*TRAFFIC_SOURCES[kernel_file]):
+            return None
+        sec = text[text.index("## `decode_tc_kernel"):]
+        rd = float(re.search(r"dram__bytes_read\.sum`\) \| ([0-9.]+) Mbyte", sec).group(1))
+        wr = float(re.search(r"dram__bytes_write\.sum`\) \| ([0-9.]+) Mbyte", sec).group(1))
+        return (rd + wr) * 1e6 * pairs / cap_pairs
     except Exception:
-        pass
-    return None
+        return None
 
 
 class L2Flush:
@@ -357,11 +369,11 @@ def run_ours(args, w, rank, world, local_rank):
         "config": config_of(w),
         "decode_hbm_gbs": step_gbs, "decode_hbm_frac": step_gbs / hbm,
         "decode_bytes_per_step": by["step"], "keys_per_query": by["keys_per_query"],
-        "roofline": {"bound": "hbm", "kernel": "decode_attn_kernel (split-KV sparse attention)",
+        "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel (tcgen05 split-KV sparse attention)",
                      "achieved": attn_gbs, "peak": hbm, "unit": "GB/s", "frac": attn_gbs / hbm,
                      "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs, burst copy)" if src == "measured" else src,
                      "algorithmic_bytes_per_launch": by["attn"], "launch_ms": attn_ms,
-                     "traffic": profiled_traffic("decode_attn.cu"),
+                     "traffic": profiled_traffic("decode_tc.cu", w.batch * w.num_kv_heads),
                      "frac_of_spec_8tbs": attn_gbs / 8000.0},
         "pool": {"kernel": "pool_kernel", "ms": pool_ms, "gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
                  "note": "compression runs once after prefill / when a block fills; not part of a decode step"},

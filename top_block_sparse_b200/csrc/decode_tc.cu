@@ -608,6 +608,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok && lane == 0) fail();
   }
 
+  // every warp reaches the final barrier converged (lane-0 drains above)
+  __syncwarp();
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 1) {

@@ -406,6 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(o_free);
     }
   }
+  // every warp reaches the final barrier converged (lane-0 drains above)
+  __syncwarp();
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 9) {

@@ -327,6 +327,8 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
       }
     }
   }
+  // every warp reaches the final barrier converged (lane-0 drains above)
+  __syncwarp();
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 1) {
@@ -356,7 +358,7 @@ __global__ void kc_split_kernel(const float* Kc, uint16_t* out, int64_t rows) {
 
 // Per (pair, tile) top-k over the candidate scores, one warp each.
 __global__ void __launch_bounds__(256) prefill_topk_kernel(PSArgs a, int top_k, int32_t* idx) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + warp;
   if (row >= static_cast<int64_t>(a.P) * a.n_tiles) return;
