@@ -94,6 +94,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// The same wait by a whole warp with one warp-wide outcome (a warp that
+// continues in lock step, e.g. to elect an issuing lane, must not split on a
+// timeout seen by some lanes only).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort));
+}
+
 // ---- 1-D bulk copy global -> shared (TMA engine, no tensor map) -----------
 // Both addresses 16-byte aligned, bytes a multiple of 16.
 
@@ -104,6 +111,13 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, u
           smem_u32(smem_dst)),
       "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Asks the TMA engine to bring `bytes` of global memory into L2 (no
+// destination, no completion to wait for); 16-byte aligned, size a multiple
+// of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* gmem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem), "r"(bytes) : "memory");
 }
 
 // ---- programmatic dependent launch ----------------------------------------

@@ -42,6 +42,7 @@ constexpr int kBBuf = 65536;                   // B operand: hi atoms 0,1 then l
 constexpr int kScoreThreadsTC = 448;
 constexpr int kBuilders = 8;                   // warps 2..9 build the B operand, 16 rows each
 constexpr uint32_t kIdesc = tc::idesc_bf16(128, 128, false, false);
+constexpr int kND = 4;                         // TMEM accumulators of 128 columns (all 512)
 
 struct PSArgs {
   const uint16_t* Q;        // [B, T, Hq, 128] bf16
@@ -92,8 +93,8 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
   uint64_t* b_full = a_empty + kNSA;
   uint64_t* b_empty = b_full + 2;
   uint64_t* d_full = b_empty + 2;
-  uint64_t* d_empty = d_full + 2;
-  uint64_t* mma_done = d_empty + 2;
+  uint64_t* d_empty = d_full + kND;
+  uint64_t* mma_done = d_empty + kND;
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
 
@@ -108,15 +109,17 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&b_full[b], kBuilders);
       mbar_init(&b_empty[b], 1);
-      mbar_init(&d_full[b], 1);
-      mbar_init(&d_empty[b], 4);
+    }
+    for (int d = 0; d < kND; ++d) {
+      mbar_init(&d_full[d], 1);
+      mbar_init(&d_empty[d], 4);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tc::tmem_alloc(tmem_base_slot, 256);
+    tc::tmem_alloc(tmem_base_slot, 128 * kND);
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
@@ -158,7 +161,9 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop in lock step so that the descriptors stay
+    // warp-uniform; one elected lane issues each MMA and commit.
+    {
       int use = 0, mc_all = 0, it = 0;
       bool ok = true;
       const uint32_t bbase = smem_u32(Bop);
@@ -169,13 +174,13 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
         const int mc = chunk_count(a, n);
         if (mc == 0) continue;
         const int b = it & 1;
-        if (!mbar_wait_bounded(&b_full[b], (it >> 1) & 1, abort_flag)) { fail(); break; }
+        if (!mbar_wait_warp(&b_full[b], (it >> 1) & 1, abort_flag)) { if (lane == 0) fail(); break; }
         tc::fence_after_sync();
         const uint32_t bhi = bbase + b * kBBuf, blo = bhi + 32768;
         for (int m = 0; m < mc; ++m, ++mc_all) {
-          const int d = mc_all & 1;
-          if (mc_all >= 2 && !mbar_wait_bounded(&d_empty[d], ((mc_all >> 1) & 1) ^ 1, abort_flag)) {
-            fail();
+          const int d = mc_all % kND;
+          if (mc_all >= kND && !mbar_wait_warp(&d_empty[d], ((mc_all / kND) & 1) ^ 1, abort_flag)) {
+            if (lane == 0) fail();
             ok = false;
             break;
           }
@@ -183,41 +188,42 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
           const uint32_t dt = tbase + d * 128;
           // hi part of Kc: hi*hi then hi*lo
           int s = use % kNSA;
-          if (!mbar_wait_bounded(&a_full[s], (use / kNSA) & 1, abort_flag)) { fail(); ok = false; break; }
+          if (!mbar_wait_warp(&a_full[s], (use / kNSA) & 1, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
           tc::fence_after_sync();
           const uint32_t ahi = abase + s * kAStage;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            tc::mma_bf16(dt, tc::smem_desc(ahi + off, 16, 1024), tc::smem_desc(bhi + off, 16, 1024), kIdesc, kk > 0);
+            tc::mma_bf16_elect(dt, tc::smem_desc(ahi + off, 16, 1024), tc::smem_desc(bhi + off, 16, 1024), kIdesc, kk > 0);
           }
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            tc::mma_bf16(dt, tc::smem_desc(ahi + off, 16, 1024), tc::smem_desc(blo + off, 16, 1024), kIdesc, true);
+            tc::mma_bf16_elect(dt, tc::smem_desc(ahi + off, 16, 1024), tc::smem_desc(blo + off, 16, 1024), kIdesc, true);
           }
-          tc::mma_commit(&a_empty[s]);
+          tc::mma_commit_elect(&a_empty[s]);
           ++use;
           // lo part of Kc: lo*hi
           s = use % kNSA;
-          if (!mbar_wait_bounded(&a_full[s], (use / kNSA) & 1, abort_flag)) { fail(); ok = false; break; }
+          if (!mbar_wait_warp(&a_full[s], (use / kNSA) & 1, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
           tc::fence_after_sync();
           const uint32_t alo = abase + s * kAStage;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            tc::mma_bf16(dt, tc::smem_desc(alo + off, 16, 1024), tc::smem_desc(bhi + off, 16, 1024), kIdesc, true);
+            tc::mma_bf16_elect(dt, tc::smem_desc(alo + off, 16, 1024), tc::smem_desc(bhi + off, 16, 1024), kIdesc, true);
           }
-          tc::mma_commit(&a_empty[s]);
+          tc::mma_commit_elect(&a_empty[s]);
           ++use;
-          tc::mma_commit(&d_full[d]);
+          tc::mma_commit_elect(&d_full[d]);
         }
-        tc::mma_commit(&b_empty[b]);
+        tc::mma_commit_elect(&b_empty[b]);
         ++it;
       }
       // every MMA issued has completed before the CTA tears TMEM down
-      tc::mma_commit(mma_done);
-      mbar_wait_bounded(mma_done, 0, nullptr);
+      tc::mma_commit_elect(mma_done);
+      mbar_wait_warp(mma_done, 0, nullptr);
+      __syncwarp();
     }
   } else if (warp < 2 + kBuilders) {
     // ---------------------------------------------------- B operand builders
@@ -227,10 +233,25 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
     const int wq = warp - 2;                       // rows wq*16 .. wq*16+15 of the item
     const int cc = lane & 15;                      // 16-byte column chunk (8 columns)
     const bool write_lo = lane >= 16;
+    // This warp's 16 rows of item kk are prefetched into L2 two items ahead
+    // of their use, so the loads below hit L2 and the HBM stream of Q runs
+    // on the TMA engine rather than on the builders' registers.
+    auto prefetch_item = [&](int kk) {
+      if (kk >= n_items || lane >= 16) return;
+      int n2, p2;
+      item_of(a, kk, &n2, &p2);
+      const int row = 128 * n2 + wq * 16 + lane;
+      if (chunk_count(a, n2) == 0 || row >= a.T) return;
+      const int bi2 = p2 / a.Hkv, h2 = p2 % a.Hkv;
+      prefetch_l2_bulk(a.Q + ((static_cast<int64_t>(bi2) * a.T + row) * a.Hq + h2 * 4) * kHeadDim, 4 * kHeadDim * 2);
+    };
+    prefetch_item(blockIdx.x);
+    prefetch_item(blockIdx.x + gridDim.x);
     int it = 0;
     for (int k = blockIdx.x; k < n_items; k += gridDim.x) {
       int n, p;
       item_of(a, k, &n, &p);
+      prefetch_item(k + 2 * gridDim.x);
       if (chunk_count(a, n) == 0) continue;
       const int b = it & 1;
       if (it >= 2 && !mbar_wait_bounded(&b_empty[b], ((it >> 1) & 1) ^ 1, abort_flag)) {
@@ -294,8 +315,8 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
       item_of(a, k, &n, &p);
       const int mc = chunk_count(a, n);
       for (int m = 0; m < mc; ++m, ++mc_all) {
-        const int d = mc_all & 1;
-        if (!mbar_wait_bounded(&d_full[d], (mc_all >> 1) & 1, abort_flag)) {
+        const int d = mc_all % kND;
+        if (!mbar_wait_bounded(&d_full[d], (mc_all / kND) & 1, abort_flag)) {
           if (lane == 0) fail();
           ok = false;
           break;
@@ -310,10 +331,15 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
           tc::tmem_wait_ld();
           const int t = 2 * n + half;
           const int rows = min(kTile, a.T - t * kTile);    // ragged last tile
-          float mx = -CUDART_INF_F;
+          float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+          if (rows == kTile) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) mx = (c < rows) ? fmaxf(mx, v[c]) : mx;
-          best[half] = mx;
+            for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], v[c]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) m4[c & 3] = (c < rows) ? fmaxf(m4[c & 3], v[c]) : m4[c & 3];
+          }
+          best[half] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         }
         tc::fence_before_sync();
         __syncwarp();
@@ -333,7 +359,7 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
   __syncthreads();
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tbase, 256);
+    tc::tmem_dealloc(tbase, 128 * kND);
   }
 }
 
@@ -357,7 +383,7 @@ __global__ void kc_split_kernel(const float* Kc, uint16_t* out, int64_t rows) {
 }
 
 // Per (pair, tile) top-k over the candidate scores, one warp each.
-__global__ void __launch_bounds__(256) prefill_topk_kernel(PSArgs a, int top_k, int32_t* idx) {
+__global__ void __launch_bounds__(256, 2) prefill_topk_kernel(PSArgs a, int top_k, int32_t* idx) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + warp;
@@ -367,19 +393,26 @@ __global__ void __launch_bounds__(256) prefill_topk_kernel(PSArgs a, int top_k, 
   const float* sc = a.scores + row * a.nb;
   // blocks at or after the tile are never candidates
   const int nb_t = min(a.nb, t);
-  for (int j0 = 0; j0 < nb_t; j0 += 8 * 32) {
-    float v[8];
+  // the candidates of tile t (context C = 64 t) are blocks [j_lo, j_hi): past
+  // the sink, starting before the window (the test of is_candidate)
+  const int64_t C = static_cast<int64_t>(t) * kTile;
+  const int64_t s_end = a.S < C ? a.S : C;
+  const int64_t w_begin = (C - a.W) > s_end ? (C - a.W) : s_end;
+  const int j_lo = static_cast<int>(s_end / kTile);
+  const int j_hi = min(nb_t, static_cast<int>((w_begin + kTile - 1) / kTile));
+  for (int j0 = 0; j0 < nb_t; j0 += 32 * 32) {
+    float v[32];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 32; ++u) {
       const int j = j0 + u * 32 + lane;
-      v[u] = (j < nb_t && is_candidate(a, t, j)) ? __ldcg(sc + j) : 0.f;
+      v[u] = (j >= j_lo && j < j_hi) ? __ldcg(sc + j) : 0.f;
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 32; ++u) {
       const int j = j0 + u * 32 + lane;
       if (j < nb_t) {
         const uint32_t key = float_key(v[u]);
-        keys[j] = is_candidate(a, t, j) ? (key == 0u ? 1u : key) : 0u;
+        keys[j] = (j >= j_lo && j < j_hi) ? (key == 0u ? 1u : key) : 0u;
       }
     }
   }
@@ -404,7 +437,7 @@ EncodeFn encode_fn() {
 }  // namespace
 
 size_t prefill_score_smem() {
-  return 1024 + kNSA * kAStage + 2 * kBBuf + 16 * 8 + 64;
+  return 1024 + kNSA * kAStage + 2 * kBBuf + (2 * kNSA + 4 + 2 * kND + 1) * 8 + 64;
 }
 
 cudaError_t launch_prefill_score(const PrefillArgs& pa, cudaStream_t s) {

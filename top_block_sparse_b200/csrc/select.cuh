@@ -47,20 +47,34 @@ __device__ inline void warp_topk_bits(const uint32_t* keys, int nb, int k, int32
   uint32_t tau = 0xffffffffu;
   unsigned need = 0;
   if (keff > 0u) {
+    // tau = the largest value with at least keff keys >= tau.  When some
+    // prefix already has exactly keff keys at or above it, those keys are the
+    // selection: stop there (tau = prefix - 1, nothing taken at equality).
     uint32_t prefix = 0u;
+    bool exact = false;
 #pragma unroll 1
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = prefix | (1u << bit);
       unsigned c = 0;
 #pragma unroll
       for (int i = 0; i < PER; ++i) c += kr[i] >= cand;
-      if (__reduce_add_sync(0xffffffffu, c) >= keff) prefix = cand;
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (c >= keff) prefix = cand;
+      if (c == keff) {
+        exact = true;
+        break;
+      }
     }
-    tau = prefix;
-    unsigned gt = 0;
+    if (exact) {
+      tau = prefix - 1u;            // prefix >= 1: it has a bit set
+      need = 0u;
+    } else {
+      tau = prefix;
+      unsigned gt = 0;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) gt += kr[i] > tau;
-    need = keff - __reduce_add_sync(0xffffffffu, gt);
+      for (int i = 0; i < PER; ++i) gt += kr[i] > tau;
+      need = keff - __reduce_add_sync(0xffffffffu, gt);
+    }
   }
   const unsigned lt_mask = (1u << lane) - 1u;
   unsigned base = 0, eq_base = 0;
@@ -90,18 +104,29 @@ __device__ inline void warp_topk_smem(const uint32_t* keys, int nb, int k, int32
   unsigned need = 0;
   if (keff > 0u) {
     uint32_t prefix = 0u;
+    bool exact = false;
 #pragma unroll 1
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = prefix | (1u << bit);
       unsigned c = 0;
 #pragma unroll 4
       for (int j = lane; j < nb; j += 32) c += keys[j] >= cand;
-      if (__reduce_add_sync(0xffffffffu, c) >= keff) prefix = cand;
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (c >= keff) prefix = cand;
+      if (c == keff) {
+        exact = true;
+        break;
+      }
     }
-    tau = prefix;
-    unsigned gt = 0;
-    for (int j = lane; j < nb; j += 32) gt += keys[j] > tau;
-    need = keff - __reduce_add_sync(0xffffffffu, gt);
+    if (exact) {
+      tau = prefix - 1u;
+      need = 0u;
+    } else {
+      tau = prefix;
+      unsigned gt = 0;
+      for (int j = lane; j < nb; j += 32) gt += keys[j] > tau;
+      need = keff - __reduce_add_sync(0xffffffffu, gt);
+    }
   }
   const unsigned lt_mask = (1u << lane) - 1u;
   unsigned base = 0, eq_base = 0;
