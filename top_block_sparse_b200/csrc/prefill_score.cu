@@ -227,12 +227,13 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
     }
   } else if (warp < 2 + kBuilders) {
     // ---------------------------------------------------- B operand builders
-    // A row's G = 4 query heads are 1 KB contiguous = 64 chunks of 16 B: lane l
-    // loads chunks l (head l / 16) and l + 32 (head l / 16 + 2), both of column
-    // chunk cc = l % 16; lanes l and l ^ 16 hold the other two heads.
+    // Lane l owns the 16-byte column chunk cc = l % 16 (8 columns) of the
+    // warp's rows of parity l / 16: it loads the chunk of all G = 4 query
+    // heads (a half-warp reads 256 contiguous bytes per head), sums them in
+    // fp32, scales, and writes both the bf16 hi part and the bf16 remainder.
     const int wq = warp - 2;                       // rows wq*16 .. wq*16+15 of the item
     const int cc = lane & 15;                      // 16-byte column chunk (8 columns)
-    const bool write_lo = lane >= 16;
+    const int rp = lane >> 4;                      // row parity
     // This warp's 16 rows of item kk are prefetched into L2 two items ahead
     // of their use, so the loads below hit L2 and the HBM stream of Q runs
     // on the TMA engine rather than on the builders' registers.
@@ -259,45 +260,40 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
         break;
       }
       const int bi = p / a.Hkv, h = p % a.Hkv;
-      unsigned char* dst = Bop + b * kBBuf + (write_lo ? 32768 : 0) + (cc >> 3) * 16384;
+      unsigned char* dst_hi = Bop + b * kBBuf + (cc >> 3) * 16384;
+      unsigned char* dst_lo = dst_hi + 32768;
 #pragma unroll 1
-      for (int rb = 0; rb < 16; rb += 8) {
-        uint4 x[8][2];
+      for (int rb = 0; rb < 8; rb += 4) {
+        uint4 x[4][4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int row = 128 * n + wq * 16 + rb + u;
-          if (row < a.T) {
-            const uint4* src = reinterpret_cast<const uint4*>(
-                a.Q + ((static_cast<int64_t>(bi) * a.T + row) * a.Hq + h * 4) * kHeadDim);
-            x[u][0] = __ldg(src + lane);
-            x[u][1] = __ldg(src + lane + 32);
-          } else {
-            x[u][0] = make_uint4(0u, 0u, 0u, 0u);
-            x[u][1] = x[u][0];
-          }
+        for (int u = 0; u < 4; ++u) {
+          const int row = 128 * n + wq * 16 + 2 * (rb + u) + rp;
+          const uint4* src = reinterpret_cast<const uint4*>(
+              a.Q + ((static_cast<int64_t>(bi) * a.T + (row < a.T ? row : 0)) * a.Hq + h * 4) * kHeadDim);
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            x[u][g] = row < a.T ? __ldg(src + g * 16 + cc) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int r = wq * 16 + rb + u;
-          float f0[8], f1[8], v[8];
-          unpack8(x[u][0], f0);
-          unpack8(x[u][1], f1);
+        for (int u = 0; u < 4; ++u) {
+          const int r = wq * 16 + 2 * (rb + u) + rp;
+          float v[8], f[8];
+          unpack8(x[u][0], v);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] = f0[e] + f1[e];
+          for (int g = 1; g < 4; ++g) {
+            unpack8(x[u][g], f);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] = (v[e] + __shfl_xor_sync(0xffffffffu, v[e], 16)) * a.scale;
-          uint32_t w[4];
+            for (int e = 0; e < 8; ++e) v[e] += f[e];
+          }
+          uint32_t whi[4], wlo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * e]), h1 = __float2bfloat16_rn(v[2 * e + 1]);
-            if (write_lo) {
-              w[e] = pack_bf16x2(v[2 * e] - __bfloat162float(h0), v[2 * e + 1] - __bfloat162float(h1));
-            } else {
-              w[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
-                     (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-            }
+            const float v0 = v[2 * e] * a.scale, v1 = v[2 * e + 1] * a.scale;
+            whi[e] = pack_bf16x2(v0, v1);
+            wlo[e] = pack_bf16x2(v0 - bf16lo(whi[e]), v1 - bf16hi(whi[e]));
           }
-          *reinterpret_cast<uint4*>(dst + tc::sw128_off(r, cc & 7)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(dst_hi + tc::sw128_off(r, cc & 7)) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
+          *reinterpret_cast<uint4*>(dst_lo + tc::sw128_off(r, cc & 7)) = make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
         }
       }
       tc::fence_proxy_async_smem();

@@ -31,17 +31,14 @@ __device__ __forceinline__ unsigned warp_exclusive_scan(unsigned v) {
 // are taken, and keys equal to tau in ascending block order until k are taken
 // (the lower-index tie rule).  Selected ids are written ascending to
 // out[0..k), -1 padded.  PER (keys per lane) bounds nb <= 32 * PER.
+// warp_topk_regs takes the keys in registers (0 also past nb);
+// warp_topk_bits loads them from shared memory first.
 template <int PER>
-__device__ inline void warp_topk_bits(const uint32_t* keys, int nb, int k, int32_t* out) {
+__device__ inline void warp_topk_regs(const uint32_t (&kr)[PER], int k, int32_t* out) {
   const int lane = threadIdx.x & 31;
-  uint32_t kr[PER];
   unsigned nc = 0;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int j = i * 32 + lane;
-    kr[i] = j < nb ? keys[j] : 0u;
-    nc += kr[i] != 0u;
-  }
+  for (int i = 0; i < PER; ++i) nc += kr[i] != 0u;
   nc = __reduce_add_sync(0xffffffffu, nc);
   const unsigned keff = nc < static_cast<unsigned>(k) ? nc : static_cast<unsigned>(k);
   uint32_t tau = 0xffffffffu;
@@ -90,6 +87,18 @@ __device__ inline void warp_topk_bits(const uint32_t* keys, int nb, int k, int32
     base += __popc(b);
   }
   for (int s = static_cast<int>(keff) + lane; s < k; s += 32) out[s] = -1;
+}
+
+template <int PER>
+__device__ inline void warp_topk_bits(const uint32_t* keys, int nb, int k, int32_t* out) {
+  const int lane = threadIdx.x & 31;
+  uint32_t kr[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int j = i * 32 + lane;
+    kr[i] = j < nb ? keys[j] : 0u;
+  }
+  warp_topk_regs<PER>(kr, k, out);
 }
 
 // The same selection for any nb, by one warp, with the keys left in shared
