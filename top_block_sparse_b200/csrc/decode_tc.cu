@@ -324,7 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // S(i) needs unit i's K and Q and a free S buffer; PV(i) needs P(i).  The
     // thread polls both and issues whichever is ready, so a unit's ring stage
     // (released when PV(i) completes) never waits for the next unit's data.
-    if (lane == 0) {
+    // The whole warp runs the loop in lock step (descriptors warp-uniform);
+    // every readiness test is made warp-wide and one elected lane issues.
+    {
       const uint32_t ring_a = smem_u32(ring), qa = smem_u32(Qs), pa = smem_u32(Ps);
       int ns = 0, npv = 0;                  // next S / PV to issue
       PairCursor cs, cp;                    // pair bookkeeping of units ns / npv
@@ -337,19 +339,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ns < nunits) {
           const bool fi = cs.first(ns);
           const int pk = cs.ordinal, qb = pk & 1, s = ns % kNS;
-          if (mbar_test_wait(&kv_full[s], (ns / kNS) & 1) &&
-              (!fi || mbar_test_wait(&q_full[qb], (pk >> 1) & 1)) &&
-              (ns < 2 || mbar_test_wait(&s_free[ns & 1], ((ns >> 1) + 1) & 1))) {
+          const bool ready = mbar_test_wait(&kv_full[s], (ns / kNS) & 1) &&
+                             (!fi || mbar_test_wait(&q_full[qb], (pk >> 1) & 1)) &&
+                             (ns < 2 || mbar_test_wait(&s_free[ns & 1], ((ns >> 1) + 1) & 1));
+          if (__all_sync(0xffffffffu, ready)) {
             tc::fence_after_sync();
             const uint32_t kst = ring_a + s * kStage, qst = qa + qb * kQBuf;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              tc::mma_bf16(tbase + (ns & 1) * kN,
+              tc::mma_bf16_elect(tbase + (ns & 1) * kN,
                            tc::smem_desc(kst + (kk >> 2) * kKVHalf + (kk & 3) * 32, 16, 1024),
                            tc::smem_desc(qst + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024), kIdescS, kk > 0);
-            tc::mma_commit(&s_full[ns & 1]);
+            tc::mma_commit_elect(&s_full[ns & 1]);
             // no later MMA reads this Q buffer for this pair
-            if (cs.last(ns, nunits)) tc::mma_commit(&q_empty[qb]);
+            if (cs.last(ns, nunits)) tc::mma_commit_elect(&q_empty[qb]);
             ++ns;
             cs.at(ns);
             did = true;
@@ -358,19 +361,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (npv < ns) {
           const bool fi = cp.first(npv);
           const int pk = cp.ordinal, ob = pk & 1;
-          if (mbar_test_wait(&p_full[npv & 1], (npv >> 1) & 1) &&
-              (!fi || pk < 2 || mbar_test_wait(&o_free[ob], ((pk >> 1) + 1) & 1))) {
+          const bool ready = mbar_test_wait(&p_full[npv & 1], (npv >> 1) & 1) &&
+                             (!fi || pk < 2 || mbar_test_wait(&o_free[ob], ((pk >> 1) + 1) & 1));
+          if (__all_sync(0xffffffffu, ready)) {
             tc::fence_after_sync();
             const uint32_t vst = ring_a + (npv % kNS) * kStage + 2 * kKVHalf;
             const uint32_t pb = pa + (npv & 1) * kPBuf;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              tc::mma_bf16(tbase + 32 + ob * kN, tc::smem_desc(vst + kk * 2048, kKVHalf, 1024),
+              tc::mma_bf16_elect(tbase + 32 + ob * kN, tc::smem_desc(vst + kk * 2048, kKVHalf, 1024),
                            tc::smem_desc(pb + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024), kIdescO,
                            !(fi && kk == 0));
-            tc::mma_commit(&kv_empty[npv % kNS]);
-            tc::mma_commit(&p_free[npv & 1]);
-            if (cp.last(npv, nunits)) tc::mma_commit(&o_full[ob]);
+            tc::mma_commit_elect(&kv_empty[npv % kNS]);
+            tc::mma_commit_elect(&p_free[npv & 1]);
+            if (cp.last(npv, nunits)) tc::mma_commit_elect(&o_full[ob]);
             ++npv;
             cp.at(npv);
             did = true;
@@ -379,16 +383,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (did) {
           t0 = global_ns();
         } else if ((spin & 63u) == 0) {
-          if (*abort_flag || global_ns() - t0 > kWaitLimitNs) {
+          if (__any_sync(0xffffffffu, *abort_flag || global_ns() - t0 > kWaitLimitNs)) {
             ok = false;
             break;
           }
         }
       }
-      if (!ok) fail();
+      if (!ok && lane == 0) fail();
       // every MMA must be complete before TMEM is released
-      tc::mma_commit(mma_done);
-      mbar_wait_bounded(mma_done, 0, nullptr);
+      tc::mma_commit_elect(mma_done);
+      mbar_wait_warp(mma_done, 0, nullptr);
     }
     __syncwarp();
   } else {

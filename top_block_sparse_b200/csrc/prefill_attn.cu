@@ -206,8 +206,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int p, t;
       item_of(a, k, &p, &t);
       const Blocks bl = blocks_of(a, p, t, lane);
-      if (lane == 0) {
-        if (!mbar_wait_bounded(q_full, it & 1, abort_flag)) { fail(); ok = false; }
+      // the whole warp runs the issue loop in lock step (descriptors stay
+      // warp-uniform); one elected lane issues each MMA and commit
+      {
+        if (!mbar_wait_warp(q_full, it & 1, abort_flag)) { if (lane == 0) fail(); ok = false; }
         tc::fence_after_sync();
         // S(b) for both halves
         auto issue_s = [&](int b_use) {
@@ -219,16 +221,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t qoff = (kk >> 2) * (kQBytes / 2) + hf * 16384 + (kk & 3) * 32;
               const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
-              tc::mma_bf16(tbase + hf * 64, tc::smem_desc(qa + qoff, 16, 1024), tc::smem_desc(kst + koff, 16, 1024),
+              tc::mma_bf16_elect(tbase + hf * 64, tc::smem_desc(qa + qoff, 16, 1024), tc::smem_desc(kst + koff, 16, 1024),
                            kIdescS, kk > 0);
             }
           }
-          tc::mma_commit(s_full);
+          tc::mma_commit_elect(s_full);
         };
         if (ok) {
           // S(0) needs the S columns free: the previous item's last S was read
-          if (nb_all > 0 && !mbar_wait_bounded(s_free, (nb_all - 1) & 1, abort_flag)) { fail(); ok = false; }
-          if (ok && !mbar_wait_bounded(&kv_full[use % kNKV], (use / kNKV) & 1, abort_flag)) { fail(); ok = false; }
+          if (nb_all > 0 && !mbar_wait_warp(s_free, (nb_all - 1) & 1, abort_flag)) { if (lane == 0) fail(); ok = false; }
+          if (ok && !mbar_wait_warp(&kv_full[use % kNKV], (use / kNKV) & 1, abort_flag)) { if (lane == 0) fail(); ok = false; }
           if (ok) {
             tc::fence_after_sync();
             issue_s(use);
@@ -237,41 +239,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < bl.n_blk && ok; ++b, ++use, ++nb_all) {
           if (b + 1 < bl.n_blk) {
             // S(b+1) as soon as the softmax has read S(b) and K(b+1) has landed
-            if (!mbar_wait_bounded(s_free, nb_all & 1, abort_flag) ||
-                !mbar_wait_bounded(&kv_full[(use + 1) % kNKV], ((use + 1) / kNKV) & 1, abort_flag)) {
-              fail();
+            if (!mbar_wait_warp(s_free, nb_all & 1, abort_flag) ||
+                !mbar_wait_warp(&kv_full[(use + 1) % kNKV], ((use + 1) / kNKV) & 1, abort_flag)) {
+              if (lane == 0) fail();
               ok = false;
               break;
             }
             tc::fence_after_sync();
             issue_s(use + 1);
           } else {
-            tc::mma_commit(q_empty);            // Q is read by no later MMA of this item
+            tc::mma_commit_elect(q_empty);            // Q is read by no later MMA of this item
           }
-          if (!mbar_wait_bounded(p_full, nb_all & 1, abort_flag)) { fail(); ok = false; break; }
-          if (b == 0 && it > 0 && !mbar_wait_bounded(o_free, (it - 1) & 1, abort_flag)) { fail(); ok = false; break; }
+          if (!mbar_wait_warp(p_full, nb_all & 1, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
+          if (b == 0 && it > 0 && !mbar_wait_warp(o_free, (it - 1) & 1, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
           tc::fence_after_sync();
           const uint32_t vst = kva + (use % kNKV) * kKVStage + 16384;
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              tc::mma_bf16(tbase + 128 + hf * 128, tc::smem_desc(pa + hf * 16384 + kk * 32, 16, 1024),
+              tc::mma_bf16_elect(tbase + 128 + hf * 128, tc::smem_desc(pa + hf * 16384 + kk * 32, 16, 1024),
                            tc::smem_desc(vst + kk * 2048, 8192, 1024), kIdescO, b > 0 || kk > 0);
             }
           }
-          tc::mma_commit(&kv_empty[use % kNKV]);
-          tc::mma_commit(pv_done);
+          tc::mma_commit_elect(&kv_empty[use % kNKV]);
+          tc::mma_commit_elect(pv_done);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       use = __shfl_sync(0xffffffffu, use, 0);
       nb_all = __shfl_sync(0xffffffffu, nb_all, 0);
     }
-    if (lane == 0) {
-      tc::mma_commit(mma_done);
-      mbar_wait_bounded(mma_done, 0, nullptr);
-    }
+    tc::mma_commit_elect(mma_done);
+    mbar_wait_warp(mma_done, 0, nullptr);
   } else {
     // ------------------------------------------------- softmax and epilogue
     const int hf = warp >> 2, q = warp & 3;
