@@ -264,20 +264,32 @@ __device__ inline void block_topk(uint32_t* keys, int nb, int k, int32_t* out, u
   uint32_t tau = 0xffffffffu;
   unsigned need = 0;
   if (keff > 0u) {
+    // as in warp_topk_regs: stop once a prefix holds exactly keff keys
     uint32_t prefix = 0u;
+    bool exact = false;
 #pragma unroll 1
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = prefix | (1u << bit);
       unsigned c = 0;
 #pragma unroll
       for (int i = 0; i < PER; ++i) c += kr[i] >= cand;
-      if (block_sum<NW>(c, red, row) >= keff) prefix = cand;
+      c = block_sum<NW>(c, red, row);
+      if (c >= keff) prefix = cand;
+      if (c == keff) {
+        exact = true;
+        break;
+      }
     }
-    tau = prefix;
-    unsigned gt = 0;
+    if (exact) {
+      tau = prefix - 1u;
+      need = 0u;
+    } else {
+      tau = prefix;
+      unsigned gt = 0;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) gt += kr[i] > tau;
-    need = keff - block_sum<NW>(gt, red, row);
+      for (int i = 0; i < PER; ++i) gt += kr[i] > tau;
+      need = keff - block_sum<NW>(gt, red, row);
+    }
   }
   // every thread has passed a barrier after loading its keys
   block_emit<NT, PER>(kr, keys, nb, k, keff, tau, need, out);
