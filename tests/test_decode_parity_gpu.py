@@ -212,6 +212,11 @@ def test_given_idx_with_oracle_indices(name, over):
     ("decode_32k", dict(batch=2)),
     ("draft_chunk_16k", dict(batch=2)),
     ("decode_1m", dict(batch=1, ctx_len=512 * 200, num_kv_heads=2, num_q_heads=8)),
+    # 8 and 16 query rows per KV head (n_q tokens x G heads): the tensor-core
+    # kernel's other row-count instantiations
+    ("draft_chunk_16k", dict(batch=3, n_q=2, num_q_heads=32, num_kv_heads=8, ctx_len=4096 + 77)),
+    ("draft_chunk_16k", dict(batch=2, n_q=4, num_q_heads=32, num_kv_heads=8, ctx_len=8192 + 5)),
+    ("draft_chunk_16k", dict(batch=2, n_q=3, num_q_heads=40, num_kv_heads=8, ctx_len=2048 + 64)),
 ])
 def test_decode_end_to_end(name, over):
     check_decode(WORKLOADS[name].scaled(**over), seed=51)

@@ -30,6 +30,7 @@
 #include "common.cuh"
 #include "decode_units.cuh"
 #include "internal.h"
+#include "select.cuh"
 #include "tc.cuh"
 
 namespace sa {
@@ -47,8 +48,10 @@ constexpr int kNumBars = 22;
 constexpr uint32_t kIdescS = tc::idesc_bf16(128, kN, false, false);
 constexpr uint32_t kIdescO = tc::idesc_bf16(128, kN, true, false);
 constexpr float kLazy = 8.f;                    // raise the running max when it grows by > 2^8
+constexpr int kMaxSelPerCta = 64;               // fused: pairs one CTA may select
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kNS) * kStage + 2 * kQBuf + 2 * kPBuf +
                               kNumBars * 8 + kNS * sizeof(StageInfo) + (2 * 4 * kN + 4 * kN) * 4 + 32;
+constexpr size_t kSmemFused = kSmemBytes;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -62,6 +65,19 @@ __device__ __forceinline__ float float_of_key(uint32_t k) {
 
 __device__ __forceinline__ void softmax_bar() {
   asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
+}
+// The same barrier, returning whether any of the softmax threads passed true.
+__device__ __forceinline__ bool softmax_bar_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(kSoftThreads)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
@@ -152,7 +168,14 @@ __device__ __forceinline__ void store_out(void* O, int64_t idx, float v) {
   else static_cast<float*>(O)[idx] = v;
 }
 
-template <bool OUT_BF16, int NR>
+// Fused mode adds the step's scoring and selection in front of the
+// attention: each CTA scores a contiguous run of the pair-major list of
+// 128-key chunks of compressed keys (cp.async.bulk through the same ring),
+// the CTA that finishes a pair's last chunk (atomic ticket) selects its top-k
+// and publishes the table with a per-pair ready flag, and the producer waits
+// for the flag of every pair before reading its table.  A cooperative launch
+// keeps every CTA resident, so the waits end.
+template <bool OUT_BF16, int NR, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                      const __grid_constant__ CUtensorMap v_map, DecodeAttnArgs a) {
@@ -179,13 +202,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* ticket = reinterpret_cast<int*>(tmem_slot + 2);
   uint64_t* mma_done = reinterpret_cast<uint64_t*>(tmem_slot + 4);    // 8-byte aligned
+  __shared__ int sel_list[kMaxSelPerCta];                               // fused: pairs this CTA selects
+  __shared__ int n_sel;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t u0 = static_cast<int64_t>(blockIdx.x) * a.tpc;
   const int64_t u1 = min(a.total_tiles, u0 + a.tpc);
   const int nunits = static_cast<int>(u1 - u0);
+  // fused: score chunks [c0, c1) of the pair-major chunk list come first and
+  // take the ring's first r0 uses
+  int c0 = 0, c1 = 0;
+  if constexpr (FUSED) {
+    const int total_chunks = a.B * a.Hkv * a.cpp;
+    c0 = min(total_chunks, static_cast<int>(blockIdx.x) * a.cpc);
+    c1 = min(total_chunks, c0 + a.cpc);
+  }
+  const int r0 = c1 - c0;
 
   if (threadIdx.x == 0) {
+    n_sel = 0;
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
@@ -239,15 +274,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     pc.init(u0, a.MT);
     int64_t pair = u0 / a.MT;
     bool stop = false;
+    if constexpr (FUSED) {
+      // this CTA's score chunks: 128 compressed keys (64 KB of fp32) each
+      for (int ci = 0; ci < r0 && !stop; ++ci) {
+        const int gc = c0 + ci;
+        const int pr = gc / a.cpp, ch = gc - pr * a.cpp;
+        const int rows = min(128, static_cast<int>(a.nb) - ch * 128);
+        const int s = ci % kNS;
+        int ok = 1;
+        if (lane == 0) {
+          if (ci >= kNS && !mbar_wait_bounded(&kv_empty[s], ((ci / kNS) & 1) ^ 1, abort_flag)) ok = 0;
+          if (ok) {
+            const uint32_t bytes = static_cast<uint32_t>(rows) * kHeadDim * 4;
+            mbar_arrive_expect_tx(&kv_full[s], bytes);
+            bulk_g2s(ring + s * kStage, a.Kc + (static_cast<int64_t>(pr) * a.nb + ch * 128) * kHeadDim, bytes,
+                     &kv_full[s]);
+          } else {
+            fail();
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) stop = true;
+      }
+    }
     for (int base = 0; base < nunits && !stop; base += 32) {
       int64_t ks0 = 0, ks1 = 0;
       int nk0 = 0, nk1 = 0;
+      bool wait_ok = true;
       if (base + lane < nunits) {
         const int64_t u = u0 + base + lane;
         const int64_t pair = u / a.MT;
         const int v = static_cast<int>(u - pair * a.MT);
-        tile_range(a, pair, 2 * v, &ks0, &nk0);
-        if (2 * v + 1 < a.n_tiles) tile_range(a, pair, 2 * v + 1, &ks1, &nk1);
+        if constexpr (FUSED) {
+          // the pair's table is published by the CTA that selected it
+          const volatile unsigned* rdy = a.ready + pair;
+          const uint64_t tw = global_ns();
+          for (uint32_t spin = 0; *rdy == 0u; ++spin) {
+            if ((spin & 63u) == 0 && (*abort_flag || global_ns() - tw > kWaitLimitNs)) {
+              wait_ok = false;
+              break;
+            }
+          }
+          __threadfence();
+          tile_range<true>(a, pair, 2 * v, &ks0, &nk0);
+          if (2 * v + 1 < a.n_tiles) tile_range<true>(a, pair, 2 * v + 1, &ks1, &nk1);
+        } else {
+          tile_range(a, pair, 2 * v, &ks0, &nk0);
+          if (2 * v + 1 < a.n_tiles) tile_range(a, pair, 2 * v + 1, &ks1, &nk1);
+        }
+      }
+      if (__any_sync(0xffffffffu, !wait_ok)) {
+        if (lane == 0) fail();
+        stop = true;
+        break;
       }
       const int cnt = min(32, nunits - base);
       for (int l = 0; l < cnt; ++l) {
@@ -256,7 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n0 = __shfl_sync(0xffffffffu, nk0, l);
         const int n1 = __shfl_sync(0xffffffffu, nk1, l);
         const int i = base + l;
-        const int s = i % kNS;
+        const int ri = r0 + i;                   // ring use
+        const int s = ri % kNS;
         const int prev_ord = pc.ordinal;
         pc.at(i);
         if (pc.ordinal != prev_ord) ++pair;
@@ -273,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc::tma_load_3d(Qs + qb * kQBuf + kN * 128, &q_map, 64, h * a.G, bi * a.n_q, &q_full[qb]);
             }
           }
-          if (ok && i >= kNS && !mbar_wait_bounded(&kv_empty[s], ((i / kNS) & 1) ^ 1, abort_flag)) ok = 0;
+          if (ok && ri >= kNS && !mbar_wait_bounded(&kv_empty[s], ((ri / kNS) & 1) ^ 1, abort_flag)) ok = 0;
           if (ok) {
             info[s].ks0 = k0;
             info[s].ks1 = k1;
@@ -315,7 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // do not leave while copies into this CTA's shared memory may be in flight
     if (lane == 0) {
-      for (int i = max(0, issued - kNS); i < issued; ++i) mbar_wait_bounded(&kv_full[i % kNS], (i / kNS) & 1, nullptr);
+      const int used = r0 + issued;
+      for (int ri = max(0, used - kNS); ri < used; ++ri) mbar_wait_bounded(&kv_full[ri % kNS], (ri / kNS) & 1, nullptr);
       for (int k = max(0, pc.ordinal - 1); k <= pc.ordinal; ++k)
         if (issued > 0) mbar_wait_bounded(&q_full[k & 1], (k >> 1) & 1, nullptr);
     }
@@ -338,8 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool did = false;
         if (ns < nunits) {
           const bool fi = cs.first(ns);
-          const int pk = cs.ordinal, qb = pk & 1, s = ns % kNS;
-          const bool ready = mbar_test_wait(&kv_full[s], (ns / kNS) & 1) &&
+          const int pk = cs.ordinal, qb = pk & 1, s = (r0 + ns) % kNS;
+          const bool ready = mbar_test_wait(&kv_full[s], ((r0 + ns) / kNS) & 1) &&
                              (!fi || mbar_test_wait(&q_full[qb], (pk >> 1) & 1)) &&
                              (ns < 2 || mbar_test_wait(&s_free[ns & 1], ((ns >> 1) + 1) & 1));
           if (__all_sync(0xffffffffu, ready)) {
@@ -365,14 +445,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                              (!fi || pk < 2 || mbar_test_wait(&o_free[ob], ((pk >> 1) + 1) & 1));
           if (__all_sync(0xffffffffu, ready)) {
             tc::fence_after_sync();
-            const uint32_t vst = ring_a + (npv % kNS) * kStage + 2 * kKVHalf;
+            const uint32_t vst = ring_a + ((r0 + npv) % kNS) * kStage + 2 * kKVHalf;
             const uint32_t pb = pa + (npv & 1) * kPBuf;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               tc::mma_bf16_elect(tbase + 32 + ob * kN, tc::smem_desc(vst + kk * 2048, kKVHalf, 1024),
                            tc::smem_desc(pb + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024), kIdescO,
                            !(fi && kk == 0));
-            tc::mma_commit_elect(&kv_empty[npv % kNS]);
+            tc::mma_commit_elect(&kv_empty[(r0 + npv) % kNS]);
             tc::mma_commit_elect(&p_free[npv & 1]);
             if (cp.last(npv, nunits)) tc::mma_commit_elect(&o_full[ob]);
             ++npv;
@@ -507,6 +587,123 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
 
+    if constexpr (FUSED) {
+      // ---- scoring: warp w scores rows 32 w .. 32 w + 31 of every chunk
+      // (q-bar = sum of the group's heads of the first new token, times the
+      // softmax scale; 8 rows per batch, a float4 per lane, shuffle sums)
+      const int sw = warp - 2;
+      const int nb = static_cast<int>(a.nb);
+      int cur = -1;
+      int seg_cnt = 0;                           // chunks of pair `cur` scored by this CTA
+      float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      // count this CTA's chunks of a pair once its run of them ends (one
+      // release fence and one atomic per run, not per chunk); the CTA that
+      // completes the pair's count selects it
+      auto close_run = [&](int pr, int n) {
+        __threadfence();
+        const unsigned old = atomicAdd(&a.score_cnt[pr], static_cast<unsigned>(n));
+        if (old + n == static_cast<unsigned>(a.cpp)) {
+          if (n_sel < kMaxSelPerCta) sel_list[n_sel++] = pr;
+          else report(a.status, kStatusTimeout);
+        }
+      };
+      for (int ci = 0; ci < r0; ++ci) {
+        const int gc = c0 + ci;
+        const int pr = gc / a.cpp, ch = gc - pr * a.cpp;
+        const int rows = min(128, nb - ch * 128);
+        const int s = ci % kNS;
+        if (pr != cur) {
+          if (t == 0 && cur >= 0) close_run(cur, seg_cnt);
+          cur = pr;
+          seg_cnt = 0;
+          const int bi = pr / a.Hkv, h = pr % a.Hkv;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int g = 0; g < G; ++g) {
+            const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(
+                static_cast<const uint16_t*>(a.Q) + (static_cast<int64_t>(bi) * a.n_q * a.Hq + h * G + g) * kHeadDim) + lane);
+            acc.x += bf16lo(w2.x);
+            acc.y += bf16hi(w2.x);
+            acc.z += bf16lo(w2.y);
+            acc.w += bf16hi(w2.y);
+          }
+          q4 = make_float4(acc.x * a.sscale, acc.y * a.sscale, acc.z * a.sscale, acc.w * a.sscale);
+        }
+        const bool got = mbar_wait_bounded(&kv_full[s], (ci / kNS) & 1, abort_flag);
+        if (got) {
+          const float* rowp = reinterpret_cast<const float*>(ring + s * kStage);
+          float* sc = a.scores + static_cast<int64_t>(pr) * nb + ch * 128;
+          // 16 rows at a time; a reduce-scatter over the lanes (each level
+          // keeps half of the rows and sends the other half to the partner
+          // lane) leaves row (lane & 15) summed over the lanes with bit 4
+          // equal, and one more exchange completes it
+          const bool b3 = lane & 8, b2 = lane & 4, b1 = lane & 2, b0 = lane & 1;
+#pragma unroll 1
+          for (int grp = 0; grp < 2; ++grp) {
+            const int rb = sw * 32 + grp * 16;
+            float d[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              // rows past the chunk hold stale data; their sums are never stored
+              const float4 v = reinterpret_cast<const float4*>(rowp + (rb + u) * kHeadDim)[lane];
+              d[u] = v.x * q4.x + v.y * q4.y + v.z * q4.z + v.w * q4.w;
+            }
+            float e8[8], e4[4], e2[2];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              e8[i] = (b3 ? d[i + 8] : d[i]) + __shfl_xor_sync(0xffffffffu, b3 ? d[i] : d[i + 8], 8);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              e4[i] = (b2 ? e8[i + 4] : e8[i]) + __shfl_xor_sync(0xffffffffu, b2 ? e8[i] : e8[i + 4], 4);
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+              e2[i] = (b1 ? e4[i + 2] : e4[i]) + __shfl_xor_sync(0xffffffffu, b1 ? e4[i] : e4[i + 2], 2);
+            float e1 = (b0 ? e2[1] : e2[0]) + __shfl_xor_sync(0xffffffffu, b0 ? e2[0] : e2[1], 1);
+            e1 += __shfl_xor_sync(0xffffffffu, e1, 16);
+            if (lane < 16 && rb + lane < rows) sc[rb + lane] = e1;
+          }
+        }
+        // every warp is done with stage s and its score stores (uniform exit)
+        if (softmax_bar_or(!got)) {
+          ok = false;
+          break;
+        }
+        if (t == 0) mbar_arrive(&kv_empty[s]);
+        ++seg_cnt;
+      }
+      if (t == 0 && ok && cur >= 0) close_run(cur, seg_cnt);
+      softmax_bar();
+      // ---- selection of the pairs whose last chunk this CTA scored (a warp each)
+      const int nsel = n_sel;
+      for (int e = sw; e < nsel && ok; e += 4) {
+        const int pr = sel_list[e];
+        __threadfence();
+        if (lane == 0) a.score_cnt[pr] = 0u;
+        const float* sc = a.scores + static_cast<int64_t>(pr) * nb;
+        // the pair's keys in registers (all loads in flight at once)
+        constexpr int PER = kFusedMaxBlocks / 32;
+        float v[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int j = i * 32 + lane;
+          v[i] = j < nb ? __ldcg(sc + j) : 0.f;
+        }
+        uint32_t kr[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int j = i * 32 + lane;
+          const int64_t lo = static_cast<int64_t>(j) * a.b, hi = lo + a.b;
+          const bool cand = j < nb && (lo < a.w_begin) && (hi > a.s_end);
+          const uint32_t key = float_key(v[i]);
+          kr[i] = cand ? (key == 0u ? 1u : key) : 0u;
+        }
+        warp_topk_regs<PER>(kr, a.top_k, a.idx_w + static_cast<int64_t>(pr) * a.top_k);
+        // publish: every lane's table entries, then the flag
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicExch(&a.ready[pr], 1u);
+      }
+    }
+
     for (int i = 0; i < nunits && ok; ++i) {
       const int prev_ord = pc.ordinal;
       pc.at(i);
@@ -519,7 +716,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_t[r] = 0.f;
         }
       }
-      const int s = i % kNS, sb = i & 1;
+      const int ri = r0 + i;                 // ring use
+      const int s = ri % kNS, sb = i & 1;
       if (!mbar_wait_bounded(&s_full[sb], (i >> 1) & 1, abort_flag)) {
         ok = false;
         break;
@@ -531,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::fence_before_sync();
       mbar_arrive(&s_free[sb]);
       // the unit's key ranges, published with the stage's full barrier
-      if (!mbar_wait_bounded(&kv_full[s], (i / kNS) & 1, abort_flag)) {
+      if (!mbar_wait_bounded(&kv_full[s], (ri / kNS) & 1, abort_flag)) {
         ok = false;
         break;
       }
@@ -620,6 +818,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tbase, 64);
   }
+  if constexpr (FUSED) {
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const unsigned done = atomicAdd(a.exit_cnt, 1u);
+      if (done == gridDim.x - 1) {
+        // every CTA is past all its flag waits: clear the flags for the next call
+        for (int p = 0; p < a.B * a.Hkv; ++p) a.ready[p] = 0u;
+        __threadfence();
+        *a.exit_cnt = 0u;
+      }
+    }
+  }
 }
 
 using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
@@ -645,53 +855,86 @@ bool decode_tc_supported(const DecodeAttnArgs& a) {
          static_cast<int64_t>(a.B) * a.n_q < (int64_t(1) << 31) && encode_fn() != nullptr;
 }
 
-cudaError_t launch_decode_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf16, cudaStream_t s) {
+namespace {
+
+bool encode_maps(const DecodeAttnArgs& a, CUtensorMap* qm, CUtensorMap* km, CUtensorMap* vm) {
   EncodeFn enc = encode_fn();
-  if (!enc) return cudaErrorNotSupported;
+  if (!enc) return false;
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUtensorMap qm, km, vm;
   {
     // Q [B * n_q tokens][Hq heads][128]: box 64 columns x G heads x n_q tokens
     cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(a.Hq), static_cast<cuuint64_t>(a.B) * a.n_q};
     cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(a.Hq) * 256};
     cuuint32_t box[3] = {64, static_cast<cuuint32_t>(a.G), static_cast<cuuint32_t>(a.n_q)};
-    if (enc(&qm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.Q), dims, strides, box, estr,
+    if (enc(qm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.Q), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
+      return false;
   }
-  {
-    // K, V [pairs][cap keys][128], rows at or past kv_end read as zeros: box 64 columns x 64 keys
-    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(a.kv_end), static_cast<cuuint64_t>(a.B) * a.Hkv};
-    cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(a.cap) * 256};
-    cuuint32_t box[3] = {64, 64, 1};
-    if (enc(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.K), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-    if (enc(&vm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.V), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
+  // K, V [pairs][cap keys][128], rows at or past kv_end read as zeros: box 64 columns x 64 keys
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(a.kv_end), static_cast<cuuint64_t>(a.B) * a.Hkv};
+  cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(a.cap) * 256};
+  cuuint32_t box[3] = {64, 64, 1};
+  if (enc(km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.K), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  return enc(vm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.V), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool FUSED>
+cudaError_t launch_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf16, cudaStream_t s) {
+  CUtensorMap qm, km, vm;
+  if (!encode_maps(a, &qm, &km, &vm)) return cudaErrorInvalidValue;
   void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, DecodeAttnArgs);
-  if (a.R <= 4) kern = out_bf16 ? decode_tc_kernel<true, 4> : decode_tc_kernel<false, 4>;
-  else if (a.R <= 8) kern = out_bf16 ? decode_tc_kernel<true, 8> : decode_tc_kernel<false, 8>;
-  else kern = out_bf16 ? decode_tc_kernel<true, 16> : decode_tc_kernel<false, 16>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
+  if (a.R <= 4) kern = out_bf16 ? decode_tc_kernel<true, 4, FUSED> : decode_tc_kernel<false, 4, FUSED>;
+  else if (a.R <= 8) kern = out_bf16 ? decode_tc_kernel<true, 8, FUSED> : decode_tc_kernel<false, 8, FUSED>;
+  else kern = out_bf16 ? decode_tc_kernel<true, 16, FUSED> : decode_tc_kernel<false, 16, FUSED>;
+  const size_t smem = FUSED ? kSmemFused : kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  if (FUSED) {
+    // every CTA resident at once: the per-pair flag waits depend on it
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = a.pdl ? 1 : 0;
+  cfg.numAttrs = (FUSED || a.pdl) ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, qm, km, vm, a);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf16, cudaStream_t s) {
+  return launch_tc<false>(a, p, out_bf16, s);
+}
+
+bool decode_fused_supported(const DecodeAttnArgs& a, int64_t nb, int lsa, int num_sms) {
+  if (lsa || nb < 1 || nb > kFusedMaxBlocks || !decode_tc_supported(a)) return false;
+  const int64_t chunks = static_cast<int64_t>(a.B) * a.Hkv * ((nb + 127) / 128);
+  // at most one CTA per SM (shared memory), at most kMaxSelPerCta tickets per CTA
+  return a.total_tiles > 0 && num_sms > 0 && (chunks + num_sms - 1) / num_sms <= kMaxSelPerCta;
+}
+
+cudaError_t launch_decode_fused(DecodeAttnArgs a, const DecodePlan& p, bool out_bf16, cudaStream_t s) {
+  a.cpp = static_cast<int>((a.nb + 127) / 128);
+  const int total_chunks = a.B * a.Hkv * a.cpp;
+  a.cpc = (total_chunks + p.grid - 1) / p.grid;
+  a.idx = a.idx_w;
+  a.idx_stride = a.top_k;
+  a.pdl = 0;
+  return launch_tc<true>(a, p, out_bf16, s);
 }
 
 }  // namespace sa

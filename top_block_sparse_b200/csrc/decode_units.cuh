@@ -17,6 +17,8 @@ struct StageInfo {
 
 // Key range of tile u (0 <= u < MT) of a pair; nkeys == 0 means empty.  The
 // index table holds valid ids or -1 (caller tables are sanitised first).
+// COHERENT: the table was written during this launch (read through L2).
+template <bool COHERENT = false>
 __device__ __forceinline__ void tile_range(const DecodeAttnArgs& a, int64_t pair, int u, int64_t* ks,
                                            int* nk) {
   int64_t s = 0, e = 0;
@@ -26,7 +28,7 @@ __device__ __forceinline__ void tile_range(const DecodeAttnArgs& a, int64_t pair
     e = min(s + T, a.s_end);
   } else if ((u -= a.n_sink_tiles) < a.idx_stride * a.tpb) {
     const int sl = u / a.tpb, sub = u - sl * a.tpb;
-    const int32_t j = __ldg(a.idx + pair * a.idx_stride + sl);
+    const int32_t j = COHERENT ? __ldcg(a.idx + pair * a.idx_stride + sl) : __ldg(a.idx + pair * a.idx_stride + sl);
     if (j >= 0) {
       const int64_t lo = max(static_cast<int64_t>(j) * a.b, a.s_end);
       const int64_t hi = min(static_cast<int64_t>(j + 1) * a.b, a.w_begin);

@@ -81,6 +81,17 @@ struct DecodeAttnArgs {
   int n_stages;
   float qscale;           // softmax scale * log2(e)
   int pdl;                // launched as a programmatic dependent of the scorer
+  // fused decode (scoring, selection and attention in one cooperative launch)
+  const float* Kc;        // [pairs, nb, 128] compressed keys
+  float* scores;          // [pairs, nb] workspace
+  unsigned* score_cnt;    // [pairs] score chunks done, zero between calls
+  unsigned* ready;        // [pairs] index table published, zero between calls
+  unsigned* exit_cnt;     // CTAs finished, zero between calls
+  int32_t* idx_w;         // [pairs, top_k] index table written by the fused kernel
+  int top_k;
+  int cpp;                // score chunks (128 compressed keys) per pair
+  int cpc;                // score chunks per CTA
+  float sscale;           // scoring scale (the softmax scale)
 };
 
 struct DecodePlan {
@@ -101,6 +112,11 @@ cudaError_t launch_decode_attn(const DecodeAttnArgs& a, const DecodePlan& p, boo
 bool decode_tc_supported(const DecodeAttnArgs& a);
 size_t decode_tc_smem_bytes();
 cudaError_t launch_decode_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf16, cudaStream_t s);
+// The whole decode step (scores, top-k, attention) in one cooperative launch
+// of the tensor-core kernel; for mean pooling and nb <= kFusedMaxBlocks.
+constexpr int kFusedMaxBlocks = 512;
+bool decode_fused_supported(const DecodeAttnArgs& a, int64_t nb, int lsa, int num_sms);
+cudaError_t launch_decode_fused(DecodeAttnArgs a, const DecodePlan& p, bool out_bf16, cudaStream_t s);
 // Copies a caller's [rows, len] index table to `out`, keeping only entries
 // that are in [0, nb) and above every earlier in-range entry of the row.
 cudaError_t launch_sanitize_idx(const int32_t* idx, int32_t* out, int rows, int len, int64_t nb,

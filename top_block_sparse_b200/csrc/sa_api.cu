@@ -101,7 +101,7 @@ float scale_of(const sa_params* p) {
 
 // Workspace layout of the decode-type ops.
 struct DecodeWs {
-  size_t score_cnt, attn_cnt, scores, idx, clean_idx, part_O, part_ml, total;
+  size_t score_cnt, attn_cnt, scores, idx, clean_idx, part_O, part_ml, ready, exit_cnt, total;
 };
 
 // idx_len: entries per row of a caller's index table (SA_OP_GIVEN_IDX).
@@ -119,7 +119,11 @@ DecodeWs decode_ws(const DecodeGeom& g, const DecodePlan& plan, int top_k, int o
   if (op == SA_OP_SCORE_TOPK || op == SA_OP_DECODE) {
     w.scores = take(pairs * static_cast<size_t>(g.nb) * 4);
   }
-  if (op == SA_OP_DECODE) w.idx = take(pairs * static_cast<size_t>(top_k) * 4);
+  if (op == SA_OP_DECODE) {
+    w.idx = take(pairs * static_cast<size_t>(top_k) * 4);
+    w.ready = take(pairs * 4);       // fused decode: per-pair table flags
+    w.exit_cnt = take(4);
+  }
   if (op == SA_OP_GIVEN_IDX) w.clean_idx = take(pairs * static_cast<size_t>(idx_len) * 4);
   if (op == SA_OP_DECODE || op == SA_OP_GIVEN_IDX) {
     const size_t slots = pairs * static_cast<size_t>(plan.n_slots) * plan.R4;
@@ -483,6 +487,26 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q, const void* K
   unsigned char* w = static_cast<unsigned char*>(ws);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + L.idx);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p->dtype == SA_BF16 && g.nb >= 1) {
+    // one cooperative launch: scores, top-k and attention
+    DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, idx, p->top_k, O, lse, w, L);
+    if (decode_fused_supported(a, g.nb, p->pool == SA_POOL_LSA, device_sms())) {
+      a.Kc = Kc;
+      a.scores = reinterpret_cast<float*>(w + L.scores);
+      a.score_cnt = reinterpret_cast<unsigned*>(w + L.score_cnt);
+      a.ready = reinterpret_cast<unsigned*>(w + L.ready);
+      a.exit_cnt = reinterpret_cast<unsigned*>(w + L.exit_cnt);
+      a.idx_w = idx;
+      a.top_k = p->top_k;
+      a.sscale = scale_of(p);
+      cudaError_t e = launch_decode_fused(a, plan, p->out_dtype == SA_BF16, s);
+      if (e == cudaSuccess) return SA_OK;
+      // a cooperative grid that cannot be resident at once (e.g. SMs taken by
+      // other work) is refused at launch: take the two-kernel path
+      if (e != cudaErrorCooperativeLaunchTooLarge) return cuda_fail(e, "fused decode launch");
+      (void)cudaGetLastError();
+    }
+  }
   ScoreArgs sa_ = score_args(p, g, Q, Kc, nullptr, idx, w, L);
   cudaError_t e = launch_score_topk_query0(sa_, p->dtype == SA_BF16, s);
   if (e != cudaSuccess) return cuda_fail(e, "score/top-k kernel launch");
