@@ -383,7 +383,7 @@ def run_ours(args, w, rank, world, local_rank):
                         "call through the C ABI, device -> pinned host copy of O; the KV cache and the "
                         "compressed keys stay resident in HBM"},
         "prefill": prefill,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": sa.decode_launches(p) * args.steps,
         "clocks": clk.summary(),
     }
     return line

@@ -173,6 +173,13 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q,
                                 void* O, float* lse, int32_t* idx_out,
                                 void* ws, size_t ws_bytes, void* stream);
 
+/* Number of kernels one sa_sparse_attn_decode call with `p` launches on this
+ * device: 1 when scoring, top-k and attention run as one cooperative launch
+ * (bf16, mean pooling, at most 512 complete blocks), else 2; 0 if p is
+ * invalid.  A cooperative launch the device refuses at run time falls back
+ * to the 2-kernel path.  Host only; launches nothing. */
+int32_t sa_decode_launches(const sa_params* p);
+
 /* Steps 1-4 for a causal prefill (select == SA_SEL_TILE_MAX, ctx_len == 0,
  * n_q = T): pools K into Kc (caller-provided, [B, Hkv, floor(T/b), d] fp32),
  * scores every query tile of b rows against the compressed keys of the

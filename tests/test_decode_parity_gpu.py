@@ -335,3 +335,10 @@ def test_full_size_sampled(name):
     w = WORKLOADS[name]
     check_decode(w, seed=91, pairs=_sampled(w), out_dtype=torch.bfloat16)
     torch.cuda.empty_cache()
+
+
+def test_decode_32k_runs_as_one_launch():
+    """The batched-decode workload takes the fused path (scores, top-k and
+    attention in one cooperative launch) on this device."""
+    assert sa.decode_launches(sa.params_for(WORKLOADS["decode_32k"])) == 1
+    assert sa.decode_launches(sa.params_for(WORKLOADS["tiny_decode"])) == 2     # fp32: two kernels

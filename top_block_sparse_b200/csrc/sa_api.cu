@@ -517,6 +517,20 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q, const void* K
   return SA_OK;
 }
 
+int32_t sa_decode_launches(const sa_params* p) {
+  if (check_params(p, false) != SA_OK) return 0;
+  DecodeGeom g;
+  DecodePlan plan;
+  if (plan_for(p, p->top_k, &g, &plan) != SA_OK) return 0;
+  if (p->dtype == SA_BF16 && g.nb >= 1) {
+    const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_DECODE);
+    DecodeAttnArgs a = attn_args(p, g, plan, nullptr, nullptr, nullptr, nullptr, p->top_k, nullptr, nullptr,
+                                 nullptr, L);
+    if (decode_fused_supported(a, g.nb, p->pool == SA_POOL_LSA, device_sms())) return 1;
+  }
+  return 2;
+}
+
 sa_status sa_sparse_attn_prefill(const sa_params* p, const void* Q, const void* K, const void* V, float* Kc,
                                  void* O, float* lse, int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
   sa_status st = check_params(p, true);

@@ -30,7 +30,8 @@ SA_FLAG_TRUSTED_IDX = 1
 
 EXPORTED = ["sa_version", "sa_workspace_size", "sa_workspace_init", "sa_pool_keys", "sa_score_topk",
             "sa_sparse_attn_given_idx", "sa_sparse_attn_decode", "sa_sparse_attn_prefill",
-            "sa_read_status", "sa_status_string", "sa_last_error", "sa_sparse_attn_given_idx_noalloc"]
+            "sa_read_status", "sa_status_string", "sa_last_error", "sa_sparse_attn_given_idx_noalloc",
+            "sa_decode_launches"]
 
 
 class SaParams(ctypes.Structure):
@@ -64,6 +65,7 @@ _sig = {
     "sa_read_status": (_i32, [_vp, _vp]),
     "sa_status_string": (ctypes.c_char_p, [_i32]),
     "sa_last_error": (ctypes.c_char_p, []),
+    "sa_decode_launches": (_i32, [_P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -184,6 +186,11 @@ def read_status(ws: torch.Tensor, stream=None) -> int:
     """Synchronises and returns (then clears) the device status of the
     workspace: SA_OK, SA_ERR_INDEX or SA_ERR_TIMEOUT."""
     return int(_lib.sa_read_status(_ptr(ws), _stream(stream)))
+
+
+def decode_launches(p: SaParams) -> int:
+    """Kernels one sparse_attn_decode call with `p` launches (1 fused, 2 split)."""
+    return int(_lib.sa_decode_launches(ctypes.byref(p)))
 
 
 def num_blocks(p: SaParams) -> int:
