@@ -156,7 +156,7 @@ def profiled_traffic(kernel_file: str, pairs: int):
         cap_pairs = int(re.search(r"captured pairs: (\d+)", text).group(1))
         if sha != src_hash(*TRAFFIC_SOURCES[kernel_file]):
             return None
-        sec = text[text.index("## `decode_tc_kernel"):]
+        sec = text[text.index("## `decode_tc_kernel<1, 4, 0>`"):]
         rd = float(re.search(r"dram__bytes_read\.sum`\) \| ([0-9.]+) Mbyte", sec).group(1))
         wr = float(re.search(r"dram__bytes_write\.sum`\) \| ([0-9.]+) Mbyte", sec).group(1))
         return (rd + wr) * 1e6 * pairs / cap_pairs
