@@ -32,6 +32,7 @@
 // (O, max, sum) to the workspace and takes an atomic ticket; the CTA that
 // arrives last for the pair merges all partials and resets the ticket.
 // Nothing ever waits on another CTA.
+#include <algorithm>
 #include <math_constants.h>
 
 #include "common.cuh"
@@ -673,6 +674,10 @@ bool plan_decode(const DecodeGeom& g, int idx_slots, bool bf16, int num_sms, Dec
   p->grid = static_cast<int>((p->total_tiles + tpc - 1) / tpc);
   if (p->grid < 1) p->grid = 1;
   p->n_slots = static_cast<int>((p->MT + tpc - 1) / tpc) + 1;
+  const int sel_tiles = idx_slots * p->tpb;
+  p->tc_plain = tc_order(g.pairs, p->n_sink_tiles, sel_tiles, p->n_wc_tiles, false, num_sms);
+  p->tc_split = tc_order(g.pairs, p->n_sink_tiles, sel_tiles, p->n_wc_tiles, true, num_sms);
+  p->n_slots = std::max(p->n_slots, std::max(p->tc_plain.slots, p->tc_split.slots));
   const size_t limit = 227 * 1024;
   int ns = 3;
   while (ns > 1 && decode_smem_bytes(p->RG, p->KG, bf16, ns) > limit) --ns;

@@ -27,6 +27,8 @@
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "decode_units.cuh"
 #include "internal.h"
@@ -43,7 +45,9 @@ constexpr int kNS = 3;                          // ring stages
 constexpr int kQBuf = 2 * kN * 128;             // two d-halves of 16 rows x 128 B
 constexpr int kPBuf = 2 * kN * 128;             // two key-halves of 16 rows x 128 B
 constexpr int kThreads = 192;
+constexpr int kThreadsFused = 256;              // fused: warps 6-7 select the top-k
 constexpr int kSoftThreads = 128;
+constexpr int kSelBarThreads = 192;             // softmax warps + selection warps
 constexpr int kNumBars = 22;
 constexpr uint32_t kIdescS = tc::idesc_bf16(128, kN, false, false);
 constexpr uint32_t kIdescO = tc::idesc_bf16(128, kN, true, false);
@@ -78,6 +82,15 @@ __device__ __forceinline__ bool softmax_bar_or(bool v) {
       : "r"(static_cast<uint32_t>(v)), "r"(kSoftThreads)
       : "memory");
   return r != 0;
+}
+
+// Named barrier 2: the softmax warps arrive once scoring is done, the
+// selection warps of the fused kernel wait for them.
+__device__ __forceinline__ void sel_bar_arrive() {
+  asm volatile("bar.arrive 2, %0;" ::"r"(kSelBarThreads) : "memory");
+}
+__device__ __forceinline__ void sel_bar_sync() {
+  asm volatile("bar.sync 2, %0;" ::"r"(kSelBarThreads) : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
@@ -140,32 +153,23 @@ __device__ __forceinline__ void tmem_stn(uint32_t taddr, const float (&v)[NR]) {
   else tmem_st16(taddr, v);
 }
 
-// Unit bookkeeping without divisions: the pair of unit i changes at
-// next_start, which advances by MT.
-struct PairCursor {
-  int next_start;   // first unit (CTA-local) of the following pair
-  int ordinal;      // pair ordinal of the current unit within this CTA
-  int MT;
-  __device__ void init(int64_t u0, int mt) {
-    MT = mt;
-    next_start = static_cast<int>((u0 / mt + 1) * mt - u0);
-    ordinal = 0;
-  }
-  // call with the unit index before using the flags of unit i (i ascending)
-  __device__ void at(int i) {
-    if (i == next_start) {
-      next_start += MT;
-      ++ordinal;
-    }
-  }
-  __device__ bool first(int i) const { return i == 0 || i == next_start - MT; }
-  __device__ bool last(int i, int nunits) const { return i == nunits - 1 || i + 1 == next_start; }
-};
-
 template <bool OUT_BF16>
 __device__ __forceinline__ void store_out(void* O, int64_t idx, float v) {
   if constexpr (OUT_BF16) static_cast<__nv_bfloat16*>(O)[idx] = __float2bfloat16_rn(v);
   else static_cast<float*>(O)[idx] = v;
+}
+// Four consecutive outputs v * s from element idx (a multiple of 4).
+template <bool OUT_BF16>
+__device__ __forceinline__ void store_out4(void* O, int64_t idx, float4 v, float s) {
+  if constexpr (OUT_BF16) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(v.x * s, v.y * s), hi = __floats2bfloat162_rn(v.z * s, v.w * s);
+    uint2 w;
+    w.x = *reinterpret_cast<uint32_t*>(&lo);
+    w.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(O) + idx) = w;
+  } else {
+    *reinterpret_cast<float4*>(static_cast<float*>(O) + idx) = make_float4(v.x * s, v.y * s, v.z * s, v.w * s);
+  }
 }
 
 // Fused mode adds the step's scoring and selection in front of the
@@ -176,7 +180,7 @@ __device__ __forceinline__ void store_out(void* O, int64_t idx, float v) {
 // for the flag of every pair before reading its table.  A cooperative launch
 // keeps every CTA resident, so the waits end.
 template <bool OUT_BF16, int NR, bool FUSED>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsFused, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                      const __grid_constant__ CUtensorMap v_map, DecodeAttnArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -206,9 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int n_sel;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t u0 = static_cast<int64_t>(blockIdx.x) * a.tpc;
-  const int64_t u1 = min(a.total_tiles, u0 + a.tpc);
-  const int nunits = static_cast<int>(u1 - u0);
+  // this CTA's units: its share of list I, then its share of list D
+  int64_t i0 = 0, d0 = 0;
+  const int nI = list_share(a.ord.totI, a.ord.gI, blockIdx.x, &i0);
+  const int nunits = nI + list_share(a.ord.totD, a.ord.gD, blockIdx.x, &d0);
   // fused: score chunks [c0, c1) of the pair-major chunk list come first and
   // take the ring's first r0 uses
   int c0 = 0, c1 = 0;
@@ -270,9 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the index table is written by the scoring kernel launched before this one
     if (a.pdl) pdl_wait_prior_grid();
     int issued = 0;
-    PairCursor pc;
-    pc.init(u0, a.MT);
-    int64_t pair = u0 / a.MT;
+    RunCursor pc;
+    pc.init(a.ord, i0, nI, d0, nunits);
     bool stop = false;
     if constexpr (FUSED) {
       // this CTA's score chunks: 128 compressed keys (64 KB of fp32) each
@@ -296,17 +300,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__shfl_sync(0xffffffffu, ok, 0)) stop = true;
       }
     }
-    for (int base = 0; base < nunits && !stop; base += 32) {
-      int64_t ks0 = 0, ks1 = 0;
-      int nk0 = 0, nk1 = 0;
+    // units in batches of up to 32 of one run: the lanes compute the key
+    // ranges together, then lane 0 issues them in order
+    for (int i = 0; i < nunits && !stop;) {
+      pc.at(i);
+      const int end = min(pc.next_start, min(nunits, i + 32));
       bool wait_ok = true;
-      if (base + lane < nunits) {
-        const int64_t u = u0 + base + lane;
-        const int64_t pair = u / a.MT;
-        const int v = static_cast<int>(u - pair * a.MT);
-        if constexpr (FUSED) {
+      if constexpr (FUSED) {
+        if (pc.in_d) {
           // the pair's table is published by the CTA that selected it
-          const volatile unsigned* rdy = a.ready + pair;
+          const volatile unsigned* rdy = a.ready + pc.pair;
           const uint64_t tw = global_ns();
           for (uint32_t spin = 0; *rdy == 0u; ++spin) {
             if ((spin & 63u) == 0 && (*abort_flag || global_ns() - tw > kWaitLimitNs)) {
@@ -315,11 +318,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           __threadfence();
-          tile_range<true>(a, pair, 2 * v, &ks0, &nk0);
-          if (2 * v + 1 < a.n_tiles) tile_range<true>(a, pair, 2 * v + 1, &ks1, &nk1);
-        } else {
-          tile_range(a, pair, 2 * v, &ks0, &nk0);
-          if (2 * v + 1 < a.n_tiles) tile_range(a, pair, 2 * v + 1, &ks1, &nk1);
         }
       }
       if (__any_sync(0xffffffffu, !wait_ok)) {
@@ -327,22 +325,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         stop = true;
         break;
       }
-      const int cnt = min(32, nunits - base);
-      for (int l = 0; l < cnt; ++l) {
+      int64_t ks0 = 0, ks1 = 0;
+      int nk0 = 0, nk1 = 0;
+      if (i + lane < end) {
+        unit_tile<FUSED>(a, pc, i + lane, 0, &ks0, &nk0);
+        unit_tile<FUSED>(a, pc, i + lane, 1, &ks1, &nk1);
+      }
+      const int64_t pair = pc.pair;
+      const int pk = pc.ordinal;
+      for (int l = 0; l < end - i; ++l) {
         const int64_t k0 = __shfl_sync(0xffffffffu, ks0, l);
         const int64_t k1 = __shfl_sync(0xffffffffu, ks1, l);
         const int n0 = __shfl_sync(0xffffffffu, nk0, l);
         const int n1 = __shfl_sync(0xffffffffu, nk1, l);
-        const int i = base + l;
-        const int ri = r0 + i;                   // ring use
+        const int ri = r0 + i + l;               // ring use
         const int s = ri % kNS;
-        const int prev_ord = pc.ordinal;
-        pc.at(i);
-        if (pc.ordinal != prev_ord) ++pair;
-        const int pk = pc.ordinal;
         int ok = 1;
         if (lane == 0) {
-          if (pc.first(i)) {
+          if (l == 0 && pc.first(i)) {
             const int qb = pk & 1;
             if (pk >= 2 && !mbar_wait_bounded(&q_empty[qb], ((pk >> 1) + 1) & 1, abort_flag)) ok = 0;
             if (ok) {
@@ -389,8 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           stop = true;
           break;
         }
-        issued = i + 1;
+        issued = i + l + 1;
       }
+      i = end;
     }
     // do not leave while copies into this CTA's shared memory may be in flight
     if (lane == 0) {
@@ -409,9 +410,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       const uint32_t ring_a = smem_u32(ring), qa = smem_u32(Qs), pa = smem_u32(Ps);
       int ns = 0, npv = 0;                  // next S / PV to issue
-      PairCursor cs, cp;                    // pair bookkeeping of units ns / npv
-      cs.init(u0, a.MT);
-      cp.init(u0, a.MT);
+      RunCursor cs, cp;                     // run bookkeeping of units ns / npv
+      cs.init(a.ord, i0, nI, d0, nunits);
+      cp.init(a.ord, i0, nI, d0, nunits);
       bool ok = true;
       uint64_t t0 = global_ns();
       for (uint32_t spin = 0; npv < nunits; ++spin) {
@@ -432,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            tc::smem_desc(qst + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024), kIdescS, kk > 0);
             tc::mma_commit_elect(&s_full[ns & 1]);
             // no later MMA reads this Q buffer for this pair
-            if (cs.last(ns, nunits)) tc::mma_commit_elect(&q_empty[qb]);
+            if (cs.last(ns)) tc::mma_commit_elect(&q_empty[qb]);
             ++ns;
             cs.at(ns);
             did = true;
@@ -454,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            !(fi && kk == 0));
             tc::mma_commit_elect(&kv_empty[(r0 + npv) % kNS]);
             tc::mma_commit_elect(&p_free[npv & 1]);
-            if (cp.last(npv, nunits)) tc::mma_commit_elect(&o_full[ob]);
+            if (cp.last(npv)) tc::mma_commit_elect(&o_full[ob]);
             ++npv;
             cp.at(npv);
             did = true;
@@ -475,6 +476,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_warp(mma_done, 0, nullptr);
     }
     __syncwarp();
+  } else if (FUSED && warp >= 6) {
+    // ------------------------------------------ top-k selection (fused only)
+    // the pairs whose last score chunk this CTA scored, a warp each, while
+    // the softmax warps attend the index-independent units
+    sel_bar_sync();
+    const int nb = static_cast<int>(a.nb);
+    const int nsel = n_sel;
+    for (int e = warp - 6; e < nsel && !*abort_flag; e += 2) {
+      const int pr = sel_list[e];
+      __threadfence();
+      if (lane == 0) a.score_cnt[pr] = 0u;
+      const float* sc = a.scores + static_cast<int64_t>(pr) * nb;
+      // the pair's keys in registers (all loads in flight at once)
+      constexpr int PER = kFusedMaxBlocks / 32;
+      float v[PER];
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int j = i * 32 + lane;
+        v[i] = j < nb ? __ldcg(sc + j) : 0.f;
+      }
+      uint32_t kr[PER];
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int j = i * 32 + lane;
+        const int64_t lo = static_cast<int64_t>(j) * a.b, hi = lo + a.b;
+        const bool cand = j < nb && (lo < a.w_begin) && (hi > a.s_end);
+        const uint32_t key = float_key(v[i]);
+        kr[i] = cand ? (key == 0u ? 1u : key) : 0u;
+      }
+      warp_topk_regs<PER>(kr, a.top_k, a.idx_w + static_cast<int64_t>(pr) * a.top_k);
+      // publish: every lane's table entries, then the flag
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) atomicExch(&a.ready[pr], 1u);
+    }
   } else {
     // ------------------------------------------------- softmax and epilogue
     const int qq = warp & 3;                  // TMEM lane quarter of this warp
@@ -489,9 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int r = 0; r < NR; ++r) poff[r] = tile * (kN * 128) + tc::sw128_off(r, kc >> 3) + (kc & 7) * 2;
     float m_run[NR], l_t[NR];
-    PairCursor pc;
-    pc.init(u0, a.MT);
-    int64_t pair = u0 / a.MT;
+    RunCursor pc;
+    pc.init(a.ord, i0, nI, d0, nunits);
     bool ok = true;
 
     auto epilogue = [&]() -> bool {
@@ -520,17 +555,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4 v = reinterpret_cast<const float4*>(lsum)[r];
         L[r] = (v.x + v.y) + (v.z + v.w);
       }
-      const int64_t first = pair * a.MT, last = first + a.MT - 1;
-      const bool whole = first >= u0 && last < u1;
-      const int64_t first_cta = first / a.tpc, last_cta = last / a.tpc;
-      const int n_ctas = static_cast<int>(last_cta - first_cta + 1);
-      const int slot = static_cast<int>(blockIdx.x - first_cta);
+      const int64_t pair = pc.pair;
+      int n_ctas, slot;
+      pair_slots(a.ord, pair, pc.in_d, &n_ctas, &slot);
       const int bi = static_cast<int>(pair / a.Hkv), h = static_cast<int>(pair % a.Hkv);
       auto out_row = [&](int r) -> int64_t {
         const int j = r / G, g = r - (r / G) * G;
         return (static_cast<int64_t>(bi) * a.n_q + j) * a.Hq + h * G + g;
       };
-      if (whole) {
+      if (n_ctas == 1) {
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
           if (r < R) {
@@ -563,22 +596,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         softmax_bar();
         if (*ticket) {
           __threadfence();
-          for (int r = 0; r < R; ++r) {
-            float M = -CUDART_INF_F;
-            for (int s2 = 0; s2 < n_ctas; ++s2)
-              M = fmaxf(M, __ldcg(a.part_ml + ((pair * a.n_slots + s2) * a.R4 + r) * 2));
-            const float Mr = (M == -CUDART_INF_F) ? 0.f : M;
-            float Ls = 0.f, acc = 0.f;
-            for (int s2 = 0; s2 < n_ctas; ++s2) {
-              const int64_t ps = (pair * a.n_slots + s2) * a.R4 + r;
-              const float sc = exp2f(__ldcg(a.part_ml + ps * 2) - Mr);
-              Ls += __ldcg(a.part_ml + ps * 2 + 1) * sc;
-              acc += __ldcg(a.part_O + ps * kHeadDim + t) * sc;
+          // thread t merges columns 4 (t % 32) .. + 3 of rows t / 32 + 4 k;
+          // the loads of up to SG slots are all in flight before their use
+          constexpr int KR = NR / 4;
+          constexpr int SG = NR >= 16 ? 2 : 4;
+          const int c4 = (t & 31) * 4, r0w = t >> 5;
+          float Mx[KR], Ls[KR];
+          float4 acc[KR];
+#pragma unroll
+          for (int k = 0; k < KR; ++k) {
+            Mx[k] = -CUDART_INF_F;
+            Ls[k] = 0.f;
+            acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          for (int s0 = 0; s0 < n_ctas; s0 += SG) {
+            float2 ml[SG][KR];
+            float4 po[SG][KR];
+#pragma unroll
+            for (int j = 0; j < SG; ++j) {
+#pragma unroll
+              for (int k = 0; k < KR; ++k) {
+                const int r = r0w + 4 * k;
+                ml[j][k] = make_float2(-CUDART_INF_F, 0.f);
+                po[j][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (s0 + j < n_ctas && r < R) {
+                  const int64_t ps = (pair * a.n_slots + s0 + j) * a.R4 + r;
+                  ml[j][k] = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + ps);
+                  po[j][k] = __ldcg(reinterpret_cast<const float4*>(a.part_O + ps * kHeadDim + c4));
+                }
+              }
             }
-            const int64_t orow = out_row(r);
-            store_out<OUT_BF16>(a.O, orow * kHeadDim + t, acc * (Ls > 0.f ? 1.f / Ls : 0.f));
-            if (t == 0 && a.lse)
-              a.lse[orow] = Ls > 0.f ? (Mr + log2f(Ls)) * 0.69314718055994531f : -CUDART_INF_F;
+#pragma unroll
+            for (int k = 0; k < KR; ++k) {
+              float mn = Mx[k];
+#pragma unroll
+              for (int j = 0; j < SG; ++j) mn = fmaxf(mn, ml[j][k].x);
+              const float mr = (mn == -CUDART_INF_F) ? 0.f : mn;
+              const float so = exp2f(Mx[k] - mr);
+              Ls[k] *= so;
+              acc[k].x *= so;
+              acc[k].y *= so;
+              acc[k].z *= so;
+              acc[k].w *= so;
+#pragma unroll
+              for (int j = 0; j < SG; ++j) {
+                const float sc = exp2f(ml[j][k].x - mr);
+                Ls[k] += ml[j][k].y * sc;
+                acc[k].x += po[j][k].x * sc;
+                acc[k].y += po[j][k].y * sc;
+                acc[k].z += po[j][k].z * sc;
+                acc[k].w += po[j][k].w * sc;
+              }
+              Mx[k] = mn;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < KR; ++k) {
+            const int r = r0w + 4 * k;
+            if (r < R) {
+              const int64_t orow = out_row(r);
+              const float inv = Ls[k] > 0.f ? 1.f / Ls[k] : 0.f;
+              store_out4<OUT_BF16>(a.O, orow * kHeadDim + c4, acc[k], inv);
+              if (c4 == 0 && a.lse)
+                a.lse[orow] = Ls[k] > 0.f ? (Mx[k] + log2f(Ls[k])) * 0.69314718055994531f : -CUDART_INF_F;
+            }
           }
           if (t == 0) a.counters[pair] = 0u;
         }
@@ -672,42 +753,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (t == 0 && ok && cur >= 0) close_run(cur, seg_cnt);
       softmax_bar();
-      // ---- selection of the pairs whose last chunk this CTA scored (a warp each)
-      const int nsel = n_sel;
-      for (int e = sw; e < nsel && ok; e += 4) {
-        const int pr = sel_list[e];
-        __threadfence();
-        if (lane == 0) a.score_cnt[pr] = 0u;
-        const float* sc = a.scores + static_cast<int64_t>(pr) * nb;
-        // the pair's keys in registers (all loads in flight at once)
-        constexpr int PER = kFusedMaxBlocks / 32;
-        float v[PER];
-#pragma unroll
-        for (int i = 0; i < PER; ++i) {
-          const int j = i * 32 + lane;
-          v[i] = j < nb ? __ldcg(sc + j) : 0.f;
-        }
-        uint32_t kr[PER];
-#pragma unroll
-        for (int i = 0; i < PER; ++i) {
-          const int j = i * 32 + lane;
-          const int64_t lo = static_cast<int64_t>(j) * a.b, hi = lo + a.b;
-          const bool cand = j < nb && (lo < a.w_begin) && (hi > a.s_end);
-          const uint32_t key = float_key(v[i]);
-          kr[i] = cand ? (key == 0u ? 1u : key) : 0u;
-        }
-        warp_topk_regs<PER>(kr, a.top_k, a.idx_w + static_cast<int64_t>(pr) * a.top_k);
-        // publish: every lane's table entries, then the flag
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) atomicExch(&a.ready[pr], 1u);
-      }
+      // sel_list is complete: hand it to the selection warps and go on
+      sel_bar_arrive();
     }
 
     for (int i = 0; i < nunits && ok; ++i) {
-      const int prev_ord = pc.ordinal;
       pc.at(i);
-      if (pc.ordinal != prev_ord) ++pair;
       const bool fi = pc.first(i);
       if (fi) {
 #pragma unroll
@@ -802,7 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::fence_proxy_async_smem();
       mbar_arrive(&p_full[sb]);
-      if (pc.last(i, nunits) && !epilogue()) {
+      if (pc.last(i) && !epilogue()) {
         ok = false;
         break;
       }
@@ -850,6 +901,34 @@ EncodeFn encode_fn() {
 
 size_t decode_tc_smem_bytes() { return kSmemBytes; }
 
+TcOrder tc_order(int64_t pairs, int n_sink_tiles, int n_sel_tiles, int n_wc_tiles, bool split, int num_sms) {
+  TcOrder o = {};
+  if (split) {
+    o.ntI = n_sink_tiles + n_wc_tiles;
+    o.ntD = n_sel_tiles;
+    o.dI = n_sel_tiles;
+    o.dD = n_sink_tiles;
+  } else {
+    o.ntD = n_sink_tiles + n_sel_tiles + n_wc_tiles;
+  }
+  o.mI = (o.ntI + 1) / 2;
+  o.mD = (o.ntD + 1) / 2;
+  o.totI = pairs * o.mI;
+  o.totD = pairs * o.mD;
+  const int64_t sms = std::max(num_sms, 1);
+  o.gI = static_cast<int>(std::min(sms, o.totI));
+  o.gD = static_cast<int>(std::min(sms, o.totD));
+  o.grid = std::max(std::max(o.gI, o.gD), 1);
+  // CTAs a run of m units can touch when every CTA holds at least q units
+  auto span = [](int m, int64_t tot, int g) -> int {
+    if (m == 0 || g == 0) return 0;
+    const int64_t q = tot / g;
+    return 1 + static_cast<int>((m - 1 + q - 1) / q);
+  };
+  o.slots = std::max(span(o.mI, o.totI, o.gI) + span(o.mD, o.totD, o.gD), 1);
+  return o;
+}
+
 bool decode_tc_supported(const DecodeAttnArgs& a) {
   return a.R >= 1 && a.R <= kN && a.kv_end < (int64_t(1) << 31) &&
          static_cast<int64_t>(a.B) * a.n_q < (int64_t(1) << 31) && encode_fn() != nullptr;
@@ -896,8 +975,8 @@ cudaError_t launch_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf1
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.gridDim = dim3(a.ord.grid);
+  cfg.blockDim = dim3(FUSED ? kThreadsFused : kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -916,21 +995,25 @@ cudaError_t launch_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf1
 
 }  // namespace
 
-cudaError_t launch_decode_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf16, cudaStream_t s) {
+cudaError_t launch_decode_tc(const DecodeAttnArgs& a0, const DecodePlan& p, bool out_bf16, cudaStream_t s) {
+  DecodeAttnArgs a = a0;
+  a.ord = p.tc_plain;
   return launch_tc<false>(a, p, out_bf16, s);
 }
 
-bool decode_fused_supported(const DecodeAttnArgs& a, int64_t nb, int lsa, int num_sms) {
+bool decode_fused_supported(const DecodeAttnArgs& a, const DecodePlan& p, int64_t nb, int lsa) {
   if (lsa || nb < 1 || nb > kFusedMaxBlocks || !decode_tc_supported(a)) return false;
   const int64_t chunks = static_cast<int64_t>(a.B) * a.Hkv * ((nb + 127) / 128);
+  const int grid = p.tc_split.grid;
   // at most one CTA per SM (shared memory), at most kMaxSelPerCta tickets per CTA
-  return a.total_tiles > 0 && num_sms > 0 && (chunks + num_sms - 1) / num_sms <= kMaxSelPerCta;
+  return a.total_tiles > 0 && grid > 0 && (chunks + grid - 1) / grid <= kMaxSelPerCta;
 }
 
 cudaError_t launch_decode_fused(DecodeAttnArgs a, const DecodePlan& p, bool out_bf16, cudaStream_t s) {
+  a.ord = p.tc_split;
   a.cpp = static_cast<int>((a.nb + 127) / 128);
   const int total_chunks = a.B * a.Hkv * a.cpp;
-  a.cpc = (total_chunks + p.grid - 1) / p.grid;
+  a.cpc = (total_chunks + a.ord.grid - 1) / a.ord.grid;
   a.idx = a.idx_w;
   a.idx_stride = a.top_k;
   a.pdl = 0;

@@ -55,6 +55,27 @@ constexpr int64_t kMaxSelectBlocks = 16384;
 cudaError_t launch_score_topk_query0(const ScoreArgs& a, bool bf16, cudaStream_t s);
 
 // ---- decode / chunk sparse attention ---------------------------------------
+// Work order of the tensor-core decode kernel: two pair-major lists of units
+// (two tiles each), each split evenly over its first g CTAs (CTA c takes
+// units [c*tot/g, (c+1)*tot/g)) and run list I first.  With `split`, list I
+// holds the tiles that need no index table (sink, window and new keys) and
+// list D the selected-block tiles, so a CTA can attend while the tables are
+// still being selected; without it list I is empty and list D is the whole
+// per-pair tile list.  Tile t of a list is tile t + off of the per-pair
+// order sink | selected | window (I: off = dI for t >= n_sink_tiles, else 0;
+// D: off = dD).  A pair's partial results take slots [0, nI) for its list-I
+// CTAs and [nI, nI + nD) for its list-D CTAs.
+struct TcOrder {
+  int mI, mD;             // units per pair
+  int ntI, ntD;           // tiles per pair
+  int dI, dD;             // tile offsets into the per-pair order
+  int gI, gD;             // CTAs sharing each list
+  int64_t totI, totD;     // units over all pairs
+  int grid;               // max(gI, gD)
+  int slots;              // partial slots a pair may need
+};
+TcOrder tc_order(int64_t pairs, int n_sink_tiles, int n_sel_tiles, int n_wc_tiles, bool split, int num_sms);
+
 struct DecodeAttnArgs {
   const void* Q;
   const void* K;
@@ -92,6 +113,7 @@ struct DecodeAttnArgs {
   int cpp;                // score chunks (128 compressed keys) per pair
   int cpc;                // score chunks per CTA
   float sscale;           // scoring scale (the softmax scale)
+  TcOrder ord;            // tensor-core kernel work order
 };
 
 struct DecodePlan {
@@ -101,6 +123,7 @@ struct DecodePlan {
   int grid, tpc, n_slots, n_stages;
   size_t smem;
   int threads;
+  TcOrder tc_plain, tc_split;   // tensor-core orders (two-kernel / fused)
 };
 // Fills `plan`; returns false (with a reason) if the shape is not built.
 bool plan_decode(const DecodeGeom& g, int idx_slots, bool bf16, int num_sms, DecodePlan* plan,
@@ -115,7 +138,7 @@ cudaError_t launch_decode_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool 
 // The whole decode step (scores, top-k, attention) in one cooperative launch
 // of the tensor-core kernel; for mean pooling and nb <= kFusedMaxBlocks.
 constexpr int kFusedMaxBlocks = 512;
-bool decode_fused_supported(const DecodeAttnArgs& a, int64_t nb, int lsa, int num_sms);
+bool decode_fused_supported(const DecodeAttnArgs& a, const DecodePlan& p, int64_t nb, int lsa);
 cudaError_t launch_decode_fused(DecodeAttnArgs a, const DecodePlan& p, bool out_bf16, cudaStream_t s);
 // Copies a caller's [rows, len] index table to `out`, keeping only entries
 // that are in [0, nb) and above every earlier in-range entry of the row.

@@ -490,7 +490,7 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q, const void* K
   if (p->dtype == SA_BF16 && g.nb >= 1) {
     // one cooperative launch: scores, top-k and attention
     DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, idx, p->top_k, O, lse, w, L);
-    if (decode_fused_supported(a, g.nb, p->pool == SA_POOL_LSA, device_sms())) {
+    if (decode_fused_supported(a, plan, g.nb, p->pool == SA_POOL_LSA)) {
       a.Kc = Kc;
       a.scores = reinterpret_cast<float*>(w + L.scores);
       a.score_cnt = reinterpret_cast<unsigned*>(w + L.score_cnt);
@@ -526,7 +526,7 @@ int32_t sa_decode_launches(const sa_params* p) {
     const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_DECODE);
     DecodeAttnArgs a = attn_args(p, g, plan, nullptr, nullptr, nullptr, nullptr, p->top_k, nullptr, nullptr,
                                  nullptr, L);
-    if (decode_fused_supported(a, g.nb, p->pool == SA_POOL_LSA, device_sms())) return 1;
+    if (decode_fused_supported(a, plan, g.nb, p->pool == SA_POOL_LSA)) return 1;
   }
   return 2;
 }
