@@ -337,6 +337,20 @@ def test_full_size_sampled(name):
     torch.cuda.empty_cache()
 
 
+def test_fused_empty_tiles_after_score_chunks():
+    """A 3-block window plus the new key gives an odd number of
+    index-independent tiles, so the last unit of each pair's run has an
+    empty second tile; at full batch every CTA first scores several chunks
+    of compressed keys through the same ring stages.  The empty tile's V rows
+    must read as zeros, not as whatever the stage last held: every output is
+    finite and sampled pairs match the oracle."""
+    w = WORKLOADS["decode_32k"].scaled(window_keys=192)
+    assert sa.decode_launches(sa.params_for(w)) == 1
+    _, _, _, O, lse, _ = check_decode(w, seed=93, pairs=_sampled(w), out_dtype=torch.bfloat16)
+    assert torch.isfinite(O.float()).all() and torch.isfinite(lse).all()
+    torch.cuda.empty_cache()
+
+
 def test_decode_32k_runs_as_one_launch():
     """The batched-decode workload takes the fused path (scores, top-k and
     attention in one cooperative launch) on this device."""

@@ -244,14 +244,11 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // V rows of a partly filled unit keep whatever the buffer held; they meet
-  // zero probabilities, so they must be finite: zero the V halves, Q and P.
+  // Q rows past the pair's R and P rows past NR only feed MMA columns that
+  // are never read; zero them once anyway.  (Every V row is written per
+  // unit: see the producer.)
   {
     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-    for (int s = 0; s < kNS; ++s) {
-      uint4* v = reinterpret_cast<uint4*>(ring + s * kStage + 2 * kKVHalf);
-      for (int i = threadIdx.x; i < 2 * kKVHalf / 16; i += kThreads) v[i] = z;
-    }
     uint4* qp = reinterpret_cast<uint4*>(Qs);
     for (int i = threadIdx.x; i < (2 * kQBuf + 2 * kPBuf) / 16; i += kThreads) qp[i] = z;
     tc::fence_proxy_async_smem();
@@ -358,28 +355,31 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
             info[s].ks1 = k1;
             info[s].n0 = n0;
             info[s].n1 = n1;
+            // Every V row of the stage meets the P^T operand (zeros for the
+            // keys of an empty tile), so an empty tile still gets V: a box
+            // at row kv_end, past the tensor map, which the copy fills with
+            // zeros without reading memory.  Stale rows could be anything
+            // (in the fused kernel, bytes of compressed keys), and 0 times a
+            // NaN is a NaN.  Its K rows are masked out of the softmax.
             const int t0 = n0 > 0, t1 = n1 > 0;
-            if (t0 + t1 > 0) {
-              unsigned char* st = ring + s * kStage;
-              const int p32 = static_cast<int>(pair);
-              mbar_arrive_expect_tx(&kv_full[s], static_cast<uint32_t>((t0 + t1) * 4 * 8192));
-              if (t0) {
-                const int r0 = static_cast<int>(k0);
-                tc::tma_load_3d(st, &k_map, 0, r0, p32, &kv_full[s]);
-                tc::tma_load_3d(st + kKVHalf, &k_map, 64, r0, p32, &kv_full[s]);
-                tc::tma_load_3d(st + 2 * kKVHalf, &v_map, 0, r0, p32, &kv_full[s]);
-                tc::tma_load_3d(st + 3 * kKVHalf, &v_map, 64, r0, p32, &kv_full[s]);
-              }
-              if (t1) {
-                const int r1 = static_cast<int>(k1);
-                tc::tma_load_3d(st + 8192, &k_map, 0, r1, p32, &kv_full[s]);
-                tc::tma_load_3d(st + kKVHalf + 8192, &k_map, 64, r1, p32, &kv_full[s]);
-                tc::tma_load_3d(st + 2 * kKVHalf + 8192, &v_map, 0, r1, p32, &kv_full[s]);
-                tc::tma_load_3d(st + 3 * kKVHalf + 8192, &v_map, 64, r1, p32, &kv_full[s]);
-              }
-            } else {
-              mbar_arrive(&kv_full[s]);
+            unsigned char* st = ring + s * kStage;
+            const int p32 = static_cast<int>(pair);
+            const int zr = static_cast<int>(a.kv_end);
+            mbar_arrive_expect_tx(&kv_full[s], static_cast<uint32_t>((t0 + t1) * 2 * 8192 + 2 * 2 * 8192));
+            const int r0 = t0 ? static_cast<int>(k0) : zr;
+            if (t0) {
+              tc::tma_load_3d(st, &k_map, 0, r0, p32, &kv_full[s]);
+              tc::tma_load_3d(st + kKVHalf, &k_map, 64, r0, p32, &kv_full[s]);
             }
+            tc::tma_load_3d(st + 2 * kKVHalf, &v_map, 0, r0, p32, &kv_full[s]);
+            tc::tma_load_3d(st + 3 * kKVHalf, &v_map, 64, r0, p32, &kv_full[s]);
+            const int r1 = t1 ? static_cast<int>(k1) : zr;
+            if (t1) {
+              tc::tma_load_3d(st + 8192, &k_map, 0, r1, p32, &kv_full[s]);
+              tc::tma_load_3d(st + kKVHalf + 8192, &k_map, 64, r1, p32, &kv_full[s]);
+            }
+            tc::tma_load_3d(st + 2 * kKVHalf + 8192, &v_map, 0, r1, p32, &kv_full[s]);
+            tc::tma_load_3d(st + 3 * kKVHalf + 8192, &v_map, 64, r1, p32, &kv_full[s]);
           } else {
             fail();
           }
