@@ -56,6 +56,15 @@ design notes of the repository):
 * R9  Multi-token chunk: the selection is made once from the chunk's FIRST
       query and reused by every token of the chunk (S3R draft chunk); token j
       of the chunk also sees chunk keys C..C+j.
+* R10 Dense verify (S3R review, "稠密验证"): every token of the chunk attends
+      causally to ALL keys 0..C+j.  The verifier's attention "mass" of a
+      complete context block is the SUM over the chunk's tokens and the KV
+      head's G query heads of the attention weights its keys receive (the
+      pages do not say how tokens and heads combine; a sum matches the
+      GQA-summed scoring of R1).  The refreshed selection is the top-k of the
+      candidate blocks by mass, with the candidates and ties of R4-R6 (the
+      KV-selection formula: recent window plus top-K by the previous verify's
+      attention scores).
 """
 from __future__ import annotations
 
@@ -308,6 +317,43 @@ def decode_pair(q_tokens: np.ndarray, K: np.ndarray, V: np.ndarray, C: int,
             wsum[j, g] = w.sum()
     return dict(Kc=Kc, qbar=qbar, scores=s, candidates=cand, sel=sel,
                 O=O, lse=lse, wsum=wsum, positions=pos_list)
+
+
+def verify_pair(q_tokens: np.ndarray, K: np.ndarray, V: np.ndarray, C: int,
+                p: OracleParams) -> Dict:
+    """Dense verify of a draft chunk for one (sequence, KV head), and the
+    block selection it refreshes (reading R10).
+
+    [S3R review, "稠密验证": the chunk's candidate tokens go through one causal
+    forward with full attention over the dense cache, and the verifier's
+    attention weights refresh the subset the drafts use; "稀疏起草",
+    KV-selection formula: recent window plus the top-K positions by the
+    previous verify's attention scores.]
+
+    q_tokens: [n_q, G, d]; token j sits at position C + j and attends to
+    keys 0..C+j.  K, V: [>= C + n_q, d].  Returns O [n_q, G, d], lse
+    [n_q, G], mass [nb] (nb = C // b complete blocks: mass_j = sum over
+    tokens j' and heads g of the weights on keys [j*b, (j+1)*b)), wtail
+    [n_q, G] (weight on the keys past the complete blocks), and the
+    Selection of the top-k candidates by mass.
+    """
+    n_q, G, d = q_tokens.shape
+    b = p.block_size
+    nb = C // b
+    scale = softmax_scale(d, p)
+    O = np.zeros((n_q, G, d))
+    lse = np.zeros((n_q, G))
+    wtail = np.zeros((n_q, G))
+    mass = np.zeros(nb)
+    for j in range(n_q):
+        pos = np.arange(C + j + 1)
+        for g in range(G):
+            O[j, g], lse[j, g], w = masked_softmax_attention(q_tokens[j, g], K, V, pos, scale)
+            mass += w[:nb * b].reshape(nb, b).sum(axis=1)
+            wtail[j, g] = w[nb * b:].sum()
+    cand = candidate_blocks(C, p)
+    sel = select_topk(mass, cand, p.top_k)
+    return dict(O=O, lse=lse, mass=mass, wtail=wtail, candidates=cand, sel=sel)
 
 
 # --------------------------------------------------------------------------

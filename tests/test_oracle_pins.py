@@ -390,6 +390,55 @@ def test_prefill_dense_equivalence_and_needles():
 
 # ---------------------------------------------- planted-mistake checks ---
 
+# ------------------------------------------------------------ dense verify ---
+
+def _verify_case(seed=21, C=2048 + 37, n_q=3, G=2):
+    w = WORKLOADS["draft_chunk_16k"].scaled(batch=1, num_kv_heads=1, num_q_heads=G, n_q=n_q,
+                                            ctx_len=C, top_k=5)
+    inp = make_inputs(w, seed=seed)
+    q, K, V = _slab(inp, 0, 0, w.group)
+    return w, inp, q, K, V
+
+
+def test_verify_mass_equals_library_softmax_block_sums():
+    """Block mass = block sums of the weights torch.softmax gives each
+    (token, head) over its causally visible keys (a library routine of the
+    same definition); O and lse equal library dense attention."""
+    w, inp, q, K, V = _verify_case()
+    C, b = w.ctx_len, w.block_size
+    r = orc.verify_pair(q, K, V, C, P(w))
+    nb = C // b
+    mass = torch.zeros(nb, dtype=torch.float64)
+    Kt, scale = torch.from_numpy(K), 1.0 / math.sqrt(128)
+    for j in range(w.n_q):
+        n = C + j + 1
+        for g in range(w.group):
+            z = Kt[:n] @ torch.from_numpy(q[j, g]) * scale
+            wt = torch.softmax(z, dim=0)
+            mass += wt[:nb * b].reshape(nb, b).sum(dim=1)
+            np.testing.assert_allclose(r["O"][j, g], _sdpa(q[j, g], K, V, n), atol=1e-12)
+            assert abs(r["lse"][j, g] - logsumexp(z.numpy())) < 1e-12
+    np.testing.assert_allclose(r["mass"], mass.numpy(), atol=1e-12, rtol=0)
+
+
+def test_verify_mass_total_needle_and_full_k():
+    """Weights of every (token, head) sum to one, so the block masses plus the
+    weight on the keys past the complete blocks total n_q * G; a block whose
+    keys point along the chunk's queries takes the most mass and is
+    selected; k >= #candidates selects every candidate."""
+    w, inp, q, K, V = _verify_case(seed=22)
+    C, b = w.ctx_len, w.block_size
+    jn = 17
+    K = K.copy()
+    K[jn * b:(jn + 1) * b] += 3.0 * q.reshape(-1, 128).mean(axis=0)
+    r = orc.verify_pair(q, K, V, C, P(w))
+    assert abs(r["mass"].sum() + r["wtail"].sum() - w.n_q * w.group) < 1e-12
+    assert int(np.argmax(r["mass"])) == jn and jn in r["sel"].selected
+    assert len(r["sel"].selected) == 5
+    r_all = orc.verify_pair(q, K, V, C, P(w, top_k=10_000))
+    assert r_all["sel"].selected == orc.candidate_blocks(C, P(w))
+
+
 def _fails(fn):
     try:
         fn()
@@ -427,7 +476,34 @@ def test_planted_mistakes_are_caught(monkeypatch):
     with monkeypatch.context() as m:
         m.setattr(orc, "softmax_scale", lambda d, p: 1.0 / d)
         assert _fails(lambda: test_hand_worked_decode("decode_k1"))
+    # verify mass of the first token only, or without the causal mask
+    orig_verify = orc.verify_pair
+
+    def mass_first_token(q, K, V, C, p):
+        r = orig_verify(q, K, V, C, p)
+        r["mass"] = orig_verify(q[:1], K, V, C, p)["mass"]
+        return r
+    for bad in (mass_first_token,
+                lambda q, K, V, C, p: _verify_noncausal(q, K, V, C, p)):
+        with monkeypatch.context() as m:
+            m.setattr(orc, "verify_pair", bad)
+            assert _fails(test_verify_mass_equals_library_softmax_block_sums)
     # summed chunk queries instead of the chunk's first query for selection
     with monkeypatch.context() as m:
         m.setattr(orc, "index_query", lambda qg: np.asarray(qg, float).sum(axis=0) * 0.0)
         assert _fails(test_needles_selected_tiny_decode)
+
+
+def _verify_noncausal(q, K, V, C, p):
+    """verify_pair with every token seeing the whole chunk (a planted mistake)."""
+    n_q, G, d = q.shape
+    b = p.block_size
+    nb = C // b
+    scale = orc.softmax_scale(d, p)
+    O, lse, mass = np.zeros((n_q, G, d)), np.zeros((n_q, G)), np.zeros(nb)
+    pos = np.arange(C + n_q)
+    for j in range(n_q):
+        for g in range(G):
+            O[j, g], lse[j, g], wt = orc.masked_softmax_attention(q[j, g], K, V, pos, scale)
+            mass += wt[:nb * b].reshape(nb, b).sum(axis=1)
+    return dict(O=O, lse=lse, mass=mass, wtail=None, candidates=None, sel=None)
