@@ -82,7 +82,8 @@ enum {                                            /* ops for sa_workspace_size *
   SA_OP_SCORE_TOPK = 0,
   SA_OP_GIVEN_IDX = 1,
   SA_OP_DECODE = 2,
-  SA_OP_PREFILL = 3
+  SA_OP_PREFILL = 3,
+  SA_OP_VERIFY = 4
 };
 
 /* Problem description shared by every entry point (88 bytes). */
@@ -172,6 +173,39 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q,
                                 const void* K, const void* V, const float* Kc,
                                 void* O, float* lse, int32_t* idx_out,
                                 void* ws, size_t ws_bytes, void* stream);
+
+/* Dense verify of a draft chunk and the block selection it refreshes
+ * (S3R review, section "稠密验证": the chunk's tokens go through one causal
+ * forward with full attention over the dense cache, and the verifier's
+ * attention weights refresh the subset the drafts read; section "稀疏起草",
+ * KV-selection formula: recent window plus the top-K positions by the
+ * previous verify's attention scores).
+ *
+ * The n_q tokens at positions C..C+n_q-1 (Q [B, n_q, Hq, d], their keys
+ * already at rows C.. of K and V) attend causally to EVERY key 0..C+j: no
+ * selection, sink_keys and window_keys do not restrict it.  Outputs:
+ *   O       [B, n_q, Hq, d] in out_dtype, lse [B, n_q, Hq] fp32 (natural
+ *           log; may be NULL);
+ *   mass    [B, Hkv, nb] fp32, nb = C / block_size: for each complete context
+ *           block, the attention weight its keys receive summed over the n_q
+ *           tokens and the KV head's G query heads (so the masses of a pair
+ *           plus the weight on the keys past the complete blocks total
+ *           n_q * G);
+ *   idx_out [B, Hkv, top_k] int32: the top_k candidate blocks by mass
+ *           (candidates and ties as in sa_score_topk: blocks not wholly
+ *           inside [0, sink_keys) or the last window_keys context keys;
+ *           higher mass first, then the lower block id), ascending, -1
+ *           padded; may be NULL when top_k == 0.
+ * Built for dtype SA_BF16, block_size a multiple of 64, n_q * (Hq / Hkv)
+ * <= 16 rows per KV head (else SA_ERR_UNSUPPORTED); pool fields are
+ * ignored; select must be SA_SEL_QUERY0.  Device buffers, 16-byte aligned;
+ * the caller owns all of them, the workspace (sa_workspace_size(p,
+ * SA_OP_VERIFY)) included.  Asynchronous on `stream`: three launches (dense
+ * attention, block mass, top-k) plus a memset of mass. */
+sa_status sa_verify_refresh(const sa_params* p, const void* Q, const void* K,
+                            const void* V, void* O, float* lse, float* mass,
+                            int32_t* idx_out, void* ws, size_t ws_bytes,
+                            void* stream);
 
 /* Number of kernels one sa_sparse_attn_decode call with `p` launches on this
  * device: 1 when scoring, top-k and attention run as one cooperative launch

@@ -108,6 +108,34 @@ def test_given_idx_validation():
     assert st == sa.SA_ERR_INVALID
 
 
+def _verify(p, ws_bytes=1 << 30, mass=FAKE, idx=FAKE):
+    return sa.raw_call("sa_verify_refresh", ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, mass, idx,
+                       FAKE, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dtype="f32"), sa.SA_ERR_UNSUPPORTED),          # tensor cores: bf16 only
+    (dict(block_size=32), sa.SA_ERR_UNSUPPORTED),        # mass tiles are 64 keys
+    (dict(n_q=5), sa.SA_ERR_UNSUPPORTED),                # 5 tokens x GQA 4 = 20 rows > 16
+    (dict(head_dim=64), sa.SA_ERR_UNSUPPORTED),
+    (dict(prefill=True), sa.SA_ERR_INVALID),
+])
+def test_verify_validation_rejects(kw, status):
+    assert _verify(_p(**kw)) == status
+    assert sa.raw_call("sa_last_error").decode() != ""
+
+
+def test_verify_null_arguments_and_workspace():
+    p = _p(n_q=3, num_q_heads=4, num_kv_heads=2)
+    assert _verify(p, mass=None) == sa.SA_ERR_INVALID
+    assert _verify(p, idx=None) == sa.SA_ERR_INVALID      # top_k > 0 needs idx_out
+    need = sa.workspace_size(p, sa.SA_OP_VERIFY)
+    assert need > 0
+    assert _verify(p, ws_bytes=need - 1) == sa.SA_ERR_WORKSPACE
+    # larger batch, larger workspace; the verify workspace holds the rows' lse
+    assert sa.workspace_size(_p(n_q=3, num_q_heads=4, num_kv_heads=2, batch=8), sa.SA_OP_VERIFY) > need
+
+
 def test_status_strings():
     for code, name in [(0, "SA_OK"), (4, "SA_ERR_INDEX"), (6, "SA_ERR_TIMEOUT")]:
         assert sa.raw_call("sa_status_string", code).decode() == name

@@ -145,6 +145,26 @@ cudaError_t launch_decode_fused(DecodeAttnArgs a, const DecodePlan& p, bool out_
 cudaError_t launch_sanitize_idx(const int32_t* idx, int32_t* out, int rows, int len, int64_t nb,
                                 unsigned* status, cudaStream_t s);
 
+// ---- dense verify: block attention mass and the refreshed selection --------
+struct BlockMassArgs {
+  const void* Q;          // [B, n_q, Hq, 128] bf16
+  const void* K;          // [pairs, cap, 128] bf16
+  const float* lse;       // [B, n_q, Hq] natural-log row sums of the dense attention
+  float* mass;            // [pairs, nb], zeroed before the launch (tiles add to it)
+  unsigned* status;
+  int B, Hq, Hkv, G, n_q, R;
+  int64_t cap, kv_end;
+  int b, nb;
+  int tiles;              // 64-key tiles of the complete blocks, nb * b / 64
+  int units;              // two tiles each, per pair
+  int upc, cpp;           // units per CTA, CTAs per pair (set by the launcher)
+  float qscale;           // softmax scale * log2(e)
+};
+bool block_mass_supported(const BlockMassArgs& a);
+cudaError_t launch_block_mass(BlockMassArgs a, int num_sms, cudaStream_t s);
+cudaError_t launch_mass_topk(const float* mass, int pairs, int nb, int b, int64_t s_end, int64_t w_begin, int k,
+                             int32_t* idx, cudaStream_t s);
+
 // ---- prefill (tensor cores) -------------------------------------------------
 struct PrefillArgs {
   const void* Q;          // [B, T, Hq, 128] bf16

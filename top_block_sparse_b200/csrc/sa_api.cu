@@ -321,7 +321,40 @@ const char* sa_status_string(sa_status s) {
   return "SA_ERR_UNKNOWN";
 }
 
+// ---- dense verify -----------------------------------------------------------
+// The dense pass is the decode attention with the whole context as its window
+// and no table: every token sees keys 0..C+j.
+sa_params verify_dense_params(const sa_params* p) {
+  sa_params d = *p;
+  d.sink_keys = 0;
+  d.window_keys = p->ctx_len;
+  d.top_k = 0;
+  d.flags = SA_FLAG_TRUSTED_IDX;
+  return d;
+}
+
+struct VerifyWs {
+  DecodeWs attn;          // the dense attention's workspace (status, tickets, partials)
+  size_t lse, total;      // lse of the rows when the caller passes none
+};
+
+VerifyWs verify_ws(const DecodeGeom& g, const DecodePlan& plan) {
+  VerifyWs w;
+  w.attn = decode_ws(g, plan, 0, SA_OP_GIVEN_IDX, 0);
+  w.lse = align_up(w.attn.total, 256);
+  w.total = w.lse + static_cast<size_t>(g.B) * g.n_q * g.Hq * 4;
+  return w;
+}
+
 size_t sa_workspace_size(const sa_params* p, int32_t op) {
+  if (op == SA_OP_VERIFY) {
+    if (check_params(p, false) != SA_OK) return 0;
+    const sa_params d = verify_dense_params(p);
+    DecodeGeom g;
+    DecodePlan plan;
+    if (plan_for(&d, 0, &g, &plan) != SA_OK) return 0;
+    return verify_ws(g, plan).total;
+  }
   const bool prefill = (op == SA_OP_PREFILL) || (p && p->select == SA_SEL_TILE_MAX);
   if (check_params(p, prefill) != SA_OK) return 0;
   if (prefill) {
@@ -514,6 +547,72 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q, const void* K
   a.pdl = 1;
   e = launch_decode_attn(a, plan, p->dtype == SA_BF16, p->out_dtype == SA_BF16, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+  return SA_OK;
+}
+
+sa_status sa_verify_refresh(const sa_params* p, const void* Q, const void* K, const void* V, void* O, float* lse,
+                            float* mass, int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  sa_status st = check_params(p, false);
+  if (st != SA_OK) return st;
+  if (!Q || !K || !V || !O || !mass) return fail(SA_ERR_INVALID, "Q, K, V, O and mass must be non-NULL");
+  if (p->top_k > 0 && !idx_out) return fail(SA_ERR_INVALID, "idx_out is NULL with top_k > 0");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return fail(SA_ERR_INVALID, "Q, K, V and O must be 16-byte aligned");
+  if (p->dtype != SA_BF16) return fail(SA_ERR_UNSUPPORTED, "verify runs on bf16 tensor cores: dtype must be SA_BF16");
+  if (p->block_size % 64 != 0) return fail(SA_ERR_UNSUPPORTED, "verify block mass needs block_size a multiple of 64");
+  const sa_params d = verify_dense_params(p);
+  DecodeGeom g;
+  DecodePlan plan;
+  if ((st = plan_for(&d, 0, &g, &plan)) != SA_OK) return st;
+  const DecodeGeom gs = decode_geom(p);          // the caller's sink and window: the candidates
+  if (gs.nb > kMaxSelectBlocks)
+    return fail(SA_ERR_UNSUPPORTED, "%lld blocks per sequence exceed the %lld the selector handles",
+                (long long)gs.nb, (long long)kMaxSelectBlocks);
+  const VerifyWs L = verify_ws(g, plan);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != SA_OK) return st;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* lse_rows = lse ? lse : reinterpret_cast<float*>(w + L.lse);
+
+  BlockMassArgs m = {};
+  m.Q = Q;
+  m.K = K;
+  m.lse = lse_rows;
+  m.mass = mass;
+  m.status = reinterpret_cast<unsigned*>(w);
+  m.B = g.B;
+  m.Hq = g.Hq;
+  m.Hkv = g.Hkv;
+  m.G = g.G;
+  m.n_q = g.n_q;
+  m.R = g.R;
+  m.cap = g.cap;
+  m.kv_end = g.kv_end;
+  m.b = g.b;
+  m.nb = static_cast<int>(gs.nb);
+  m.tiles = static_cast<int>(gs.nb * g.b / 64);
+  m.units = (m.tiles + 1) / 2;
+  m.qscale = scale_of(p) * 1.4426950408889634f;
+  if (!block_mass_supported(m))
+    return fail(SA_ERR_UNSUPPORTED, "verify block mass needs n_q * G <= 16 rows per KV head");
+
+  // 1. dense attention (O, lse)
+  DecodeAttnArgs a = attn_args(&d, g, plan, Q, K, V, nullptr, 0, O, lse_rows, w, L.attn);
+  a.pdl = 0;
+  cudaError_t e = launch_decode_attn(a, plan, true, p->out_dtype == SA_BF16, s);
+  if (e != cudaSuccess) return cuda_fail(e, "dense attention launch");
+  // 2. block mass (tiles add into a cleared array)
+  if (gs.nb > 0) {
+    e = cudaMemsetAsync(mass, 0, static_cast<size_t>(g.pairs) * gs.nb * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    e = launch_block_mass(m, device_sms(), s);
+    if (e != cudaSuccess) return cuda_fail(e, "block mass launch");
+  }
+  // 3. the refreshed selection: top-k candidates by mass
+  if (p->top_k > 0) {
+    e = launch_mass_topk(mass, g.pairs, static_cast<int>(gs.nb), g.b, gs.s_end, gs.w_begin, p->top_k, idx_out, s);
+    if (e != cudaSuccess) return cuda_fail(e, "mass top-k launch");
+  }
   return SA_OK;
 }
 

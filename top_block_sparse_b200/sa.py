@@ -25,13 +25,13 @@ SA_OK, SA_ERR_INVALID, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_INDEX, SA_ER
 SA_F32, SA_BF16 = 0, 1
 SA_POOL_MEAN, SA_POOL_LSA = 0, 1
 SA_SEL_QUERY0, SA_SEL_TILE_MAX = 0, 1
-SA_OP_SCORE_TOPK, SA_OP_GIVEN_IDX, SA_OP_DECODE, SA_OP_PREFILL = 0, 1, 2, 3
+SA_OP_SCORE_TOPK, SA_OP_GIVEN_IDX, SA_OP_DECODE, SA_OP_PREFILL, SA_OP_VERIFY = 0, 1, 2, 3, 4
 SA_FLAG_TRUSTED_IDX = 1
 
 EXPORTED = ["sa_version", "sa_workspace_size", "sa_workspace_init", "sa_pool_keys", "sa_score_topk",
             "sa_sparse_attn_given_idx", "sa_sparse_attn_decode", "sa_sparse_attn_prefill",
             "sa_read_status", "sa_status_string", "sa_last_error", "sa_sparse_attn_given_idx_noalloc",
-            "sa_decode_launches"]
+            "sa_decode_launches", "sa_verify_refresh"]
 
 
 class SaParams(ctypes.Structure):
@@ -66,6 +66,7 @@ _sig = {
     "sa_status_string": (ctypes.c_char_p, [_i32]),
     "sa_last_error": (ctypes.c_char_p, []),
     "sa_decode_launches": (_i32, [_P]),
+    "sa_verify_refresh": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -180,6 +181,13 @@ def sparse_attn_prefill(p: SaParams, Q, K, V, Kc, O, lse=None, idx_out=None, ws=
     _check(_lib.sa_sparse_attn_prefill(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kc), _ptr(O),
                                        _ptr(lse), _ptr(idx_out), _ptr(ws),
                                        0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def verify_refresh(p: SaParams, Q, K, V, O, mass, lse=None, idx_out=None, ws=None, stream=None):
+    """Dense verify of a draft chunk: O, lse, per-block attention mass and the
+    top_k blocks by mass (sa_verify_refresh)."""
+    _check(_lib.sa_verify_refresh(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse), _ptr(mass),
+                                  _ptr(idx_out), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def read_status(ws: torch.Tensor, stream=None) -> int:
