@@ -1,7 +1,7 @@
 """Benchmark of the sparse-attention decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_32k] [--no-cpu-baseline] [--no-prefill]
+                    [--workload decode_32k] [--no-cpu-baseline] [--no-prefill] [--no-verify]
 
 Workload (default): batched decode, batch 32, 32 query / 8 KV heads, d = 128,
 context T = 32768, bf16 KV cache with fp32 accumulation, block 64, top-k 32 +
@@ -22,7 +22,8 @@ data path); the per-rank device times are max-reduced.
 Printed: one JSON line (rank 0).  ``value`` = sequences decoded per second
 (whole job).  Also: the roofline of the step's one kernel (algorithmic bytes
 over the timed launch, against the measured copy bandwidth), the attention
-kernel alone on the same table, the end-to-end number
+kernel alone on the same table, the causal prefill and the dense verify of
+a draft chunk (each with its kernels' rooflines), the end-to-end number
 through the C ABI with host buffers, clocks sampled during the timed region,
 and the float64 CPU oracle timed on a bounded sample (rank 0, N = 1).
 """
@@ -352,6 +353,10 @@ def run_ours(args, w, rank, world, local_rank):
     prefill = None
     if not args.no_prefill:
         prefill = run_prefill_bench(args, dev, stream, flush)
+    # --- dense verify of a draft chunk, rank-local ----------------------------
+    verify = None
+    if not args.no_verify:
+        verify = run_verify_bench(args, dev, stream, flush)
     # --- end to end through the C ABI with host buffers -------------------
     e2e = e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush)
     if world > 1:
@@ -398,6 +403,7 @@ def run_ours(args, w, rank, world, local_rank):
                         "call through the C ABI, device -> pinned host copy of O; the KV cache and the "
                         "compressed keys stay resident in HBM"},
         "prefill": prefill,
+        "verify": verify,
         "gpu_launches": sa.decode_launches(p) * args.steps,
         "clocks": clk.summary(),
     }
@@ -496,6 +502,65 @@ def run_prefill_bench(args, dev, stream, flush):
     }
 
 
+def run_verify_bench(args, dev, stream, flush):
+    """Times the dense verify of a draft chunk (sa_verify_refresh) on the
+    draft-chunk workload with the chunk's 6 tokens plus one (n_q = 7), and
+    the dense attention alone (the same kernel through
+    sa_sparse_attn_given_idx with the whole context as window)."""
+    from top_block_sparse_b200 import sa
+    w = WORKLOADS["draft_chunk_16k"].scaled(n_q=7)
+    if args.batch:
+        w = w.scaled(batch=args.batch)
+    inp = make_inputs(w, seed=3001, device=dev)
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    del inp
+    p = sa.params_for(w, out_dtype="bf16")
+    nb = w.ctx_len // w.block_size
+    O = torch.empty((w.batch, w.n_q, w.num_q_heads, 128), device=dev, dtype=torch.bfloat16)
+    lse = torch.empty((w.batch, w.n_q, w.num_q_heads), device=dev)
+    mass = torch.empty((w.batch, w.num_kv_heads, nb), device=dev)
+    idx = torch.empty((w.batch, w.num_kv_heads, w.top_k), device=dev, dtype=torch.int32)
+    ws = sa.alloc_workspace(p, sa.SA_OP_VERIFY, device=dev)
+    pd = sa.params_for(w, out_dtype="bf16")
+    pd.sink_keys, pd.window_keys, pd.top_k, pd.flags = 0, w.ctx_len, 0, sa.SA_FLAG_TRUSTED_IDX
+    ws_d = sa.alloc_workspace(pd, sa.SA_OP_GIVEN_IDX, device=dev)
+
+    def full():
+        sa.verify_refresh(p, Q, K, V, O, mass, lse, idx, ws, stream=stream)
+
+    def dense():
+        sa.sparse_attn_given_idx(pd, Q, K, V, None, O, lse, ws_d, stream=stream)
+
+    n = args.verify_steps
+    full_ms = statistics.mean(timed_steps(full, n, 3, stream, flush))
+    dense_ms = statistics.mean(timed_steps(dense, n, 3, stream, flush))
+    if sa.read_status(ws, stream) != sa.SA_OK:
+        raise RuntimeError("device status word set during the verify runs")
+    hbm, _, _, src = peaks()
+    pairs = w.batch * w.num_kv_heads
+    kv = w.ctx_len + w.n_q
+    qo = 2 * w.batch * w.n_q * w.num_q_heads * 128 * 2
+    alg = pairs * kv * 128 * 2 * 2 + qo + pairs * nb * 4 + pairs * w.top_k * 4
+    k_blocks = pairs * nb * w.block_size * 128 * 2          # K of the complete blocks, read again for the mass
+    return {
+        "workload": f"draft_chunk_16k dense verify: B={w.batch}, n_q={w.n_q} (6 draft tokens + 1), Hq={w.num_q_heads}, "
+                    f"Hkv={w.num_kv_heads}, C={w.ctx_len}, d=128, bf16, block 64, refreshed top-k {w.top_k}",
+        "ms": full_ms,
+        "algorithmic_bytes": alg,
+        "achieved_gbs": alg / (full_ms * 1e-3) / 1e9,
+        "frac": alg / (full_ms * 1e-3) / 1e9 / hbm,
+        "note": "algorithmic bytes = every K and V row once + Q, O, mass, table; the block-mass pass reads K "
+                "of the complete blocks a second time (executed, not algorithmic)",
+        "dense_attention": {"kernel": "decode_tc_kernel (the whole context as window)", "ms": dense_ms,
+                            "gbs": (pairs * kv * 128 * 2 * 2 + qo) / (dense_ms * 1e-3) / 1e9,
+                            "frac": (pairs * kv * 128 * 2 * 2 + qo) / (dense_ms * 1e-3) / 1e9 / hbm},
+        "mass_and_topk": {"kernel": "block_mass_kernel (tcgen05) + mass_topk_kernel",
+                          "ms": full_ms - dense_ms,
+                          "k_gbs": k_blocks / ((full_ms - dense_ms) * 1e-3) / 1e9},
+        "peak_gbs": hbm, "peak_source": src,
+    }
+
+
 def e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush):
     from top_block_sparse_b200 import sa
     C = w.ctx_len
@@ -536,6 +601,8 @@ def main():
     ap.add_argument("--ref-pairs", type=int, default=4)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--prefill-steps", type=int, default=10)
+    ap.add_argument("--verify-steps", type=int, default=10)
+    ap.add_argument("--no-verify", action="store_true")
     ap.add_argument("--prefill-tokens", type=int, default=None,
                     help="override the prefill length (smaller cases for ncu captures)")
     ap.add_argument("--batch", type=int, default=None,
