@@ -200,8 +200,9 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q,
  * <= 16 rows per KV head (else SA_ERR_UNSUPPORTED); pool fields are
  * ignored; select must be SA_SEL_QUERY0.  Device buffers, 16-byte aligned;
  * the caller owns all of them, the workspace (sa_workspace_size(p,
- * SA_OP_VERIFY)) included.  Asynchronous on `stream`: three launches (dense
- * attention, block mass, top-k) plus a memset of mass. */
+ * SA_OP_VERIFY)) included.  Asynchronous on `stream`: three launches (the
+ * dense attention, which also keeps per-32-key row sums of the complete
+ * blocks, the block masses, the top-k); K and V are read once. */
 sa_status sa_verify_refresh(const sa_params* p, const void* Q, const void* K,
                             const void* V, void* O, float* lse, float* mass,
                             int32_t* idx_out, void* ws, size_t ws_bytes,

@@ -179,7 +179,7 @@ __device__ __forceinline__ void store_out4(void* O, int64_t idx, float4 v, float
 // and publishes the table with a per-pair ready flag, and the producer waits
 // for the flag of every pair before reading its table.  A cooperative launch
 // keeps every CTA resident, so the waits end.
-template <bool OUT_BF16, int NR, bool FUSED>
+template <bool OUT_BF16, int NR, bool FUSED, bool MASS>
 __global__ void __launch_bounds__(kThreadsFused, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                      const __grid_constant__ CUtensorMap v_map, DecodeAttnArgs a) {
@@ -785,6 +785,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         break;
       }
       const int n = tile ? info[s].n1 : info[s].n0;
+      const int64_t kst = tile ? info[s].ks1 : info[s].ks0;
       const int dnew = static_cast<int>(tile ? info[s].ks1 : info[s].ks0) + kc - C;   // >= 0: a new key
       const int dn = dnew < 0 ? -1 : min(dnew, 64);
       const bool kv = kc < n;
@@ -845,14 +846,47 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         break;
       }
       unsigned char* pbuf = Ps + sb * kPBuf;
+      float pm[NR];
 #pragma unroll
       for (int r = 0; r < NR; ++r) {
         const float p = ex2(x[r] - (m_run[r] == -CUDART_INF_F ? 0.f : m_run[r]));
+        pm[r] = p;
         l_t[r] += p;
         *reinterpret_cast<__nv_bfloat16*>(pbuf + poff[r]) = __float2bfloat16_rn(p);
       }
       tc::fence_proxy_async_smem();
       mbar_arrive(&p_full[sb]);
+      if constexpr (MASS) {
+        // dense verify: this warp's 32 keys, when they are keys of the tile
+        // (an empty tile has no key range) and lie in the complete blocks
+        // (the dense mode's tiles start at multiples of 64): each row's
+        // probability sum, reduce-scattered so that lane r holds row r
+        const int64_t k32 = kst + (qq & 1) * 32;
+        if (n >= (qq & 1) * 32 + 32 && k32 + 32 <= a.mass_keys) {
+          float d[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) d[u] = u < NR ? pm[u] : 0.f;
+          const bool b3 = lane & 8, b2 = lane & 4, b1 = lane & 2, b0 = lane & 1;
+          float e8[8], e4[4], e2[2];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            e8[u] = (b3 ? d[u + 8] : d[u]) + __shfl_xor_sync(0xffffffffu, b3 ? d[u] : d[u + 8], 8);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            e4[u] = (b2 ? e8[u + 4] : e8[u]) + __shfl_xor_sync(0xffffffffu, b2 ? e8[u] : e8[u + 4], 4);
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+            e2[u] = (b1 ? e4[u + 2] : e4[u]) + __shfl_xor_sync(0xffffffffu, b1 ? e4[u] : e4[u + 2], 2);
+          float e1 = (b0 ? e2[1] : e2[0]) + __shfl_xor_sync(0xffffffffu, b0 ? e2[0] : e2[1], 1);
+          e1 += __shfl_xor_sync(0xffffffffu, e1, 16);
+          const int r = lane & 15;
+          float mr = 0.f;
+#pragma unroll
+          for (int u = 0; u < NR; ++u) mr = (u == r && m_run[u] != -CUDART_INF_F) ? m_run[u] : mr;
+          if (lane < 16 && r < R)
+            a.mass_part[(pc.pair * a.mass_hts + k32 / 32) * 16 + r] = make_float2(e1, mr);
+        }
+      }
       if (pc.last(i) && !epilogue()) {
         ok = false;
         break;
@@ -968,9 +1002,18 @@ cudaError_t launch_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf1
   CUtensorMap qm, km, vm;
   if (!encode_maps(a, &qm, &km, &vm)) return cudaErrorInvalidValue;
   void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, DecodeAttnArgs);
-  if (a.R <= 4) kern = out_bf16 ? decode_tc_kernel<true, 4, FUSED> : decode_tc_kernel<false, 4, FUSED>;
-  else if (a.R <= 8) kern = out_bf16 ? decode_tc_kernel<true, 8, FUSED> : decode_tc_kernel<false, 8, FUSED>;
-  else kern = out_bf16 ? decode_tc_kernel<true, 16, FUSED> : decode_tc_kernel<false, 16, FUSED>;
+  if (!FUSED && a.mass_part) {
+    // dense verify: the row sums of the complete blocks ride along
+    if (a.R <= 4) kern = out_bf16 ? decode_tc_kernel<true, 4, false, true> : decode_tc_kernel<false, 4, false, true>;
+    else if (a.R <= 8) kern = out_bf16 ? decode_tc_kernel<true, 8, false, true> : decode_tc_kernel<false, 8, false, true>;
+    else kern = out_bf16 ? decode_tc_kernel<true, 16, false, true> : decode_tc_kernel<false, 16, false, true>;
+  } else if (a.R <= 4) {
+    kern = out_bf16 ? decode_tc_kernel<true, 4, FUSED, false> : decode_tc_kernel<false, 4, FUSED, false>;
+  } else if (a.R <= 8) {
+    kern = out_bf16 ? decode_tc_kernel<true, 8, FUSED, false> : decode_tc_kernel<false, 8, FUSED, false>;
+  } else {
+    kern = out_bf16 ? decode_tc_kernel<true, 16, FUSED, false> : decode_tc_kernel<false, 16, FUSED, false>;
+  }
   const size_t smem = FUSED ? kSmemFused : kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;

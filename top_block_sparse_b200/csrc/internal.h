@@ -114,6 +114,11 @@ struct DecodeAttnArgs {
   int cpc;                // score chunks per CTA
   float sscale;           // scoring scale (the softmax scale)
   TcOrder ord;            // tensor-core kernel work order
+  // dense verify: per 32-key half-tile of the complete blocks and query row,
+  // (sum of the row's probabilities, the running max they are taken against)
+  float2* mass_part;      // [pairs, mass_hts, 16], or null
+  int64_t mass_keys;      // keys of the complete blocks, nb * b
+  int mass_hts;           // mass_keys / 32
 };
 
 struct DecodePlan {
@@ -146,22 +151,10 @@ cudaError_t launch_sanitize_idx(const int32_t* idx, int32_t* out, int rows, int 
                                 unsigned* status, cudaStream_t s);
 
 // ---- dense verify: block attention mass and the refreshed selection --------
-struct BlockMassArgs {
-  const void* Q;          // [B, n_q, Hq, 128] bf16
-  const void* K;          // [pairs, cap, 128] bf16
-  const float* lse;       // [B, n_q, Hq] natural-log row sums of the dense attention
-  float* mass;            // [pairs, nb], zeroed before the launch (tiles add to it)
-  unsigned* status;
-  int B, Hq, Hkv, G, n_q, R;
-  int64_t cap, kv_end;
-  int b, nb;
-  int tiles;              // 64-key tiles of the complete blocks, nb * b / 64
-  int units;              // two tiles each, per pair
-  int upc, cpp;           // units per CTA, CTAs per pair (set by the launcher)
-  float qscale;           // softmax scale * log2(e)
-};
-bool block_mass_supported(const BlockMassArgs& a);
-cudaError_t launch_block_mass(BlockMassArgs a, int num_sms, cudaStream_t s);
+// mass[pair][j] = sum over j's half-tiles h and rows r < R of
+// part[pair][h][r].x * 2^(part[pair][h][r].y - lse_r * log2 e).
+cudaError_t launch_mass_finalize(const float2* part, const float* lse, float* mass, int B, int Hkv, int G, int n_q,
+                                 int nb, int b, cudaStream_t s);
 cudaError_t launch_mass_topk(const float* mass, int pairs, int nb, int b, int64_t s_end, int64_t w_begin, int k,
                              int32_t* idx, cudaStream_t s);
 

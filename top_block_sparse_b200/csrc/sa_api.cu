@@ -335,14 +335,18 @@ sa_params verify_dense_params(const sa_params* p) {
 
 struct VerifyWs {
   DecodeWs attn;          // the dense attention's workspace (status, tickets, partials)
-  size_t lse, total;      // lse of the rows when the caller passes none
+  size_t lse;             // lse of the rows when the caller passes none
+  size_t part;            // [pairs, nb * b / 32, 16] float2 half-tile row sums
+  size_t total;
 };
 
-VerifyWs verify_ws(const DecodeGeom& g, const DecodePlan& plan) {
+// nb: complete blocks of the caller's context
+VerifyWs verify_ws(const DecodeGeom& g, const DecodePlan& plan, int64_t nb) {
   VerifyWs w;
   w.attn = decode_ws(g, plan, 0, SA_OP_GIVEN_IDX, 0);
   w.lse = align_up(w.attn.total, 256);
-  w.total = w.lse + static_cast<size_t>(g.B) * g.n_q * g.Hq * 4;
+  w.part = align_up(w.lse + static_cast<size_t>(g.B) * g.n_q * g.Hq * 4, 256);
+  w.total = w.part + static_cast<size_t>(g.pairs) * static_cast<size_t>(nb * g.b / 32) * 16 * 8;
   return w;
 }
 
@@ -353,7 +357,7 @@ size_t sa_workspace_size(const sa_params* p, int32_t op) {
     DecodeGeom g;
     DecodePlan plan;
     if (plan_for(&d, 0, &g, &plan) != SA_OK) return 0;
-    return verify_ws(g, plan).total;
+    return verify_ws(g, plan, decode_geom(p).nb).total;
   }
   const bool prefill = (op == SA_OP_PREFILL) || (p && p->select == SA_SEL_TILE_MAX);
   if (check_params(p, prefill) != SA_OK) return 0;
@@ -568,46 +572,27 @@ sa_status sa_verify_refresh(const sa_params* p, const void* Q, const void* K, co
   if (gs.nb > kMaxSelectBlocks)
     return fail(SA_ERR_UNSUPPORTED, "%lld blocks per sequence exceed the %lld the selector handles",
                 (long long)gs.nb, (long long)kMaxSelectBlocks);
-  const VerifyWs L = verify_ws(g, plan);
+  if (g.R > 16) return fail(SA_ERR_UNSUPPORTED, "verify needs n_q * G <= 16 rows per KV head");
+  const VerifyWs L = verify_ws(g, plan, gs.nb);
   if ((st = check_ws(ws, ws_bytes, L.total)) != SA_OK) return st;
   unsigned char* w = static_cast<unsigned char*>(ws);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* lse_rows = lse ? lse : reinterpret_cast<float*>(w + L.lse);
+  float2* part = reinterpret_cast<float2*>(w + L.part);
 
-  BlockMassArgs m = {};
-  m.Q = Q;
-  m.K = K;
-  m.lse = lse_rows;
-  m.mass = mass;
-  m.status = reinterpret_cast<unsigned*>(w);
-  m.B = g.B;
-  m.Hq = g.Hq;
-  m.Hkv = g.Hkv;
-  m.G = g.G;
-  m.n_q = g.n_q;
-  m.R = g.R;
-  m.cap = g.cap;
-  m.kv_end = g.kv_end;
-  m.b = g.b;
-  m.nb = static_cast<int>(gs.nb);
-  m.tiles = static_cast<int>(gs.nb * g.b / 64);
-  m.units = (m.tiles + 1) / 2;
-  m.qscale = scale_of(p) * 1.4426950408889634f;
-  if (!block_mass_supported(m))
-    return fail(SA_ERR_UNSUPPORTED, "verify block mass needs n_q * G <= 16 rows per KV head");
-
-  // 1. dense attention (O, lse)
+  // 1. dense attention (O, lse) with the half-tile row sums of the complete
+  //    blocks (tensor-core kernel only)
   DecodeAttnArgs a = attn_args(&d, g, plan, Q, K, V, nullptr, 0, O, lse_rows, w, L.attn);
   a.pdl = 0;
-  cudaError_t e = launch_decode_attn(a, plan, true, p->out_dtype == SA_BF16, s);
+  a.mass_part = part;
+  a.mass_keys = gs.nb * g.b;
+  a.mass_hts = static_cast<int>(a.mass_keys / 32);
+  if (!decode_tc_supported(a)) return fail(SA_ERR_UNSUPPORTED, "verify needs the tensor-core attention kernel");
+  cudaError_t e = launch_decode_tc(a, plan, p->out_dtype == SA_BF16, s);
   if (e != cudaSuccess) return cuda_fail(e, "dense attention launch");
-  // 2. block mass (tiles add into a cleared array)
-  if (gs.nb > 0) {
-    e = cudaMemsetAsync(mass, 0, static_cast<size_t>(g.pairs) * gs.nb * 4, s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-    e = launch_block_mass(m, device_sms(), s);
-    if (e != cudaSuccess) return cuda_fail(e, "block mass launch");
-  }
+  // 2. block masses
+  e = launch_mass_finalize(part, lse_rows, mass, g.B, g.Hkv, g.G, g.n_q, static_cast<int>(gs.nb), g.b, s);
+  if (e != cudaSuccess) return cuda_fail(e, "block mass launch");
   // 3. the refreshed selection: top-k candidates by mass
   if (p->top_k > 0) {
     e = launch_mass_topk(mass, g.pairs, static_cast<int>(gs.nb), g.b, gs.s_end, gs.w_begin, p->top_k, idx_out, s);
