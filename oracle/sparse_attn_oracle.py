@@ -56,7 +56,7 @@ design notes of the repository):
 * R9  Multi-token chunk: the selection is made once from the chunk's FIRST
       query and reused by every token of the chunk (S3R draft chunk); token j
       of the chunk also sees chunk keys C..C+j.
-* R10 Dense verify (S3R review, "稠密验证"): every token of the chunk attends
+* R15 Dense verify (S3R review, "稠密验证"): every token of the chunk attends
       causally to ALL keys 0..C+j.  The verifier's attention "mass" of a
       complete context block is the SUM over the chunk's tokens and the KV
       head's G query heads of the attention weights its keys receive (the
@@ -322,7 +322,7 @@ def decode_pair(q_tokens: np.ndarray, K: np.ndarray, V: np.ndarray, C: int,
 def verify_pair(q_tokens: np.ndarray, K: np.ndarray, V: np.ndarray, C: int,
                 p: OracleParams) -> Dict:
     """Dense verify of a draft chunk for one (sequence, KV head), and the
-    block selection it refreshes (reading R10).
+    block selection it refreshes (reading R15).
 
     [S3R review, "稠密验证": the chunk's candidate tokens go through one causal
     forward with full attention over the dense cache, and the verifier's
