@@ -56,6 +56,11 @@ design notes of the repository):
 * R9  Multi-token chunk: the selection is made once from the chunk's FIRST
       query and reused by every token of the chunk (S3R draft chunk); token j
       of the chunk also sees chunk keys C..C+j.
+* R17 Column-sparse attention (PulseCol §3.1 eq. (2) with a column mask): the
+      mask is token-granular and shared by a group of 64 consecutive query
+      tokens and the KV head's query heads; each listed key is attended once
+      (duplicates and -1 entries are ignored); no causal mask, no sink or
+      window.  An empty list gives O = 0, lse = -inf.
 * R15 Dense verify (S3R review, "稠密验证"): every token of the chunk attends
       causally to ALL keys 0..C+j.  The verifier's attention "mass" of a
       complete context block is the SUM over the chunk's tokens and the KV
@@ -354,6 +359,31 @@ def verify_pair(q_tokens: np.ndarray, K: np.ndarray, V: np.ndarray, C: int,
     cand = candidate_blocks(C, p)
     sel = select_topk(mass, cand, p.top_k)
     return dict(O=O, lse=lse, mass=mass, wtail=wtail, candidates=cand, sel=sel)
+
+
+def column_attention_group(q_rows: np.ndarray, K: np.ndarray, V: np.ndarray,
+                           cols: Sequence[int], p: OracleParams) -> Dict:
+    """Column-sparse attention of one group of query tokens of one (sequence,
+    KV head) (reading R17) [PulseCol §3.1: eq. (1) logits Q K^T / sqrt(d_h);
+    eq. (2) softmax(Z + M(S)) V with S(i, j) = 1 for the kept key columns j of
+    row i: here the same columns for every row of the group, and every key
+    position may be kept, before or after the query (bidirectional)].
+
+    q_rows: [n, G, d] the group's tokens x the KV head's query heads; cols:
+    key positions (duplicates and negative entries ignored).  Returns O
+    [n, G, d], lse [n, G] (O = 0, lse = -inf when no column is kept).
+    """
+    n, G, d = q_rows.shape
+    pos = np.array(sorted({int(c) for c in cols if int(c) >= 0}), dtype=np.int64)
+    O = np.zeros((n, G, d))
+    lse = np.full((n, G), -np.inf)
+    if len(pos) == 0:
+        return dict(O=O, lse=lse, positions=pos)
+    scale = softmax_scale(d, p)
+    for i in range(n):
+        for g in range(G):
+            O[i, g], lse[i, g], _ = masked_softmax_attention(q_rows[i, g], K, V, pos, scale)
+    return dict(O=O, lse=lse, positions=pos)
 
 
 # --------------------------------------------------------------------------

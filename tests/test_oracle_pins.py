@@ -439,6 +439,52 @@ def test_verify_mass_total_needle_and_full_k():
     assert r_all["sel"].selected == orc.candidate_blocks(C, P(w))
 
 
+# ------------------------------------------------------------ column-sparse ---
+
+_COLP = orc.OracleParams(block_size=64, top_k=0, sink_keys=0, window_keys=0)
+
+
+def _col_case(seed=31, T=300, G=4):
+    r = rng(seed)
+    q = r.standard_normal((64, G, 128))
+    K = r.standard_normal((T, 128))
+    V = r.standard_normal((T, 128))
+    return q, K, V
+
+
+def test_column_attention_all_columns_is_library_bidirectional_attention():
+    """Every key kept: plain bidirectional attention (torch SDPA without a
+    mask), whatever the order of the list or its duplicates."""
+    q, K, V = _col_case()
+    T = len(K)
+    cols = list(range(T))[::-1] + [5, 5, -1]
+    r = orc.column_attention_group(q, K, V, cols, _COLP)
+    for i in (0, 17, 63):
+        for g in range(4):
+            np.testing.assert_allclose(r["O"][i, g], _sdpa(q[i, g], K, V, T), atol=1e-12)
+            z = K @ q[i, g] / math.sqrt(128)
+            assert abs(r["lse"][i, g] - logsumexp(z)) < 1e-12
+
+
+def test_column_attention_subset_and_edge_cases():
+    """A subset of columns equals library attention over those rows only
+    (keys after the query included); one column gives that column's V; an
+    empty list gives O = 0 and lse = -inf."""
+    q, K, V = _col_case(seed=32)
+    cols = [3, 250, 7, 299, 120, 64]
+    r = orc.column_attention_group(q, K, V, cols, _COLP)
+    sub = sorted(cols)
+    for i in (0, 40):
+        for g in (0, 3):
+            ref = _sdpa(q[i, g], K[sub], V[sub], len(sub))
+            np.testing.assert_allclose(r["O"][i, g], ref, atol=1e-12)
+    one = orc.column_attention_group(q, K, V, [42], _COLP)
+    np.testing.assert_allclose(one["O"][5, 1], V[42], atol=1e-12)
+    assert abs(one["lse"][5, 1] - float(K[42] @ q[5, 1]) / math.sqrt(128)) < 1e-12
+    none = orc.column_attention_group(q, K, V, [-1, -1], _COLP)
+    assert np.all(none["O"] == 0) and np.all(np.isneginf(none["lse"]))
+
+
 def _fails(fn):
     try:
         fn()
@@ -488,6 +534,15 @@ def test_planted_mistakes_are_caught(monkeypatch):
         with monkeypatch.context() as m:
             m.setattr(orc, "verify_pair", bad)
             assert _fails(test_verify_mass_equals_library_softmax_block_sums)
+    # a causal mask applied to the column-sparse attention
+    orig_col = orc.column_attention_group
+
+    def causal_cols(q, K, V, cols, p):
+        r = orig_col(q, K, V, [c for c in cols if 0 <= c <= 63], p)
+        return r
+    with monkeypatch.context() as m:
+        m.setattr(orc, "column_attention_group", causal_cols)
+        assert _fails(test_column_attention_subset_and_edge_cases)
     # summed chunk queries instead of the chunk's first query for selection
     with monkeypatch.context() as m:
         m.setattr(orc, "index_query", lambda qg: np.asarray(qg, float).sum(axis=0) * 0.0)
