@@ -83,7 +83,8 @@ enum {                                            /* ops for sa_workspace_size *
   SA_OP_GIVEN_IDX = 1,
   SA_OP_DECODE = 2,
   SA_OP_PREFILL = 3,
-  SA_OP_VERIFY = 4
+  SA_OP_VERIFY = 4,
+  SA_OP_COLUMN = 5
 };
 
 /* Problem description shared by every entry point (88 bytes). */
@@ -207,6 +208,30 @@ sa_status sa_verify_refresh(const sa_params* p, const void* Q, const void* K,
                             const void* V, void* O, float* lse, float* mass,
                             int32_t* idx_out, void* ws, size_t ws_bytes,
                             void* stream);
+
+/* Column-sparse attention (PulseCol §3.1, eq. (1) logits QK^T/sqrt(d_h) and
+ * eq. (2) softmax(Z + M(S)) V, with a token-granular column mask S): every
+ * group of 64 consecutive query tokens of a (sequence, KV head) and the
+ * KV head's 4 query heads attend to the key positions listed for the group,
+ * before or after them alike (no causal mask, no sink or window).
+ *
+ * p describes a full sequence as in prefill: select = SA_SEL_TILE_MAX,
+ * ctx_len = 0, n_q = T tokens, block_size = 64 (the group), GQA 4, bf16;
+ * top_k, sink_keys, window_keys and pool are ignored.  Q [B, T, Hq, d];
+ * K, V [B, Hkv, kv_capacity, d] (rows 0..T-1 are the keys); cols [B, Hkv,
+ * ceil(T/64), n_cols] int32: per group, key positions in [0, T), ascending,
+ * -1 padded.  Unless p->flags has SA_FLAG_TRUSTED_IDX the table is checked
+ * first: entries out of range or not above every earlier kept entry are
+ * dropped and set SA_ERR_INDEX in the workspace status (the rest are used).
+ * An empty list gives O = 0 and lse = -inf for its rows.  Outputs O
+ * [B, T, Hq, d] in out_dtype, lse [B, T, Hq] fp32 (may be NULL).
+ * Workspace: sa_workspace_size(p, SA_OP_COLUMN) sized for n_cols ==
+ * p->top_k.  Asynchronous on `stream`: one tensor-core launch (the K and V
+ * rows gathered by 16-byte copies), plus the table check. */
+sa_status sa_column_attn(const sa_params* p, const void* Q, const void* K,
+                         const void* V, const int32_t* cols, int32_t n_cols,
+                         void* O, float* lse, void* ws, size_t ws_bytes,
+                         void* stream);
 
 /* Number of kernels one sa_sparse_attn_decode call with `p` launches on this
  * device: 1 when scoring, top-k and attention run as one cooperative launch

@@ -136,6 +136,40 @@ def test_verify_null_arguments_and_workspace():
     assert sa.workspace_size(_p(n_q=3, num_q_heads=4, num_kv_heads=2, batch=8), sa.SA_OP_VERIFY) > need
 
 
+def _pcol(**kw):
+    base = dict(batch=1, num_q_heads=8, num_kv_heads=2, ctx_len=0, n_q=1000, block_size=64, top_k=70,
+                sink_keys=0, window_keys=0, dtype="bf16", prefill=True)
+    base.update(kw)
+    return sa.make_params(**base)
+
+
+def _column(p, n_cols=70, cols=FAKE, ws_bytes=1 << 30):
+    return sa.raw_call("sa_column_attn", ctypes.byref(p), FAKE, FAKE, FAKE, cols, n_cols, FAKE, None,
+                       FAKE, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,n_cols,status", [
+    (dict(dtype="f32"), 70, sa.SA_ERR_UNSUPPORTED),           # tensor cores: bf16 only
+    (dict(num_q_heads=4), 70, sa.SA_ERR_UNSUPPORTED),         # GQA 2: built for groups of 4 heads
+    (dict(block_size=128), 70, sa.SA_ERR_UNSUPPORTED),        # the query group is 64 tokens
+    (dict(prefill=False), 70, sa.SA_ERR_INVALID),             # sequence-type params needed
+    ({}, -1, sa.SA_ERR_INVALID),
+])
+def test_column_validation_rejects(kw, n_cols, status):
+    assert _column(_pcol(**kw), n_cols=n_cols) == status
+    assert sa.raw_call("sa_last_error").decode() != ""
+
+
+def test_column_null_table_and_workspace():
+    p = _pcol()
+    assert _column(p, cols=None) == sa.SA_ERR_INVALID            # n_cols > 0 needs a table
+    need = sa.workspace_size(p, sa.SA_OP_COLUMN)
+    assert need > 0
+    assert _column(p, ws_bytes=need - 1) == sa.SA_ERR_WORKSPACE
+    # top_k is the column count for sizing, beyond the selection limit too
+    assert sa.workspace_size(_pcol(top_k=13120), sa.SA_OP_COLUMN) > need
+
+
 def test_status_strings():
     for code, name in [(0, "SA_OK"), (4, "SA_ERR_INDEX"), (6, "SA_ERR_TIMEOUT")]:
         assert sa.raw_call("sa_status_string", code).decode() == name

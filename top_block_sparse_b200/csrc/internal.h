@@ -180,6 +180,13 @@ cudaError_t launch_prefill_score(const PrefillArgs& pa, cudaStream_t s);
 cudaError_t launch_prefill_attn(const PrefillArgs& pa, cudaStream_t s);
 size_t prefill_score_smem();
 size_t prefill_attn_smem();
+// Column-sparse attention (PulseCol eq. (2) with a column mask): every
+// 64-token group attends to the columns pa.idx lists for it ([P, n_tiles,
+// pa.top_k], ascending from the front, -1 padded), no causal mask.
+cudaError_t launch_column_attn(const PrefillArgs& pa, cudaStream_t s);
+// Caller column tables: kept entries in [0, T), ascending, packed, -1 padded.
+cudaError_t launch_sanitize_cols(const int32_t* in, int32_t* out, int64_t rows, int len, int T, unsigned* status,
+                                 cudaStream_t s);
 // Caller prefill tables [P, n_tiles, len]: keeps ids j < tile that are above
 // every earlier such id of the row and outside sink / window of the tile.
 cudaError_t launch_sanitize_prefill_idx(const int32_t* idx, int32_t* out, int P, int n_tiles, int len,

@@ -18,6 +18,16 @@
 // item, then K and V blocks through a 4-stage ring), warp 9 TMEM owner and
 // MMA issuer.  S(b + 1) is issued as soon as the softmax has read S(b), so
 // the tensor cores overlap the softmax.
+//
+// Column mode (PulseCol §3.1 eq. (2) with a token-granular column mask): the
+// item's 64 tokens x 4 heads attend to the key columns listed for the group
+// (ascending, -1 padded), before or after them alike.  The producer warp
+// gathers each chunk of 64 listed K and V rows with 16-byte cp.async copies
+// into the same 128-byte-swizzled stage layout the tensor maps produce,
+// keeps up to three chunks in flight (cp.async groups), and, once a chunk
+// has landed, fences it for the tensor cores and arrives on the stage's
+// barrier (one arrival per lane).  The last chunk's unused columns are
+// masked; an empty list is one fully masked chunk (O = 0, lse = -inf).
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
@@ -56,7 +66,10 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
 }
 
 struct PAArgs {
-  const int32_t* idx;       // [P, n_tiles, k]
+  const int32_t* idx;       // [P, n_tiles, k] (column mode: the column lists, k = n_cols)
+  const void* K;            // column mode: [P, cap, 128] bf16 (gathered by cp.async)
+  const void* V;
+  int64_t cap;
   void* O;                  // [B, T, Hq, 128]
   float* lse;               // [B, T, Hq] or null
   unsigned* status;
@@ -89,12 +102,44 @@ __device__ __forceinline__ Blocks blocks_of(const PAArgs& a, int p, int t, int l
   return bl;
 }
 
+// Column mode: n_sel = the group's listed columns (entries >= 0, which lead
+// the row), n_blk = chunks of 64 of them, at least one.
+__device__ __forceinline__ Blocks col_blocks_of(const PAArgs& a, int p, int t, int lane) {
+  Blocks bl;
+  const int32_t* row = a.idx + (static_cast<int64_t>(p) * a.n_tiles + t) * a.top_k;
+  int cnt = 0;
+  for (int s = lane; s < a.top_k; s += 32) cnt += __ldg(row + s) >= 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  bl.n_sink = 0;
+  bl.n_sel = cnt;
+  bl.w_first = 0;
+  bl.n_blk = cnt > 0 ? (cnt + kT - 1) / kT : 1;
+  return bl;
+}
+
+template <bool COL>
+__device__ __forceinline__ Blocks item_blocks(const PAArgs& a, int p, int t, int lane) {
+  if constexpr (COL) return col_blocks_of(a, p, t, lane);
+  else return blocks_of(a, p, t, lane);
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Item k -> (pair p, tile t), most expensive tiles first.
 __device__ __forceinline__ void item_of(const PAArgs& a, int k, int* p, int* t) {
   *t = a.n_tiles - 1 - k / a.P;
   *p = k % a.P;
 }
 
+template <bool COL>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_attn_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                         const __grid_constant__ CUtensorMap v_map, PAArgs a) {
@@ -122,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNKV; ++s) {
-      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_full[s], COL ? 32 : 1);         // column mode: one arrival per producer lane
       mbar_init(&kv_empty[s], 1);
     }
     mbar_init(q_full, 1);
@@ -157,9 +202,67 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = blockIdx.x; k < n_items && ok; k += gridDim.x, ++it) {
       int p, t;
       item_of(a, k, &p, &t);
-      const Blocks bl = blocks_of(a, p, t, lane);
+      const Blocks bl = item_blocks<COL>(a, p, t, lane);
       const int32_t* row = a.idx + (static_cast<int64_t>(p) * a.n_tiles + t) * a.top_k;
       const int bi = p / a.Hkv, h = p % a.Hkv;
+      if constexpr (COL) {
+        if (lane == 0) {
+          if (it > 0 && !mbar_wait_bounded(q_empty, (it - 1) & 1, abort_flag)) { fail(); ok = false; }
+          if (ok) {
+            mbar_arrive_expect_tx(q_full, kQBytes);
+            const int tok = bi * a.T + t * kT;
+            tc::tma_load_3d(Qs, &q_map, 0, h * kG, tok, q_full);
+            tc::tma_load_3d(Qs + kQBytes / 2, &q_map, 64, h * kG, tok, q_full);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        const unsigned char* kb = static_cast<const unsigned char*>(a.K) + static_cast<int64_t>(p) * a.cap * 256;
+        const unsigned char* vb = static_cast<const unsigned char*>(a.V) + static_cast<int64_t>(p) * a.cap * 256;
+        int pend = 0;                               // chunks copied but not yet signalled
+        for (int b = 0; b < bl.n_blk && ok; ++b, ++use) {
+          const int s = use % kNKV;
+          int fine = 1;
+          if (lane == 0 && use >= kNKV && !mbar_wait_bounded(&kv_empty[s], ((use / kNKV) & 1) ^ 1, abort_flag)) {
+            fail();
+            fine = 0;
+          }
+          if (!__shfl_sync(0xffffffffu, fine, 0)) {
+            ok = false;
+            break;
+          }
+          unsigned char* st = KV + s * kKVStage;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            // key slot r of the chunk <- listed column b * 64 + r (past the
+            // list: column 0, masked; clamped into the sequence either way)
+            const int r = hh * 32 + lane;
+            const int e = b * kT + r;
+            int col = e < bl.n_sel ? __ldg(row + e) : 0;
+            col = min(max(col, 0), a.T - 1);
+            const unsigned char* ks = kb + static_cast<int64_t>(col) * 256;
+            const unsigned char* vs = vb + static_cast<int64_t>(col) * 256;
+#pragma unroll
+            for (int c16 = 0; c16 < 16; ++c16) {
+              const uint32_t off = (c16 >> 3) * 8192 + tc::sw128_off(r, c16 & 7);
+              cp_async16(st + off, ks + c16 * 16);
+              cp_async16(st + 16384 + off, vs + c16 * 16);
+            }
+          }
+          cp_async_commit();
+          if (++pend == 3) {
+            // chunk use - 2 has landed: make it visible to the tensor cores
+            cp_async_wait<2>();
+            tc::fence_proxy_async_smem();
+            mbar_arrive(&kv_full[(use - 2) % kNKV]);
+            --pend;
+          }
+        }
+        // the item's last chunks (also after an error: every copy must land)
+        cp_async_wait<0>();
+        tc::fence_proxy_async_smem();
+        for (int q = pend; q > 0; --q) mbar_arrive(&kv_full[(use - q) % kNKV]);
+        continue;
+      }
       if (lane == 0) {
         if (it > 0 && !mbar_wait_bounded(q_empty, (it - 1) & 1, abort_flag)) { fail(); ok = false; }
         if (ok) {
@@ -205,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = blockIdx.x; k < n_items && ok; k += gridDim.x, ++it) {
       int p, t;
       item_of(a, k, &p, &t);
-      const Blocks bl = blocks_of(a, p, t, lane);
+      const Blocks bl = item_blocks<COL>(a, p, t, lane);
       // the whole warp runs the issue loop in lock step (descriptors stay
       // warp-uniform); one elected lane issues each MMA and commit
       {
@@ -285,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = blockIdx.x; k < n_items && ok; k += gridDim.x, ++it) {
       int p, t;
       item_of(a, k, &p, &t);
-      const Blocks bl = blocks_of(a, p, t, lane);
+      const Blocks bl = item_blocks<COL>(a, p, t, lane);
       float m_ref = -CUDART_INF_F, l = 0.f;
       for (int b = 0; b < bl.n_blk; ++b, ++nb_all) {
         if (!mbar_wait_bounded(s_full, nb_all & 1, abort_flag)) {
@@ -300,10 +403,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);
-        const bool diag = b == bl.n_blk - 1;          // the tile's own block: causal
-        if (diag) {
+        if constexpr (COL) {
+          // the last chunk's slots past the list are masked
+          const int nlast = bl.n_sel - b * kT;
+          if (nlast < kT) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = (c <= r) ? s[c] : -CUDART_INF_F;
+            for (int c = 0; c < 64; ++c) s[c] = (c < nlast) ? s[c] : -CUDART_INF_F;
+          }
+        } else {
+          const bool diag = b == bl.n_blk - 1;        // the tile's own block: causal
+          if (diag) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s[c] = (c <= r) ? s[c] : -CUDART_INF_F;
+          }
         }
         // row max of the raw logits (8 independent chains; the scale is > 0)
         float m8[8];
@@ -346,7 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // p = 2^(s * scale_log2 - m_ref): one FFMA and one ex2 per element; the
         // row sum uses the fp32 values, P goes to the tensor cores in bf16
         float ls0 = 0.f, ls1 = 0.f;
-        const float neg_m = -m_ref;
+        // (column mode: a row may have no key yet; 2^-inf = 0 then)
+        const float neg_m = (COL && m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
           uint32_t w[4];
@@ -480,12 +593,104 @@ cudaError_t launch_prefill_attn(const PrefillArgs& pa, cudaStream_t s) {
       return cudaErrorInvalidValue;
   }
   const size_t smem = prefill_attn_smem();
-  cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int items = pa.n_tiles * a.P;
   const int grid = items < pa.num_sms ? items : pa.num_sms;
-  prefill_attn_kernel<<<grid, kThreads, smem, s>>>(qm, km, vm, a);
+  prefill_attn_kernel<false><<<grid, kThreads, smem, s>>>(qm, km, vm, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_column_attn(const PrefillArgs& pa, cudaStream_t s) {
+  EncodeFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  PAArgs a = {};
+  a.idx = pa.idx;
+  a.K = pa.K;
+  a.V = pa.V;
+  a.cap = pa.cap;
+  a.O = pa.O;
+  a.lse = pa.lse;
+  a.status = pa.status;
+  a.B = pa.B;
+  a.Hq = pa.Hq;
+  a.Hkv = pa.Hkv;
+  a.T = pa.T;
+  a.n_tiles = pa.n_tiles;
+  a.P = pa.B * pa.Hkv;
+  a.top_k = pa.top_k;
+  a.out_bf16 = pa.out_bf16;
+  a.scale_log2 = pa.scale * 1.4426950408889634f;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUtensorMap qm;
+  {
+    // Q [B*T tokens][Hq heads][128]: box 64 columns x 4 heads x 64 tokens
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(pa.Hq), static_cast<cuuint64_t>(pa.B) * pa.T};
+    cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(pa.Hq) * 256};
+    cuuint32_t box[3] = {64, kG, kT};
+    if (enc(&qm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pa.Q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  const size_t smem = prefill_attn_smem();
+  cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int items = pa.n_tiles * a.P;
+  const int grid = items < pa.num_sms ? items : pa.num_sms;
+  // K and V are gathered by cp.async: their tensor-map slots are unused
+  prefill_attn_kernel<true><<<grid, kThreads, smem, s>>>(qm, qm, qm, a);
+  return cudaGetLastError();
+}
+
+namespace {
+
+// One warp per row of a caller's column table: keeps the entries in [0, T)
+// that are above every earlier kept entry (ascending, no repeats), packed
+// to the front and -1 padded; any other entry except -1 reports the index
+// status bit.
+__global__ void __launch_bounds__(256) sanitize_cols_kernel(const int32_t* __restrict__ in, int32_t* __restrict__ out,
+                                                            int64_t rows, int len, int T, unsigned* status) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * 8) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int lane = threadIdx.x & 31;
+  const int32_t* src = in + row * len;
+  int32_t* dst = out + row * len;
+  int last = -1, n = 0;
+  bool bad = false;
+  for (int base = 0; base < len; base += 32) {
+    const int e = base + lane;
+    const int v = e < len ? __ldg(src + e) : -1;
+    const bool in_range = v >= 0 && v < T;
+    bad |= e < len && v != -1 && !in_range;
+    // largest in-range entry strictly before this lane (carried across chunks)
+    int m = in_range ? v : -1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, m, o);
+      if (lane >= o) m = max(m, y);
+    }
+    int before = __shfl_up_sync(0xffffffffu, m, 1);
+    before = lane == 0 ? last : max(before, last);
+    const bool keep = in_range && v > before;
+    bad |= in_range && !keep;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) dst[n + __popc(bal & ((1u << lane) - 1u))] = v;
+    n += __popc(bal);
+    last = max(last, __shfl_sync(0xffffffffu, m, 31));
+  }
+  for (int e = n + lane; e < len; e += 32) dst[e] = -1;
+  if (__any_sync(0xffffffffu, bad) && lane == 0) report(status, kStatusIndex);
+}
+
+}  // namespace
+
+cudaError_t launch_sanitize_cols(const int32_t* in, int32_t* out, int64_t rows, int len, int T, unsigned* status,
+                                 cudaStream_t s) {
+  if (rows == 0 || len == 0) return cudaSuccess;
+  sanitize_cols_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(in, out, rows, len, T, status);
   return cudaGetLastError();
 }
 

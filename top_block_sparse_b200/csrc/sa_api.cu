@@ -350,7 +350,40 @@ VerifyWs verify_ws(const DecodeGeom& g, const DecodePlan& plan, int64_t nb) {
   return w;
 }
 
+// ---- column-sparse attention ------------------------------------------------
+sa_status check_column(const sa_params* p, PrefillGeom* g) {
+  if (p->dtype != SA_BF16) return fail(SA_ERR_UNSUPPORTED, "column attention runs on bf16 tensor cores");
+  if (p->num_q_heads != 4 * p->num_kv_heads)
+    return fail(SA_ERR_UNSUPPORTED, "column attention is built for GQA groups of 4 query heads per KV head");
+  if (p->block_size != 64) return fail(SA_ERR_UNSUPPORTED, "column attention groups 64 query tokens: block_size 64");
+  g->B = p->batch;
+  g->Hq = p->num_q_heads;
+  g->Hkv = p->num_kv_heads;
+  g->G = 4;
+  g->T = p->n_q;
+  g->nb = p->n_q / 64;
+  g->n_tiles = (p->n_q + 63) / 64;
+  g->P = p->batch * p->num_kv_heads;
+  g->cap = p->kv_capacity;
+  if (static_cast<int64_t>(g->B) * g->T > 0x7fffffff) return fail(SA_ERR_UNSUPPORTED, "too many tokens");
+  return SA_OK;
+}
+
+size_t column_ws(const PrefillGeom& g, int n_cols) {
+  return align_up(kWsHeader, 1024) + static_cast<size_t>(g.P) * g.n_tiles * static_cast<size_t>(n_cols) * 4;
+}
+
 size_t sa_workspace_size(const sa_params* p, int32_t op) {
+  if (op == SA_OP_COLUMN) {
+    // top_k is the column count here (checked against its own limit)
+    if (!p || p->top_k < 0 || p->top_k > (1 << 20)) return 0;
+    sa_params q = *p;
+    q.top_k = 0;
+    if (check_params(&q, true) != SA_OK) return 0;
+    PrefillGeom g;
+    if (check_column(&q, &g) != SA_OK) return 0;
+    return column_ws(g, p->top_k);
+  }
   if (op == SA_OP_VERIFY) {
     if (check_params(p, false) != SA_OK) return 0;
     const sa_params d = verify_dense_params(p);
@@ -598,6 +631,47 @@ sa_status sa_verify_refresh(const sa_params* p, const void* Q, const void* K, co
     e = launch_mass_topk(mass, g.pairs, static_cast<int>(gs.nb), g.b, gs.s_end, gs.w_begin, p->top_k, idx_out, s);
     if (e != cudaSuccess) return cuda_fail(e, "mass top-k launch");
   }
+  return SA_OK;
+}
+
+sa_status sa_column_attn(const sa_params* p0, const void* Q, const void* K, const void* V, const int32_t* cols,
+                         int32_t n_cols, void* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!p0) return fail(SA_ERR_INVALID, "params is NULL");
+  sa_params pc = *p0;
+  pc.top_k = 0;                               // not used by this call
+  const sa_params* p = &pc;
+  sa_status st = check_params(p, true);
+  if (st != SA_OK) return st;
+  if (!Q || !K || !V || !O) return fail(SA_ERR_INVALID, "Q, K, V and O must be non-NULL");
+  if (n_cols < 0 || n_cols > (1 << 20)) return fail(SA_ERR_INVALID, "n_cols %d must be in [0, 2^20]", n_cols);
+  if (n_cols > 0 && !cols) return fail(SA_ERR_INVALID, "cols is NULL with n_cols > 0");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return fail(SA_ERR_INVALID, "Q, K, V and O must be 16-byte aligned");
+  PrefillGeom g;
+  if ((st = check_column(p, &g)) != SA_OK) return st;
+  const size_t need = column_ws(g, n_cols);
+  if ((st = check_ws(ws, ws_bytes, need)) != SA_OK) return st;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int32_t* table = cols;
+  if (n_cols > 0 && !(p->flags & SA_FLAG_TRUSTED_IDX)) {
+    int32_t* clean = reinterpret_cast<int32_t*>(w + align_up(kWsHeader, 1024));
+    cudaError_t e = launch_sanitize_cols(cols, clean, static_cast<int64_t>(g.P) * g.n_tiles, n_cols, g.T,
+                                         reinterpret_cast<unsigned*>(w), s);
+    if (e != cudaSuccess) return cuda_fail(e, "column-table check launch");
+    table = clean;
+  }
+  PrefillArgs a = prefill_args(p, g);
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.idx = const_cast<int32_t*>(table);
+  a.top_k = n_cols;
+  a.O = O;
+  a.lse = lse;
+  a.status = reinterpret_cast<unsigned*>(w);
+  cudaError_t e = launch_column_attn(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "column attention launch");
   return SA_OK;
 }
 

@@ -71,7 +71,38 @@ WORKLOADS: Dict[str, Workload] = {
     # batch 64, 6-token draft chunk, 16 / 8 heads, C = 16384
     "draft_chunk_16k": Workload("draft_chunk_16k", 64, 6, 16, 8, 128, 16384,
                                 "bf16", 64, "mean", 16, 64, 256, 8),
+    # column-sparse (bidirectional) attention over T = 65536 tokens, 32 / 8
+    # heads, bf16: top_k = the columns listed per 64-token group (20% of T)
+    "column_64k": Workload("column_64k", 1, 65536, 32, 8, 128, 0, "bf16",
+                           64, "mean", 13120, 0, 0, 0, prefill=True),
 }
+
+
+def make_columns(w: Workload, seed: int, n_cols: Optional[int] = None, device="cpu") -> torch.Tensor:
+    """Column lists [B, Hkv, ceil(T/64), n_cols] int32 for column-sparse
+    attention over T = w.n_q tokens: per (sequence, KV head) one random set
+    of n_cols - 64 key positions shared by all its 64-token groups (the
+    important columns recur across rows), joined for each group with the
+    group's own tokens; ascending, -1 padded.  n_cols defaults to w.top_k."""
+    n_cols = w.top_k if n_cols is None else int(n_cols)
+    T, B, Hkv = w.n_q, w.batch, w.num_kv_heads
+    groups = (T + 63) // 64
+    out = torch.full((B, Hkv, groups, n_cols), -1, dtype=torch.int32)
+    n_shared = max(min(n_cols - 64, T), 0)
+    for bi in range(B):
+        for h in range(Hkv):
+            g = _gen("cpu", seed * 1000003 + (bi * Hkv + h) * 4 + 5)
+            shared = torch.randperm(T, generator=g)[:n_shared]
+            mark = torch.zeros(T, dtype=torch.bool)
+            mark[shared] = True
+            for t in range(groups):
+                m = mark.clone()
+                lo, hi = t * 64, min(t * 64 + 64, T)
+                if n_cols >= 64:
+                    m[lo:hi] = True
+                cols = torch.nonzero(m).flatten()[:n_cols].to(torch.int32)
+                out[bi, h, t, :len(cols)] = cols
+    return out.to(device)
 
 
 def _gen(device, seed: int) -> torch.Generator:

@@ -25,13 +25,13 @@ SA_OK, SA_ERR_INVALID, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_INDEX, SA_ER
 SA_F32, SA_BF16 = 0, 1
 SA_POOL_MEAN, SA_POOL_LSA = 0, 1
 SA_SEL_QUERY0, SA_SEL_TILE_MAX = 0, 1
-SA_OP_SCORE_TOPK, SA_OP_GIVEN_IDX, SA_OP_DECODE, SA_OP_PREFILL, SA_OP_VERIFY = 0, 1, 2, 3, 4
+SA_OP_SCORE_TOPK, SA_OP_GIVEN_IDX, SA_OP_DECODE, SA_OP_PREFILL, SA_OP_VERIFY, SA_OP_COLUMN = 0, 1, 2, 3, 4, 5
 SA_FLAG_TRUSTED_IDX = 1
 
 EXPORTED = ["sa_version", "sa_workspace_size", "sa_workspace_init", "sa_pool_keys", "sa_score_topk",
             "sa_sparse_attn_given_idx", "sa_sparse_attn_decode", "sa_sparse_attn_prefill",
             "sa_read_status", "sa_status_string", "sa_last_error", "sa_sparse_attn_given_idx_noalloc",
-            "sa_decode_launches", "sa_verify_refresh"]
+            "sa_decode_launches", "sa_verify_refresh", "sa_column_attn"]
 
 
 class SaParams(ctypes.Structure):
@@ -67,6 +67,7 @@ _sig = {
     "sa_last_error": (ctypes.c_char_p, []),
     "sa_decode_launches": (_i32, [_P]),
     "sa_verify_refresh": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "sa_column_attn": (_i32, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -188,6 +189,14 @@ def verify_refresh(p: SaParams, Q, K, V, O, mass, lse=None, idx_out=None, ws=Non
     top_k blocks by mass (sa_verify_refresh)."""
     _check(_lib.sa_verify_refresh(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse), _ptr(mass),
                                   _ptr(idx_out), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def column_attn(p: SaParams, Q, K, V, cols, O, lse=None, ws=None, stream=None):
+    """Column-sparse attention of every 64-token group over its listed key
+    columns (sa_column_attn); cols [B, Hkv, groups, n_cols] int32 or None."""
+    n_cols = 0 if cols is None else int(cols.shape[-1])
+    _check(_lib.sa_column_attn(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(cols), n_cols, _ptr(O), _ptr(lse),
+                               _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def read_status(ws: torch.Tensor, stream=None) -> int:
