@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload decode_32k] [--no-cpu-baseline] [--no-prefill] [--no-verify]
+                    [--no-column]
 
 Workload (default): batched decode, batch 32, 32 query / 8 KV heads, d = 128,
 context T = 32768, bf16 KV cache with fp32 accumulation, block 64, top-k 32 +
@@ -22,8 +23,9 @@ data path); the per-rank device times are max-reduced.
 Printed: one JSON line (rank 0).  ``value`` = sequences decoded per second
 (whole job).  Also: the roofline of the step's one kernel (algorithmic bytes
 over the timed launch, against the measured copy bandwidth), the attention
-kernel alone on the same table, the causal prefill and the dense verify of
-a draft chunk (each with its kernels' rooflines), the end-to-end number
+kernel alone on the same table, the causal prefill, the dense verify of a
+draft chunk and column-sparse attention (each with its kernels' rooflines),
+the end-to-end number
 through the C ABI with host buffers, clocks sampled during the timed region,
 and the float64 CPU oracle timed on a bounded sample (rank 0, N = 1).
 """
@@ -357,6 +359,10 @@ def run_ours(args, w, rank, world, local_rank):
     verify = None
     if not args.no_verify:
         verify = run_verify_bench(args, dev, stream, flush)
+    # --- column-sparse attention, rank-local ----------------------------------
+    column = None
+    if not args.no_column:
+        column = run_column_bench(args, dev, stream, flush)
     # --- end to end through the C ABI with host buffers -------------------
     e2e = e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush)
     if world > 1:
@@ -404,6 +410,7 @@ def run_ours(args, w, rank, world, local_rank):
                         "compressed keys stay resident in HBM"},
         "prefill": prefill,
         "verify": verify,
+        "column": column,
         "gpu_launches": sa.decode_launches(p) * args.steps,
         "clocks": clk.summary(),
     }
@@ -560,6 +567,52 @@ def run_verify_bench(args, dev, stream, flush):
     }
 
 
+def run_column_bench(args, dev, stream, flush):
+    """Times column-sparse attention (sa_column_attn) on the 64k-token
+    workload: every 64-token group attends to its 13120 listed columns."""
+    from top_block_sparse_b200 import sa
+    from top_block_sparse_b200.inputs import make_columns
+    w = WORKLOADS["column_64k"]
+    if args.column_tokens:
+        # a smaller sequence (ncu captures) keeps the 20% of columns per group
+        T = args.column_tokens
+        w = w.scaled(n_q=T, top_k=max(64, (T // 5 + 63) // 64 * 64))
+    inp = make_inputs(w, seed=4001, device=dev)
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    del inp
+    cols = make_columns(w, seed=4002, device=dev)
+    n_valid = int((cols >= 0).sum().item())
+    p = sa.params_for(w, out_dtype="bf16")
+    p.flags = sa.SA_FLAG_TRUSTED_IDX
+    O = torch.empty((1, w.n_q, w.num_q_heads, 128), device=dev, dtype=torch.bfloat16)
+    lse = torch.empty((1, w.n_q, w.num_q_heads), device=dev)
+    ws = sa.alloc_workspace(p, sa.SA_OP_COLUMN, device=dev)
+
+    def run():
+        sa.column_attn(p, Q, K, V, cols, O, lse, ws, stream=stream)
+
+    ms = statistics.mean(timed_steps(run, args.column_steps, 3, stream, flush))
+    if sa.read_status(ws, stream) != sa.SA_OK:
+        raise RuntimeError("device status word set during the column-sparse runs")
+    _, tfl, _, src = peaks()
+    rows = 64 * w.group                                   # query rows of one group
+    alg = 2 * 2 * rows * 128 * n_valid                    # QK^T and PV over the listed columns
+    chunks = int(((cols >= 0).sum(-1) + 63).div(64, rounding_mode="floor").clamp(min=1).sum().item())
+    exe = 2 * 2 * rows * 128 * 64 * chunks                # 64-column chunks as executed
+    return {
+        "workload": f"column_64k: bidirectional column-sparse attention, T={w.n_q}, Hq={w.num_q_heads}, "
+                    f"Hkv={w.num_kv_heads}, d=128, bf16, {w.top_k} columns per 64-token group (20% of T: a shared "
+                    "random set per (sequence, KV head) plus the group's own tokens)",
+        "ms": ms,
+        "alg_tflops": alg / (ms * 1e-3) / 1e12,
+        "exec_tflops": exe / (ms * 1e-3) / 1e12,
+        "frac_of_bf16_peak": exe / (ms * 1e-3) / 1e12 / tfl,
+        "kernel": "prefill_attn_kernel<column mode> (tcgen05; K and V rows gathered by cp.async)",
+        "gathered_gb": n_valid * 512 / 1e9,
+        "peak_bf16_tflops": tfl, "peak_source": src,
+    }
+
+
 def e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush):
     from top_block_sparse_b200 import sa
     C = w.ctx_len
@@ -602,6 +655,10 @@ def main():
     ap.add_argument("--prefill-steps", type=int, default=10)
     ap.add_argument("--verify-steps", type=int, default=10)
     ap.add_argument("--no-verify", action="store_true")
+    ap.add_argument("--column-steps", type=int, default=5)
+    ap.add_argument("--no-column", action="store_true")
+    ap.add_argument("--column-tokens", type=int, default=None,
+                    help="override the column workload's sequence length (smaller cases for ncu captures)")
     ap.add_argument("--prefill-tokens", type=int, default=None,
                     help="override the prefill length (smaller cases for ncu captures)")
     ap.add_argument("--batch", type=int, default=None,
