@@ -219,7 +219,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const unsigned char* kb = static_cast<const unsigned char*>(a.K) + static_cast<int64_t>(p) * a.cap * 256;
         const unsigned char* vb = static_cast<const unsigned char*>(a.V) + static_cast<int64_t>(p) * a.cap * 256;
         int pend = 0;                               // chunks copied but not yet signalled
+        // slot r of chunk b <- listed column b * 64 + r (past the list:
+        // column 0, masked; clamped into the sequence either way); lane l
+        // loads slots l and l + 32, one chunk ahead of the copies
+        auto load_cols = [&](int b, int (&c)[2]) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int e = b * kT + hh * 32 + lane;
+            c[hh] = e < bl.n_sel ? __ldg(row + e) : 0;
+          }
+        };
+        int nxt[2];
+        load_cols(0, nxt);
         for (int b = 0; b < bl.n_blk && ok; ++b, ++use) {
+          int cur[2] = {nxt[0], nxt[1]};
+          if (b + 1 < bl.n_blk) load_cols(b + 1, nxt);
           const int s = use % kNKV;
           int fine = 1;
           if (lane == 0 && use >= kNKV && !mbar_wait_bounded(&kv_empty[s], ((use / kNKV) & 1) ^ 1, abort_flag)) {
@@ -233,12 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           unsigned char* st = KV + s * kKVStage;
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
-            // key slot r of the chunk <- listed column b * 64 + r (past the
-            // list: column 0, masked; clamped into the sequence either way)
             const int r = hh * 32 + lane;
-            const int e = b * kT + r;
-            int col = e < bl.n_sel ? __ldg(row + e) : 0;
-            col = min(max(col, 0), a.T - 1);
+            const int col = min(max(cur[hh], 0), a.T - 1);
             const unsigned char* ks = kb + static_cast<int64_t>(col) * 256;
             const unsigned char* vs = vb + static_cast<int64_t>(col) * 256;
 #pragma unroll
