@@ -255,6 +255,23 @@ def cpu_info():
     return model, os.cpu_count()
 
 
+# ---------------------------------------------------------------- ranks ---
+
+def rank_seed(rank: int) -> int:
+    """Input seed of a rank: every rank decodes its own batch (weak scaling)."""
+    return 1000 + 1 + rank
+
+
+def reduce_max(value: float, world: int, device) -> float:
+    """Max over the ranks of a per-rank device time: the job takes as long as
+    its slowest rank."""
+    if world <= 1:
+        return value
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ------------------------------------------------------------------- arms ---
 
 def run_reference(args, w, rank, world):
@@ -308,7 +325,7 @@ def run_ours(args, w, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.Stream(device=dev)
-    inp = make_inputs(w, seed=1000 + 1 + rank, device=dev)
+    inp = make_inputs(w, seed=rank_seed(rank), device=dev)
     Q, K, V = inp["Q"], inp["K"], inp["V"]
     p = sa.params_for(w)
     nb = w.ctx_len // w.block_size
@@ -343,11 +360,7 @@ def run_ours(args, w, rank, world, local_rank):
         step_ms = timed_steps(step, args.steps, args.warmup, stream, flush)
     if sa.read_status(ws, stream) != sa.SA_OK:
         raise RuntimeError("device status word set during the timed steps")
-    ms = sum(step_ms) / len(step_ms)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(sum(step_ms) / len(step_ms), world, dev)
     # --- the attention kernel alone, rank-local ----------------------------
     attn_ms = statistics.mean(timed_steps(attn_only, max(50, args.steps // 4), 3, stream, flush))
     pool_ms = statistics.mean(timed_steps(pool_only, 10, 2, stream, flush))
@@ -365,10 +378,7 @@ def run_ours(args, w, rank, world, local_rank):
         column = run_column_bench(args, dev, stream, flush)
     # --- end to end through the C ABI with host buffers -------------------
     e2e = e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush)
-    if world > 1:
-        t = torch.tensor([e2e["ms"]], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e["ms"] = float(t.item())
+    e2e["ms"] = reduce_max(e2e["ms"], world, dev)
     if rank != 0:
         return None
 
