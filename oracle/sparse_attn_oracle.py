@@ -70,6 +70,12 @@ design notes of the repository):
       candidate blocks by mass, with the candidates and ties of R4-R6 (the
       KV-selection formula: recent window plus top-K by the previous verify's
       attention scores).
+* R18 Overlapping compressed keys (SparDA, "方法": InfLLM-V2 mean-pools the
+      keys into OVERLAPPING compressed representations, coarse to fine; the
+      window length and stride are not given, so they are parameters):
+      compressed key c is the mean of the l keys starting at c*s (complete
+      windows only), and the score of selectable block j is the MAX of the
+      scores of the compressed keys whose windows share a key with block j.
 """
 from __future__ import annotations
 
@@ -90,8 +96,11 @@ class OracleParams:
     top_k: int                 # k: blocks chosen by score
     sink_keys: int             # S: keys [0, S) always attended
     window_keys: int           # W: keys [C-W, C) always attended
-    pool: str = "mean"         # "mean" (SparDA) or "lsa" (LSA §2.2)
-    pool_stride: int = 4       # raw keys summed into one LSA pool key
+    pool: str = "mean"         # "mean" (SparDA), "lsa" (LSA §2.2) or
+                               # "overlap" (SparDA / InfLLM-V2, reading R18)
+    pool_stride: int = 4       # LSA: raw keys summed into one pool key;
+                               # overlap: keys between window starts (s)
+    pool_kernel: int = 0       # overlap: keys per compressed key (l)
     scale: Optional[float] = None   # softmax scale; None -> 1/sqrt(d)
 
 
@@ -140,11 +149,32 @@ def pool_lsa(K: np.ndarray, b: int, stride: int = 4) -> np.ndarray:
     return _normalise(cent)
 
 
+def pool_overlap(K: np.ndarray, kernel: int, stride: int) -> np.ndarray:
+    """Overlapping mean-pooled compressed keys  [SparDA, "方法": the keys
+    are average-pooled into overlapping compressed representations]
+    (reading R18 for the window geometry):
+
+        Kc[c] = (1/kernel) * sum_{t = c*stride}^{c*stride + kernel - 1} K[t]
+
+    for every c whose window lies wholly inside the rows given.  Returns
+    [n_c, d] with n_c = (T - kernel) // stride + 1 if T >= kernel, else 0.
+    """
+    K = np.asarray(K, dtype=np.float64)
+    T = K.shape[0]
+    n_c = (T - kernel) // stride + 1 if T >= kernel else 0
+    out = np.zeros((n_c, K.shape[1]), dtype=np.float64)
+    for c in range(n_c):
+        out[c] = K[c * stride:c * stride + kernel].sum(axis=0) / kernel
+    return out
+
+
 def compress(K: np.ndarray, p: OracleParams) -> np.ndarray:
     if p.pool == "mean":
         return pool_mean(K, p.block_size)
     if p.pool == "lsa":
         return pool_lsa(K, p.block_size, p.pool_stride)
+    if p.pool == "overlap":
+        return pool_overlap(K, p.pool_kernel, p.pool_stride)
     raise ValueError(p.pool)
 
 
@@ -177,6 +207,22 @@ def block_scores(qbar: np.ndarray, Kc: np.ndarray, p: OracleParams) -> np.ndarra
     if p.pool == "lsa":
         return Kc @ _normalise(qbar)
     return (Kc @ qbar) * softmax_scale(Kc.shape[1], p)
+
+
+def blocks_from_compressed(sigma: np.ndarray, C: int, p: OracleParams) -> np.ndarray:
+    """Coarse-to-fine step of overlapping compression (reading R18; SparDA
+    "方法"): the score of complete block j, keys [j*b, j*b + b), is the
+    largest score among the compressed keys whose window
+    [c*s, c*s + l) shares at least one key with the block.  Returns [nb]
+    with nb = C // b (-inf for a block no window reaches)."""
+    b, l, s = p.block_size, p.pool_kernel, p.pool_stride
+    starts = np.arange(len(sigma)) * s
+    out = np.full(C // b, -np.inf)
+    for j in range(C // b):
+        hit = (starts < (j + 1) * b) & (starts + l > j * b)
+        if hit.any():
+            out[j] = np.max(np.asarray(sigma)[hit])
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -306,6 +352,8 @@ def decode_pair(q_tokens: np.ndarray, K: np.ndarray, V: np.ndarray, C: int,
         Kc = compress(K[:C], p)
     qbar = index_query(q_tokens[0])
     s = block_scores(qbar, Kc, p)
+    if p.pool == "overlap":
+        s = blocks_from_compressed(s, C, p)
     cand = candidate_blocks(C, p)
     sel = select_topk(s, cand, p.top_k)
     scale = softmax_scale(d, p)
@@ -393,6 +441,8 @@ def column_attention_group(q_rows: np.ndarray, K: np.ndarray, V: np.ndarray,
 def prefill_tile_scores(q_rows: np.ndarray, Kc: np.ndarray, p: OracleParams) -> np.ndarray:
     """Tile score of each block: max over the tile's rows of the row's
     GQA-summed block score (readings R1, R2).  q_rows: [rows, G, d]."""
+    if p.pool == "overlap":
+        raise NotImplementedError("overlapping compression is defined here for decode and draft chunks only")
     per_row = np.stack([block_scores(index_query(q_rows[r]), Kc, p)
                         for r in range(q_rows.shape[0])])
     return per_row.max(axis=0)

@@ -19,7 +19,8 @@ F32_MAX_ABS = 1e-5
 
 def oracle_params(w, **kw) -> orc.OracleParams:
     p = orc.OracleParams(block_size=w.block_size, top_k=w.top_k, sink_keys=w.sink_keys,
-                         window_keys=w.window_keys, pool=w.pool)
+                         window_keys=w.window_keys, pool=w.pool, pool_stride=w.pool_stride,
+                         pool_kernel=w.pool_kernel)
     for k, v in kw.items():
         setattr(p, k, v)
     return p

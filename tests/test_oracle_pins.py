@@ -27,7 +27,7 @@ GOLD = json.load(open(os.path.join(HERE, "golden", "hand_worked.json")))["cases"
 def P(w, **kw):
     p = orc.OracleParams(block_size=w.block_size, top_k=w.top_k,
                          sink_keys=w.sink_keys, window_keys=w.window_keys,
-                         pool=w.pool)
+                         pool=w.pool, pool_stride=w.pool_stride, pool_kernel=w.pool_kernel)
     for k, v in kw.items():
         setattr(p, k, v)
     return p
@@ -280,13 +280,15 @@ def test_sink_window_always_attended_and_chunk_causal():
         assert len(pos) == (16 + 1 + 4) * 64 + j + 1
 
 
-@pytest.mark.parametrize("pool", ["mean", "lsa"])
+@pytest.mark.parametrize("pool", ["mean", "lsa", "overlap"])
 def test_dense_equivalence_when_topk_covers_all(pool):
     """With k >= #candidates the sparse result is dense causal attention
     (the special case S = all-ones causal of the masked softmax)."""
-    b = 64 if pool == "mean" else 512
+    b = 512 if pool == "lsa" else 64
     w = WORKLOADS["draft_chunk_16k"].scaled(batch=1, num_kv_heads=1, num_q_heads=3,
-                                            ctx_len=2048 + 37, block_size=b, pool=pool)
+                                            ctx_len=2048 + 37, block_size=b, pool=pool,
+                                            pool_stride=16 if pool == "overlap" else 4,
+                                            pool_kernel=32 if pool == "overlap" else 0)
     inp = make_inputs(w, seed=14)
     q, K, V = _slab(inp, 0, 0, w.group)
     p = P(w, top_k=10_000)
@@ -386,6 +388,76 @@ def test_prefill_dense_equivalence_and_needles():
     r = orc.prefill_tile(q[i * 64:], K, V, i, p, Kc)
     assert set(inp["needles"][0, 0].tolist()) <= set(r["sel"].selected)
     assert len(r["sel"].selected) == min(64, i - 5)
+
+
+# ------------------------------------------- overlapping compression ---
+
+_OVL_CASES = [(64, 32, 16, 320), (64, 32, 16, 333), (64, 64, 16, 300), (64, 16, 16, 256),
+              (32, 24, 8, 200), (64, 64, 64, 256), (64, 48, 16, 64 * 7 + 40)]
+
+
+def _ovl_params(b, l, s):
+    return orc.OracleParams(block_size=b, top_k=1, sink_keys=0, window_keys=0, pool="overlap",
+                            pool_stride=s, pool_kernel=l, scale=0.5)
+
+
+@pytest.mark.parametrize("b,l,s,C", _OVL_CASES)
+def test_overlap_pool_is_library_avg_pool(b, l, s, C):
+    """Overlapping mean pooling is avg_pool1d with kernel l and stride s
+    (windows running past the rows are dropped by both)."""
+    K = rng(5).standard_normal((C, 8))
+    ref = torch.nn.functional.avg_pool1d(torch.from_numpy(K).T[None], l, s)[0].T.numpy()
+    got = orc.compress(K, _ovl_params(b, l, s))
+    assert got.shape == ref.shape == ((C - l) // s + 1, 8)
+    np.testing.assert_allclose(got, ref, atol=1e-14)
+
+
+@pytest.mark.parametrize("b,l,s,C", _OVL_CASES)
+def test_overlap_block_scores_closed_form(b, l, s, C):
+    """Keys on a ramp K_t = +-(t+1) v: compressed key c is
+    +-(c*s + (l+1)/2) v, so with qbar.v > 0 a block's score is taken from the
+    LAST window touching it on a rising ramp (c = min(n_c-1, ((j+1)b-1)//s):
+    complete windows only) and from the FIRST on a falling one
+    (c = max(0, ceil((jb-l+1)/s)): the window reaching in from the block
+    before counts)."""
+    d = 8
+    p = _ovl_params(b, l, s)
+    n_c = (C - l) // s + 1
+    v = rng(6).standard_normal(d)
+    qbar = 2.0 * v
+    qv = float(qbar @ v) * 0.5
+    for sign in (1.0, -1.0):
+        K = sign * (np.arange(C)[:, None] + 1.0) * v[None, :]
+        S = orc.blocks_from_compressed(orc.block_scores(qbar, orc.compress(K, p), p), C, p)
+        assert S.shape == (C // b,)
+        for j in range(C // b):
+            if sign > 0:
+                c = min(n_c - 1, ((j + 1) * b - 1) // s)
+            else:
+                c = max(0, -(-(j * b - l + 1) // s))
+            assert S[j] == pytest.approx(sign * qv * (c * s + (l + 1) / 2), rel=1e-12), (sign, j)
+
+
+def test_overlap_without_overlap_is_block_mean():
+    """l = s = b: one window per block, the plain block-mean scores."""
+    r = rng(7)
+    K = r.standard_normal((64 * 9 + 5, 16))
+    q = r.standard_normal(16)
+    p_ovl = _ovl_params(64, 64, 64)
+    p_mean = orc.OracleParams(block_size=64, top_k=1, sink_keys=0, window_keys=0, scale=0.5)
+    got = orc.blocks_from_compressed(orc.block_scores(q, orc.compress(K, p_ovl), p_ovl), len(K), p_ovl)
+    np.testing.assert_allclose(got, orc.block_scores(q, orc.pool_mean(K, 64), p_mean), atol=1e-14)
+
+
+def test_overlap_needles_selected():
+    """Needle blocks (keys pulled towards the index query) win the block
+    max of their own windows, so the 32k overlapping decode slab keeps
+    them."""
+    w = WORKLOADS["decode_32k_overlap"].scaled(batch=1, num_kv_heads=1, num_q_heads=4, ctx_len=8192, n_needles=6)
+    inp = make_inputs(w, seed=15)
+    q, K, V = _slab(inp, 0, 0, w.group)
+    r = orc.decode_pair(q, K, V, w.ctx_len, P(w))
+    assert set(inp["needles"][0, 0].tolist()) <= set(r["sel"].selected)
 
 
 # ---------------------------------------------- planted-mistake checks ---
@@ -495,6 +567,7 @@ def _fails(fn):
 
 def test_planted_mistakes_are_caught(monkeypatch):
     """Each plausible mistake planted in the oracle makes some pin fail."""
+    orig_pool_ovl = orc.pool_overlap
     mistakes = {
         "mean instead of sum over the GQA group":
             ("index_query", lambda qg: np.asarray(qg, float).mean(axis=0),
@@ -543,6 +616,27 @@ def test_planted_mistakes_are_caught(monkeypatch):
     with monkeypatch.context() as m:
         m.setattr(orc, "column_attention_group", causal_cols)
         assert _fails(test_column_attention_subset_and_edge_cases)
+    # overlapping compression: windows inside the block only, incomplete
+    # windows kept, the sum over the stride instead of the mean over the window
+    orig_b2c = orc.blocks_from_compressed
+
+    def contained_only(sigma, C, p):
+        b, l, s_ = p.block_size, p.pool_kernel, p.pool_stride
+        st = np.arange(len(sigma)) * s_
+        return np.array([np.max(np.asarray(sigma)[(st >= j * b) & (st + l <= (j + 1) * b)])
+                         for j in range(C // b)])
+
+    def with_partial(K, kernel, stride):
+        K = np.asarray(K, float)
+        return np.stack([K[c:c + kernel].mean(0) for c in range(0, len(K) - stride + 1, stride)])
+    ovl = lambda: [test_overlap_block_scores_closed_form(*c) for c in _OVL_CASES]
+    for name, bad in (("blocks_from_compressed", contained_only),
+                      ("pool_overlap", with_partial),
+                      ("pool_overlap", lambda K, l, s_: orig_pool_ovl(K, l, s_) * l / s_)):
+        with monkeypatch.context() as m:
+            m.setattr(orc, name, bad)
+            assert _fails(ovl), name
+    assert orig_b2c is orc.blocks_from_compressed
     # summed chunk queries instead of the chunk's first query for selection
     with monkeypatch.context() as m:
         m.setattr(orc, "index_query", lambda qg: np.asarray(qg, float).sum(axis=0) * 0.0)

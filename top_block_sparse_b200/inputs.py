@@ -42,6 +42,8 @@ class Workload:
     window_keys: int
     n_needles: int
     prefill: bool = False
+    pool_stride: int = 4  # LSA: raw keys per pool key; overlap: keys between window starts
+    pool_kernel: int = 0  # overlap: keys per compressed key
 
     @property
     def group(self) -> int:
@@ -68,6 +70,10 @@ WORKLOADS: Dict[str, Workload] = {
     # batch 4, C = 1,048,576, LSA pooling (4 -> 1, 128 pool keys per block)
     "decode_1m": Workload("decode_1m", 4, 1, 32, 8, 128, 1048576, "bf16",
                           512, "lsa", 4, 4, 512, 32),
+    # decode_32k with overlapping compressed keys: windows of 32 keys every
+    # 16 keys (two windows per half block, neighbours sharing half their keys)
+    "decode_32k_overlap": Workload("decode_32k_overlap", 32, 1, 32, 8, 128, 32768, "bf16",
+                                   64, "overlap", 32, 64, 256, 16, pool_stride=16, pool_kernel=32),
     # batch 64, 6-token draft chunk, 16 / 8 heads, C = 16384
     "draft_chunk_16k": Workload("draft_chunk_16k", 64, 6, 16, 8, 128, 16384,
                                 "bf16", 64, "mean", 16, 64, 256, 8),
