@@ -9,7 +9,9 @@
  *      average-pooled into compressed keys), or LSA-style: each key
  *      L2-normalised, 4 consecutive unit keys summed into a pool key, the
  *      block centroid = the normalised sum of its pool keys (LSA review,
- *      §2.2);
+ *      §2.2); or into OVERLAPPING windows (SparDA "方法": InfLLM-V2 pools
+ *      keys into overlapping compressed representations, coarse to fine),
+ *      a block then scoring as the best window that touches it;
  *   2. one index query per (sequence, KV head) = the SUM of the query vectors
  *      of the GQA group (LSA review §2.4; SparDA "方法": one forecast head per
  *      GQA group) scores every compressed key: s_j = qbar.Kc_j * scale, or the
@@ -34,7 +36,9 @@
  *   O    : [B, n_q, Hq, d]            dtype = params.out_dtype
  *   lse  : [B, n_q, Hq] float32, natural log of the softmax denominator
  *   Kc   : [B, Hkv, nb, d] float32, nb = number of complete blocks
- *          (decode: floor(ctx_len / b); prefill: floor(n_q / b))
+ *          (decode: floor(ctx_len / b); prefill: floor(n_q / b));
+ *          SA_POOL_OVERLAP: [B, Hkv, n_c, d], n_c = the number of complete
+ *          windows = floor((ctx_len - l) / s) + 1 if ctx_len >= l, else 0
  *   idx  : decode / chunk: [B, Hkv, top_k] int32; prefill: [B, Hkv,
  *          n_tiles, top_k] int32 with n_tiles = ceil(n_q / b).  Block ids in
  *          ascending order, unused entries -1 at the end.
@@ -76,7 +80,7 @@ typedef enum {
 } sa_status;
 
 enum { SA_F32 = 0, SA_BF16 = 1 };                 /* element types */
-enum { SA_POOL_MEAN = 0, SA_POOL_LSA = 1 };       /* compression (step 1) */
+enum { SA_POOL_MEAN = 0, SA_POOL_LSA = 1, SA_POOL_OVERLAP = 2 };  /* compression (step 1) */
 enum { SA_SEL_QUERY0 = 0, SA_SEL_TILE_MAX = 1 };  /* how the index query is formed */
 enum {                                            /* ops for sa_workspace_size */
   SA_OP_SCORE_TOPK = 0,
@@ -87,7 +91,7 @@ enum {                                            /* ops for sa_workspace_size *
   SA_OP_COLUMN = 5
 };
 
-/* Problem description shared by every entry point (88 bytes). */
+/* Problem description shared by every entry point (96 bytes). */
 typedef struct sa_params {
   int32_t batch;          /* B >= 1 */
   int32_t num_q_heads;    /* Hq, a multiple of Hkv */
@@ -97,8 +101,10 @@ typedef struct sa_params {
   int64_t kv_capacity;    /* token stride of K and V, >= ctx_len + n_q */
   int32_t n_q;            /* new tokens per sequence (decode 1, draft chunk m, prefill T) */
   int32_t block_size;     /* b: keys per selectable block (a multiple of 16) */
-  int32_t pool;           /* SA_POOL_MEAN or SA_POOL_LSA */
-  int32_t pool_stride;    /* LSA: raw keys per pool key (divides b); ignored for mean */
+  int32_t pool;           /* SA_POOL_MEAN, SA_POOL_LSA or SA_POOL_OVERLAP */
+  int32_t pool_stride;    /* LSA: raw keys per pool key (divides b);
+                             OVERLAP: s, keys between window starts (divides b);
+                             ignored for mean */
   int32_t top_k;          /* k >= 0 blocks chosen by score */
   int32_t dtype;          /* SA_F32 or SA_BF16: element type of Q, K, V */
   int32_t out_dtype;      /* SA_F32 or SA_BF16: element type of O */
@@ -109,6 +115,8 @@ typedef struct sa_params {
   int64_t window_keys;    /* W >= 0 */
   float softmax_scale;    /* <= 0 selects 1/sqrt(head_dim) */
   int32_t flags;          /* OR of SA_FLAG_* (other bits must be 0) */
+  int32_t pool_kernel;    /* OVERLAP: l, keys per window, s <= l <= b; must be
+                             0 for the other pool modes */
 } sa_params;
 
 /* sa_params.flags: the caller's index table is known to hold only
@@ -131,6 +139,9 @@ sa_status sa_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Step 1 (compression) for every complete block of the context:
  * SA_POOL_MEAN: Kc[j] = (1/b) sum_{t=jb}^{jb+b-1} K[t] (SparDA "方法");
+ * SA_POOL_OVERLAP (decode / chunk only): Kc[c] = (1/l) sum_{t=cs}^{cs+l-1}
+ *               K[t] for every complete window c (l = pool_kernel,
+ *               s = pool_stride; SparDA "方法", overlapping compressed keys);
  * SA_POOL_LSA : Kc[j] = normalise(sum over the block's pool keys), a pool
  *               key being the sum of pool_stride consecutive L2-normalised
  *               keys (LSA review §2.2).
@@ -146,7 +157,11 @@ sa_status sa_pool_keys(const sa_params* p, const void* K, float* Kc, void* strea
  * layouts).  scores (optional, may be NULL): fp32 block scores,
  * [B, Hkv, nb] for SA_SEL_QUERY0 or [B, Hkv, n_tiles, nb] for
  * SA_SEL_TILE_MAX.  Kc may be NULL when the context holds no complete
- * block. */
+ * block.  SA_POOL_OVERLAP (SA_SEL_QUERY0 only): every window is scored as
+ * above and block j takes the largest score among the complete windows
+ * [cs, cs + l) that share a key with [jb, jb + b) (the coarse-to-fine step;
+ * the pages do not fix the rule, the max is this library's reading);
+ * scores then holds those block scores. */
 sa_status sa_score_topk(const sa_params* p, const void* Q, const float* Kc,
                         int32_t* idx, float* scores, void* ws, size_t ws_bytes,
                         void* stream);
@@ -235,7 +250,7 @@ sa_status sa_column_attn(const sa_params* p, const void* Q, const void* K,
 
 /* Number of kernels one sa_sparse_attn_decode call with `p` launches on this
  * device: 1 when scoring, top-k and attention run as one cooperative launch
- * (bf16, mean pooling, at most 512 complete blocks), else 2; 0 if p is
+ * (bf16, SA_POOL_MEAN or SA_POOL_LSA, at most 512 complete blocks), else 2; 0 if p is
  * invalid.  A cooperative launch the device refuses at run time falls back
  * to the 2-kernel path.  Host only; launches nothing. */
 int32_t sa_decode_launches(const sa_params* p);
@@ -245,7 +260,8 @@ int32_t sa_decode_launches(const sa_params* p);
  * scores every query tile of b rows against the compressed keys of the
  * blocks before it, selects per (tile, KV head) and runs causal sparse
  * attention: tile i attends sink U window U selected U its own keys
- * (causal).  Writes O, lse (optional), idx_out (optional). */
+ * (causal).  Writes O, lse (optional), idx_out (optional).  SA_POOL_LSA
+ * and SA_POOL_OVERLAP return SA_ERR_UNSUPPORTED here. */
 sa_status sa_sparse_attn_prefill(const sa_params* p, const void* Q,
                                  const void* K, const void* V, float* Kc,
                                  void* O, float* lse, int32_t* idx_out,

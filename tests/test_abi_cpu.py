@@ -33,11 +33,11 @@ def test_library_exports_every_declared_symbol():
     for name in declared_functions():
         assert hasattr(lib, name), name
     assert set(declared_functions()) <= set(sa.EXPORTED) | set(declared_functions())
-    assert sa.version() == 101
+    assert sa.version() == 102
 
 
 def test_params_struct_layout():
-    assert ctypes.sizeof(sa.SaParams) == 88
+    assert ctypes.sizeof(sa.SaParams) == 96
     assert sa.SaParams.sink_keys.offset == 64
     assert sa.SaParams.softmax_scale.offset == 80
 
@@ -68,6 +68,36 @@ def _decode(p, ws_bytes=1 << 30, q=FAKE, kc=FAKE):
 def test_validation_rejects(kw, status):
     assert _decode(_p(**kw)) == status
     assert sa.raw_call("sa_last_error").decode() != ""
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(pool="overlap", pool_stride=24, pool_kernel=32), sa.SA_ERR_INVALID),   # s does not divide b
+    (dict(pool="overlap", pool_stride=16, pool_kernel=8), sa.SA_ERR_INVALID),    # l < s
+    (dict(pool="overlap", pool_stride=16, pool_kernel=80), sa.SA_ERR_INVALID),   # l > b
+    (dict(pool="overlap", pool_stride=0, pool_kernel=32), sa.SA_ERR_INVALID),
+])
+def test_overlap_validation_rejects(kw, status):
+    assert _decode(_p(**kw)) == status
+    assert "pool" in sa.raw_call("sa_last_error").decode()
+
+
+def test_overlap_params_and_workspace():
+    """pool_kernel must be 0 outside the overlap mode; the overlap mode runs
+    as two kernels (scoring, attention), its prefill is not built, and its
+    scoring workspace holds one score per window."""
+    p = _p()
+    p.pool_kernel = 8
+    assert _decode(p) == sa.SA_ERR_INVALID
+    ov = _p(pool="overlap", pool_stride=16, pool_kernel=32)
+    assert sa.raw_call("sa_decode_launches", ctypes.byref(ov)) == 2
+    assert sa.raw_call("sa_decode_launches", ctypes.byref(_p())) in (1, 2)
+    pf = _p(pool="overlap", pool_stride=16, pool_kernel=32, prefill=True, ctx_len=0, n_q=4096,
+            num_q_heads=8, num_kv_heads=2)
+    assert sa.raw_call("sa_pool_keys", ctypes.byref(pf), FAKE, FAKE, None) == sa.SA_ERR_UNSUPPORTED
+    w_mean = sa.raw_call("sa_workspace_size", ctypes.byref(_p()), sa.SA_OP_SCORE_TOPK)
+    w_ovl = sa.raw_call("sa_workspace_size", ctypes.byref(ov), sa.SA_OP_SCORE_TOPK)
+    n_c = (4096 - 32) // 16 + 1
+    assert w_ovl >= w_mean + 4 * 4 * (n_c - 4096 // 64) - 1024
 
 
 def test_validation_null_and_alignment():

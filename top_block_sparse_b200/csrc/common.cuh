@@ -152,6 +152,11 @@ __device__ __forceinline__ uint32_t float_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Inverse of float_key.
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 // ---- workspace header ------------------------------------------------------
 // [0, 256): status word at offset 0, rest reserved.
 constexpr size_t kWsHeader = 256;

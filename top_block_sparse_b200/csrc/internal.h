@@ -16,32 +16,44 @@ struct DecodeGeom {
   int64_t C, cap, kv_end;          // context length, token stride, C + n_q
   int b;                           // block size
   int64_t nb;                      // complete blocks of the context
+  int64_t kc_rows;                 // rows of Kc per pair (nb, or the windows of SA_POOL_OVERLAP)
+  int64_t n_rows;                  // rows of Kc that scoring reads (the windows touching a complete block)
+  int ov_s, ov_l;                  // SA_POOL_OVERLAP window stride and length (0 otherwise)
   int64_t s_end, w_begin;          // sink [0, s_end), window [w_begin, C)
   int pairs;                       // B * Hkv
 };
 
 // ---- pooling ----------------------------------------------------------------
+// Row j of a pair's Kc compresses keys [j * stride, j * stride + len).
 struct PoolArgs {
   const void* K;
   float* Kc;
   int pairs;
   int64_t cap;      // token stride of K
-  int64_t nb;       // blocks per pair
-  int b;
-  int lsa;          // 0 mean, 1 LSA centroid
+  int64_t nb;       // rows of Kc per pair
+  int64_t stride;   // keys between row starts (b, or s of SA_POOL_OVERLAP)
+  int len;          // keys per row (b, or l of SA_POOL_OVERLAP)
+  int lsa;          // 0 mean, 1 LSA centroid (len == stride)
 };
 cudaError_t launch_pool(const PoolArgs& a, bool bf16, cudaStream_t s);
 
 // ---- decode scoring + top-k --------------------------------------------------
+// SA_POOL_OVERLAP (ov_s > 0): the rows are windows of ov_l keys every ov_s
+// keys; block j's score is the max over the windows touching it.
 struct ScoreArgs {
   const void* Q;
-  const float* Kc;
-  float* scores;          // [pairs, nb]; may be null when chunks == 1
+  const float* Kc;        // [pairs, kc_rows, d]
+  float* scores;          // [pairs, nb] block scores; may be null when chunks == 1
+                          // (or, with ov_s > 0, when the caller wants none)
+  float* cscores;         // ov_s > 0 and chunks > 1: [pairs, n_rows] window scores
   int32_t* idx;           // [pairs, top_k]
   unsigned* counters;     // [pairs], zero between calls
   unsigned* status;       // workspace status word
   int B, Hq, Hkv, G, n_q;
   int64_t nb;
+  int64_t kc_rows;        // Kc rows per pair
+  int64_t n_rows;         // rows scored per pair (a prefix of the kc_rows)
+  int ov_s, ov_l;         // window stride and length; 0 = one row per block
   int b;
   int64_t s_end, w_begin;
   int top_k;

@@ -3,11 +3,15 @@
 //   mean : Kc[j] = (1/b) * sum of the b keys of block j
 //          (SparDA summary, section "方法": keys average-pooled into
 //          compressed keys)
+//   overlapping windows: Kc[c] = (1/l) * sum of the l keys from c*s, for
+//          every complete window (same section: InfLLM-V2 pools into
+//          overlapping compressed representations); the same kernel with
+//          row start c*s and row length l
 //   LSA  : Kc[j] = normalise(sum_t K_t / |K_t|) over the block's keys, which
 //          equals the normalised sum of its pool keys (each pool key being the
 //          sum of 4 consecutive unit keys) (LSA review §2.2)
 //
-// One warp per block, one pass over K with 128-bit coalesced loads: for bf16
+// One warp per row, one pass over K with 128-bit coalesced loads: for bf16
 // a row of 128 elements is 256 B = 16 lanes x 16 B, so one warp load covers
 // two rows; for fp32 a row is 512 B = 32 lanes x 16 B.  Sums are kept in
 // fp32 registers; the output is fp32 (set parity of the later top-k needs
@@ -28,17 +32,17 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(PoolArgs a) {
   if (w >= total) return;
   const int64_t pair = w / a.nb;
   const int64_t j = w - pair * a.nb;
-  const int b = a.b;
+  const int len = a.len;
   float* out = a.Kc + (pair * a.nb + j) * kHeadDim;
 
   if constexpr (BF16) {
     // lane -> row parity (lane >> 4), 16-byte chunk (lane & 15) = elements 8c..8c+7
-    const uint16_t* base = static_cast<const uint16_t*>(a.K) + (pair * a.cap + j * b) * kHeadDim;
+    const uint16_t* base = static_cast<const uint16_t*>(a.K) + (pair * a.cap + j * a.stride) * kHeadDim;
     const int half = lane >> 4, c = lane & 15;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    const int rows2 = b >> 1;                      // row pairs
+    const int rows2 = len >> 1;                    // row pairs
     int i = 0;
     for (; i + 4 <= rows2; i += 4) {
       uint4 u[4];
@@ -62,6 +66,15 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(PoolArgs a) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) acc[e] += f[e];
         }
+      }
+    }
+    if constexpr (!LSA) {
+      // an odd row count leaves one row for the lower half-warp
+      if ((len & 1) && half == 0) {
+        float f[8];
+        unpack8(__ldg(reinterpret_cast<const uint4*>(base + (len - 1) * kHeadDim) + c), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += f[e];
       }
     }
     for (; i < rows2; ++i) {
@@ -93,7 +106,7 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(PoolArgs a) {
       for (int o = 1; o < 16; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       mul = ss > 0.f ? rsqrtf(ss) : 0.f;
     } else {
-      mul = 1.f / static_cast<float>(b);
+      mul = 1.f / static_cast<float>(len);
     }
     if (half == 0) {
       float4* o4 = reinterpret_cast<float4*>(out + 8 * c);
@@ -102,10 +115,10 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(PoolArgs a) {
     }
   } else {
     // fp32: lane -> 16-byte chunk = elements 4*lane..4*lane+3 of every row
-    const float* base = static_cast<const float*>(a.K) + (pair * a.cap + j * b) * kHeadDim;
+    const float* base = static_cast<const float*>(a.K) + (pair * a.cap + j * a.stride) * kHeadDim;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     int i = 0;
-    for (; i + 4 <= b; i += 4) {
+    for (; i + 4 <= len; i += 4) {
       float4 u[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k)
@@ -123,7 +136,7 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(PoolArgs a) {
         acc[2] += u[k].z * inv; acc[3] += u[k].w * inv;
       }
     }
-    for (; i < b; ++i) {
+    for (; i < len; ++i) {
       float4 u = __ldg(reinterpret_cast<const float4*>(base + i * kHeadDim) + lane);
       float inv = 1.f;
       if constexpr (LSA) {
@@ -141,7 +154,7 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(PoolArgs a) {
       for (int o = 1; o < 32; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       mul = ss > 0.f ? rsqrtf(ss) : 0.f;
     } else {
-      mul = 1.f / static_cast<float>(b);
+      mul = 1.f / static_cast<float>(len);
     }
     reinterpret_cast<float4*>(out)[lane] =
         make_float4(acc[0] * mul, acc[1] * mul, acc[2] * mul, acc[3] * mul);

@@ -60,9 +60,16 @@ sa_status check_params(const sa_params* p, bool prefill) {
                 (long long)(p->ctx_len + p->n_q));
   if (p->block_size < 16 || p->block_size % 16 != 0 || p->block_size > 65536)
     return fail(SA_ERR_INVALID, "block_size %d must be a multiple of 16 in [16, 65536]", p->block_size);
-  if (p->pool != SA_POOL_MEAN && p->pool != SA_POOL_LSA) return fail(SA_ERR_INVALID, "pool %d", p->pool);
-  if (p->pool == SA_POOL_LSA && (p->pool_stride < 1 || p->block_size % p->pool_stride != 0))
+  if (p->pool != SA_POOL_MEAN && p->pool != SA_POOL_LSA && p->pool != SA_POOL_OVERLAP)
+    return fail(SA_ERR_INVALID, "pool %d", p->pool);
+  if ((p->pool == SA_POOL_LSA || p->pool == SA_POOL_OVERLAP) &&
+      (p->pool_stride < 1 || p->block_size % p->pool_stride != 0))
     return fail(SA_ERR_INVALID, "pool_stride %d must divide block_size %d", p->pool_stride, p->block_size);
+  if (p->pool == SA_POOL_OVERLAP && (p->pool_kernel < p->pool_stride || p->pool_kernel > p->block_size))
+    return fail(SA_ERR_INVALID, "pool_kernel %d must lie in [pool_stride %d, block_size %d]", p->pool_kernel,
+                p->pool_stride, p->block_size);
+  if (p->pool != SA_POOL_OVERLAP && p->pool_kernel != 0)
+    return fail(SA_ERR_INVALID, "pool_kernel must be 0 unless pool = SA_POOL_OVERLAP");
   if (p->top_k < 0 || p->top_k > 4096) return fail(SA_ERR_INVALID, "top_k %d must be in [0, 4096]", p->top_k);
   if (p->sink_keys < 0 || p->window_keys < 0) return fail(SA_ERR_INVALID, "sink_keys and window_keys must be >= 0");
   if (p->select != SA_SEL_QUERY0 && p->select != SA_SEL_TILE_MAX) return fail(SA_ERR_INVALID, "select %d", p->select);
@@ -88,6 +95,17 @@ DecodeGeom decode_geom(const sa_params* p) {
   g.kv_end = p->ctx_len + p->n_q;
   g.b = p->block_size;
   g.nb = p->ctx_len / p->block_size;
+  g.kc_rows = g.nb;
+  g.n_rows = g.nb;
+  g.ov_s = g.ov_l = 0;
+  if (p->pool == SA_POOL_OVERLAP) {
+    g.ov_s = p->pool_stride;
+    g.ov_l = p->pool_kernel;
+    g.kc_rows = g.C >= g.ov_l ? (g.C - g.ov_l) / g.ov_s + 1 : 0;
+    // windows starting at or past the last complete block's end touch no
+    // complete block (s divides b, so block j's windows start below (j+1)b)
+    g.n_rows = std::min<int64_t>(g.kc_rows, g.nb * (g.b / g.ov_s));
+  }
   g.s_end = p->sink_keys < g.C ? p->sink_keys : g.C;
   const int64_t wb = g.C - p->window_keys;
   g.w_begin = wb > g.s_end ? wb : g.s_end;
@@ -117,7 +135,7 @@ DecodeWs decode_ws(const DecodeGeom& g, const DecodePlan& plan, int top_k, int o
   w.score_cnt = take(pairs * 4);
   w.attn_cnt = take(pairs * 4);
   if (op == SA_OP_SCORE_TOPK || op == SA_OP_DECODE) {
-    w.scores = take(pairs * static_cast<size_t>(g.nb) * 4);
+    w.scores = take(pairs * static_cast<size_t>(std::max(g.nb, g.n_rows)) * 4);
   }
   if (op == SA_OP_DECODE) {
     w.idx = take(pairs * static_cast<size_t>(top_k) * 4);
@@ -167,6 +185,10 @@ ScoreArgs score_args(const sa_params* p, const DecodeGeom& g, const void* Q, con
   a.G = g.G;
   a.n_q = g.n_q;
   a.nb = g.nb;
+  a.kc_rows = g.kc_rows;
+  a.n_rows = g.n_rows;
+  a.ov_s = g.ov_s;
+  a.ov_l = g.ov_l;
   a.b = g.b;
   a.s_end = g.s_end;
   a.w_begin = g.w_begin;
@@ -175,12 +197,17 @@ ScoreArgs score_args(const sa_params* p, const DecodeGeom& g, const void* Q, con
   a.lsa = p->pool == SA_POOL_LSA;
   // as many chunks per pair as keep every CTA resident (two per SM)
   const int64_t pairs = std::max<int64_t>(1, g.pairs);
-  const int64_t passes = std::max<int64_t>(1, (g.nb + kScoreRowsPerPass - 1) / kScoreRowsPerPass);
+  const int64_t passes = std::max<int64_t>(1, (g.n_rows + kScoreRowsPerPass - 1) / kScoreRowsPerPass);
   const int64_t want = std::min<int64_t>(passes, std::max<int64_t>(1, 2 * device_sms() / pairs));
   const int64_t per = (passes + want - 1) / want;
   a.rows_per_chunk = per * kScoreRowsPerPass;
   a.chunks = static_cast<int>((passes + per - 1) / per);
-  a.scores = caller_scores ? caller_scores : (a.chunks > 1 ? ws_scores : nullptr);
+  if (g.ov_s > 0) {
+    a.scores = caller_scores;
+    a.cscores = a.chunks > 1 ? ws_scores : nullptr;
+  } else {
+    a.scores = caller_scores ? caller_scores : (a.chunks > 1 ? ws_scores : nullptr);
+  }
   return a;
 }
 
@@ -304,7 +331,7 @@ using namespace sa;
 
 extern "C" {
 
-int32_t sa_version(void) { return 101; }
+int32_t sa_version(void) { return 102; }
 
 const char* sa_last_error(void) { return g_err; }
 
@@ -419,8 +446,13 @@ sa_status sa_pool_keys(const sa_params* p, const void* K, float* Kc, void* strea
   const bool prefill = p && p->select == SA_SEL_TILE_MAX;
   sa_status st = check_params(p, prefill);
   if (st != SA_OK) return st;
-  const int64_t nb = (prefill ? static_cast<int64_t>(p->n_q) : p->ctx_len) / p->block_size;
-  if (nb == 0) return SA_OK;   // no complete block: nothing to write
+  if (prefill && p->pool == SA_POOL_OVERLAP)
+    return fail(SA_ERR_UNSUPPORTED, "overlapping windows are built for decode and draft chunks");
+  const int64_t keys = prefill ? static_cast<int64_t>(p->n_q) : p->ctx_len;
+  const bool ovl = p->pool == SA_POOL_OVERLAP;
+  const int64_t rows = ovl ? (keys >= p->pool_kernel ? (keys - p->pool_kernel) / p->pool_stride + 1 : 0)
+                           : keys / p->block_size;
+  if (rows == 0) return SA_OK;   // no complete block / window: nothing to write
   if (!K || !Kc) return fail(SA_ERR_INVALID, "K and Kc must be non-NULL");
   if (!aligned16(K) || !aligned16(Kc)) return fail(SA_ERR_INVALID, "K and Kc must be 16-byte aligned");
   PoolArgs a = {};
@@ -428,8 +460,9 @@ sa_status sa_pool_keys(const sa_params* p, const void* K, float* Kc, void* strea
   a.Kc = Kc;
   a.pairs = p->batch * p->num_kv_heads;
   a.cap = p->kv_capacity;
-  a.nb = nb;
-  a.b = p->block_size;
+  a.nb = rows;
+  a.stride = ovl ? p->pool_stride : p->block_size;
+  a.len = ovl ? p->pool_kernel : p->block_size;
   a.lsa = p->pool == SA_POOL_LSA;
   cudaError_t e = launch_pool(a, p->dtype == SA_BF16, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "pool kernel launch");
@@ -560,7 +593,7 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q, const void* K
   if (p->dtype == SA_BF16 && g.nb >= 1) {
     // one cooperative launch: scores, top-k and attention
     DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, idx, p->top_k, O, lse, w, L);
-    if (decode_fused_supported(a, plan, g.nb, p->pool == SA_POOL_LSA)) {
+    if (p->pool != SA_POOL_OVERLAP && decode_fused_supported(a, plan, g.nb, p->pool == SA_POOL_LSA)) {
       a.Kc = Kc;
       a.scores = reinterpret_cast<float*>(w + L.scores);
       a.score_cnt = reinterpret_cast<unsigned*>(w + L.score_cnt);
@@ -684,7 +717,7 @@ int32_t sa_decode_launches(const sa_params* p) {
     const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_DECODE);
     DecodeAttnArgs a = attn_args(p, g, plan, nullptr, nullptr, nullptr, nullptr, p->top_k, nullptr, nullptr,
                                  nullptr, L);
-    if (decode_fused_supported(a, plan, g.nb, p->pool == SA_POOL_LSA)) return 1;
+    if (p->pool != SA_POOL_OVERLAP && decode_fused_supported(a, plan, g.nb, p->pool == SA_POOL_LSA)) return 1;
   }
   return 2;
 }

@@ -5,6 +5,10 @@
 // group, here the sum of the group's queries of the first new token):
 //   mean pooling: s_j = qbar . Kc_j * scale
 //   LSA         : s_j = (qbar / |qbar|) . Kc_j   (cosine, LSA review §2.3)
+// Overlapping compressed keys (SparDA "方法": InfLLM-V2 pools keys into
+// overlapping compressed representations, coarse to fine): every window is
+// scored the same way and block j takes the max over the windows that share
+// a key with it.
 // Candidates: complete blocks not wholly inside sink [0, s_end) or window
 // [w_begin, C) (SparDA "方法": initial + local + top-k blocks).
 // Selection: the k largest by (score desc, block id asc), written in
@@ -16,9 +20,10 @@
 // cp.async.bulk (the TMA engine keeps far more bytes in flight per SM than
 // per-thread loads); a warp scores 8 rows of a stage with a shuffle reduction
 // per row.  With one chunk per pair the CTA builds the selection keys in
-// shared memory and selects; with several, CTAs write scores and the CTA that
-// finishes last for the pair (atomic ticket, no waiting) reads them back and
-// selects.
+// shared memory (windows: an atomicMax of the order-preserving key into each
+// block they touch) and selects; with several, CTAs write scores and the CTA
+// that finishes last for the pair (atomic ticket, no waiting) reads them back
+// and selects.
 #include <math_constants.h>
 
 #include "common.cuh"
@@ -63,12 +68,14 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_topk_query0_kernel(Sco
   const int bi = pair / a.Hkv, h = pair % a.Hkv;
   const bool single = a.chunks == 1;
 
-  const int64_t j_begin = min(a.nb, static_cast<int64_t>(chunk) * a.rows_per_chunk);
-  const int64_t j_end = min(a.nb, j_begin + a.rows_per_chunk);
+  const bool ovl = a.ov_s > 0;
+  const int64_t j_begin = min(a.n_rows, static_cast<int64_t>(chunk) * a.rows_per_chunk);
+  const int64_t j_end = min(a.n_rows, j_begin + a.rows_per_chunk);
   const int nrows = static_cast<int>(j_end - j_begin);
   const int nst = (nrows + kStageRows - 1) / kStageRows;
-  const float* kc = a.Kc + (static_cast<int64_t>(pair) * a.nb + j_begin) * kHeadDim;
+  const float* kc = a.Kc + (static_cast<int64_t>(pair) * a.kc_rows + j_begin) * kHeadDim;
   float* sc = a.scores ? a.scores + static_cast<int64_t>(pair) * a.nb : nullptr;
+  float* csc = a.cscores ? a.cscores + static_cast<int64_t>(pair) * a.n_rows : nullptr;
 
   if (tid == 0) {
     for (int s = 0; s < kScoreStages; ++s) mbar_init(&full[s], 1);
@@ -98,6 +105,8 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_topk_query0_kernel(Sco
     }
     qs[tid] = s;
   }
+  if (ovl && single)
+    for (int64_t j = tid; j < a.nb; j += kScoreThreads) keys[j] = 0u;
   __syncthreads();
   if (a.lsa) {
     if (warp == 0) {
@@ -139,8 +148,19 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_topk_query0_kernel(Sco
       for (int u = 1; u < kRowsPerWarp; ++u) mine = (lane == u) ? d[u] : mine;
       const int64_t j = j_begin + static_cast<int64_t>(st) * kStageRows + r0 + lane;
       if (lane < kRowsPerWarp && j < j_end) {
-        if (sc) sc[j] = mine;
-        if (single) keys[j] = block_key(a, j, mine);
+        if (!ovl) {
+          if (sc) sc[j] = mine;
+          if (single) keys[j] = block_key(a, j, mine);
+        } else {
+          if (csc) csc[j] = mine;
+          if (single) {
+            // window j covers keys [j*s, j*s + l): blocks t0/b .. (t0+l-1)/b
+            const uint32_t key = float_key(mine);
+            const int64_t t0 = j * a.ov_s;
+            const int64_t last = min(a.nb - 1, (t0 + a.ov_l - 1) / a.b);
+            for (int64_t jb = t0 / a.b; jb <= last; ++jb) atomicMax(&keys[jb], key);
+          }
+        }
       }
     } else if (lane == 0) {
       report(a.status, kStatusTimeout);
@@ -174,7 +194,27 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_topk_query0_kernel(Sco
     __threadfence();
     if (tid == 0) a.counters[pair] = 0u;
     // the pair's scores come back from L2
-    for (int64_t j = tid; j < a.nb; j += kScoreThreads) keys[j] = block_key(a, j, __ldcg(sc + j));
+    if (!ovl) {
+      for (int64_t j = tid; j < a.nb; j += kScoreThreads) keys[j] = block_key(a, j, __ldcg(sc + j));
+    } else {
+      // block j: windows c_lo = ceil((jb - l + 1) / s) .. c_hi = ((j+1)b - 1) / s
+      for (int64_t j = tid; j < a.nb; j += kScoreThreads) {
+        const int64_t lo = j * a.b - a.ov_l + 1;
+        const int64_t c_lo = lo <= 0 ? 0 : (lo + a.ov_s - 1) / a.ov_s;
+        const int64_t c_hi = min(a.n_rows - 1, ((j + 1) * a.b - 1) / a.ov_s);
+        float m = -CUDART_INF_F;
+        for (int64_t c = c_lo; c <= c_hi; ++c) m = fmaxf(m, __ldcg(csc + c));
+        if (sc) sc[j] = m;
+        keys[j] = block_key(a, j, m);
+      }
+    }
+  } else if (ovl) {
+    __syncthreads();
+    for (int64_t j = tid; j < a.nb; j += kScoreThreads) {
+      const float m = key_float(keys[j]);
+      if (sc) sc[j] = m;
+      keys[j] = block_key(a, j, m);
+    }
   }
   __syncthreads();
   const int nb = static_cast<int>(a.nb);

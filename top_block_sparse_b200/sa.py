@@ -23,7 +23,7 @@ _lib = ctypes.CDLL(_LIB_PATH)
 # ---- constants mirrored from sa.h ------------------------------------------
 SA_OK, SA_ERR_INVALID, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_INDEX, SA_ERR_CUDA, SA_ERR_TIMEOUT = range(7)
 SA_F32, SA_BF16 = 0, 1
-SA_POOL_MEAN, SA_POOL_LSA = 0, 1
+SA_POOL_MEAN, SA_POOL_LSA, SA_POOL_OVERLAP = 0, 1, 2
 SA_SEL_QUERY0, SA_SEL_TILE_MAX = 0, 1
 SA_OP_SCORE_TOPK, SA_OP_GIVEN_IDX, SA_OP_DECODE, SA_OP_PREFILL, SA_OP_VERIFY, SA_OP_COLUMN = 0, 1, 2, 3, 4, 5
 SA_FLAG_TRUSTED_IDX = 1
@@ -45,10 +45,11 @@ class SaParams(ctypes.Structure):
         ("out_dtype", ctypes.c_int32), ("select", ctypes.c_int32),
         ("sink_keys", ctypes.c_int64), ("window_keys", ctypes.c_int64),
         ("softmax_scale", ctypes.c_float), ("flags", ctypes.c_int32),
+        ("pool_kernel", ctypes.c_int32),
     ]
 
 
-assert ctypes.sizeof(SaParams) == 88
+assert ctypes.sizeof(SaParams) == 96
 
 _vp, _sz, _i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
 _P = ctypes.POINTER(SaParams)
@@ -92,7 +93,7 @@ def version() -> int:
 
 def make_params(*, batch, num_q_heads, num_kv_heads, ctx_len, n_q, block_size, top_k,
                 sink_keys, window_keys, dtype="bf16", out_dtype=None, pool="mean",
-                pool_stride=4, kv_capacity=None, prefill=False, softmax_scale=0.0,
+                pool_stride=4, pool_kernel=0, kv_capacity=None, prefill=False, softmax_scale=0.0,
                 head_dim=128) -> SaParams:
     dt = SA_BF16 if dtype == "bf16" else SA_F32
     odt = dt if out_dtype is None else (SA_BF16 if out_dtype == "bf16" else SA_F32)
@@ -100,7 +101,8 @@ def make_params(*, batch, num_q_heads, num_kv_heads, ctx_len, n_q, block_size, t
                     head_dim=head_dim, ctx_len=ctx_len,
                     kv_capacity=(ctx_len + n_q) if kv_capacity is None else kv_capacity,
                     n_q=n_q, block_size=block_size,
-                    pool=SA_POOL_LSA if pool == "lsa" else SA_POOL_MEAN, pool_stride=pool_stride,
+                    pool={"mean": SA_POOL_MEAN, "lsa": SA_POOL_LSA, "overlap": SA_POOL_OVERLAP}[pool],
+                    pool_stride=pool_stride, pool_kernel=pool_kernel if pool == "overlap" else 0,
                     top_k=top_k, dtype=dt, out_dtype=odt,
                     select=SA_SEL_TILE_MAX if prefill else SA_SEL_QUERY0,
                     sink_keys=sink_keys, window_keys=window_keys,
@@ -112,7 +114,8 @@ def params_for(w, kv_capacity=None, out_dtype=None) -> SaParams:
     return make_params(batch=w.batch, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
                        ctx_len=w.ctx_len, n_q=w.n_q, block_size=w.block_size, top_k=w.top_k,
                        sink_keys=w.sink_keys, window_keys=w.window_keys, dtype=w.dtype,
-                       out_dtype=out_dtype, pool=w.pool, kv_capacity=kv_capacity,
+                       out_dtype=out_dtype, pool=w.pool, pool_stride=w.pool_stride,
+                       pool_kernel=w.pool_kernel, kv_capacity=kv_capacity,
                        prefill=w.prefill, head_dim=w.head_dim)
 
 
