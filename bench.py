@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload decode_32k] [--no-cpu-baseline] [--no-prefill] [--no-verify]
-                    [--no-column]
+                    [--no-column] [--no-overlap]
 
 Workload (default): batched decode, batch 32, 32 query / 8 KV heads, d = 128,
 context T = 32768, bf16 KV cache with fp32 accumulation, block 64, top-k 32 +
@@ -24,7 +24,8 @@ Printed: one JSON line (rank 0).  ``value`` = sequences decoded per second
 (whole job).  Also: the roofline of the step's one kernel (algorithmic bytes
 over the timed launch, against the measured copy bandwidth), the attention
 kernel alone on the same table, the causal prefill, the dense verify of a
-draft chunk and column-sparse attention (each with its kernels' rooflines),
+draft chunk, column-sparse attention and the decode step with overlapping
+compressed keys (each with its kernels' rooflines),
 the end-to-end number
 through the C ABI with host buffers, clocks sampled during the timed region,
 and the float64 CPU oracle timed on a bounded sample (rank 0, N = 1).
@@ -376,6 +377,10 @@ def run_ours(args, w, rank, world, local_rank):
     column = None
     if not args.no_column:
         column = run_column_bench(args, dev, stream, flush)
+    # --- decode with overlapping compressed keys, rank-local ------------------
+    overlap = None
+    if not args.no_overlap:
+        overlap = run_overlap_bench(args, dev, stream, flush)
     # --- end to end through the C ABI with host buffers -------------------
     e2e = e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush)
     e2e["ms"] = reduce_max(e2e["ms"], world, dev)
@@ -421,6 +426,7 @@ def run_ours(args, w, rank, world, local_rank):
         "prefill": prefill,
         "verify": verify,
         "column": column,
+        "overlap": overlap,
         "gpu_launches": sa.decode_launches(p) * args.steps,
         "clocks": clk.summary(),
     }
@@ -623,6 +629,75 @@ def run_column_bench(args, dev, stream, flush):
     }
 
 
+def run_overlap_bench(args, dev, stream, flush):
+    """Times the decode step with overlapping compressed keys on the 32k
+    decode workload (windows of 32 keys every 16 keys, block = max over the
+    windows touching it): one sa_sparse_attn_decode call = the scoring +
+    top-k kernel over the windows, then the attention kernel.  Also the
+    scoring kernel alone (sa_score_topk) and the window pooling."""
+    from top_block_sparse_b200 import sa
+    w = WORKLOADS["decode_32k_overlap"]
+    if args.batch:
+        w = w.scaled(batch=args.batch)
+    inp = make_inputs(w, seed=5001, device=dev)
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    del inp
+    p = sa.params_for(w, out_dtype="bf16")
+    pairs = w.batch * w.num_kv_heads
+    nb = w.ctx_len // w.block_size
+    n_c = (w.ctx_len - w.pool_kernel) // w.pool_stride + 1
+    n_rows = min(n_c, nb * (w.block_size // w.pool_stride))     # windows touching a complete block
+    Kc = torch.empty((w.batch, w.num_kv_heads, n_c, 128), device=dev)
+    O = torch.empty((w.batch, w.n_q, w.num_q_heads, 128), device=dev, dtype=torch.bfloat16)
+    lse = torch.empty((w.batch, w.n_q, w.num_q_heads), device=dev)
+    idx = torch.empty((w.batch, w.num_kv_heads, w.top_k), device=dev, dtype=torch.int32)
+    idx2 = torch.empty_like(idx)
+    ws = sa.alloc_workspace(p, sa.SA_OP_DECODE, device=dev)
+    ws_s = sa.alloc_workspace(p, sa.SA_OP_SCORE_TOPK, device=dev)
+
+    def pool():
+        sa.pool_keys(p, K, Kc, stream=stream)
+
+    def step():
+        sa.sparse_attn_decode(p, Q, K, V, Kc, O, lse, idx, ws, stream=stream)
+
+    def score():
+        sa.score_topk(p, Q, Kc, idx2, None, ws_s, stream=stream)
+
+    n = args.overlap_steps
+    pool_ms = statistics.mean(timed_steps(pool, 5, 3, stream, flush))
+    step_ms = statistics.mean(timed_steps(step, n, 3, stream, flush))
+    score_ms = statistics.mean(timed_steps(score, n, 3, stream, flush))
+    if sa.read_status(ws, stream) != sa.SA_OK or sa.read_status(ws_s, stream) != sa.SA_OK:
+        raise RuntimeError("device status word set during the overlapping-window runs")
+    if not torch.equal(idx, idx2):
+        raise RuntimeError("the decode step and sa_score_topk selected different blocks")
+    hbm, _, _, src = peaks()
+    by = decode_bytes(w)
+    win = pairs * n_rows * w.head_dim * 4
+    step_b = by["kv"] + win + 2 * by["q"] + by["o"]
+    score_b = win + by["q"] + pairs * w.top_k * 4
+    pool_b = pairs * (n_c * w.pool_stride * w.head_dim * 2 + n_c * w.head_dim * 4)
+    gbs = lambda b, ms: b / (ms * 1e-3) / 1e9
+    return {
+        "workload": f"decode_32k_overlap: B={w.batch}, Hq={w.num_q_heads}, Hkv={w.num_kv_heads}, C={w.ctx_len}, "
+                    f"d=128, bf16, block {w.block_size}, windows of {w.pool_kernel} keys every {w.pool_stride} "
+                    f"({n_rows} scored per pair, fp32), top-k {w.top_k}, sink {w.sink_keys}, window {w.window_keys}",
+        "ms": step_ms,
+        "queries_per_s": w.batch * w.n_q / (step_ms * 1e-3),
+        "launches": sa.decode_launches(p),
+        "algorithmic_bytes": step_b,
+        "achieved_gbs": gbs(step_b, step_ms), "frac": gbs(step_b, step_ms) / hbm,
+        "note": "algorithmic bytes = the scored windows (fp32) + the retained K and V rows + Q, O",
+        "scoring": {"kernel": "score_topk_query0_kernel (window scores, block max, radix top-k)", "ms": score_ms,
+                    "algorithmic_bytes": score_b, "gbs": gbs(score_b, score_ms),
+                    "frac": gbs(score_b, score_ms) / hbm},
+        "pool": {"kernel": "pool_kernel (overlapping windows)", "ms": pool_ms, "gbs": gbs(pool_b, pool_ms),
+                 "note": "bytes = each key once + the windows written; runs when blocks fill, not per step"},
+        "peak_gbs": hbm, "peak_source": src,
+    }
+
+
 def e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush):
     from top_block_sparse_b200 import sa
     C = w.ctx_len
@@ -667,6 +742,8 @@ def main():
     ap.add_argument("--no-verify", action="store_true")
     ap.add_argument("--column-steps", type=int, default=5)
     ap.add_argument("--no-column", action="store_true")
+    ap.add_argument("--overlap-steps", type=int, default=50)
+    ap.add_argument("--no-overlap", action="store_true")
     ap.add_argument("--column-tokens", type=int, default=None,
                     help="override the column workload's sequence length (smaller cases for ncu captures)")
     ap.add_argument("--prefill-tokens", type=int, default=None,
