@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload decode_32k] [--no-cpu-baseline] [--no-prefill] [--no-verify]
-                    [--no-column] [--no-overlap]
+                    [--no-column] [--no-overlap] [--no-configs]
 
 Workload (default): batched decode, batch 32, 32 query / 8 KV heads, d = 128,
 context T = 32768, bf16 KV cache with fp32 accumulation, block 64, top-k 32 +
@@ -24,8 +24,9 @@ Printed: one JSON line (rank 0).  ``value`` = sequences decoded per second
 (whole job).  Also: the roofline of the step's one kernel (algorithmic bytes
 over the timed launch, against the measured copy bandwidth), the attention
 kernel alone on the same table, the causal prefill, the dense verify of a
-draft chunk, column-sparse attention and the decode step with overlapping
-compressed keys (each with its kernels' rooflines),
+draft chunk, column-sparse attention, the decode step with overlapping
+compressed keys and the other decode workloads (tiny fp32, the 6-token draft
+chunk, the 1M-token LSA decode), each with its kernels' rooflines,
 the end-to-end number
 through the C ABI with host buffers, clocks sampled during the timed region,
 and the float64 CPU oracle timed on a bounded sample (rank 0, N = 1).
@@ -381,6 +382,10 @@ def run_ours(args, w, rank, world, local_rank):
     overlap = None
     if not args.no_overlap:
         overlap = run_overlap_bench(args, dev, stream, flush)
+    # --- the other decode workloads, rank-local ---------------------------------
+    configs = None
+    if not args.no_configs:
+        configs = run_decode_configs(args, dev, stream, flush)
     # --- end to end through the C ABI with host buffers -------------------
     e2e = e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush)
     e2e["ms"] = reduce_max(e2e["ms"], world, dev)
@@ -427,6 +432,7 @@ def run_ours(args, w, rank, world, local_rank):
         "verify": verify,
         "column": column,
         "overlap": overlap,
+        "decode_configs": configs,
         "gpu_launches": sa.decode_launches(p) * args.steps,
         "clocks": clk.summary(),
     }
@@ -629,6 +635,58 @@ def run_column_bench(args, dev, stream, flush):
     }
 
 
+def run_decode_configs(args, dev, stream, flush):
+    """Times one sa_sparse_attn_decode call (compressed keys maintained) on
+    each of the other decode workloads: the tiny fp32 decode, the 6-token
+    draft chunk and the 1M-token decode with LSA centroids (whose one-time
+    pooling of the whole context is timed too).  Median of
+    --config-steps L2-flushed steps after 5 warm-ups."""
+    from top_block_sparse_b200 import sa
+    hbm, _, _, src = peaks()
+    out = {"peak_gbs": hbm, "peak_source": src}
+    for name, seed in (("tiny_decode", 6001), ("draft_chunk_16k", 6002), ("decode_1m", 6003)):
+        w = WORKLOADS[name]
+        inp = make_inputs(w, seed=seed, device=dev)
+        Q, K, V = inp["Q"], inp["K"], inp["V"]
+        del inp
+        p = sa.params_for(w)
+        nb = w.ctx_len // w.block_size
+        Kc = torch.empty((w.batch, w.num_kv_heads, nb, 128), device=dev)
+        odt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+        O = torch.empty((w.batch, w.n_q, w.num_q_heads, 128), device=dev, dtype=odt)
+        lse = torch.empty((w.batch, w.n_q, w.num_q_heads), device=dev)
+        idx = torch.empty((w.batch, w.num_kv_heads, w.top_k), device=dev, dtype=torch.int32)
+        ws = sa.alloc_workspace(p, sa.SA_OP_DECODE, device=dev)
+
+        def pool():
+            sa.pool_keys(p, K, Kc, stream=stream)
+
+        def step():
+            sa.sparse_attn_decode(p, Q, K, V, Kc, O, lse, idx, ws, stream=stream)
+
+        pool_ms = statistics.median(timed_steps(pool, 3, 3, stream, flush))
+        ms = statistics.median(timed_steps(step, args.config_steps, 5, stream, flush))
+        if sa.read_status(ws, stream) != sa.SA_OK:
+            raise RuntimeError(f"device status word set during the {name} runs")
+        by = decode_bytes(w)
+        el = 2 if w.dtype == "bf16" else 4
+        pool_b = w.batch * w.num_kv_heads * (nb * w.block_size * w.head_dim * el + nb * w.head_dim * 4)
+        out[name] = {
+            "workload": f"B={w.batch}, n_q={w.n_q}, Hq={w.num_q_heads}, Hkv={w.num_kv_heads}, C={w.ctx_len}, "
+                        f"{w.dtype}, block {w.block_size}, {w.pool} pooling, top-k {w.top_k}, sink {w.sink_keys}, "
+                        f"window {w.window_keys}",
+            "ms": ms, "launches": sa.decode_launches(p),
+            "token_queries_per_s": w.batch * w.n_q / (ms * 1e-3),
+            "keys_per_query": by["keys_per_query"], "algorithmic_bytes": by["step"],
+            "gbs": by["step"] / (ms * 1e-3) / 1e9, "frac": by["step"] / (ms * 1e-3) / 1e9 / hbm,
+            "pool": {"ms": pool_ms, "gbs": pool_b / (pool_ms * 1e-3) / 1e9,
+                     "note": "one-time compression of the whole context (each key read once)"},
+        }
+        del Q, K, V, Kc, O, lse, idx, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_overlap_bench(args, dev, stream, flush):
     """Times the decode step with overlapping compressed keys on the 32k
     decode workload (windows of 32 keys every 16 keys, block = max over the
@@ -743,6 +801,8 @@ def main():
     ap.add_argument("--column-steps", type=int, default=5)
     ap.add_argument("--no-column", action="store_true")
     ap.add_argument("--overlap-steps", type=int, default=50)
+    ap.add_argument("--config-steps", type=int, default=30)
+    ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--no-overlap", action="store_true")
     ap.add_argument("--column-tokens", type=int, default=None,
                     help="override the column workload's sequence length (smaller cases for ncu captures)")

@@ -353,6 +353,13 @@ def test_fused_empty_tiles_after_score_chunks():
 
 def test_decode_32k_runs_as_one_launch():
     """The batched-decode workload takes the fused path (scores, top-k and
-    attention in one cooperative launch) on this device."""
-    assert sa.decode_launches(sa.params_for(WORKLOADS["decode_32k"])) == 1
-    assert sa.decode_launches(sa.params_for(WORKLOADS["tiny_decode"])) == 2     # fp32: two kernels
+    attention in one cooperative launch) on this device; draft chunks (12
+    query rows per KV head), more than two pairs per SM, fp32 and LSA
+    centroids take the scoring kernel and then the attention kernel."""
+    n = lambda w: sa.decode_launches(sa.params_for(w))
+    assert n(WORKLOADS["decode_32k"]) == 1
+    assert n(WORKLOADS["draft_chunk_16k"]) == 2
+    assert n(WORKLOADS["draft_chunk_16k"].scaled(n_q=2)) == 2        # 512 pairs
+    assert n(WORKLOADS["draft_chunk_16k"].scaled(n_q=2, batch=16)) == 1
+    assert n(WORKLOADS["tiny_decode"]) == 2                            # fp32
+    assert n(WORKLOADS["decode_1m"]) == 2                              # LSA centroids

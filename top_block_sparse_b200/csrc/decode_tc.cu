@@ -937,19 +937,25 @@ size_t decode_tc_smem_bytes() { return kSmemBytes; }
 
 TcOrder tc_order(int64_t pairs, int n_sink_tiles, int n_sel_tiles, int n_wc_tiles, bool split, int num_sms) {
   TcOrder o = {};
+  const int64_t sms = std::max(num_sms, 1);
+  int64_t pairs_i = pairs, pairs_d = pairs;
   if (split) {
     o.ntI = n_sink_tiles + n_wc_tiles;
     o.ntD = n_sel_tiles;
     o.dI = n_sel_tiles;
     o.dD = n_sink_tiles;
+    o.pI = pairs;
   } else {
-    o.ntD = n_sink_tiles + n_sel_tiles + n_wc_tiles;
+    // whole pairs first (the same number for every CTA), the rest split
+    o.ntI = o.ntD = n_sink_tiles + n_sel_tiles + n_wc_tiles;
+    o.pI = o.pD0 = (pairs / sms) * sms;
+    pairs_i = o.pI;
+    pairs_d = pairs - o.pI;
   }
   o.mI = (o.ntI + 1) / 2;
   o.mD = (o.ntD + 1) / 2;
-  o.totI = pairs * o.mI;
-  o.totD = pairs * o.mD;
-  const int64_t sms = std::max(num_sms, 1);
+  o.totI = pairs_i * o.mI;
+  o.totD = pairs_d * o.mD;
   o.gI = static_cast<int>(std::min(sms, o.totI));
   o.gD = static_cast<int>(std::min(sms, o.totD));
   o.grid = std::max(std::max(o.gI, o.gD), 1);
@@ -1046,8 +1052,14 @@ cudaError_t launch_decode_tc(const DecodeAttnArgs& a0, const DecodePlan& p, bool
 
 bool decode_fused_supported(const DecodeAttnArgs& a, const DecodePlan& p, int64_t nb, int lsa) {
   if (lsa || nb < 1 || nb > kFusedMaxBlocks || !decode_tc_supported(a)) return false;
-  const int64_t chunks = static_cast<int64_t>(a.B) * a.Hkv * ((nb + 127) / 128);
+  const int64_t pairs = static_cast<int64_t>(a.B) * a.Hkv;
+  const int64_t chunks = pairs * ((nb + 127) / 128);
   const int grid = p.tc_split.grid;
+  // Measured on B200: with more than 4 query rows per KV head (draft chunks)
+  // or more than two pairs per CTA, the per-pair partial results of the two
+  // split lists cost more than the second launch saves, and the scoring
+  // kernel + attention kernel (whole pairs first) is faster.
+  if (a.R > 4 || pairs > 2 * static_cast<int64_t>(grid)) return false;
   // at most one CTA per SM (shared memory), at most kMaxSelPerCta tickets per CTA
   return a.total_tiles > 0 && grid > 0 && (chunks + grid - 1) / grid <= kMaxSelPerCta;
 }

@@ -66,7 +66,7 @@ __device__ __forceinline__ int list_share(int64_t tot, int g, int c, int64_t* fi
 // [nI, n) list D from global unit d0.  A run is the CTA's consecutive units of
 // one pair in one list; the divisions happen once per run.
 struct RunCursor {
-  int64_t i0, d0;
+  int64_t i0, d0, pD0;
   int nI, n, mI, mD;
   int run_start, next_start, ordinal;
   int64_t pair;
@@ -80,13 +80,15 @@ struct RunCursor {
       next_start = static_cast<int>(e < nI ? e : nI);
     } else {
       in_d = true;
-      pair = (d0 + (i - nI)) / mD;
-      next_start = nI + static_cast<int>((pair + 1) * mD - d0);
+      const int64_t pd = (d0 + (i - nI)) / mD;         // pair index within list D
+      pair = pD0 + pd;
+      next_start = nI + static_cast<int>((pd + 1) * mD - d0);
     }
   }
   __device__ void init(const TcOrder& o, int64_t i0_, int nI_, int64_t d0_, int n_) {
     i0 = i0_;
     d0 = d0_;
+    pD0 = o.pD0;
     nI = nI_;
     n = n_;
     mI = o.mI;
@@ -117,7 +119,8 @@ __device__ __forceinline__ void unit_tile(const DecodeAttnArgs& a, const RunCurs
   const TcOrder& o = a.ord;
   const int64_t u = c.in_d ? c.d0 + (i - c.nI) : c.i0 + i;
   const int M = c.in_d ? o.mD : o.mI, nt = c.in_d ? o.ntD : o.ntI;
-  const int t = 2 * static_cast<int>(u - c.pair * M) + e;
+  const int64_t lp = c.in_d ? c.pair - o.pD0 : c.pair;   // pair index within the list
+  const int t = 2 * static_cast<int>(u - lp * M) + e;
   if (t >= nt) {
     *ks = 0;
     *nk = 0;
@@ -132,13 +135,14 @@ __device__ __forceinline__ void unit_tile(const DecodeAttnArgs& a, const RunCurs
 __device__ __forceinline__ void pair_slots(const TcOrder& o, int64_t pair, bool in_d, int* n, int* mine) {
   int nI = 0, nD = 0;
   int64_t fI = 0, fD = 0;
-  if (o.mI > 0) {
+  if (o.mI > 0 && pair < o.pI) {
     fI = list_owner(pair * o.mI, o.totI, o.gI);
     nI = static_cast<int>(list_owner(pair * o.mI + o.mI - 1, o.totI, o.gI) - fI) + 1;
   }
-  if (o.mD > 0) {
-    fD = list_owner(pair * o.mD, o.totD, o.gD);
-    nD = static_cast<int>(list_owner(pair * o.mD + o.mD - 1, o.totD, o.gD) - fD) + 1;
+  if (o.mD > 0 && pair >= o.pD0) {
+    const int64_t pd = pair - o.pD0;
+    fD = list_owner(pd * o.mD, o.totD, o.gD);
+    nD = static_cast<int>(list_owner(pd * o.mD + o.mD - 1, o.totD, o.gD) - fD) + 1;
   }
   *n = nI + nD;
   *mine = in_d ? nI + static_cast<int>(blockIdx.x - fD) : static_cast<int>(blockIdx.x - fI);

@@ -71,18 +71,23 @@ cudaError_t launch_score_topk_query0(const ScoreArgs& a, bool bf16, cudaStream_t
 // (two tiles each), each split evenly over its first g CTAs (CTA c takes
 // units [c*tot/g, (c+1)*tot/g)) and run list I first.  With `split`, list I
 // holds the tiles that need no index table (sink, window and new keys) and
-// list D the selected-block tiles, so a CTA can attend while the tables are
-// still being selected; without it list I is empty and list D is the whole
-// per-pair tile list.  Tile t of a list is tile t + off of the per-pair
-// order sink | selected | window (I: off = dI for t >= n_sink_tiles, else 0;
-// D: off = dD).  A pair's partial results take slots [0, nI) for its list-I
-// CTAs and [nI, nI + nD) for its list-D CTAs.
+// list D the selected-block tiles of every pair, so a CTA can attend while
+// the tables are still being selected.  Without it both lists hold whole
+// per-pair tile lists: list I the first floor(pairs / SMs) * SMs pairs, so
+// that every CTA attends the same number of pairs alone and writes their
+// outputs directly, list D the remaining pairs, split evenly over the CTAs.
+// List I covers pairs [0, pI), list D pairs [pD0, pD0 + totD / mD).  Tile t
+// of a list is tile t + off of the per-pair order sink | selected | window
+// (I: off = dI for t >= n_sink_tiles, else 0; D: off = dD).  A pair's
+// partial results take slots [0, nI) for its list-I CTAs and [nI, nI + nD)
+// for its list-D CTAs.
 struct TcOrder {
   int mI, mD;             // units per pair
   int ntI, ntD;           // tiles per pair
   int dI, dD;             // tile offsets into the per-pair order
   int gI, gD;             // CTAs sharing each list
   int64_t totI, totD;     // units over all pairs
+  int64_t pI, pD0;        // pairs [0, pI) are in list I; list D starts at pair pD0
   int grid;               // max(gI, gD)
   int slots;              // partial slots a pair may need
 };
