@@ -140,6 +140,31 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const float (&v)[4]) {
                : "memory");
 }
 // The first NR columns of this warp's 32 TMEM lanes.
+// Reduction of each of NR rows over the 32 lanes of a warp (max or sum) by a
+// reduce-scatter: at each level a lane keeps half of the rows it still holds
+// and trades the other half with the lane that differs in that bit, so NR
+// rows take NR shuffles in all (not 5 NR); lane l ends with row l % NR.
+template <int NR, bool MAX>
+__device__ __forceinline__ float rows_reduce(float (&v)[NR], int lane) {
+#pragma unroll
+  for (int h = NR / 2; h >= 1; h >>= 1) {
+    const bool up = (lane & h) != 0;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float keep = up ? v[i + h] : v[i];
+      const float other = __shfl_xor_sync(0xffffffffu, up ? v[i] : v[i + h], h);
+      v[i] = MAX ? fmaxf(keep, other) : keep + other;
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (int o = NR; o < 32; o <<= 1) {
+    const float other = __shfl_xor_sync(0xffffffffu, r, o);
+    r = MAX ? fmaxf(r, other) : r + other;
+  }
+  return r;
+}
+
 template <int NR>
 __device__ __forceinline__ void tmem_ldn(uint32_t taddr, float (&v)[NR]) {
   if constexpr (NR == 4) tmem_ld4(taddr, v);
@@ -532,12 +557,19 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     auto epilogue = [&]() -> bool {
       // row sums over the unit's 128 key slots
       float mine = 0.f;
+      if constexpr (NR >= 8) {
+        float lt[NR];
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        float v = l_t[r];
+        for (int r = 0; r < NR; ++r) lt[r] = l_t[r];
+        mine = rows_reduce<NR, false>(lt, lane);
+      } else {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        mine = (lane == r) ? v : mine;
+        for (int r = 0; r < NR; ++r) {
+          float v = l_t[r];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          mine = (lane == r) ? v : mine;
+        }
       }
       if (lane < NR) lsum[lane * 4 + qq] = mine;
       const int pkk = pc.ordinal, ob = pkk & 1;
@@ -799,24 +831,57 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       // unit max of every row: warp reduction, then the four warps through
       // shared memory (row r of this warp stored by lane r)
       float* wm = wmax + sb * (kN * 4);
-      uint32_t mk = 0u;
+      if constexpr (NR >= 8) {
+        float xm[NR];
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        const uint32_t k = __reduce_max_sync(0xffffffffu, float_key(x[r]));
-        mk = (lane == r) ? k : mk;
+        for (int r = 0; r < NR; ++r) xm[r] = x[r];
+        const float mx = rows_reduce<NR, true>(xm, lane);
+        if (lane < NR) wm[lane * 4 + qq] = mx;
+      } else {
+        uint32_t mk = 0u;
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          const uint32_t k = __reduce_max_sync(0xffffffffu, float_key(x[r]));
+          mk = (lane == r) ? k : mk;
+        }
+        if (lane < NR) wm[lane * 4 + qq] = float_of_key(mk);
       }
-      if (lane < NR) wm[lane * 4 + qq] = float_of_key(mk);
       softmax_bar();
       float alpha[NR];
       bool grow_any = false;
-#pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        const float4 w4 = reinterpret_cast<const float4*>(wm)[r];
+      if constexpr (NR >= 8) {
+        // lane l combines row l % NR alone (the unit max over the four
+        // warps, the growth test, the factor); every lane then takes the
+        // rows from their lanes
+        const int rr = lane & (NR - 1);
+        const float4 w4 = reinterpret_cast<const float4*>(wm)[rr];
         const float M = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
-        const bool grow = M > m_run[r] + kLazy;
-        alpha[r] = grow ? ex2(m_run[r] - M) : 1.f;     // 0 for the first keys of a row
-        m_run[r] = grow ? M : m_run[r];
-        grow_any |= grow;
+        float mo = m_run[0];
+#pragma unroll
+        for (int r = 1; r < NR; ++r) mo = (rr == r) ? m_run[r] : mo;
+        const bool grow = M > mo + kLazy;
+        const float al = grow ? ex2(mo - M) : 1.f;     // 0 for the first keys of a row
+        const float mn = grow ? M : mo;
+        grow_any = __any_sync(0xffffffffu, grow);
+#pragma unroll
+        for (int r = 0; r < NR; ++r) m_run[r] = __shfl_sync(0xffffffffu, mn, r);
+        if (grow_any) {
+#pragma unroll
+          for (int r = 0; r < NR; ++r) alpha[r] = __shfl_sync(0xffffffffu, al, r);
+        } else {
+#pragma unroll
+          for (int r = 0; r < NR; ++r) alpha[r] = 1.f;
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          const float4 w4 = reinterpret_cast<const float4*>(wm)[r];
+          const float M = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
+          const bool grow = M > m_run[r] + kLazy;
+          alpha[r] = grow ? ex2(m_run[r] - M) : 1.f;     // 0 for the first keys of a row
+          m_run[r] = grow ? M : m_run[r];
+          grow_any |= grow;
+        }
       }
       if (grow_any) {
         if (!fi) {
