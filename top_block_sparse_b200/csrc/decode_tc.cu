@@ -1080,10 +1080,12 @@ cudaError_t launch_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf1
     else kern = out_bf16 ? decode_tc_kernel<true, 16, false, true> : decode_tc_kernel<false, 16, false, true>;
   } else if (a.R <= 4) {
     kern = out_bf16 ? decode_tc_kernel<true, 4, FUSED, false> : decode_tc_kernel<false, 4, FUSED, false>;
+  } else if constexpr (FUSED) {
+    return cudaErrorInvalidValue;      // the fused step is built for at most 4 rows (decode_fused_supported)
   } else if (a.R <= 8) {
-    kern = out_bf16 ? decode_tc_kernel<true, 8, FUSED, false> : decode_tc_kernel<false, 8, FUSED, false>;
+    kern = out_bf16 ? decode_tc_kernel<true, 8, false, false> : decode_tc_kernel<false, 8, false, false>;
   } else {
-    kern = out_bf16 ? decode_tc_kernel<true, 16, FUSED, false> : decode_tc_kernel<false, 16, FUSED, false>;
+    kern = out_bf16 ? decode_tc_kernel<true, 16, false, false> : decode_tc_kernel<false, 16, false, false>;
   }
   const size_t smem = FUSED ? kSmemFused : kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
