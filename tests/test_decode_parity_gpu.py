@@ -246,6 +246,24 @@ def test_decode_edge_cases(over):
     check_decode(w, seed=61)
 
 
+@pytest.mark.parametrize("batch,n_q", [
+    (74, 3),      # 148 pairs, 6 rows: one whole pair per CTA on a 148-SM B200, nothing split
+    (74, 6),      # the same with 12 rows per KV head (draft chunk)
+    (149, 1),     # 298 pairs, 2 rows: two whole pairs per CTA, two split over every CTA
+    (150, 6),     # 300 pairs: two whole pairs per CTA, four split
+])
+def test_attention_whole_pairs_then_split(batch, n_q):
+    """The attention kernel gives each CTA floor(pairs / SMs) whole pairs and
+    splits the rest evenly; at these pair counts (all above what the fused
+    launch takes, so scoring and attention run as two kernels) every output
+    row is checked (2 KV heads, a 2085-key context)."""
+    assert sa.decode_launches(sa.params_for(WORKLOADS["decode_32k"].scaled(batch=batch, num_q_heads=4,
+                                                                           num_kv_heads=2, n_q=n_q))) == 2
+    w = WORKLOADS["decode_32k"].scaled(batch=batch, num_q_heads=4, num_kv_heads=2, ctx_len=2048 + 37,
+                                       n_q=n_q, top_k=5, n_needles=0)
+    check_decode(w, seed=67, out_dtype=torch.bfloat16)
+
+
 def test_decode_fp32_dense_equivalence_torch():
     """k covering every candidate: the GPU result equals dense attention
     computed by torch in float64 (a library routine, independent of both)."""
