@@ -76,6 +76,28 @@ design notes of the repository):
       compressed key c is the mean of the l keys starting at c*s (complete
       windows only), and the score of selectable block j is the MAX of the
       scores of the compressed keys whose windows share a key with block j.
+* R19 LSA flat bucket retrieval (LSA review §2.2-2.3).  Pool keys as in R7
+      (each raw key L2-normalised, ``pool_stride`` = 4 consecutive unit keys
+      summed).  A cluster block is ``block_size`` = 512 RAW keys (128 pool
+      keys): the page's 512-key window is "exactly one cluster block", and 64
+      buckets of 8 keys on average fill 512 raw keys.  Inside a complete
+      cluster block every pool key starts as its own bucket; each round
+      every bucket finds its cheapest partner by Ward's criterion (the rise
+      of the within-bucket sum of squares, n_a n_b / (n_a + n_b) |mean_a -
+      mean_b|^2 over the member pool keys) among the buckets it may join
+      without passing 16 raw keys (lower bucket index first on equal cost),
+      and all pairs that are each other's cheapest partner merge at once; if
+      that would leave fewer than block_size / 8 buckets, only the cheapest
+      such pairs merge (cost, then lower indices).  Buckets are indexed by
+      their lowest member within the block, and globally block by block.
+      Centroid = the normalised sum of the members' pool keys.  The index
+      query (R1) is normalised and scores every centroid (cosine); the
+      candidates are the buckets with a key outside sink and window (R4);
+      the top ``top_k`` buckets (R6 ties) are expanded to their raw keys.
+      With ``bucket_keys`` = N > 0 only the N / pool_stride best member pool
+      keys by their own cosine with the query (lower position first on
+      ties) are kept ("expanded by within-bucket merit to N long-range
+      keys"); with 0 every member key is kept.
 """
 from __future__ import annotations
 
@@ -101,6 +123,7 @@ class OracleParams:
     pool_stride: int = 4       # LSA: raw keys summed into one pool key;
                                # overlap: keys between window starts (s)
     pool_kernel: int = 0       # overlap: keys per compressed key (l)
+    bucket_keys: int = 0       # LSA buckets: long-range key budget N (0 = all)
     scale: Optional[float] = None   # softmax scale; None -> 1/sqrt(d)
 
 
@@ -493,3 +516,123 @@ def prefill_head_selection(q_head_rows: np.ndarray, Kc_all: np.ndarray,
         s = prefill_tile_scores(q_tile, Kc, p) if C // b > 0 else np.zeros(0)
         out[i] = select_topk(s, candidate_blocks(C, p), p.top_k)
     return out
+
+
+# --------------------------------------------------------------------------
+# 7. LSA flat bucket retrieval (reading R19)
+# --------------------------------------------------------------------------
+
+def lsa_pool_keys(K: np.ndarray, stride: int = 4) -> np.ndarray:
+    """Pool keys [LSA review §2.2]: each raw key L2-normalised, then every
+    ``stride`` consecutive unit keys summed.  Returns [len(K) // stride, d]."""
+    K = np.asarray(K, dtype=np.float64)
+    m = K.shape[0] // stride
+    return _normalise(K[:m * stride]).reshape(m, stride, -1).sum(axis=1)
+
+
+def ward_cost(sum_a: np.ndarray, n_a: int, sum_b: np.ndarray, n_b: int) -> float:
+    """Ward's merge cost of two buckets given their member sums and sizes:
+    the rise of the within-bucket sum of squares, n_a n_b / (n_a + n_b) *
+    |mean_a - mean_b|^2."""
+    diff = sum_a / n_a - sum_b / n_b
+    return n_a * n_b / (n_a + n_b) * float(diff @ diff)
+
+
+def ward_buckets(P: np.ndarray, n_buckets: int, cap: int, history: Optional[list] = None) -> List[List[int]]:
+    """Bottom-up Ward clustering of one cluster block's pool keys P [m, d]
+    into n_buckets buckets of at most ``cap`` pool keys  [LSA review §2.2:
+    every pool key its own bucket; each round, buckets that are each other's
+    cheapest merge merge in parallel; 64 buckets per block, at most 16 keys
+    each] (reading R19 for ties and the last round).  Returns the buckets
+    as ascending member lists, ordered by their lowest member.  ``history``
+    (optional) receives, per round, (bucket list, merged index pairs)."""
+    P = np.asarray(P, dtype=np.float64)
+    buckets = [[i] for i in range(P.shape[0])]
+    while len(buckets) > n_buckets:
+        sums = [P[b].sum(axis=0) for b in buckets]
+        nb = len(buckets)
+        best = []
+        for a in range(nb):
+            cost_a, part_a = math.inf, -1
+            for b in range(nb):
+                if b == a or len(buckets[a]) + len(buckets[b]) > cap:
+                    continue
+                c = ward_cost(sums[a], len(buckets[a]), sums[b], len(buckets[b]))
+                if c < cost_a:                  # ascending b: ties keep the lower index
+                    cost_a, part_a = c, b
+            best.append((part_a, cost_a))
+        pairs = [(best[a][1], a, best[a][0]) for a in range(nb)
+                 if best[a][0] > a and best[best[a][0]][0] == a]
+        if not pairs:
+            raise RuntimeError("no pair of buckets may merge under the size cap")
+        pairs.sort()
+        pairs = pairs[:nb - n_buckets]
+        if history is not None:
+            history.append(([list(b) for b in buckets], [(a, b) for _, a, b in pairs]))
+        gone = set()
+        merged = []
+        for _, a, b in pairs:
+            merged.append(sorted(buckets[a] + buckets[b]))
+            gone.update((a, b))
+        buckets = sorted([bk for i, bk in enumerate(buckets) if i not in gone] + merged, key=lambda x: x[0])
+    return buckets
+
+
+def lsa_bucket_index(K: np.ndarray, C: int, p: OracleParams):
+    """The bucket cache of a context of C keys (reading R19): for every
+    complete cluster block of ``block_size`` raw keys, its block_size / 8
+    buckets.  Returns (members, centroids): members[g] = ascending global
+    pool-key ids of bucket g, centroids [n, d] unit vectors."""
+    b, stride = p.block_size, p.pool_stride
+    per = b // stride
+    P = lsa_pool_keys(K[:(C // b) * b], stride)
+    members, cents = [], []
+    for j in range(C // b):
+        for bk in ward_buckets(P[j * per:(j + 1) * per], b // 8, 16 // stride):
+            ids = [j * per + i for i in bk]
+            members.append(ids)
+            cents.append(P[ids].sum(axis=0))
+    d = K.shape[1]
+    cents = _normalise(np.array(cents)) if cents else np.zeros((0, d))
+    return members, cents
+
+
+def bucket_decode_pair(q_tokens: np.ndarray, K: np.ndarray, V: np.ndarray, C: int,
+                       p: OracleParams) -> Dict:
+    """Decode / draft chunk for one (sequence, KV head) with LSA's flat bucket
+    retrieval [LSA review §2.2-2.3] (reading R19): normalised index query of
+    the first new token scores every bucket centroid; the top-k candidate
+    buckets are expanded to raw keys and joined with sink, window and the
+    chunk (R3, R9); masked softmax attention as in decode_pair."""
+    n_q, G, d = q_tokens.shape
+    stride = p.pool_stride
+    members, cents = lsa_bucket_index(K, C, p)
+    qhat = _normalise(index_query(q_tokens[0]))
+    scores = cents @ qhat if len(members) else np.zeros(0)
+    s_end, w_begin = sink_window(C, p)
+    cand = [g for g, ids in enumerate(members)
+            if any(s_end <= 4 * m + r < w_begin for m in ids for r in range(stride))]
+    sel = select_topk(scores, cand, p.top_k)
+    kept = sorted(m for g in sel.selected for m in members[g])
+    if p.bucket_keys > 0:
+        P = lsa_pool_keys(K[:(C // p.block_size) * p.block_size], stride)
+        own = {m: float(_normalise(P[m]) @ qhat) for m in kept}
+        kept = sorted(sorted(kept, key=lambda m: (-own[m], m))[:p.bucket_keys // stride])
+    scale = softmax_scale(d, p)
+    O = np.zeros((n_q, G, d))
+    lse = np.zeros((n_q, G))
+    pos_list = []
+    for j in range(n_q):
+        mask = np.zeros(C + j + 1, dtype=bool)
+        mask[0:s_end] = True
+        mask[w_begin:C] = True
+        for m in kept:
+            mask[m * stride:(m + 1) * stride] = True
+        mask[C:C + j + 1] = True
+        pos = np.flatnonzero(mask)
+        pos_list.append(pos)
+        for g in range(G):
+            O[j, g], lse[j, g], _ = masked_softmax_attention(q_tokens[j, g], K, V, pos, scale)
+    return dict(members=members, centroids=cents, scores=scores, candidates=cand, sel=sel,
+                kept=kept, O=O, lse=lse, positions=pos_list)
+

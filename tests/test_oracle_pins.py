@@ -460,6 +460,145 @@ def test_overlap_needles_selected():
     assert set(inp["needles"][0, 0].tolist()) <= set(r["sel"].selected)
 
 
+# ------------------------------------------- LSA flat bucket retrieval ---
+
+def _sse(X):
+    X = np.asarray(X, float)
+    return float(((X - X.mean(axis=0)) ** 2).sum())
+
+
+def test_ward_cost_is_the_rise_in_sum_of_squares():
+    """Ward's criterion: merging A and B raises the within-bucket sum of
+    squared distances to the mean by exactly the cost (brute force)."""
+    r = rng(21)
+    for na, nb in [(1, 1), (1, 3), (2, 2), (3, 4), (5, 1)]:
+        A, B = r.standard_normal((na, 16)), r.standard_normal((nb, 16)) + 0.3
+        rise = _sse(np.vstack([A, B])) - _sse(A) - _sse(B)
+        assert orc.ward_cost(A.sum(0), na, B.sum(0), nb) == pytest.approx(rise, rel=1e-10)
+
+
+def _bases(n, d, seed):
+    return 10.0 * orc._normalise(rng(seed).standard_normal((n, d)))
+
+
+def test_ward_recovers_planted_pairs_and_quartets():
+    """Tight pairs far apart are exactly the 64 buckets; tight groups of four
+    (the cap) end as two buckets each, none mixing groups."""
+    r = rng(22)
+    perm = r.permutation(128)
+    pts = np.repeat(_bases(64, 32, 23), 2, axis=0) + 1e-3 * r.standard_normal((128, 32))
+    P = np.empty_like(pts)
+    P[perm] = pts                                  # point i of pair i // 2 sits at perm[i]
+    got = {frozenset(b) for b in orc.ward_buckets(P, 64, 4)}
+    want = {frozenset((int(perm[2 * k]), int(perm[2 * k + 1]))) for k in range(64)}
+    assert got == want
+    pts = np.repeat(_bases(32, 32, 24), 4, axis=0) + 1e-3 * r.standard_normal((128, 32))
+    P = np.empty_like(pts)
+    P[perm] = pts
+    group = {int(perm[i]): i // 4 for i in range(128)}
+    out = orc.ward_buckets(P, 64, 4)
+    assert len(out) == 64
+    per_group = {}
+    for b in out:
+        assert len({group[m] for m in b}) == 1
+        per_group[group[b[0]]] = per_group.get(group[b[0]], 0) + 1
+    assert all(v == 2 for v in per_group.values()) and len(per_group) == 32
+
+
+@pytest.mark.parametrize("seed,n,target,cap", [(25, 128, 64, 4), (26, 128, 64, 4), (27, 40, 20, 8), (28, 33, 17, 2)])
+def test_ward_rounds_merge_mutual_cheapest_pairs(seed, n, target, cap):
+    """Every round merges only pairs of buckets that are each other's
+    cheapest partner within the cap (costs by brute force on the members),
+    all such pairs unless that would pass the bucket target (then the
+    cheapest); the result partitions the keys into `target` buckets of at
+    most `cap`, ordered by their lowest member."""
+    P = rng(seed).standard_normal((n, 24))
+    hist = []
+    out = orc.ward_buckets(P, target, cap, hist)
+    for buckets, merged in hist:
+        nb = len(buckets)
+        cost = np.full((nb, nb), np.inf)
+        for a in range(nb):
+            for b in range(nb):
+                if a != b and len(buckets[a]) + len(buckets[b]) <= cap:
+                    cost[a, b] = _sse(P[buckets[a] + buckets[b]]) - _sse(P[buckets[a]]) - _sse(P[buckets[b]])
+        best = [int(np.argmin(cost[a])) if np.isfinite(cost[a]).any() else -1 for a in range(nb)]
+        mutual = {(a, best[a]) for a in range(nb) if best[a] > a and best[best[a]] == a}
+        assert set(merged) <= mutual
+        if len(merged) < len(mutual):
+            assert nb - len(merged) == target
+            worst = max(cost[a, b] for a, b in merged)
+            assert all(cost[a, b] >= worst - 1e-12 for a, b in mutual - set(merged))
+    flat = sorted(m for b in out for m in b)
+    assert flat == list(range(n)) and len(out) == target
+    assert all(len(b) <= cap and b == sorted(b) for b in out)
+    assert [b[0] for b in out] == sorted(b[0] for b in out)
+
+
+def _lsa_params(**kw):
+    base = dict(block_size=512, top_k=4, sink_keys=4, window_keys=512, pool="lsa", pool_stride=4)
+    base.update(kw)
+    return orc.OracleParams(**base)
+
+
+def test_bucket_index_covers_blocks_and_ignores_key_scale():
+    """The bucket cache of the complete cluster blocks: every pool key of
+    them in exactly one bucket, 64 per block, unit centroids; scaling raw
+    keys by positive factors (which the L2 normalisation removes) changes
+    nothing."""
+    r = rng(29)
+    C = 512 * 3 + 100
+    K = r.standard_normal((C, 32))
+    p = _lsa_params()
+    members, cents = orc.lsa_bucket_index(K, C, p)
+    assert len(members) == 3 * 64
+    assert sorted(m for b in members for m in b) == list(range(3 * 128))
+    assert all(len(b) <= 4 for b in members)
+    assert np.allclose(np.linalg.norm(cents, axis=1), 1.0)
+    members2, cents2 = orc.lsa_bucket_index(K * r.uniform(0.1, 10.0, (C, 1)), C, p)
+    assert members2 == members
+    np.testing.assert_allclose(cents2, cents, atol=1e-12)
+
+
+def test_bucket_decode_with_every_bucket_is_dense_attention():
+    """With k above the number of candidate buckets and a context of whole
+    cluster blocks, the attended set is every key: library dense attention
+    (torch SDPA in float64); also for a 3-token chunk."""
+    r = rng(30)
+    C, d = 512 * 3, 32
+    K, V = r.standard_normal((C + 3, d)), r.standard_normal((C + 3, d))
+    q = r.standard_normal((3, 2, d))
+    res = orc.bucket_decode_pair(q, K, V, C, _lsa_params(top_k=10_000))
+    assert len(res["sel"].selected) == len(res["candidates"]) == 2 * 64     # the last block is the window
+    for j in range(3):
+        for g in range(2):
+            np.testing.assert_allclose(res["O"][j, g], _sdpa(q[j, g], K, V, C + j + 1), atol=1e-12)
+
+
+def test_bucket_decode_selects_a_planted_needle_and_keeps_the_budget():
+    """Eight raw keys (two pool keys) pulled towards the query in an early
+    cluster block land in the selected buckets; with a budget of N keys only
+    the N / 4 member pool keys of best own cosine stay, every kept one at
+    least as good as every dropped one."""
+    r = rng(31)
+    C, d = 512 * 6, 64
+    K, V = r.standard_normal((C + 1, d)), r.standard_normal((C + 1, d))
+    q = r.standard_normal((1, 4, d))
+    u = q[0].mean(axis=0)
+    needle = list(range(512 + 100, 512 + 108))
+    K[needle] = 0.5 * u * 4 + 0.3 * r.standard_normal((8, d))
+    res = orc.bucket_decode_pair(q, K, V, C, _lsa_params(top_k=6))
+    assert set(needle) <= set(res["positions"][0].tolist())
+    full = res["kept"]
+    res2 = orc.bucket_decode_pair(q, K, V, C, _lsa_params(top_k=6, bucket_keys=16))
+    kept = res2["kept"]
+    assert len(kept) == min(4, len(full)) and set(kept) <= set(full)
+    P = orc.lsa_pool_keys(K[:C])
+    qhat = orc._normalise(q[0].sum(axis=0))
+    own = {m: float(orc._normalise(P[m]) @ qhat) for m in full}
+    assert min(own[m] for m in kept) >= max([own[m] for m in set(full) - set(kept)] + [-2.0])
+
+
 # ---------------------------------------------- planted-mistake checks ---
 
 # ------------------------------------------------------------ dense verify ---
@@ -637,6 +776,38 @@ def test_planted_mistakes_are_caught(monkeypatch):
             m.setattr(orc, name, bad)
             assert _fails(ovl), name
     assert orig_b2c is orc.blocks_from_compressed
+    # Ward clustering: centroid distance without the size weights; every
+    # bucket merging with its cheapest partner whether or not that is mutual;
+    # the size cap ignored
+    with monkeypatch.context() as m:
+        m.setattr(orc, "ward_cost", lambda sa, na, sb, nb: float(((sa / na - sb / nb) ** 2).sum()))
+        assert _fails(test_ward_cost_is_the_rise_in_sum_of_squares)
+    orig_wb = orc.ward_buckets
+
+    def greedy(P, n_buckets, cap, history=None):
+        P = np.asarray(P, float)
+        buckets = [[i] for i in range(len(P))]
+        while len(buckets) > n_buckets:
+            nb = len(buckets)
+            used, merged = set(), []
+            for a in range(nb):
+                if a in used:
+                    continue
+                cands = [b for b in range(nb) if b != a and b not in used and len(buckets[a]) + len(buckets[b]) <= cap]
+                if not cands or nb - len(merged) <= n_buckets:
+                    continue
+                b = min(cands, key=lambda b: (orc.ward_cost(P[buckets[a]].sum(0), len(buckets[a]), P[buckets[b]].sum(0), len(buckets[b])), b))
+                used.update((a, b))
+                merged.append((a, b))
+            if history is not None:
+                history.append(([list(x) for x in buckets], merged))
+            buckets = sorted([bk for i, bk in enumerate(buckets) if i not in used]
+                             + [sorted(buckets[a] + buckets[b]) for a, b in merged], key=lambda x: x[0])
+        return buckets
+    for bad in (greedy, lambda P, n, cap, history=None: orig_wb(P, n, 10 ** 6, history)):
+        with monkeypatch.context() as m:
+            m.setattr(orc, "ward_buckets", bad)
+            assert _fails(lambda: test_ward_rounds_merge_mutual_cheapest_pairs(25, 128, 64, 4))
     # summed chunk queries instead of the chunk's first query for selection
     with monkeypatch.context() as m:
         m.setattr(orc, "index_query", lambda qg: np.asarray(qg, float).sum(axis=0) * 0.0)
