@@ -184,7 +184,9 @@ sa_status sa_sparse_attn_given_idx(const sa_params* p, const void* Q,
 
 /* Steps 2-4 for decode and draft chunks (select == SA_SEL_QUERY0) with the
  * compressed keys Kc kept up to date by the caller (sa_pool_keys).  Writes
- * O, lse (optional) and the index table (optional idx_out, [B, Hkv, top_k]). */
+ * O, lse (optional) and the index table (optional idx_out, [B, Hkv, top_k]).
+ * Runs as one cooperative launch where sa_decode_launches(p) == 1, else as
+ * the scoring + top-k kernel followed by the attention kernel. */
 sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q,
                                 const void* K, const void* V, const float* Kc,
                                 void* O, float* lse, int32_t* idx_out,
