@@ -425,9 +425,9 @@ def run_ours(args, w, rank, world, local_rank):
                  "note": "compression runs once after prefill / when a block fills; not part of a decode step"},
         "e2e": {"value": world * w.batch * w.n_q / (e2e["ms"] * 1e-3), "unit": "queries/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                "note": "per step: pinned host -> device copy of the new tokens' Q, K, V rows, the decode "
-                        "call through the C ABI, device -> pinned host copy of O; the KV cache and the "
-                        "compressed keys stay resident in HBM"},
+                "note": "per step: one pinned host -> device copy of the new tokens' Q, K, V rows (packed), "
+                        "sa_append_kv into the cache and the decode call through the C ABI, device -> pinned "
+                        "host copy of O; the KV cache and the compressed keys stay resident in HBM"},
         "prefill": prefill,
         "verify": verify,
         "column": column,
@@ -757,31 +757,34 @@ def run_overlap_bench(args, dev, stream, flush):
 
 
 def e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush):
+    """One decode step as a serving loop runs it: the new tokens' Q, K and V
+    arrive packed in one pinned host buffer, one copy takes them to the
+    device, sa_append_kv writes the K and V rows into the cache, the decode
+    runs on the staged Q, and O is copied back to pinned host memory."""
     from top_block_sparse_b200 import sa
     C = w.ctx_len
-    hQ = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
-    hK = torch.empty((w.batch, w.num_kv_heads, w.n_q, w.head_dim), dtype=K.dtype, pin_memory=True)
-    hV = torch.empty_like(hK, pin_memory=True)
+    shape_new = (w.batch, w.num_kv_heads, w.n_q, w.head_dim)
+    nq, nk = Q.numel(), w.batch * w.num_kv_heads * w.n_q * w.head_dim
+    h_stage = torch.empty(nq + 2 * nk, dtype=Q.dtype, pin_memory=True)
+    d_stage = torch.empty(nq + 2 * nk, dtype=Q.dtype, device=Q.device)
+    h_stage[:nq].copy_(Q.flatten().cpu())
+    h_stage[nq:nq + nk].copy_(K[:, :, C:C + w.n_q].flatten().cpu())
+    h_stage[nq + nk:].copy_(V[:, :, C:C + w.n_q].flatten().cpu())
+    Qs = d_stage[:nq].view(Q.shape)
+    Kn = d_stage[nq:nq + nk].view(shape_new)
+    Vn = d_stage[nq + nk:].view(shape_new)
     hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
-    hQ.copy_(Q.cpu())
-    hK.copy_(K[:, :, C:C + w.n_q].cpu())
-    hV.copy_(V[:, :, C:C + w.n_q].cpu())
-    Kn = K[:, :, C:C + w.n_q]
-    Vn = V[:, :, C:C + w.n_q]
 
     def one():
-        Q.copy_(hQ, non_blocking=True)
-        Kn.copy_(hK, non_blocking=True)
-        Vn.copy_(hV, non_blocking=True)
-        sa.sparse_attn_decode(p, Q, K, V, Kc, O, lse, idx, ws, stream=stream)
+        d_stage.copy_(h_stage, non_blocking=True)
+        sa.append_kv(p, Kn, Vn, K, V, stream=stream)
+        sa.sparse_attn_decode(p, Qs, K, V, Kc, O, lse, idx, ws, stream=stream)
         hO.copy_(O, non_blocking=True)
 
     n = max(50, args.steps // 4)
     with torch.cuda.stream(stream):
         ms = statistics.mean(timed_steps(one, n, args.warmup, stream, flush))
-    el = Q.element_size()
-    h2d = hQ.numel() * el + 2 * hK.numel() * el
-    return {"ms": ms, "h2d": h2d, "d2h": hO.numel() * O.element_size()}
+    return {"ms": ms, "h2d": h_stage.numel() * h_stage.element_size(), "d2h": hO.numel() * O.element_size()}
 
 
 def main():

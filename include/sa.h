@@ -149,6 +149,16 @@ sa_status sa_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * writes Kc (fp32, see layouts).  No workspace. */
 sa_status sa_pool_keys(const sa_params* p, const void* K, float* Kc, void* stream);
 
+/* Cache append for decode / draft chunks (select == SA_SEL_QUERY0): the n_q
+ * new tokens' keys and values go to rows ctx_len .. ctx_len + n_q - 1 of the
+ * cache, K[b, h, ctx_len + t, :] = K_new[b, h, t, :] and the same for V.
+ * K_new, V_new: [B, Hkv, n_q, d] in dtype, contiguous, 16-byte aligned; K, V
+ * as in the layouts (ctx_len + n_q <= kv_capacity is checked).  Compressed
+ * keys are not touched: call sa_pool_keys when a block fills.  Asynchronous
+ * on `stream`; one kernel, no workspace. */
+sa_status sa_append_kv(const sa_params* p, const void* K_new, const void* V_new,
+                       void* K, void* V, void* stream);
+
 /* Steps 2-3 (scoring and selection).  SA_SEL_QUERY0: one table row per
  * (sequence, KV head) from the first new token's GQA-summed query.
  * SA_SEL_TILE_MAX: one row per (sequence, KV head, query tile of b rows),

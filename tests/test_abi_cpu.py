@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
     for name in declared_functions():
         assert hasattr(lib, name), name
     assert set(declared_functions()) <= set(sa.EXPORTED) | set(declared_functions())
-    assert sa.version() == 102
+    assert sa.version() == 103
 
 
 def test_params_struct_layout():

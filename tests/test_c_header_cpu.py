@@ -30,7 +30,7 @@ static sa_params decode_params(void) {
 int main(void) {
   sa_params p = decode_params();
   if (sizeof(sa_params) != 96) return 10;
-  if (sa_version() != 102) return 11;
+  if (sa_version() != 103) return 11;
   if (sa_workspace_size(&p, SA_OP_DECODE) == 0) return 12;
   if (sa_workspace_size(&p, SA_OP_SCORE_TOPK) == 0) return 13;
   p.head_dim = 64;                                   /* not built */
@@ -42,6 +42,7 @@ int main(void) {
   if (sa_pool_keys(&p, (const void*)0x10000, (float*)0x10000, NULL) != SA_ERR_INVALID) return 17;
   if (sa_pool_keys(NULL, NULL, NULL, NULL) != SA_ERR_INVALID) return 18;
   if (strcmp(sa_status_string(SA_OK), sa_status_string(SA_ERR_INDEX)) == 0) return 19;
+  if (sa_append_kv(&p, NULL, NULL, NULL, NULL, NULL) != SA_ERR_INVALID) return 20;
   printf("ok %d\n", sa_version());
   return 0;
 }
@@ -62,4 +63,4 @@ def test_c99_program_uses_the_header_and_library(tmp_path):
     assert build.returncode == 0, build.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
-    assert run.stdout.strip() == "ok 102"
+    assert run.stdout.strip() == "ok 103"

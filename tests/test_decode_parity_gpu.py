@@ -264,6 +264,29 @@ def test_attention_whole_pairs_then_split(batch, n_q):
     check_decode(w, seed=67, out_dtype=torch.bfloat16)
 
 
+@pytest.mark.parametrize("dtype,n_q", [("bf16", 1), ("bf16", 6), ("f32", 3)])
+def test_append_kv(dtype, n_q):
+    """sa_append_kv puts the new tokens' rows at rows ctx_len.. of every
+    pair, bit for bit, and leaves every other row of the cache as it was."""
+    w = WORKLOADS["decode_32k"].scaled(batch=3, num_q_heads=8, num_kv_heads=2, ctx_len=1000, n_q=n_q,
+                                       dtype=dtype, n_needles=0)
+    cap = w.kv_len + 37
+    inp = make_inputs(w, seed=69, device="cuda", kv_capacity=cap)
+    K, V = inp["K"], inp["V"]
+    K0, V0 = K.clone(), V.clone()
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    Kn = torch.randn((w.batch, w.num_kv_heads, n_q, 128), device="cuda", generator=g).to(K.dtype)
+    Vn = torch.randn((w.batch, w.num_kv_heads, n_q, 128), device="cuda", generator=g).to(K.dtype)
+    sa.append_kv(sa.params_for(w, kv_capacity=cap), Kn, Vn, K, V)
+    torch.cuda.synchronize()
+    C = w.ctx_len
+    assert torch.equal(K[:, :, C:C + n_q], Kn) and torch.equal(V[:, :, C:C + n_q], Vn)
+    keep = torch.ones(cap, dtype=torch.bool, device="cuda")
+    keep[C:C + n_q] = False
+    assert torch.equal(K[:, :, keep], K0[:, :, keep]) and torch.equal(V[:, :, keep], V0[:, :, keep])
+
+
 def test_decode_fp32_dense_equivalence_torch():
     """k covering every candidate: the GPU result equals dense attention
     computed by torch in float64 (a library routine, independent of both)."""

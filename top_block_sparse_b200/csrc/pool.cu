@@ -1,4 +1,5 @@
-// Compression of complete key blocks (step 1 of the method).
+// Cache maintenance: compression of complete key blocks (step 1 of the
+// method) and the append of new tokens' keys and values.
 //
 //   mean : Kc[j] = (1/b) * sum of the b keys of block j
 //          (SparDA summary, section "方法": keys average-pooled into
@@ -161,7 +162,37 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(PoolArgs a) {
   }
 }
 
+// Append of the new tokens' rows to the cache: row t of pair q in K_new goes
+// to row C + t of pair q in K (the same for V).  One thread per 16 bytes,
+// K's rows first, then V's.
+__global__ void __launch_bounds__(256) append_kv_kernel(const uint4* __restrict__ kn, const uint4* __restrict__ vn,
+                                                        uint4* __restrict__ K, uint4* __restrict__ V, int64_t rows,
+                                                        int n_q, int64_t cap, int64_t C, int chunks) {
+  const int64_t per = rows * chunks;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= 2 * per) return;
+  const bool is_v = i >= per;
+  const int64_t j = is_v ? i - per : i;
+  const int64_t row = j / chunks, c = j - row * chunks;
+  const int64_t pair = row / n_q, t = row - pair * n_q;
+  const uint4 v = is_v ? __ldg(vn + j) : __ldg(kn + j);
+  (is_v ? V : K)[(pair * cap + C + t) * chunks + c] = v;
+}
+
 }  // namespace
+
+cudaError_t launch_append_kv(const void* K_new, const void* V_new, void* K, void* V, int pairs, int n_q, int64_t cap,
+                             int64_t C, int row_bytes, cudaStream_t s) {
+  const int chunks = row_bytes / 16;
+  const int64_t total = 2 * static_cast<int64_t>(pairs) * n_q * chunks;
+  if (total == 0) return cudaSuccess;
+  const int64_t grid = (total + 255) / 256;
+  if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  append_kv_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(
+      static_cast<const uint4*>(K_new), static_cast<const uint4*>(V_new), static_cast<uint4*>(K),
+      static_cast<uint4*>(V), static_cast<int64_t>(pairs) * n_q, n_q, cap, C, chunks);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pool(const PoolArgs& a, bool bf16, cudaStream_t s) {
   const int64_t total = static_cast<int64_t>(a.pairs) * a.nb;

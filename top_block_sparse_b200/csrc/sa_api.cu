@@ -331,7 +331,7 @@ using namespace sa;
 
 extern "C" {
 
-int32_t sa_version(void) { return 102; }
+int32_t sa_version(void) { return 103; }
 
 const char* sa_last_error(void) { return g_err; }
 
@@ -439,6 +439,19 @@ sa_status sa_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (!ws) return fail(SA_ERR_INVALID, "workspace is NULL");
   cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  return SA_OK;
+}
+
+sa_status sa_append_kv(const sa_params* p, const void* K_new, const void* V_new, void* K, void* V, void* stream) {
+  sa_status st = check_params(p, false);
+  if (st != SA_OK) return st;
+  if (!K_new || !V_new || !K || !V) return fail(SA_ERR_INVALID, "K_new, V_new, K and V must be non-NULL");
+  if (!aligned16(K_new) || !aligned16(V_new) || !aligned16(K) || !aligned16(V))
+    return fail(SA_ERR_INVALID, "K_new, V_new, K and V must be 16-byte aligned");
+  const int row_bytes = p->head_dim * (p->dtype == SA_BF16 ? 2 : 4);
+  cudaError_t e = launch_append_kv(K_new, V_new, K, V, p->batch * p->num_kv_heads, p->n_q, p->kv_capacity,
+                                   p->ctx_len, row_bytes, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
   return SA_OK;
 }
 

@@ -31,7 +31,7 @@ SA_FLAG_TRUSTED_IDX = 1
 EXPORTED = ["sa_version", "sa_workspace_size", "sa_workspace_init", "sa_pool_keys", "sa_score_topk",
             "sa_sparse_attn_given_idx", "sa_sparse_attn_decode", "sa_sparse_attn_prefill",
             "sa_read_status", "sa_status_string", "sa_last_error", "sa_sparse_attn_given_idx_noalloc",
-            "sa_decode_launches", "sa_verify_refresh", "sa_column_attn"]
+            "sa_decode_launches", "sa_verify_refresh", "sa_column_attn", "sa_append_kv"]
 
 
 class SaParams(ctypes.Structure):
@@ -69,6 +69,7 @@ _sig = {
     "sa_decode_launches": (_i32, [_P]),
     "sa_verify_refresh": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "sa_column_attn": (_i32, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "sa_append_kv": (_i32, [_P, _vp, _vp, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -153,6 +154,11 @@ def workspace_init(ws: torch.Tensor, stream=None):
 
 def pool_keys(p: SaParams, K: torch.Tensor, Kc: torch.Tensor, stream=None):
     _check(_lib.sa_pool_keys(ctypes.byref(p), _ptr(K), _ptr(Kc), _stream(stream)))
+
+
+def append_kv(p: SaParams, K_new, V_new, K, V, stream=None):
+    """The new tokens' keys and values [B, Hkv, n_q, d] into cache rows ctx_len.."""
+    _check(_lib.sa_append_kv(ctypes.byref(p), _ptr(K_new), _ptr(V_new), _ptr(K), _ptr(V), _stream(stream)))
 
 
 def score_topk(p: SaParams, Q, Kc, idx, scores=None, ws=None, stream=None):
