@@ -36,10 +36,6 @@ struct PoolArgs {
   int lsa;          // 0 mean, 1 LSA centroid (len == stride)
 };
 cudaError_t launch_pool(const PoolArgs& a, bool bf16, cudaStream_t s);
-// rows [pairs * n_q] of row_bytes (a multiple of 16) from K_new / V_new to
-// rows C.. of each pair's cap rows in K / V
-cudaError_t launch_append_kv(const void* K_new, const void* V_new, void* K, void* V, int pairs, int n_q, int64_t cap,
-                             int64_t C, int row_bytes, cudaStream_t s);
 
 // ---- decode scoring + top-k --------------------------------------------------
 // SA_POOL_OVERLAP (ov_s > 0): the rows are windows of ov_l keys every ov_s

@@ -18,6 +18,7 @@
 // fp32 registers; the output is fp32 (set parity of the later top-k needs
 // compressed keys far more precise than bf16).
 #include "common.cuh"
+#include "cache_ops.h"
 #include "internal.h"
 
 namespace sa {

@@ -8,6 +8,7 @@
 #include <string.h>
 
 #include "common.cuh"
+#include "cache_ops.h"
 #include "internal.h"
 #include "sa.h"
 
