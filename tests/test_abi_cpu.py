@@ -64,10 +64,16 @@ def _decode(p, ws_bytes=1 << 30, q=FAKE, kc=FAKE):
     (dict(n_q=0), sa.SA_ERR_INVALID),
     (dict(n_q=5), sa.SA_ERR_UNSUPPORTED),       # 5 tokens x GQA 4 = 20 rows > 16
     (dict(prefill=True), sa.SA_ERR_INVALID),     # decode entry point with the prefill selector
+    (dict(batch=2 ** 31 - 1), sa.SA_ERR_UNSUPPORTED),            # pairs past 32-bit counts
+    (dict(ctx_len=2 ** 41), sa.SA_ERR_UNSUPPORTED),              # cache rows past 2^40
+    (dict(batch=2 ** 20, ctx_len=2 ** 30), sa.SA_ERR_UNSUPPORTED),   # pairs x rows past 2^48
 ])
 def test_validation_rejects(kw, status):
     assert _decode(_p(**kw)) == status
     assert sa.raw_call("sa_last_error").decode() != ""
+    # no workspace size for a problem the library refuses
+    for op in range(6):
+        assert sa.raw_call("sa_workspace_size", ctypes.byref(_p(**kw)), op) == 0
 
 
 @pytest.mark.parametrize("kw,status", [

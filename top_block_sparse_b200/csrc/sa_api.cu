@@ -59,6 +59,18 @@ sa_status check_params(const sa_params* p, bool prefill) {
   if (p->kv_capacity < p->ctx_len + p->n_q)
     return fail(SA_ERR_INVALID, "kv_capacity (%lld) < ctx_len + n_q (%lld)", (long long)p->kv_capacity,
                 (long long)(p->ctx_len + p->n_q));
+  // index arithmetic: (sequence, KV head) pairs and query rows are counted in
+  // 32-bit integers, cache rows in 64-bit ones
+  {
+    const int64_t pairs = static_cast<int64_t>(p->batch) * p->num_kv_heads;
+    const int64_t q_rows = static_cast<int64_t>(p->batch) * p->n_q * p->num_q_heads;
+    if (pairs > INT32_MAX || q_rows > INT32_MAX)
+      return fail(SA_ERR_UNSUPPORTED, "batch x heads x n_q too large (%lld query rows, %lld pairs)",
+                  (long long)q_rows, (long long)pairs);
+    if (p->kv_capacity > (int64_t(1) << 40) || pairs * p->kv_capacity > (int64_t(1) << 48))
+      return fail(SA_ERR_UNSUPPORTED, "cache of %lld pairs x %lld rows too large", (long long)pairs,
+                  (long long)p->kv_capacity);
+  }
   if (p->block_size < 16 || p->block_size % 16 != 0 || p->block_size > 65536)
     return fail(SA_ERR_INVALID, "block_size %d must be a multiple of 16 in [16, 65536]", p->block_size);
   if (p->pool != SA_POOL_MEAN && p->pool != SA_POOL_LSA && p->pool != SA_POOL_OVERLAP)
