@@ -53,7 +53,9 @@
  *
  * Errors: arguments are validated on the host before any launch
  * (SA_ERR_INVALID / SA_ERR_UNSUPPORTED / SA_ERR_WORKSPACE, with a message in
- * sa_last_error()); a failed launch returns SA_ERR_CUDA.  Conditions found on
+ * sa_last_error(); sizes are refused as SA_ERR_UNSUPPORTED when B x Hkv or
+ * B x n_q x Hq reaches 2^31, kv_capacity passes 2^40 or B x Hkv x
+ * kv_capacity passes 2^48); a failed launch returns SA_ERR_CUDA.  Conditions found on
  * the device (an out-of-range or repeated block id in a caller's index table,
  * a bounded wait that ran out) set bits of a status word kept in the
  * workspace; the affected block is skipped and sa_read_status() reports
@@ -127,7 +129,7 @@ typedef struct sa_params {
 /* Version of this ABI (major * 100 + minor). */
 int32_t sa_version(void);
 
-/* Bytes of workspace `op` needs for `p` (0 if p is invalid).  The workspace
+/* Bytes of workspace `op` needs for `p` (0 if p is invalid or refused).  The workspace
  * also carries the device status word and self-resetting counters, so it
  * must be zero-filled once before its first use (sa_workspace_init) and may
  * then be reused by later calls on the same stream.  Calls that share one
