@@ -530,12 +530,13 @@ def lsa_pool_keys(K: np.ndarray, stride: int = 4) -> np.ndarray:
     return _normalise(K[:m * stride]).reshape(m, stride, -1).sum(axis=1)
 
 
-def ward_cost(sum_a: np.ndarray, n_a: int, sum_b: np.ndarray, n_b: int) -> float:
-    """Ward's merge cost of two buckets given their member sums and sizes:
-    the rise of the within-bucket sum of squares, n_a n_b / (n_a + n_b) *
-    |mean_a - mean_b|^2."""
-    diff = sum_a / n_a - sum_b / n_b
-    return n_a * n_b / (n_a + n_b) * float(diff @ diff)
+def ward_cost(sum_a, n_a, sum_b, n_b):
+    """Ward's merge cost of two buckets given their member sums (last axis)
+    and sizes: the rise of the within-bucket sum of squares,
+    n_a n_b / (n_a + n_b) * |mean_a - mean_b|^2.  Broadcasts over leading
+    axes (all pairs of a round at once)."""
+    diff = np.asarray(sum_a) / np.asarray(n_a)[..., None] - np.asarray(sum_b) / np.asarray(n_b)[..., None]
+    return np.asarray(n_a) * n_b / (np.asarray(n_a) + n_b) * (diff * diff).sum(axis=-1)
 
 
 def ward_buckets(P: np.ndarray, n_buckets: int, cap: int, history: Optional[list] = None) -> List[List[int]]:
@@ -549,18 +550,16 @@ def ward_buckets(P: np.ndarray, n_buckets: int, cap: int, history: Optional[list
     P = np.asarray(P, dtype=np.float64)
     buckets = [[i] for i in range(P.shape[0])]
     while len(buckets) > n_buckets:
-        sums = [P[b].sum(axis=0) for b in buckets]
         nb = len(buckets)
+        sums = np.stack([P[b].sum(axis=0) for b in buckets])
+        size = np.array([len(b) for b in buckets], dtype=np.float64)
+        # cost[a, b] for every pair; a pair may merge if b != a and it fits the cap
+        cost = ward_cost(sums[:, None, :], size[:, None], sums[None, :, :], size[None, :])
+        cost = np.where((size[:, None] + size[None, :] <= cap) & ~np.eye(nb, dtype=bool), cost, math.inf)
         best = []
         for a in range(nb):
-            cost_a, part_a = math.inf, -1
-            for b in range(nb):
-                if b == a or len(buckets[a]) + len(buckets[b]) > cap:
-                    continue
-                c = ward_cost(sums[a], len(buckets[a]), sums[b], len(buckets[b]))
-                if c < cost_a:                  # ascending b: ties keep the lower index
-                    cost_a, part_a = c, b
-            best.append((part_a, cost_a))
+            part_a = int(np.argmin(cost[a]))            # the first of equal costs: the lower index
+            best.append((part_a, float(cost[a, part_a])) if math.isfinite(cost[a, part_a]) else (-1, math.inf))
         pairs = [(best[a][1], a, best[a][0]) for a in range(nb)
                  if best[a][0] > a and best[best[a][0]][0] == a]
         if not pairs:
