@@ -6,12 +6,6 @@
 
 namespace sa {
 
-__device__ __forceinline__ unsigned warp_sum(unsigned v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 __device__ __forceinline__ unsigned warp_exclusive_scan(unsigned v) {
   const int lane = threadIdx.x & 31;
   unsigned x = v;
@@ -166,23 +160,6 @@ __device__ inline void warp_topk(const uint32_t* keys, int nb, int k, int32_t* o
   else warp_topk_smem(keys, nb, k, out);
 }
 
-// Sum over a CTA of NW warps.  `red` holds two rows of NW words used in turn,
-// so one barrier per call suffices: a row is rewritten two calls later, after
-// the barrier of the call in between, when every thread has read it.
-template <int NW>
-__device__ __forceinline__ unsigned block_sum(unsigned v, unsigned* red, int& row) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  v = __reduce_add_sync(0xffffffffu, v);
-  unsigned* r = red + row * NW;
-  row ^= 1;
-  if (lane == 0) r[warp] = v;
-  __syncthreads();
-  unsigned s = 0;
-#pragma unroll
-  for (int w = 0; w < NW; ++w) s += r[w];
-  return s;
-}
-
 // Ascending ids of the keys above tau plus the first `need` keys equal to
 // tau (lowest ids first), -1 padded to k; the CTA's keys are in registers
 // (thread t holds keys t, t + NT, ...).  The keys array (nb words) is reused
@@ -242,60 +219,8 @@ __device__ inline void block_emit(const uint32_t (&kr)[PER], uint32_t* keys, int
   for (int s = static_cast<int>(keff) + lane; s < k; s += 32) out[s] = -1;
 }
 
-// Exact top-k of nb <= NT * PER keys (in shared memory) by a whole CTA of NT
-// threads; the same rules as warp_topk_bits.  The k-th largest key tau is
-// found bit by bit (32 steps of a CTA-wide count); `red` is 2 * NT / 32 words
-// of shared memory.
-template <int NT, int PER>
-__device__ inline void block_topk(uint32_t* keys, int nb, int k, int32_t* out, unsigned* red) {
-  constexpr int NW = NT / 32;
-  const int tid = threadIdx.x;
-  int row = 0;
-  uint32_t kr[PER];
-  unsigned nc = 0;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int j = i * NT + tid;
-    kr[i] = j < nb ? keys[j] : 0u;
-    nc += kr[i] != 0u;
-  }
-  nc = block_sum<NW>(nc, red, row);
-  const unsigned keff = nc < static_cast<unsigned>(k) ? nc : static_cast<unsigned>(k);
-  uint32_t tau = 0xffffffffu;
-  unsigned need = 0;
-  if (keff > 0u) {
-    // as in warp_topk_regs: stop once a prefix holds exactly keff keys
-    uint32_t prefix = 0u;
-    bool exact = false;
-#pragma unroll 1
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = prefix | (1u << bit);
-      unsigned c = 0;
-#pragma unroll
-      for (int i = 0; i < PER; ++i) c += kr[i] >= cand;
-      c = block_sum<NW>(c, red, row);
-      if (c >= keff) prefix = cand;
-      if (c == keff) {
-        exact = true;
-        break;
-      }
-    }
-    if (exact) {
-      tau = prefix - 1u;
-      need = 0u;
-    } else {
-      tau = prefix;
-      unsigned gt = 0;
-#pragma unroll
-      for (int i = 0; i < PER; ++i) gt += kr[i] > tau;
-      need = keff - block_sum<NW>(gt, red, row);
-    }
-  }
-  // every thread has passed a barrier after loading its keys
-  block_emit<NT, PER>(kr, keys, nb, k, keff, tau, need, out);
-}
-
-// The same selection by a CTA of 256 threads with an 8-bit radix search for
+// Exact top-k of nb <= 256 * PER keys (in shared memory) by a whole CTA of
+// 256 threads, with the rules of warp_topk_bits and an 8-bit radix search for
 // tau: four passes, each a histogram of the next 8 bits of the keys that
 // still agree with tau on the bits above (one private histogram per warp,
 // then one bin per thread), and a suffix scan over the 256 bins that picks
