@@ -1,0 +1,53 @@
+"""The algorithmic byte and FLOP counts behind the benchmark's roofline
+figures, derived here independently from the workload shapes: keys
+attended per query (sink + k blocks + window + the new keys), the bytes of
+one decode step (retained K and V rows, compressed keys, Q and O) and the
+algorithmic FLOPs of the causal prefill."""
+import bench
+from top_block_sparse_b200.inputs import WORKLOADS
+
+
+def _keys(S, k, b, W, n_new):
+    return S + k * b + W + n_new
+
+
+def test_decode_step_bytes():
+    # 32k decode: 64 sink + 32 blocks of 64 + 256 window + the new key
+    w = WORKLOADS["decode_32k"]
+    by = bench.decode_bytes(w)
+    pairs = 32 * 8
+    assert by["keys_per_query"] == _keys(64, 32, 64, 256, 1) == 2369
+    assert by["kv"] == pairs * 2369 * 128 * 2 * 2                # 310.5 MB
+    assert by["kc"] == pairs * (32768 // 64) * 128 * 4           # 67.1 MB
+    qo = 32 * 1 * 32 * 128 * 2
+    assert by["step"] == by["kv"] + by["kc"] + 2 * qo + qo
+    assert abs(by["step"] / 1e6 - 378.4) < 0.1
+    # draft chunk: 16 blocks, 6 new keys; 1M-token LSA: 4 sink keys, 4 blocks of 512, 512 window
+    assert bench.decode_bytes(WORKLOADS["draft_chunk_16k"])["keys_per_query"] == _keys(64, 16, 64, 256, 6) == 1350
+    d1m = bench.decode_bytes(WORKLOADS["decode_1m"])
+    assert d1m["keys_per_query"] == _keys(4, 4, 512, 512, 1) == 2565
+    assert d1m["kc"] == 4 * 8 * 2048 * 128 * 4
+    assert bench.decode_bytes(WORKLOADS["tiny_decode"])["keys_per_query"] == _keys(64, 8, 64, 128, 1) == 705
+
+
+def test_prefill_flops():
+    """Tile i of 64 queries (context C = 64 i) attends the sink block, the
+    top-64 of its max(0, i - 5) candidate blocks, the 4 window blocks before
+    it and its own keys causally; QK^T and PV are 4 d FLOP per (query, key,
+    head).  Scoring: each (tile, candidate block) pair costs 64 rows x 2 d
+    per KV head."""
+    w = WORKLOADS["prefill_64k"]
+    d, Hq, Hkv = 128, 32, 8
+    attn = score = 0
+    for i in range(65536 // 64):
+        C = 64 * i
+        sink = min(64, C)
+        window = C - max(C - 256, sink)
+        cand = max(0, i - 5)
+        ctx_keys = sink + 64 * min(64, cand) + window
+        attn += Hq * 4 * d * (64 * ctx_keys + 64 * 65 // 2)
+        score += Hkv * cand * 64 * 2 * d
+    c = bench.prefill_counts(w)
+    assert c["attn_alg"] == attn and abs(attn / 1e12 - 4.61) < 0.01
+    assert c["score_alg"] == score and abs(score / 1e9 - 68.0) < 0.1
+    assert c["attn_exec"] >= c["attn_alg"] and c["score_exec"] >= c["score_alg"]
