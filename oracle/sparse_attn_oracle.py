@@ -610,7 +610,7 @@ def bucket_decode_pair(q_tokens: np.ndarray, K: np.ndarray, V: np.ndarray, C: in
     scores = cents @ qhat if len(members) else np.zeros(0)
     s_end, w_begin = sink_window(C, p)
     cand = [g for g, ids in enumerate(members)
-            if any(s_end <= 4 * m + r < w_begin for m in ids for r in range(stride))]
+            if any(s_end <= stride * m + r < w_begin for m in ids for r in range(stride))]
     sel = select_topk(scores, cand, p.top_k)
     kept = sorted(m for g in sel.selected for m in members[g])
     if p.bucket_keys > 0:

@@ -390,6 +390,38 @@ def test_prefill_dense_equivalence_and_needles():
     assert len(r["sel"].selected) == min(64, i - 5)
 
 
+def test_prefill_head_selection_matches_tiles_and_brute_force():
+    """The selection-only helper picks, for every tile of a ragged case, the
+    same blocks as the full tile computation, and the same blocks as a brute
+    force: tile score = max over the rows of the hand-summed group logits,
+    candidates by key enumeration, then an exhaustive sort."""
+    r_ = rng(61)
+    G, d, b = 2, 16, 8
+    T = 13 * b + 5
+    K = r_.standard_normal((T, d))
+    V = r_.standard_normal((T, d))
+    q = r_.standard_normal((T, G, d))
+    p = orc.OracleParams(block_size=b, top_k=3, sink_keys=b, window_keys=2 * b)
+    Kc_all = orc.pool_mean(K, b)
+    nt = (T + b - 1) // b
+    sels = orc.prefill_head_selection(q, Kc_all, p, range(nt))
+    for i in range(nt):
+        full = orc.prefill_tile(q[i * b:(i + 1) * b], K, V, i, p, Kc_all)
+        assert sels[i].selected == full["sel"].selected, i
+        C = i * b
+        rows = range(i * b, min((i + 1) * b, T))
+        brute = []
+        for j in range(C // b):
+            keys = range(j * b, (j + 1) * b)
+            if all(t < b or t >= C - 2 * b for t in keys):
+                continue                                       # wholly inside sink or window
+            mean = [sum(K[t, c] for t in keys) / b for c in range(d)]
+            s = max(sum(sum(q[rr, g, c] for g in range(G)) * mean[c] for c in range(d)) for rr in rows)
+            brute.append((-s / math.sqrt(d), j))
+        brute.sort()
+        assert sels[i].selected == sorted(j for _, j in brute[:3]), i
+
+
 # ------------------------------------------- overlapping compression ---
 
 _OVL_CASES = [(64, 32, 16, 320), (64, 32, 16, 333), (64, 64, 16, 300), (64, 16, 16, 256),
@@ -597,6 +629,34 @@ def test_bucket_decode_selects_a_planted_needle_and_keeps_the_budget():
     qhat = orc._normalise(q[0].sum(axis=0))
     own = {m: float(orc._normalise(P[m]) @ qhat) for m in full}
     assert min(own[m] for m in kept) >= max([own[m] for m in set(full) - set(kept)] + [-2.0])
+
+
+@pytest.mark.parametrize("stride", [2, 4, 8])
+def test_bucket_candidates_by_key_enumeration(stride):
+    """A bucket is a candidate iff one of its raw keys lies outside sink and
+    window, for any pool stride: expected sets built key by key (raw key t
+    belongs to pool key t // stride, which belongs to one bucket), with a
+    sink and a window that cut through buckets."""
+    r = rng(60 + stride)
+    b, d = 512, 16
+    C = 3 * b
+    K, V = r.standard_normal((C + 1, d)), r.standard_normal((C + 1, d))
+    q = r.standard_normal((1, 2, d))
+    p = _lsa_params(pool_stride=stride, sink_keys=6, window_keys=300, top_k=10_000)
+    res = orc.bucket_decode_pair(q, K, V, C, p)
+    owner = {}
+    for g, ids in enumerate(res["members"]):
+        for m in ids:
+            owner[m] = g
+    expected = set()
+    for t in range(C):
+        if 6 <= t < C - 300:
+            expected.add(owner[t // stride])
+    assert sorted(expected) == res["candidates"]
+    assert all(len(ids) <= 16 // stride for ids in res["members"])
+    # every candidate selected: every key of the context is attended (dense)
+    for g in range(2):
+        np.testing.assert_allclose(res["O"][0, g], _sdpa(q[0, g], K, V, C + 1), atol=1e-12)
 
 
 # ---------------------------------------------- planted-mistake checks ---
