@@ -68,43 +68,73 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """nvidia-smi clock / throttle sampling during the timed region.
+
+    nvidia-smi is started first and the timed work begins only once it has
+    printed its first samples: its start-up (driver queries on the GPU) would
+    otherwise fall inside a short timed region and slow the first steps."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 20
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.lines = []
+        self.marks = []
+
+    def _reader(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.lines.append((time.perf_counter(), ln))
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.PERIOD_MS)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
-        time.sleep(0.25)
+        if self.proc is not None:
+            self.thread = threading.Thread(target=self._reader, daemon=True)
+            self.thread.start()
+            t0 = time.perf_counter()
+            while len(self.lines) < 3 and time.perf_counter() - t0 < 10.0 and self.proc.poll() is None:
+                time.sleep(0.01)
         return self
 
+    def mark(self):
+        """Host time stamp taken right after a synchronize: the timed region
+        lies between the first and the last mark."""
+        self.marks.append(time.perf_counter())
+
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
-            time.sleep(0.15)
+            time.sleep(2.5 * self.PERIOD_MS / 1000)
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-                out = ""
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            self.thread.join(timeout=5)
         return False
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        """Median SM clock and active throttle reasons of the samples taken
+        inside the timed region (between the marks, widened by one sampling
+        period), or of all samples if none falls inside."""
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        rows = list(self.lines)
+        if len(self.marks) >= 2:
+            lo, hi = self.marks[0], self.marks[-1] + self.PERIOD_MS / 1000
+            inside = [r for r in rows if lo <= r[0] <= hi]
+            if inside:
+                rows = inside
+        sm, mx, reasons = [], None, set()
+        for _, ln in rows:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -119,7 +149,16 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "sample_period_ms": self.PERIOD_MS}
+
+
+def spread(ms_list):
+    """Spread of per-step device times (ms): min, median, 90th percentile,
+    max and mean."""
+    s = sorted(ms_list)
+    p90 = s[min(len(s) - 1, int(math.ceil(0.9 * len(s))) - 1)]
+    return {"min": s[0], "median": statistics.median(s), "p90": p90, "max": s[-1],
+            "mean": statistics.mean(s), "n": len(s)}
 
 
 def decode_bytes(w) -> dict:
@@ -190,13 +229,16 @@ class L2Flush:
         torch.sum(self.r, dim=0, out=self.sink)
 
 
-def timed_steps(fn, steps, warmup, stream, flush):
+def timed_steps(fn, steps, warmup, stream, flush, clk=None):
     """W warm-ups, then K steps each preceded by an L2 flush; returns the
-    per-step device times (ms) from CUDA events on `stream`."""
+    per-step device times (ms) from CUDA events on `stream`.  `clk` (a
+    ClockSampler) gets host marks at both ends of the timed region."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    if clk is not None:
+        clk.mark()
     with torch.cuda.stream(stream):
         for s, e in evs:
             flush()
@@ -204,7 +246,35 @@ def timed_steps(fn, steps, warmup, stream, flush):
             fn()
             e.record(stream)
     torch.cuda.synchronize()
+    if clk is not None:
+        clk.mark()
     return [s.elapsed_time(e) for s, e in evs]
+
+
+def timed_interleaved(fns, steps, warmup, stream, flush, clk=None):
+    """Like timed_steps for several functions at once: every round runs each
+    function once (each after its own L2 flush), so they all see the same
+    clocks and temperature.  Returns one list of per-step times (ms) per
+    function."""
+    for _ in range(warmup):
+        for fn in fns:
+            fn()
+    torch.cuda.synchronize()
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in fns]
+           for _ in range(steps)]
+    if clk is not None:
+        clk.mark()
+    with torch.cuda.stream(stream):
+        for row in evs:
+            for fn, (s, e) in zip(fns, row):
+                flush()
+                s.record(stream)
+                fn()
+                e.record(stream)
+    torch.cuda.synchronize()
+    if clk is not None:
+        clk.mark()
+    return [[row[i][0].elapsed_time(row[i][1]) for row in evs] for i in range(len(fns))]
 
 
 # ------------------------------------------------------------- CPU oracle --
@@ -359,7 +429,7 @@ def run_ours(args, w, rank, world, local_rank):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
-        step_ms = timed_steps(step, args.steps, args.warmup, stream, flush)
+        step_ms = timed_steps(step, args.steps, args.warmup, stream, flush, clk)
     if sa.read_status(ws, stream) != sa.SA_OK:
         raise RuntimeError("device status word set during the timed steps")
     ms = reduce_max(sum(step_ms) / len(step_ms), world, dev)
@@ -436,6 +506,14 @@ def run_ours(args, w, rank, world, local_rank):
         "gpu_launches": sa.decode_launches(p) * args.steps,
         "clocks": clk.summary(),
     }
+    # per-step spread of the timed steps, and the mean step in SM clock
+    # cycles at the sampled median clock (a slower clock shows as fewer
+    # cycles per step, not as a slower kernel)
+    sp = spread(step_ms)
+    line["step_ms_min"], line["step_ms_median"], line["step_ms_p90"] = sp["min"], sp["median"], sp["p90"]
+    line["step_ms_max"] = sp["max"]
+    mhz = line["clocks"].get("sm_mhz")
+    line["step_kcycles_at_median_sm_mhz"] = ms * mhz if mhz else None
     return line
 
 
@@ -473,6 +551,54 @@ def prefill_counts(w):
     return dict(attn_alg=attn_alg, attn_exec=attn_exec, score_alg=score_alg, score_exec=score_exec)
 
 
+def prefill_report(w, full_l, score_l, attn_l, pk):
+    """The prefill object of the benchmark line from the per-step times (ms)
+    of the full call, the scoring call and the attention call, and the peaks
+    (hbm GB/s, bf16 TFLOP/s, sustained TFLOP/s, source)."""
+    T = w.n_q
+    nb = T // 64
+    full_ms, score_ms, attn_ms = (statistics.mean(x) for x in (full_l, score_l, attn_l))
+    c = prefill_counts(w)
+    hbm, tfl, tfl_s, src = pk
+    q_bytes = T * w.num_q_heads * 128 * 2
+    kc_bytes = w.num_kv_heads * nb * 128 * 4
+    tf = lambda flop, ms: flop / (ms * 1e-3) / 1e12
+    return {
+        "workload": f"prefill_64k: causal prefill T={w.n_q}, Hq=32, Hkv=8, d=128, bf16, tile = block 64, "
+                    "top-k 64 + sink 64 keys + window 256 keys",
+        "ms": full_ms,
+        "ms_spread": spread(full_l),
+        "tflops": tf(c["attn_alg"] + c["score_alg"], full_ms),
+        "tflops_note": "algorithmic attention + scoring FLOPs / whole prefill time (pool, score, top-k, attention)",
+        "timing": "the full call, the scoring call and the attention call interleaved step by step (each after "
+                  "its own L2 flush), so all three see the same clocks",
+        "attention": {"kernel": "prefill_attn_kernel (tcgen05)", "ms": attn_ms, "ms_spread": spread(attn_l),
+                      "alg_tflops": tf(c["attn_alg"], attn_ms),
+                      "exec_tflops": tf(c["attn_exec"], attn_ms),
+                      "frac_of_bf16_peak": tf(c["attn_alg"], attn_ms) / tfl,
+                      "exec_frac_of_bf16_peak": tf(c["attn_exec"], attn_ms) / tfl,
+                      "exec_flop": c["attn_exec"], "alg_flop": c["attn_alg"],
+                      "note": "frac_of_bf16_peak counts the algorithmic FLOPs (attended keys only); the executed "
+                              "count adds the masked half of each diagonal block"},
+        "scoring": {"kernel": "kc_split + prefill_score_kernel (tcgen05, split bf16 x3) + prefill_topk_kernel",
+                    "ms": score_ms, "ms_spread": spread(score_l),
+                    "alg_tflops": tf(c["score_alg"], score_ms),
+                    "exec_tflops": tf(c["score_exec"], score_ms),
+                    "frac_of_bf16_peak": tf(c["score_alg"], score_ms) / tfl,
+                    "exec_frac_of_bf16_peak": tf(c["score_exec"], score_ms) / tfl,
+                    "hbm_bytes": q_bytes + kc_bytes,
+                    "hbm_gbs": (q_bytes + kc_bytes) / (score_ms * 1e-3) / 1e9,
+                    "hbm_frac": (q_bytes + kc_bytes) / (score_ms * 1e-3) / 1e9 / hbm,
+                    "alg_gflop": c["score_alg"] / 1e9, "exec_gflop": c["score_exec"] / 1e9,
+                    "note": "three readings: frac_of_bf16_peak = algorithmic FLOPs (GQA-summed query rows x the "
+                            "causally visible compressed keys); exec_frac_of_bf16_peak = the MMA FLOPs executed "
+                            "(three bf16 products per fp32 product for the split-precision scores, whole 128-block "
+                            "chunks); hbm_frac = Q and Kc read once over the call"},
+        "attention_plus_scoring_ms": attn_ms + score_ms,
+        "peak_bf16_tflops": tfl, "peak_hbm_gbs": hbm, "peak_source": src,
+    }
+
+
 def run_prefill_bench(args, dev, stream, flush):
     """Times the full causal prefill and its two tensor-core kernels alone."""
     from top_block_sparse_b200 import sa
@@ -505,30 +631,16 @@ def run_prefill_bench(args, dev, stream, flush):
         sa.sparse_attn_given_idx(pt, Q, K, V, idx, O, lse, ws_g, stream=stream)
 
     n = args.prefill_steps
-    full_ms = statistics.mean(timed_steps(full, n, 3, stream, flush))
-    score_ms = statistics.mean(timed_steps(score, n, 3, stream, flush))
-    attn_ms = statistics.mean(timed_steps(attn, n, 3, stream, flush))
+    # the three calls interleaved step by step: a long run of tensor-core work
+    # lowers the clock under the power cap, so timing them one after another
+    # would give the later ones a lower clock
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        full_l, score_l, attn_l = timed_interleaved([full, score, attn], n, 3, stream, flush, clk)
     if sa.read_status(ws, stream) != sa.SA_OK:
         raise RuntimeError("device status word set during the prefill runs")
-    c = prefill_counts(w)
-    hbm, tfl, tfl_s, src = peaks()
-    return {
-        "workload": f"prefill_64k: causal prefill T={w.n_q}, Hq=32, Hkv=8, d=128, bf16, tile = block 64, "
-                    "top-k 64 + sink 64 keys + window 256 keys",
-        "ms": full_ms,
-        "tflops": (c["attn_alg"] + c["score_alg"]) / (full_ms * 1e-3) / 1e12,
-        "tflops_note": "algorithmic attention + scoring FLOPs / whole prefill time (pool, score, top-k, attention)",
-        "attention": {"kernel": "prefill_attn_kernel (tcgen05)", "ms": attn_ms,
-                      "exec_tflops": c["attn_exec"] / (attn_ms * 1e-3) / 1e12,
-                      "alg_tflops": c["attn_alg"] / (attn_ms * 1e-3) / 1e12,
-                      "frac_of_bf16_peak": c["attn_exec"] / (attn_ms * 1e-3) / 1e12 / tfl,
-                      "exec_flop": c["attn_exec"], "alg_flop": c["attn_alg"]},
-        "scoring": {"kernel": "kc_split + prefill_score_kernel (tcgen05, split bf16 x3) + prefill_topk_kernel",
-                    "ms": score_ms, "exec_tflops": c["score_exec"] / (score_ms * 1e-3) / 1e12,
-                    "frac_of_bf16_peak": c["score_exec"] / (score_ms * 1e-3) / 1e12 / tfl,
-                    "alg_gflop": c["score_alg"] / 1e9, "exec_gflop": c["score_exec"] / 1e9},
-        "peak_bf16_tflops": tfl, "peak_source": src,
-    }
+    rep = prefill_report(w, full_l, score_l, attn_l, peaks())
+    rep["clocks"] = clk.summary()
+    return rep
 
 
 def run_verify_bench(args, dev, stream, flush):

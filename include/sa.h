@@ -297,7 +297,13 @@ sa_status sa_sparse_attn_prefill(const sa_params* p, const void* Q,
  * stream or otherwise order them.  Each call clears the array's status word
  * and tickets first; bad index entries are skipped exactly as in
  * sa_sparse_attn_given_idx but cannot be read back (there is no workspace to
- * pass to sa_read_status).  Calls no allocating routine. */
+ * pass to sa_read_status).  Only decode and draft-chunk tables
+ * (select == SA_SEL_QUERY0) are taken: prefill tables (SA_SEL_TILE_MAX)
+ * return SA_ERR_UNSUPPORTED; pass those to sa_sparse_attn_given_idx.  The
+ * array's address is looked up once per device ordinal and kept: after a
+ * cudaDeviceReset of that device the kept address is stale, so reload the
+ * library before calling this entry point again.  Calls no allocating
+ * routine. */
 sa_status sa_sparse_attn_given_idx_noalloc(const sa_params* p, const void* Q,
                                            const void* K, const void* V,
                                            const int32_t* idx, int32_t idx_len,

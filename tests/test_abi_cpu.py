@@ -1,11 +1,14 @@
 """CPU-only checks of the C ABI: the library loads without a GPU, exports
 every symbol include/sa.h declares, the params struct matches, and host-side
-validation rejects bad arguments before any launch."""
+validation rejects bad arguments before any launch.  The validation tests
+pass fake device pointers, so they are skipped wherever a GPU could run a
+kernel on them (only the symbol and layout checks run there)."""
 import ctypes
 import os
 import re
 
 import pytest
+import torch
 
 from top_block_sparse_b200 import sa
 
@@ -14,6 +17,9 @@ HEADER = open(os.path.join(ROOT, "include", "sa.h")).read()
 
 FAKE = ctypes.c_void_p(0x10000)          # 16-byte aligned, never dereferenced
 FAKE_ODD = ctypes.c_void_p(0x10008)
+
+# tests that hand the library FAKE addresses run on hosts without a GPU only
+host_only = pytest.mark.skipif(torch.cuda.is_available(), reason="fake device pointers: host-only test")
 
 
 def declared_functions():
@@ -54,6 +60,7 @@ def _decode(p, ws_bytes=1 << 30, q=FAKE, kc=FAKE):
                        FAKE, ws_bytes, None)
 
 
+@host_only
 @pytest.mark.parametrize("kw,status", [
     (dict(head_dim=64), sa.SA_ERR_UNSUPPORTED),
     (dict(num_q_heads=7), sa.SA_ERR_INVALID),
@@ -76,6 +83,7 @@ def test_validation_rejects(kw, status):
         assert sa.raw_call("sa_workspace_size", ctypes.byref(_p(**kw)), op) == 0
 
 
+@host_only
 @pytest.mark.parametrize("kw,status", [
     (dict(pool="overlap", pool_stride=24, pool_kernel=32), sa.SA_ERR_INVALID),   # s does not divide b
     (dict(pool="overlap", pool_stride=16, pool_kernel=8), sa.SA_ERR_INVALID),    # l < s
@@ -87,6 +95,7 @@ def test_overlap_validation_rejects(kw, status):
     assert "pool" in sa.raw_call("sa_last_error").decode()
 
 
+@host_only
 def test_overlap_params_and_workspace():
     """pool_kernel must be 0 outside the overlap mode; the overlap mode runs
     as two kernels (scoring, attention), its prefill is not built, and its
@@ -106,6 +115,7 @@ def test_overlap_params_and_workspace():
     assert w_ovl >= w_mean + 4 * 4 * (n_c - 4096 // 64) - 1024
 
 
+@host_only
 def test_validation_null_and_alignment():
     p = _p()
     assert sa.raw_call("sa_sparse_attn_decode", None, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
@@ -117,6 +127,7 @@ def test_validation_null_and_alignment():
     assert _decode(p2) == sa.SA_ERR_INVALID
 
 
+@host_only
 def test_workspace_too_small():
     p = _p()
     need = sa.workspace_size(p, sa.SA_OP_DECODE)
@@ -134,6 +145,7 @@ def test_workspace_sizes_grow_with_the_problem():
     assert sa.workspace_size(_p(), sa.SA_OP_SCORE_TOPK) > 0
 
 
+@host_only
 def test_given_idx_validation():
     p = _p()
     st = sa.raw_call("sa_sparse_attn_given_idx", ctypes.byref(p), FAKE, FAKE, FAKE, None, 4, FAKE, None,
@@ -149,6 +161,7 @@ def _verify(p, ws_bytes=1 << 30, mass=FAKE, idx=FAKE):
                        FAKE, ws_bytes, None)
 
 
+@host_only
 @pytest.mark.parametrize("kw,status", [
     (dict(dtype="f32"), sa.SA_ERR_UNSUPPORTED),          # tensor cores: bf16 only
     (dict(block_size=32), sa.SA_ERR_UNSUPPORTED),        # mass tiles are 64 keys
@@ -161,6 +174,7 @@ def test_verify_validation_rejects(kw, status):
     assert sa.raw_call("sa_last_error").decode() != ""
 
 
+@host_only
 def test_verify_null_arguments_and_workspace():
     p = _p(n_q=3, num_q_heads=4, num_kv_heads=2)
     assert _verify(p, mass=None) == sa.SA_ERR_INVALID
@@ -184,6 +198,7 @@ def _column(p, n_cols=70, cols=FAKE, ws_bytes=1 << 30):
                        FAKE, ws_bytes, None)
 
 
+@host_only
 @pytest.mark.parametrize("kw,n_cols,status", [
     (dict(dtype="f32"), 70, sa.SA_ERR_UNSUPPORTED),           # tensor cores: bf16 only
     (dict(num_q_heads=4), 70, sa.SA_ERR_UNSUPPORTED),         # GQA 2: built for groups of 4 heads
@@ -196,6 +211,7 @@ def test_column_validation_rejects(kw, n_cols, status):
     assert sa.raw_call("sa_last_error").decode() != ""
 
 
+@host_only
 def test_column_null_table_and_workspace():
     p = _pcol()
     assert _column(p, cols=None) == sa.SA_ERR_INVALID            # n_cols > 0 needs a table
@@ -209,3 +225,15 @@ def test_column_null_table_and_workspace():
 def test_status_strings():
     for code, name in [(0, "SA_OK"), (4, "SA_ERR_INDEX"), (6, "SA_ERR_TIMEOUT")]:
         assert sa.raw_call("sa_status_string", code).decode() == name
+
+
+def test_noalloc_refuses_prefill_tables():
+    """The allocation-free entry point takes decode and draft-chunk tables
+    only: a prefill table is refused before the pointers are looked at (NULL
+    pointers here, so nothing could be launched on any host)."""
+    p = _p(prefill=True, ctx_len=0, n_q=4096)
+    st = sa.raw_call("sa_sparse_attn_given_idx_noalloc", ctypes.byref(p), None, None, None, None, 8, None, None,
+                     None)
+    assert st == sa.SA_ERR_UNSUPPORTED
+    msg = sa.raw_call("sa_last_error").decode()
+    assert "SA_SEL_QUERY0" in msg and "sa_sparse_attn_given_idx" in msg

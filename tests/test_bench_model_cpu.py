@@ -51,3 +51,32 @@ def test_prefill_flops():
     assert c["attn_alg"] == attn and abs(attn / 1e12 - 4.61) < 0.01
     assert c["score_alg"] == score and abs(score / 1e9 - 68.0) < 0.1
     assert c["attn_exec"] >= c["attn_alg"] and c["score_exec"] >= c["score_alg"]
+
+
+def test_prefill_report_fractions():
+    """The prefill line's headline fractions count algorithmic FLOPs; the
+    executed-FLOP fractions are separate fields, and the scoring call also
+    reports Q and Kc read once against the HBM peak."""
+    w = WORKLOADS["prefill_64k"]
+    c = bench.prefill_counts(w)
+    pk = (6000.0, 1500.0, 1400.0, "test")
+    rep = bench.prefill_report(w, [5.0, 5.2], [0.25, 0.27], [4.9, 4.7], pk)
+    a, s = rep["attention"], rep["scoring"]
+    assert abs(a["ms"] - 4.8) < 1e-12 and abs(s["ms"] - 0.26) < 1e-12
+    assert abs(a["frac_of_bf16_peak"] - c["attn_alg"] / 4.8e-3 / 1e12 / 1500.0) < 1e-12
+    assert abs(a["exec_frac_of_bf16_peak"] - c["attn_exec"] / 4.8e-3 / 1e12 / 1500.0) < 1e-12
+    assert abs(s["frac_of_bf16_peak"] - c["score_alg"] / 0.26e-3 / 1e12 / 1500.0) < 1e-12
+    assert abs(s["exec_frac_of_bf16_peak"] - c["score_exec"] / 0.26e-3 / 1e12 / 1500.0) < 1e-12
+    # split precision: three bf16 products per fp32 product, so executed > 3x algorithmic
+    assert s["exec_frac_of_bf16_peak"] > 3 * s["frac_of_bf16_peak"]
+    q_bytes = 65536 * 32 * 128 * 2
+    kc_bytes = 8 * 1024 * 128 * 4
+    assert s["hbm_bytes"] == q_bytes + kc_bytes
+    assert abs(s["hbm_frac"] - (q_bytes + kc_bytes) / 0.26e-3 / 1e9 / 6000.0) < 1e-12
+    assert rep["ms_spread"]["min"] == 5.0 and rep["ms_spread"]["max"] == 5.2
+
+
+def test_step_spread():
+    sp = bench.spread([3.0, 1.0, 2.0, 10.0, 4.0, 5.0, 6.0, 7.0, 8.0, 9.0])
+    assert sp["min"] == 1.0 and sp["max"] == 10.0 and sp["median"] == 5.5
+    assert sp["p90"] == 9.0 and sp["n"] == 10 and abs(sp["mean"] - 5.5) < 1e-12

@@ -70,10 +70,21 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(name, over):
 
 
 def test_noalloc_refuses_problems_larger_than_its_array():
-    w = WORKLOADS["draft_chunk_16k"].scaled(batch=256)
+    """A problem whose scratch exceeds the static array is refused before
+    any launch.  Every buffer is a real allocation of its full layout (256
+    draft chunks over a 256-key context), so even a launch would stay in
+    bounds."""
+    w = WORKLOADS["draft_chunk_16k"].scaled(batch=256, ctx_len=256)
     p = sa.params_for(w)
-    fake = ctypes.c_void_p(0x10000)
-    st = sa.raw_call("sa_sparse_attn_given_idx_noalloc", ctypes.byref(p), fake, fake, fake, fake, w.top_k,
-                     fake, None, None)
+    assert sa.workspace_size(p, sa.SA_OP_GIVEN_IDX) > 16 << 20
+    cap = w.ctx_len + w.n_q
+    Q = torch.zeros((w.batch, w.n_q, w.num_q_heads, 128), device="cuda", dtype=torch.bfloat16)
+    K = torch.zeros((w.batch, w.num_kv_heads, cap, 128), device="cuda", dtype=torch.bfloat16)
+    V = torch.zeros_like(K)
+    O = torch.empty_like(Q)
+    idx = torch.full((w.batch, w.num_kv_heads, w.top_k), -1, device="cuda", dtype=torch.int32)
+    st = sa.raw_call("sa_sparse_attn_given_idx_noalloc", ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
+                     w.top_k, _ptr(O), None, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == sa.SA_ERR_WORKSPACE
     assert "static" in sa.raw_call("sa_last_error").decode()
+    torch.cuda.synchronize()

@@ -849,7 +849,10 @@ extern "C" sa_status sa_sparse_attn_given_idx_noalloc(const sa_params* p, const 
   const bool prefill = p && p->select == SA_SEL_TILE_MAX;
   sa_status st = check_params(p, prefill);
   if (st != SA_OK) return st;
-  if (prefill) return fail(SA_ERR_UNSUPPORTED, "prefill index tables are not built in this library version");
+  if (prefill)
+    return fail(SA_ERR_UNSUPPORTED,
+                "the allocation-free entry point takes decode and draft-chunk index tables (SA_SEL_QUERY0) only; "
+                "pass prefill tables (SA_SEL_TILE_MAX) to sa_sparse_attn_given_idx with a workspace");
   if (!Q || !K || !V || !O) return fail(SA_ERR_INVALID, "Q, K, V and O must be non-NULL");
   if (idx_len < 0 || idx_len > 4096) return fail(SA_ERR_INVALID, "idx_len %d must be in [0, 4096]", idx_len);
   if (idx_len > 0 && !idx) return fail(SA_ERR_INVALID, "idx is NULL");
