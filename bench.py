@@ -229,17 +229,30 @@ class L2Flush:
         torch.sum(self.r, dim=0, out=self.sink)
 
 
+def queue_ahead(steps):
+    """Holds the stream for a few ms (a GPU spin, outside every timed
+    region) so that the host enqueues the first steps before the GPU reaches
+    them: without it the first step's start event fires while the host is
+    still issuing that step's launch, and the host's launch latency would be
+    timed as device time."""
+    ms = min(50.0, 1.0 + 0.3 * steps)
+    torch.cuda._sleep(int(ms * 1e-3 * 2.0e9))
+
+
 def timed_steps(fn, steps, warmup, stream, flush, clk=None):
     """W warm-ups, then K steps each preceded by an L2 flush; returns the
     per-step device times (ms) from CUDA events on `stream`.  `clk` (a
     ClockSampler) gets host marks at both ends of the timed region."""
-    for _ in range(warmup):
-        fn()
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush()
+            fn()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     if clk is not None:
         clk.mark()
     with torch.cuda.stream(stream):
+        queue_ahead(steps)
         for s, e in evs:
             flush()
             s.record(stream)
@@ -256,15 +269,18 @@ def timed_interleaved(fns, steps, warmup, stream, flush, clk=None):
     function once (each after its own L2 flush), so they all see the same
     clocks and temperature.  Returns one list of per-step times (ms) per
     function."""
-    for _ in range(warmup):
-        for fn in fns:
-            fn()
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            for fn in fns:
+                flush()
+                fn()
     torch.cuda.synchronize()
     evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in fns]
            for _ in range(steps)]
     if clk is not None:
         clk.mark()
     with torch.cuda.stream(stream):
+        queue_ahead(steps * len(fns))
         for row in evs:
             for fn, (s, e) in zip(fns, row):
                 flush()
@@ -428,6 +444,7 @@ def run_ours(args, w, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    ClockSampler.PERIOD_MS = args.clock_period_ms
     with ClockSampler(local_rank) as clk:
         step_ms = timed_steps(step, args.steps, args.warmup, stream, flush, clk)
     if sa.read_status(ws, stream) != sa.SA_OK:
@@ -512,6 +529,7 @@ def run_ours(args, w, rank, world, local_rank):
     sp = spread(step_ms)
     line["step_ms_min"], line["step_ms_median"], line["step_ms_p90"] = sp["min"], sp["median"], sp["p90"]
     line["step_ms_max"] = sp["max"]
+    line["step_us"] = [round(x * 1000, 1) for x in step_ms]
     mhz = line["clocks"].get("sm_mhz")
     line["step_kcycles_at_median_sm_mhz"] = ms * mhz if mhz else None
     return line
@@ -907,6 +925,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode_32k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-period-ms", type=int, default=20, help="nvidia-smi sampling period")
     ap.add_argument("--cpu-pairs", type=int, default=16)
     ap.add_argument("--ref-pairs", type=int, default=4)
     ap.add_argument("--no-prefill", action="store_true")
