@@ -527,6 +527,8 @@ def lsa_pool_keys(K: np.ndarray, stride: int = 4) -> np.ndarray:
     ``stride`` consecutive unit keys summed.  Returns [len(K) // stride, d]."""
     K = np.asarray(K, dtype=np.float64)
     m = K.shape[0] // stride
+    if m == 0:
+        return np.zeros((0, K.shape[1]))
     return _normalise(K[:m * stride]).reshape(m, stride, -1).sum(axis=1)
 
 
@@ -597,15 +599,17 @@ def lsa_bucket_index(K: np.ndarray, C: int, p: OracleParams):
 
 
 def bucket_decode_pair(q_tokens: np.ndarray, K: np.ndarray, V: np.ndarray, C: int,
-                       p: OracleParams) -> Dict:
+                       p: OracleParams, index=None) -> Dict:
     """Decode / draft chunk for one (sequence, KV head) with LSA's flat bucket
     retrieval [LSA review §2.2-2.3] (reading R19): normalised index query of
     the first new token scores every bucket centroid; the top-k candidate
     buckets are expanded to raw keys and joined with sink, window and the
-    chunk (R3, R9); masked softmax attention as in decode_pair."""
+    chunk (R3, R9); masked softmax attention as in decode_pair.  ``index``
+    (optional) is this context's (members, centroids) as lsa_bucket_index
+    returns them, when the caller has built it already."""
     n_q, G, d = q_tokens.shape
     stride = p.pool_stride
-    members, cents = lsa_bucket_index(K, C, p)
+    members, cents = lsa_bucket_index(K, C, p) if index is None else index
     qhat = _normalise(index_query(q_tokens[0]))
     scores = cents @ qhat if len(members) else np.zeros(0)
     s_end, w_begin = sink_window(C, p)

@@ -631,6 +631,24 @@ def test_bucket_decode_selects_a_planted_needle_and_keeps_the_budget():
     assert min(own[m] for m in kept) >= max([own[m] for m in set(full) - set(kept)] + [-2.0])
 
 
+def test_bucket_decode_before_the_first_cluster_block():
+    """A context shorter than one cluster block has no pool keys, no buckets
+    and nothing to select: with a window covering it, every key is attended
+    (library dense attention); with none, only the sink and the chunk."""
+    r = rng(62)
+    C, d = 300, 16
+    K, V = r.standard_normal((C + 2, d)), r.standard_normal((C + 2, d))
+    q = r.standard_normal((2, 2, d))
+    assert orc.lsa_pool_keys(K[:0]).shape == (0, d)
+    res = orc.bucket_decode_pair(q, K, V, C, _lsa_params(top_k=8))
+    assert res["members"] == [] and res["kept"] == [] and res["sel"].selected == []
+    for j in range(2):
+        for g in range(2):
+            np.testing.assert_allclose(res["O"][j, g], _sdpa(q[j, g], K, V, C + j + 1), atol=1e-12)
+    res = orc.bucket_decode_pair(q, K, V, C, _lsa_params(top_k=8, window_keys=0))
+    assert res["positions"][1].tolist() == [0, 1, 2, 3, C, C + 1]
+
+
 @pytest.mark.parametrize("stride", [2, 4, 8])
 def test_bucket_candidates_by_key_enumeration(stride):
     """A bucket is a candidate iff one of its raw keys lies outside sink and
