@@ -318,6 +318,116 @@ def oracle_sample(w, inp_cpu_pairs, n_pairs_total, min_seconds=10.0):
     return per_pair * n_pairs_total, dt, done
 
 
+class ParityTally:
+    """Per-config parity of the timed GPU results against the float64 oracle
+    (one host core): selected sets identical / near-ties / mismatches, and
+    the output errors of the pairs whose sets match (max abs, relative L2;
+    for bf16 outputs also the max abs beyond half a bf16 step of the exact
+    value, which the output format cannot come closer than)."""
+
+    def __init__(self):
+        self.n = self.match = self.near = self.mismatch = 0
+        self.max_abs = self.max_abs_fmt = 0.0
+        self.se = self.sr = 0.0
+        self.oracle_s = 0.0
+
+    def sets(self, got, sel):
+        self.n += 1
+        if got == sel.selected:
+            self.match += 1
+            return True
+        if sel.near_tie:
+            self.near += 1
+        else:
+            self.mismatch += 1
+        return False
+
+    def out(self, got, ref):
+        import numpy as np
+        g = got.double().cpu().numpy().reshape(ref.shape)
+        d = np.abs(g - ref)
+        self.max_abs = max(self.max_abs, float(d.max()) if d.size else 0.0)
+        if got.dtype == torch.bfloat16:
+            ax = np.abs(ref)
+            half = np.where(ax > 0, np.exp2(np.floor(np.log2(np.where(ax > 0, ax, 1.0))) - 8), 0.0)
+            d = np.maximum(d - half, 0.0)
+        self.max_abs_fmt = max(self.max_abs_fmt, float(d.max()) if d.size else 0.0)
+        self.se += float(((g - ref) ** 2).sum())
+        self.sr += float((ref ** 2).sum())
+
+    def report(self, sample, extrapolate=1.0):
+        rel = math.sqrt(self.se / self.sr) if self.sr > 0 else 0.0
+        return {"checked": self.n, "sets_match": self.match, "near_ties": self.near, "mismatches": self.mismatch,
+                "max_abs": self.max_abs, "max_abs_beyond_bf16_rounding": self.max_abs_fmt, "rel_l2": rel,
+                "oracle_s": self.oracle_s, "oracle_s_full_config": self.oracle_s * extrapolate,
+                "oracle_cores": 1, "sample": sample}
+
+
+def decode_parity(w, inp, O, idx, pairs, n_pairs_total, min_pairs_note=""):
+    """Oracle decode of the sampled pairs on one core, compared with the
+    GPU's index table and output of the same inputs."""
+    from threadpoolctl import threadpool_limits
+    from oracle import sparse_attn_oracle as orc
+    op = orc.OracleParams(block_size=w.block_size, top_k=w.top_k, sink_keys=w.sink_keys,
+                          window_keys=w.window_keys, pool=w.pool, pool_stride=w.pool_stride,
+                          pool_kernel=w.pool_kernel)
+    G = w.group
+    t = ParityTally()
+    with threadpool_limits(limits=1):
+        for (b, h) in pairs:
+            q = inp["Q"][b, :, h * G:(h + 1) * G].cpu().double().numpy()
+            K = inp["K"][b, h, :w.kv_len].cpu().double().numpy()
+            V = inp["V"][b, h, :w.kv_len].cpu().double().numpy()
+            t0 = time.perf_counter()
+            r = orc.decode_pair(q, K, V, w.ctx_len, op)
+            t.oracle_s += time.perf_counter() - t0
+            got = [int(x) for x in idx[b, h].tolist() if x >= 0]
+            if t.sets(got, r["sel"]):
+                t.out(O[b, :, h * G:(h + 1) * G], r["O"])
+    sample = (f"every (sequence, KV head) pair ({len(pairs)})" if len(pairs) == n_pairs_total else
+              f"{len(pairs)} of {n_pairs_total} (sequence, KV head) pairs, evenly spaced{min_pairs_note}")
+    return t.report(sample, n_pairs_total / max(1, len(pairs)))
+
+
+def prefill_parity(w, Q, K, V, O, idx, heads, tiles):
+    """Oracle of sampled prefill tiles (selection and attention, one core)
+    against the GPU's per-tile tables and output rows."""
+    from threadpoolctl import threadpool_limits
+    from oracle import sparse_attn_oracle as orc
+    op = orc.OracleParams(block_size=w.block_size, top_k=w.top_k, sink_keys=w.sink_keys,
+                          window_keys=w.window_keys)
+    G, b = w.group, w.block_size
+    t = ParityTally()
+    with threadpool_limits(limits=1):
+        for h in heads:
+            Kh = K[0, h, :w.n_q].cpu().double().numpy()
+            Vh = V[0, h, :w.n_q].cpu().double().numpy()
+            t0 = time.perf_counter()
+            Kc = orc.compress(Kh, op)
+            t.oracle_s += time.perf_counter() - t0
+            for i in tiles:
+                q = Q[0, i * b:(i + 1) * b, h * G:(h + 1) * G].cpu().double().numpy()
+                t0 = time.perf_counter()
+                r = orc.prefill_tile(q, Kh, Vh, i, op, Kc)
+                t.oracle_s += time.perf_counter() - t0
+                got = [int(x) for x in idx[0, h, i].tolist() if x >= 0]
+                if t.sets(got, r["sel"]):
+                    t.out(O[0, i * b:(i + 1) * b, h * G:(h + 1) * G], r["O"])
+    n_tiles = (w.n_q + b - 1) // b
+    return t.report(f"{len(tiles)} of {n_tiles} query tiles (evenly spaced, the last included) x KV heads "
+                    f"{list(heads)} of {w.num_kv_heads}; oracle_s_full_config extrapolates per tile, and later "
+                    f"tiles cost more",
+                    w.num_kv_heads * n_tiles / (len(heads) * len(tiles)))
+
+
+def even_pairs(w, n):
+    allp = [(b, h) for b in range(w.batch) for h in range(w.num_kv_heads)]
+    if n >= len(allp):
+        return allp
+    step = len(allp) / n
+    return [allp[int(i * step)] for i in range(n)]
+
+
 def cpu_pairs(w, inp, n):
     G = w.group
     out = []
@@ -450,6 +560,11 @@ def run_ours(args, w, rank, world, local_rank):
     if sa.read_status(ws, stream) != sa.SA_OK:
         raise RuntimeError("device status word set during the timed steps")
     ms = reduce_max(sum(step_ms) / len(step_ms), world, dev)
+    parity = None
+    if rank == 0 and not args.no_parity:
+        torch.cuda.synchronize()
+        parity = decode_parity(w, inp, O, idx, even_pairs(w, w.batch * w.num_kv_heads),
+                               w.batch * w.num_kv_heads)
     # --- the attention kernel alone, rank-local ----------------------------
     attn_ms = statistics.mean(timed_steps(attn_only, max(50, args.steps // 4), 3, stream, flush))
     pool_ms = statistics.mean(timed_steps(pool_only, 10, 2, stream, flush))
@@ -473,6 +588,11 @@ def run_ours(args, w, rank, world, local_rank):
     configs = None
     if not args.no_configs:
         configs = run_decode_configs(args, dev, stream, flush)
+    # --- LSA flat bucket retrieval, rank-local -----------------------------------
+    buckets = None
+    if not args.no_buckets:
+        buckets = run_bucket_bench(args, dev, stream, flush)
+        torch.cuda.empty_cache()
     # --- end to end through the C ABI with host buffers -------------------
     e2e = e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush)
     e2e["ms"] = reduce_max(e2e["ms"], world, dev)
@@ -520,6 +640,8 @@ def run_ours(args, w, rank, world, local_rank):
         "column": column,
         "overlap": overlap,
         "decode_configs": configs,
+        "buckets": buckets,
+        "parity": parity,
         "gpu_launches": sa.decode_launches(p) * args.steps,
         "clocks": clk.summary(),
     }
@@ -658,6 +780,12 @@ def run_prefill_bench(args, dev, stream, flush):
         raise RuntimeError("device status word set during the prefill runs")
     rep = prefill_report(w, full_l, score_l, attn_l, peaks())
     rep["clocks"] = clk.summary()
+    if not args.no_parity:
+        full()                     # the table and output of the full call
+        torch.cuda.synchronize()
+        nt = (T + 63) // 64
+        tiles = sorted(set([int(i * (nt - 1) / 15) for i in range(16)] + [nt - 1]))
+        rep["parity"] = prefill_parity(w, Q, K, V, O, idx, [0, w.num_kv_heads - 1], tiles)
     return rep
 
 
@@ -776,6 +904,8 @@ def run_decode_configs(args, dev, stream, flush):
     out = {"peak_gbs": hbm, "peak_source": src}
     for name, seed in (("tiny_decode", 6001), ("draft_chunk_16k", 6002), ("decode_1m", 6003)):
         w = WORKLOADS[name]
+        if args.small and name != "tiny_decode":
+            w = w.scaled(batch=max(1, w.batch // 8), ctx_len=min(w.ctx_len, 262144))
         inp = make_inputs(w, seed=seed, device=dev)
         Q, K, V = inp["Q"], inp["K"], inp["V"]
         del inp
@@ -798,6 +928,12 @@ def run_decode_configs(args, dev, stream, flush):
         ms = statistics.median(timed_steps(step, args.config_steps, 5, stream, flush))
         if sa.read_status(ws, stream) != sa.SA_OK:
             raise RuntimeError(f"device status word set during the {name} runs")
+        parity = None
+        if not args.no_parity:
+            torch.cuda.synchronize()
+            n_all = w.batch * w.num_kv_heads
+            n_chk = n_all if name != "decode_1m" else 4
+            parity = decode_parity(w, {"Q": Q, "K": K, "V": V}, O, idx, even_pairs(w, n_chk), n_all)
         by = decode_bytes(w)
         el = 2 if w.dtype == "bf16" else 4
         pool_b = w.batch * w.num_kv_heads * (nb * w.block_size * w.head_dim * el + nb * w.head_dim * 4)
@@ -811,6 +947,7 @@ def run_decode_configs(args, dev, stream, flush):
             "gbs": by["step"] / (ms * 1e-3) / 1e9, "frac": by["step"] / (ms * 1e-3) / 1e9 / hbm,
             "pool": {"ms": pool_ms, "gbs": pool_b / (pool_ms * 1e-3) / 1e9,
                      "note": "one-time compression of the whole context (each key read once)"},
+            "parity": parity,
         }
         del Q, K, V, Kc, O, lse, idx, ws
         torch.cuda.empty_cache()
@@ -886,6 +1023,81 @@ def run_overlap_bench(args, dev, stream, flush):
     }
 
 
+def run_bucket_bench(args, dev, stream, flush):
+    """Times LSA flat bucket retrieval on the 1M-token workload: the bucket
+    cache build of all 2048 cluster blocks of every (sequence, KV head) pair
+    (one-time, then per new cluster block), and one decode step
+    (sa_bucket_decode: centroid scores, top-256 buckets, expansion to the
+    2048 long-range keys of best own cosine, attention)."""
+    from top_block_sparse_b200 import sa
+    w = WORKLOADS["decode_1m_buckets"]
+    if args.small:
+        w = w.scaled(batch=1, ctx_len=262144)
+    bucket_keys = 2048
+    inp = make_inputs(w, seed=8001, device=dev)
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    del inp
+    p = sa.params_for(w, out_dtype="bf16")
+    R = sa.bucket_rows(p)
+    mcap = 16 // w.pool_stride
+    cents = torch.empty((w.batch, w.num_kv_heads, R, 128), device=dev)
+    members = torch.empty((w.batch, w.num_kv_heads, R, mcap), device=dev, dtype=torch.int32)
+    kcap = bucket_keys // w.pool_stride
+    O = torch.empty((w.batch, w.n_q, w.num_q_heads, 128), device=dev, dtype=torch.bfloat16)
+    lse = torch.empty((w.batch, w.n_q, w.num_q_heads), device=dev)
+    sel = torch.empty((w.batch, w.num_kv_heads, w.top_k), device=dev, dtype=torch.int32)
+    kept = torch.empty((w.batch, w.num_kv_heads, kcap), device=dev, dtype=torch.int32)
+    ws = sa.alloc_workspace(p, sa.SA_OP_BUCKET_DECODE, device=dev)
+
+    def build():
+        sa.bucket_build(p, K, cents, members, stream=stream)
+
+    def step():
+        sa.bucket_decode(p, Q, K, V, cents, members, O, lse, sel, kept, bucket_keys, ws, stream=stream)
+
+    build_ms = statistics.median(timed_steps(build, 3, 1, stream, flush))
+    ms_l = timed_steps(step, args.bucket_steps, 3, stream, flush)
+    ms = statistics.mean(ms_l)
+    if sa.read_status(ws, stream) != sa.SA_OK:
+        raise RuntimeError("device status word set during the bucket runs")
+    hbm, _, _, src = peaks()
+    pairs = w.batch * w.num_kv_heads
+    nblk = w.ctx_len // w.block_size
+    n_bkt = nblk * (w.block_size // 8)
+    n_kept = int((kept >= 0).sum().item())
+    s_end = min(w.sink_keys, w.ctx_len)
+    w_keys = min(w.window_keys, w.ctx_len - s_end)
+    attn_keys = pairs * (s_end + w_keys + w.n_q) + n_kept * w.pool_stride
+    by = {"centroids": pairs * n_bkt * 128 * 4,
+          "members_of_selected": pairs * w.top_k * mcap * 4,
+          "own_cosine_keys": pairs * w.top_k * mcap * w.pool_stride * 128 * 2,
+          "attention_kv": attn_keys * 128 * 2 * 2,
+          "q_o": 2 * w.batch * w.n_q * w.num_q_heads * 128 * 2}
+    step_b = sum(by.values())
+    build_b = pairs * nblk * w.block_size * 128 * 2 + pairs * n_bkt * (128 * 4 + mcap * 4)
+    gbs = lambda b, t: b / (t * 1e-3) / 1e9
+    return {
+        "workload": f"decode_1m_buckets: B={w.batch}, Hq={w.num_q_heads}, Hkv={w.num_kv_heads}, C={w.ctx_len}, "
+                    f"d=128, bf16, LSA pool keys of {w.pool_stride} keys, {w.block_size // 8} Ward buckets per "
+                    f"{w.block_size}-key cluster block ({n_bkt} per pair), top-{w.top_k} buckets by centroid "
+                    f"cosine, {bucket_keys} long-range keys by own cosine, sink {w.sink_keys}, window "
+                    f"{w.window_keys}",
+        "ms": ms, "ms_spread": spread(ms_l),
+        "queries_per_s": w.batch * w.n_q / (ms * 1e-3),
+        "launches": 5,
+        "algorithmic_bytes": step_b, "bytes": by,
+        "achieved_gbs": gbs(step_b, ms), "frac": gbs(step_b, ms) / hbm,
+        "kept_pool_keys_per_pair": n_kept / pairs,
+        "build": {"kernel": "ward_kernel (pool keys, Ward rounds, centroids, one CTA per cluster block)",
+                  "ms": build_ms, "blocks": pairs * nblk, "us_per_block_per_sm":
+                      build_ms * 1e3 * torch.cuda.get_device_properties(dev).multi_processor_count / (pairs * nblk),
+                  "hbm_bytes": build_b, "gbs": gbs(build_b, build_ms),
+                  "note": "one-time per context (then per new cluster block): reads every key once, writes "
+                          "the centroids and member lists"},
+        "peak_gbs": hbm, "peak_source": src,
+    }
+
+
 def e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush):
     """One decode step as a serving loop runs it: the new tokens' Q, K and V
     arrive packed in one pinned host buffer, one copy takes them to the
@@ -938,15 +1150,26 @@ def main():
     ap.add_argument("--config-steps", type=int, default=30)
     ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--no-overlap", action="store_true")
+    ap.add_argument("--no-buckets", action="store_true")
+    ap.add_argument("--no-parity", action="store_true",
+                    help="skip the per-config comparison of the timed results with the float64 oracle")
+    ap.add_argument("--bucket-steps", type=int, default=20)
     ap.add_argument("--column-tokens", type=int, default=None,
                     help="override the column workload's sequence length (smaller cases for ncu captures)")
     ap.add_argument("--prefill-tokens", type=int, default=None,
                     help="override the prefill length (smaller cases for ncu captures)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for ncu captures)")
+    ap.add_argument("--small", action="store_true",
+                    help="every leg at a reduced size (a few GB on the device, inputs still larger than L2), "
+                         "for ncu captures of single kernels; its numbers are not the benchmark's")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.small:
+        args.batch = args.batch or 16
+        args.prefill_tokens = args.prefill_tokens or 16384
+        args.column_tokens = args.column_tokens or 16384
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

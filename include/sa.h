@@ -90,7 +90,8 @@ enum {                                            /* ops for sa_workspace_size *
   SA_OP_DECODE = 2,
   SA_OP_PREFILL = 3,
   SA_OP_VERIFY = 4,
-  SA_OP_COLUMN = 5
+  SA_OP_COLUMN = 5,
+  SA_OP_BUCKET_DECODE = 6
 };
 
 /* Problem description shared by every entry point (96 bytes). */
@@ -282,6 +283,60 @@ sa_status sa_sparse_attn_prefill(const sa_params* p, const void* Q,
                                  const void* K, const void* V, float* Kc,
                                  void* O, float* lse, int32_t* idx_out,
                                  void* ws, size_t ws_bytes, void* stream);
+
+/* LSA flat bucket retrieval, building the bucket cache (LSA review
+ * "精读:LSA", §2.2 "语义聚类:流式 Ward 装桶").  Needs pool == SA_POOL_LSA,
+ * pool_stride (raw keys per pool key) 1, 2 or 4, and block_size = b raw keys
+ * per cluster block with b / pool_stride <= 128.  For every (sequence, KV
+ * head) and every complete cluster block c in [first_block, ctx_len / b):
+ * each raw key is L2-normalised (a zero key stays zero), pool_stride
+ * consecutive unit keys are summed into a pool key, and the block's
+ * b / pool_stride pool keys are clustered bottom-up by Ward's criterion (the
+ * rise n_a n_b / (n_a + n_b) |mean_a - mean_b|^2 of the within-bucket sum of
+ * squares): all start as singletons; every round each bucket takes the
+ * cheapest partner it may join without passing 16 raw keys (lower index on
+ * equal cost), and all pairs that chose each other merge, unless that would
+ * leave fewer than b / 8 buckets, in which case only the cheapest such pairs
+ * merge (cost, then lower index); rounds repeat until b / 8 buckets remain.
+ * Buckets are ordered by their lowest pool key.  Blocks before first_block
+ * are left as they are (a cluster block's buckets never change once built,
+ * so a decode loop calls this with first_block = the blocks built so far).
+ * Writes, per pair, rows [c * b / 8, (c + 1) * b / 8) of
+ *   centroids [B, Hkv, R, d] fp32: the normalised sum of the bucket's pool keys;
+ *   members   [B, Hkv, R, 16 / pool_stride] int32: the bucket's global pool-key
+ *             ids ascending (pool key i = raw keys [i * pool_stride, (i + 1) *
+ *             pool_stride)), -1 padded;
+ * with R = floor(kv_capacity / b) * b / 8 rows per pair (room for every
+ * cluster block the cache can hold).  Reads K only; no workspace.  One launch,
+ * one CTA per (pair, cluster block). */
+sa_status sa_bucket_build(const sa_params* p, const void* K, int64_t first_block,
+                          float* centroids, int32_t* members, void* stream);
+
+/* LSA flat bucket retrieval, a decode / draft-chunk step (LSA review §2.3
+ * "检索:flat 打分与 tree 下降"; S3R review "稀疏起草" for the chunk), on the
+ * bucket cache sa_bucket_build wrote for the ctx_len / b complete cluster
+ * blocks.  The index query of (sequence, KV head) is the sum of its query
+ * heads of the chunk's FIRST token, normalised; it scores every bucket's
+ * centroid (cosine).  A bucket is a candidate if one of its raw keys lies
+ * outside sink [0, S) and window [C - W, C); the top_k candidates by score
+ * (lower bucket first on ties) are selected.  Their member pool keys are
+ * expanded: with bucket_keys = N > 0 (a multiple of pool_stride) only the
+ * N / pool_stride members of best own cosine with the index query are kept
+ * (lower position first on ties), with 0 every member is kept.  Every token j
+ * of the chunk then attends sink U window U the kept pool keys' raw keys U
+ * chunk keys C..C+j (a key counted once), softmax scale as in decode.
+ * Writes O [B, n_q, Hq, d], lse (optional) [B, n_q, Hq], sel_out (optional)
+ * [B, Hkv, top_k] selected buckets ascending, -1 padded, kept_out (optional)
+ * [B, Hkv, K'] kept pool keys ascending, -1 padded, K' = min(N / pool_stride,
+ * top_k * 16 / pool_stride) if N > 0, else top_k * 16 / pool_stride.
+ * top_k * 16 / pool_stride <= 4096.  Workspace: sa_workspace_size(p,
+ * SA_OP_BUCKET_DECODE) (enough for any bucket_keys), zero-filled once.
+ * Kernels: centroid scores, top-k, (own cosines,) expansion, attention. */
+sa_status sa_bucket_decode(const sa_params* p, const void* Q, const void* K,
+                           const void* V, const float* centroids,
+                           const int32_t* members, int32_t bucket_keys, void* O,
+                           float* lse, int32_t* sel_out, int32_t* kept_out,
+                           void* ws, size_t ws_bytes, void* stream);
 
 /* Allocation-free variant of sa_sparse_attn_given_idx (the paper has no
  * counterpart; it exists for callers that cannot allocate device memory,

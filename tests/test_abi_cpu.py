@@ -237,3 +237,50 @@ def test_noalloc_refuses_prefill_tables():
     assert st == sa.SA_ERR_UNSUPPORTED
     msg = sa.raw_call("sa_last_error").decode()
     assert "SA_SEL_QUERY0" in msg and "sa_sparse_attn_given_idx" in msg
+
+
+def _pb(**kw):
+    base = dict(batch=2, num_q_heads=8, num_kv_heads=2, ctx_len=512 * 6 + 5, n_q=1, block_size=512, top_k=16,
+                sink_keys=4, window_keys=512, dtype="bf16", pool="lsa", pool_stride=4)
+    base.update(kw)
+    return sa.make_params(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(pool="mean"), sa.SA_ERR_INVALID),               # buckets are built on LSA pool keys
+    (dict(pool_stride=8, block_size=512), sa.SA_ERR_UNSUPPORTED),    # pool keys of 1, 2 or 4 raw keys
+    (dict(block_size=1024), sa.SA_ERR_UNSUPPORTED),       # 256 pool keys per cluster block > 128
+    (dict(top_k=2048), sa.SA_ERR_UNSUPPORTED),            # 2048 x 4 members > 4096 expansion entries
+])
+def test_bucket_validation_rejects(kw, status):
+    """Host-side checks of the bucket entry points run before any pointer is
+    used (NULL pointers here) and agree with the workspace size query."""
+    p = _pb(**kw)
+    st_b = sa.raw_call("sa_bucket_build", ctypes.byref(p), None, 0, None, None, None)
+    st_d = sa.raw_call("sa_bucket_decode", ctypes.byref(p), None, None, None, None, None, 0, None, None, None,
+                       None, None, 0, None)
+    assert st_b == status
+    assert st_d == status
+    assert sa.raw_call("sa_workspace_size", ctypes.byref(p), sa.SA_OP_BUCKET_DECODE) == 0
+
+
+def test_bucket_arguments_and_workspace():
+    p = _pb()
+    # first_block past the complete cluster blocks; NULL buffers with blocks to build
+    assert sa.raw_call("sa_bucket_build", ctypes.byref(p), None, 7, None, None, None) == sa.SA_ERR_INVALID
+    assert sa.raw_call("sa_bucket_build", ctypes.byref(p), None, 0, None, None, None) == sa.SA_ERR_INVALID
+    # nothing left to build: no launch, no pointer needed
+    assert sa.raw_call("sa_bucket_build", ctypes.byref(p), None, 6, None, None, None) == sa.SA_OK
+    # bucket_keys must be a multiple of the pool stride
+    st = sa.raw_call("sa_bucket_decode", ctypes.byref(p), None, None, None, None, None, 6, None, None, None,
+                     None, None, 0, None)
+    assert st == sa.SA_ERR_INVALID and "bucket_keys" in sa.raw_call("sa_last_error").decode()
+    a = sa.workspace_size(p, sa.SA_OP_BUCKET_DECODE)
+    b = sa.workspace_size(_pb(top_k=64), sa.SA_OP_BUCKET_DECODE)
+    c = sa.workspace_size(_pb(ctx_len=512 * 60), sa.SA_OP_BUCKET_DECODE)
+    assert 0 < a < b and a < c
+    # the scores of every bucket of the context: 64 per cluster block, 4 bytes each
+    assert c - a >= 2 * 2 * 54 * 64 * 4
+    assert sa.bucket_rows(p) == ((512 * 6 + 6) // 512) * 64
+    # 5 tokens x GQA 4 = 20 query rows per KV head: the attention is not built
+    assert sa.workspace_size(_pb(n_q=5), sa.SA_OP_BUCKET_DECODE) == 0

@@ -80,3 +80,33 @@ def test_step_spread():
     sp = bench.spread([3.0, 1.0, 2.0, 10.0, 4.0, 5.0, 6.0, 7.0, 8.0, 9.0])
     assert sp["min"] == 1.0 and sp["max"] == 10.0 and sp["median"] == 5.5
     assert sp["p90"] == 9.0 and sp["n"] == 10 and abs(sp["mean"] - 5.5) < 1e-12
+
+
+def test_parity_tally_counts_and_errors():
+    """The benchmark's per-config parity record: sets counted as matching,
+    near-tie or mismatching; errors only over matching pairs; a bf16 output's
+    format rounding reported apart from the plain max abs."""
+    import numpy as np
+    import torch
+    from oracle.sparse_attn_oracle import Selection
+
+    t = bench.ParityTally()
+    sel = Selection([1, 4], 10, 0.5, 0.2, False)
+    tie = Selection([1, 5], 10, 0.5, 1e-9, True)
+    assert t.sets([1, 4], sel) and not t.sets([1, 6], tie) and not t.sets([2, 4], sel)
+    ref = np.array([[1.0, -2.0], [0.5, 0.25]])
+    t.out(torch.tensor(ref + 1e-3, dtype=torch.float32), ref)
+    r = t.report("test", 4.0)
+    assert (r["checked"], r["sets_match"], r["near_ties"], r["mismatches"]) == (3, 1, 1, 1)
+    assert abs(r["max_abs"] - 1e-3) < 1e-7 and abs(r["max_abs_beyond_bf16_rounding"] - 1e-3) < 1e-7
+    assert abs(r["rel_l2"] - 2e-3 / np.sqrt((ref ** 2).sum())) < 1e-7
+    t2 = bench.ParityTally()
+    t2.out(torch.tensor(ref, dtype=torch.bfloat16), ref + 4e-4)    # within half a bf16 step (>= 2^-10 here)
+    assert t2.max_abs > 0 and t2.max_abs_fmt == 0.0
+
+
+def test_even_pairs_sampling():
+    w = WORKLOADS["decode_1m"]
+    ps = bench.even_pairs(w, 4)
+    assert len(ps) == 4 and ps[0] == (0, 0) and len(set(ps)) == 4
+    assert bench.even_pairs(w, 100) == [(b, h) for b in range(4) for h in range(8)]

@@ -23,7 +23,7 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libsa.so")
 INCLUDE = os.path.join(ROOT, "include")
 
-SOURCES = ["sa_api.cu", "pool.cu", "score_topk.cu", "decode_attn.cu", "decode_tc.cu", "prefill_score.cu", "prefill_attn.cu", "verify.cu"]
+SOURCES = ["sa_api.cu", "pool.cu", "score_topk.cu", "decode_attn.cu", "decode_tc.cu", "prefill_score.cu", "prefill_attn.cu", "verify.cu", "bucket.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

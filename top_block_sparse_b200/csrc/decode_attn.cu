@@ -120,6 +120,25 @@ __device__ __forceinline__ void qk_two_keys(const unsigned char* krow_a, const u
   }
 }
 
+// Run mode: entry e of gathered tile `sl` of `pair` (rpt entries per tile).
+// Returns the number of keys of its run inside [s_end, w_begin) and their
+// first key in *start (0 keys for -1 entries and entries past the row).
+__device__ __forceinline__ int run_entry(const DecodeAttnArgs& a, int64_t pair, int sl, int e, int rpt,
+                                         int64_t* start) {
+  const int64_t at = static_cast<int64_t>(sl) * rpt + e;
+  const int32_t m = (e < rpt && at < a.runs_stride) ? __ldg(a.runs + pair * a.runs_stride + at) : -1;
+  *start = 0;
+  if (m < 0) return 0;
+  const int64_t lo = max(static_cast<int64_t>(m) * a.run_len, a.s_end);
+  const int64_t hi = min(static_cast<int64_t>(m) * a.run_len + a.run_len, a.w_begin);
+  *start = lo;
+  return hi > lo ? static_cast<int>(hi - lo) : 0;
+}
+
+// Key position given to gathered tiles: below every context key, so the
+// causal rule of the new tokens never applies to them.
+constexpr int64_t kRunTilePos = -(int64_t(1) << 40);
+
 template <bool BF16, bool OUT_BF16, int RG, int KG>
 __global__ void __launch_bounds__((RG * KG + 1) * 32, 1) decode_attn_kernel(DecodeAttnArgs a) {
   constexpr int NWC = RG * KG;                 // consumer warps
@@ -188,26 +207,49 @@ __global__ void __launch_bounds__((RG * KG + 1) * 32, 1) decode_attn_kernel(Deco
         const int n1 = __shfl_sync(0xffffffffu, nk1, l);
         const int i = base + l;
         const int s = i % NS;
+        const int64_t pair = (u0 + i) / a.MT;
+        unsigned char* st = stages + static_cast<size_t>(s) * STAGE;
+        const unsigned char* kb = static_cast<const unsigned char*>(a.K) + pair * a.cap * ROWB;
+        const unsigned char* vb = static_cast<const unsigned char*>(a.V) + pair * a.cap * ROWB;
+        // run mode: tiles of the selected section are packed from key runs
+        // by the whole warp (their sizes first, the copies after the barrier
+        // expects their bytes)
+        bool gat[2] = {false, false};
+        int sl[2] = {0, 0};
+        int tot[2] = {n0, n1};
+        const int rpt = a.runs ? HALF / a.run_len : 0;
+        if (a.runs) {
+          const int v = static_cast<int>((u0 + i) - pair * a.MT);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            sl[h] = 2 * v + h - a.n_sink_tiles;
+            gat[h] = (2 * v + h < a.n_tiles) && sl[h] >= 0 && sl[h] < a.idx_stride;
+            if (!gat[h]) continue;
+            int t = 0;
+            for (int c0 = 0; c0 < rpt; c0 += 32) {
+              int64_t st0;
+              const int len = run_entry(a, pair, sl[h], c0 + lane, rpt, &st0);
+              t += __reduce_add_sync(0xffffffffu, static_cast<unsigned>(len));
+            }
+            tot[h] = t;
+          }
+        }
         int ok = 1;
         if (lane == 0) {
           if (i >= NS && !mbar_wait_bounded(&empty[s], ((i / NS) & 1) ^ 1, abort_flag)) ok = 0;
           if (ok && *abort_flag) ok = 0;
           if (ok) {
-            info[s].ks0 = k0;
-            info[s].ks1 = k1;
-            info[s].n0 = n0;
-            info[s].n1 = n1;
-            if (n0 + n1 > 0) {
-              const int64_t pair = (u0 + i) / a.MT;
-              mbar_arrive_expect_tx(&full[s], 2u * static_cast<uint32_t>(n0 + n1) * ROWB);
-              unsigned char* st = stages + static_cast<size_t>(s) * STAGE;
-              const unsigned char* kb = static_cast<const unsigned char*>(a.K) + pair * a.cap * ROWB;
-              const unsigned char* vb = static_cast<const unsigned char*>(a.V) + pair * a.cap * ROWB;
-              if (n0 > 0) {
+            info[s].ks0 = gat[0] ? kRunTilePos : k0;
+            info[s].ks1 = gat[1] ? kRunTilePos : k1;
+            info[s].n0 = tot[0];
+            info[s].n1 = tot[1];
+            if (tot[0] + tot[1] > 0) {
+              mbar_arrive_expect_tx(&full[s], 2u * static_cast<uint32_t>(tot[0] + tot[1]) * ROWB);
+              if (!gat[0] && n0 > 0) {
                 bulk_g2s(st, kb + k0 * ROWB, n0 * ROWB, &full[s]);
                 bulk_g2s(st + KBYTES, vb + k0 * ROWB, n0 * ROWB, &full[s]);
               }
-              if (n1 > 0) {
+              if (!gat[1] && n1 > 0) {
                 bulk_g2s(st + HALF * ROWB, kb + k1 * ROWB, n1 * ROWB, &full[s]);
                 bulk_g2s(st + KBYTES + HALF * ROWB, vb + k1 * ROWB, n1 * ROWB, &full[s]);
               }
@@ -223,6 +265,32 @@ __global__ void __launch_bounds__((RG * KG + 1) * 32, 1) decode_attn_kernel(Deco
         if (!ok) {
           stop = true;
           break;
+        }
+        __syncwarp();
+        if (gat[0] || gat[1]) {
+          // each lane copies its runs' K and V rows to the packed positions
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (!gat[h]) continue;
+            int carry = 0;
+            for (int c0 = 0; c0 < rpt; c0 += 32) {
+              int64_t ks;
+              const int len = run_entry(a, pair, sl[h], c0 + lane, rpt, &ks);
+              int incl = len;
+#pragma unroll
+              for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += y;
+              }
+              const int off = carry + incl - len;
+              if (len > 0) {
+                const uint32_t by = static_cast<uint32_t>(len) * ROWB;
+                bulk_g2s(st + (h * HALF + off) * ROWB, kb + ks * ROWB, by, &full[s]);
+                bulk_g2s(st + KBYTES + (h * HALF + off) * ROWB, vb + ks * ROWB, by, &full[s]);
+              }
+              carry += __shfl_sync(0xffffffffu, incl, 31);
+            }
+          }
         }
         issued = i + 1;
       }

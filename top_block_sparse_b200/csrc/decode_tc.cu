@@ -1035,7 +1035,7 @@ TcOrder tc_order(int64_t pairs, int n_sink_tiles, int n_sel_tiles, int n_wc_tile
 }
 
 bool decode_tc_supported(const DecodeAttnArgs& a) {
-  return a.R >= 1 && a.R <= kN && a.kv_end < (int64_t(1) << 31) &&
+  return a.runs == nullptr && a.R >= 1 && a.R <= kN && a.kv_end < (int64_t(1) << 31) &&
          static_cast<int64_t>(a.B) * a.n_q < (int64_t(1) << 31) && encode_fn() != nullptr;
 }
 

@@ -136,6 +136,15 @@ struct DecodeAttnArgs {
   float2* mass_part;      // [pairs, mass_hts, 16], or null
   int64_t mass_keys;      // keys of the complete blocks, nb * b
   int mass_hts;           // mass_keys / 32
+  // run mode (CUDA-core kernel only): the selected section is a list of
+  // key runs instead of blocks.  Entry e of a pair's row names the run of
+  // keys [e_id * run_len, e_id * run_len + run_len), clipped to [s_end,
+  // w_begin); -1 entries are empty.  Tile t of the section packs the runs of
+  // entries [t * tile / run_len, (t + 1) * tile / run_len) back to back
+  // (idx_stride = tiles of the section, tpb = 1).
+  const int32_t* runs;    // [pairs, runs_stride], or null
+  int runs_stride;
+  int run_len;
 };
 
 struct DecodePlan {
@@ -166,6 +175,55 @@ cudaError_t launch_decode_fused(DecodeAttnArgs a, const DecodePlan& p, bool out_
 // that are in [0, nb) and above every earlier in-range entry of the row.
 cudaError_t launch_sanitize_idx(const int32_t* idx, int32_t* out, int rows, int len, int64_t nb,
                                 unsigned* status, cudaStream_t s);
+
+// ---- LSA flat bucket retrieval (bucket.cu) ----------------------------------
+// Bucket cache of a pair: rows_per_pair rows, nbk per cluster block of b raw
+// keys (block c's buckets are rows [c * nbk, (c + 1) * nbk)), ordered by their
+// lowest member; centroids [rows, 128] fp32 unit vectors, members [rows,
+// mcap] int32 global pool-key ids (pool key i = raw keys [i * stride, (i + 1)
+// * stride)), ascending, -1 padded.
+struct WardArgs {
+  const void* K;          // [pairs, cap, 128]
+  float* cents;
+  int32_t* members;
+  int64_t cap;            // token stride of K
+  int64_t rows_per_pair;
+  int64_t first_block;    // cluster blocks [first_block, first_block + gridDim.x) are built
+  int b, stride, m, nbk, mcap;   // raw keys per block, per pool key; pool keys per block; buckets; cap
+};
+cudaError_t launch_ward(const WardArgs& a, int pairs, int64_t n_blocks, bool bf16, cudaStream_t s);
+size_t ward_smem_bytes();
+
+struct BucketScoreArgs {
+  const void* Q;
+  const float* cents;
+  const int32_t* members;
+  uint32_t* keys;         // [pairs, n_bkt] order-preserving cosine keys, 0 = not a candidate
+  int Hq, Hkv, G, n_q;
+  int64_t rows_per_pair;
+  int64_t n_bkt;          // buckets of the context's complete cluster blocks
+  int nbk, b, stride, mcap;
+  int64_t s_end, w_begin;
+  int64_t rows_per_cta;
+};
+struct BucketExpandArgs {
+  const void* Q;
+  const void* K;
+  const int32_t* members;
+  int32_t* sel;           // [pairs, top_k] selected buckets, ascending, -1 padded
+  unsigned long long* own;  // [pairs, top_k * mcap] expansion keys (workspace)
+  int32_t* kept;          // [pairs, kept_cap] kept pool keys, ascending, -1 padded
+  int Hq, Hkv, G, n_q;
+  int64_t cap, rows_per_pair;
+  int top_k, mcap, stride;
+  int keep_pool;          // pool keys kept (0: every member of the selected buckets)
+  int kept_cap;
+};
+// Scores of every bucket and the top-k selection into ea.sel.
+cudaError_t launch_bucket_select(const BucketScoreArgs& sa_, const BucketExpandArgs& ea, int pairs, bool bf16,
+                                 cudaStream_t s);
+// Expansion of the selected buckets into ea.kept.
+cudaError_t launch_bucket_expand(const BucketExpandArgs& a, int pairs, bool bf16, cudaStream_t s);
 
 // ---- dense verify: block attention mass and the refreshed selection --------
 // mass[pair][j] = sum over j's half-tiles h and rows r < R of

@@ -337,6 +337,92 @@ PrefillArgs prefill_args(const sa_params* p, const PrefillGeom& g) {
   return a;
 }
 
+// ---- LSA flat bucket retrieval ------------------------------------------------
+struct BucketGeom {
+  int stride, m, nbk, mcap;
+  int64_t nblk;            // complete cluster blocks of the context
+  int64_t rows_per_pair;   // bucket rows per pair: every cluster block the cache can hold
+  int64_t n_bkt;           // buckets of the context's complete cluster blocks
+};
+
+sa_status check_bucket(const sa_params* p, BucketGeom* g) {
+  sa_status st = check_params(p, false);
+  if (st != SA_OK) return st;
+  if (p->pool != SA_POOL_LSA) return fail(SA_ERR_INVALID, "bucket retrieval needs pool = SA_POOL_LSA");
+  if (p->pool_stride != 1 && p->pool_stride != 2 && p->pool_stride != 4)
+    return fail(SA_ERR_UNSUPPORTED, "pool_stride %d: bucket retrieval is built for pool keys of 1, 2 or 4 raw keys",
+                p->pool_stride);
+  g->stride = p->pool_stride;
+  g->m = p->block_size / p->pool_stride;
+  if (g->m > 128)
+    return fail(SA_ERR_UNSUPPORTED, "a cluster block holds at most 128 pool keys (block_size / pool_stride = %d)",
+                g->m);
+  g->nbk = p->block_size / 8;
+  g->mcap = 16 / p->pool_stride;
+  g->nblk = p->ctx_len / p->block_size;
+  g->rows_per_pair = (p->kv_capacity / p->block_size) * g->nbk;
+  g->n_bkt = g->nblk * g->nbk;
+  if (p->kv_capacity / p->pool_stride >= (int64_t(1) << 31))
+    return fail(SA_ERR_UNSUPPORTED, "pool-key ids of a %lld-row cache do not fit 32 bits", (long long)p->kv_capacity);
+  if (g->rows_per_pair > (int64_t(1) << 26))
+    return fail(SA_ERR_UNSUPPORTED, "%lld buckets per sequence exceed the 2^26 built", (long long)g->rows_per_pair);
+  if (static_cast<int64_t>(p->top_k) * g->mcap > 4096)
+    return fail(SA_ERR_UNSUPPORTED, "top_k x %d members = %d entries exceed the 4096 the expansion sorts", g->mcap,
+                p->top_k * g->mcap);
+  if (static_cast<int64_t>(p->batch) * p->num_kv_heads > 65535)
+    return fail(SA_ERR_UNSUPPORTED, "more than 65535 (sequence, KV head) pairs");
+  return SA_OK;
+}
+
+struct BucketWs {
+  DecodeWs attn;
+  size_t keys, sel, own, kept, total;
+};
+
+// Attention plan of the run mode: the selected section holds kept_cap runs,
+// tile / stride of them per tile.
+sa_status bucket_plan(const sa_params* p, const BucketGeom& bg, int kept_cap, DecodeGeom* g, DecodePlan* plan) {
+  *g = decode_geom(p);
+  const int T = p->dtype == SA_BF16 ? 64 : 32;
+  g->b = T;
+  const int rpt = T / bg.stride;
+  const int n_sel = (kept_cap + rpt - 1) / rpt;
+  const char* why = "";
+  if (!plan_decode(*g, n_sel, p->dtype == SA_BF16, device_sms(), plan, &why))
+    return fail(SA_ERR_UNSUPPORTED, "%s", why);
+  return SA_OK;
+}
+
+BucketWs bucket_ws(const sa_params* p, const BucketGeom& bg, const DecodeGeom& g, const DecodePlan& plan) {
+  BucketWs w;
+  w.attn = decode_ws(g, plan, 0, SA_OP_GIVEN_IDX, 0);
+  const size_t pairs = static_cast<size_t>(g.pairs);
+  const size_t n_ent = static_cast<size_t>(p->top_k) * bg.mcap;
+  w.keys = align_up(w.attn.total, 256);
+  w.sel = align_up(w.keys + pairs * static_cast<size_t>(bg.n_bkt) * 4, 256);
+  w.own = align_up(w.sel + pairs * static_cast<size_t>(p->top_k) * 4, 256);
+  w.kept = align_up(w.own + pairs * n_ent * 8, 256);
+  w.total = align_up(w.kept + pairs * n_ent * 4, 256);
+  return w;
+}
+
+// Workspace for any bucket_keys: the largest over the run counts the kept
+// table can have.
+size_t bucket_ws_bytes(const sa_params* p, const BucketGeom& bg) {
+  const int n_ent = p->top_k * bg.mcap;
+  const int rpt = (p->dtype == SA_BF16 ? 64 : 32) / bg.stride;
+  size_t best = 0;
+  for (int kc = 0;; kc += rpt) {
+    const int cap = kc < n_ent ? kc : n_ent;
+    DecodeGeom g;
+    DecodePlan plan;
+    if (bucket_plan(p, bg, cap, &g, &plan) != SA_OK) return 0;
+    best = std::max(best, bucket_ws(p, bg, g, plan).total);
+    if (cap >= n_ent) break;
+  }
+  return best;
+}
+
 }  // namespace
 }  // namespace sa
 
@@ -431,6 +517,11 @@ size_t sa_workspace_size(const sa_params* p, int32_t op) {
     DecodePlan plan;
     if (plan_for(&d, 0, &g, &plan) != SA_OK) return 0;
     return verify_ws(g, plan, decode_geom(p).nb).total;
+  }
+  if (op == SA_OP_BUCKET_DECODE) {
+    BucketGeom bg;
+    if (check_bucket(p, &bg) != SA_OK) return 0;
+    return bucket_ws_bytes(p, bg);
   }
   const bool prefill = (op == SA_OP_PREFILL) || (p && p->select == SA_SEL_TILE_MAX);
   if (check_params(p, prefill) != SA_OK) return 0;
@@ -799,6 +890,130 @@ sa_status sa_read_status(void* ws, void* stream) {
 }
 
 }  // extern "C"
+
+// ---- LSA flat bucket retrieval (LSA review §2.2-2.3) --------------------------
+extern "C" sa_status sa_bucket_build(const sa_params* p, const void* K, int64_t first_block, float* centroids,
+                                     int32_t* members, void* stream) {
+  BucketGeom bg;
+  sa_status st = check_bucket(p, &bg);
+  if (st != SA_OK) return st;
+  if (first_block < 0 || first_block > bg.nblk)
+    return fail(SA_ERR_INVALID, "first_block %lld must be in [0, %lld]", (long long)first_block, (long long)bg.nblk);
+  if (first_block == bg.nblk) return SA_OK;
+  if (!K || !centroids || !members) return fail(SA_ERR_INVALID, "K, centroids and members must be non-NULL");
+  if (!aligned16(K) || !aligned16(centroids) || !aligned16(members))
+    return fail(SA_ERR_INVALID, "K, centroids and members must be 16-byte aligned");
+  WardArgs a = {};
+  a.K = K;
+  a.cents = centroids;
+  a.members = members;
+  a.cap = p->kv_capacity;
+  a.rows_per_pair = bg.rows_per_pair;
+  a.first_block = first_block;
+  a.b = p->block_size;
+  a.stride = bg.stride;
+  a.m = bg.m;
+  a.nbk = bg.nbk;
+  a.mcap = bg.mcap;
+  cudaError_t e = launch_ward(a, p->batch * p->num_kv_heads, bg.nblk - first_block, p->dtype == SA_BF16,
+                              static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "bucket clustering launch");
+  return SA_OK;
+}
+
+extern "C" sa_status sa_bucket_decode(const sa_params* p, const void* Q, const void* K, const void* V,
+                                      const float* centroids, const int32_t* members, int32_t bucket_keys, void* O,
+                                      float* lse, int32_t* sel_out, int32_t* kept_out, void* ws, size_t ws_bytes,
+                                      void* stream) {
+  BucketGeom bg;
+  sa_status st = check_bucket(p, &bg);
+  if (st != SA_OK) return st;
+  if (bucket_keys < 0 || bucket_keys % bg.stride != 0)
+    return fail(SA_ERR_INVALID, "bucket_keys %d must be >= 0 and a multiple of pool_stride %d", bucket_keys,
+                bg.stride);
+  const bool retrieve = p->top_k > 0 && bg.n_bkt > 0;
+  if (!Q || !K || !V || !O || (retrieve && (!centroids || !members)))
+    return fail(SA_ERR_INVALID, "Q, K, V, O (and centroids, members with buckets to score) must be non-NULL");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(centroids) ||
+      !aligned16(members))
+    return fail(SA_ERR_INVALID, "Q, K, V, O, centroids and members must be 16-byte aligned");
+  const int n_ent = p->top_k * bg.mcap;
+  const int keep_pool = bucket_keys / bg.stride;
+  const int kept_cap = keep_pool > 0 ? std::min(keep_pool, n_ent) : n_ent;
+  DecodeGeom g;
+  DecodePlan plan;
+  if ((st = bucket_plan(p, bg, kept_cap, &g, &plan)) != SA_OK) return st;
+  const BucketWs L = bucket_ws(p, bg, g, plan);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != SA_OK) return st;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bf16 = p->dtype == SA_BF16;
+  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w + L.sel);
+  int32_t* kept = kept_out ? kept_out : reinterpret_cast<int32_t*>(w + L.kept);
+  BucketScoreArgs sc = {};
+  sc.Q = Q;
+  sc.cents = centroids;
+  sc.members = members;
+  sc.keys = reinterpret_cast<uint32_t*>(w + L.keys);
+  sc.Hq = p->num_q_heads;
+  sc.Hkv = p->num_kv_heads;
+  sc.G = p->num_q_heads / p->num_kv_heads;
+  sc.n_q = p->n_q;
+  sc.rows_per_pair = bg.rows_per_pair;
+  sc.n_bkt = retrieve ? bg.n_bkt : 0;
+  sc.nbk = bg.nbk;
+  sc.b = p->block_size;
+  sc.stride = bg.stride;
+  sc.mcap = bg.mcap;
+  sc.s_end = g.s_end;
+  sc.w_begin = g.w_begin;
+  sc.rows_per_cta = 2048;
+  BucketExpandArgs ex = {};
+  ex.Q = Q;
+  ex.K = K;
+  ex.members = members;
+  ex.sel = sel;
+  ex.own = reinterpret_cast<unsigned long long*>(w + L.own);
+  ex.kept = kept;
+  ex.Hq = sc.Hq;
+  ex.Hkv = sc.Hkv;
+  ex.G = sc.G;
+  ex.n_q = sc.n_q;
+  ex.cap = p->kv_capacity;
+  ex.rows_per_pair = bg.rows_per_pair;
+  ex.top_k = retrieve ? p->top_k : 0;
+  ex.mcap = bg.mcap;
+  ex.stride = bg.stride;
+  ex.keep_pool = keep_pool;
+  ex.kept_cap = kept_cap;
+  const int pairs = g.pairs;
+  cudaError_t e = cudaSuccess;
+  if (retrieve) {
+    e = launch_bucket_select(sc, ex, pairs, bf16, s);
+    if (e != cudaSuccess) return cuda_fail(e, "bucket scoring launch");
+  } else if (sel_out && p->top_k > 0) {
+    e = cudaMemsetAsync(sel_out, 0xff, static_cast<size_t>(pairs) * p->top_k * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  }
+  if (kept_cap > 0) {
+    if (retrieve) {
+      e = launch_bucket_expand(ex, pairs, bf16, s);
+      if (e != cudaSuccess) return cuda_fail(e, "bucket expansion launch");
+    } else {
+      e = cudaMemsetAsync(kept, 0xff, static_cast<size_t>(pairs) * kept_cap * 4, s);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    }
+  }
+  const int rpt = (bf16 ? 64 : 32) / bg.stride;
+  DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, kept, (kept_cap + rpt - 1) / rpt, O, lse, w, L.attn);
+  a.pdl = 0;
+  a.runs = kept;
+  a.runs_stride = kept_cap;
+  a.run_len = bg.stride;
+  e = launch_decode_attn(a, plan, bf16, p->out_dtype == SA_BF16, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+  return SA_OK;
+}
 
 // ---- allocation-free variant of sa_sparse_attn_given_idx --------------------
 // For callers that cannot call cudaMalloc themselves: code running inside a

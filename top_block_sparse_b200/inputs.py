@@ -74,6 +74,11 @@ WORKLOADS: Dict[str, Workload] = {
     # 16 keys (two windows per half block, neighbours sharing half their keys)
     "decode_32k_overlap": Workload("decode_32k_overlap", 32, 1, 32, 8, 128, 32768, "bf16",
                                    64, "overlap", 32, 64, 256, 16, pool_stride=16, pool_kernel=32),
+    # decode_1m with LSA flat bucket retrieval: 64 Ward buckets per 512-key
+    # cluster block, top-256 buckets by centroid cosine, expanded to the 2048
+    # long-range keys of best own cosine (sa_bucket_decode, bucket_keys 2048)
+    "decode_1m_buckets": Workload("decode_1m_buckets", 4, 1, 32, 8, 128, 1048576, "bf16",
+                                  512, "lsa", 256, 4, 512, 32),
     # batch 64, 6-token draft chunk, 16 / 8 heads, C = 16384
     "draft_chunk_16k": Workload("draft_chunk_16k", 64, 6, 16, 8, 128, 16384,
                                 "bf16", 64, "mean", 16, 64, 256, 8),

@@ -26,12 +26,14 @@ SA_F32, SA_BF16 = 0, 1
 SA_POOL_MEAN, SA_POOL_LSA, SA_POOL_OVERLAP = 0, 1, 2
 SA_SEL_QUERY0, SA_SEL_TILE_MAX = 0, 1
 SA_OP_SCORE_TOPK, SA_OP_GIVEN_IDX, SA_OP_DECODE, SA_OP_PREFILL, SA_OP_VERIFY, SA_OP_COLUMN = 0, 1, 2, 3, 4, 5
+SA_OP_BUCKET_DECODE = 6
 SA_FLAG_TRUSTED_IDX = 1
 
 EXPORTED = ["sa_version", "sa_workspace_size", "sa_workspace_init", "sa_pool_keys", "sa_score_topk",
             "sa_sparse_attn_given_idx", "sa_sparse_attn_decode", "sa_sparse_attn_prefill",
             "sa_read_status", "sa_status_string", "sa_last_error", "sa_sparse_attn_given_idx_noalloc",
-            "sa_decode_launches", "sa_verify_refresh", "sa_column_attn", "sa_append_kv"]
+            "sa_decode_launches", "sa_verify_refresh", "sa_column_attn", "sa_append_kv",
+            "sa_bucket_build", "sa_bucket_decode"]
 
 
 class SaParams(ctypes.Structure):
@@ -70,6 +72,8 @@ _sig = {
     "sa_verify_refresh": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "sa_column_attn": (_i32, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     "sa_append_kv": (_i32, [_P, _vp, _vp, _vp, _vp, _vp]),
+    "sa_bucket_build": (_i32, [_P, _vp, ctypes.c_int64, _vp, _vp, _vp]),
+    "sa_bucket_decode": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -206,6 +210,28 @@ def column_attn(p: SaParams, Q, K, V, cols, O, lse=None, ws=None, stream=None):
     n_cols = 0 if cols is None else int(cols.shape[-1])
     _check(_lib.sa_column_attn(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(cols), n_cols, _ptr(O), _ptr(lse),
                                _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def bucket_rows(p: SaParams) -> int:
+    """Bucket-cache rows per (sequence, KV head): every cluster block the
+    cache can hold, block_size / 8 buckets each."""
+    return (p.kv_capacity // p.block_size) * (p.block_size // 8)
+
+
+def bucket_build(p: SaParams, K, centroids, members, first_block=0, stream=None):
+    """LSA bucket cache of the complete cluster blocks from first_block on
+    (sa_bucket_build): centroids [B, Hkv, R, d] fp32, members [B, Hkv, R,
+    16 // pool_stride] int32, R = bucket_rows(p)."""
+    _check(_lib.sa_bucket_build(ctypes.byref(p), _ptr(K), int(first_block), _ptr(centroids), _ptr(members),
+                                _stream(stream)))
+
+
+def bucket_decode(p: SaParams, Q, K, V, centroids, members, O, lse=None, sel_out=None, kept_out=None,
+                  bucket_keys=0, ws=None, stream=None):
+    """Decode / draft chunk with LSA flat bucket retrieval (sa_bucket_decode)."""
+    _check(_lib.sa_bucket_decode(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(centroids), _ptr(members),
+                                 int(bucket_keys), _ptr(O), _ptr(lse), _ptr(sel_out), _ptr(kept_out), _ptr(ws),
+                                 0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def read_status(ws: torch.Tensor, stream=None) -> int:
