@@ -152,6 +152,21 @@ class ClockSampler:
                 "samples": len(sm), "sample_period_ms": self.PERIOD_MS}
 
 
+class nvtx_range:
+    """An NVTX range around one benchmark leg (ncu --nvtx-include selects a
+    leg's kernels by it)."""
+
+    def __init__(self, name):
+        self.name = name
+
+    def __enter__(self):
+        torch.cuda.nvtx.range_push(self.name)
+
+    def __exit__(self, *exc):
+        torch.cuda.nvtx.range_pop()
+        return False
+
+
 def spread(ms_list):
     """Spread of per-step device times (ms): min, median, 90th percentile,
     max and mean."""
@@ -536,6 +551,7 @@ def run_ours(args, w, rank, world, local_rank):
     flush = L2Flush(dev)
     p_trusted = sa.params_for(w)
     p_trusted.flags = sa.SA_FLAG_TRUSTED_IDX
+    torch.cuda.nvtx.range_push(w.name)
     with torch.cuda.stream(stream):
         sa.pool_keys(p, K, Kc, stream=stream)
     torch.cuda.synchronize()
@@ -568,22 +584,27 @@ def run_ours(args, w, rank, world, local_rank):
     # --- the attention kernel alone, rank-local ----------------------------
     attn_ms = statistics.mean(timed_steps(attn_only, max(50, args.steps // 4), 3, stream, flush))
     pool_ms = statistics.mean(timed_steps(pool_only, 10, 2, stream, flush))
+    torch.cuda.nvtx.range_pop()
     # --- causal prefill (tensor cores), rank-local --------------------------
     prefill = None
     if not args.no_prefill:
-        prefill = run_prefill_bench(args, dev, stream, flush)
+        with nvtx_range("prefill"):
+            prefill = run_prefill_bench(args, dev, stream, flush)
     # --- dense verify of a draft chunk, rank-local ----------------------------
     verify = None
     if not args.no_verify:
-        verify = run_verify_bench(args, dev, stream, flush)
+        with nvtx_range("verify"):
+            verify = run_verify_bench(args, dev, stream, flush)
     # --- column-sparse attention, rank-local ----------------------------------
     column = None
     if not args.no_column:
-        column = run_column_bench(args, dev, stream, flush)
+        with nvtx_range("column"):
+            column = run_column_bench(args, dev, stream, flush)
     # --- decode with overlapping compressed keys, rank-local ------------------
     overlap = None
     if not args.no_overlap:
-        overlap = run_overlap_bench(args, dev, stream, flush)
+        with nvtx_range("overlap"):
+            overlap = run_overlap_bench(args, dev, stream, flush)
     # --- the other decode workloads, rank-local ---------------------------------
     configs = None
     if not args.no_configs:
@@ -591,10 +612,12 @@ def run_ours(args, w, rank, world, local_rank):
     # --- LSA flat bucket retrieval, rank-local -----------------------------------
     buckets = None
     if not args.no_buckets:
-        buckets = run_bucket_bench(args, dev, stream, flush)
+        with nvtx_range("buckets"):
+            buckets = run_bucket_bench(args, dev, stream, flush)
         torch.cuda.empty_cache()
     # --- end to end through the C ABI with host buffers -------------------
-    e2e = e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush)
+    with nvtx_range("e2e"):
+        e2e = e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush)
     e2e["ms"] = reduce_max(e2e["ms"], world, dev)
     if rank != 0:
         return None
@@ -903,6 +926,7 @@ def run_decode_configs(args, dev, stream, flush):
     hbm, _, _, src = peaks()
     out = {"peak_gbs": hbm, "peak_source": src}
     for name, seed in (("tiny_decode", 6001), ("draft_chunk_16k", 6002), ("decode_1m", 6003)):
+        torch.cuda.nvtx.range_push(name)
         w = WORKLOADS[name]
         if args.small and name != "tiny_decode":
             w = w.scaled(batch=max(1, w.batch // 8), ctx_len=min(w.ctx_len, 262144))
@@ -951,6 +975,7 @@ def run_decode_configs(args, dev, stream, flush):
         }
         del Q, K, V, Kc, O, lse, idx, ws
         torch.cuda.empty_cache()
+        torch.cuda.nvtx.range_pop()
     return out
 
 

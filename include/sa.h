@@ -329,7 +329,10 @@ sa_status sa_bucket_build(const sa_params* p, const void* K, int64_t first_block
  * [B, Hkv, top_k] selected buckets ascending, -1 padded, kept_out (optional)
  * [B, Hkv, K'] kept pool keys ascending, -1 padded, K' = min(N / pool_stride,
  * top_k * 16 / pool_stride) if N > 0, else top_k * 16 / pool_stride.
- * top_k * 16 / pool_stride <= 4096.  Workspace: sa_workspace_size(p,
+ * top_k * 16 / pool_stride <= 4096, and ceil(buckets / 8192) * min(top_k,
+ * 8192) <= 28672 (the selection keeps each 8192 buckets' top-k, then the
+ * top-k of those in shared memory; with top_k = 256, contexts up to 7.3M
+ * keys at b = 512).  Workspace: sa_workspace_size(p,
  * SA_OP_BUCKET_DECODE) (enough for any bucket_keys), zero-filled once.
  * Kernels: centroid scores, top-k, (own cosines,) expansion, attention. */
 sa_status sa_bucket_decode(const sa_params* p, const void* Q, const void* K,

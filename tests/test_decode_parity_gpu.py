@@ -378,6 +378,17 @@ def test_full_size_sampled(name):
     torch.cuda.empty_cache()
 
 
+def test_full_size_sampled_fp32_output():
+    """decode_32k at full size in the benchmark's launch configuration (the
+    fused cooperative launch) with fp32 outputs: the sampled pairs meet max
+    abs <= 5e-3 and relative L2 <= 1e-2 on the plain error, with nothing
+    discounted for an output format."""
+    w = WORKLOADS["decode_32k"]
+    assert sa.decode_launches(sa.params_for(w, out_dtype="f32")) == 1
+    check_decode(w, seed=92, pairs=_sampled(w), out_dtype=torch.float32)
+    torch.cuda.empty_cache()
+
+
 def test_fused_empty_tiles_after_score_chunks():
     """A 3-block window plus the new key gives an odd number of
     index-independent tiles, so the last unit of each pair's run has an

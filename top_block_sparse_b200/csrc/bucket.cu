@@ -39,6 +39,7 @@ constexpr int kWardThreads = 512;
 constexpr int kWardWarps = kWardThreads / 32;
 constexpr int kWardMaxMembers = 16;            // pool keys per bucket at most (16 raw keys, stride 1)
 constexpr int kOwnPerCta = 64;                 // expansion entries per CTA of bucket_own_kernel
+constexpr int kStageBytes = 131072;            // raw keys staged per bulk copy (inside M and the costs)
 
 typedef unsigned long long u64;
 
@@ -91,6 +92,31 @@ __device__ __forceinline__ void pool_key(const void* K, int64_t row0, int stride
   }
 }
 
+// The same from raw key rows staged in shared memory (row bytes 128 x el).
+template <bool BF16>
+__device__ __forceinline__ void pool_key_smem(const unsigned char* row0, int stride, int lane, float (&acc)[4]) {
+  constexpr int kRowBytes = kHeadDim * (BF16 ? 2 : 4);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) acc[e] = 0.f;
+#pragma unroll 4
+  for (int r = 0; r < stride; ++r) {
+    const unsigned char* row = row0 + r * kRowBytes;
+    float x[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if constexpr (BF16) {
+        x[e] = __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(row)[lane + 32 * e]) << 16);
+      } else {
+        x[e] = reinterpret_cast<const float*>(row)[lane + 32 * e];
+      }
+    }
+    const float s2 = warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
+    const float sc = s2 > 0.f ? 1.f / sqrtf(s2) : 0.f;      // normalise(0) = 0
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] += x[e] * sc;
+  }
+}
+
 // The normalised index query of `pair`: the sum of its G query heads of the
 // first new token, divided by its norm (0 stays 0); coordinates lane + 32 e.
 template <bool BF16>
@@ -120,7 +146,8 @@ template <bool BF16>
 __global__ void __launch_bounds__(kWardThreads, 1) ward_kernel(WardArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   float* S = reinterpret_cast<float*>(smem);
-  float* cost = S + kHeadDim * kWardRow;
+  float* M = S + kHeadDim * kWardRow;                      // bucket means, same layout as S
+  float* cost = M + kHeadDim * kWardRow;
   float* inv = cost + kWardMaxPool * kWardCost;
   float* bestc = inv + kWardMaxPool;
   float* pc = bestc + kWardMaxPool;                        // [64] pair costs
@@ -132,6 +159,10 @@ __global__ void __launch_bounds__(kWardThreads, 1) ward_kernel(WardArgs a) {
   int* rank = keep + kWardMaxPool / 2;                     // [128]
   int* misc = rank + kWardMaxPool;                         // [8]
   uint8_t* mem = reinterpret_cast<uint8_t*>(misc + 8);     // [128][16]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(mem + kWardMaxPool * kWardMaxMembers);
+  // the block's raw keys are staged (one or two bulk copies of up to 128 KB)
+  // in the space of M and the cost matrix, which are filled only afterwards
+  unsigned char* stage = reinterpret_cast<unsigned char*>(M);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t pair = blockIdx.y;
@@ -144,89 +175,157 @@ __global__ void __launch_bounds__(kWardThreads, 1) ward_kernel(WardArgs a) {
     inv[t] = 1.f;
     mem[t * kWardMaxMembers] = static_cast<uint8_t>(t);
   }
-  // pool keys (§2.2: normalise, sum `stride` consecutive keys)
-  for (int i = warp; i < m; i += kWardWarps) {
-    float acc[4];
-    const int64_t row0 = (pair * a.cap + blk * a.b + static_cast<int64_t>(i) * a.stride) * kHeadDim;
-    pool_key<BF16>(a.K, row0, a.stride, lane, acc);
+  // pool keys (§2.2: normalise, sum `stride` consecutive keys) from the
+  // staged raw keys
+  {
+    constexpr int kRowBytes = kHeadDim * (BF16 ? 2 : 4);
+    constexpr int kChunkRows = kStageBytes / kRowBytes;              // a multiple of every stride
+    if (threadIdx.x == 0) {
+      mbar_init(bar, 1);
+      fence_mbar_init();
+    }
+    __syncthreads();
+    const unsigned char* src = static_cast<const unsigned char*>(a.K) + (pair * a.cap + blk * a.b) * kRowBytes;
+    for (int r0 = 0, c = 0; r0 < a.b; r0 += kChunkRows, ++c) {
+      const int rows = min(kChunkRows, a.b - r0);
+      if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * kRowBytes);
+        bulk_g2s(stage, src + static_cast<int64_t>(r0) * kRowBytes, static_cast<uint32_t>(rows) * kRowBytes, bar);
+      }
+      const bool ok = mbar_wait_bounded(bar, c & 1, nullptr);
+      if (__syncthreads_or(!ok)) {
+        // the copy did not land in time: leave this block's buckets empty
+        // (members -1) after a last bounded wait for the copy in flight
+        if (threadIdx.x == 0) mbar_wait_bounded(bar, c & 1, nullptr);
+        int32_t* out = a.members + (pair * a.rows_per_pair + blk * a.nbk) * a.mcap;
+        for (int t = threadIdx.x; t < a.nbk * a.mcap; t += kWardThreads) out[t] = -1;
+        __syncthreads();
+        return;
+      }
+      for (int i = r0 / a.stride + warp; i < (r0 + rows) / a.stride; i += kWardWarps) {
+        float acc[4];
+        pool_key_smem<BF16>(stage + (i * a.stride - r0) * kRowBytes, a.stride, lane, acc);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) S[(lane + 32 * e) * kWardRow + i] = acc[e];
+        for (int e = 0; e < 4; ++e) S[(lane + 32 * e) * kWardRow + i] = acc[e];
+      }
+      __syncthreads();                   // the stage is free for the next copy
+    }
+    for (int item = threadIdx.x; item < kHeadDim * kWardMaxPool; item += kWardThreads) {
+      const int d = item >> 7, i = item & (kWardMaxPool - 1);
+      M[d * kWardRow + i] = S[d * kWardRow + i];
+    }
+    __syncthreads();
   }
-  __syncthreads();
 
-  // initial costs: singletons, n_a n_b / (n_a + n_b) = 1/2; thread (warp, lane)
-  // computes buckets 4 lane .. 4 lane + 3 against 4 w .. 4 w + 3 and 4 (w + 16) ..
+  // initial costs of singletons (n_a n_b / (n_a + n_b) = 1/2), upper
+  // triangle of 4 x 4 bucket tiles, both halves of the matrix written.  Warp w
+  // takes the column blocks w (rows 0..w) and 31 - w (rows 0..30 - w), one
+  // tile per lane; the 16 diagonal tiles of blocks 16..31 left over are 96
+  // single pairs done after.
   {
     const u64 neg1 = pk2(-1.f, -1.f);
-    u64 acc[2][4][2];
+    const int ib = lane <= warp ? lane : lane - warp - 1;          // row block
+    const int jb = lane <= warp ? warp : 31 - warp;                // column block
+    u64 acc[4][2];
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
-#pragma unroll
-      for (int u = 0; u < 4; ++u) acc[t][u][0] = acc[t][u][1] = 0ull;
-    const int cb0 = 4 * warp, cb1 = 4 * (warp + kWardWarps);
-#pragma unroll 2
+    for (int u = 0; u < 4; ++u) acc[u][0] = acc[u][1] = 0ull;
+#pragma unroll 4
     for (int d = 0; d < kHeadDim; ++d) {
       const float* row = S + d * kWardRow;
-      const float4 av = *reinterpret_cast<const float4*>(row + 4 * lane);
-      const float4 b0 = *reinterpret_cast<const float4*>(row + cb0);
-      const float4 b1 = *reinterpret_cast<const float4*>(row + cb1);
-      const u64 b[2][2] = {{pk2(b0.x, b0.y), pk2(b0.z, b0.w)}, {pk2(b1.x, b1.y), pk2(b1.z, b1.w)}};
+      const float4 av = *reinterpret_cast<const float4*>(row + 4 * ib);
+      const float4 bv = *reinterpret_cast<const float4*>(row + 4 * jb);
+      const u64 b0 = pk2(bv.x, bv.y), b1 = pk2(bv.z, bv.w);
       const float ar[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const u64 a2 = pk2(ar[u], ar[u]);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const u64 df = fma2(b[t][v], neg1, a2);        // a - b, rounded once
-            acc[t][u][v] = fma2(df, df, acc[t][u][v]);
-          }
+        const u64 d0 = fma2(b0, neg1, a2), d1 = fma2(b1, neg1, a2);   // a - b, rounded once
+        acc[u][0] = fma2(d0, d0, acc[u][0]);
+        acc[u][1] = fma2(d1, d1, acc[u][1]);
       }
     }
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
+    for (int u = 0; u < 4; ++u)
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          const int ra = 4 * lane + u, cb = (t ? cb1 : cb0) + 2 * v;
-          if (ra < m && cb < m && ra != cb) cost[ra * kWardCost + cb] = 0.5f * lo2(acc[t][u][v]);
-          if (ra < m && cb + 1 < m && ra != cb + 1) cost[ra * kWardCost + cb + 1] = 0.5f * hi2(acc[t][u][v]);
+      for (int v = 0; v < 4; ++v) {
+        const int ra = 4 * ib + u, cb = 4 * jb + v;
+        if (ra < cb && cb < m) {
+          const float c = 0.5f * ((v & 1) ? hi2(acc[u][v >> 1]) : lo2(acc[u][v >> 1]));
+          cost[ra * kWardCost + cb] = c;
+          cost[cb * kWardCost + ra] = c;
         }
+      }
+    if (threadIdx.x < 96) {
+      // pairs (u, v), u < v, inside diagonal tile 16 + t / 6
+      const int t = threadIdx.x, jd = 16 + t / 6, q = t % 6;
+      const int u = q < 3 ? 0 : (q < 5 ? 1 : 2);
+      const int v = q < 3 ? q + 1 : (q < 5 ? q - 1 : 3);
+      const int ra = 4 * jd + u, cb = 4 * jd + v;
+      float s = 0.f;
+      for (int d = 0; d < kHeadDim; ++d) {
+        const float df = S[d * kWardRow + ra] - S[d * kWardRow + cb];
+        s = fmaf(df, df, s);
+      }
+      if (cb < m) {
+        cost[ra * kWardCost + cb] = 0.5f * s;
+        cost[cb * kWardCost + ra] = 0.5f * s;
+      }
+    }
   }
 
   // rounds of mutual cheapest merges
   int alive = m;
   for (int round = 0; alive > a.nbk && round < m; ++round) {
     __syncthreads();
-    for (int r = warp; r < m; r += kWardWarps) {
-      const int nr = n[r];
-      if (nr == 0) continue;
-      float bc = CUDART_INF_F;
-      int bi = -1;
-      for (int c = lane; c < m; c += 32) {
-        const int nc = n[c];
-        if (c != r && nc > 0 && nr + nc <= a.mcap) {
-          const float v = cost[r * kWardCost + c];
-          if (v < bc) {
-            bc = v;
-            bi = c;
+    {
+      // the warp's 8 rows r = warp + 16 j side by side (their reductions
+      // overlap); lane l holds candidates 4 l .. 4 l + 3, ascending
+      constexpr int kRows = kWardMaxPool / kWardWarps;
+      const int4 nn = *reinterpret_cast<const int4*>(n + 4 * lane);
+      const int nv[4] = {nn.x, nn.y, nn.z, nn.w};
+      float bc[kRows];
+      int bi[kRows];
+#pragma unroll
+      for (int j = 0; j < kRows; ++j) {
+        const int r = warp + kWardWarps * j;
+        const int nr = r < m ? n[r] : 0;
+        bc[j] = CUDART_INF_F;
+        bi[j] = -1;
+        if (nr > 0) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * lane + e;
+            if (c != r && nv[e] > 0 && nr + nv[e] <= a.mcap) {
+              const float v = cost[r * kWardCost + c];
+              if (v < bc[j]) {
+                bc[j] = v;
+                bi[j] = c;
+              }
+            }
           }
         }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bc, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (oi >= 0 && (bi < 0 || ov < bc || (ov == bc && oi < bi))) {
-          bc = ov;
-          bi = oi;
+#pragma unroll
+        for (int j = 0; j < kRows; ++j) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bc[j], o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi[j], o);
+          if (oi >= 0 && (bi[j] < 0 || ov < bc[j] || (ov == bc[j] && oi < bi[j]))) {
+            bc[j] = ov;
+            bi[j] = oi;
+          }
         }
       }
       if (lane == 0) {
-        best[r] = bi;
-        bestc[r] = bc;
+#pragma unroll
+        for (int j = 0; j < kRows; ++j) {
+          const int r = warp + kWardWarps * j;
+          if (r < m && n[r] > 0) {
+            best[r] = bi[j];
+            bestc[r] = bc[j];
+          }
+        }
       }
     }
     if (threadIdx.x == 0) misc[0] = 0;
@@ -280,35 +379,45 @@ __global__ void __launch_bounds__(kWardThreads, 1) ward_kernel(WardArgs a) {
       inv[r] = 1.f / static_cast<float>(na + nb2);
     }
     __syncthreads();
-    // costs of every merged bucket against every live one (both halves of
-    // the symmetric matrix; two merged buckets compute their shared entry
-    // twice, to the same value)
-    for (int i = warp; i < np; i += kWardWarps) {
-      if (!keep[i]) continue;
-      const int r = pa[i];
-      const float ir = inv[r];
-      const int nr = n[r];
-      float ic[4], acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) ic[e] = inv[lane + 32 * e];
-#pragma unroll 2
-      for (int d = 0; d < kHeadDim; ++d) {
-        const float* row = S + d * kWardRow;
-        const float sr = row[r] * ir;
+    for (int item = threadIdx.x; item < np * kHeadDim; item += kWardThreads) {
+      const int i = item >> 7, d = item & (kHeadDim - 1);
+      if (keep[i]) M[d * kWardRow + pa[i]] = S[d * kWardRow + pa[i]] / static_cast<float>(n[pa[i]]);
+    }
+    __syncthreads();
+    // costs of every merged bucket against every live one from the means
+    // (both halves of the symmetric matrix; two merged buckets compute their
+    // shared entry twice, to the same value); lane l takes buckets 4 l .. 4 l + 3
+    {
+      // costs of every merged bucket against every live one from the means
+      // (both halves of the symmetric matrix; two merged buckets compute
+      // their shared entry twice, to the same value); lane l takes buckets
+      // 4 l .. 4 l + 3
+      const u64 neg1 = pk2(-1.f, -1.f);
+      for (int i = warp; i < np; i += kWardWarps) {
+        if (!keep[i]) continue;
+        const int r = pa[i];
+        const int nr = n[r];
+        u64 acc0 = 0ull, acc1 = 0ull;
+#pragma unroll 4
+        for (int d = 0; d < kHeadDim; ++d) {
+          const float* row = M + d * kWardRow;
+          const float mr = row[r];
+          const float4 mc = *reinterpret_cast<const float4*>(row + 4 * lane);
+          const u64 r2 = pk2(mr, mr);
+          const u64 d0 = fma2(pk2(mc.x, mc.y), neg1, r2), d1 = fma2(pk2(mc.z, mc.w), neg1, r2);
+          acc0 = fma2(d0, d0, acc0);
+          acc1 = fma2(d1, d1, acc1);
+        }
+        const float accv[4] = {lo2(acc0), hi2(acc0), lo2(acc1), hi2(acc1)};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float df = sr - row[lane + 32 * e] * ic[e];
-          acc[e] = fmaf(df, df, acc[e]);
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = lane + 32 * e;
-        if (c < m && c != r && n[c] > 0) {
-          const float w = static_cast<float>(nr * n[c]) / static_cast<float>(nr + n[c]);
-          const float v = w * acc[e];
-          cost[r * kWardCost + c] = v;
-          cost[c * kWardCost + r] = v;
+          const int c = 4 * lane + e;
+          if (c < m && c != r && n[c] > 0) {
+            const float w = static_cast<float>(nr * n[c]) / static_cast<float>(nr + n[c]);
+            const float v = w * accv[e];
+            cost[r * kWardCost + c] = v;
+            cost[c * kWardCost + r] = v;
+          }
         }
       }
     }
@@ -410,35 +519,45 @@ __global__ void __launch_bounds__(256) bucket_score_kernel(BucketScoreArgs a) {
 }
 
 // ---- §2.3: top-k buckets -------------------------------------------------------
-// One CTA per pair: the k-th largest candidate key by four 8-bit radix passes
-// over the pair's keys (L2-resident), then the selected ids in ascending
-// order: every key above the threshold and, of the keys equal to it, the
-// lowest ids (a warp per contiguous segment, two scans over the warps).
-constexpr int kSelThreads = 1024;
-__global__ void __launch_bounds__(kSelThreads) bucket_select_kernel(const uint32_t* keys_all, int64_t n, int k,
-                                                                     int32_t* sel_all) {
+// Exact top-k of n order-preserving keys held in shared memory by one CTA of
+// THREADS threads (key 0 = not a candidate): the k-th largest key tau by four
+// 8-bit radix passes (lanes of a warp that fall into one bin add once), then
+// the positions of the selected keys in ascending order: every key above
+// tau and, of the keys equal to it, the lowest positions (a warp per
+// contiguous segment, two scans over the warps).  Writes min(k, candidates)
+// positions to out[0..), -1 up to k.
+template <int THREADS>
+__device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out) {
+  constexpr int W = THREADS / 32;
+  constexpr int HG = 8;                // warps sharing one private histogram
   __shared__ unsigned hist[256];
-  __shared__ unsigned wgt[32], weq[32];
-  __shared__ unsigned bc[4];     // prefix, need (keys equal to tau to take), keff
+  __shared__ unsigned phist[W / HG][256];
+  __shared__ unsigned wgt[W], weq[W];
+  __shared__ unsigned bc[3];     // prefix, keys equal to tau still to take, keff
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t pair = blockIdx.x;
-  const uint32_t* keys = keys_all + pair * n;
-  int32_t* sel = sel_all + pair * static_cast<int64_t>(k);
   uint32_t prefix = 0, pmask = 0;
   unsigned remaining = 0, keff = 0;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    if (threadIdx.x < 256) hist[threadIdx.x] = 0;
+    for (int t = threadIdx.x; t < (W / HG) * 256; t += THREADS) (&phist[0][0])[t] = 0;
     __syncthreads();
-    // lanes of a warp that fall into the same bin add once (scores crowd a
-    // few bins of the leading digits)
-    for (int64_t b0 = static_cast<int64_t>(warp) * 32; b0 < n; b0 += kSelThreads) {
-      const int64_t i = b0 + lane;
-      const uint32_t key = i < n ? __ldg(keys + i) : 0u;
+    // the scores crowd a few bins of the leading digits: lanes of a warp in
+    // one bin add once, and groups of HG warps count into their own copy
+    unsigned* my = phist[warp / HG];
+    for (int b0 = warp * 32; b0 < n; b0 += THREADS) {
+      const int i = b0 + lane;
+      const uint32_t key = i < n ? keys[i] : 0u;
       const bool want = key != 0u && (key & pmask) == prefix;
       const unsigned bin = want ? (key >> shift) & 255u : 256u;
       const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (want && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<unsigned>(__popc(peers)));
+      if (want && lane == __ffs(peers) - 1) atomicAdd(&my[bin], static_cast<unsigned>(__popc(peers)));
+    }
+    __syncthreads();
+    if (threadIdx.x < 256) {
+      unsigned t = 0;
+#pragma unroll
+      for (int g = 0; g < W / HG; ++g) t += phist[g][threadIdx.x];
+      hist[threadIdx.x] = t;
     }
     __syncthreads();
     if (warp == 0) {
@@ -460,7 +579,7 @@ __global__ void __launch_bounds__(kSelThreads) bucket_select_kernel(const uint32
         const unsigned y = __shfl_down_sync(0xffffffffu, above, o);
         if (lane + o < 32) above += y;
       }
-      const unsigned higher = above - own;      // lanes above this one
+      const unsigned higher = above - own;
       int digit = -1;
       unsigned cnt_above_digit = 0;
       if (remaining > 0 && higher < remaining && above >= remaining) {
@@ -495,16 +614,17 @@ __global__ void __launch_bounds__(kSelThreads) bucket_select_kernel(const uint32
     remaining = bc[1];
     keff = bc[2];
     pmask |= 255u << shift;
+    __syncthreads();             // bc is rewritten by the next pass
     if (keff == 0) break;
   }
   const uint32_t tau = prefix;
   const unsigned need = remaining;
-  const int64_t seg = (n + 31) / 32;
-  const int64_t s0 = warp * seg, s1 = min(n, s0 + seg);
+  const int seg = (n + W - 1) / W;
+  const int s0 = warp * seg, s1 = min(n, s0 + seg);
   unsigned gt = 0, eq = 0;
   if (keff > 0)
-    for (int64_t i = s0 + lane; i < s1; i += 32) {
-      const uint32_t key = __ldg(keys + i);
+    for (int i = s0 + lane; i < s1; i += 32) {
+      const uint32_t key = keys[i];
       gt += key > tau;
       eq += key == tau;
     }
@@ -516,7 +636,8 @@ __global__ void __launch_bounds__(kSelThreads) bucket_select_kernel(const uint32
   }
   __syncthreads();
   if (warp == 0) {
-    unsigned g = wgt[lane], e = weq[lane];
+    unsigned g = lane < W ? wgt[lane] : 0u, e = lane < W ? weq[lane] : 0u;
+    const unsigned g0 = g, e0 = e;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const unsigned yg = __shfl_up_sync(0xffffffffu, g, o);
@@ -526,30 +647,73 @@ __global__ void __launch_bounds__(kSelThreads) bucket_select_kernel(const uint32
         e += ye;
       }
     }
-    wgt[lane] = g - wgt[lane];
-    weq[lane] = e - weq[lane];
+    if (lane < W) {
+      wgt[lane] = g - g0;
+      weq[lane] = e - e0;
+    }
   }
   __syncthreads();
   if (keff > 0) {
     unsigned gt_before = wgt[warp], eq_before = weq[warp];
     const unsigned lt = (1u << lane) - 1u;
-    for (int64_t b0 = s0; b0 < s1; b0 += 32) {
-      const int64_t i = b0 + lane;
-      const uint32_t key = i < s1 ? __ldg(keys + i) : 0u;
+    for (int b0 = s0; b0 < s1; b0 += 32) {
+      const int i = b0 + lane;
+      const uint32_t key = i < s1 ? keys[i] : 0u;
       const bool is_gt = i < s1 && key > tau;
       const bool is_eq = i < s1 && key == tau;
       const unsigned bg = __ballot_sync(0xffffffffu, is_gt), be = __ballot_sync(0xffffffffu, is_eq);
       const unsigned my_eq = eq_before + __popc(be & lt);
-      const bool take = is_gt || (is_eq && my_eq < need);
-      if (take) {
-        const unsigned pos = gt_before + __popc(bg & lt) + min(my_eq, need);
-        sel[pos] = static_cast<int32_t>(i);
-      }
+      if (is_gt || (is_eq && my_eq < need)) out[gt_before + __popc(bg & lt) + min(my_eq, need)] = i;
       gt_before += __popc(bg);
       eq_before += __popc(be);
     }
   }
-  for (int i = keff + threadIdx.x; i < k; i += kSelThreads) sel[i] = -1;
+  for (int i = keff + threadIdx.x; i < k; i += THREADS) out[i] = -1;
+  __syncthreads();
+}
+
+// First level: the top min(k, 8192) of each chunk of kLocalKeys buckets (one
+// CTA per (chunk, pair)).  Every key of the global top-k is among the top-k of
+// its own chunk (same order), so the chunks' winners, kept in bucket order,
+// are the candidates of the second level.
+constexpr int kLocalKeys = kBucketChunk;
+constexpr int kLocalThreads = 512;
+__global__ void __launch_bounds__(kLocalThreads) bucket_local_topk_kernel(const uint32_t* keys_all, int64_t n, int kl,
+                                                                          uint32_t* cand_key, int32_t* cand_id) {
+  extern __shared__ __align__(16) uint32_t keys[];         // [kLocalKeys], then the positions
+  int32_t* pos = reinterpret_cast<int32_t*>(keys + kLocalKeys);
+  const int64_t pair = blockIdx.y;
+  const int64_t g0 = static_cast<int64_t>(blockIdx.x) * kLocalKeys;
+  const int64_t left = n - g0;
+  const int nl = left < kLocalKeys ? static_cast<int>(left) : kLocalKeys;
+  const uint32_t* src = keys_all + pair * n + g0;
+  for (int i = threadIdx.x; i < kLocalKeys; i += kLocalThreads) keys[i] = i < nl ? __ldg(src + i) : 0u;
+  __syncthreads();
+  smem_topk<kLocalThreads>(keys, nl, kl, pos);
+  const int64_t ob = (pair * gridDim.x + blockIdx.x) * kl;
+  for (int j = threadIdx.x; j < kl; j += kLocalThreads) {
+    const int q = pos[j];
+    cand_key[ob + j] = q >= 0 ? keys[q] : 0u;
+    cand_id[ob + j] = q >= 0 ? static_cast<int32_t>(g0 + q) : -1;
+  }
+}
+
+// Second level: one CTA per pair selects the top k of its chunks' candidates
+// (in shared memory, bucket order), ties to the lower bucket.
+constexpr int kSelThreads = 1024;
+__global__ void __launch_bounds__(kSelThreads) bucket_select_kernel(const uint32_t* cand_key, const int32_t* cand_id,
+                                                                     int nc, int k, int32_t* sel_all) {
+  extern __shared__ __align__(16) uint32_t ck[];
+  int32_t* pos = reinterpret_cast<int32_t*>(ck + nc);
+  const int64_t pair = blockIdx.x;
+  for (int i = threadIdx.x; i < nc; i += kSelThreads) ck[i] = __ldg(cand_key + pair * nc + i);
+  __syncthreads();
+  smem_topk<kSelThreads>(ck, nc, k, pos);
+  int32_t* sel = sel_all + pair * static_cast<int64_t>(k);
+  for (int j = threadIdx.x; j < k; j += kSelThreads) {
+    const int q = pos[j];
+    sel[j] = q >= 0 ? __ldg(cand_id + pair * nc + q) : -1;
+  }
 }
 
 // ---- §2.3: expansion by within-bucket merit ------------------------------------
@@ -665,8 +829,9 @@ __global__ void __launch_bounds__(512) bucket_keep_kernel(BucketExpandArgs a) {
 }  // namespace
 
 size_t ward_smem_bytes() {
-  return sizeof(float) * (kHeadDim * kWardRow + kWardMaxPool * kWardCost + 2 * kWardMaxPool + kWardMaxPool / 2) +
-         sizeof(int) * (3 * kWardMaxPool + 3 * (kWardMaxPool / 2) + 8) + kWardMaxPool * kWardMaxMembers;
+  return sizeof(float) * (2 * kHeadDim * kWardRow + kWardMaxPool * kWardCost + 2 * kWardMaxPool + kWardMaxPool / 2) +
+         sizeof(int) * (3 * kWardMaxPool + 3 * (kWardMaxPool / 2) + 8) + kWardMaxPool * kWardMaxMembers +
+         sizeof(uint64_t);
 }
 
 cudaError_t launch_ward(const WardArgs& a, int pairs, int64_t n_blocks, bool bf16, cudaStream_t s) {
@@ -690,8 +855,22 @@ cudaError_t launch_bucket_select(const BucketScoreArgs& sa_, const BucketExpandA
     if (e != cudaSuccess) return e;
   }
   if (ea.top_k > 0) {
-    bucket_select_kernel<<<pairs, kSelThreads, 0, s>>>(sa_.keys, sa_.n_bkt, ea.top_k, ea.sel);
-    cudaError_t e = cudaGetLastError();
+    const int chunks = static_cast<int>((sa_.n_bkt + kLocalKeys - 1) / kLocalKeys);
+    const int kl = ea.top_k < kLocalKeys ? ea.top_k : kLocalKeys;
+    const int nc = chunks * kl;
+    constexpr size_t kLocalSmem = static_cast<size_t>(kLocalKeys) * 8;
+    cudaError_t e = cudaFuncSetAttribute(bucket_local_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kLocalSmem));
+    if (e != cudaSuccess) return e;
+    bucket_local_topk_kernel<<<dim3(chunks, pairs), kLocalThreads, kLocalSmem, s>>>(sa_.keys, sa_.n_bkt, kl,
+                                                                                     sa_.cand_key, sa_.cand_id);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t smem = static_cast<size_t>(nc) * 8;     // keys and positions
+    e = cudaFuncSetAttribute(bucket_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    bucket_select_kernel<<<pairs, kSelThreads, smem, s>>>(sa_.cand_key, sa_.cand_id, nc, ea.top_k, ea.sel);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -199,6 +199,8 @@ struct BucketScoreArgs {
   const float* cents;
   const int32_t* members;
   uint32_t* keys;         // [pairs, n_bkt] order-preserving cosine keys, 0 = not a candidate
+  uint32_t* cand_key;     // [pairs, chunks * min(top_k, kBucketChunk)] first-level winners (workspace)
+  int32_t* cand_id;       // their bucket ids
   int Hq, Hkv, G, n_q;
   int64_t rows_per_pair;
   int64_t n_bkt;          // buckets of the context's complete cluster blocks
@@ -219,7 +221,11 @@ struct BucketExpandArgs {
   int keep_pool;          // pool keys kept (0: every member of the selected buckets)
   int kept_cap;
 };
-// Scores of every bucket and the top-k selection into ea.sel.
+// Scores of every bucket and the top-k selection into ea.sel (two levels:
+// the top-k of every kBucketChunk buckets, then of those winners, at most
+// kBucketMaxCand per pair, in shared memory).
+constexpr int kBucketChunk = 8192;
+constexpr int kBucketMaxCand = 28672;
 cudaError_t launch_bucket_select(const BucketScoreArgs& sa_, const BucketExpandArgs& ea, int pairs, bool bf16,
                                  cudaStream_t s);
 // Expansion of the selected buckets into ea.kept.

@@ -345,6 +345,12 @@ struct BucketGeom {
   int64_t n_bkt;           // buckets of the context's complete cluster blocks
 };
 
+// First-level winners of the bucket selection per pair.
+int64_t bucket_cands(const sa_params* p, const BucketGeom& g) {
+  const int64_t chunks = (g.n_bkt + kBucketChunk - 1) / kBucketChunk;
+  return chunks * std::min(p->top_k, kBucketChunk);
+}
+
 sa_status check_bucket(const sa_params* p, BucketGeom* g) {
   sa_status st = check_params(p, false);
   if (st != SA_OK) return st;
@@ -371,12 +377,16 @@ sa_status check_bucket(const sa_params* p, BucketGeom* g) {
                 p->top_k * g->mcap);
   if (static_cast<int64_t>(p->batch) * p->num_kv_heads > 65535)
     return fail(SA_ERR_UNSUPPORTED, "more than 65535 (sequence, KV head) pairs");
+  if (bucket_cands(p, *g) > kBucketMaxCand)
+    return fail(SA_ERR_UNSUPPORTED,
+                "%lld buckets with top_k %d: the selection's %lld first-level winners per sequence exceed %d",
+                (long long)g->n_bkt, p->top_k, (long long)bucket_cands(p, *g), kBucketMaxCand);
   return SA_OK;
 }
 
 struct BucketWs {
   DecodeWs attn;
-  size_t keys, sel, own, kept, total;
+  size_t keys, cand_key, cand_id, sel, own, kept, total;
 };
 
 // Attention plan of the run mode: the selected section holds kept_cap runs,
@@ -398,8 +408,11 @@ BucketWs bucket_ws(const sa_params* p, const BucketGeom& bg, const DecodeGeom& g
   w.attn = decode_ws(g, plan, 0, SA_OP_GIVEN_IDX, 0);
   const size_t pairs = static_cast<size_t>(g.pairs);
   const size_t n_ent = static_cast<size_t>(p->top_k) * bg.mcap;
+  const size_t nc = static_cast<size_t>(bucket_cands(p, bg));
   w.keys = align_up(w.attn.total, 256);
-  w.sel = align_up(w.keys + pairs * static_cast<size_t>(bg.n_bkt) * 4, 256);
+  w.cand_key = align_up(w.keys + pairs * static_cast<size_t>(bg.n_bkt) * 4, 256);
+  w.cand_id = align_up(w.cand_key + pairs * nc * 4, 256);
+  w.sel = align_up(w.cand_id + pairs * nc * 4, 256);
   w.own = align_up(w.sel + pairs * static_cast<size_t>(p->top_k) * 4, 256);
   w.kept = align_up(w.own + pairs * n_ent * 8, 256);
   w.total = align_up(w.kept + pairs * n_ent * 4, 256);
@@ -955,6 +968,8 @@ extern "C" sa_status sa_bucket_decode(const sa_params* p, const void* Q, const v
   sc.cents = centroids;
   sc.members = members;
   sc.keys = reinterpret_cast<uint32_t*>(w + L.keys);
+  sc.cand_key = reinterpret_cast<uint32_t*>(w + L.cand_key);
+  sc.cand_id = reinterpret_cast<int32_t*>(w + L.cand_id);
   sc.Hq = p->num_q_heads;
   sc.Hkv = p->num_kv_heads;
   sc.G = p->num_q_heads / p->num_kv_heads;
