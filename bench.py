@@ -655,6 +655,7 @@ def run_ours(args, w, rank, world, local_rank):
                  "note": "compression runs once after prefill / when a block fills; not part of a decode step"},
         "e2e": {"value": world * w.batch * w.n_q / (e2e["ms"] * 1e-3), "unit": "queries/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                "ms_per_step": e2e["ms"], "breakdown_us": e2e["breakdown_us"],
                 "note": "per step: one pinned host -> device copy of the new tokens' Q, K, V rows (packed), "
                         "sa_append_kv into the cache and the decode call through the C ABI, device -> pinned "
                         "host copy of O; the KV cache and the compressed keys stay resident in HBM"},
@@ -1151,7 +1152,33 @@ def e2e_decode(args, w, p, Q, K, V, Kc, O, lse, idx, ws, stream, flush):
     n = max(50, args.steps // 4)
     with torch.cuda.stream(stream):
         ms = statistics.mean(timed_steps(one, n, args.warmup, stream, flush))
-    return {"ms": ms, "h2d": h_stage.numel() * h_stage.element_size(), "d2h": hO.numel() * O.element_size()}
+    # where the step's time goes: the same four operations with an event
+    # between each, in a loop of their own (the events add a little)
+    parts = ["h2d_copy", "append_kv", "decode", "d2h_copy"]
+    ops = [lambda: d_stage.copy_(h_stage, non_blocking=True),
+           lambda: sa.append_kv(p, Kn, Vn, K, V, stream=stream),
+           lambda: sa.sparse_attn_decode(p, Qs, K, V, Kc, O, lse, idx, ws, stream=stream),
+           lambda: hO.copy_(O, non_blocking=True)]
+    rec = []
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            for op in ops:
+                op()
+        torch.cuda.synchronize()
+        queue_ahead(20)
+        for _ in range(20):
+            flush()
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(ops) + 1)]
+            evs[0].record(stream)
+            for op, ev in zip(ops, evs[1:]):
+                op()
+                ev.record(stream)
+            rec.append(evs)
+    torch.cuda.synchronize()
+    breakdown = {name: statistics.median(r[i].elapsed_time(r[i + 1]) for r in rec) * 1e3
+                 for i, name in enumerate(parts)}
+    return {"ms": ms, "h2d": h_stage.numel() * h_stage.element_size(), "d2h": hO.numel() * O.element_size(),
+            "breakdown_us": breakdown}
 
 
 def main():

@@ -46,6 +46,10 @@ constexpr int kQBytes = kRows * 256;           // 64 KB (two 32 KB boxes: d 0-63
 constexpr int kKVStage = 32768;                // K 16 KB (two 8 KB boxes) + V 16 KB
 constexpr int kPBytes = 2 * 16384;             // P: two halves of 128 rows x 64 keys
 constexpr int kThreads = 320;
+constexpr int kGatherWarps = 2;                // column mode: warps 8 and 10 gather K and V rows
+constexpr int kGatherRows = kT / kGatherWarps;  // rows of a chunk per gathering warp
+constexpr int kLanesPerRow = 32 / kGatherRows;
+constexpr int kThreadsCol = kThreads + (kGatherWarps - 1) * 32;
 constexpr uint32_t kIdescS = tc::idesc_bf16(128, 64, false, false);
 constexpr uint32_t kIdescO = tc::idesc_bf16(128, 128, false, true);
 constexpr float kLazy = 8.f;                   // rescale when the max grows by > 2^8
@@ -140,7 +144,7 @@ __device__ __forceinline__ void item_of(const PAArgs& a, int k, int* p, int* t) 
 }
 
 template <bool COL>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(COL ? kThreadsCol : kThreads, 1)
     prefill_attn_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                         const __grid_constant__ CUtensorMap v_map, PAArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -167,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNKV; ++s) {
-      mbar_init(&kv_full[s], COL ? 32 : 1);         // column mode: one arrival per producer lane
+      mbar_init(&kv_full[s], COL ? 32 * kGatherWarps : 1);   // column mode: one arrival per gathering lane
       mbar_init(&kv_empty[s], 1);
     }
     mbar_init(q_full, 1);
@@ -195,8 +199,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 1;
   };
 
-  if (warp == 8) {
+  if (warp == 8 || (COL && warp >= 10)) {
     // -------------------------------------------------------- TMA producer
+    // column mode: warps 8 and 10 (and more with kGatherWarps) gather
+    // kGatherRows of every chunk's rows each; warp 8 also loads Q
+    const int gw = warp == 8 ? 0 : warp - 9;
     int use = 0, it = 0;
     bool ok = true;
     for (int k = blockIdx.x; k < n_items && ok; k += gridDim.x, ++it) {
@@ -206,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t* row = a.idx + (static_cast<int64_t>(p) * a.n_tiles + t) * a.top_k;
       const int bi = p / a.Hkv, h = p % a.Hkv;
       if constexpr (COL) {
-        if (lane == 0) {
+        if (warp == 8 && lane == 0) {
           if (it > 0 && !mbar_wait_bounded(q_empty, (it - 1) & 1, abort_flag)) { fail(); ok = false; }
           if (ok) {
             mbar_arrive_expect_tx(q_full, kQBytes);
@@ -220,20 +227,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const unsigned char* vb = static_cast<const unsigned char*>(a.V) + static_cast<int64_t>(p) * a.cap * 256;
         int pend = 0;                               // chunks copied but not yet signalled
         // slot r of chunk b <- listed column b * 64 + r (past the list:
-        // column 0, masked; clamped into the sequence either way); lane l
-        // loads slots l and l + 32, one chunk ahead of the copies
-        auto load_cols = [&](int b, int (&c)[2]) {
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int e = b * kT + hh * 32 + lane;
-            c[hh] = e < bl.n_sel ? __ldg(row + e) : 0;
-          }
+        // column 0, masked; clamped into the sequence either way); this
+        // warp copies slots kGatherRows gw .. + kGatherRows - 1, kLanesPerRow
+        // lanes a slot, its column id loaded one chunk ahead of the copies
+        const int r = gw * kGatherRows + lane % kGatherRows;
+        auto load_col = [&](int b) -> int {
+          const int e = b * kT + r;
+          return e < bl.n_sel ? __ldg(row + e) : 0;
         };
-        int nxt[2];
-        load_cols(0, nxt);
+        int nxt = load_col(0);
         for (int b = 0; b < bl.n_blk && ok; ++b, ++use) {
-          int cur[2] = {nxt[0], nxt[1]};
-          if (b + 1 < bl.n_blk) load_cols(b + 1, nxt);
+          const int cur = nxt;
+          if (b + 1 < bl.n_blk) nxt = load_col(b + 1);
           const int s = use % kNKV;
           int fine = 1;
           if (lane == 0 && use >= kNKV && !mbar_wait_bounded(&kv_empty[s], ((use / kNKV) & 1) ^ 1, abort_flag)) {
@@ -245,14 +250,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           unsigned char* st = KV + s * kKVStage;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int r = hh * 32 + lane;
-            const int col = min(max(cur[hh], 0), a.T - 1);
+          {
+            const int col = min(max(cur, 0), a.T - 1);
             const unsigned char* ks = kb + static_cast<int64_t>(col) * 256;
             const unsigned char* vs = vb + static_cast<int64_t>(col) * 256;
+            constexpr int kPer = 16 / kLanesPerRow;   // this lane's share of the row's 16 chunks of 16 bytes
+            const int hb = (lane / kGatherRows) * kPer;
 #pragma unroll
-            for (int c16 = 0; c16 < 16; ++c16) {
+            for (int c = 0; c < kPer; ++c) {
+              const int c16 = hb + c;
               const uint32_t off = (c16 >> 3) * 8192 + tc::sw128_off(r, c16 & 7);
               cp_async16(st + off, ks + c16 * 16);
               cp_async16(st + 16384 + off, vs + c16 * 16);
@@ -651,7 +657,7 @@ cudaError_t launch_column_attn(const PrefillArgs& pa, cudaStream_t s) {
   const int items = pa.n_tiles * a.P;
   const int grid = items < pa.num_sms ? items : pa.num_sms;
   // K and V are gathered by cp.async: their tensor-map slots are unused
-  prefill_attn_kernel<true><<<grid, kThreads, smem, s>>>(qm, qm, qm, a);
+  prefill_attn_kernel<true><<<grid, kThreadsCol, smem, s>>>(qm, qm, qm, a);
   return cudaGetLastError();
 }
 
