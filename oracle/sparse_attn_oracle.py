@@ -51,7 +51,8 @@ design notes of the repository):
       near-tie; more than one selected set is then correct.
 * R7  LSA pooling order: normalise each raw key, sum 4 consecutive unit keys
       into a pool key, centroid = normalise(sum of the block's pool keys);
-      score = (qbar/|qbar|) . c_j (cosine).  normalise(0) = 0.
+      score = (qbar/|qbar|) . c_j (cosine).  normalise(0) = 0.  In a causal
+      prefill each row's index query is normalised before the tile max (R2).
 * R8  Softmax scale 1/sqrt(d) unless given (PulseCol eq. (1)).
 * R9  Multi-token chunk: the selection is made once from the chunk's FIRST
       query and reused by every token of the chunk (S3R draft chunk); token j
@@ -76,6 +77,9 @@ design notes of the repository):
       compressed key c is the mean of the l keys starting at c*s (complete
       windows only), and the score of selectable block j is the MAX of the
       scores of the compressed keys whose windows share a key with block j.
+      In a causal prefill, query tile i (context C = i*b) sees the windows
+      complete inside its context, and block j's tile score is the max over
+      those windows of the max over the tile's rows (R2).
 * R19 LSA flat bucket retrieval (LSA review §2.2-2.3).  Pool keys as in R7
       (each raw key L2-normalised, ``pool_stride`` = 4 consecutive unit keys
       summed).  A cluster block is ``block_size`` = 512 RAW keys (128 pool
@@ -461,14 +465,35 @@ def column_attention_group(q_rows: np.ndarray, K: np.ndarray, V: np.ndarray,
 # 6. Prefill (one KV head): 64-query tiles, tile-max scoring
 # --------------------------------------------------------------------------
 
-def prefill_tile_scores(q_rows: np.ndarray, Kc: np.ndarray, p: OracleParams) -> np.ndarray:
-    """Tile score of each block: max over the tile's rows of the row's
-    GQA-summed block score (readings R1, R2).  q_rows: [rows, G, d]."""
+def context_rows(C: int, p: OracleParams) -> int:
+    """Compressed keys a context of C keys holds: its complete blocks (mean
+    and LSA pooling, reading R5) or its complete windows (overlapping
+    compression, reading R18)."""
     if p.pool == "overlap":
-        raise NotImplementedError("overlapping compression is defined here for decode and draft chunks only")
+        return (C - p.pool_kernel) // p.pool_stride + 1 if C >= p.pool_kernel else 0
+    return C // p.block_size
+
+
+def prefill_tile_scores(q_rows: np.ndarray, Kc: np.ndarray, p: OracleParams,
+                        C: Optional[int] = None) -> np.ndarray:
+    """Tile score of each complete block of the context: max over the tile's
+    rows of the row's GQA-summed block score (readings R1, R2).  q_rows:
+    [rows, G, d]; Kc: the context's compressed keys (context_rows(C, p) of
+    them).
+
+    Overlapping compression (readings R2 and R18 together): every window
+    takes the max over the rows, then block j the max over the complete
+    windows touching it; both steps are maxima, so this is also the max over
+    rows of each row's own block score.  C (the tile's context length) is
+    needed in that mode only."""
     per_row = np.stack([block_scores(index_query(q_rows[r]), Kc, p)
                         for r in range(q_rows.shape[0])])
-    return per_row.max(axis=0)
+    tile = per_row.max(axis=0)
+    if p.pool == "overlap":
+        if C is None:
+            raise ValueError("overlapping compression needs the context length C")
+        return blocks_from_compressed(tile, C, p)
+    return tile
 
 
 def prefill_tile(q_tile: np.ndarray, K: np.ndarray, V: np.ndarray, i: int,
@@ -486,8 +511,8 @@ def prefill_tile(q_tile: np.ndarray, K: np.ndarray, V: np.ndarray, i: int,
     rows, G, d = q_tile.shape
     if Kc_all is None:
         Kc_all = compress(K, p)
-    Kc = Kc_all[:C // b]
-    s = prefill_tile_scores(q_tile, Kc, p) if C // b > 0 else np.zeros(0)
+    Kc = Kc_all[:context_rows(C, p)]
+    s = prefill_tile_scores(q_tile, Kc, p, C) if C // b > 0 else np.zeros(0)
     cand = candidate_blocks(C, p)
     sel = select_topk(s, cand, p.top_k)
     scale = softmax_scale(d, p)
@@ -512,8 +537,8 @@ def prefill_head_selection(q_head_rows: np.ndarray, Kc_all: np.ndarray,
     for i in tiles:
         q_tile = q_head_rows[i * b:(i + 1) * b]
         C = i * b
-        Kc = Kc_all[:C // b]
-        s = prefill_tile_scores(q_tile, Kc, p) if C // b > 0 else np.zeros(0)
+        Kc = Kc_all[:context_rows(C, p)]
+        s = prefill_tile_scores(q_tile, Kc, p, C) if C // b > 0 else np.zeros(0)
         out[i] = select_topk(s, candidate_blocks(C, p), p.top_k)
     return out
 

@@ -422,6 +422,106 @@ def test_prefill_head_selection_matches_tiles_and_brute_force():
         assert sels[i].selected == sorted(j for _, j in brute[:3]), i
 
 
+def _prefill_ovl_brute(q, K, i, b, l, s_, scale):
+    """Tile scores of tile i by enumeration: for each complete context block
+    j, the max over the tile's rows and over the windows lying wholly inside
+    the context [0, i b) that share a key with the block, of the hand-summed
+    group logit against the window's hand-averaged keys."""
+    C = i * b
+    T, G, d = q.shape
+    rows = range(i * b, min((i + 1) * b, T))
+    out = []
+    for j in range(C // b):
+        block = set(range(j * b, (j + 1) * b))
+        best = -math.inf
+        for c in range(C):
+            keys = range(c * s_, c * s_ + l)
+            if c * s_ + l > C or not block.intersection(keys):
+                continue
+            mean = [sum(K[t, e] for t in keys) / l for e in range(d)]
+            for rr in rows:
+                best = max(best, scale * sum(sum(q[rr, g, e] for g in range(G)) * mean[e] for e in range(d)))
+        out.append(best)
+    return np.array(out)
+
+
+@pytest.mark.parametrize("b,l,s_", [(8, 6, 2), (8, 8, 4), (8, 4, 4), (16, 12, 4)])
+def test_prefill_overlap_tile_scores_brute_force(b, l, s_):
+    """Overlapping compression in a causal prefill (readings R2 and R18): the
+    oracle's tile scores and selections equal an enumeration over rows,
+    windows complete inside the tile's context and blocks; an exhaustive
+    sort with candidates by key enumeration gives the same sets."""
+    r_ = rng(62 + b + l + s_)
+    G, d = 2, 6
+    T = 9 * b + 3
+    K = r_.standard_normal((T, d))
+    V = r_.standard_normal((T, d))
+    q = r_.standard_normal((T, G, d))
+    p = orc.OracleParams(block_size=b, top_k=2, sink_keys=b, window_keys=b, pool="overlap",
+                         pool_stride=s_, pool_kernel=l, scale=0.5)
+    Kc_all = orc.compress(K, p)
+    nt = (T + b - 1) // b
+    sels = orc.prefill_head_selection(q, Kc_all, p, range(nt))
+    for i in range(1, nt):
+        C = i * b
+        ref = _prefill_ovl_brute(q, K, i, b, l, s_, 0.5)
+        got = orc.prefill_tile_scores(q[i * b:(i + 1) * b], Kc_all[:orc.context_rows(C, p)], p, C)
+        np.testing.assert_allclose(got, ref, atol=1e-12)
+        full = orc.prefill_tile(q[i * b:(i + 1) * b], K, V, i, p, Kc_all)
+        np.testing.assert_allclose(full["scores"], ref, atol=1e-12)
+        cand = [j for j in range(C // b)
+                if any(not (t < b or t >= C - b) for t in range(j * b, (j + 1) * b))]
+        brute = sorted(sorted(cand, key=lambda j: (-ref[j], j))[:2])
+        assert full["sel"].selected == brute == sels[i].selected, i
+
+
+def test_prefill_overlap_without_overlap_is_mean_prefill():
+    """l = s = b: one window per block, so the overlapping prefill gives the
+    block-mean prefill's scores, selections and outputs on every tile."""
+    w = WORKLOADS["prefill_64k"].scaled(n_q=64 * 11 + 9, num_q_heads=2, num_kv_heads=1, top_k=3, n_needles=2)
+    inp = make_inputs(w, seed=63)
+    q = inp["Q"][0, :, 0:2].double().numpy()
+    K = inp["K"][0, 0].double().numpy()
+    V = inp["V"][0, 0].double().numpy()
+    p_mean = P(w)
+    p_ovl = P(w, pool="overlap", pool_stride=64, pool_kernel=64)
+    Kc_m, Kc_o = orc.compress(K, p_mean), orc.compress(K, p_ovl)
+    for i in (1, 5, 8, 11):
+        rows = slice(i * 64, (i + 1) * 64)
+        a = orc.prefill_tile(q[rows], K, V, i, p_mean, Kc_m)
+        o = orc.prefill_tile(q[rows], K, V, i, p_ovl, Kc_o)
+        np.testing.assert_allclose(o["scores"], a["scores"], atol=1e-13)
+        assert o["sel"].selected == a["sel"].selected
+        np.testing.assert_allclose(o["O"], a["O"], atol=1e-13)
+
+
+def test_prefill_lsa_tile_scores_are_row_cosines():
+    """LSA pooling in a causal prefill (readings R2 and R7): each row's index
+    query is normalised, so scaling a row's group of queries by a positive
+    factor leaves the tile scores unchanged, every score is a cosine
+    against a unit centroid (|s| <= 1), a tile whose rows all point along
+    one centroid scores it 1, and a single-row tile equals the decode score
+    of that row."""
+    r_ = rng(64)
+    G, d, b = 2, 8, 16
+    T = 7 * b
+    K = r_.standard_normal((T, d))
+    q = r_.standard_normal((b, G, d))
+    p = orc.OracleParams(block_size=b, top_k=2, sink_keys=0, window_keys=0, pool="lsa", pool_stride=4)
+    Kc = orc.compress(K, p)[:6]
+    s = orc.prefill_tile_scores(q, Kc, p)
+    f = r_.uniform(0.1, 10.0, size=(b, 1, 1))
+    np.testing.assert_allclose(orc.prefill_tile_scores(q * f, Kc, p), s, atol=1e-13)
+    assert np.all(np.abs(s) <= 1 + 1e-12)
+    for j in range(6):
+        rows = [float(q[r].sum(0) @ Kc[j]) / math.sqrt(float(q[r].sum(0) @ q[r].sum(0))) for r in range(b)]
+        assert abs(s[j] - max(rows)) < 1e-12
+    along = np.repeat((3.0 * Kc[4] / G)[None, None], G, axis=1).repeat(b, axis=0)
+    assert abs(orc.prefill_tile_scores(along, Kc, p)[4] - 1.0) < 1e-12
+    np.testing.assert_allclose(orc.prefill_tile_scores(q[5:6], Kc, p),
+                               orc.block_scores(q[5].sum(0), Kc, p), atol=1e-15)
+
+
 # ------------------------------------------- overlapping compression ---
 
 _OVL_CASES = [(64, 32, 16, 320), (64, 32, 16, 333), (64, 64, 16, 300), (64, 16, 16, 256),
@@ -854,6 +954,13 @@ def test_planted_mistakes_are_caught(monkeypatch):
             m.setattr(orc, name, bad)
             assert _fails(ovl), name
     assert orig_b2c is orc.blocks_from_compressed
+    # prefill with overlapping windows: the context's windows counted like
+    # its blocks, or windows reaching past the context kept
+    for bad in (lambda C, p: C // p.block_size,
+                lambda C, p: (C - p.pool_stride) // p.pool_stride + 1 if p.pool == "overlap" else C // p.block_size):
+        with monkeypatch.context() as m:
+            m.setattr(orc, "context_rows", bad)
+            assert _fails(lambda: test_prefill_overlap_tile_scores_brute_force(8, 6, 2)), "context_rows"
     # Ward clustering: centroid distance without the size weights; every
     # bucket merging with its cheapest partner whether or not that is mutual;
     # the size cap ignored
