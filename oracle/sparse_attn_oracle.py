@@ -167,6 +167,8 @@ def pool_lsa(K: np.ndarray, b: int, stride: int = 4) -> np.ndarray:
     assert b % stride == 0
     K = np.asarray(K, dtype=np.float64)
     nb = K.shape[0] // b
+    if nb == 0:
+        return np.zeros((0, K.shape[1]))                            # no complete block (R5)
     khat = _normalise(K[:nb * b])                                   # (1)
     pool_keys = khat.reshape(nb * b // stride, stride, -1).sum(1)   # (2)
     per_block = b // stride

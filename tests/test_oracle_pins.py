@@ -422,6 +422,18 @@ def test_prefill_head_selection_matches_tiles_and_brute_force():
         assert sels[i].selected == sorted(j for _, j in brute[:3]), i
 
 
+@pytest.mark.parametrize("pool", ["mean", "lsa", "overlap"])
+def test_compress_without_a_complete_block_is_empty(pool):
+    """Fewer keys than one block (or one window) give no compressed key in
+    every pooling mode (reading R5: only complete blocks are compressed)."""
+    p = orc.OracleParams(block_size=64, top_k=1, sink_keys=0, window_keys=0, pool=pool,
+                         pool_stride=16 if pool == "overlap" else 4, pool_kernel=32 if pool == "overlap" else 0)
+    short = 31 if pool == "overlap" else 63
+    for T in (0, 1, short):
+        assert orc.compress(rng(65).standard_normal((T, 8)), p).shape == (0, 8)
+    assert orc.compress(rng(65).standard_normal((short + 1, 8)), p).shape == (1, 8)
+
+
 def _prefill_ovl_brute(q, K, i, b, l, s_, scale):
     """Tile scores of tile i by enumeration: for each complete context block
     j, the max over the tile's rows and over the windows lying wholly inside
