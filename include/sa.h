@@ -38,7 +38,8 @@
  *   Kc   : [B, Hkv, nb, d] float32, nb = number of complete blocks
  *          (decode: floor(ctx_len / b); prefill: floor(n_q / b));
  *          SA_POOL_OVERLAP: [B, Hkv, n_c, d], n_c = the number of complete
- *          windows = floor((ctx_len - l) / s) + 1 if ctx_len >= l, else 0
+ *          windows = floor((L - l) / s) + 1 if L >= l, else 0, with L =
+ *          ctx_len (decode) or n_q (prefill)
  *   idx  : decode / chunk: [B, Hkv, top_k] int32; prefill: [B, Hkv,
  *          n_tiles, top_k] int32 with n_tiles = ceil(n_q / b).  Block ids in
  *          ascending order, unused entries -1 at the end.
@@ -142,7 +143,7 @@ sa_status sa_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Step 1 (compression) for every complete block of the context:
  * SA_POOL_MEAN: Kc[j] = (1/b) sum_{t=jb}^{jb+b-1} K[t] (SparDA "方法");
- * SA_POOL_OVERLAP (decode / chunk only): Kc[c] = (1/l) sum_{t=cs}^{cs+l-1}
+ * SA_POOL_OVERLAP: Kc[c] = (1/l) sum_{t=cs}^{cs+l-1}
  *               K[t] for every complete window c (l = pool_kernel,
  *               s = pool_stride; SparDA "方法", overlapping compressed keys);
  * SA_POOL_LSA : Kc[j] = normalise(sum over the block's pool keys), a pool
@@ -170,11 +171,14 @@ sa_status sa_append_kv(const sa_params* p, const void* K_new, const void* V_new,
  * layouts).  scores (optional, may be NULL): fp32 block scores,
  * [B, Hkv, nb] for SA_SEL_QUERY0 or [B, Hkv, n_tiles, nb] for
  * SA_SEL_TILE_MAX.  Kc may be NULL when the context holds no complete
- * block.  SA_POOL_OVERLAP (SA_SEL_QUERY0 only): every window is scored as
- * above and block j takes the largest score among the complete windows
- * [cs, cs + l) that share a key with [jb, jb + b) (the coarse-to-fine step;
- * the pages do not fix the rule, the max is this library's reading);
- * scores then holds those block scores. */
+ * block.  SA_POOL_OVERLAP: every window is scored as above and block j
+ * takes the largest score among the complete windows [cs, cs + l) that
+ * share a key with [jb, jb + b) (the coarse-to-fine step; the pages do not
+ * fix the rule, the max is this library's reading); with SA_SEL_TILE_MAX a
+ * tile sees the windows complete inside its context (keys before the tile),
+ * each window taking the max over the tile's rows first.  scores then holds
+ * those block scores.  SA_POOL_LSA with SA_SEL_TILE_MAX: each row's index
+ * query is normalised, so the tile score is the largest row cosine. */
 sa_status sa_score_topk(const sa_params* p, const void* Q, const float* Kc,
                         int32_t* idx, float* scores, void* ws, size_t ws_bytes,
                         void* stream);
@@ -273,12 +277,15 @@ sa_status sa_column_attn(const sa_params* p, const void* Q, const void* K,
 int32_t sa_decode_launches(const sa_params* p);
 
 /* Steps 1-4 for a causal prefill (select == SA_SEL_TILE_MAX, ctx_len == 0,
- * n_q = T): pools K into Kc (caller-provided, [B, Hkv, floor(T/b), d] fp32),
- * scores every query tile of b rows against the compressed keys of the
- * blocks before it, selects per (tile, KV head) and runs causal sparse
+ * n_q = T): pools K into Kc (caller-provided, [B, Hkv, floor(T/b), d] fp32;
+ * SA_POOL_OVERLAP: [B, Hkv, n_c, d] as in the layouts), scores every query
+ * tile of b rows against the compressed keys before it (the tile max over
+ * its rows; LSA centroids by each row's cosine; overlapping windows as in
+ * sa_score_topk), selects per (tile, KV head) and runs causal sparse
  * attention: tile i attends sink U window U selected U its own keys
- * (causal).  Writes O, lse (optional), idx_out (optional).  SA_POOL_LSA
- * and SA_POOL_OVERLAP return SA_ERR_UNSUPPORTED here. */
+ * (causal).  Writes O, lse (optional), idx_out (optional).  Built for bf16,
+ * b = 64, Hq = 4 Hkv, sink and window multiples of 64 (else
+ * SA_ERR_UNSUPPORTED). */
 sa_status sa_sparse_attn_prefill(const sa_params* p, const void* Q,
                                  const void* K, const void* V, float* Kc,
                                  void* O, float* lse, int32_t* idx_out,

@@ -98,8 +98,9 @@ def test_overlap_validation_rejects(kw, status):
 @host_only
 def test_overlap_params_and_workspace():
     """pool_kernel must be 0 outside the overlap mode; the overlap mode runs
-    as two kernels (scoring, attention), its prefill is not built, and its
-    scoring workspace holds one score per window."""
+    as two kernels (scoring, attention), and its scoring workspace holds one
+    score per window, in decode and in prefill (per tile: the windows that
+    touch a complete block)."""
     p = _p()
     p.pool_kernel = 8
     assert _decode(p) == sa.SA_ERR_INVALID
@@ -108,7 +109,13 @@ def test_overlap_params_and_workspace():
     assert sa.raw_call("sa_decode_launches", ctypes.byref(_p())) in (1, 2)
     pf = _p(pool="overlap", pool_stride=16, pool_kernel=32, prefill=True, ctx_len=0, n_q=4096,
             num_q_heads=8, num_kv_heads=2)
-    assert sa.raw_call("sa_pool_keys", ctypes.byref(pf), FAKE, FAKE, None) == sa.SA_ERR_UNSUPPORTED
+    pf_mean = _p(prefill=True, ctx_len=0, n_q=4096, num_q_heads=8, num_kv_heads=2)
+    nt, nb = 4096 // 64, 4096 // 64
+    nc = min((4096 - 32) // 16 + 1, nb * 4)
+    for op in (sa.SA_OP_PREFILL, sa.SA_OP_SCORE_TOPK):
+        wm = sa.raw_call("sa_workspace_size", ctypes.byref(pf_mean), op)
+        wo = sa.raw_call("sa_workspace_size", ctypes.byref(pf), op)
+        assert wm > 0 and wo >= wm + 2 * (nt * 4 + 512) * (nc - nb) - 2048
     w_mean = sa.raw_call("sa_workspace_size", ctypes.byref(_p()), sa.SA_OP_SCORE_TOPK)
     w_ovl = sa.raw_call("sa_workspace_size", ctypes.byref(ov), sa.SA_OP_SCORE_TOPK)
     n_c = (4096 - 32) // 16 + 1

@@ -244,14 +244,19 @@ struct PrefillArgs {
   const void* Q;          // [B, T, Hq, 128] bf16
   const void* K;          // [B, Hkv, cap, 128] bf16
   const void* V;
-  const float* Kc;        // [B, Hkv, nb, 128] fp32
-  uint16_t* kc2;          // workspace: [B*Hkv, nb, 256] bf16 (hi | lo)
-  float* scores;          // workspace or caller: [B*Hkv, n_tiles, nb]
+  const float* Kc;        // [B, Hkv, kc_rows, 128] fp32 (blocks, or windows when ov_s > 0)
+  uint16_t* kc2;          // workspace: [B*Hkv, nc, 256] bf16 (hi | lo)
+  float* scores;          // scorer output [B*Hkv, n_tiles, nc]: workspace, or the caller's when nc is per block
+  float* bscores;         // overlapping windows: the caller's block scores [B*Hkv, n_tiles, nb] or null
   int32_t* idx;           // [B*Hkv, n_tiles, top_k]
   void* O;                // [B, T, Hq, 128]
   float* lse;             // [B, T, Hq] or null
   unsigned* status;
   int B, Hq, Hkv, T, nb, n_tiles, top_k, out_bf16, num_sms;
+  int nc;                 // compressed rows scored per pair: nb, or the windows that touch a complete block
+  int kc_rows;            // rows per pair of the caller's Kc
+  int lsa;                // LSA centroids: each query row normalised instead of scaled
+  int ov_s, ov_l;         // overlapping windows (stride, length), 0 otherwise
   int64_t cap, S, W;
   float scale;
 };

@@ -5,7 +5,13 @@
 // a 64-query tile are combined -- the reading taken is the max over rows):
 //   s[t][j] = max_{r in tile t} ( sum_g q_{r,g} ) . Kc_j * scale
 // for every candidate block j of tile t (complete, before the tile, not
-// wholly inside sink / window).
+// wholly inside sink / window).  LSA centroids (LSA review §2.3): each row's
+// index query is normalised instead of scaled, so s is a cosine.
+// Overlapping windows (SparDA "方法", overlapping compressed keys): the rows
+// of Kc are windows of l keys every s keys; the scorer takes the tile max of
+// every window complete inside the tile's context that touches a candidate
+// block, and the top-k kernel gives block j the max over the windows that
+// share a key with it.
 //
 // This is a dense contraction, so it runs on tcgen05 tensor cores.  The GEMM
 // is transposed -- M = 128 compressed keys (TMEM lanes), N = 128 query rows
@@ -46,32 +52,59 @@ constexpr int kND = 4;                         // TMEM accumulators of 128 colum
 
 struct PSArgs {
   const uint16_t* Q;        // [B, T, Hq, 128] bf16
-  float* scores;            // [P, n_tiles, nb]
+  float* scores;            // [P, n_tiles, nc]: per compressed row
+  float* bscores;           // overlapping windows: block scores [P, n_tiles, nb] or null
   unsigned* status;
   int B, Hq, Hkv, G, T, nb, n_tiles, n_tpairs, P;
+  int nc;                   // compressed rows per pair (blocks, or windows)
+  int lsa;                  // normalise each row's index query
+  int ov_s, ov_l;           // overlapping windows: stride and length (0: blocks)
   int64_t S, W;
   float scale;
 };
 
-// Candidate test of block j for query tile t (context C = 64 t).
-__device__ __forceinline__ bool is_candidate(const PSArgs& a, int t, int j) {
+// Candidate blocks of query tile t (context C = 64 t): [*j_lo, *j_hi), the
+// complete blocks that reach past the sink and start before the window
+// (none when *j_hi <= *j_lo).
+__device__ __forceinline__ void cand_range(const PSArgs& a, int t, int* j_lo, int* j_hi) {
   const int64_t C = static_cast<int64_t>(t) * kTile;
   const int64_t s_end = a.S < C ? a.S : C;
   const int64_t w_begin = (C - a.W) > s_end ? (C - a.W) : s_end;
-  const int64_t lo = static_cast<int64_t>(j) * kTile;
-  return j < a.nb && lo < w_begin && lo + kTile > s_end;
+  const int64_t jh = (w_begin + kTile - 1) / kTile;
+  *j_lo = static_cast<int>(s_end / kTile);
+  *j_hi = static_cast<int>(jh < a.nb ? jh : a.nb);
 }
 
-// Blocks [0, j_lim) contain every candidate of tiles 2n and 2n+1.
+// Windows complete inside the context of tile t.
+__device__ __forceinline__ int windows_in(const PSArgs& a, int t) {
+  const int C = t * kTile;
+  return C >= a.ov_l ? (C - a.ov_l) / a.ov_s + 1 : 0;
+}
+
+// Whether tile t needs the score of compressed row c: a candidate block, or
+// a window complete inside the tile's context that shares a key with one.
+__device__ __forceinline__ bool row_needed(const PSArgs& a, int t, int c) {
+  int j_lo, j_hi;
+  cand_range(a, t, &j_lo, &j_hi);
+  if (a.ov_s == 0) return c >= j_lo && c < j_hi;
+  const int64_t k0 = static_cast<int64_t>(c) * a.ov_s;
+  return j_hi > j_lo && c < windows_in(a, t) && k0 < static_cast<int64_t>(j_hi) * kTile &&
+         k0 + a.ov_l > static_cast<int64_t>(j_lo) * kTile;
+}
+
+// Rows [0, lim) hold every row tiles 2n and 2n+1 need; chunks of 128 of them.
 __device__ __forceinline__ int chunk_count(const PSArgs& a, int n) {
-  int t = min(2 * n + 1, a.n_tiles - 1);
-  const int64_t C = static_cast<int64_t>(t) * kTile;
-  const int64_t s_end = a.S < C ? a.S : C;
-  const int64_t w_begin = (C - a.W) > s_end ? (C - a.W) : s_end;
-  int64_t j_lim = (w_begin + kTile - 1) / kTile;
-  if (j_lim > a.nb) j_lim = a.nb;
-  if (j_lim * kTile <= s_end) return 0;      // no block reaches past the sink
-  return static_cast<int>((j_lim + 127) / 128);
+  const int t = min(2 * n + 1, a.n_tiles - 1);
+  int j_lo, j_hi;
+  cand_range(a, t, &j_lo, &j_hi);
+  if (j_hi <= j_lo) return 0;                // no block reaches past the sink
+  int lim = j_hi;
+  if (a.ov_s > 0) {
+    // windows starting before the last candidate block's end (s divides 64)
+    lim = min(windows_in(a, t), j_hi * (kTile / a.ov_s));
+  }
+  lim = min(lim, a.nc);
+  return (lim + 127) / 128;
 }
 
 // Work item k -> (tile pair n, pair p), most expensive first.
@@ -285,10 +318,20 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) v[e] += f[e];
           }
+          float mul = a.scale;
+          if (a.lsa) {
+            // the row's 128 columns sit on the 16 lanes of this half-warp
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss += v[e] * v[e];
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            mul = ss > 0.f ? rsqrtf(ss) : 0.f;
+          }
           uint32_t whi[4], wlo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float v0 = v[2 * e] * a.scale, v1 = v[2 * e + 1] * a.scale;
+            const float v0 = v[2 * e] * mul, v1 = v[2 * e + 1] * mul;
             whi[e] = pack_bf16x2(v0, v1);
             wlo[e] = pack_bf16x2(v0 - bf16lo(whi[e]), v1 - bf16hi(whi[e]));
           }
@@ -318,7 +361,7 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
           break;
         }
         tc::fence_after_sync();
-        const int j = 128 * m + 32 * q + lane;      // this thread's block
+        const int j = 128 * m + 32 * q + lane;      // this thread's compressed row
         float best[2];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -343,8 +386,8 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           const int t = 2 * n + half;
-          if (t < a.n_tiles && is_candidate(a, t, j))
-            a.scores[(static_cast<int64_t>(p) * a.n_tiles + t) * a.nb + j] = best[half];
+          if (t < a.n_tiles && row_needed(a, t, j))
+            a.scores[(static_cast<int64_t>(p) * a.n_tiles + t) * a.nc + j] = best[half];
         }
       }
     }
@@ -359,12 +402,14 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
   }
 }
 
-// Kc (fp32) -> [hi | lo] bf16 rows of 256 elements for the TMA loads.
-__global__ void kc_split_kernel(const float* Kc, uint16_t* out, int64_t rows) {
+// Kc (fp32, kc_rows rows per pair) -> [hi | lo] bf16 rows of 256 elements,
+// the first nc rows of every pair, for the TMA loads.
+__global__ void kc_split_kernel(const float* Kc, uint16_t* out, int64_t rows, int nc, int kc_rows) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;   // one float4 each
   if (i >= rows * 32) return;
   const int64_t r = i / 32, c = i % 32;
-  const float4 x = reinterpret_cast<const float4*>(Kc)[i];
+  const int64_t pr = r / nc, row = r - pr * nc;
+  const float4 x = reinterpret_cast<const float4*>(Kc + (pr * kc_rows + row) * kHeadDim)[c];
   const float v[4] = {x.x, x.y, x.z, x.w};
   uint16_t hi[4], lo[4];
 #pragma unroll
@@ -386,17 +431,32 @@ __global__ void __launch_bounds__(256, 2) prefill_topk_kernel(PSArgs a, int top_
   if (row >= static_cast<int64_t>(a.P) * a.n_tiles) return;
   const int t = static_cast<int>(row % a.n_tiles);
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw) + warp * a.nb;
-  const float* sc = a.scores + row * a.nb;
+  const float* sc = a.scores + row * a.nc;
   // blocks at or after the tile are never candidates
   const int nb_t = min(a.nb, t);
-  // the candidates of tile t (context C = 64 t) are blocks [j_lo, j_hi): past
-  // the sink, starting before the window (the test of is_candidate)
-  const int64_t C = static_cast<int64_t>(t) * kTile;
-  const int64_t s_end = a.S < C ? a.S : C;
-  const int64_t w_begin = (C - a.W) > s_end ? (C - a.W) : s_end;
-  const int j_lo = static_cast<int>(s_end / kTile);
-  const int j_hi = min(nb_t, static_cast<int>((w_begin + kTile - 1) / kTile));
-  for (int j0 = 0; j0 < nb_t; j0 += 32 * 32) {
+  int j_lo, j_hi;
+  cand_range(a, t, &j_lo, &j_hi);
+  j_hi = min(j_hi, nb_t);
+  if (a.ov_s > 0) {
+    // block j: the max over the windows complete inside the context that
+    // share a key with it, c s + l > 64 j and c s < 64 (j + 1); every
+    // candidate has one (the window starting at its first key)
+    const int s = a.ov_s, l = a.ov_l, last = windows_in(a, t) - 1;
+    for (int j = lane; j < nb_t; j += 32) {
+      uint32_t key = 0u;
+      if (j >= j_lo && j < j_hi) {
+        const int ca = j * kTile - l >= 0 ? (j * kTile - l) / s + 1 : 0;
+        const int cb = min(last, ((j + 1) * kTile - 1) / s);
+        float m = -CUDART_INF_F;
+        for (int c = ca; c <= cb; ++c) m = fmaxf(m, __ldcg(sc + c));
+        if (a.bscores) a.bscores[row * a.nb + j] = m;
+        key = float_key(m);
+        key = key == 0u ? 1u : key;
+      }
+      keys[j] = key;
+    }
+  }
+  for (int j0 = 0; a.ov_s == 0 && j0 < nb_t; j0 += 32 * 32) {
     float v[32];
 #pragma unroll
     for (int u = 0; u < 32; ++u) {
@@ -442,6 +502,7 @@ cudaError_t launch_prefill_score(const PrefillArgs& pa, cudaStream_t s) {
   PSArgs a = {};
   a.Q = static_cast<const uint16_t*>(pa.Q);
   a.scores = pa.scores;
+  a.bscores = pa.bscores;
   a.status = pa.status;
   a.B = pa.B;
   a.Hq = pa.Hq;
@@ -449,21 +510,26 @@ cudaError_t launch_prefill_score(const PrefillArgs& pa, cudaStream_t s) {
   a.G = pa.Hq / pa.Hkv;
   a.T = pa.T;
   a.nb = pa.nb;
+  a.nc = pa.nc;
+  a.lsa = pa.lsa;
+  a.ov_s = pa.ov_s;
+  a.ov_l = pa.ov_l;
   a.n_tiles = pa.n_tiles;
   a.n_tpairs = (pa.n_tiles + 1) / 2;
   a.P = pa.B * pa.Hkv;
   a.S = pa.S;
   a.W = pa.W;
   a.scale = pa.scale;
-  if (a.nb > 0) {
+  if (a.nc > 0) {
     // Kc -> hi / lo bf16
-    const int64_t rows = static_cast<int64_t>(a.P) * a.nb;
-    kc_split_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, s>>>(pa.Kc, pa.kc2, rows);
+    const int64_t rows = static_cast<int64_t>(a.P) * a.nc;
+    kc_split_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, s>>>(pa.Kc, pa.kc2, rows, a.nc,
+                                                                                    pa.kc_rows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     CUtensorMap map;
-    cuuint64_t dims[3] = {256, static_cast<cuuint64_t>(a.nb), static_cast<cuuint64_t>(a.P)};
-    cuuint64_t strides[2] = {256 * 2, static_cast<cuuint64_t>(a.nb) * 256 * 2};
+    cuuint64_t dims[3] = {256, static_cast<cuuint64_t>(a.nc), static_cast<cuuint64_t>(a.P)};
+    cuuint64_t strides[2] = {256 * 2, static_cast<cuuint64_t>(a.nc) * 256 * 2};
     cuuint32_t box[3] = {64, 128, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, pa.kc2, dims, strides, box, estr,

@@ -270,6 +270,9 @@ DecodeAttnArgs attn_args(const sa_params* p, const DecodeGeom& g, const DecodePl
 // ---- prefill -------------------------------------------------------------------
 struct PrefillGeom {
   int B, Hq, Hkv, G, T, nb, n_tiles, P;
+  int nc;          // compressed rows scored per pair (blocks, or windows touching a complete block)
+  int kc_rows;     // rows per pair of the caller's Kc
+  int ov_s, ov_l;  // overlapping windows, 0 otherwise
   int64_t cap;
 };
 
@@ -281,7 +284,6 @@ sa_status check_prefill(const sa_params* p, PrefillGeom* g) {
   if (p->block_size != 64) return fail(SA_ERR_UNSUPPORTED, "prefill is built for block_size 64 (= query tile)");
   if (p->sink_keys % 64 != 0 || p->window_keys % 64 != 0)
     return fail(SA_ERR_UNSUPPORTED, "prefill needs sink_keys and window_keys to be multiples of 64");
-  if (p->pool != SA_POOL_MEAN) return fail(SA_ERR_UNSUPPORTED, "prefill scoring is built for mean pooling");
   g->B = p->batch;
   g->Hq = p->num_q_heads;
   g->Hkv = p->num_kv_heads;
@@ -291,6 +293,16 @@ sa_status check_prefill(const sa_params* p, PrefillGeom* g) {
   g->n_tiles = (p->n_q + 63) / 64;
   g->P = p->batch * p->num_kv_heads;
   g->cap = p->kv_capacity;
+  g->nc = g->kc_rows = g->nb;
+  g->ov_s = g->ov_l = 0;
+  if (p->pool == SA_POOL_OVERLAP) {
+    // windows starting at or past the last complete block's end touch no
+    // complete block (s divides b)
+    g->ov_s = p->pool_stride;
+    g->ov_l = p->pool_kernel;
+    g->kc_rows = g->T >= g->ov_l ? (g->T - g->ov_l) / g->ov_s + 1 : 0;
+    g->nc = std::min(g->kc_rows, g->nb * (64 / g->ov_s));
+  }
   if (g->nb > 6144) return fail(SA_ERR_UNSUPPORTED, "prefill is built for sequences up to 393216 tokens");
   if (static_cast<int64_t>(g->B) * g->T > 0x7fffffff) return fail(SA_ERR_UNSUPPORTED, "too many tokens");
   return SA_OK;
@@ -310,8 +322,8 @@ PrefillWs prefill_ws(const PrefillGeom& g, int top_k, int op, int idx_len) {
   };
   const size_t rows = static_cast<size_t>(g.P) * g.n_tiles;
   if (op == SA_OP_PREFILL || op == SA_OP_SCORE_TOPK) {
-    w.kc2 = take(static_cast<size_t>(g.P) * g.nb * 512);
-    w.scores = take(rows * g.nb * 4);
+    w.kc2 = take(static_cast<size_t>(g.P) * g.nc * 512);
+    w.scores = take(rows * g.nc * 4);
   }
   if (op == SA_OP_PREFILL) w.idx = take(rows * static_cast<size_t>(top_k) * 4);
   if (op == SA_OP_GIVEN_IDX) w.clean = take(rows * static_cast<size_t>(idx_len) * 4);
@@ -326,6 +338,11 @@ PrefillArgs prefill_args(const sa_params* p, const PrefillGeom& g) {
   a.Hkv = g.Hkv;
   a.T = g.T;
   a.nb = g.nb;
+  a.nc = g.nc;
+  a.kc_rows = g.kc_rows;
+  a.lsa = p->pool == SA_POOL_LSA;
+  a.ov_s = g.ov_s;
+  a.ov_l = g.ov_l;
   a.n_tiles = g.n_tiles;
   a.top_k = p->top_k;
   a.out_bf16 = p->out_dtype == SA_BF16;
@@ -576,8 +593,6 @@ sa_status sa_pool_keys(const sa_params* p, const void* K, float* Kc, void* strea
   const bool prefill = p && p->select == SA_SEL_TILE_MAX;
   sa_status st = check_params(p, prefill);
   if (st != SA_OK) return st;
-  if (prefill && p->pool == SA_POOL_OVERLAP)
-    return fail(SA_ERR_UNSUPPORTED, "overlapping windows are built for decode and draft chunks");
   const int64_t keys = prefill ? static_cast<int64_t>(p->n_q) : p->ctx_len;
   const bool ovl = p->pool == SA_POOL_OVERLAP;
   const int64_t rows = ovl ? (keys >= p->pool_kernel ? (keys - p->pool_kernel) / p->pool_stride + 1 : 0)
@@ -616,7 +631,14 @@ sa_status sa_score_topk(const sa_params* p, const void* Q, const float* Kc, int3
     a.Q = Q;
     a.Kc = Kc;
     a.kc2 = reinterpret_cast<uint16_t*>(w + L.kc2);
-    a.scores = scores ? scores : reinterpret_cast<float*>(w + L.scores);
+    // per-block scores go straight to the caller's buffer; window scores
+    // stay in the workspace and the caller gets the block scores
+    if (g.ov_s > 0) {
+      a.scores = reinterpret_cast<float*>(w + L.scores);
+      a.bscores = scores;
+    } else {
+      a.scores = scores ? scores : reinterpret_cast<float*>(w + L.scores);
+    }
     a.idx = idx;
     a.status = reinterpret_cast<unsigned*>(w);
     cudaError_t e = launch_prefill_score(a, static_cast<cudaStream_t>(stream));
