@@ -22,7 +22,10 @@
 // V as 64-row x 128-byte boxes, two d-halves per tile, into a 3-stage ring of
 // 64 KB units; rows at or past the end of the cache are zero-filled by the
 // tensor map), warp 1 TMEM owner and MMA issuer, warps 2-5 softmax and
-// epilogue.  TMEM columns: S in [0,16) / [16,32) by unit parity, O^T in
+// epilogue.  With 9-16 rows (draft chunks, dense verify) warps 6-9 join as a
+// second softmax warpgroup: warps w and w + 4 share a TMEM lane quarter (the
+// same keys) and take rows 0-7 and 8-15, which halves each unit's softmax
+// chain.  TMEM columns: S in [0,16) / [16,32) by unit parity, O^T in
 // [32,48) / [48,64) by pair parity.  All waits are bounded.
 #include <cudaTypedefs.h>
 #include <math_constants.h>
@@ -46,6 +49,7 @@ constexpr int kQBuf = 2 * kN * 128;             // two d-halves of 16 rows x 128
 constexpr int kPBuf = 2 * kN * 128;             // two key-halves of 16 rows x 128 B
 constexpr int kThreads = 192;
 constexpr int kThreadsFused = 256;              // fused: warps 6-7 select the top-k
+constexpr int kThreadsSplit = 320;              // 9-16 rows: warps 6-9 are a second softmax warpgroup
 constexpr int kSoftThreads = 128;
 constexpr int kSelBarThreads = 192;             // softmax warps + selection warps
 constexpr int kNumBars = 22;
@@ -70,6 +74,21 @@ __device__ __forceinline__ float float_of_key(uint32_t k) {
 __device__ __forceinline__ void softmax_bar() {
   asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
 }
+// Split rows: barrier 1 (warps 2-5) or 3 (warps 6-9) for one warpgroup's
+// rows, barrier 4 for both warpgroups.
+__device__ __forceinline__ void group_bar(int grp) {
+  asm volatile("bar.sync %0, %1;" ::"r"(grp ? 3 : 1), "r"(kSoftThreads) : "memory");
+}
+__device__ __forceinline__ void groups_bar() {
+  asm volatile("bar.sync 4, %0;" ::"r"(2 * kSoftThreads) : "memory");
+}
+
+// Threads of an instantiation, and whether its softmax rows are split over
+// two warpgroups.
+template <int NR, bool FUSED>
+constexpr bool kSplitRows = NR == 16 && !FUSED;
+template <int NR, bool FUSED>
+constexpr int kThreadsOf = FUSED ? kThreadsFused : (kSplitRows<NR, FUSED> ? kThreadsSplit : kThreads);
 // The same barrier, returning whether any of the softmax threads passed true.
 __device__ __forceinline__ bool softmax_bar_or(bool v) {
   uint32_t r;
@@ -205,7 +224,7 @@ __device__ __forceinline__ void store_out4(void* O, int64_t idx, float4 v, float
 // for the flag of every pair before reading its table.  A cooperative launch
 // keeps every CTA resident, so the waits end.
 template <bool OUT_BF16, int NR, bool FUSED, bool MASS>
-__global__ void __launch_bounds__(kThreadsFused, 1)
+__global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                      const __grid_constant__ CUtensorMap v_map, DecodeAttnArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -259,11 +278,11 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       mbar_init(&q_full[b], 1);
       mbar_init(&q_empty[b], 1);
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], kSoftThreads);
-      mbar_init(&p_full[b], kSoftThreads);
+      mbar_init(&s_free[b], kSplitRows<NR, FUSED> ? 2 * kSoftThreads : kSoftThreads);
+      mbar_init(&p_full[b], kSplitRows<NR, FUSED> ? 2 * kSoftThreads : kSoftThreads);
       mbar_init(&p_free[b], 1);
       mbar_init(&o_full[b], 1);
-      mbar_init(&o_free[b], kSoftThreads);
+      mbar_init(&o_free[b], kSplitRows<NR, FUSED> ? 2 * kSoftThreads : kSoftThreads);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -275,7 +294,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
   {
     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
     uint4* qp = reinterpret_cast<uint4*>(Qs);
-    for (int i = threadIdx.x; i < (2 * kQBuf + 2 * kPBuf) / 16; i += kThreads) qp[i] = z;
+    for (int i = threadIdx.x; i < (2 * kQBuf + 2 * kPBuf) / 16; i += blockDim.x) qp[i] = z;
     tc::fence_proxy_async_smem();
   }
   if (warp == 1) {
@@ -540,16 +559,30 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     // ------------------------------------------------- softmax and epilogue
     const int qq = warp & 3;                  // TMEM lane quarter of this warp
     const int t = qq * 32 + lane;             // key slot of the unit; output column d in the epilogue
+    constexpr bool SPLIT = kSplitRows<NR, FUSED>;
+    constexpr int NH = SPLIT ? NR / 2 : NR;   // rows of this thread's warpgroup
+    const int grp = SPLIT ? (warp - 2) >> 2 : 0;
+    const int rb = grp * NH;                  // its first row
+    // one warpgroup's barrier (its rows' maxima and sums), and the barrier of
+    // every softmax thread (the pair's ticket)
+    auto gbar = [&]() {
+      if constexpr (SPLIT) group_bar(grp);
+      else softmax_bar();
+    };
+    auto abar = [&]() {
+      if constexpr (SPLIT) groups_bar();
+      else softmax_bar();
+    };
     const uint32_t tl = tbase + (static_cast<uint32_t>(qq * 32) << 16);
     const int R = a.R, G = a.G;
     const int C = static_cast<int>(a.C);
     const float qscale = a.qscale;
     const int tile = t >> 6, kc = t & 63;
     // byte offsets of this key's P^T entries (row r, key kc of its 64-key half)
-    uint32_t poff[NR];
+    uint32_t poff[NH];
 #pragma unroll
-    for (int r = 0; r < NR; ++r) poff[r] = tile * (kN * 128) + tc::sw128_off(r, kc >> 3) + (kc & 7) * 2;
-    float m_run[NR], l_t[NR];
+    for (int r = 0; r < NH; ++r) poff[r] = tile * (kN * 128) + tc::sw128_off(rb + r, kc >> 3) + (kc & 7) * 2;
+    float m_run[NH], l_t[NH];
     RunCursor pc;
     pc.init(a.ord, i0, nI, d0, nunits);
     bool ok = true;
@@ -557,34 +590,34 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     auto epilogue = [&]() -> bool {
       // row sums over the unit's 128 key slots
       float mine = 0.f;
-      if constexpr (NR >= 8) {
-        float lt[NR];
+      if constexpr (NH >= 8) {
+        float lt[NH];
 #pragma unroll
-        for (int r = 0; r < NR; ++r) lt[r] = l_t[r];
-        mine = rows_reduce<NR, false>(lt, lane);
+        for (int r = 0; r < NH; ++r) lt[r] = l_t[r];
+        mine = rows_reduce<NH, false>(lt, lane);
       } else {
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
+        for (int r = 0; r < NH; ++r) {
           float v = l_t[r];
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
           mine = (lane == r) ? v : mine;
         }
       }
-      if (lane < NR) lsum[lane * 4 + qq] = mine;
+      if (lane < NH) lsum[(rb + lane) * 4 + qq] = mine;
       const int pkk = pc.ordinal, ob = pkk & 1;
       if (!mbar_wait_bounded(&o_full[ob], (pkk >> 1) & 1, abort_flag)) return false;
       tc::fence_after_sync();
-      float ov[NR];
-      tmem_ldn<NR>(tl + 32 + ob * kN, ov);
+      float ov[NH];
+      tmem_ldn<NH>(tl + 32 + ob * kN + rb, ov);
       tc::tmem_wait_ld();
       tc::fence_before_sync();
       mbar_arrive(&o_free[ob]);
-      softmax_bar();
-      float L[NR];
+      gbar();
+      float L[NH];
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        const float4 v = reinterpret_cast<const float4*>(lsum)[r];
+      for (int r = 0; r < NH; ++r) {
+        const float4 v = reinterpret_cast<const float4*>(lsum)[rb + r];
         L[r] = (v.x + v.y) + (v.z + v.w);
       }
       const int64_t pair = pc.pair;
@@ -597,9 +630,9 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       };
       if (n_ctas == 1) {
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
-          if (r < R) {
-            const int64_t orow = out_row(r);
+        for (int r = 0; r < NH; ++r) {
+          if (rb + r < R) {
+            const int64_t orow = out_row(rb + r);
             store_out<OUT_BF16>(a.O, orow * kHeadDim + t, ov[r] * (L[r] > 0.f ? 1.f / L[r] : 0.f));
             if (t == r && a.lse)
               a.lse[orow] = L[r] > 0.f ? (m_run[r] + log2f(L[r])) * 0.69314718055994531f : -CUDART_INF_F;
@@ -607,9 +640,9 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         }
       } else {
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
-          if (r < R) {
-            const int64_t ps = (pair * a.n_slots + slot) * a.R4 + r;
+        for (int r = 0; r < NH; ++r) {
+          if (rb + r < R) {
+            const int64_t ps = (pair * a.n_slots + slot) * a.R4 + rb + r;
             a.part_O[ps * kHeadDim + t] = ov[r];
             if (t == r) {
               a.part_ml[ps * 2 + 0] = m_run[r];
@@ -619,20 +652,21 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         }
         // the barrier orders every thread's partial stores before thread 0's
         // release fence and ticket
-        softmax_bar();
-        if (t == 0) {
+        abar();
+        if (t == 0 && grp == 0) {
           __threadfence();
           const unsigned tk = atomicAdd(&a.counters[pair], 1u);
           *ticket = (tk == static_cast<unsigned>(n_ctas - 1));
         }
-        softmax_bar();
+        abar();
         if (*ticket) {
           __threadfence();
-          // thread t merges columns 4 (t % 32) .. + 3 of rows t / 32 + 4 k;
-          // the loads of up to SG slots are all in flight before their use
-          constexpr int KR = NR / 4;
-          constexpr int SG = NR >= 16 ? 2 : 4;
-          const int c4 = (t & 31) * 4, r0w = t >> 5;
+          // thread t merges columns 4 (t % 32) .. + 3 of its warpgroup's rows
+          // t / 32 + 4 k; the loads of up to SG slots are all in flight
+          // before their use
+          constexpr int KR = NH / 4;
+          constexpr int SG = NH >= 16 ? 2 : 4;
+          const int c4 = (t & 31) * 4, r0w = rb + (t >> 5);
           float Mx[KR], Ls[KR];
           float4 acc[KR];
 #pragma unroll
@@ -693,10 +727,10 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
                 a.lse[orow] = Ls[k] > 0.f ? (Mx[k] + log2f(Ls[k])) * 0.69314718055994531f : -CUDART_INF_F;
             }
           }
-          if (t == 0) a.counters[pair] = 0u;
+          if (t == 0 && grp == 0) a.counters[pair] = 0u;
         }
       }
-      softmax_bar();     // lsum and the ticket are reused by the next pair
+      abar();            // lsum and the ticket are reused by the next pair
       return true;
     };
 
@@ -794,7 +828,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       const bool fi = pc.first(i);
       if (fi) {
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
+        for (int r = 0; r < NH; ++r) {
           m_run[r] = -CUDART_INF_F;
           l_t[r] = 0.f;
         }
@@ -806,8 +840,8 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         break;
       }
       tc::fence_after_sync();
-      float sv[NR];
-      tmem_ldn<NR>(tl + sb * kN, sv);
+      float sv[NH];
+      tmem_ldn<NH>(tl + sb * kN + rb, sv);
       tc::tmem_wait_ld();
       tc::fence_before_sync();
       mbar_arrive(&s_free[sb]);
@@ -821,61 +855,62 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       const int dnew = static_cast<int>(tile ? info[s].ks1 : info[s].ks0) + kc - C;   // >= 0: a new key
       const int dn = dnew < 0 ? -1 : min(dnew, 64);
       const bool kv = kc < n;
-      float x[NR];
+      float x[NH];
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        // new key C + dnew is seen by token r / G iff dnew <= r / G, i.e. dnew * G <= r
-        const bool v = kv && r < R && (dn < 0 || dn * G <= r);
+      for (int r = 0; r < NH; ++r) {
+        // new key C + dnew is seen by token row / G iff dnew <= row / G, i.e. dnew * G <= row
+        const int row = rb + r;
+        const bool v = kv && row < R && (dn < 0 || dn * G <= row);
         x[r] = v ? sv[r] * qscale : -CUDART_INF_F;
       }
       // unit max of every row: warp reduction, then the four warps through
       // shared memory (row r of this warp stored by lane r)
       float* wm = wmax + sb * (kN * 4);
-      if constexpr (NR >= 8) {
-        float xm[NR];
+      if constexpr (NH >= 8) {
+        float xm[NH];
 #pragma unroll
-        for (int r = 0; r < NR; ++r) xm[r] = x[r];
-        const float mx = rows_reduce<NR, true>(xm, lane);
-        if (lane < NR) wm[lane * 4 + qq] = mx;
+        for (int r = 0; r < NH; ++r) xm[r] = x[r];
+        const float mx = rows_reduce<NH, true>(xm, lane);
+        if (lane < NH) wm[(rb + lane) * 4 + qq] = mx;
       } else {
         uint32_t mk = 0u;
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
+        for (int r = 0; r < NH; ++r) {
           const uint32_t k = __reduce_max_sync(0xffffffffu, float_key(x[r]));
           mk = (lane == r) ? k : mk;
         }
-        if (lane < NR) wm[lane * 4 + qq] = float_of_key(mk);
+        if (lane < NH) wm[(rb + lane) * 4 + qq] = float_of_key(mk);
       }
-      softmax_bar();
-      float alpha[NR];
+      gbar();
+      float alpha[NH];
       bool grow_any = false;
-      if constexpr (NR >= 8) {
-        // lane l combines row l % NR alone (the unit max over the four
+      if constexpr (NH >= 8) {
+        // lane l combines row l % NH alone (the unit max over the four
         // warps, the growth test, the factor); every lane then takes the
         // rows from their lanes
-        const int rr = lane & (NR - 1);
-        const float4 w4 = reinterpret_cast<const float4*>(wm)[rr];
+        const int rr = lane & (NH - 1);
+        const float4 w4 = reinterpret_cast<const float4*>(wm)[rb + rr];
         const float M = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
         float mo = m_run[0];
 #pragma unroll
-        for (int r = 1; r < NR; ++r) mo = (rr == r) ? m_run[r] : mo;
+        for (int r = 1; r < NH; ++r) mo = (rr == r) ? m_run[r] : mo;
         const bool grow = M > mo + kLazy;
         const float al = grow ? ex2(mo - M) : 1.f;     // 0 for the first keys of a row
         const float mn = grow ? M : mo;
         grow_any = __any_sync(0xffffffffu, grow);
 #pragma unroll
-        for (int r = 0; r < NR; ++r) m_run[r] = __shfl_sync(0xffffffffu, mn, r);
+        for (int r = 0; r < NH; ++r) m_run[r] = __shfl_sync(0xffffffffu, mn, r);
         if (grow_any) {
 #pragma unroll
-          for (int r = 0; r < NR; ++r) alpha[r] = __shfl_sync(0xffffffffu, al, r);
+          for (int r = 0; r < NH; ++r) alpha[r] = __shfl_sync(0xffffffffu, al, r);
         } else {
 #pragma unroll
-          for (int r = 0; r < NR; ++r) alpha[r] = 1.f;
+          for (int r = 0; r < NH; ++r) alpha[r] = 1.f;
         }
       } else {
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
-          const float4 w4 = reinterpret_cast<const float4*>(wm)[r];
+        for (int r = 0; r < NH; ++r) {
+          const float4 w4 = reinterpret_cast<const float4*>(wm)[rb + r];
           const float M = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
           const bool grow = M > m_run[r] + kLazy;
           alpha[r] = grow ? ex2(m_run[r] - M) : 1.f;     // 0 for the first keys of a row
@@ -892,18 +927,18 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
             break;
           }
           tc::fence_after_sync();
-          float ov[NR];
-          const uint32_t to = tl + 32 + (pc.ordinal & 1) * kN;
-          tmem_ldn<NR>(to, ov);
+          float ov[NH];
+          const uint32_t to = tl + 32 + (pc.ordinal & 1) * kN + rb;
+          tmem_ldn<NH>(to, ov);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int r = 0; r < NR; ++r) ov[r] *= alpha[r];
-          tmem_stn<NR>(to, ov);
+          for (int r = 0; r < NH; ++r) ov[r] *= alpha[r];
+          tmem_stn<NH>(to, ov);
           tc::tmem_wait_st();
           tc::fence_before_sync();
         }
 #pragma unroll
-        for (int r = 0; r < NR; ++r) l_t[r] *= alpha[r];
+        for (int r = 0; r < NH; ++r) l_t[r] *= alpha[r];
       }
       // P^T into this unit's P buffer once PV(i-2) has read it
       if (i >= 2 && !mbar_wait_bounded(&p_free[sb], ((i >> 1) + 1) & 1, abort_flag)) {
@@ -911,9 +946,9 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         break;
       }
       unsigned char* pbuf = Ps + sb * kPBuf;
-      float pm[NR];
+      float pm[NH];
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
+      for (int r = 0; r < NH; ++r) {
         const float p = ex2(x[r] - (m_run[r] == -CUDART_INF_F ? 0.f : m_run[r]));
         pm[r] = p;
         l_t[r] += p;
@@ -925,17 +960,21 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         // dense verify: this warp's 32 keys, when they are keys of the tile
         // (an empty tile has no key range) and lie in the complete blocks
         // (the dense mode's tiles start at multiples of 64): each row's
-        // probability sum, reduce-scattered so that lane r holds row r
+        // probability sum, reduce-scattered so that lane r holds the
+        // warpgroup's row r (16 rows: lanes 0-15; at most 8: lanes 0-7)
         const int64_t k32 = kst + (qq & 1) * 32;
         if (n >= (qq & 1) * 32 + 32 && k32 + 32 <= a.mass_keys) {
-          float d[16];
-#pragma unroll
-          for (int u = 0; u < 16; ++u) d[u] = u < NR ? pm[u] : 0.f;
+          constexpr int W = NH > 8 ? 16 : 8;
           const bool b3 = lane & 8, b2 = lane & 4, b1 = lane & 2, b0 = lane & 1;
           float e8[8], e4[4], e2[2];
+          if constexpr (W == 16) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            e8[u] = (b3 ? d[u + 8] : d[u]) + __shfl_xor_sync(0xffffffffu, b3 ? d[u] : d[u + 8], 8);
+            for (int u = 0; u < 8; ++u)
+              e8[u] = (b3 ? pm[u + 8] : pm[u]) + __shfl_xor_sync(0xffffffffu, b3 ? pm[u] : pm[u + 8], 8);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) e8[u] = u < NH ? pm[u < NH ? u : 0] : 0.f;
+          }
 #pragma unroll
           for (int u = 0; u < 4; ++u)
             e4[u] = (b2 ? e8[u + 4] : e8[u]) + __shfl_xor_sync(0xffffffffu, b2 ? e8[u] : e8[u + 4], 4);
@@ -943,13 +982,14 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
           for (int u = 0; u < 2; ++u)
             e2[u] = (b1 ? e4[u + 2] : e4[u]) + __shfl_xor_sync(0xffffffffu, b1 ? e4[u] : e4[u + 2], 2);
           float e1 = (b0 ? e2[1] : e2[0]) + __shfl_xor_sync(0xffffffffu, b0 ? e2[0] : e2[1], 1);
+          if constexpr (W == 8) e1 += __shfl_xor_sync(0xffffffffu, e1, 8);
           e1 += __shfl_xor_sync(0xffffffffu, e1, 16);
-          const int r = lane & 15;
+          const int r = lane & (W - 1);
           float mr = 0.f;
 #pragma unroll
-          for (int u = 0; u < NR; ++u) mr = (u == r && m_run[u] != -CUDART_INF_F) ? m_run[u] : mr;
-          if (lane < 16 && r < R)
-            a.mass_part[(pc.pair * a.mass_hts + k32 / 32) * 16 + r] = make_float2(e1, mr);
+          for (int u = 0; u < NH; ++u) mr = (u == r && m_run[u] != -CUDART_INF_F) ? m_run[u] : mr;
+          if (lane < W && r < NH && rb + r < R)
+            a.mass_part[(pc.pair * a.mass_hts + k32 / 32) * 16 + rb + r] = make_float2(e1, mr);
         }
       }
       if (pc.last(i) && !epilogue()) {
@@ -1073,6 +1113,9 @@ cudaError_t launch_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf1
   CUtensorMap qm, km, vm;
   if (!encode_maps(a, &qm, &km, &vm)) return cudaErrorInvalidValue;
   void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, DecodeAttnArgs);
+  // more than 8 rows: the 16-row instantiations, whose softmax rows are split
+  // over two warpgroups
+  const unsigned threads = FUSED ? kThreadsFused : (a.R > 8 ? kThreadsOf<16, false> : kThreads);
   if (!FUSED && a.mass_part) {
     // dense verify: the row sums of the complete blocks ride along
     if (a.R <= 4) kern = out_bf16 ? decode_tc_kernel<true, 4, false, true> : decode_tc_kernel<false, 4, false, true>;
@@ -1092,7 +1135,7 @@ cudaError_t launch_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf1
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.ord.grid);
-  cfg.blockDim = dim3(FUSED ? kThreadsFused : kThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
