@@ -212,6 +212,9 @@ def test_given_idx_with_oracle_indices(name, over):
     ("decode_32k", dict(batch=2)),
     ("draft_chunk_16k", dict(batch=2)),
     ("decode_1m", dict(batch=1, ctx_len=512 * 200, num_kv_heads=2, num_q_heads=8)),
+    # LSA centroids past 512 blocks (scoring kernel, then attention)
+    ("decode_1m", dict(batch=2, ctx_len=512 * 1500 + 77, num_kv_heads=4, num_q_heads=16)),
+    ("decode_1m", dict(batch=1, ctx_len=512 * 2000 + 300, num_kv_heads=1, num_q_heads=4, top_k=8)),
     # 8 and 16 query rows per KV head (n_q tokens x G heads): the tensor-core
     # kernel's other row-count instantiations
     ("draft_chunk_16k", dict(batch=3, n_q=2, num_q_heads=32, num_kv_heads=8, ctx_len=4096 + 77)),
@@ -405,13 +408,56 @@ def test_fused_empty_tiles_after_score_chunks():
 
 def test_decode_32k_runs_as_one_launch():
     """The batched-decode workload takes the fused path (scores, top-k and
-    attention in one cooperative launch) on this device; draft chunks (12
-    query rows per KV head), more than two pairs per SM, fp32 and LSA
-    centroids take the scoring kernel and then the attention kernel."""
+    attention in one cooperative launch) on this device, and so does LSA
+    pooling up to 512 blocks; draft chunks (12 query rows per KV head), more
+    than two pairs per SM, fp32, overlapping windows and more than 512
+    blocks (the 1M-token workload) take the scoring kernel and then the
+    attention kernel."""
     n = lambda w: sa.decode_launches(sa.params_for(w))
     assert n(WORKLOADS["decode_32k"]) == 1
     assert n(WORKLOADS["draft_chunk_16k"]) == 2
     assert n(WORKLOADS["draft_chunk_16k"].scaled(n_q=2)) == 2        # 512 pairs
     assert n(WORKLOADS["draft_chunk_16k"].scaled(n_q=2, batch=16)) == 1
     assert n(WORKLOADS["tiny_decode"]) == 2                            # fp32
-    assert n(WORKLOADS["decode_1m"]) == 2                              # LSA centroids
+    assert n(WORKLOADS["decode_32k_overlap"]) == 2                     # windows
+    assert n(WORKLOADS["decode_1m"]) == 2                              # 2048 blocks
+    assert n(WORKLOADS["decode_1m"].scaled(ctx_len=512 * 512, top_k=64)) == 1
+    assert n(WORKLOADS["decode_1m"].scaled(ctx_len=512 * 513, top_k=64)) == 2
+
+
+@pytest.mark.parametrize("nb,k,pool,launches", [(500, 8, "lsa", 1), (400, 32, "lsa", 1), (450, 6, "mean", 1),
+                                                 (2048, 4, "lsa", 2), (1500, 6, "mean", 2)])
+def test_decode_selection_with_exact_ties(nb, k, pool, launches):
+    """The decode step's selection (the fused step's warp bit search up to
+    512 blocks, the scoring kernel's CTA radix select past them) on
+    compressed keys whose odd rows repeat the even rows: exact ties go to
+    the lower block id, so a selected odd block always comes with its even
+    twin; the sets and outputs match the oracle's."""
+    b = 512 if pool == "lsa" else 64
+    C = nb * b + 33
+    base = WORKLOADS["decode_1m"] if pool == "lsa" else WORKLOADS["decode_32k"]
+    w = base.scaled(batch=2, num_kv_heads=2, num_q_heads=8, ctx_len=C, top_k=k, n_needles=0)
+    p = sa.params_for(w, out_dtype="f32")
+    assert sa.decode_launches(p) == launches
+    inp = dev_inputs(w, seed=97)
+    Kc = run_pool(w, inp, p)
+    Kc[:, :, 1::2] = Kc[:, :, 0::2]
+    O, lse, idx, _ = run_decode(w, inp, p, Kc, torch.float32)
+    torch.cuda.synchronize()
+    op = oracle_params(w)
+    cand = orc.candidate_blocks(C, op)
+    for bi in range(w.batch):
+        for h in range(w.num_kv_heads):
+            q, K, V = slab(inp, bi, h, w.group, w.kv_len)
+            ref = orc.block_scores(orc.index_query(q[0]), Kc[bi, h].double().cpu().numpy(), op)
+            sel = orc.select_topk(ref, cand, k)
+            v = compare_sets(idx[bi, h].cpu().numpy(), sel)
+            assert v != "mismatch", (bi, h, idx[bi, h].tolist(), sel.selected)
+            got = set(int(j) for j in idx[bi, h] if j >= 0)
+            for j in got:
+                if j % 2 == 1 and (j - 1) in cand:
+                    assert j - 1 in got, (bi, h, j, sorted(got))
+            if v == "match":
+                pos = orc.attended_positions(C, op, sel.selected, C)
+                Oref, lref, _ = orc.masked_softmax_attention(q[0, 0], K, V, pos, orc.softmax_scale(128, op))
+                assert_close(O[bi, 0, h * w.group], Oref[None], "bf16", f"pair {(bi, h)}")

@@ -773,7 +773,16 @@ __global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
             acc.z += bf16lo(w2.y);
             acc.w += bf16hi(w2.y);
           }
-          q4 = make_float4(acc.x * a.sscale, acc.y * a.sscale, acc.z * a.sscale, acc.w * a.sscale);
+          // mean pooling: qbar times the softmax scale; LSA centroids:
+          // qbar / |qbar| (cosine scores)
+          float mul = a.sscale;
+          if (a.lsa) {
+            float ss = acc.x * acc.x + acc.y * acc.y + acc.z * acc.z + acc.w * acc.w;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            mul = ss > 0.f ? rsqrtf(ss) : 0.f;
+          }
+          q4 = make_float4(acc.x * mul, acc.y * mul, acc.z * mul, acc.w * mul);
         }
         const bool got = mbar_wait_bounded(&kv_full[s], (ci / kNS) & 1, abort_flag);
         if (got) {
@@ -1160,8 +1169,8 @@ cudaError_t launch_decode_tc(const DecodeAttnArgs& a0, const DecodePlan& p, bool
   return launch_tc<false>(a, p, out_bf16, s);
 }
 
-bool decode_fused_supported(const DecodeAttnArgs& a, const DecodePlan& p, int64_t nb, int lsa) {
-  if (lsa || nb < 1 || nb > kFusedMaxBlocks || !decode_tc_supported(a)) return false;
+bool decode_fused_supported(const DecodeAttnArgs& a, const DecodePlan& p, int64_t nb) {
+  if (nb < 1 || nb > kFusedMaxBlocks || !decode_tc_supported(a)) return false;
   const int64_t pairs = static_cast<int64_t>(a.B) * a.Hkv;
   const int64_t chunks = pairs * ((nb + 127) / 128);
   const int grid = p.tc_split.grid;

@@ -130,6 +130,7 @@ struct DecodeAttnArgs {
   int cpp;                // score chunks (128 compressed keys) per pair
   int cpc;                // score chunks per CTA
   float sscale;           // scoring scale (the softmax scale)
+  int lsa;                // LSA centroids: the index query is normalised instead of scaled
   TcOrder ord;            // tensor-core kernel work order
   // dense verify: per 32-key half-tile of the complete blocks and query row,
   // (sum of the row's probabilities, the running max they are taken against)
@@ -167,9 +168,10 @@ bool decode_tc_supported(const DecodeAttnArgs& a);
 size_t decode_tc_smem_bytes();
 cudaError_t launch_decode_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf16, cudaStream_t s);
 // The whole decode step (scores, top-k, attention) in one cooperative launch
-// of the tensor-core kernel; for mean pooling and nb <= kFusedMaxBlocks.
+// of the tensor-core kernel; for mean pooling or LSA centroids and nb <=
+// kFusedMaxBlocks.
 constexpr int kFusedMaxBlocks = 512;
-bool decode_fused_supported(const DecodeAttnArgs& a, const DecodePlan& p, int64_t nb, int lsa);
+bool decode_fused_supported(const DecodeAttnArgs& a, const DecodePlan& p, int64_t nb);
 cudaError_t launch_decode_fused(DecodeAttnArgs a, const DecodePlan& p, bool out_bf16, cudaStream_t s);
 // Copies a caller's [rows, len] index table to `out`, keeping only entries
 // that are in [0, nb) and above every earlier in-range entry of the row.

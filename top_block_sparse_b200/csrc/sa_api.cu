@@ -233,6 +233,7 @@ DecodeAttnArgs attn_args(const sa_params* p, const DecodeGeom& g, const DecodePl
   a.V = V;
   a.idx = idx;
   a.idx_stride = idx_stride;
+  a.top_k = p->top_k;
   a.O = O;
   a.lse = lse;
   a.part_O = reinterpret_cast<float*>(ws + L.part_O);
@@ -745,7 +746,7 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q, const void* K
   if (p->dtype == SA_BF16 && g.nb >= 1) {
     // one cooperative launch: scores, top-k and attention
     DecodeAttnArgs a = attn_args(p, g, plan, Q, K, V, idx, p->top_k, O, lse, w, L);
-    if (p->pool != SA_POOL_OVERLAP && decode_fused_supported(a, plan, g.nb, p->pool == SA_POOL_LSA)) {
+    if (p->pool != SA_POOL_OVERLAP && decode_fused_supported(a, plan, g.nb)) {
       a.Kc = Kc;
       a.scores = reinterpret_cast<float*>(w + L.scores);
       a.score_cnt = reinterpret_cast<unsigned*>(w + L.score_cnt);
@@ -754,6 +755,7 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q, const void* K
       a.idx_w = idx;
       a.top_k = p->top_k;
       a.sscale = scale_of(p);
+      a.lsa = p->pool == SA_POOL_LSA;
       cudaError_t e = launch_decode_fused(a, plan, p->out_dtype == SA_BF16, s);
       if (e == cudaSuccess) return SA_OK;
       // a cooperative grid that cannot be resident at once (e.g. SMs taken by
@@ -869,7 +871,7 @@ int32_t sa_decode_launches(const sa_params* p) {
     const DecodeWs L = decode_ws(g, plan, p->top_k, SA_OP_DECODE);
     DecodeAttnArgs a = attn_args(p, g, plan, nullptr, nullptr, nullptr, nullptr, p->top_k, nullptr, nullptr,
                                  nullptr, L);
-    if (p->pool != SA_POOL_OVERLAP && decode_fused_supported(a, plan, g.nb, p->pool == SA_POOL_LSA)) return 1;
+    if (p->pool != SA_POOL_OVERLAP && decode_fused_supported(a, plan, g.nb)) return 1;
   }
   return 2;
 }
