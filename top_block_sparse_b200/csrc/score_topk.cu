@@ -221,7 +221,10 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_topk_query0_kernel(Sco
   int32_t* out = a.idx + static_cast<int64_t>(pair) * a.top_k;
   // the ring is idle now: its first words hold the selection's histograms
   unsigned* scratch = reinterpret_cast<unsigned*>(ring);
-  if (nb <= 2048) block_radix_topk<2048 / kScoreThreads>(keys, nb, a.top_k, out, scratch);
+  // keys per thread sized to the table (the radix passes loop over them)
+  if (nb <= kScoreThreads) block_radix_topk<1>(keys, nb, a.top_k, out, scratch);
+  else if (nb <= 2 * kScoreThreads) block_radix_topk<2>(keys, nb, a.top_k, out, scratch);
+  else if (nb <= 2048) block_radix_topk<2048 / kScoreThreads>(keys, nb, a.top_k, out, scratch);
   else block_radix_topk<kMaxSelectBlocks / kScoreThreads>(keys, nb, a.top_k, out, scratch);
 }
 
