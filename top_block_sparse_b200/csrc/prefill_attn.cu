@@ -21,8 +21,8 @@
 //
 // Column mode (PulseCol §3.1 eq. (2) with a token-granular column mask): the
 // item's 64 tokens x 4 heads attend to the key columns listed for the group
-// (ascending, -1 padded), before or after them alike.  The producer warp
-// gathers each chunk of 64 listed K and V rows with 16-byte cp.async copies
+// (ascending, -1 padded), before or after them alike.  Four producer warps
+// gather each chunk of 64 listed K and V rows with 16-byte cp.async copies
 // into the same 128-byte-swizzled stage layout the tensor maps produce,
 // keeps up to three chunks in flight (cp.async groups), and, once a chunk
 // has landed, fences it for the tensor cores and arrives on the stage's
@@ -46,7 +46,7 @@ constexpr int kQBytes = kRows * 256;           // 64 KB (two 32 KB boxes: d 0-63
 constexpr int kKVStage = 32768;                // K 16 KB (two 8 KB boxes) + V 16 KB
 constexpr int kPBytes = 2 * 16384;             // P: two halves of 128 rows x 64 keys
 constexpr int kThreads = 320;
-constexpr int kGatherWarps = 2;                // column mode: warps 8 and 10 gather K and V rows
+constexpr int kGatherWarps = 4;                // column mode: warps 8, 10, 11 and 12 gather K and V rows
 constexpr int kGatherRows = kT / kGatherWarps;  // rows of a chunk per gathering warp
 constexpr int kLanesPerRow = 32 / kGatherRows;
 constexpr int kThreadsCol = kThreads + (kGatherWarps - 1) * 32;
@@ -201,8 +201,8 @@ __global__ void __launch_bounds__(COL ? kThreadsCol : kThreads, 1)
 
   if (warp == 8 || (COL && warp >= 10)) {
     // -------------------------------------------------------- TMA producer
-    // column mode: warps 8 and 10 (and more with kGatherWarps) gather
-    // kGatherRows of every chunk's rows each; warp 8 also loads Q
+    // column mode: warps 8, 10, 11 and 12 gather kGatherRows of every
+    // chunk's rows each, two lanes a row; warp 8 also loads Q
     const int gw = warp == 8 ? 0 : warp - 9;
     int use = 0, it = 0;
     bool ok = true;
