@@ -936,7 +936,7 @@ def run_decode_configs(args, dev, stream, flush):
         torch.cuda.nvtx.range_push(name)
         w = WORKLOADS[name]
         if args.small and name != "tiny_decode":
-            w = w.scaled(batch=max(1, w.batch // 8), ctx_len=min(w.ctx_len, 262144))
+            w = w.scaled(batch=max(1, w.batch // 8), ctx_len=min(w.ctx_len, 524288))
         inp = make_inputs(w, seed=seed, device=dev)
         Q, K, V = inp["Q"], inp["K"], inp["V"]
         del inp

@@ -112,25 +112,6 @@ __device__ __forceinline__ void sel_bar_sync() {
   asm volatile("bar.sync 2, %0;" ::"r"(kSelBarThreads) : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t* r = reinterpret_cast<uint32_t*>(v);
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
-  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
 
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
   uint32_t* r = reinterpret_cast<uint32_t*>(v);
@@ -158,7 +139,6 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const float (&v)[4]) {
                "r"(r[2]), "r"(r[3])
                : "memory");
 }
-// The first NR columns of this warp's 32 TMEM lanes.
 // Reduction of each of NR rows over the 32 lanes of a warp (max or sum) by a
 // reduce-scatter: at each level a lane keeps half of the rows it still holds
 // and trades the other half with the lane that differs in that bit, so NR
@@ -184,17 +164,19 @@ __device__ __forceinline__ float rows_reduce(float (&v)[NR], int lane) {
   return r;
 }
 
+// The first NR columns of this warp's 32 TMEM lanes.  A thread reads at
+// most 8 rows: 16-row instantiations split their rows over two warpgroups.
 template <int NR>
 __device__ __forceinline__ void tmem_ldn(uint32_t taddr, float (&v)[NR]) {
+  static_assert(NR == 4 || NR == 8, "a thread reads at most 8 rows");
   if constexpr (NR == 4) tmem_ld4(taddr, v);
-  else if constexpr (NR == 8) tmem_ld8(taddr, v);
-  else tmem_ld16(taddr, v);
+  else tmem_ld8(taddr, v);
 }
 template <int NR>
 __device__ __forceinline__ void tmem_stn(uint32_t taddr, const float (&v)[NR]) {
+  static_assert(NR == 4 || NR == 8, "a thread rescales at most 8 rows");
   if constexpr (NR == 4) tmem_st4(taddr, v);
-  else if constexpr (NR == 8) tmem_st8(taddr, v);
-  else tmem_st16(taddr, v);
+  else tmem_st8(taddr, v);
 }
 
 template <bool OUT_BF16>
