@@ -269,9 +269,11 @@ sa_status sa_column_attn(const sa_params* p, const void* Q, const void* K,
 
 /* Number of kernels one sa_sparse_attn_decode call with `p` launches on this
  * device: 1 when scoring, top-k and attention run as one cooperative launch
- * (bf16, SA_POOL_MEAN or SA_POOL_LSA, at most 512 complete blocks, at most
- * 4 query rows (n_q x Hq / Hkv) per KV head and at most two (sequence, KV
- * head) pairs per SM), else 2; 0 if p is
+ * (bf16, SA_POOL_MEAN or SA_POOL_LSA, at most 512 complete blocks or, for
+ * top_k <= 8, up to 16384 while each SM scores at most 4 x 128 of them and a
+ * (sequence, KV head) pair's are scored on at most 31 SMs, at most 4 query rows (n_q x Hq /
+ * Hkv) per KV head and at most two (sequence, KV head) pairs per SM), else
+ * 2; 0 if p is
  * invalid.  A cooperative launch the device refuses at run time falls back
  * to the 2-kernel path.  Host only; launches nothing. */
 int32_t sa_decode_launches(const sa_params* p);

@@ -212,7 +212,8 @@ def test_given_idx_with_oracle_indices(name, over):
     ("decode_32k", dict(batch=2)),
     ("draft_chunk_16k", dict(batch=2)),
     ("decode_1m", dict(batch=1, ctx_len=512 * 200, num_kv_heads=2, num_q_heads=8)),
-    # LSA centroids past 512 blocks (scoring kernel, then attention)
+    # LSA centroids past 512 blocks: the fused step, each CTA publishing the
+    # top k of its own score chunks and the last of a pair merging them
     ("decode_1m", dict(batch=2, ctx_len=512 * 1500 + 77, num_kv_heads=4, num_q_heads=16)),
     ("decode_1m", dict(batch=1, ctx_len=512 * 2000 + 300, num_kv_heads=1, num_q_heads=4, top_k=8)),
     # 8 and 16 query rows per KV head (n_q tokens x G heads): the tensor-core
@@ -407,11 +408,11 @@ def test_fused_empty_tiles_after_score_chunks():
 
 
 def test_decode_32k_runs_as_one_launch():
-    """The batched-decode workload takes the fused path (scores, top-k and
-    attention in one cooperative launch) on this device, and so does LSA
-    pooling up to 512 blocks; draft chunks (12 query rows per KV head), more
-    than two pairs per SM, fp32, overlapping windows and more than 512
-    blocks (the 1M-token workload) take the scoring kernel and then the
+    """The batched-decode and 1M-token workloads take the fused path (scores,
+    top-k and attention in one cooperative launch) on this device, LSA
+    pooling too, past 512 blocks for k <= 8; draft chunks (12 query rows per
+    KV head), more than two pairs per SM, fp32, overlapping windows and more
+    than 512 blocks with k > 8 take the scoring kernel and then the
     attention kernel."""
     n = lambda w: sa.decode_launches(sa.params_for(w))
     assert n(WORKLOADS["decode_32k"]) == 1
@@ -420,19 +421,21 @@ def test_decode_32k_runs_as_one_launch():
     assert n(WORKLOADS["draft_chunk_16k"].scaled(n_q=2, batch=16)) == 1
     assert n(WORKLOADS["tiny_decode"]) == 2                            # fp32
     assert n(WORKLOADS["decode_32k_overlap"]) == 2                     # windows
-    assert n(WORKLOADS["decode_1m"]) == 2                              # 2048 blocks
+    assert n(WORKLOADS["decode_1m"]) == 1                              # 2048 blocks, k = 4
+    assert n(WORKLOADS["decode_1m"].scaled(top_k=9)) == 2              # 2048 blocks, k > 8
     assert n(WORKLOADS["decode_1m"].scaled(ctx_len=512 * 512, top_k=64)) == 1
     assert n(WORKLOADS["decode_1m"].scaled(ctx_len=512 * 513, top_k=64)) == 2
 
 
 @pytest.mark.parametrize("nb,k,pool,launches", [(500, 8, "lsa", 1), (400, 32, "lsa", 1), (450, 6, "mean", 1),
-                                                 (2048, 4, "lsa", 2), (1500, 6, "mean", 2)])
+                                                 (2048, 4, "lsa", 1), (1500, 6, "mean", 1), (1500, 12, "mean", 2)])
 def test_decode_selection_with_exact_ties(nb, k, pool, launches):
     """The decode step's selection (the fused step's warp bit search up to
-    512 blocks, the scoring kernel's CTA radix select past them) on
-    compressed keys whose odd rows repeat the even rows: exact ties go to
-    the lower block id, so a selected odd block always comes with its even
-    twin; the sets and outputs match the oracle's."""
+    512 blocks, its per-CTA candidates and merge past them for k <= 8, the
+    scoring kernel's CTA radix select otherwise) on compressed keys whose
+    odd rows repeat the even rows: exact ties go to the lower block id, so a
+    selected odd block always comes with its even twin; the sets and outputs
+    match the oracle's."""
     b = 512 if pool == "lsa" else 64
     C = nb * b + 33
     base = WORKLOADS["decode_1m"] if pool == "lsa" else WORKLOADS["decode_32k"]

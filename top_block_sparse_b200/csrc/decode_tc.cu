@@ -85,9 +85,9 @@ __device__ __forceinline__ void groups_bar() {
 
 // Threads of an instantiation, and whether its softmax rows are split over
 // two warpgroups.
-template <int NR, bool FUSED>
-constexpr bool kSplitRows = NR == 16 && !FUSED;
-template <int NR, bool FUSED>
+template <int NR, int FUSED>
+constexpr bool kSplitRows = NR == 16 && FUSED == 0;
+template <int NR, int FUSED>
 constexpr int kThreadsOf = FUSED ? kThreadsFused : (kSplitRows<NR, FUSED> ? kThreadsSplit : kThreads);
 // The same barrier, returning whether any of the softmax threads passed true.
 __device__ __forceinline__ bool softmax_bar_or(bool v) {
@@ -205,7 +205,12 @@ __device__ __forceinline__ void store_out4(void* O, int64_t idx, float4 v, float
 // and publishes the table with a per-pair ready flag, and the producer waits
 // for the flag of every pair before reading its table.  A cooperative launch
 // keeps every CTA resident, so the waits end.
-template <bool OUT_BF16, int NR, bool FUSED, bool MASS>
+// FUSED: 0 attention only; 1 the whole step, each pair selected by the CTA
+// that scored its last chunk (a warp bit search over <= kFusedMaxBlocks
+// scores); 2 the whole step for long contexts and k <= kFusedSmallK: every
+// CTA that scored chunks of a pair publishes the top k of its own rows, and
+// the CTA completing the pair's count selects among those candidates.
+template <bool OUT_BF16, int NR, int FUSED, bool MASS>
 __global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                      const __grid_constant__ CUtensorMap v_map, DecodeAttnArgs a) {
@@ -233,6 +238,8 @@ __global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
   int* ticket = reinterpret_cast<int*>(tmem_slot + 2);
   uint64_t* mma_done = reinterpret_cast<uint64_t*>(tmem_slot + 4);    // 8-byte aligned
   __shared__ int sel_list[kMaxSelPerCta];                               // fused: pairs this CTA selects
+  __shared__ int sel_first[kMaxSelPerCta];                              // FUSED 2: a run's first chunk
+  __shared__ int sel_cnt[kMaxSelPerCta];                                // FUSED 2: its chunks
   __shared__ int n_sel;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -351,8 +358,8 @@ __global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
       int64_t ks0 = 0, ks1 = 0;
       int nk0 = 0, nk1 = 0;
       if (i + lane < end) {
-        unit_tile<FUSED>(a, pc, i + lane, 0, &ks0, &nk0);
-        unit_tile<FUSED>(a, pc, i + lane, 1, &ks1, &nk1);
+        unit_tile<FUSED != 0>(a, pc, i + lane, 0, &ks0, &nk0);
+        unit_tile<FUSED != 0>(a, pc, i + lane, 1, &ks1, &nk1);
       }
       const int64_t pair = pc.pair;
       const int pk = pc.ordinal;
@@ -509,7 +516,107 @@ __global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
     sel_bar_sync();
     const int nb = static_cast<int>(a.nb);
     const int nsel = n_sel;
-    for (int e = warp - 6; e < nsel && !*abort_flag; e += 2) {
+    for (int e = warp - 6; e < nsel && !*abort_flag && FUSED == 2; e += 2) {
+      // FUSED 2: this CTA's run of chunks of pair pr -> the top k of its own
+      // rows into the pair's candidate slot, then the pair's chunk count
+      const int pr = sel_list[e], first = sel_first[e], n = sel_cnt[e];
+      const int row0 = (first - pr * a.cpp) * 128, row1 = min(nb, row0 + n * 128);
+      const float* sc = a.scores + static_cast<int64_t>(pr) * nb;
+      constexpr int PR = kFusedRunChunks * 128 / 32;
+      uint32_t kr[PR];
+#pragma unroll
+      for (int i = 0; i < PR; ++i) {
+        const int j = row0 + i * 32 + lane;
+        const float v = j < row1 ? __ldcg(sc + j) : 0.f;
+        const int64_t lo = static_cast<int64_t>(j) * a.b, hi = lo + a.b;
+        const bool cand = j < row1 && (lo < a.w_begin) && (hi > a.s_end);
+        const uint32_t key = float_key(v);
+        kr[i] = cand ? (key == 0u ? 1u : key) : 0u;
+      }
+      const int slot = static_cast<int>(blockIdx.x) - (pr * a.cpp) / a.cpc;
+      uint2* cs = a.cand + (static_cast<int64_t>(pr) * kFusedCandSlots + slot) * kFusedSmallK;
+      // k passes, each taking the largest key left (the lowest id on ties)
+#pragma unroll 1
+      for (int q = 0; q < kFusedSmallK; ++q) {
+        uint32_t best = 0u;
+        int bi = 0;
+#pragma unroll
+        for (int i = 0; i < PR; ++i) {
+          const bool gt = kr[i] > best;
+          best = gt ? kr[i] : best;
+          bi = gt ? i : bi;
+        }
+        const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+        unsigned jm = 0xffffffffu;
+        if (m != 0u && q < a.top_k) {
+          jm = __reduce_min_sync(0xffffffffu, best == m ? static_cast<unsigned>(bi * 32 + lane) : 0xffffffffu);
+#pragma unroll
+          for (int i = 0; i < PR; ++i) kr[i] = (static_cast<unsigned>(i * 32 + lane) == jm) ? 0u : kr[i];
+        }
+        if (lane == 0) cs[q] = make_uint2(jm == 0xffffffffu ? 0u : m, jm == 0xffffffffu ? 0u : row0 + jm);
+      }
+      __threadfence();
+      __syncwarp();
+      unsigned old = 0u;
+      if (lane == 0) old = atomicAdd(&a.score_cnt[pr], static_cast<unsigned>(n));
+      old = __shfl_sync(0xffffffffu, old, 0);
+      if (old + n != static_cast<unsigned>(a.cpp)) continue;
+      // the last run of the pair: merge the slots' candidates
+      __threadfence();
+      if (lane == 0) a.score_cnt[pr] = 0u;
+      const int nslots = ((pr + 1) * a.cpp - 1) / a.cpc - (pr * a.cpp) / a.cpc + 1;
+      const uint2* cp = a.cand + static_cast<int64_t>(pr) * kFusedCandSlots * kFusedSmallK;
+      constexpr int PM = kFusedCandSlots * kFusedSmallK / 32;
+      uint32_t mk[PM], mi[PM];
+#pragma unroll
+      for (int i = 0; i < PM; ++i) {
+        const int c = i * 32 + lane;
+        const uint2 v = c < nslots * kFusedSmallK ? __ldcg(cp + c) : make_uint2(0u, 0u);
+        mk[i] = v.x;
+        mi[i] = v.y;
+      }
+      int got[kFusedSmallK];
+      int ng = 0;
+#pragma unroll
+      for (int q = 0; q < kFusedSmallK; ++q) {
+        got[q] = 0x7fffffff;
+        uint32_t best = 0u, bid = 0xffffffffu;
+#pragma unroll
+        for (int i = 0; i < PM; ++i) {
+          const bool better = mk[i] > best || (mk[i] == best && mk[i] != 0u && mi[i] < bid);
+          best = better ? mk[i] : best;
+          bid = better ? mi[i] : bid;
+        }
+        const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+        if (m != 0u && q < a.top_k) {
+          const unsigned jm = __reduce_min_sync(0xffffffffu, best == m ? bid : 0xffffffffu);
+#pragma unroll
+          for (int i = 0; i < PM; ++i) mk[i] = (mk[i] == m && mi[i] == jm) ? 0u : mk[i];
+          got[q] = static_cast<int>(jm);
+          ++ng;
+        }
+      }
+      if (lane == 0) {
+        // ascending ids (absent ones sort last)
+#pragma unroll
+        for (int q = 1; q < kFusedSmallK; ++q) {
+#pragma unroll
+          for (int r = q; r > 0; --r) {
+            const int lo = min(got[r - 1], got[r]), hi = max(got[r - 1], got[r]);
+            got[r - 1] = lo;
+            got[r] = hi;
+          }
+        }
+        int32_t* out = a.idx_w + static_cast<int64_t>(pr) * a.top_k;
+#pragma unroll
+        for (int q = 0; q < kFusedSmallK; ++q)
+          if (q < a.top_k) out[q] = q < ng ? got[q] : -1;
+      }
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) atomicExch(&a.ready[pr], 1u);
+    }
+    for (int e = warp - 6; e < nsel && !*abort_flag && FUSED == 1; e += 2) {
       const int pr = sel_list[e];
       __threadfence();
       if (lane == 0) a.score_cnt[pr] = 0u;
@@ -728,12 +835,23 @@ __global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
       // count this CTA's chunks of a pair once its run of them ends (one
       // release fence and one atomic per run, not per chunk); the CTA that
       // completes the pair's count selects it
+      int run_first = 0;                         // FUSED 2: the run's first chunk
       auto close_run = [&](int pr, int n) {
-        __threadfence();
-        const unsigned old = atomicAdd(&a.score_cnt[pr], static_cast<unsigned>(n));
-        if (old + n == static_cast<unsigned>(a.cpp)) {
-          if (n_sel < kMaxSelPerCta) sel_list[n_sel++] = pr;
-          else report(a.status, kStatusTimeout);
+        if constexpr (FUSED == 1) {
+          __threadfence();
+          const unsigned old = atomicAdd(&a.score_cnt[pr], static_cast<unsigned>(n));
+          if (old + n == static_cast<unsigned>(a.cpp)) {
+            if (n_sel < kMaxSelPerCta) sel_list[n_sel++] = pr;
+            else report(a.status, kStatusTimeout);
+          }
+        } else if (n_sel < kMaxSelPerCta) {
+          // every run goes to the selection warps, which count it
+          sel_list[n_sel] = pr;
+          sel_first[n_sel] = run_first;
+          sel_cnt[n_sel] = n;
+          ++n_sel;
+        } else {
+          report(a.status, kStatusTimeout);
         }
       };
       for (int ci = 0; ci < r0; ++ci) {
@@ -745,6 +863,7 @@ __global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
           if (t == 0 && cur >= 0) close_run(cur, seg_cnt);
           cur = pr;
           seg_cnt = 0;
+          run_first = gc;
           const int bi = pr / a.Hkv, h = pr % a.Hkv;
           float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
           for (int g = 0; g < G; ++g) {
@@ -1099,7 +1218,7 @@ bool encode_maps(const DecodeAttnArgs& a, CUtensorMap* qm, CUtensorMap* km, CUte
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool FUSED>
+template <int FUSED>
 cudaError_t launch_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf16, cudaStream_t s) {
   CUtensorMap qm, km, vm;
   if (!encode_maps(a, &qm, &km, &vm)) return cudaErrorInvalidValue;
@@ -1148,14 +1267,22 @@ cudaError_t launch_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf1
 cudaError_t launch_decode_tc(const DecodeAttnArgs& a0, const DecodePlan& p, bool out_bf16, cudaStream_t s) {
   DecodeAttnArgs a = a0;
   a.ord = p.tc_plain;
-  return launch_tc<false>(a, p, out_bf16, s);
+  return launch_tc<0>(a, p, out_bf16, s);
 }
 
 bool decode_fused_supported(const DecodeAttnArgs& a, const DecodePlan& p, int64_t nb) {
-  if (nb < 1 || nb > kFusedMaxBlocks || !decode_tc_supported(a)) return false;
+  if (nb < 1 || nb > kMaxSelectBlocks || !decode_tc_supported(a)) return false;
   const int64_t pairs = static_cast<int64_t>(a.B) * a.Hkv;
-  const int64_t chunks = pairs * ((nb + 127) / 128);
+  const int64_t cpp = (nb + 127) / 128;
+  const int64_t chunks = pairs * cpp;
   const int grid = p.tc_split.grid;
+  if (grid < 1) return false;
+  if (nb > kFusedMaxBlocks) {
+    // past 512 blocks: runs of at most kFusedRunChunks chunks publish their
+    // own top k (k <= kFusedSmallK) into at most kFusedCandSlots slots a pair
+    const int64_t cpc = (chunks + grid - 1) / grid;
+    if (a.top_k > kFusedSmallK || cpc > kFusedRunChunks || (cpp + cpc - 1) / cpc + 1 > kFusedCandSlots) return false;
+  }
   // Measured on B200: with more than 4 query rows per KV head (draft chunks)
   // or more than two pairs per CTA, the per-pair partial results of the two
   // split lists cost more than the second launch saves, and the scoring
@@ -1173,7 +1300,7 @@ cudaError_t launch_decode_fused(DecodeAttnArgs a, const DecodePlan& p, bool out_
   a.idx = a.idx_w;
   a.idx_stride = a.top_k;
   a.pdl = 0;
-  return launch_tc<true>(a, p, out_bf16, s);
+  return a.nb <= kFusedMaxBlocks ? launch_tc<1>(a, p, out_bf16, s) : launch_tc<2>(a, p, out_bf16, s);
 }
 
 }  // namespace sa

@@ -126,6 +126,7 @@ struct DecodeAttnArgs {
   unsigned* ready;        // [pairs] index table published, zero between calls
   unsigned* exit_cnt;     // CTAs finished, zero between calls
   int32_t* idx_w;         // [pairs, top_k] index table written by the fused kernel
+  uint2* cand;            // [pairs, kFusedCandSlots, kFusedSmallK] (key, block id) per run of score chunks
   int top_k;
   int cpp;                // score chunks (128 compressed keys) per pair
   int cpc;                // score chunks per CTA
@@ -169,8 +170,13 @@ size_t decode_tc_smem_bytes();
 cudaError_t launch_decode_tc(const DecodeAttnArgs& a, const DecodePlan& p, bool out_bf16, cudaStream_t s);
 // The whole decode step (scores, top-k, attention) in one cooperative launch
 // of the tensor-core kernel; for mean pooling or LSA centroids and nb <=
-// kFusedMaxBlocks.
+// kFusedMaxBlocks, or past it for k <= kFusedSmallK when every CTA scores at
+// most kFusedRunChunks chunks and a pair's chunks span at most
+// kFusedCandSlots CTAs.
 constexpr int kFusedMaxBlocks = 512;
+constexpr int kFusedSmallK = 8;
+constexpr int kFusedRunChunks = 4;
+constexpr int kFusedCandSlots = 32;
 bool decode_fused_supported(const DecodeAttnArgs& a, const DecodePlan& p, int64_t nb);
 cudaError_t launch_decode_fused(DecodeAttnArgs a, const DecodePlan& p, bool out_bf16, cudaStream_t s);
 // Copies a caller's [rows, len] index table to `out`, keeping only entries

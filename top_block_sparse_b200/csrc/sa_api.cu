@@ -132,7 +132,7 @@ float scale_of(const sa_params* p) {
 
 // Workspace layout of the decode-type ops.
 struct DecodeWs {
-  size_t score_cnt, attn_cnt, scores, idx, clean_idx, part_O, part_ml, ready, exit_cnt, total;
+  size_t score_cnt, attn_cnt, scores, idx, clean_idx, part_O, part_ml, ready, exit_cnt, cand, total;
 };
 
 // idx_len: entries per row of a caller's index table (SA_OP_GIVEN_IDX).
@@ -154,6 +154,7 @@ DecodeWs decode_ws(const DecodeGeom& g, const DecodePlan& plan, int top_k, int o
     w.idx = take(pairs * static_cast<size_t>(top_k) * 4);
     w.ready = take(pairs * 4);       // fused decode: per-pair table flags
     w.exit_cnt = take(4);
+    w.cand = take(pairs * kFusedCandSlots * kFusedSmallK * 8);   // fused decode past 512 blocks
   }
   if (op == SA_OP_GIVEN_IDX) w.clean_idx = take(pairs * static_cast<size_t>(idx_len) * 4);
   if (op == SA_OP_DECODE || op == SA_OP_GIVEN_IDX) {
@@ -752,6 +753,7 @@ sa_status sa_sparse_attn_decode(const sa_params* p, const void* Q, const void* K
       a.score_cnt = reinterpret_cast<unsigned*>(w + L.score_cnt);
       a.ready = reinterpret_cast<unsigned*>(w + L.ready);
       a.exit_cnt = reinterpret_cast<unsigned*>(w + L.exit_cnt);
+      a.cand = reinterpret_cast<uint2*>(w + L.cand);
       a.idx_w = idx;
       a.top_k = p->top_k;
       a.sscale = scale_of(p);
