@@ -250,7 +250,8 @@ sa_status sa_verify_refresh(const sa_params* p, const void* Q, const void* K,
  * before or after them alike (no causal mask, no sink or window).
  *
  * p describes a full sequence as in prefill: select = SA_SEL_TILE_MAX,
- * ctx_len = 0, n_q = T tokens, block_size = 64 (the group), GQA 4, bf16;
+ * ctx_len = 0, n_q = T tokens, block_size = 64 (the group), Hq / Hkv a
+ * multiple of 4, bf16;
  * top_k, sink_keys, window_keys and pool are ignored.  Q [B, T, Hq, d];
  * K, V [B, Hkv, kv_capacity, d] (rows 0..T-1 are the keys); cols [B, Hkv,
  * ceil(T/64), n_cols] int32: per group, key positions in [0, T), ascending,
@@ -286,7 +287,7 @@ int32_t sa_decode_launches(const sa_params* p);
  * sa_score_topk), selects per (tile, KV head) and runs causal sparse
  * attention: tile i attends sink U window U selected U its own keys
  * (causal).  Writes O, lse (optional), idx_out (optional).  Built for bf16,
- * b = 64, Hq = 4 Hkv, sink and window multiples of 64 (else
+ * b = 64, Hq / Hkv a multiple of 4, sink and window multiples of 64 (else
  * SA_ERR_UNSUPPORTED). */
 sa_status sa_sparse_attn_prefill(const sa_params* p, const void* Q,
                                  const void* K, const void* V, float* Kc,

@@ -208,7 +208,8 @@ def _column(p, n_cols=70, cols=FAKE, ws_bytes=1 << 30):
 @host_only
 @pytest.mark.parametrize("kw,n_cols,status", [
     (dict(dtype="f32"), 70, sa.SA_ERR_UNSUPPORTED),           # tensor cores: bf16 only
-    (dict(num_q_heads=4), 70, sa.SA_ERR_UNSUPPORTED),         # GQA 2: built for groups of 4 heads
+    (dict(num_q_heads=4), 70, sa.SA_ERR_UNSUPPORTED),         # GQA 2: built for multiples of 4 heads
+    (dict(num_q_heads=12), 70, sa.SA_ERR_UNSUPPORTED),        # GQA 6 (not a multiple of 4)
     (dict(block_size=128), 70, sa.SA_ERR_UNSUPPORTED),        # the query group is 64 tokens
     (dict(prefill=False), 70, sa.SA_ERR_INVALID),             # sequence-type params needed
     ({}, -1, sa.SA_ERR_INVALID),
@@ -291,3 +292,15 @@ def test_bucket_arguments_and_workspace():
     assert sa.bucket_rows(p) == ((512 * 6 + 6) // 512) * 64
     # 5 tokens x GQA 4 = 20 query rows per KV head: the attention is not built
     assert sa.workspace_size(_pb(n_q=5), sa.SA_OP_BUCKET_DECODE) == 0
+
+
+@host_only
+def test_prefill_head_group_sizes():
+    """Prefill and column attention take GQA groups of a multiple of 4 query
+    heads (4 heads of a tile per work item): groups of 4, 8 and 16 get a
+    workspace size, 2 and 6 are refused."""
+    for G, ok in ((4, True), (8, True), (16, True), (2, False), (6, False)):
+        pf = _p(prefill=True, ctx_len=0, n_q=4096, num_q_heads=2 * G, num_kv_heads=2)
+        for op in (sa.SA_OP_PREFILL, sa.SA_OP_SCORE_TOPK, sa.SA_OP_GIVEN_IDX):
+            assert (sa.raw_call("sa_workspace_size", ctypes.byref(pf), op) > 0) == ok, (G, op)
+        assert (sa.workspace_size(_pcol(num_q_heads=2 * G), sa.SA_OP_COLUMN) > 0) == ok, G

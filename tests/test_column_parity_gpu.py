@@ -68,6 +68,7 @@ def _all_groups(w):
     (dict(n_q=256), 64),                                # one full chunk per group
     (dict(n_q=64 * 3, batch=2), 200),                   # lists longer than the sequence: -1 padding
     (dict(n_q=128), 1),                                 # one column
+    (dict(num_q_heads=16), 70),                         # 8 query heads per KV head: two head groups per item
 ])
 def test_column_parity(over, n_cols):
     w = _w(**over)

@@ -19,13 +19,14 @@ pytestmark = pytest.mark.gpu
 sa = pytest.importorskip("top_block_sparse_b200.sa")
 
 
-def pf(T, Hkv=2, k=8, **kw):
-    return WORKLOADS["prefill_64k"].scaled(n_q=T, num_kv_heads=Hkv, num_q_heads=4 * Hkv, top_k=k,
+def pf(T, Hkv=2, k=8, G=4, **kw):
+    return WORKLOADS["prefill_64k"].scaled(n_q=T, num_kv_heads=Hkv, num_q_heads=G * Hkv, top_k=k,
                                            n_needles=min(k, 4), **kw)
 
 
 def head_arrays(inp, h, w):
-    q = inp["Q"][0, :, 4 * h:4 * h + 4].double().cpu().numpy()     # [T, G, d]
+    G = w.group
+    q = inp["Q"][0, :, G * h:G * h + G].double().cpu().numpy()     # [T, G, d]
     K = inp["K"][0, h, :w.n_q].double().cpu().numpy()
     V = inp["V"][0, h, :w.n_q].double().cpu().numpy()
     return q, K, V
@@ -62,8 +63,9 @@ def check_tiles(w, inp, O, lse, idx, tiles, Kc_gpu=None):
             if v == "near_tie":
                 ties += 1
                 continue
-            assert_close(O[0, rows, 4 * h:4 * h + 4], r["O"], "bf16", f"head {h} tile {i}")
-            lerr = np.abs(lse[0, rows, 4 * h:4 * h + 4].double().cpu().numpy() - r["lse"]).max()
+            G = w.group
+            assert_close(O[0, rows, G * h:G * h + G], r["O"], "bf16", f"head {h} tile {i}")
+            lerr = np.abs(lse[0, rows, G * h:G * h + G].double().cpu().numpy() - r["lse"]).max()
             assert lerr < 2e-3, (h, i, lerr)
     return ties
 
@@ -134,6 +136,18 @@ def test_prefill_end_to_end(T, k):
     _, Kc, O, lse, idx = run_prefill(w, inp)
     ties = check_tiles(w, inp, O, lse, idx, range((T + 63) // 64), Kc)
     print(f"\nprefill T={T}: near-ties {ties}")
+
+
+@pytest.mark.parametrize("G,T", [(8, 64 * 14 + 9), (12, 64 * 9)])
+def test_prefill_head_groups(G, T):
+    """8 and 12 query heads per KV head: the scorer sums all G heads of a
+    row, and each tile's attention runs as G / 4 items of four heads that
+    share its block list; every tile matches the oracle."""
+    w = pf(T, G=G, k=5)
+    inp = make_inputs(w, seed=74, device="cuda")
+    _, Kc, O, lse, idx = run_prefill(w, inp)
+    ties = check_tiles(w, inp, O, lse, idx, range((T + 63) // 64), Kc)
+    print(f"\nprefill G={G}: near-ties {ties}")
 
 
 def test_prefill_bf16_output_and_reuse():

@@ -5,9 +5,10 @@
 //   sink [0, min(S, C)) U selected blocks U window [max(C - W, sink end), C)
 //   U its own block, causally (query row r sees keys 64 t .. 64 t + r).
 //
-// One work item = (sequence x KV head, tile): 64 tokens x G = 4 heads = 256
-// query rows = two M = 128 halves (row m = 4 * token + head, the order a 3-D
-// TMA box of Q lands in).  Per 64-key block:
+// One work item = (sequence x KV head, tile, group of 4 of the KV head's G
+// query heads): 64 tokens x 4 heads = 256 query rows = two M = 128 halves
+// (row m = 4 * token + head, the order a 3-D TMA box of Q lands in); G a
+// multiple of 4, the G / 4 items of a tile sharing its block list.  Per 64-key block:
 //   S   = Q K^T          tcgen05.mma, M 128, N 64, K 128 per half, fp32 in TMEM
 //   P   = softmax(S)     8 warps, one query row per thread (online, lazy
 //                        rescale when the row max grows by more than 2^8),
@@ -39,7 +40,7 @@ namespace sa {
 namespace {
 
 constexpr int kT = 64;                         // tile = block = 64
-constexpr int kG = 4;                          // query heads per KV head handled here
+constexpr int kG = 4;                          // query heads of one work item
 constexpr int kRows = kT * kG;                 // 256 query rows per item
 constexpr int kNKV = 4;                        // K/V ring stages
 constexpr int kQBytes = kRows * 256;           // 64 KB (two 32 KB boxes: d 0-63, d 64-127)
@@ -78,6 +79,7 @@ struct PAArgs {
   float* lse;               // [B, T, Hq] or null
   unsigned* status;
   int B, Hq, Hkv, T, n_tiles, P, top_k, out_bf16;
+  int HG;                   // groups of kG query heads per KV head (G / 4)
   int64_t S, W;
   float scale_log2;         // softmax scale * log2(e)
 };
@@ -137,10 +139,14 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Item k -> (pair p, tile t), most expensive tiles first.
-__device__ __forceinline__ void item_of(const PAArgs& a, int k, int* p, int* t) {
-  *t = a.n_tiles - 1 - k / a.P;
-  *p = k % a.P;
+// Item k -> (pair p, tile t, head group hg), most expensive tiles first, a
+// tile's head groups next to each other (they read the same K and V blocks).
+__device__ __forceinline__ void item_of(const PAArgs& a, int k, int* p, int* t, int* hg) {
+  const int per_tile = a.P * a.HG;
+  *t = a.n_tiles - 1 - k / per_tile;
+  const int q = k - (k / per_tile) * per_tile;
+  *p = q / a.HG;
+  *hg = q - *p * a.HG;
 }
 
 template <bool COL>
@@ -167,7 +173,7 @@ __global__ void __launch_bounds__(COL ? kThreadsCol : kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_items = a.n_tiles * a.P;
+  const int n_items = a.n_tiles * a.P * a.HG;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNKV; ++s) {
@@ -207,19 +213,20 @@ __global__ void __launch_bounds__(COL ? kThreadsCol : kThreads, 1)
     int use = 0, it = 0;
     bool ok = true;
     for (int k = blockIdx.x; k < n_items && ok; k += gridDim.x, ++it) {
-      int p, t;
-      item_of(a, k, &p, &t);
+      int p, t, hg;
+      item_of(a, k, &p, &t, &hg);
       const Blocks bl = item_blocks<COL>(a, p, t, lane);
       const int32_t* row = a.idx + (static_cast<int64_t>(p) * a.n_tiles + t) * a.top_k;
       const int bi = p / a.Hkv, h = p % a.Hkv;
+      const int h0 = (h * a.HG + hg) * kG;           // the item's first query head
       if constexpr (COL) {
         if (warp == 8 && lane == 0) {
           if (it > 0 && !mbar_wait_bounded(q_empty, (it - 1) & 1, abort_flag)) { fail(); ok = false; }
           if (ok) {
             mbar_arrive_expect_tx(q_full, kQBytes);
             const int tok = bi * a.T + t * kT;
-            tc::tma_load_3d(Qs, &q_map, 0, h * kG, tok, q_full);
-            tc::tma_load_3d(Qs + kQBytes / 2, &q_map, 64, h * kG, tok, q_full);
+            tc::tma_load_3d(Qs, &q_map, 0, h0, tok, q_full);
+            tc::tma_load_3d(Qs + kQBytes / 2, &q_map, 64, h0, tok, q_full);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -284,8 +291,8 @@ __global__ void __launch_bounds__(COL ? kThreadsCol : kThreads, 1)
         if (ok) {
           mbar_arrive_expect_tx(q_full, kQBytes);
           const int tok = bi * a.T + t * kT;
-          tc::tma_load_3d(Qs, &q_map, 0, h * kG, tok, q_full);
-          tc::tma_load_3d(Qs + kQBytes / 2, &q_map, 64, h * kG, tok, q_full);
+          tc::tma_load_3d(Qs, &q_map, 0, h0, tok, q_full);
+          tc::tma_load_3d(Qs + kQBytes / 2, &q_map, 64, h0, tok, q_full);
         }
         int sel = 0;   // position in the index row
         for (int b = 0; b < bl.n_blk && ok; ++b, ++use) {
@@ -322,8 +329,8 @@ __global__ void __launch_bounds__(COL ? kThreadsCol : kThreads, 1)
     bool ok = true;
     const uint32_t qa = smem_u32(Qs), kva = smem_u32(KV), pa = smem_u32(Ps);
     for (int k = blockIdx.x; k < n_items && ok; k += gridDim.x, ++it) {
-      int p, t;
-      item_of(a, k, &p, &t);
+      int p, t, hg;
+      item_of(a, k, &p, &t, &hg);
       const Blocks bl = item_blocks<COL>(a, p, t, lane);
       // the whole warp runs the issue loop in lock step (descriptors stay
       // warp-uniform); one elected lane issues each MMA and commit
@@ -402,8 +409,8 @@ __global__ void __launch_bounds__(COL ? kThreadsCol : kThreads, 1)
     int it = 0, nb_all = 0;
     bool ok = true;
     for (int k = blockIdx.x; k < n_items && ok; k += gridDim.x, ++it) {
-      int p, t;
-      item_of(a, k, &p, &t);
+      int p, t, hg;
+      item_of(a, k, &p, &t, &hg);
       const Blocks bl = item_blocks<COL>(a, p, t, lane);
       float m_ref = -CUDART_INF_F, l = 0.f;
       for (int b = 0; b < bl.n_blk; ++b, ++nb_all) {
@@ -506,7 +513,7 @@ __global__ void __launch_bounds__(COL ? kThreadsCol : kThreads, 1)
       const int bi = p / a.Hkv, h = p % a.Hkv;
       const int tok = t * kT + r;
       const bool valid = tok < a.T;
-      const int64_t orow = (static_cast<int64_t>(bi) * a.T + tok) * a.Hq + h * kG + g;
+      const int64_t orow = (static_cast<int64_t>(bi) * a.T + tok) * a.Hq + (h * a.HG + hg) * kG + g;
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
       for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -574,6 +581,7 @@ cudaError_t launch_prefill_attn(const PrefillArgs& pa, cudaStream_t s) {
   a.B = pa.B;
   a.Hq = pa.Hq;
   a.Hkv = pa.Hkv;
+  a.HG = pa.Hq / pa.Hkv / kG;
   a.T = pa.T;
   a.n_tiles = pa.n_tiles;
   a.P = pa.B * pa.Hkv;
@@ -612,7 +620,7 @@ cudaError_t launch_prefill_attn(const PrefillArgs& pa, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int items = pa.n_tiles * a.P;
+  const int items = pa.n_tiles * a.P * a.HG;
   const int grid = items < pa.num_sms ? items : pa.num_sms;
   prefill_attn_kernel<false><<<grid, kThreads, smem, s>>>(qm, km, vm, a);
   return cudaGetLastError();
@@ -632,6 +640,7 @@ cudaError_t launch_column_attn(const PrefillArgs& pa, cudaStream_t s) {
   a.B = pa.B;
   a.Hq = pa.Hq;
   a.Hkv = pa.Hkv;
+  a.HG = pa.Hq / pa.Hkv / kG;
   a.T = pa.T;
   a.n_tiles = pa.n_tiles;
   a.P = pa.B * pa.Hkv;
@@ -654,7 +663,7 @@ cudaError_t launch_column_attn(const PrefillArgs& pa, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int items = pa.n_tiles * a.P;
+  const int items = pa.n_tiles * a.P * a.HG;
   const int grid = items < pa.num_sms ? items : pa.num_sms;
   // K and V are gathered by cp.async: their tensor-map slots are unused
   prefill_attn_kernel<true><<<grid, kThreadsCol, smem, s>>>(qm, qm, qm, a);

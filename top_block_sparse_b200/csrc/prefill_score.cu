@@ -25,9 +25,10 @@
 // pair of query tiles) in decreasing-cost order):
 //   warp 0      TMA producer: Kc hi / lo chunks of 128 blocks (128-byte swizzle)
 //   warp 1      TMEM owner and MMA issuer (one thread)
-//   warps 2-9   build the B operand: GQA sum x scale of 128 query rows, split
-//               into hi / lo, written to swizzled shared memory (16 rows per
-//               warp, 8 rows of loads in flight: Q is the kernel's HBM stream)
+//   warps 2-9   build the B operand: GQA sum (G a multiple of 4) x scale of
+//               128 query rows, split into hi / lo, written to swizzled shared
+//               memory (16 rows per warp, 4 rows x 4 heads of loads in flight
+//               per round: Q is the kernel's HBM stream)
 //   warps 10-13 epilogue: TMEM -> registers, max over each 64-row tile,
 //               candidate mask, fp32 scores to global
 #include <cudaTypedefs.h>
@@ -277,7 +278,8 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
       const int row = 128 * n2 + wq * 16 + lane;
       if (chunk_count(a, n2) == 0 || row >= a.T) return;
       const int bi2 = p2 / a.Hkv, h2 = p2 % a.Hkv;
-      prefetch_l2_bulk(a.Q + ((static_cast<int64_t>(bi2) * a.T + row) * a.Hq + h2 * 4) * kHeadDim, 4 * kHeadDim * 2);
+      prefetch_l2_bulk(a.Q + ((static_cast<int64_t>(bi2) * a.T + row) * a.Hq + h2 * a.G) * kHeadDim,
+                       static_cast<uint32_t>(a.G) * kHeadDim * 2);
     };
     prefetch_item(blockIdx.x);
     prefetch_item(blockIdx.x + gridDim.x);
@@ -297,27 +299,41 @@ __global__ void __launch_bounds__(kScoreThreadsTC, 1)
       unsigned char* dst_lo = dst_hi + 32768;
 #pragma unroll 1
       for (int rb = 0; rb < 8; rb += 4) {
-        uint4 x[4][4];
+        // the GQA sum over the group's G heads, four heads of four rows per round
+        float vs[4][8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int row = 128 * n + wq * 16 + 2 * (rb + u) + rp;
-          const uint4* src = reinterpret_cast<const uint4*>(
-              a.Q + ((static_cast<int64_t>(bi) * a.T + (row < a.T ? row : 0)) * a.Hq + h * 4) * kHeadDim);
+        for (int u = 0; u < 4; ++u)
 #pragma unroll
-          for (int g = 0; g < 4; ++g)
-            x[u][g] = row < a.T ? __ldg(src + g * 16 + cc) : make_uint4(0u, 0u, 0u, 0u);
+          for (int e = 0; e < 8; ++e) vs[u][e] = 0.f;
+#pragma unroll 1
+        for (int hb = 0; hb < a.G; hb += 4) {
+          uint4 x[4][4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int row = 128 * n + wq * 16 + 2 * (rb + u) + rp;
+            const uint4* src = reinterpret_cast<const uint4*>(
+                a.Q + ((static_cast<int64_t>(bi) * a.T + (row < a.T ? row : 0)) * a.Hq + h * a.G + hb) * kHeadDim);
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              x[u][g] = row < a.T ? __ldg(src + g * 16 + cc) : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float f[8];
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              unpack8(x[u][g], f);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) vs[u][e] += f[e];
+            }
+          }
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int r = wq * 16 + 2 * (rb + u) + rp;
-          float v[8], f[8];
-          unpack8(x[u][0], v);
+          float v[8];
 #pragma unroll
-          for (int g = 1; g < 4; ++g) {
-            unpack8(x[u][g], f);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] += f[e];
-          }
+          for (int e = 0; e < 8; ++e) v[e] = vs[u][e];
           float mul = a.scale;
           if (a.lsa) {
             // the row's 128 columns sit on the 16 lanes of this half-warp

@@ -281,15 +281,15 @@ struct PrefillGeom {
 // Shape limits of the tensor-core prefill path (besides check_params).
 sa_status check_prefill(const sa_params* p, PrefillGeom* g) {
   if (p->dtype != SA_BF16) return fail(SA_ERR_UNSUPPORTED, "prefill runs on bf16 tensor cores: dtype must be SA_BF16");
-  if (p->num_q_heads != 4 * p->num_kv_heads)
-    return fail(SA_ERR_UNSUPPORTED, "prefill is built for GQA groups of 4 query heads per KV head");
+  if ((p->num_q_heads / p->num_kv_heads) % 4 != 0)
+    return fail(SA_ERR_UNSUPPORTED, "prefill is built for GQA groups of a multiple of 4 query heads per KV head");
   if (p->block_size != 64) return fail(SA_ERR_UNSUPPORTED, "prefill is built for block_size 64 (= query tile)");
   if (p->sink_keys % 64 != 0 || p->window_keys % 64 != 0)
     return fail(SA_ERR_UNSUPPORTED, "prefill needs sink_keys and window_keys to be multiples of 64");
   g->B = p->batch;
   g->Hq = p->num_q_heads;
   g->Hkv = p->num_kv_heads;
-  g->G = 4;
+  g->G = p->num_q_heads / p->num_kv_heads;
   g->T = p->n_q;
   g->nb = p->n_q / 64;
   g->n_tiles = (p->n_q + 63) / 64;
@@ -511,13 +511,13 @@ VerifyWs verify_ws(const DecodeGeom& g, const DecodePlan& plan, int64_t nb) {
 // ---- column-sparse attention ------------------------------------------------
 sa_status check_column(const sa_params* p, PrefillGeom* g) {
   if (p->dtype != SA_BF16) return fail(SA_ERR_UNSUPPORTED, "column attention runs on bf16 tensor cores");
-  if (p->num_q_heads != 4 * p->num_kv_heads)
-    return fail(SA_ERR_UNSUPPORTED, "column attention is built for GQA groups of 4 query heads per KV head");
+  if ((p->num_q_heads / p->num_kv_heads) % 4 != 0)
+    return fail(SA_ERR_UNSUPPORTED, "column attention is built for GQA groups of a multiple of 4 query heads per KV head");
   if (p->block_size != 64) return fail(SA_ERR_UNSUPPORTED, "column attention groups 64 query tokens: block_size 64");
   g->B = p->batch;
   g->Hq = p->num_q_heads;
   g->Hkv = p->num_kv_heads;
-  g->G = 4;
+  g->G = p->num_q_heads / p->num_kv_heads;
   g->T = p->n_q;
   g->nb = p->n_q / 64;
   g->n_tiles = (p->n_q + 63) / 64;
