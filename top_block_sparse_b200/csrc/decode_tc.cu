@@ -52,11 +52,14 @@ constexpr int kThreadsFused = 256;              // fused: warps 6-7 select the t
 constexpr int kThreadsSplit = 320;              // 9-16 rows: warps 6-9 are a second softmax warpgroup
 constexpr int kSoftThreads = 128;
 constexpr int kSelBarThreads = 192;             // softmax warps + selection warps
-constexpr int kNumBars = 22;
+constexpr int kNumBars = 24;                    // 23 used; an even count keeps what follows 16-byte aligned
 constexpr uint32_t kIdescS = tc::idesc_bf16(128, kN, false, false);
 constexpr uint32_t kIdescO = tc::idesc_bf16(128, kN, true, false);
 constexpr float kLazy = 8.f;                    // raise the running max when it grows by > 2^8
 constexpr int kMaxSelPerCta = 64;               // fused: pairs one CTA may select
+// wmax and lsum follow the barriers and the stage records and are read as float4
+static_assert((kNumBars * 8 + kNS * sizeof(StageInfo)) % 16 == 0,
+              "shared memory after the stage records must stay 16-byte aligned");
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kNS) * kStage + 2 * kQBuf + 2 * kPBuf +
                               kNumBars * 8 + kNS * sizeof(StageInfo) + (2 * 4 * kN + 4 * kN) * 4 + 32;
 constexpr size_t kSmemFused = kSmemBytes;
@@ -230,6 +233,7 @@ __global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
   uint64_t* p_free = bars + 16;
   uint64_t* o_full = bars + 18;
   uint64_t* o_free = bars + 20;
+  uint64_t* score_done = bars + 22;      // fused: every score chunk consumed
   StageInfo* info = reinterpret_cast<StageInfo*>(bars + kNumBars);
   float* wmax = reinterpret_cast<float*>(info + kNS);          // [2][16 rows][4 warps]
   float* lsum = wmax + 2 * 4 * kN;                              // [16 rows][4 warps]
@@ -274,6 +278,7 @@ __global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
       mbar_init(&o_free[b], kSplitRows<NR, FUSED> ? 2 * kSoftThreads : kSoftThreads);
     }
     mbar_init(mma_done, 1);
+    mbar_init(score_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -447,8 +452,17 @@ __global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
       cs.init(a.ord, i0, nI, d0, nunits);
       cp.init(a.ord, i0, nI, d0, nunits);
       bool ok = true;
+      // Fused: the ring's first r0 uses carry score chunks, which land in
+      // order of use as far as the softmax warps' waits see them.  Only once
+      // the last one has landed does each stage's full barrier stand at or
+      // past its last score-chunk phase; polled earlier, a completed phase of
+      // the same parity one use back would read as an attention unit's
+      // arrival.
+      if constexpr (FUSED) {
+        if (!mbar_wait_warp(score_done, 0, abort_flag)) ok = false;
+      }
       uint64_t t0 = global_ns();
-      for (uint32_t spin = 0; npv < nunits; ++spin) {
+      for (uint32_t spin = 0; ok && npv < nunits; ++spin) {
         bool did = false;
         if (ns < nunits) {
           const bool fi = cs.first(ns);
@@ -886,6 +900,9 @@ __global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
           q4 = make_float4(acc.x * mul, acc.y * mul, acc.z * mul, acc.w * mul);
         }
         const bool got = mbar_wait_bounded(&kv_full[s], (ci / kNS) & 1, abort_flag);
+        // the last score chunk has landed, so every stage's full barrier has
+        // passed its score-chunk phases: the MMA warp may poll the ring
+        if (got && t == 0 && ci == r0 - 1) mbar_arrive(score_done);
         if (got) {
           const float* rowp = reinterpret_cast<const float*>(ring + s * kStage);
           float* sc = a.scores + static_cast<int64_t>(pr) * nb + ch * 128;
@@ -929,6 +946,7 @@ __global__ void __launch_bounds__(kThreadsOf<NR, FUSED>, 1)
       }
       if (t == 0 && ok && cur >= 0) close_run(cur, seg_cnt);
       softmax_bar();
+      if (t == 0 && r0 == 0) mbar_arrive(score_done);    // no score chunks
       // sel_list is complete: hand it to the selection warps and go on
       sel_bar_arrive();
     }
